@@ -1,0 +1,349 @@
+"""Benchmark of the TQP MoE layer forward on B200 (one process per GPU).
+
+python bench.py [--gpus N --steps K --warmup W --config full|skewed|mid|tiny] [--impl tqp|reference]
+
+A step is one full layer forward (router GEMM, top-k routing, permutation,
+grouped int4+LoRA SwiGLU experts, combine) over one batch of T synthetic
+tokens, issued as the library's public C-ABI calls. Inputs are resident in HBM
+when the timed region starts; L2 is flushed between steps by writing a buffer
+larger than L2 (the layer's weights, 1.4 GB for the 460-expert config, are
+larger than L2 as well). Per-step CUDA events on the launching stream time
+every call; the timed region is bracketed by a barrier and a device
+synchronisation on both sides; multi-GPU time is the max over ranks. Each rank
+processes its own batch (weak scaling, no collective on the data path).
+
+The `e2e` leg measures the same metric through the Python API with the token
+batch copied from pinned host memory and the layer output copied back inside
+the timed region. `cpu_baseline` times the fp64 oracle on a bounded sample of
+the same workload on this host's cores. `--impl reference` times that oracle
+as the reference arm (there is no other implementation of this layer).
+"""
+from __future__ import annotations
+
+import argparse
+import json
+import os
+import statistics
+import subprocess
+import sys
+import tempfile
+import time
+
+import numpy as np
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+if ROOT not in sys.path:
+    sys.path.insert(0, ROOT)
+
+import synth  # noqa: E402
+
+METRIC = "routed tokens/s and TFLOP/s, 460-expert top-12 TQP MoE layer; % of roofline"
+UNIT = "tokens/s"
+L2_FLUSH_BYTES = 512 << 20
+
+
+def layer_flops(cfg: synth.LayerConfig) -> dict:
+    """Algorithmic FLOPs of one layer forward (router, experts, LoRA)."""
+    A = cfg.T * cfg.k
+    router = 2.0 * cfg.T * cfg.d * cfg.E
+    expert = A * 6.0 * cfg.d * cfg.f
+    lora = A * 2.0 * cfg.r * (cfg.d + cfg.f) * 3
+    return {"router": router, "expert": expert, "lora": lora, "total": router + expert + lora,
+            "ffn": expert + lora}
+
+
+def peaks() -> dict:
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(p):
+        d = json.load(open(p))
+        return {"hbm_gbs": d["hbm_gbs"], "bf16_tflops": d["bf16_tflops"],
+                "bf16_tflops_sustained": d.get("bf16_tflops_sustained"), "source": "measured"}
+    return {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0, "source": "fallback"}
+
+
+def cores() -> int:
+    try:
+        return len(os.sched_getaffinity(0))
+    except AttributeError:
+        return os.cpu_count() or 1
+
+
+# ---------------------------------------------------------------- CPU oracle timing
+
+
+def time_oracle(cfg: synth.LayerConfig, host: dict, x_bits: np.ndarray, sample_tokens: int) -> dict:
+    """Time the fp64 oracle's layer forward on the first `sample_tokens` tokens."""
+    from oracle import tqp_oracle as O
+    L = O.Layer(host)
+    x = O.bf16_to_f64(x_bits[:sample_tokens])
+    t0 = time.perf_counter()
+    O.layer_forward(x, L)
+    dt = time.perf_counter() - t0
+    return {"value": sample_tokens / dt, "unit": UNIT, "cores": cores(), "kind": "oracle",
+            "sample": f"first {sample_tokens} of {cfg.T} tokens of the {cfg.name} workload, fp64 NumPy "
+                      f"(dequantises every touched expert), {dt:.1f} s wall"}
+
+
+# ---------------------------------------------------------------- clocks
+
+
+class ClockSampler:
+    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, gpu_index: int):
+        self.idx = gpu_index
+        self.proc = None
+        self.path = tempfile.mktemp(suffix=".csv")
+
+    def start(self):
+        try:
+            self.f = open(self.path, "w")
+            self.proc = subprocess.Popen(["nvidia-smi", "-i", str(self.idx), f"--query-gpu={self.FIELDS}",
+                                          "--format=csv,noheader,nounits", "-lms", "200"], stdout=self.f,
+                                         stderr=subprocess.DEVNULL)
+        except (OSError, FileNotFoundError):
+            self.proc = None
+
+    def stop(self) -> dict:
+        if self.proc is None:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["nvidia-smi unavailable"]}
+        self.proc.terminate()
+        try:
+            self.proc.wait(timeout=5)
+        except subprocess.TimeoutExpired:
+            self.proc.kill()
+        self.f.close()
+        sm, smax, reasons = [], None, set()
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        for line in open(self.path):
+            parts = [p.strip() for p in line.split(",")]
+            if len(parts) < 9:
+                continue
+            try:
+                sm.append(float(parts[1]))
+                smax = float(parts[2])
+            except ValueError:
+                continue
+            for n, v in zip(names, parts[5:9]):
+                if v.lower().startswith("active"):
+                    reasons.add(n)
+        os.unlink(self.path)
+        load = [v for v in sm if smax and v > 0.3 * smax] or sm
+        return {"sm_mhz": statistics.median(load) if load else None, "sm_max_mhz": smax,
+                "samples": len(sm), "reasons": sorted(reasons)}
+
+
+# ---------------------------------------------------------------- GPU arm
+
+
+def run_tqp(args, rank: int, world: int, local_rank: int) -> dict | None:
+    import torch
+    import quantized_base_lora_moe_b200 as Q
+    torch.cuda.set_device(local_rank)
+    dev = torch.device("cuda", local_rank)
+    cfg = synth.CONFIGS[args.config]
+    host = synth.make_layer(cfg)
+    x_bits = synth.make_tokens(cfg.T, cfg.d, cfg.seed + rank)
+    L = Q.DeviceLayer(host, device=dev)
+    T, E, k, d, f = cfg.T, cfg.E, cfg.k, cfg.d, cfg.f
+    A = T * k
+    x = torch.from_numpy(x_bits.view(np.int16)).to(dev)
+    y = torch.empty(T, d, dtype=torch.int16, device=dev)
+    logits = torch.empty(T, E, dtype=torch.float32, device=dev)
+    ids = torch.empty(T, k, dtype=torch.int32, device=dev)
+    gates = torch.empty(T, k, dtype=torch.float32, device=dev)
+    offsets = torch.empty(E + 1, dtype=torch.int32, device=dev)
+    perm = torch.empty(A, dtype=torch.int32, device=dev)
+    inv = torch.empty(A, dtype=torch.int32, device=dev)
+    h = torch.empty(A, f, dtype=torch.int16, device=dev)
+    o = torch.empty(A, d, dtype=torch.int16, device=dev)
+    lib = Q.lib()
+    ws_r = Q.workspace(lib.moe_router_gemm_workspace_size(T, L.ref()), dev)
+    ws_p = Q.workspace(lib.moe_permute_workspace_size(T, E, k), dev)
+    ws_f = Q.workspace(lib.tqp_grouped_ffn_workspace_size(T, L.ref()), dev)
+    ws_l = Q.workspace(lib.tqp_moe_layer_workspace_size(T, L.ref()), dev)
+    st = Q.Status(dev)
+    flush = torch.empty(L2_FLUSH_BYTES, dtype=torch.uint8, device=dev)
+    stream = torch.cuda.current_stream(dev)
+    names = ["router_gemm", "route", "permute", "grouped_ffn", "combine"]
+    launches_per_step = {"router_gemm": 2, "route": 1, "permute": 3, "grouped_ffn": 6 if cfg.r > 0 else 4,
+                         "combine": 1}
+
+    def step(evs=None):
+        def mark(i):
+            if evs is not None:
+                evs[i].record(stream)
+        mark(0)
+        Q.moe_router_gemm(x, L, logits, ws_r, st)
+        mark(1)
+        Q.moe_route(logits, k, ids, gates, st)
+        mark(2)
+        Q.moe_permute(ids, E, offsets, perm, inv, ws_p, st)
+        mark(3)
+        Q.tqp_grouped_ffn(x, offsets, perm, L, h, o, ws_f, st)
+        mark(4)
+        Q.moe_combine(o, inv, gates, y)
+        mark(5)
+
+    dist = world > 1
+    for _ in range(args.warmup):
+        flush.zero_()
+        step()
+    torch.cuda.synchronize(dev)
+    if st.read() != 0:
+        raise RuntimeError(f"device status {st.read()} after warm-up")
+    evs = [[torch.cuda.Event(enable_timing=True) for _ in range(6)] for _ in range(args.steps)]
+    clocks = ClockSampler(int(os.environ.get("CUDA_VISIBLE_DEVICES", str(local_rank)).split(",")[0])
+                          if "CUDA_VISIBLE_DEVICES" in os.environ else local_rank)
+    if rank == 0:
+        clocks.start()
+        time.sleep(0.4)
+    if dist:
+        torch.distributed.barrier()
+    torch.cuda.synchronize(dev)
+    for i in range(args.steps):
+        flush.zero_()                       # L2 flush, outside the per-step events
+        step(evs[i])
+    torch.cuda.synchronize(dev)
+    if dist:
+        torch.distributed.barrier()
+    clk = clocks.stop() if rank == 0 else None
+    per_call = {n: [] for n in names}
+    step_ms = []
+    for e in evs:
+        for j, n in enumerate(names):
+            per_call[n].append(e[j].elapsed_time(e[j + 1]))
+        step_ms.append(e[0].elapsed_time(e[5]))
+    total_ms = float(sum(step_ms))
+    t = torch.tensor([total_ms], dtype=torch.float64, device=dev)
+    if dist:
+        torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
+    max_ms = float(t.item())
+
+    # e2e through the public API: pinned host tokens in, layer output back to host, each step
+    e2e = None
+    if not args.no_e2e:
+        x_host = torch.from_numpy(x_bits.view(np.int16)).pin_memory()
+        y_host = torch.empty(T, d, dtype=torch.int16).pin_memory()
+        x_dev = torch.empty_like(x)
+        for _ in range(2):
+            x_dev.copy_(x_host, non_blocking=True)
+            Q.tqp_moe_layer_fwd(x_dev, L, y, ws_l, st)
+            y_host.copy_(y, non_blocking=True)
+        torch.cuda.synchronize(dev)
+        if dist:
+            torch.distributed.barrier()
+        e0 = torch.cuda.Event(enable_timing=True)
+        e1 = torch.cuda.Event(enable_timing=True)
+        e0.record(stream)
+        for _ in range(args.steps):
+            x_dev.copy_(x_host, non_blocking=True)
+            Q.tqp_moe_layer_fwd(x_dev, L, y, ws_l, st)
+            y_host.copy_(y, non_blocking=True)
+        e1.record(stream)
+        torch.cuda.synchronize(dev)
+        te = torch.tensor([e0.elapsed_time(e1)], dtype=torch.float64, device=dev)
+        if dist:
+            torch.distributed.all_reduce(te, op=torch.distributed.ReduceOp.MAX)
+        e2e_ms = float(te.item()) / args.steps
+        e2e = {"value": world * T / (e2e_ms * 1e-3), "unit": UNIT, "h2d_bytes_per_step": int(T * d * 2),
+               "d2h_bytes_per_step": int(T * d * 2), "ms_per_step": e2e_ms}
+    if st.read() != 0:
+        raise RuntimeError(f"device status {st.read()} after the timed steps")
+    if rank != 0:
+        return None
+
+    ms = max_ms / args.steps
+    fl = layer_flops(cfg)
+    pk = peaks()
+    ffn_ms = statistics.mean(per_call["grouped_ffn"])
+    ffn_tflops = fl["ffn"] / (ffn_ms * 1e-3) / 1e12
+    result = {
+        "metric": METRIC, "value": world * T / (ms * 1e-3), "unit": UNIT, "n_gpus": world,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms, "higher_is_better": True,
+        "scaling": "weak", "vs_baseline": None, "dtype": "f16",
+        "data": "synthetic (seeded N(0,1) tokens, N(0,1/d) weights int4-quantised, random-init LoRA)",
+        "config": {"workload": f"{cfg.name}: T={T} d={d} E={E} top-{k} ffn={f} int4 g{cfg.g} LoRA r{cfg.r}"
+                               f"{' zipf-bias' if cfg.zipf_s else ''}, layer forward",
+                   "T": T, "d": d, "E": E, "k": k, "ffn": f, "group": cfg.g, "rank": cfg.r,
+                   "l2": "flushed before every step (512 MB write); weights 1.4 GB > L2",
+                   "parallelism": f"dp{world} (independent token batches, replicated weights)"},
+        "tflops": fl["total"] / (ms * 1e-3) / 1e12 * world,
+        "assignments_per_s": world * A / (ms * 1e-3),
+        "per_call_ms": {n: statistics.mean(v) for n, v in per_call.items()},
+        "roofline": {"bound": "tensor", "kernel": "tqp_grouped_ffn (int4-dequant + fp16 tcgen05 grouped GEMMs)",
+                     "achieved": ffn_tflops, "peak": pk["bf16_tflops"], "unit": "TFLOP/s",
+                     "frac": ffn_tflops / pk["bf16_tflops"], "traffic": None,
+                     "peak_source": f"{pk['source']} bf16 dense burst (fp16 has the same nominal rate)",
+                     "flop_per_launch": fl["ffn"]},
+        "layer_roofline_frac_nominal": (fl["total"] / 2.25e15) / (ms * 1e-3),
+        "gpu_launches": args.steps * sum(launches_per_step.values()),
+        "clocks": clk,
+        "e2e": e2e,
+    }
+    if world == 1 and not args.no_cpu_baseline:
+        sample = min(T, args.cpu_sample)
+        result["cpu_baseline"] = time_oracle(cfg, host, x_bits, sample)
+    return result
+
+
+def run_reference(args, rank: int) -> dict | None:
+    """The reference arm: the fp64 CPU oracle (the only other implementation)."""
+    if rank != 0:
+        return None
+    cfg = synth.CONFIGS[args.config]
+    host = synth.make_layer(cfg)
+    x_bits = synth.make_tokens(cfg.T, cfg.d, cfg.seed)
+    sample = min(cfg.T, args.ref_sample)
+    for _ in range(args.warmup):
+        time_oracle(cfg, host, x_bits, 1)    # untimed
+    vals = []
+    for _ in range(args.steps):
+        vals.append(time_oracle(cfg, host, x_bits, sample))
+    v = statistics.mean(r["value"] for r in vals)
+    return {"impl": "reference", "metric": METRIC, "value": v, "unit": UNIT, "n_gpus": 1,
+            "steps": args.steps, "warmup": args.warmup, "ms_per_step": sample / v * 1e3,
+            "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
+            "data": "synthetic", "config": {"workload": f"{cfg.name}, layer forward, oracle on a {sample}-token sample"},
+            "cpu_baseline": {"value": v, "unit": UNIT, "cores": cores(), "kind": "oracle", "sample": vals[0]["sample"]},
+            "e2e": {"value": v, "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
+
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=20)
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--config", default="full", choices=sorted(synth.CONFIGS))
+    ap.add_argument("--impl", default="tqp", choices=["tqp", "reference"])
+    ap.add_argument("--cpu-sample", type=int, default=256, help="tokens of the cpu_baseline sample")
+    ap.add_argument("--ref-sample", type=int, default=8, help="tokens per step of the reference arm")
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--no-e2e", action="store_true")
+    args = ap.parse_args()
+    rank = int(os.environ.get("RANK", 0))
+    world = int(os.environ.get("WORLD_SIZE", 1))
+    local_rank = int(os.environ.get("LOCAL_RANK", 0))
+    if args.impl == "reference":
+        res = run_reference(args, rank)
+        if res is not None:
+            print(json.dumps(res))
+        return
+    import torch
+    if world > 1:
+        import datetime
+        torch.cuda.set_device(local_rank)
+        torch.distributed.init_process_group("nccl", timeout=datetime.timedelta(seconds=120))
+    try:
+        res = run_tqp(args, rank, world, local_rank)
+    finally:
+        if world > 1:
+            torch.distributed.destroy_process_group()
+    if res is not None:
+        print(json.dumps(res))
+
+
+if __name__ == "__main__":
+    main()

@@ -1,0 +1,243 @@
+/*
+ * tqp_moe.h - C ABI of the B200 (sm_100a) TQP MoE layer and its reversible coupling.
+ *
+ * The layer is the routed-expert block of the reversible sparse MoE described in
+ * "Reversible Sparse MoE Single Node" (skills-directory page) and the abstract
+ * of "Reversible Foundations: Training a 120B Sparse MoE through
+ * State-Preserving Scaling":
+ *   - 460 routed experts with top-12 routing ("Architecture Details"; Abstract),
+ *   - TQP: frozen quantised base expert weights plus trained low-rank adapters
+ *     per expert, full-precision router ("Principle 3: TQP Optimizer Strategy";
+ *     "TQP Quantization"; Abstract, "Single-node economics"),
+ *   - stateless routing, recomputed during the inverse ("Reversibility
+ *     Implementation"),
+ *   - reversible residual blocks whose inverse is a subtraction, used to
+ *     reconstruct activations in the backward pass instead of storing them
+ *     ("Principle 1: Reversible Recurrence Stack"; "Pattern 1"; Abstract,
+ *     "Reversibility").
+ * The pages fix neither equations nor formats; the readings used here are:
+ * gates = softmax over the k chosen fp32 logits (ties -> lower expert id),
+ * SwiGLU experts, LoRA W' = W + s*A*B on gate, up and down, symmetric int4
+ * base weights with one bf16 scale per group of `group` input positions, and
+ * the additive coupling y1 = x1 + F(x2), y2 = x2 + G(y1).
+ *
+ * Conventions (all entry points)
+ *   - Return value: TQP_OK (0) or a negative TQP_ERR_* code. Argument errors
+ *     are detected on the host before anything is enqueued.
+ *   - Data-dependent errors are OR-ed asynchronously into `dev_status`, a
+ *     caller-owned int32 in device memory that the caller zeroes and reads
+ *     after synchronising: TQP_STATUS_NONFINITE (a NaN/Inf router logit),
+ *     TQP_STATUS_BAD_ID (an expert id outside [0, E)), TQP_STATUS_TIMEOUT (a
+ *     device-side wait hit its limit; outputs are then undefined). Nothing
+ *     traps, prints or exits.
+ *   - Every pointer argument is caller-owned DEVICE memory (unless stated),
+ *     16-byte aligned, dense row-major. The library never allocates device
+ *     memory: scratch comes from `ws` of at least the size returned by the
+ *     matching *_workspace_size query (which needs no GPU).
+ *   - Work is enqueued on `stream` (a cudaStream_t; NULL = legacy default
+ *     stream) and the call returns at once. Calls hold no global state and may
+ *     run concurrently on different streams with disjoint workspaces.
+ *   - bf16 tensors are uint16_t bit patterns.
+ *   - Outputs are overwritten (never accumulated into).
+ *
+ * Weight formats (one tqp_moe_weights per layer; p = 0 gate, 1 up, 2 down;
+ * in_p / out_p = d / ffn for gate and up, ffn / d for down)
+ *   router_w   [E][d] fp32.
+ *   router_bias[E] fp32 or NULL: additive per-expert bias, added to the logits
+ *              before top-k and gates.
+ *   wq[p]      [E][out_p][in_p/2] uint8: int4 codes of the frozen base weight
+ *              W_p[out][in]. Each little-endian 32-bit word holds 8 consecutive
+ *              input positions k0..k7 of one output row as two's-complement
+ *              nibbles: k(2i) in bits [4i,4i+4), k(2i+1) in bits [16+4i,16+4i+4).
+ *   wscale[p]  [E][in_p/group][out_p] bf16: W_p[n][k] = q[n][k] * wscale[k/group][n].
+ *   lora_a[p]  [E][rank][in_p] bf16: A_p^T.
+ *   lora_b[p]  [E][out_p][rank] bf16: B_p^T.
+ *   The projection is  x -> x W_p^T + lora_scale * (x A_p) B_p.
+ *
+ * Validity (host-checked, else TQP_ERR_INVALID_ARG / TQP_ERR_UNSUPPORTED):
+ *   1 <= top_k <= E <= 4096; d % 128 == 0; ffn % 64 == 0; 64 <= d, ffn <= 16384;
+ *   group in {32, 64, 128, 256} dividing d and ffn; rank % 8 == 0 and
+ *   0 <= rank <= 64 (rank 0 skips the adapter path); T >= 0 (T == 0 is a no-op).
+ */
+#ifndef TQP_MOE_H_
+#define TQP_MOE_H_
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+#define TQP_OK 0
+#define TQP_ERR_INVALID_ARG (-1)
+#define TQP_ERR_UNSUPPORTED (-2)
+#define TQP_ERR_WORKSPACE (-3)
+#define TQP_ERR_CUDA (-4)
+
+#define TQP_STATUS_NONFINITE 1
+#define TQP_STATUS_BAD_ID 2
+#define TQP_STATUS_TIMEOUT 4
+
+#define TQP_DTYPE_BF16 0
+#define TQP_DTYPE_F32 1
+
+typedef struct tqp_moe_weights {
+  int E;            /* routed experts */
+  int d;            /* model width */
+  int ffn;          /* expert SwiGLU hidden width */
+  int group;        /* quantisation group along the input dimension */
+  int rank;         /* LoRA rank */
+  int top_k;        /* experts per token */
+  float lora_scale; /* s = alpha / rank */
+  const float* router_w;
+  const float* router_bias;
+  const uint8_t* wq[3];
+  const uint16_t* wscale[3];
+  const uint16_t* lora_a[3];
+  const uint16_t* lora_b[3];
+} tqp_moe_weights;
+
+/* Adapter gradients of one layer, fp32, same layouts as lora_a / lora_b:
+ * dA[p] [E][rank][in_p], dB[p] [E][out_p][rank]. Overwritten. */
+typedef struct tqp_adapter_grads {
+  float* dA[3];
+  float* dB[3];
+} tqp_adapter_grads;
+
+/* Library version (major*10000 + minor*100 + patch) and error names. */
+int tqp_version(void);
+const char* tqp_error_string(int code);
+
+/* ---------------------------------------------------------------------------
+ * moe_router_gemm: full-precision router logits.
+ * "Router: Full precision (critical for routing quality)" (TQP Quantization).
+ *   logits[t][e] = sum_i x[t][i] * router_w[e][i] (+ router_bias[e]), accurate to
+ *   fp32 (the fp32 weights are split exactly into three bf16 parts and the
+ *   products accumulated in fp32 on the tensor cores).
+ *   x [T][d] bf16; logits [T][E] fp32. ws: moe_router_gemm_workspace_size.
+ * ------------------------------------------------------------------------- */
+size_t moe_router_gemm_workspace_size(int T, const tqp_moe_weights* w);
+int moe_router_gemm(const uint16_t* x, int T, const tqp_moe_weights* w, float* logits, void* ws,
+                    size_t ws_bytes, int32_t* dev_status, void* stream);
+
+/* ---------------------------------------------------------------------------
+ * moe_route: top-k expert selection and gates ("Top-12 routing", Architecture
+ * Details; stateless, so a replay from the same logits gives the same ids).
+ *   ids[t][j]: the k experts with the largest logits, in descending order;
+ *   exact ties -> lower id first; +0.0 ties with -0.0; NaN ranks lowest.
+ *   gates[t][j] = exp(l_j - l_0) / sum_j' exp(l_j' - l_0) over the chosen ones.
+ *   A NaN or +-Inf logit anywhere in the row raises TQP_STATUS_NONFINITE.
+ *   logits [T][E] fp32; ids [T][k] int32; gates [T][k] fp32.
+ * ------------------------------------------------------------------------- */
+int moe_route(const float* logits, int T, int E, int k, int32_t* ids, float* gates, int32_t* dev_status,
+              void* stream);
+
+/* ---------------------------------------------------------------------------
+ * moe_permute: stable counting sort of the T*k assignments by expert (the
+ * dispatch step of sparse MoE routing, "Related Methods": Switch, GShard).
+ *   offsets[e] = #assignments to experts < e, offsets[E] = T*k;
+ *   rows of one expert are in increasing token order;
+ *   perm_token[row] = token of that row; inv[t*k + j] = row of assignment (t, j).
+ *   ids outside [0, E) raise TQP_STATUS_BAD_ID (those assignments are dropped
+ *   and the outputs are then incomplete).
+ *   ws: moe_permute_workspace_size.
+ * ------------------------------------------------------------------------- */
+size_t moe_permute_workspace_size(int T, int E, int k);
+int moe_permute(const int32_t* ids, int T, int E, int k, int32_t* offsets, int32_t* perm_token, int32_t* inv,
+                void* ws, size_t ws_bytes, int32_t* dev_status, void* stream);
+
+/* ---------------------------------------------------------------------------
+ * tqp_grouped_ffn: the routed experts ("Train low-rank adapters per expert"
+ * over "Quantize base expert weights", Pattern 3). For each expert e and each
+ * of its rows (row r holds token perm_token[r]):
+ *   G = X Wg^T + s (X Ag) Bg ;  U = X Wu^T + s (X Au) Bu ;  H = bf16(silu(G) * U)
+ *   O = bf16(H Wd^T + s (H Ad) Bd)
+ * with the int4 base dequantised in shared memory and all contractions on the
+ * tensor cores (bf16 x bf16 -> fp32). X A and H A are rounded to bf16.
+ *   x [T][d] bf16 (tokens, gathered through perm_token); offsets [E+1];
+ *   h [T*k][ffn] bf16 output (permuted row order); out_perm [T*k][d] bf16 output.
+ *   ws: tqp_grouped_ffn_workspace_size.
+ * ------------------------------------------------------------------------- */
+size_t tqp_grouped_ffn_workspace_size(int T, const tqp_moe_weights* w);
+int tqp_grouped_ffn(const uint16_t* x, int T, const int32_t* offsets, const int32_t* perm_token,
+                    const tqp_moe_weights* w, uint16_t* h, uint16_t* out_perm, void* ws, size_t ws_bytes,
+                    int32_t* dev_status, void* stream);
+
+/* ---------------------------------------------------------------------------
+ * moe_combine: gate-weighted un-permute (scatter back to tokens), plus the
+ * additive coupling when a residual is given ("Pattern 1": addition and
+ * subtraction are the invertible primitives).
+ *   m[t] = bf16( sum_{j<k} gates[t][j] * out_perm[inv[t*k + j]] )  (fixed j order,
+ *   fp32 accumulation, no atomics: deterministic)
+ *   y[t] = m[t]                         if residual == NULL
+ *   y[t] = residual[t] + sign * m[t]    otherwise (fp32 arithmetic)
+ *   residual_dtype / y_dtype: TQP_DTYPE_BF16 or TQP_DTYPE_F32 (bf16 output is
+ *   rounded to nearest even). y_bf16 (nullable): extra bf16 copy of y.
+ * ------------------------------------------------------------------------- */
+int moe_combine(const uint16_t* out_perm, const int32_t* inv, const float* gates, int T, int k, int d,
+                const void* residual, int residual_dtype, float sign, void* y, int y_dtype, uint16_t* y_bf16,
+                void* stream);
+
+/* ---------------------------------------------------------------------------
+ * tqp_moe_layer_fwd: router GEMM -> route -> permute -> grouped FFN -> combine.
+ *   x [T][d] bf16 -> y [T][d] bf16 (the MoE output, no residual).
+ *   ws: tqp_moe_layer_workspace_size.
+ * ------------------------------------------------------------------------- */
+size_t tqp_moe_layer_workspace_size(int T, const tqp_moe_weights* w);
+int tqp_moe_layer_fwd(const uint16_t* x, int T, const tqp_moe_weights* w, uint16_t* y, void* ws,
+                      size_t ws_bytes, int32_t* dev_status, void* stream);
+
+/* ---------------------------------------------------------------------------
+ * Reversible additive coupling ("Principle 1"; "Reversibility
+ * Implementation": reversible residual blocks, RevNet).
+ *   rev_couple_fwd: y1 = x1 + F(x2); y2 = x2 + G(bf16(y1)).
+ *     x1, x2 [T][d] bf16 in; y1, y2 [T][d] fp32 out.
+ *   rev_couple_inv: x2 = y2 - G(bf16(y1)); x1 = y1 - F(x2), rounded to bf16.
+ *     y1, y2 fp32 in; x1, x2 bf16 out. Routing is recomputed (stateless).
+ *   F and G must share d. ws: rev_couple_workspace_size (both calls).
+ * ------------------------------------------------------------------------- */
+size_t rev_couple_workspace_size(int T, const tqp_moe_weights* F, const tqp_moe_weights* G);
+int rev_couple_fwd(const uint16_t* x1, const uint16_t* x2, int T, const tqp_moe_weights* F,
+                   const tqp_moe_weights* G, float* y1, float* y2, void* ws, size_t ws_bytes,
+                   int32_t* dev_status, void* stream);
+int rev_couple_inv(const float* y1, const float* y2, int T, const tqp_moe_weights* F, const tqp_moe_weights* G,
+                   uint16_t* x1, uint16_t* x2, void* ws, size_t ws_bytes, int32_t* dev_status, void* stream);
+
+/* ---------------------------------------------------------------------------
+ * tqp_moe_layer_bwd: gradients of <dy, layer(x)> (base weights and router
+ * frozen: "Base expert weights: Quantized (fixed)"; optimizer state on the
+ * adapters only).
+ *   x [T][d] bf16; dy [T][d] fp32 -> dx [T][d] fp32 (through the experts and,
+ *   via the softmax over the chosen logits, through the frozen router), and the
+ *   adapter gradients `grads`. Top-k selection is treated as constant.
+ *   ws: tqp_moe_layer_bwd_workspace_size.
+ * ------------------------------------------------------------------------- */
+size_t tqp_moe_layer_bwd_workspace_size(int T, const tqp_moe_weights* w);
+int tqp_moe_layer_bwd(const uint16_t* x, const float* dy, int T, const tqp_moe_weights* w, float* dx,
+                      const tqp_adapter_grads* grads, void* ws, size_t ws_bytes, int32_t* dev_status,
+                      void* stream);
+
+/* ---------------------------------------------------------------------------
+ * tqp_adapter_bwd: reversible block backward from the block outputs only
+ * ("Backward: reconstruct from final state ... compute gradients locally",
+ * Principle 1).
+ *   G-step: z = bf16(y1); x2 = y2 - G(z); G's adapter grads for cotangent dy2;
+ *           dz1 = dy1 + J_G(z)^T dy2.
+ *   F-step: x1 = y1 - F(x2); F's adapter grads for cotangent dz1;
+ *           dx2 = dy2 + J_F(x2)^T dz1; dx1 = dz1.
+ *   y1, y2, dy1, dy2 [T][d] fp32 in; x1, x2 [T][d] bf16 out (reconstructed);
+ *   dx1, dx2 [T][d] fp32 out; gF, gG adapter gradients of F and G.
+ *   ws: tqp_adapter_bwd_workspace_size.
+ * ------------------------------------------------------------------------- */
+size_t tqp_adapter_bwd_workspace_size(int T, const tqp_moe_weights* F, const tqp_moe_weights* G);
+int tqp_adapter_bwd(const float* y1, const float* y2, const float* dy1, const float* dy2, int T,
+                    const tqp_moe_weights* F, const tqp_moe_weights* G, uint16_t* x1, uint16_t* x2, float* dx1,
+                    float* dx2, const tqp_adapter_grads* gF, const tqp_adapter_grads* gG, void* ws,
+                    size_t ws_bytes, int32_t* dev_status, void* stream);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* TQP_MOE_H_ */

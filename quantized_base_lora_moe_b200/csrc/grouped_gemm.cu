@@ -1,0 +1,848 @@
+// Grouped tensor-core GEMM engine for the TQP MoE layer (sm_100a, tcgen05).
+//
+// One persistent, warp-specialised kernel template serves every contraction of
+// the forward path:
+//   GATEUP  : [G|U] = X_e Wg/u^T (+ s (X Ag/u) Bg/u), H = bf16(silu(G) * U)
+//   DOWN    : O = bf16(H_e Wd^T + s (H Ad) Bd)
+//   LORA_XA : xa = bf16(s * X_e [Ag | Au])        (rank-space input of gate/up)
+//   LORA_HA : ha = bf16(s * H_e Ad)               (rank-space input of down)
+//   ROUTER  : logits = x W_r^T (+ bias), W_r split exactly into 3 bf16 parts
+// ("Train low-rank adapters per expert" over "Quantize base expert weights",
+// Pattern 3; "Router: Full precision", TQP Quantization.)
+//
+// Work unit = (expert e, n-tile, m-block of up to 256 routed rows). Per CTA (1
+// per SM, 576 threads):
+//   warps 0-3   epilogue: tcgen05.ld from TMEM, activation, bf16 stores
+//   warp  4     TMEM allocation + one thread issuing tcgen05.mma (M=128 per
+//               sub-tile, two sub-tiles share each B tile)
+//   warp  5     TMA producer: int4 code tiles + bf16 group scales
+//   warps 6-9   A producer: cp.async 16-byte row gathers into 128B-swizzled tiles
+//   warps 10-17 B producer: int4 -> bf16 dequant (or bf16 copies) into
+//               128B-swizzled K-major tiles
+// Accumulators are double-buffered in TMEM (2 x 2 x 128 fp32 columns), so the
+// epilogue of one unit overlaps the main loop of the next.
+#include <cstdint>
+#include <cuda.h>
+#include <cudaTypedefs.h>
+#include <cuda_runtime.h>
+
+#include "tqp_device.cuh"
+#include "tqp_launch.h"
+
+namespace tqp {
+
+enum Mode : int { GATEUP = 0, DOWN = 1, LORA_XA = 2, LORA_HA = 3, ROUTER = 4 };
+
+constexpr int kThreads = 576;
+constexpr int kStages = 4;          // operand ring (A: 2 x 16 KB, B: 16 KB)
+constexpr int kQStages = 4;         // int4 + scale ring
+constexpr int kAStageBytes = 32768;
+constexpr int kBStageBytes = 16384;
+constexpr int kOpStageBytes = kAStageBytes + kBStageBytes;
+constexpr int kQStageBytes = 5120;  // 4096 B codes + up to 1024 B scales
+constexpr int kMBlock = 256;
+
+struct GemmArgs {
+  int E;
+  int nkb_main;        // main K-blocks (64 wide)
+  int kb_per_piece;    // ROUTER: K-blocks per bf16 piece (A columns repeat)
+  int nkb_lora;        // extra K-blocks of the LoRA term
+  int lora_k;          // LoRA contraction extent (2r gate/up, r down)
+  int n_tiles;         // n-tiles per m-block
+  int ntile;           // MMA N
+  int g;               // quantisation group
+  int r;               // LoRA rank
+  int in_dim;          // K of the int4 projection (for scale rows)
+  int out_dim;         // rows of one expert's int4 projection
+  float lora_scale;
+  const int32_t* offsets;
+  const int32_t* mb_prefix;
+  const int32_t* perm_token;
+  const uint16_t* a_src;
+  int a_ld;
+  const uint16_t* a_lora;
+  int lora_ld;
+  const uint16_t* b0;   // bf16 B source 0 (Ag^T / Ad^T / router parts) or lora B^T (gate / down)
+  const uint16_t* b1;   // bf16 B source 1 (Au^T) or lora Bu^T
+  const uint8_t* wq0;   // int4 codes (gate or down) and scales, for direct loads
+  const uint8_t* wq1;
+  const uint16_t* ws0;
+  const uint16_t* ws1;
+  void* out;
+  int out_ld;
+  int n_valid;          // valid output columns (ROUTER: E)
+  const float* bias;
+  int32_t* status;
+};
+
+struct SmemCtl {
+  uint64_t op_full[kStages];
+  uint64_t op_empty[kStages];
+  uint64_t q_full[kQStages];
+  uint64_t q_empty[kQStages];
+  uint64_t acc_full[2];
+  uint64_t acc_empty[2];
+  uint64_t drain;
+  uint32_t tmem_base;
+  int abort_flag;
+};
+
+constexpr size_t kSmemBytes = 1024 /*align slack*/ + size_t(kStages) * kOpStageBytes +
+                              size_t(kQStages) * kQStageBytes + sizeof(SmemCtl);
+
+struct Unit {
+  int e, nt, mb, rows, base;
+};
+
+__device__ __forceinline__ int total_units(const GemmArgs& a) { return __ldg(a.mb_prefix + a.E) * a.n_tiles; }
+
+__device__ __forceinline__ Unit decode_unit(const GemmArgs& a, int u) {
+  int lo = 0, hi = a.E;  // find e with mb_prefix[e]*nt <= u < mb_prefix[e+1]*nt
+  while (hi - lo > 1) {
+    const int mid = (lo + hi) >> 1;
+    if (__ldg(a.mb_prefix + mid) * a.n_tiles <= u) lo = mid;
+    else hi = mid;
+  }
+  Unit un;
+  un.e = lo;
+  const int p0 = __ldg(a.mb_prefix + lo);
+  const int nmb = __ldg(a.mb_prefix + lo + 1) - p0;
+  const int idx = u - p0 * a.n_tiles;
+  un.nt = idx / nmb;
+  un.mb = idx - un.nt * nmb;
+  const int o0 = __ldg(a.offsets + lo);
+  const int cnt = __ldg(a.offsets + lo + 1) - o0;
+  un.rows = min(kMBlock, cnt - un.mb * kMBlock);
+  un.base = o0 + un.mb * kMBlock;
+  return un;
+}
+
+struct Ring {
+  int stage = 0;
+  uint32_t phase = 0;
+  template <int N>
+  __device__ __forceinline__ void next() {
+    if (++stage == N) { stage = 0; phase ^= 1u; }
+  }
+};
+
+__device__ __forceinline__ uint32_t f16x2_sub(uint32_t a, uint32_t b) {
+  uint32_t d;
+  asm("sub.rn.f16x2 %0, %1, %2;" : "=r"(d) : "r"(a), "r"(b));
+  return d;
+}
+
+__device__ __forceinline__ uint32_t f16x2_mul(uint32_t a, uint32_t b) {
+  uint32_t d;
+  asm("mul.rn.f16x2 %0, %1, %2;" : "=r"(d) : "r"(a), "r"(b));
+  return d;
+}
+
+// 8 int4 codes (one storage word) -> 8 fp16 values q * s as a 16-byte chunk.
+// (n & 0xF) ^ 8 = q + 8 for a two's-complement nibble n, and 0x6400 | m is the
+// fp16 value 1024 + m, so one AND/XOR gives the pair (1032 + q); subtracting
+// 1032 is exact and q * s (3-bit code times 8-bit scale) is exact in fp16.
+__device__ __forceinline__ uint4 dequant_word(uint32_t w, uint32_t s2) {
+  const uint32_t k1032 = 0x64086408u;  // fp16 pair (1032, 1032)
+  uint32_t o[4];
+#pragma unroll
+  for (int i = 0; i < 4; ++i) {
+    const uint32_t v = ((w >> (4 * i)) & 0x000F000Fu) ^ 0x64086408u;  // fp16 pair 1032 + q
+    o[i] = f16x2_mul(f16x2_sub(v, k1032), s2);
+  }
+  return make_uint4(o[0], o[1], o[2], o[3]);
+}
+
+template <int MODE>
+__global__ void __launch_bounds__(kThreads, 1)
+    grouped_gemm_kernel(const GemmArgs a, const __grid_constant__ CUtensorMap tq0,
+                        const __grid_constant__ CUtensorMap tq1, const __grid_constant__ CUtensorMap ts0,
+                        const __grid_constant__ CUtensorMap ts1) {
+  constexpr bool kDequant = (MODE == GATEUP || MODE == DOWN);
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  uint8_t* op_base = smem;
+  uint8_t* q_base = smem + size_t(kStages) * kOpStageBytes;
+  SmemCtl* ctl = reinterpret_cast<SmemCtl*>(q_base + size_t(kQStages) * kQStageBytes);
+  volatile int* abort_flag = &ctl->abort_flag;
+
+  const int warp = threadIdx.x >> 5;
+  const int lane = threadIdx.x & 31;
+
+  if (threadIdx.x == 0) {
+    for (int i = 0; i < kStages; ++i) {
+      mbar_init(&ctl->op_full[i], 128 + 256);
+      mbar_init(&ctl->op_empty[i], 1);
+    }
+    for (int i = 0; i < kQStages; ++i) {
+      mbar_init(&ctl->q_full[i], 1);
+      mbar_init(&ctl->q_empty[i], 256);
+    }
+    for (int i = 0; i < 2; ++i) {
+      mbar_init(&ctl->acc_full[i], 1);
+      mbar_init(&ctl->acc_empty[i], 128);
+    }
+    mbar_init(&ctl->drain, 1);
+    ctl->abort_flag = 0;
+    fence_barrier_init();
+  }
+  if (warp == 4) {
+    tmem_alloc(&ctl->tmem_base, 512);
+    tmem_relinquish();
+  }
+  if (warp == 5 && lane == 0 && kDequant) {
+    prefetch_tmap(&tq0);
+    prefetch_tmap(&ts0);
+    if (MODE == GATEUP) {
+      prefetch_tmap(&tq1);
+      prefetch_tmap(&ts1);
+    }
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem_base = ctl->tmem_base;
+
+  const int nunits = total_units(a);
+  const int nkb = a.nkb_main + a.nkb_lora;
+
+  if (warp < 4) {
+    // ------------------------------------------------------------ epilogue
+    const int row_in_sub = warp * 32 + lane;
+    int it = 0;
+    for (int u = blockIdx.x; u < nunits; u += gridDim.x, ++it) {
+      const Unit un = decode_unit(a, u);
+      const int ab = it & 1;
+      const uint32_t aph = uint32_t(it >> 1) & 1u;
+      if (!mbar_wait(&ctl->acc_full[ab], aph, abort_flag, a.status)) break;
+      tc_fence_after();
+      const int nsub = un.rows > 128 ? 2 : 1;
+      for (int sub = 0; sub < nsub; ++sub) {
+        const int row = sub * 128 + row_in_sub;
+        const bool valid = row < un.rows;
+        const size_t grow = size_t(un.base) + row;
+        const uint32_t tacc = tmem_base + (uint32_t(warp * 32) << 16) + uint32_t(ab * 256 + sub * 128);
+        if (MODE == GATEUP) {
+          uint16_t* hrow = static_cast<uint16_t*>(a.out) + grow * a.out_ld + un.nt * 64;
+#pragma unroll 1
+          for (int c = 0; c < 64; c += 32) {
+            float gv[32], uv[32];
+            tmem_ld32(tacc + c, gv);
+            tmem_ld32(tacc + 64 + c, uv);
+            uint32_t pk[16];
+#pragma unroll
+            for (int i = 0; i < 16; ++i) {
+              const float g0 = gv[2 * i], g1 = gv[2 * i + 1];
+              const float h0 = g0 / (1.0f + __expf(-g0)) * uv[2 * i];
+              const float h1 = g1 / (1.0f + __expf(-g1)) * uv[2 * i + 1];
+              pk[i] = pack_f16x2(h0, h1);
+            }
+            if (valid) {
+              uint4* dst = reinterpret_cast<uint4*>(hrow + c);
+#pragma unroll
+              for (int i = 0; i < 4; ++i) dst[i] = make_uint4(pk[4 * i], pk[4 * i + 1], pk[4 * i + 2], pk[4 * i + 3]);
+            }
+          }
+        } else if (MODE == ROUTER) {
+          float* lrow = static_cast<float*>(a.out) + grow * a.out_ld;
+#pragma unroll 1
+          for (int c = 0; c < a.ntile; c += 32) {
+            float v[32];
+            tmem_ld32(tacc + c, v);
+            const int n0 = un.nt * a.ntile + c;
+            if (valid) {
+#pragma unroll
+              for (int i = 0; i < 32; ++i) {
+                const int n = n0 + i;
+                if (n < a.n_valid) lrow[n] = v[i] + (a.bias ? __ldg(a.bias + n) : 0.0f);
+              }
+            }
+          }
+        } else {
+          // DOWN / LORA_XA / LORA_HA: fp16 output, optional scale
+          const float sc = (MODE == DOWN) ? 1.0f : a.lora_scale;
+          uint16_t* orow = static_cast<uint16_t*>(a.out) + grow * a.out_ld + un.nt * a.ntile;
+#pragma unroll 1
+          for (int c = 0; c < a.ntile; c += 32) {
+            float v[32];
+            tmem_ld32(tacc + c, v);
+            uint32_t pk[16];
+#pragma unroll
+            for (int i = 0; i < 16; ++i) pk[i] = pack_f16x2(sc * v[2 * i], sc * v[2 * i + 1]);
+            if (valid) {
+              const int ncol = min(32, a.n_valid - (un.nt * a.ntile + c));
+              if (ncol >= 32) {
+                uint4* dst = reinterpret_cast<uint4*>(orow + c);
+#pragma unroll
+                for (int i = 0; i < 4; ++i)
+                  dst[i] = make_uint4(pk[4 * i], pk[4 * i + 1], pk[4 * i + 2], pk[4 * i + 3]);
+              } else {
+                for (int i = 0; i < ncol / 8; ++i)
+                  reinterpret_cast<uint4*>(orow + c)[i] =
+                      make_uint4(pk[4 * i], pk[4 * i + 1], pk[4 * i + 2], pk[4 * i + 3]);
+              }
+            }
+          }
+        }
+      }
+      tc_fence_before();
+      mbar_arrive(&ctl->acc_empty[ab]);
+    }
+  } else if (warp == 4) {
+    // ------------------------------------------------------------ MMA issuer
+    if (lane == 0) {
+      Ring ring;
+      int it = 0;
+      bool ok = true;
+      const uint32_t idesc = (MODE == ROUTER) ? idesc_bf16(128, a.ntile) : idesc_f16(128, a.ntile);
+      for (int u = blockIdx.x; u < nunits && ok; u += gridDim.x, ++it) {
+        const Unit un = decode_unit(a, u);
+        const int nsub = un.rows > 128 ? 2 : 1;
+        const int ab = it & 1;
+        const uint32_t aph = uint32_t(it >> 1) & 1u;
+        if (!mbar_wait(&ctl->acc_empty[ab], aph ^ 1u, abort_flag, a.status)) { ok = false; break; }
+        tc_fence_after();
+        for (int kb = 0; kb < nkb; ++kb) {
+          if (!mbar_wait(&ctl->op_full[ring.stage], ring.phase, abort_flag, a.status)) { ok = false; break; }
+          fence_proxy_async_smem();
+          tc_fence_after();
+          int ksteps = 4;
+          if (kb >= a.nkb_main) ksteps = (min(64, a.lora_k - (kb - a.nkb_main) * 64) + 15) / 16;
+          uint8_t* st = op_base + size_t(ring.stage) * kOpStageBytes;
+          const uint64_t bdesc = sdesc_k_sw128(smem_u32(st + kAStageBytes));
+          for (int sub = 0; sub < nsub; ++sub) {
+            const uint64_t adesc = sdesc_k_sw128(smem_u32(st + sub * 16384));
+            const uint32_t dt = tmem_base + uint32_t(ab * 256 + sub * 128);
+            for (int kk = 0; kk < ksteps; ++kk)
+              umma_bf16(dt, adesc + uint64_t(2 * kk), bdesc + uint64_t(2 * kk), idesc,
+                        (kb > 0 || kk > 0) ? 1u : 0u);
+          }
+          umma_commit(&ctl->op_empty[ring.stage]);
+          ring.next<kStages>();
+        }
+        if (!ok) break;
+        umma_commit(&ctl->acc_full[ab]);
+      }
+      // make sure no MMA is still writing TMEM before teardown
+      umma_commit(&ctl->drain);
+      mbar_wait(&ctl->drain, 0, abort_flag, a.status);
+    }
+    __syncwarp();
+  } else if (warp == 5) {
+    // ------------------------------------------------------------ TMA producer (int4 + scales)
+    if (kDequant && lane == 0) {
+      Ring q;
+      const int ngrp = a.g >= 64 ? 1 : 64 / a.g;
+      const int rows_box = (MODE == GATEUP) ? 64 : 128;
+      const uint32_t bytes = 4096u + uint32_t(ngrp * 128 * 2);
+      const int gpe = a.in_dim / a.g;  // scale rows per expert
+      int issued = 0;
+      uint32_t last_phase = 0;
+      int last_stage = 0;
+      for (int u = blockIdx.x; u < nunits; u += gridDim.x) {
+        const Unit un = decode_unit(a, u);
+        const int nrow0 = un.e * a.out_dim + un.nt * rows_box;
+        bool ok = true;
+        for (int kb = 0; kb < a.nkb_main; ++kb) {
+          if (!mbar_wait(&ctl->q_empty[q.stage], q.phase ^ 1u, abort_flag, a.status)) { ok = false; break; }
+          uint8_t* qs = q_base + size_t(q.stage) * kQStageBytes;
+          uint64_t* bar = &ctl->q_full[q.stage];
+          mbar_arrive_expect_tx(bar, bytes);
+          const int srow = un.e * gpe + (kb * 64) / a.g;
+          tma_load_2d(smem_u32(qs), &tq0, bar, kb * 32, nrow0);
+          tma_load_2d(smem_u32(qs + 4096), &ts0, bar, un.nt * rows_box, srow);
+          if (MODE == GATEUP) {
+            tma_load_2d(smem_u32(qs + 2048), &tq1, bar, kb * 32, nrow0);
+            tma_load_2d(smem_u32(qs + 4096 + ngrp * 128), &ts1, bar, un.nt * rows_box, srow);
+          }
+          ++issued;
+          last_stage = q.stage;
+          last_phase = q.phase;
+          q.next<kQStages>();
+        }
+        if (!ok) break;
+      }
+      // drain: wait until the last issued stage has landed (bounded)
+      if (issued > 0 && *abort_flag) mbar_wait(&ctl->q_full[last_stage], last_phase, abort_flag, a.status);
+    }
+  } else if (warp < 10) {
+    // ------------------------------------------------------------ A producer (cp.async)
+    const int tid = threadIdx.x - 6 * 32;  // 0..127
+    Ring ring;
+    CpAsyncLagArrive<2> lag;
+    for (int u = blockIdx.x; u < nunits; u += gridDim.x) {
+      const Unit un = decode_unit(a, u);
+      const uint16_t* src[2];
+      const uint16_t* lsrc[2];
+      bool valid[2];
+#pragma unroll
+      for (int sub = 0; sub < 2; ++sub) {
+        const int row = sub * 128 + tid;
+        valid[sub] = row < un.rows;
+        const int grow = un.base + (valid[sub] ? row : 0);
+        int srow = grow;
+        if (MODE == GATEUP || MODE == LORA_XA) srow = valid[sub] ? __ldg(a.perm_token + grow) : 0;
+        src[sub] = a.a_src + size_t(srow) * a.a_ld;
+        lsrc[sub] = a.a_lora ? a.a_lora + size_t(grow) * a.lora_ld : nullptr;
+      }
+      bool ok = true;
+      for (int kb = 0; kb < nkb; ++kb) {
+        if (!mbar_wait(&ctl->op_empty[ring.stage], ring.phase ^ 1u, abort_flag, a.status)) { ok = false; break; }
+        const uint32_t st = smem_u32(op_base + size_t(ring.stage) * kOpStageBytes);
+        if (kb < a.nkb_main) {
+          const int kcol = (MODE == ROUTER ? (kb % a.kb_per_piece) : kb) * 64;
+#pragma unroll
+          for (int sub = 0; sub < 2; ++sub) {
+            if (!valid[sub]) continue;
+            const uint16_t* p = src[sub] + kcol;
+#pragma unroll
+            for (int c = 0; c < 8; ++c) cp_async16(st + sub * 16384 + sw128_offset(tid, c), p + c * 8, 16);
+          }
+        } else {
+          const int lb = kb - a.nkb_main;
+#pragma unroll
+          for (int sub = 0; sub < 2; ++sub) {
+            if (!valid[sub]) continue;
+#pragma unroll
+            for (int c = 0; c < 8; ++c) {
+              const int col = lb * 64 + c * 8;
+              const bool in = col < a.lora_k;
+              cp_async16(st + sub * 16384 + sw128_offset(tid, c), lsrc[sub] + (in ? col : 0), in ? 16u : 0u);
+            }
+          }
+        }
+        lag.stage_done(&ctl->op_full[ring.stage]);
+        ring.next<kStages>();
+      }
+      if (!ok) break;
+    }
+    lag.flush();
+  } else {
+    // ------------------------------------------------------------ B producer
+    const int tid = threadIdx.x - 10 * 32;  // 0..255
+    const int row = tid >> 1;               // 0..127
+    const int half = tid & 1;
+    Ring ring, q;
+    CpAsyncLagArrive<2> lag;
+    for (int u = blockIdx.x; u < nunits; u += gridDim.x) {
+      const Unit un = decode_unit(a, u);
+      bool ok = true;
+      for (int kb = 0; kb < nkb; ++kb) {
+        if (!mbar_wait(&ctl->op_empty[ring.stage], ring.phase ^ 1u, abort_flag, a.status)) { ok = false; break; }
+        uint8_t* bst = op_base + size_t(ring.stage) * kOpStageBytes + kAStageBytes;
+        const uint32_t bst_u = smem_u32(bst);
+        if (kDequant && kb < a.nkb_main) {
+          if (!mbar_wait(&ctl->q_full[q.stage], q.phase, abort_flag, a.status)) { ok = false; break; }
+          const uint8_t* qs = q_base + size_t(q.stage) * kQStageBytes;
+          const uint4 words = *reinterpret_cast<const uint4*>(qs + row * 32 + half * 16);
+          const int ngrp = a.g >= 64 ? 1 : 64 / a.g;
+          const int gl = (a.g == 32) ? half : 0;
+          const uint16_t* sc = reinterpret_cast<const uint16_t*>(qs + 4096);
+          uint16_t sbits;
+          if (MODE == GATEUP) {
+            const int blk = row >> 6;
+            sbits = sc[blk * ngrp * 64 + gl * 64 + (row & 63)];
+          } else {
+            sbits = sc[gl * 128 + row];
+          }
+          const uint32_t sh = __half_as_ushort(__float2half_rn(bf16_to_f32(sbits)));
+          const uint32_t s2 = sh | (sh << 16);
+          const uint32_t wv[4] = {words.x, words.y, words.z, words.w};
+#pragma unroll
+          for (int i = 0; i < 4; ++i) {
+            const uint4 v = dequant_word(wv[i], s2);
+            *reinterpret_cast<uint4*>(bst + sw128_offset(row, half * 4 + i)) = v;
+          }
+          // The ring slot is handed back only after its values were consumed and
+          // a proxy fence ordered these generic-proxy reads (and the B-tile writes)
+          // before the async-proxy accesses that follow: the next TMA fill of the
+          // slot and the tensor-core reads of the B tile.
+          fence_proxy_async_smem();
+          mbar_arrive(&ctl->q_empty[q.stage]);
+          q.next<kQStages>();
+          mbar_arrive(&ctl->op_full[ring.stage]);
+        } else if (kDequant) {
+          // LoRA B^T tile: K' columns [lb*64, lb*64 + 64) of the rank space
+          const int lb = kb - a.nkb_main;
+#pragma unroll
+          for (int i = 0; i < 4; ++i) {
+            const int c = half * 4 + i;
+            const int col = lb * 64 + c * 8;
+            uint4 v = make_uint4(0, 0, 0, 0);
+            if (MODE == GATEUP) {
+              const int n = un.nt * 64 + (row & 63);
+              if (row < 64) {
+                if (col < a.r) v = __ldg(reinterpret_cast<const uint4*>(a.b0 + (size_t(un.e) * a.out_dim + n) * a.r + col));
+              } else {
+                if (col >= a.r && col < 2 * a.r)
+                  v = __ldg(reinterpret_cast<const uint4*>(a.b1 + (size_t(un.e) * a.out_dim + n) * a.r + (col - a.r)));
+              }
+            } else {
+              const int n = un.nt * 128 + row;
+              if (col < a.r) v = __ldg(reinterpret_cast<const uint4*>(a.b0 + (size_t(un.e) * a.out_dim + n) * a.r + col));
+            }
+            *reinterpret_cast<uint4*>(bst + sw128_offset(row, c)) = bf16x8_to_f16x8(v);
+          }
+          fence_proxy_async_smem();
+          mbar_arrive(&ctl->op_full[ring.stage]);
+        } else if (MODE == LORA_XA || MODE == LORA_HA) {
+          // rank-space B^T = A^T rows (bf16 in memory) -> fp16 tile rows [0, ntile)
+          if (row < a.ntile) {
+            const uint16_t* p = nullptr;
+            if (MODE == LORA_XA) {
+              if (row < a.r) p = a.b0 + (size_t(un.e) * a.r + row) * a.a_ld;
+              else if (row < 2 * a.r) p = a.b1 + (size_t(un.e) * a.r + (row - a.r)) * a.a_ld;
+            } else if (row < a.r) {
+              p = a.b0 + (size_t(un.e) * a.r + row) * a.a_ld;
+            }
+#pragma unroll
+            for (int i = 0; i < 4; ++i) {
+              const int c = half * 4 + i;
+              uint4 v = make_uint4(0, 0, 0, 0);
+              if (p) v = bf16x8_to_f16x8(__ldg(reinterpret_cast<const uint4*>(p + kb * 64 + c * 8)));
+              *reinterpret_cast<uint4*>(bst + sw128_offset(row, c)) = v;
+            }
+          }
+          fence_proxy_async_smem();
+          mbar_arrive(&ctl->op_full[ring.stage]);
+        } else {
+          // ROUTER: bf16 parts of W_r, rows [0, ntile) x 64 K, via cp.async (zero-filled padding)
+          if (row < a.ntile) {
+            const uint16_t* p = nullptr;
+            const int n = un.nt * a.ntile + row;
+            const int piece = kb / a.kb_per_piece;
+            const int kcol = (kb % a.kb_per_piece) * 64;
+            if (n < a.n_valid) p = a.b0 + (size_t(piece) * a.n_valid + n) * a.a_ld;
+#pragma unroll
+            for (int i = 0; i < 4; ++i) {
+              const int c = half * 4 + i;
+              cp_async16(bst_u + sw128_offset(row, c), p ? p + kcol + c * 8 : a.a_src, p ? 16u : 0u);
+            }
+          }
+          lag.stage_done(&ctl->op_full[ring.stage]);
+        }
+        ring.next<kStages>();
+      }
+      if (!ok) break;
+    }
+    lag.flush();
+  }
+
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 4) {
+    tc_fence_after();
+    tmem_dealloc(tmem_base, 512);
+  }
+}
+
+// ----------------------------------------------------------------------------
+// small helper kernels
+// ----------------------------------------------------------------------------
+
+// mb_prefix[e] = sum_{e' < e} ceil(count(e') / 256), one block.
+__global__ void schedule_kernel(const int32_t* __restrict__ offsets, int E, int32_t* __restrict__ mb_prefix) {
+  __shared__ int32_t warp_sums[32];
+  const int nt = blockDim.x;
+  const int per = (E + nt - 1) / nt;
+  const int lo = threadIdx.x * per;
+  const int hi = min(E, lo + per);
+  int local = 0;
+  for (int e = lo; e < hi; ++e) local += (offsets[e + 1] - offsets[e] + kMBlock - 1) / kMBlock;
+  const int lane = threadIdx.x & 31, wid = threadIdx.x >> 5;
+  int v = local;
+#pragma unroll
+  for (int o = 1; o < 32; o <<= 1) {
+    const int u = __shfl_up_sync(0xFFFFFFFFu, v, o);
+    if (lane >= o) v += u;
+  }
+  if (lane == 31) warp_sums[wid] = v;
+  __syncthreads();
+  if (wid == 0) {
+    int s = (lane < (nt >> 5)) ? warp_sums[lane] : 0;
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+      const int u = __shfl_up_sync(0xFFFFFFFFu, s, o);
+      if (lane >= o) s += u;
+    }
+    if (lane < (nt >> 5)) warp_sums[lane] = s;
+  }
+  __syncthreads();
+  int run = v - local + (wid > 0 ? warp_sums[wid - 1] : 0);
+  for (int e = lo; e < hi; ++e) {
+    mb_prefix[e] = run;
+    run += (offsets[e + 1] - offsets[e] + kMBlock - 1) / kMBlock;
+  }
+  if (threadIdx.x == nt - 1) mb_prefix[E] = run;
+}
+
+// Token activations bf16 -> fp16 (the operand type of the expert contractions);
+// values beyond the fp16 range raise TQP_STATUS_NONFINITE.
+__global__ void x_to_f16_kernel(const uint16_t* __restrict__ x, uint16_t* __restrict__ x16, size_t n8,
+                                int32_t* status) {
+  const size_t i = size_t(blockIdx.x) * blockDim.x + threadIdx.x;
+  if (i >= n8) return;
+  const uint4 v = __ldg(reinterpret_cast<const uint4*>(x) + i);
+  const uint4 o = bf16x8_to_f16x8(v);
+  reinterpret_cast<uint4*>(x16)[i] = o;
+  const uint32_t w[4] = {o.x, o.y, o.z, o.w};
+  bool bad = false;
+#pragma unroll
+  for (int j = 0; j < 4; ++j) bad |= ((w[j] & 0x7C00u) == 0x7C00u) || ((w[j] & 0x7C000000u) == 0x7C000000u);
+  if (bad) raise_status(status, TQP_STATUS_NONFINITE);
+}
+
+// Router: one group covering all T tokens; split W_r into three exact bf16 parts.
+__global__ void router_prep_kernel(const float* __restrict__ wr, int n, int T, uint16_t* __restrict__ parts,
+                                   int32_t* __restrict__ offsets2, int32_t* __restrict__ mbp2) {
+  const int i = blockIdx.x * blockDim.x + threadIdx.x;
+  if (i == 0) {
+    offsets2[0] = 0;
+    offsets2[1] = T;
+    mbp2[0] = 0;
+    mbp2[1] = (T + kMBlock - 1) / kMBlock;
+  }
+  if (i >= n) return;
+  const float w = wr[i];
+  const uint16_t hi = f32_to_bf16(w);
+  const float r1 = w - bf16_to_f32(hi);
+  const uint16_t mid = f32_to_bf16(r1);
+  const float r2 = r1 - bf16_to_f32(mid);
+  const uint16_t lo = f32_to_bf16(r2);
+  parts[i] = hi;
+  parts[size_t(n) + i] = mid;
+  parts[2 * size_t(n) + i] = lo;
+}
+
+// ----------------------------------------------------------------------------
+// host side
+// ----------------------------------------------------------------------------
+
+static PFN_cuTensorMapEncodeTiled_v12000 encode_fn() {
+  static PFN_cuTensorMapEncodeTiled_v12000 fn = nullptr;
+  if (!fn) {
+    void* p = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) == cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(p);
+  }
+  return fn;
+}
+
+static bool make_map(CUtensorMap* m, CUtensorMapDataType dt, const void* ptr, uint64_t inner, uint64_t outer,
+                     uint64_t row_bytes, uint32_t box_inner, uint32_t box_outer) {
+  auto fn = encode_fn();
+  if (!fn) return false;
+  cuuint64_t dims[2] = {inner, outer};
+  cuuint64_t strides[1] = {row_bytes};
+  cuuint32_t box[2] = {box_inner, box_outer};
+  cuuint32_t estr[2] = {1, 1};
+  return fn(m, dt, 2, const_cast<void*>(ptr), dims, strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
+            CU_TENSOR_MAP_SWIZZLE_NONE, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+            CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+int num_sms() {
+  int dev = 0, n = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess) return 148;
+  if (cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess || n <= 0) return 148;
+  return n;
+}
+
+template <int MODE>
+static int run_gemm(const GemmArgs& a, const CUtensorMap* maps, int units_upper, cudaStream_t s) {
+  static bool attr_set = false;
+  if (!attr_set) {
+    if (cudaFuncSetAttribute(grouped_gemm_kernel<MODE>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                             int(kSmemBytes)) != cudaSuccess)
+      return TQP_ERR_CUDA;
+    attr_set = true;
+  }
+  const int grid = units_upper < num_sms() ? (units_upper > 0 ? units_upper : 1) : num_sms();
+  grouped_gemm_kernel<MODE><<<grid, kThreads, kSmemBytes, s>>>(a, maps[0], maps[1], maps[2], maps[3]);
+  return cudaGetLastError() == cudaSuccess ? TQP_OK : TQP_ERR_CUDA;
+}
+
+size_t router_ws_bytes(int T, const tqp_moe_weights* w) {
+  (void)T;
+  return align_up(size_t(3) * w->E * w->d * 2, 256) + 256;
+}
+
+int launch_router_gemm(const uint16_t* x, int T, const tqp_moe_weights* w, float* logits, void* ws,
+                       int32_t* status, cudaStream_t s) {
+  if (T == 0) return TQP_OK;
+  uint16_t* parts = static_cast<uint16_t*>(ws);
+  int32_t* ctl = reinterpret_cast<int32_t*>(static_cast<char*>(ws) + align_up(size_t(3) * w->E * w->d * 2, 256));
+  const int n = w->E * w->d;
+  router_prep_kernel<<<(n + 255) / 256, 256, 0, s>>>(w->router_w, n, T, parts, ctl, ctl + 2);
+  GemmArgs a{};
+  a.E = 1;
+  a.kb_per_piece = w->d / 64;
+  a.nkb_main = 3 * a.kb_per_piece;
+  a.nkb_lora = 0;
+  a.lora_k = 0;
+  a.ntile = 128;
+  a.n_tiles = (w->E + 127) / 128;
+  a.g = 64;
+  a.offsets = ctl;
+  a.mb_prefix = ctl + 2;
+  a.perm_token = nullptr;
+  a.a_src = x;
+  a.a_ld = w->d;
+  a.b0 = parts;
+  a.out = logits;
+  a.out_ld = w->E;
+  a.n_valid = w->E;
+  a.bias = w->router_bias;
+  a.status = status;
+  CUtensorMap maps[4];
+  memset(maps, 0, sizeof(maps));
+  const int units = ((T + kMBlock - 1) / kMBlock) * a.n_tiles;
+  return run_gemm<ROUTER>(a, maps, units, s);
+}
+
+size_t ffn_ws_bytes(int T, const tqp_moe_weights* w) {
+  const size_t A = size_t(T) * w->top_k;
+  size_t b = align_up(size_t(w->E + 1) * 4, 256);              // mb_prefix
+  b += align_up(size_t(T) * w->d * 2, 256);                    // x in fp16
+  if (w->rank > 0) {
+    b += align_up(A * 2 * w->rank * 2, 256);                    // xa [A][2r]
+    b += align_up(A * w->rank * 2, 256);                        // ha [A][r]
+  }
+  return b + 256;
+}
+
+int launch_grouped_ffn(const uint16_t* x, int T, const int32_t* offsets, const int32_t* perm_token,
+                       const tqp_moe_weights* w, uint16_t* h, uint16_t* out_perm, void* ws, int32_t* status,
+                       cudaStream_t s) {
+  if (T == 0) return TQP_OK;
+  const size_t A = size_t(T) * w->top_k;
+  char* p = static_cast<char*>(ws);
+  int32_t* mb_prefix = reinterpret_cast<int32_t*>(p);
+  p += align_up(size_t(w->E + 1) * 4, 256);
+  uint16_t* x16 = reinterpret_cast<uint16_t*>(p);
+  p += align_up(size_t(T) * w->d * 2, 256);
+  uint16_t* xa = nullptr;
+  uint16_t* ha = nullptr;
+  if (w->rank > 0) {
+    xa = reinterpret_cast<uint16_t*>(p);
+    p += align_up(A * 2 * w->rank * 2, 256);
+    ha = reinterpret_cast<uint16_t*>(p);
+  }
+  schedule_kernel<<<1, 1024, 0, s>>>(offsets, w->E, mb_prefix);
+  {
+    const size_t n8 = size_t(T) * w->d / 8;
+    x_to_f16_kernel<<<unsigned((n8 + 255) / 256), 256, 0, s>>>(x, x16, n8, status);
+  }
+  if (cudaGetLastError() != cudaSuccess) return TQP_ERR_CUDA;
+  // an upper bound on the number of work units (grid sizing only)
+  const int mb_upper = int((A + kMBlock - 1) / kMBlock) + w->E;
+  const int d = w->d, f = w->ffn, r = w->rank;
+
+  GemmArgs base{};
+  base.E = w->E;
+  base.g = w->group;
+  base.r = r;
+  base.lora_scale = w->lora_scale;
+  base.offsets = offsets;
+  base.mb_prefix = mb_prefix;
+  base.perm_token = perm_token;
+  base.status = status;
+  base.kb_per_piece = 1;
+  int rc;
+  CUtensorMap maps[4];
+  memset(maps, 0, sizeof(maps));
+
+  if (r > 0) {  // xa = s * X [Ag | Au]
+    GemmArgs a = base;
+    a.nkb_main = d / 64;
+    a.ntile = 2 * r;
+    a.n_tiles = 1;
+    a.a_src = x16;
+    a.a_ld = d;
+    a.b0 = w->lora_a[0];
+    a.b1 = w->lora_a[1];
+    a.out = xa;
+    a.out_ld = 2 * r;
+    a.n_valid = 2 * r;
+    if ((rc = run_gemm<LORA_XA>(a, maps, mb_upper, s)) != TQP_OK) return rc;
+  }
+  {  // H = silu(G) * U
+    GemmArgs a = base;
+    a.nkb_main = d / 64;
+    a.nkb_lora = r > 0 ? (2 * r + 63) / 64 : 0;
+    a.lora_k = 2 * r;
+    a.ntile = 128;
+    a.n_tiles = f / 64;
+    a.in_dim = d;
+    a.out_dim = f;
+    a.a_src = x16;
+    a.a_ld = d;
+    a.a_lora = xa;
+    a.lora_ld = 2 * r;
+    a.b0 = w->lora_b[0];
+    a.b1 = w->lora_b[1];
+    a.wq0 = w->wq[0];
+    a.wq1 = w->wq[1];
+    a.ws0 = w->wscale[0];
+    a.ws1 = w->wscale[1];
+    a.out = h;
+    a.out_ld = f;
+    a.n_valid = f;
+    const int ngrp = w->group >= 64 ? 1 : 64 / w->group;
+    bool ok = make_map(&maps[0], CU_TENSOR_MAP_DATA_TYPE_UINT8, w->wq[0], d / 2, uint64_t(w->E) * f, d / 2, 32, 64) &&
+              make_map(&maps[1], CU_TENSOR_MAP_DATA_TYPE_UINT8, w->wq[1], d / 2, uint64_t(w->E) * f, d / 2, 32, 64) &&
+              make_map(&maps[2], CU_TENSOR_MAP_DATA_TYPE_UINT16, w->wscale[0], f, uint64_t(w->E) * (d / w->group),
+                       uint64_t(f) * 2, 64, ngrp) &&
+              make_map(&maps[3], CU_TENSOR_MAP_DATA_TYPE_UINT16, w->wscale[1], f, uint64_t(w->E) * (d / w->group),
+                       uint64_t(f) * 2, 64, ngrp);
+    if (!ok) return TQP_ERR_CUDA;
+    if ((rc = run_gemm<GATEUP>(a, maps, mb_upper * a.n_tiles, s)) != TQP_OK) return rc;
+  }
+  if (r > 0) {  // ha = s * H Ad
+    GemmArgs a = base;
+    memset(maps, 0, sizeof(maps));
+    a.nkb_main = f / 64;
+    a.ntile = r < 16 ? 16 : r;
+    a.n_tiles = 1;
+    a.a_src = h;
+    a.a_ld = f;
+    a.b0 = w->lora_a[2];
+    a.out = ha;
+    a.out_ld = r;
+    a.n_valid = r;
+    if ((rc = run_gemm<LORA_HA>(a, maps, mb_upper, s)) != TQP_OK) return rc;
+  }
+  {  // O = H Wd^T + (s H Ad) Bd
+    GemmArgs a = base;
+    a.nkb_main = f / 64;
+    a.nkb_lora = r > 0 ? (r + 63) / 64 : 0;
+    a.lora_k = r;
+    a.ntile = 128;
+    a.n_tiles = d / 128;
+    a.in_dim = f;
+    a.out_dim = d;
+    a.a_src = h;
+    a.a_ld = f;
+    a.a_lora = ha;
+    a.lora_ld = r;
+    a.b0 = w->lora_b[2];
+    a.wq0 = w->wq[2];
+    a.ws0 = w->wscale[2];
+    a.out = out_perm;
+    a.out_ld = d;
+    a.n_valid = d;
+    const int ngrp = w->group >= 64 ? 1 : 64 / w->group;
+    bool ok = make_map(&maps[0], CU_TENSOR_MAP_DATA_TYPE_UINT8, w->wq[2], f / 2, uint64_t(w->E) * d, f / 2, 32, 128) &&
+              make_map(&maps[2], CU_TENSOR_MAP_DATA_TYPE_UINT16, w->wscale[2], d, uint64_t(w->E) * (f / w->group),
+                       uint64_t(d) * 2, 128, ngrp);
+    maps[1] = maps[0];
+    maps[3] = maps[2];
+    if (!ok) return TQP_ERR_CUDA;
+    if ((rc = run_gemm<DOWN>(a, maps, mb_upper * a.n_tiles, s)) != TQP_OK) return rc;
+  }
+  return TQP_OK;
+}
+
+}  // namespace tqp

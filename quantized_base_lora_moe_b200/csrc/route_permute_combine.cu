@@ -1,0 +1,344 @@
+// Routing, permutation and combine kernels of the TQP MoE layer (sm_100a).
+//
+//  moe_route    : one warp per token; top-k by repeated warp arg-max on a 64-bit
+//                 key (orderable logit, then lower expert id), renormalised
+//                 softmax over the chosen logits ("Top-12 routing",
+//                 Architecture Details; stateless routing, Reversibility
+//                 Implementation).
+//  moe_permute  : stable counting sort by expert in three passes: per 32-token
+//                 chunk expert bitmaps -> per-expert column prefix over chunks
+//                 -> scatter with rank = popcount of earlier tokens' bits.
+//  moe_combine  : gate-weighted gather back to token order (fixed j order, fp32,
+//                 no atomics) with the additive coupling fused in ("Pattern 1":
+//                 addition/subtraction are invertible).
+#include <cstdint>
+#include <cuda_runtime.h>
+
+#include "tqp_device.cuh"
+#include "tqp_launch.h"
+
+namespace tqp {
+
+// ----------------------------------------------------------------------------
+// moe_route
+// ----------------------------------------------------------------------------
+
+// Orderable key: larger key = larger logit; +0.0 == -0.0; NaN lowest.
+__device__ __forceinline__ uint32_t logit_key(float v) {
+  if (v != v) return 0u;
+  if (v == 0.0f) v = 0.0f;
+  const uint32_t b = __float_as_uint(v);
+  return (b & 0x80000000u) ? (~b) : (b | 0x80000000u);
+}
+
+__device__ __forceinline__ uint64_t pack_key(float v, int e) {
+  return (uint64_t(logit_key(v)) << 32) | uint64_t(0xFFFFFFFFu - uint32_t(e));
+}
+
+__device__ __forceinline__ uint64_t warp_max_u64(uint64_t v) {
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) {
+    const uint64_t w = __shfl_xor_sync(0xFFFFFFFFu, v, o);
+    v = w > v ? w : v;
+  }
+  return v;
+}
+
+template <int EPL>  // logits per lane kept in registers (E <= 32 * EPL)
+__global__ void __launch_bounds__(256) route_kernel(const float* __restrict__ logits, int T, int E, int k,
+                                                    int32_t* __restrict__ ids, float* __restrict__ gates,
+                                                    int32_t* status) {
+  const int lane = threadIdx.x & 31;
+  const int t = blockIdx.x * (blockDim.x >> 5) + (threadIdx.x >> 5);
+  if (t >= T) return;
+  const float* row = logits + size_t(t) * E;
+  uint64_t key[EPL];
+  bool nonfinite = false;
+#pragma unroll
+  for (int i = 0; i < EPL; ++i) {
+    const int e = lane + 32 * i;
+    if (e < E) {
+      const float v = __ldg(row + e);
+      nonfinite |= !isfinite(v);
+      key[i] = pack_key(v, e);
+    } else {
+      key[i] = 0ull;  // below every real entry (a real key has a non-zero low word)
+    }
+  }
+  if (__any_sync(0xFFFFFFFFu, nonfinite) && lane == 0) raise_status(status, TQP_STATUS_NONFINITE);
+
+  uint64_t bound = ~0ull;
+  int my_id = 0;
+  float my_val = 0.0f;
+  for (int j = 0; j < k; ++j) {
+    uint64_t best = 0ull;
+#pragma unroll
+    for (int i = 0; i < EPL; ++i) best = (key[i] < bound && key[i] > best) ? key[i] : best;
+    best = warp_max_u64(best);
+    bound = best;
+    if (lane == j) {
+      my_id = int(0xFFFFFFFFu - uint32_t(best & 0xFFFFFFFFull));
+      my_val = __ldg(row + my_id);
+    }
+  }
+  const float m = __shfl_sync(0xFFFFFFFFu, my_val, 0);
+  float ex = (lane < k) ? expf(my_val - m) : 0.0f;
+  float sum = ex;
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) sum += __shfl_xor_sync(0xFFFFFFFFu, sum, o);
+  if (lane < k) {
+    ids[size_t(t) * k + lane] = my_id;
+    gates[size_t(t) * k + lane] = ex / sum;
+  }
+}
+
+int launch_route(const float* logits, int T, int E, int k, int32_t* ids, float* gates, int32_t* status,
+                 cudaStream_t s) {
+  if (T == 0) return TQP_OK;
+  const dim3 block(256);
+  const dim3 grid((T + 7) / 8);
+  const int epl = (E + 31) / 32;
+#define TQP_ROUTE(N) route_kernel<N><<<grid, block, 0, s>>>(logits, T, E, k, ids, gates, status)
+  if (epl <= 1) TQP_ROUTE(1);
+  else if (epl <= 2) TQP_ROUTE(2);
+  else if (epl <= 4) TQP_ROUTE(4);
+  else if (epl <= 8) TQP_ROUTE(8);
+  else if (epl <= 16) TQP_ROUTE(16);
+  else if (epl <= 32) TQP_ROUTE(32);
+  else if (epl <= 64) TQP_ROUTE(64);
+  else TQP_ROUTE(128);
+#undef TQP_ROUTE
+  return cudaGetLastError() == cudaSuccess ? TQP_OK : TQP_ERR_CUDA;
+}
+
+// ----------------------------------------------------------------------------
+// moe_permute
+// ----------------------------------------------------------------------------
+
+// Pass 1: per 32-token chunk w, count[w][e] = #tokens of the chunk routed to e.
+__global__ void permute_count_kernel(const int32_t* __restrict__ ids, int T, int E, int k,
+                                     int32_t* __restrict__ count, int32_t* status) {
+  extern __shared__ uint32_t bits_all[];
+  const int lane = threadIdx.x & 31;
+  const int wib = threadIdx.x >> 5;
+  const int w = blockIdx.x * (blockDim.x >> 5) + wib;
+  const int W = (T + 31) / 32;
+  if (w >= W) return;
+  uint32_t* bits = bits_all + size_t(wib) * E;
+  for (int e = lane; e < E; e += 32) bits[e] = 0u;
+  __syncwarp();
+  const int t = w * 32 + lane;
+  bool bad = false;
+  if (t < T) {
+    for (int j = 0; j < k; ++j) {
+      const int e = ids[size_t(t) * k + j];
+      if (e >= 0 && e < E) atomicOr(&bits[e], 1u << lane);
+      else bad = true;
+    }
+  }
+  if (__any_sync(0xFFFFFFFFu, bad) && lane == 0) raise_status(status, TQP_STATUS_BAD_ID);
+  __syncwarp();
+  for (int e = lane; e < E; e += 32) count[size_t(w) * E + e] = __popc(bits[e]);
+}
+
+// Pass 2: one thread per expert: exclusive prefix of count[.][e] over chunks
+// (in place) and the expert total.
+__global__ void permute_colscan_kernel(int32_t* __restrict__ count, int W, int E, int32_t* __restrict__ total) {
+  const int e = blockIdx.x * blockDim.x + threadIdx.x;
+  if (e >= E) return;
+  int run = 0;
+  for (int w = 0; w < W; ++w) {
+    const size_t i = size_t(w) * E + e;
+    const int c = count[i];
+    count[i] = run;
+    run += c;
+  }
+  total[e] = run;
+}
+
+// Block-wide exclusive scan of total[0..E) into off[0..E] (shared memory).
+__device__ void block_exclusive_scan(const int32_t* __restrict__ total, int E, int32_t* off, int32_t* warp_sums) {
+  const int nt = blockDim.x;
+  const int per = (E + nt - 1) / nt;
+  const int lo = threadIdx.x * per;
+  const int hi = min(E, lo + per);
+  int local = 0;
+  for (int e = lo; e < hi; ++e) local += total[e];
+  // inclusive warp scan of the per-thread sums
+  const int lane = threadIdx.x & 31, wid = threadIdx.x >> 5;
+  int v = local;
+#pragma unroll
+  for (int o = 1; o < 32; o <<= 1) {
+    const int u = __shfl_up_sync(0xFFFFFFFFu, v, o);
+    if (lane >= o) v += u;
+  }
+  if (lane == 31) warp_sums[wid] = v;
+  __syncthreads();
+  if (wid == 0) {
+    int s = (lane < (nt >> 5)) ? warp_sums[lane] : 0;
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+      const int u = __shfl_up_sync(0xFFFFFFFFu, s, o);
+      if (lane >= o) s += u;
+    }
+    if (lane < (nt >> 5)) warp_sums[lane] = s;  // inclusive
+  }
+  __syncthreads();
+  int run = v - local + (wid > 0 ? warp_sums[wid - 1] : 0);
+  for (int e = lo; e < hi; ++e) {
+    off[e] = run;
+    run += total[e];
+  }
+  if (threadIdx.x == nt - 1) off[E] = run;
+  __syncthreads();
+}
+
+// Pass 3: scatter. Row of (t, j) with expert e = offsets[e] + prefix[w][e] +
+// #earlier tokens of the chunk routed to e.
+__global__ void permute_scatter_kernel(const int32_t* __restrict__ ids, int T, int E, int k,
+                                       const int32_t* __restrict__ prefix, const int32_t* __restrict__ total,
+                                       int32_t* __restrict__ offsets, int32_t* __restrict__ perm_token,
+                                       int32_t* __restrict__ inv, int warps_per_block) {
+  extern __shared__ int32_t smem_i[];
+  int32_t* off = smem_i;                       // E + 1
+  int32_t* warp_sums = smem_i + E + 1;         // 32
+  uint32_t* bits_all = reinterpret_cast<uint32_t*>(smem_i + E + 1 + 32);
+  block_exclusive_scan(total, E, off, warp_sums);
+  if (blockIdx.x == 0)
+    for (int e = threadIdx.x; e <= E; e += blockDim.x) offsets[e] = off[e];
+
+  const int lane = threadIdx.x & 31;
+  const int wib = threadIdx.x >> 5;
+  const int w = blockIdx.x * warps_per_block + wib;
+  const int W = (T + 31) / 32;
+  if (w >= W) return;
+  uint32_t* bits = bits_all + size_t(wib) * E;
+  for (int e = lane; e < E; e += 32) bits[e] = 0u;
+  __syncwarp();
+  const int t = w * 32 + lane;
+  if (t < T) {
+    for (int j = 0; j < k; ++j) {
+      const int e = ids[size_t(t) * k + j];
+      if (e >= 0 && e < E) atomicOr(&bits[e], 1u << lane);
+    }
+  }
+  __syncwarp();
+  if (t < T) {
+    const uint32_t lt = (1u << lane) - 1u;
+    for (int j = 0; j < k; ++j) {
+      const int e = ids[size_t(t) * k + j];
+      if (e < 0 || e >= E) continue;
+      const int row = off[e] + prefix[size_t(w) * E + e] + __popc(bits[e] & lt);
+      perm_token[row] = t;
+      inv[size_t(t) * k + j] = row;
+    }
+  }
+}
+
+size_t permute_ws_bytes(int T, int E) {
+  const size_t W = (size_t(T) + 31) / 32;
+  return align_up(W * E * 4, 256) + align_up(size_t(E) * 4, 256);
+}
+
+int launch_permute(const int32_t* ids, int T, int E, int k, int32_t* offsets, int32_t* perm_token, int32_t* inv,
+                   void* ws, int32_t* status, cudaStream_t s) {
+  if (T == 0) {
+    return cudaMemsetAsync(offsets, 0, sizeof(int32_t) * (E + 1), s) == cudaSuccess ? TQP_OK : TQP_ERR_CUDA;
+  }
+  const int W = (T + 31) / 32;
+  int32_t* count = static_cast<int32_t*>(ws);
+  int32_t* total = reinterpret_cast<int32_t*>(static_cast<char*>(ws) + align_up(size_t(W) * E * 4, 256));
+  // pass 1
+  int wpb = 8;
+  while (wpb > 1 && size_t(wpb) * E * 4 > 64 * 1024) wpb >>= 1;
+  const size_t smem1 = size_t(wpb) * E * 4;
+  if (smem1 > 48 * 1024) cudaFuncSetAttribute(permute_count_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, int(smem1));
+  permute_count_kernel<<<(W + wpb - 1) / wpb, wpb * 32, smem1, s>>>(ids, T, E, k, count, status);
+  // pass 2
+  permute_colscan_kernel<<<(E + 127) / 128, 128, 0, s>>>(count, W, E, total);
+  // pass 3
+  const size_t smem3 = size_t(E + 1 + 32) * 4 + size_t(wpb) * E * 4;
+  if (smem3 > 48 * 1024)
+    cudaFuncSetAttribute(permute_scatter_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, int(smem3));
+  permute_scatter_kernel<<<(W + wpb - 1) / wpb, wpb * 32, smem3, s>>>(ids, T, E, k, count, total, offsets,
+                                                                      perm_token, inv, wpb);
+  return cudaGetLastError() == cudaSuccess ? TQP_OK : TQP_ERR_CUDA;
+}
+
+// ----------------------------------------------------------------------------
+// moe_combine
+// ----------------------------------------------------------------------------
+
+// One block per token row; each thread owns 8 consecutive columns (16 B of bf16).
+__global__ void __launch_bounds__(256) combine_kernel(const uint16_t* __restrict__ out_perm,
+                                                      const int32_t* __restrict__ inv,
+                                                      const float* __restrict__ gates, int T, int k, int d,
+                                                      const void* __restrict__ residual, int residual_f32,
+                                                      float sign, void* __restrict__ y, int y_f32,
+                                                      uint16_t* __restrict__ y_bf16) {
+  const int t = blockIdx.x;
+  const int c0 = threadIdx.x * 8;
+  for (int c = c0; c < d; c += blockDim.x * 8) {
+    float acc[8];
+#pragma unroll
+    for (int i = 0; i < 8; ++i) acc[i] = 0.0f;
+    for (int j = 0; j < k; ++j) {
+      const int row = __ldg(inv + size_t(t) * k + j);
+      const float gmm = __ldg(gates + size_t(t) * k + j);
+      const uint4 v = __ldg(reinterpret_cast<const uint4*>(out_perm + size_t(row) * d + c));
+      const uint32_t w[4] = {v.x, v.y, v.z, v.w};
+#pragma unroll
+      for (int i = 0; i < 4; ++i) {
+        acc[2 * i] = fmaf(gmm, f16_to_f32(uint16_t(w[i] & 0xFFFFu)), acc[2 * i]);
+        acc[2 * i + 1] = fmaf(gmm, f16_to_f32(uint16_t(w[i] >> 16)), acc[2 * i + 1]);
+      }
+    }
+    float out[8];
+#pragma unroll
+    for (int i = 0; i < 8; ++i) out[i] = bf16_to_f32(f32_to_bf16(acc[i]));   // m = bf16(sum)
+    if (residual) {
+      float res[8];
+      if (residual_f32) {
+        const float4* rp = reinterpret_cast<const float4*>(static_cast<const float*>(residual) + size_t(t) * d + c);
+        const float4 a = __ldg(rp), b = __ldg(rp + 1);
+        res[0] = a.x; res[1] = a.y; res[2] = a.z; res[3] = a.w;
+        res[4] = b.x; res[5] = b.y; res[6] = b.z; res[7] = b.w;
+      } else {
+        const uint4 v = __ldg(reinterpret_cast<const uint4*>(static_cast<const uint16_t*>(residual) + size_t(t) * d + c));
+        const uint32_t w[4] = {v.x, v.y, v.z, v.w};
+#pragma unroll
+        for (int i = 0; i < 4; ++i) {
+          res[2 * i] = __uint_as_float(w[i] << 16);
+          res[2 * i + 1] = __uint_as_float(w[i] & 0xFFFF0000u);
+        }
+      }
+#pragma unroll
+      for (int i = 0; i < 8; ++i) out[i] = res[i] + sign * out[i];
+    }
+    uint4 ob;
+    ob.x = pack_bf16x2(out[0], out[1]);
+    ob.y = pack_bf16x2(out[2], out[3]);
+    ob.z = pack_bf16x2(out[4], out[5]);
+    ob.w = pack_bf16x2(out[6], out[7]);
+    if (y_f32) {
+      float4* yp = reinterpret_cast<float4*>(static_cast<float*>(y) + size_t(t) * d + c);
+      yp[0] = make_float4(out[0], out[1], out[2], out[3]);
+      yp[1] = make_float4(out[4], out[5], out[6], out[7]);
+    } else {
+      *reinterpret_cast<uint4*>(static_cast<uint16_t*>(y) + size_t(t) * d + c) = ob;
+    }
+    if (y_bf16) *reinterpret_cast<uint4*>(y_bf16 + size_t(t) * d + c) = ob;
+  }
+}
+
+int launch_combine(const uint16_t* out_perm, const int32_t* inv, const float* gates, int T, int k, int d,
+                   const void* residual, int residual_f32, float sign, void* y, int y_f32, uint16_t* y_bf16,
+                   cudaStream_t s) {
+  if (T == 0) return TQP_OK;
+  const int threads = d / 8 < 256 ? d / 8 : 256;
+  combine_kernel<<<T, threads, 0, s>>>(out_perm, inv, gates, T, k, d, residual, residual_f32, sign, y, y_f32,
+                                       y_bf16);
+  return cudaGetLastError() == cudaSuccess ? TQP_OK : TQP_ERR_CUDA;
+}
+
+}  // namespace tqp

@@ -1,0 +1,342 @@
+// C ABI of the TQP MoE library: argument validation, workspace layout and the
+// composition of the per-step kernels into the layer, the reversible coupling
+// and its backward. Declarations and contracts: include/tqp_moe.h.
+#include <cstdint>
+#include <cstring>
+#include <cuda_runtime.h>
+
+#include "../../include/tqp_moe.h"
+#include "tqp_device.cuh"
+#include "tqp_launch.h"
+
+using namespace tqp;
+
+namespace {
+
+constexpr int kMaxE = 4096;
+constexpr int kMaxTopK = 32;
+
+inline bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+int check_weights(const tqp_moe_weights* w) {
+  if (!w) return TQP_ERR_INVALID_ARG;
+  if (w->E < 1 || w->E > kMaxE || w->top_k < 1 || w->top_k > w->E || w->top_k > kMaxTopK)
+    return TQP_ERR_INVALID_ARG;
+  if (w->d < 128 || w->d > 16384 || w->d % 128 != 0) return TQP_ERR_INVALID_ARG;
+  if (w->ffn < 64 || w->ffn > 16384 || w->ffn % 64 != 0) return TQP_ERR_INVALID_ARG;
+  if (!(w->group == 32 || w->group == 64 || w->group == 128 || w->group == 256)) return TQP_ERR_UNSUPPORTED;
+  if (w->d % w->group != 0 || w->ffn % w->group != 0) return TQP_ERR_INVALID_ARG;
+  if (w->rank < 0 || w->rank > 64 || w->rank % 8 != 0) return TQP_ERR_UNSUPPORTED;
+  if (!w->router_w || !aligned16(w->router_w)) return TQP_ERR_INVALID_ARG;
+  if (w->router_bias && !aligned16(w->router_bias)) return TQP_ERR_INVALID_ARG;
+  for (int p = 0; p < 3; ++p) {
+    if (!w->wq[p] || !w->wscale[p] || !aligned16(w->wq[p]) || !aligned16(w->wscale[p])) return TQP_ERR_INVALID_ARG;
+    if (w->rank > 0 && (!w->lora_a[p] || !w->lora_b[p] || !aligned16(w->lora_a[p]) || !aligned16(w->lora_b[p])))
+      return TQP_ERR_INVALID_ARG;
+  }
+  return TQP_OK;
+}
+
+inline bool ptr_ok(const void* p, bool need) { return need ? (p && aligned16(p)) : true; }
+
+// Workspace of one full layer forward (kept for the backward's recompute too).
+struct LayerWs {
+  float* logits;
+  int32_t* ids;
+  float* gates;
+  int32_t* offsets;
+  int32_t* perm;
+  int32_t* inv;
+  uint16_t* h;
+  uint16_t* out_perm;
+  void* router_ws;
+  void* permute_ws;
+  void* ffn_ws;
+};
+
+size_t layer_ws_size(int T, const tqp_moe_weights* w) {
+  const size_t A = size_t(T) * w->top_k;
+  size_t b = 0;
+  b += align_up(size_t(T) * w->E * 4, 256);
+  b += align_up(A * 4, 256) * 2;                 // ids, gates
+  b += align_up(size_t(w->E + 1) * 4, 256);
+  b += align_up(A * 4, 256) * 2;                 // perm, inv
+  b += align_up(A * w->ffn * 2, 256);            // h
+  b += align_up(A * w->d * 2, 256);              // out_perm
+  b += align_up(router_ws_bytes(T, w), 256);
+  b += align_up(permute_ws_bytes(T, w->E), 256);
+  b += align_up(ffn_ws_bytes(T, w), 256);
+  return b + 256;
+}
+
+LayerWs carve_layer_ws(void* ws, int T, const tqp_moe_weights* w) {
+  const size_t A = size_t(T) * w->top_k;
+  char* p = reinterpret_cast<char*>(align_up(reinterpret_cast<uintptr_t>(ws), 256));
+  LayerWs L;
+  auto take = [&](size_t bytes) {
+    char* q = p;
+    p += align_up(bytes, 256);
+    return static_cast<void*>(q);
+  };
+  L.logits = static_cast<float*>(take(size_t(T) * w->E * 4));
+  L.ids = static_cast<int32_t*>(take(A * 4));
+  L.gates = static_cast<float*>(take(A * 4));
+  L.offsets = static_cast<int32_t*>(take(size_t(w->E + 1) * 4));
+  L.perm = static_cast<int32_t*>(take(A * 4));
+  L.inv = static_cast<int32_t*>(take(A * 4));
+  L.h = static_cast<uint16_t*>(take(A * w->ffn * 2));
+  L.out_perm = static_cast<uint16_t*>(take(A * w->d * 2));
+  L.router_ws = take(router_ws_bytes(T, w));
+  L.permute_ws = take(permute_ws_bytes(T, w->E));
+  L.ffn_ws = take(ffn_ws_bytes(T, w));
+  return L;
+}
+
+// router -> route -> permute -> experts (leaves everything in the workspace)
+int layer_experts(const uint16_t* x, int T, const tqp_moe_weights* w, const LayerWs& L, int32_t* status,
+                  cudaStream_t s) {
+  int rc;
+  if ((rc = launch_router_gemm(x, T, w, L.logits, L.router_ws, status, s)) != TQP_OK) return rc;
+  if ((rc = launch_route(L.logits, T, w->E, w->top_k, L.ids, L.gates, status, s)) != TQP_OK) return rc;
+  if ((rc = launch_permute(L.ids, T, w->E, w->top_k, L.offsets, L.perm, L.inv, L.permute_ws, status, s)) != TQP_OK)
+    return rc;
+  return launch_grouped_ffn(x, T, L.offsets, L.perm, w, L.h, L.out_perm, L.ffn_ws, status, s);
+}
+
+int layer_forward(const uint16_t* x, int T, const tqp_moe_weights* w, const void* residual, int res_f32,
+                  float sign, void* y, int y_f32, uint16_t* y_bf16, void* ws, int32_t* status, cudaStream_t s) {
+  const LayerWs L = carve_layer_ws(ws, T, w);
+  int rc = layer_experts(x, T, w, L, status, s);
+  if (rc != TQP_OK) return rc;
+  return launch_combine(L.out_perm, L.inv, L.gates, T, w->top_k, w->d, residual, res_f32, sign, y, y_f32, y_bf16, s);
+}
+
+__global__ void f32_to_bf16_kernel(const float* __restrict__ in, uint16_t* __restrict__ out, size_t n) {
+  const size_t i = (size_t(blockIdx.x) * blockDim.x + threadIdx.x) * 4;
+  if (i + 3 < n) {
+    const float4 v = *reinterpret_cast<const float4*>(in + i);
+    uint2 o;
+    o.x = pack_bf16x2(v.x, v.y);
+    o.y = pack_bf16x2(v.z, v.w);
+    *reinterpret_cast<uint2*>(out + i) = o;
+  } else {
+    for (size_t j = i; j < n; ++j) out[j] = f32_to_bf16(in[j]);
+  }
+}
+
+int to_bf16(const float* in, uint16_t* out, size_t n, cudaStream_t s) {
+  if (n == 0) return TQP_OK;
+  const size_t threads = (n + 3) / 4;
+  f32_to_bf16_kernel<<<unsigned((threads + 255) / 256), 256, 0, s>>>(in, out, n);
+  return cudaGetLastError() == cudaSuccess ? TQP_OK : TQP_ERR_CUDA;
+}
+
+}  // namespace
+
+extern "C" {
+
+int tqp_version(void) { return 100; }
+
+const char* tqp_error_string(int code) {
+  switch (code) {
+    case TQP_OK: return "ok";
+    case TQP_ERR_INVALID_ARG: return "invalid argument";
+    case TQP_ERR_UNSUPPORTED: return "unsupported configuration";
+    case TQP_ERR_WORKSPACE: return "workspace too small";
+    case TQP_ERR_CUDA: return "CUDA launch or runtime error";
+    default: return "unknown error";
+  }
+}
+
+size_t moe_router_gemm_workspace_size(int T, const tqp_moe_weights* w) {
+  if (check_weights(w) != TQP_OK || T < 0) return 0;
+  return router_ws_bytes(T, w);
+}
+
+int moe_router_gemm(const uint16_t* x, int T, const tqp_moe_weights* w, float* logits, void* ws, size_t ws_bytes,
+                    int32_t* dev_status, void* stream) {
+  int rc = check_weights(w);
+  if (rc != TQP_OK) return rc;
+  if (T < 0 || !ptr_ok(x, T > 0) || !ptr_ok(logits, T > 0) || !ptr_ok(ws, T > 0)) return TQP_ERR_INVALID_ARG;
+  if (T > 0 && ws_bytes < router_ws_bytes(T, w)) return TQP_ERR_WORKSPACE;
+  return launch_router_gemm(x, T, w, logits, ws, dev_status, static_cast<cudaStream_t>(stream));
+}
+
+int moe_route(const float* logits, int T, int E, int k, int32_t* ids, float* gates, int32_t* dev_status,
+              void* stream) {
+  if (T < 0 || E < 1 || E > kMaxE || k < 1 || k > E || k > kMaxTopK) return TQP_ERR_INVALID_ARG;
+  if (T > 0 && (!logits || !ids || !gates)) return TQP_ERR_INVALID_ARG;
+  return launch_route(logits, T, E, k, ids, gates, dev_status, static_cast<cudaStream_t>(stream));
+}
+
+size_t moe_permute_workspace_size(int T, int E, int k) {
+  if (T < 0 || E < 1 || E > kMaxE || k < 1 || k > E) return 0;
+  return permute_ws_bytes(T, E);
+}
+
+int moe_permute(const int32_t* ids, int T, int E, int k, int32_t* offsets, int32_t* perm_token, int32_t* inv,
+                void* ws, size_t ws_bytes, int32_t* dev_status, void* stream) {
+  if (T < 0 || E < 1 || E > kMaxE || k < 1 || k > E || !offsets) return TQP_ERR_INVALID_ARG;
+  if (T > 0 && (!ids || !perm_token || !inv || !ws)) return TQP_ERR_INVALID_ARG;
+  if (T > 0 && ws_bytes < permute_ws_bytes(T, E)) return TQP_ERR_WORKSPACE;
+  return launch_permute(ids, T, E, k, offsets, perm_token, inv, ws, dev_status, static_cast<cudaStream_t>(stream));
+}
+
+size_t tqp_grouped_ffn_workspace_size(int T, const tqp_moe_weights* w) {
+  if (check_weights(w) != TQP_OK || T < 0) return 0;
+  return ffn_ws_bytes(T, w);
+}
+
+int tqp_grouped_ffn(const uint16_t* x, int T, const int32_t* offsets, const int32_t* perm_token,
+                    const tqp_moe_weights* w, uint16_t* h, uint16_t* out_perm, void* ws, size_t ws_bytes,
+                    int32_t* dev_status, void* stream) {
+  int rc = check_weights(w);
+  if (rc != TQP_OK) return rc;
+  const bool n = T > 0;
+  if (T < 0 || !ptr_ok(x, n) || !ptr_ok(offsets, n) || !ptr_ok(perm_token, n) || !ptr_ok(h, n) ||
+      !ptr_ok(out_perm, n) || !ptr_ok(ws, n))
+    return TQP_ERR_INVALID_ARG;
+  if (n && ws_bytes < ffn_ws_bytes(T, w)) return TQP_ERR_WORKSPACE;
+  return launch_grouped_ffn(x, T, offsets, perm_token, w, h, out_perm, ws, dev_status,
+                            static_cast<cudaStream_t>(stream));
+}
+
+int moe_combine(const uint16_t* out_perm, const int32_t* inv, const float* gates, int T, int k, int d,
+                const void* residual, int residual_dtype, float sign, void* y, int y_dtype, uint16_t* y_bf16,
+                void* stream) {
+  if (T < 0 || k < 1 || k > kMaxTopK || d < 8 || d % 8 != 0) return TQP_ERR_INVALID_ARG;
+  if ((residual_dtype != TQP_DTYPE_BF16 && residual_dtype != TQP_DTYPE_F32) ||
+      (y_dtype != TQP_DTYPE_BF16 && y_dtype != TQP_DTYPE_F32))
+    return TQP_ERR_INVALID_ARG;
+  const bool n = T > 0;
+  if (!ptr_ok(out_perm, n) || !ptr_ok(inv, n) || !ptr_ok(gates, n) || !ptr_ok(y, n) || !ptr_ok(residual, false) ||
+      (residual && !aligned16(residual)) || (y_bf16 && !aligned16(y_bf16)))
+    return TQP_ERR_INVALID_ARG;
+  return launch_combine(out_perm, inv, gates, T, k, d, residual, residual_dtype == TQP_DTYPE_F32, sign, y,
+                        y_dtype == TQP_DTYPE_F32, y_bf16, static_cast<cudaStream_t>(stream));
+}
+
+size_t tqp_moe_layer_workspace_size(int T, const tqp_moe_weights* w) {
+  if (check_weights(w) != TQP_OK || T < 0) return 0;
+  return layer_ws_size(T, w);
+}
+
+int tqp_moe_layer_fwd(const uint16_t* x, int T, const tqp_moe_weights* w, uint16_t* y, void* ws, size_t ws_bytes,
+                      int32_t* dev_status, void* stream) {
+  int rc = check_weights(w);
+  if (rc != TQP_OK) return rc;
+  const bool n = T > 0;
+  if (T < 0 || !ptr_ok(x, n) || !ptr_ok(y, n) || !ptr_ok(ws, n)) return TQP_ERR_INVALID_ARG;
+  if (!n) return TQP_OK;
+  if (ws_bytes < layer_ws_size(T, w)) return TQP_ERR_WORKSPACE;
+  return layer_forward(x, T, w, nullptr, 0, 1.0f, y, 0, nullptr, ws, dev_status, static_cast<cudaStream_t>(stream));
+}
+
+size_t rev_couple_workspace_size(int T, const tqp_moe_weights* F, const tqp_moe_weights* G) {
+  if (check_weights(F) != TQP_OK || check_weights(G) != TQP_OK || T < 0 || F->d != G->d) return 0;
+  const size_t a = layer_ws_size(T, F), b = layer_ws_size(T, G);
+  return (a > b ? a : b) + align_up(size_t(T) * F->d * 2, 256) + 256;
+}
+
+int rev_couple_fwd(const uint16_t* x1, const uint16_t* x2, int T, const tqp_moe_weights* F, const tqp_moe_weights* G,
+                   float* y1, float* y2, void* ws, size_t ws_bytes, int32_t* dev_status, void* stream) {
+  int rc;
+  if ((rc = check_weights(F)) != TQP_OK || (rc = check_weights(G)) != TQP_OK) return rc;
+  if (F->d != G->d || T < 0) return TQP_ERR_INVALID_ARG;
+  const bool n = T > 0;
+  if (!ptr_ok(x1, n) || !ptr_ok(x2, n) || !ptr_ok(y1, n) || !ptr_ok(y2, n) || !ptr_ok(ws, n))
+    return TQP_ERR_INVALID_ARG;
+  if (!n) return TQP_OK;
+  if (ws_bytes < rev_couple_workspace_size(T, F, G)) return TQP_ERR_WORKSPACE;
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  char* base = reinterpret_cast<char*>(align_up(reinterpret_cast<uintptr_t>(ws), 256));
+  uint16_t* y1b = reinterpret_cast<uint16_t*>(base);
+  void* lws = base + align_up(size_t(T) * F->d * 2, 256);
+  // y1 = x1 + F(x2) (fp32), plus its bf16 copy as G's input
+  if ((rc = layer_forward(x2, T, F, x1, 0, 1.0f, y1, 1, y1b, lws, dev_status, s)) != TQP_OK) return rc;
+  // y2 = x2 + G(bf16(y1))
+  return layer_forward(y1b, T, G, x2, 0, 1.0f, y2, 1, nullptr, lws, dev_status, s);
+}
+
+int rev_couple_inv(const float* y1, const float* y2, int T, const tqp_moe_weights* F, const tqp_moe_weights* G,
+                   uint16_t* x1, uint16_t* x2, void* ws, size_t ws_bytes, int32_t* dev_status, void* stream) {
+  int rc;
+  if ((rc = check_weights(F)) != TQP_OK || (rc = check_weights(G)) != TQP_OK) return rc;
+  if (F->d != G->d || T < 0) return TQP_ERR_INVALID_ARG;
+  const bool n = T > 0;
+  if (!ptr_ok(x1, n) || !ptr_ok(x2, n) || !ptr_ok(y1, n) || !ptr_ok(y2, n) || !ptr_ok(ws, n))
+    return TQP_ERR_INVALID_ARG;
+  if (!n) return TQP_OK;
+  if (ws_bytes < rev_couple_workspace_size(T, F, G)) return TQP_ERR_WORKSPACE;
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  char* base = reinterpret_cast<char*>(align_up(reinterpret_cast<uintptr_t>(ws), 256));
+  uint16_t* y1b = reinterpret_cast<uint16_t*>(base);
+  void* lws = base + align_up(size_t(T) * F->d * 2, 256);
+  if ((rc = to_bf16(y1, y1b, size_t(T) * F->d, s)) != TQP_OK) return rc;
+  // x2 = y2 - G(bf16(y1)), rounded to bf16
+  if ((rc = layer_forward(y1b, T, G, y2, 1, -1.0f, x2, 0, nullptr, lws, dev_status, s)) != TQP_OK) return rc;
+  // x1 = y1 - F(x2)
+  return layer_forward(x2, T, F, y1, 1, -1.0f, x1, 0, nullptr, lws, dev_status, s);
+}
+
+size_t tqp_moe_layer_bwd_workspace_size(int T, const tqp_moe_weights* w) {
+  if (check_weights(w) != TQP_OK || T < 0) return 0;
+  return layer_ws_size(T, w) + layer_bwd_ws_bytes(T, w);
+}
+
+int tqp_moe_layer_bwd(const uint16_t* x, const float* dy, int T, const tqp_moe_weights* w, float* dx,
+                      const tqp_adapter_grads* grads, void* ws, size_t ws_bytes, int32_t* dev_status, void* stream) {
+  int rc = check_weights(w);
+  if (rc != TQP_OK) return rc;
+  const bool n = T > 0;
+  if (T < 0 || !ptr_ok(x, n) || !ptr_ok(dy, n) || !ptr_ok(dx, n) || !grads) return TQP_ERR_INVALID_ARG;
+  if (w->rank > 0)
+    for (int p = 0; p < 3; ++p)
+      if (!grads->dA[p] || !grads->dB[p] || !aligned16(grads->dA[p]) || !aligned16(grads->dB[p]))
+        return TQP_ERR_INVALID_ARG;
+  if (n && (!ws || ws_bytes < tqp_moe_layer_bwd_workspace_size(T, w))) return TQP_ERR_WORKSPACE;
+  return launch_layer_bwd(x, dy, T, w, dx, grads, ws, dev_status, static_cast<cudaStream_t>(stream));
+}
+
+size_t tqp_adapter_bwd_workspace_size(int T, const tqp_moe_weights* F, const tqp_moe_weights* G) {
+  if (check_weights(F) != TQP_OK || check_weights(G) != TQP_OK || T < 0 || F->d != G->d) return 0;
+  const size_t a = tqp_moe_layer_bwd_workspace_size(T, F), b = tqp_moe_layer_bwd_workspace_size(T, G);
+  const size_t fw = rev_couple_workspace_size(T, F, G);
+  size_t m = a > b ? a : b;
+  m = m > fw ? m : fw;
+  return m + align_up(size_t(T) * F->d * 2, 256) + align_up(size_t(T) * F->d * 4, 256) + 512;
+}
+
+int tqp_adapter_bwd(const float* y1, const float* y2, const float* dy1, const float* dy2, int T,
+                    const tqp_moe_weights* F, const tqp_moe_weights* G, uint16_t* x1, uint16_t* x2, float* dx1,
+                    float* dx2, const tqp_adapter_grads* gF, const tqp_adapter_grads* gG, void* ws, size_t ws_bytes,
+                    int32_t* dev_status, void* stream) {
+  int rc;
+  if ((rc = check_weights(F)) != TQP_OK || (rc = check_weights(G)) != TQP_OK) return rc;
+  if (F->d != G->d || T < 0 || !gF || !gG) return TQP_ERR_INVALID_ARG;
+  const bool n = T > 0;
+  if (!ptr_ok(y1, n) || !ptr_ok(y2, n) || !ptr_ok(dy1, n) || !ptr_ok(dy2, n) || !ptr_ok(x1, n) || !ptr_ok(x2, n) ||
+      !ptr_ok(dx1, n) || !ptr_ok(dx2, n))
+    return TQP_ERR_INVALID_ARG;
+  if (!n) return TQP_OK;
+  if (ws_bytes < tqp_adapter_bwd_workspace_size(T, F, G)) return TQP_ERR_WORKSPACE;
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  const size_t Td = size_t(T) * F->d;
+  char* base = reinterpret_cast<char*>(align_up(reinterpret_cast<uintptr_t>(ws), 256));
+  uint16_t* zb = reinterpret_cast<uint16_t*>(base);                     // bf16(y1)
+  float* dxG = reinterpret_cast<float*>(base + align_up(Td * 2, 256));  // J_G^T dy2
+  void* lws = base + align_up(Td * 2, 256) + align_up(Td * 4, 256);
+  const size_t lws_bytes = ws_bytes - size_t((char*)lws - (char*)ws);
+  // G-step: reconstruct x2 = y2 - G(bf16(y1)); G's grads for cotangent dy2
+  if ((rc = to_bf16(y1, zb, Td, s)) != TQP_OK) return rc;
+  if ((rc = layer_forward(zb, T, G, y2, 1, -1.0f, x2, 0, nullptr, lws, dev_status, s)) != TQP_OK) return rc;
+  if ((rc = tqp_moe_layer_bwd(zb, dy2, T, G, dxG, gG, lws, lws_bytes, dev_status, stream)) != TQP_OK) return rc;
+  // dz1 = dy1 + J_G^T dy2 -> dx1 (dx1 = dz1)
+  if ((rc = launch_add_f32(dy1, dxG, dx1, Td, s)) != TQP_OK) return rc;
+  // F-step: x1 = y1 - F(x2); F's grads for cotangent dz1; dx2 = dy2 + J_F^T dz1
+  if ((rc = layer_forward(x2, T, F, y1, 1, -1.0f, x1, 0, nullptr, lws, dev_status, s)) != TQP_OK) return rc;
+  if ((rc = tqp_moe_layer_bwd(x2, dx1, T, F, dxG, gF, lws, lws_bytes, dev_status, stream)) != TQP_OK) return rc;
+  return launch_add_f32(dy2, dxG, dx2, Td, s);
+}
+
+}  // extern "C"

@@ -256,3 +256,22 @@ def make_rev_inputs(cfgF: LayerConfig = REV_F, cfgG: LayerConfig = REV_G, T: int
         "dy1": make_grad(T, cfgF.d, seeds["dy"], "dy1"),
         "dy2": make_grad(T, cfgF.d, seeds["dy"], "dy2"),
     }
+
+
+def make_logits(T: int, E: int, seed: int, ties: bool = False, bias: np.ndarray | None = None) -> np.ndarray:
+    """Router-logit stand-ins [T][E] fp32 ~ N(0, 1) (the router's logit scale).
+
+    ties=True snaps every other token's row to a coarse grid (multiples of 1/4)
+    and plants +0.0 / -0.0 pairs, so exact ties are frequent. bias (optional)
+    is added in fp32, as the skewed-load workload's router does.
+    """
+    rng = _rng(seed, "x", 7)
+    l = rng.standard_normal((T, E), dtype=np.float32)
+    if ties:
+        l[::2] = np.round(l[::2] * 4) / 4
+        if E >= 4:
+            l[::3, 1] = np.float32(0.0)
+            l[::3, 2] = np.float32(-0.0)
+    if bias is not None:
+        l = (l + bias[None, :].astype(np.float32)).astype(np.float32)
+    return np.ascontiguousarray(l)

@@ -1,0 +1,85 @@
+"""Host-only checks of the C-ABI library: it loads, exports every function the
+header declares, answers workspace queries, and rejects bad arguments before
+touching the GPU. No compute call is made."""
+import ctypes
+
+import pytest
+
+import synth
+import quantized_base_lora_moe_b200 as Q
+
+
+def _struct(cfg, **over):
+    w = Q.Weights()
+    w.E, w.d, w.ffn, w.group, w.rank, w.top_k = cfg.E, cfg.d, cfg.f, cfg.g, cfg.r, cfg.k
+    w.lora_scale = cfg.lora_scale
+    fake = 0x10000
+    w.router_w = fake
+    for p in range(3):
+        w.wq[p] = fake
+        w.wscale[p] = fake
+        w.lora_a[p] = fake
+        w.lora_b[p] = fake
+    for k_, v in over.items():
+        setattr(w, k_, v)
+    return w
+
+
+def test_library_loads_and_exports_header_functions():
+    L = Q.lib()
+    names = Q.header_functions()
+    assert len(names) >= 19
+    for n in names:
+        assert hasattr(L, n), n
+    assert L.tqp_version() >= 100
+    assert L.tqp_error_string(-3) == b"workspace too small"
+
+
+@pytest.mark.parametrize("cfg", [synth.TINY, synth.MID, synth.FULL, synth.SKEWED], ids=lambda c: c.name)
+def test_workspace_queries(cfg):
+    L = Q.lib()
+    w = _struct(cfg)
+    assert L.moe_router_gemm_workspace_size(cfg.T, ctypes.byref(w)) >= 3 * cfg.E * cfg.d * 2
+    assert L.moe_permute_workspace_size(cfg.T, cfg.E, cfg.k) >= ((cfg.T + 31) // 32) * cfg.E * 4
+    assert L.tqp_grouped_ffn_workspace_size(cfg.T, ctypes.byref(w)) >= cfg.T * cfg.k * 3 * cfg.r * 2
+    lw = L.tqp_moe_layer_workspace_size(cfg.T, ctypes.byref(w))
+    assert lw >= cfg.T * cfg.k * (cfg.f + cfg.d) * 2
+    assert L.rev_couple_workspace_size(cfg.T, ctypes.byref(w), ctypes.byref(w)) > lw
+    assert L.tqp_adapter_bwd_workspace_size(cfg.T, ctypes.byref(w), ctypes.byref(w)) > lw
+
+
+BAD = [
+    dict(E=0), dict(top_k=0), dict(top_k=33), dict(d=100), dict(d=192), dict(ffn=96), dict(group=48),
+    dict(rank=12), dict(rank=72), dict(router_w=None), dict(router_w=0x10004),
+]
+
+
+@pytest.mark.parametrize("over", BAD, ids=[str(b) for b in BAD])
+def test_invalid_weights_rejected_on_host(over):
+    L = Q.lib()
+    w = _struct(synth.TINY, **over)
+    assert L.tqp_moe_layer_workspace_size(64, ctypes.byref(w)) == 0
+    rc = L.tqp_moe_layer_fwd(0x20000, 64, ctypes.byref(w), 0x30000, 0x40000, 1 << 30, None, None)
+    assert rc in (-1, -2)
+
+
+def test_small_workspace_and_null_pointers_rejected():
+    L = Q.lib()
+    w = _struct(synth.TINY)
+    assert L.tqp_moe_layer_fwd(0x20000, 64, ctypes.byref(w), 0x30000, 0x40000, 16, None, None) == -3
+    assert L.tqp_moe_layer_fwd(None, 64, ctypes.byref(w), 0x30000, 0x40000, 1 << 30, None, None) == -1
+    assert L.moe_route(None, 4, 8, 2, None, None, None, None) == -1
+    assert L.moe_route(0x1000, 4, 8, 9, 0x1000, 0x1000, None, None) == -1
+    assert L.moe_permute(0x1000, 4, 8, 2, 0x1000, 0x1000, 0x1000, 0x1000, 0, None, None) == -3
+    assert L.moe_combine(0x1000, 0x1000, 0x1000, 4, 2, 12, None, 0, 1.0, 0x1000, 0, None, None) == -1
+    # T == 0 is a no-op that succeeds without touching the device
+    assert L.tqp_moe_layer_fwd(None, 0, ctypes.byref(w), None, None, 0, None, None) == 0
+
+
+def test_mismatched_coupling_widths_rejected():
+    L = Q.lib()
+    F = _struct(synth.TINY)
+    G = _struct(synth.MID)
+    assert L.rev_couple_workspace_size(64, ctypes.byref(F), ctypes.byref(G)) == 0
+    assert L.rev_couple_fwd(0x1000, 0x1000, 64, ctypes.byref(F), ctypes.byref(G), 0x1000, 0x1000, 0x1000,
+                            1 << 30, None, None) == -1
