@@ -148,6 +148,30 @@ int moe_permute(const int32_t* ids, int T, int E, int k, int32_t* offsets, int32
                 void* ws, size_t ws_bytes, int32_t* dev_status, void* stream);
 
 /* ---------------------------------------------------------------------------
+ * moe_permute_noalloc: moe_permute for callers that cannot allocate device
+ * memory (a runtime that only hands out memory from its own fixed pool, a
+ * serving process that must never block in the driver's allocator, code with
+ * nowhere to keep a workspace between calls). The pages have no counterpart:
+ * this is a library convenience, not part of the method.
+ *   Same arguments and results as moe_permute, minus the workspace: the
+ *   scratch lives in a fixed array inside this library's device image, of
+ *   moe_permute_noalloc_max_bytes() bytes (about 1 MiB), which every GPU that
+ *   loads the library holds until the process exits.
+ *   Limits: T <= 16384 and E <= 512, else TQP_ERR_UNSUPPORTED (nothing is
+ *   enqueued). Allocates nothing: no cudaMalloc, no cudaFree, no allocating
+ *   library call.
+ *   The first call on a device looks up the array's device address with that
+ *   device current (cudaGetSymbolAddress); make that first call before any
+ *   stream capture.
+ *   All calls share the one array, and every call overwrites it before reading
+ *   it; calls that overlap on the GPU (concurrent streams) race on it and must
+ *   be serialised by the caller.
+ * ------------------------------------------------------------------------- */
+size_t moe_permute_noalloc_max_bytes(void);
+int moe_permute_noalloc(const int32_t* ids, int T, int E, int k, int32_t* offsets, int32_t* perm_token,
+                        int32_t* inv, int32_t* dev_status, void* stream);
+
+/* ---------------------------------------------------------------------------
  * tqp_grouped_ffn: the routed experts ("Train low-rank adapters per expert"
  * over "Quantize base expert weights", Pattern 3). For each expert e and each
  * of its rows (row r holds token perm_token[r]):

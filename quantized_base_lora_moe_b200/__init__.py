@@ -15,7 +15,7 @@ import numpy as np
 
 __all__ = [
     "lib", "TQPError", "DeviceLayer", "Status", "workspace",
-    "moe_router_gemm", "moe_route", "moe_permute", "tqp_grouped_ffn", "moe_combine", "tqp_moe_layer_fwd",
+    "moe_router_gemm", "moe_route", "moe_permute", "moe_permute_noalloc", "tqp_grouped_ffn", "moe_combine", "tqp_moe_layer_fwd",
     "rev_couple_fwd", "rev_couple_inv", "tqp_moe_layer_bwd", "tqp_adapter_bwd",
     "header_functions",
 ]
@@ -63,6 +63,8 @@ _SIGS = {
     "moe_route": (_I, [_VP, _I, _I, _I, _VP, _VP, _VP, _VP]),
     "moe_permute_workspace_size": (_SZ, [_I, _I, _I]),
     "moe_permute": (_I, [_VP, _I, _I, _I, _VP, _VP, _VP, _VP, _SZ, _VP, _VP]),
+    "moe_permute_noalloc_max_bytes": (_SZ, []),
+    "moe_permute_noalloc": (_I, [_VP, _I, _I, _I, _VP, _VP, _VP, _VP, _VP]),
     "tqp_grouped_ffn_workspace_size": (_SZ, [_I, _WP]),
     "tqp_grouped_ffn": (_I, [_VP, _I, _VP, _VP, _WP, _VP, _VP, _VP, _SZ, _VP, _VP]),
     "moe_combine": (_I, [_VP, _VP, _VP, _I, _I, _I, _VP, _I, _F, _VP, _I, _VP, _VP]),
@@ -234,6 +236,16 @@ def moe_permute(ids, E: int, offsets, perm_token, inv, ws=None, status: Status |
     _check("moe_permute", lib().moe_permute(ids.data_ptr(), T, E, k, offsets.data_ptr(), perm_token.data_ptr(),
                                             inv.data_ptr(), ws.data_ptr(), ws.numel(),
                                             status.ptr() if status else None, _stream(stream)))
+    return offsets, perm_token, inv
+
+
+def moe_permute_noalloc(ids, E: int, offsets, perm_token, inv, status: Status | None = None, stream=None):
+    """moe_permute with its scratch in the library's fixed device array (no workspace)."""
+    _require_cuda(ids, offsets, perm_token, inv)
+    T, k = ids.shape
+    _check("moe_permute_noalloc", lib().moe_permute_noalloc(ids.data_ptr(), T, E, k, offsets.data_ptr(),
+                                                            perm_token.data_ptr(), inv.data_ptr(),
+                                                            status.ptr() if status else None, _stream(stream)))
     return offsets, perm_token, inv
 
 
