@@ -31,7 +31,7 @@
 
 namespace tqp {
 
-enum Mode : int { GATEUP = 0, DOWN = 1, LORA_XA = 2, LORA_HA = 3, ROUTER = 4 };
+enum Mode : int { GATEUP = 0, DOWN = 1, LORA_XA = 2, LORA_HA = 3, ROUTER = 4, DH = 5, DX = 6 };
 
 constexpr int kThreads = 576;
 constexpr int kStages = 4;          // operand ring (A: 2 x 16 KB, B: 16 KB)
@@ -71,6 +71,12 @@ struct GemmArgs {
   void* out;
   int out_ld;
   int n_valid;          // valid output columns (ROUTER: E)
+  uint16_t* aux;        // GATEUP: optional G|U pre-activations out [A][2f]; DH: G|U in
+  int f_dim;            // ffn (GATEUP aux / DH epilogue)
+  int half_kb;          // DX: K-blocks of the gate part (then the up part)
+  const uint16_t* lb0;  // DH / DX LoRA step: A^T sources read transposed (Ad^T | Ag^T)
+  const uint16_t* lb1;  // DX: Au^T
+  int lb_ld;            // row length of lb0 / lb1
   const float* bias;
   int32_t* status;
 };
@@ -158,7 +164,8 @@ __global__ void __launch_bounds__(kThreads, 1)
     grouped_gemm_kernel(const GemmArgs a, const __grid_constant__ CUtensorMap tq0,
                         const __grid_constant__ CUtensorMap tq1, const __grid_constant__ CUtensorMap ts0,
                         const __grid_constant__ CUtensorMap ts1) {
-  constexpr bool kDequant = (MODE == GATEUP || MODE == DOWN);
+  constexpr bool kTrans = (MODE == DH || MODE == DX);   // B = W^T: dequantised transposed
+  constexpr bool kDequant = (MODE == GATEUP || MODE == DOWN || kTrans);
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   uint8_t* op_base = smem;
@@ -193,7 +200,7 @@ __global__ void __launch_bounds__(kThreads, 1)
   if (warp == 5 && lane == 0 && kDequant) {
     prefetch_tmap(&tq0);
     prefetch_tmap(&ts0);
-    if (MODE == GATEUP) {
+    if (MODE == GATEUP || MODE == DX) {
       prefetch_tmap(&tq1);
       prefetch_tmap(&ts1);
     }
@@ -241,6 +248,54 @@ __global__ void __launch_bounds__(kThreads, 1)
               uint4* dst = reinterpret_cast<uint4*>(hrow + c);
 #pragma unroll
               for (int i = 0; i < 4; ++i) dst[i] = make_uint4(pk[4 * i], pk[4 * i + 1], pk[4 * i + 2], pk[4 * i + 3]);
+              if (a.aux) {  // keep the pre-activations for the backward
+                uint4* ga = reinterpret_cast<uint4*>(a.aux + grow * (2 * size_t(a.f_dim)) + un.nt * 64 + c);
+                uint4* ua = reinterpret_cast<uint4*>(a.aux + grow * (2 * size_t(a.f_dim)) + a.f_dim + un.nt * 64 + c);
+#pragma unroll
+                for (int i = 0; i < 4; ++i) {
+                  ga[i] = make_uint4(pack_f16x2(gv[8 * i], gv[8 * i + 1]), pack_f16x2(gv[8 * i + 2], gv[8 * i + 3]),
+                                     pack_f16x2(gv[8 * i + 4], gv[8 * i + 5]), pack_f16x2(gv[8 * i + 6], gv[8 * i + 7]));
+                  ua[i] = make_uint4(pack_f16x2(uv[8 * i], uv[8 * i + 1]), pack_f16x2(uv[8 * i + 2], uv[8 * i + 3]),
+                                     pack_f16x2(uv[8 * i + 4], uv[8 * i + 5]), pack_f16x2(uv[8 * i + 6], uv[8 * i + 7]));
+                }
+              }
+            }
+          }
+        } else if (MODE == DH) {
+          // dH -> dG = dH * U * silu'(G), dU = dH * silu(G); G, U from the recompute
+          const size_t ld2 = 2 * size_t(a.f_dim);
+          const uint16_t* grow_gu = a.aux + grow * ld2 + un.nt * 128;
+          uint16_t* drow = static_cast<uint16_t*>(a.out) + grow * ld2 + un.nt * 128;
+#pragma unroll 1
+          for (int c = 0; c < 128; c += 32) {
+            float v[32];
+            tmem_ld32(tacc + c, v);
+            if (valid) {
+#pragma unroll
+              for (int q = 0; q < 4; ++q) {
+                const uint4 gq = *reinterpret_cast<const uint4*>(grow_gu + c + 8 * q);
+                const uint4 uq = *reinterpret_cast<const uint4*>(grow_gu + a.f_dim + c + 8 * q);
+                const uint32_t gw[4] = {gq.x, gq.y, gq.z, gq.w};
+                const uint32_t uw[4] = {uq.x, uq.y, uq.z, uq.w};
+                uint32_t dg[4], du[4];
+#pragma unroll
+                for (int t = 0; t < 4; ++t) {
+                  float res_g[2], res_u[2];
+#pragma unroll
+                  for (int hh = 0; hh < 2; ++hh) {
+                    const float g = f16_to_f32(uint16_t(hh ? (gw[t] >> 16) : (gw[t] & 0xFFFFu)));
+                    const float u = f16_to_f32(uint16_t(hh ? (uw[t] >> 16) : (uw[t] & 0xFFFFu)));
+                    const float dh = v[8 * q + 2 * t + hh];
+                    const float sg = 1.0f / (1.0f + __expf(-g));
+                    res_g[hh] = dh * u * sg * (1.0f + g * (1.0f - sg));
+                    res_u[hh] = dh * g * sg;
+                  }
+                  dg[t] = pack_f16x2(res_g[0], res_g[1]);
+                  du[t] = pack_f16x2(res_u[0], res_u[1]);
+                }
+                *reinterpret_cast<uint4*>(drow + c + 8 * q) = make_uint4(dg[0], dg[1], dg[2], dg[3]);
+                *reinterpret_cast<uint4*>(drow + a.f_dim + c + 8 * q) = make_uint4(du[0], du[1], du[2], du[3]);
+              }
             }
           }
         } else if (MODE == ROUTER) {
@@ -260,7 +315,7 @@ __global__ void __launch_bounds__(kThreads, 1)
           }
         } else {
           // DOWN / LORA_XA / LORA_HA: fp16 output, optional scale
-          const float sc = (MODE == DOWN) ? 1.0f : a.lora_scale;
+          const float sc = (MODE == DOWN || MODE == DX) ? 1.0f : a.lora_scale;
           uint16_t* orow = static_cast<uint16_t*>(a.out) + grow * a.out_ld + un.nt * a.ntile;
 #pragma unroll 1
           for (int c = 0; c < a.ntile; c += 32) {
@@ -332,9 +387,11 @@ __global__ void __launch_bounds__(kThreads, 1)
     // ------------------------------------------------------------ TMA producer (int4 + scales)
     if (kDequant && lane == 0) {
       Ring q;
-      const int ngrp = a.g >= 64 ? 1 : 64 / a.g;
+      const int ngrp = kTrans ? (a.g >= 128 ? 1 : 128 / a.g) : (a.g >= 64 ? 1 : 64 / a.g);
       const int rows_box = (MODE == GATEUP) ? 64 : 128;
-      const uint32_t bytes = 4096u + uint32_t(ngrp * 128 * 2);
+      // codes 4096 B + scale boxes: forward {64|128 out cols x ngrp} twice or once (256*ngrp B),
+      // transposed {64 K x ngrp} once (128*ngrp B)
+      const uint32_t bytes = 4096u + uint32_t(ngrp * (kTrans ? 128 : 256));
       const int gpe = a.in_dim / a.g;  // scale rows per expert
       int issued = 0;
       uint32_t last_phase = 0;
@@ -348,6 +405,18 @@ __global__ void __launch_bounds__(kThreads, 1)
           uint8_t* qs = q_base + size_t(q.stage) * kQStageBytes;
           uint64_t* bar = &ctl->q_full[q.stage];
           mbar_arrive_expect_tx(bar, bytes);
+          if (kTrans) {
+            // B = W^T: int4 rows = K (output index of W), bytes = N (input index)
+            const bool up = (MODE == DX) && kb >= a.half_kb;
+            const int kl = up ? kb - a.half_kb : kb;
+            tma_load_2d(smem_u32(qs), up ? &tq1 : &tq0, bar, un.nt * 64, un.e * a.out_dim + kl * 64);
+            tma_load_2d(smem_u32(qs + 4096), up ? &ts1 : &ts0, bar, kl * 64, un.e * gpe + (un.nt * 128) / a.g);
+            ++issued;
+            last_stage = q.stage;
+            last_phase = q.phase;
+            q.next<kQStages>();
+            continue;
+          }
           const int srow = un.e * gpe + (kb * 64) / a.g;
           tma_load_2d(smem_u32(qs), &tq0, bar, kb * 32, nrow0);
           tma_load_2d(smem_u32(qs + 4096), &ts0, bar, un.nt * rows_box, srow);
@@ -431,7 +500,61 @@ __global__ void __launch_bounds__(kThreads, 1)
         if (!mbar_wait(&ctl->op_empty[ring.stage], ring.phase ^ 1u, abort_flag, a.status)) { ok = false; break; }
         uint8_t* bst = op_base + size_t(ring.stage) * kOpStageBytes + kAStageBytes;
         const uint32_t bst_u = smem_u32(bst);
-        if (kDequant && kb < a.nkb_main) {
+        if (kTrans && kb < a.nkb_main) {
+          // transposed dequant: thread = 4 K rows x 8 N columns of the int4 tile [64 K][128 N]
+          if (!mbar_wait(&ctl->q_full[q.stage], q.phase, abort_flag, a.status)) { ok = false; break; }
+          const uint8_t* qs = q_base + size_t(q.stage) * kQStageBytes;
+          const int kq = tid >> 4, no = tid & 15;
+          const int n0 = un.nt * 128;
+          const int gi = (n0 + no * 8) / a.g - n0 / a.g;
+          const uint16_t* sc = reinterpret_cast<const uint16_t*>(qs + 4096);
+          uint32_t hv[4][4];
+#pragma unroll
+          for (int r = 0; r < 4; ++r) {
+            const int k = kq * 4 + r;
+            const uint32_t wv = *reinterpret_cast<const uint32_t*>(qs + k * 64 + no * 4);
+            const uint32_t sh = __half_as_ushort(__float2half_rn(bf16_to_f32(sc[gi * 64 + k])));
+            const uint4 d4 = dequant_word(wv, sh | (sh << 16));
+            hv[r][0] = d4.x; hv[r][1] = d4.y; hv[r][2] = d4.z; hv[r][3] = d4.w;
+          }
+#pragma unroll
+          for (int nn = 0; nn < 8; ++nn) {
+            const uint32_t sel = (nn & 1) ? 0x7632u : 0x5410u;
+            const uint32_t p01 = __byte_perm(hv[0][nn >> 1], hv[1][nn >> 1], sel);
+            const uint32_t p23 = __byte_perm(hv[2][nn >> 1], hv[3][nn >> 1], sel);
+            *reinterpret_cast<uint2*>(bst + sw128_offset(no * 8 + nn, kq >> 1) + (kq & 1) * 8) = make_uint2(p01, p23);
+          }
+          fence_proxy_async_smem();
+          mbar_arrive(&ctl->q_empty[q.stage]);
+          q.next<kQStages>();
+          mbar_arrive(&ctl->op_full[ring.stage]);
+        } else if (kTrans) {
+          // LoRA step of a dgrad: B[n][rr] = A^T[rr][n0 + n] (bf16, read transposed) as fp16
+          const int lb = kb - a.nkb_main;
+          const int n = un.nt * 128 + row;
+#pragma unroll 1
+          for (int i = 0; i < 4; ++i) {
+            const int c = half * 4 + i;
+            uint32_t pk[4];
+#pragma unroll
+            for (int t = 0; t < 4; ++t) {
+              float vv[2];
+#pragma unroll
+              for (int hh = 0; hh < 2; ++hh) {
+                const int rr = lb * 64 + c * 8 + 2 * t + hh;
+                float val = 0.0f;
+                if (rr < a.r) val = bf16_to_f32(__ldg(a.lb0 + (size_t(un.e) * a.r + rr) * a.lb_ld + n));
+                else if (MODE == DX && rr < 2 * a.r)
+                  val = bf16_to_f32(__ldg(a.lb1 + (size_t(un.e) * a.r + (rr - a.r)) * a.lb_ld + n));
+                vv[hh] = val;
+              }
+              pk[t] = pack_f16x2(vv[0], vv[1]);
+            }
+            *reinterpret_cast<uint4*>(bst + sw128_offset(row, c)) = make_uint4(pk[0], pk[1], pk[2], pk[3]);
+          }
+          fence_proxy_async_smem();
+          mbar_arrive(&ctl->op_full[ring.stage]);
+        } else if (kDequant && kb < a.nkb_main) {
           if (!mbar_wait(&ctl->q_full[q.stage], q.phase, abort_flag, a.status)) { ok = false; break; }
           const uint8_t* qs = q_base + size_t(q.stage) * kQStageBytes;
           const uint4 words = *reinterpret_cast<const uint4*>(qs + row * 32 + half * 16);
@@ -713,23 +836,32 @@ size_t ffn_ws_bytes(int T, const tqp_moe_weights* w) {
   return b + 256;
 }
 
-int launch_grouped_ffn(const uint16_t* x, int T, const int32_t* offsets, const int32_t* perm_token,
-                       const tqp_moe_weights* w, uint16_t* h, uint16_t* out_perm, void* ws, int32_t* status,
-                       cudaStream_t s) {
-  if (T == 0) return TQP_OK;
+FfnBufs ffn_carve(void* ws, int T, const tqp_moe_weights* w) {
   const size_t A = size_t(T) * w->top_k;
   char* p = static_cast<char*>(ws);
-  int32_t* mb_prefix = reinterpret_cast<int32_t*>(p);
+  FfnBufs b{};
+  b.mb_prefix = reinterpret_cast<int32_t*>(p);
   p += align_up(size_t(w->E + 1) * 4, 256);
-  uint16_t* x16 = reinterpret_cast<uint16_t*>(p);
+  b.x16 = reinterpret_cast<uint16_t*>(p);
   p += align_up(size_t(T) * w->d * 2, 256);
-  uint16_t* xa = nullptr;
-  uint16_t* ha = nullptr;
   if (w->rank > 0) {
-    xa = reinterpret_cast<uint16_t*>(p);
+    b.xa = reinterpret_cast<uint16_t*>(p);
     p += align_up(A * 2 * w->rank * 2, 256);
-    ha = reinterpret_cast<uint16_t*>(p);
+    b.ha = reinterpret_cast<uint16_t*>(p);
   }
+  return b;
+}
+
+int launch_grouped_ffn(const uint16_t* x, int T, const int32_t* offsets, const int32_t* perm_token,
+                       const tqp_moe_weights* w, uint16_t* h, uint16_t* out_perm, void* ws, int32_t* status,
+                       cudaStream_t s, uint16_t* aux_gu) {
+  if (T == 0) return TQP_OK;
+  const size_t A = size_t(T) * w->top_k;
+  const FfnBufs fb = ffn_carve(ws, T, w);
+  int32_t* mb_prefix = fb.mb_prefix;
+  uint16_t* x16 = fb.x16;
+  uint16_t* xa = fb.xa;
+  uint16_t* ha = fb.ha;
   schedule_kernel<<<1, 1024, 0, s>>>(offsets, w->E, mb_prefix);
   {
     const size_t n8 = size_t(T) * w->d / 8;
@@ -790,6 +922,8 @@ int launch_grouped_ffn(const uint16_t* x, int T, const int32_t* offsets, const i
     a.out = h;
     a.out_ld = f;
     a.n_valid = f;
+    a.aux = aux_gu;
+    a.f_dim = f;
     const int ngrp = w->group >= 64 ? 1 : 64 / w->group;
     bool ok = make_map(&maps[0], CU_TENSOR_MAP_DATA_TYPE_UINT8, w->wq[0], d / 2, uint64_t(w->E) * f, d / 2, 32, 64) &&
               make_map(&maps[1], CU_TENSOR_MAP_DATA_TYPE_UINT8, w->wq[1], d / 2, uint64_t(w->E) * f, d / 2, 32, 64) &&
@@ -843,6 +977,80 @@ int launch_grouped_ffn(const uint16_t* x, int T, const int32_t* offsets, const i
     if ((rc = run_gemm<DOWN>(a, maps, mb_upper * a.n_tiles, s)) != TQP_OK) return rc;
   }
   return TQP_OK;
+}
+
+// dH = dO Wd + dhA Ad^T (SwiGLU backward fused: writes dG | dU) or
+// dX = [dG | dU] [Wg ; Wu] + dxa [Ag^T ; Au^T]^T, per expert, on the tensor cores
+// with the int4 base dequantised transposed in shared memory.
+int launch_dgrad(int which, const uint16_t* a_src, const uint16_t* a_lora, const int32_t* offsets,
+                 const int32_t* mb_prefix, const tqp_moe_weights* w, int T, const uint16_t* aux_gu, uint16_t* out,
+                 int32_t* status, cudaStream_t s) {
+  if (T == 0) return TQP_OK;
+  const size_t A = size_t(T) * w->top_k;
+  const int d = w->d, f = w->ffn, r = w->rank;
+  const int mb_upper = int((A + kMBlock - 1) / kMBlock) + w->E;
+  GemmArgs a{};
+  a.E = w->E;
+  a.g = w->group;
+  a.r = r;
+  a.lora_scale = w->lora_scale;
+  a.offsets = offsets;
+  a.mb_prefix = mb_prefix;
+  a.kb_per_piece = 1;
+  a.status = status;
+  a.ntile = 128;
+  a.f_dim = f;
+  a.a_src = a_src;
+  a.a_lora = a_lora;
+  a.out = out;
+  CUtensorMap maps[4];
+  memset(maps, 0, sizeof(maps));
+  const int ngn = w->group >= 128 ? 1 : 128 / w->group;
+  if (which == 0) {  // DH: K = d (rows of Wd), N = f
+    a.nkb_main = d / 64;
+    a.nkb_lora = r > 0 ? (r + 63) / 64 : 0;
+    a.lora_k = r;
+    a.lora_ld = r;
+    a.n_tiles = f / 128;
+    a.in_dim = f;
+    a.out_dim = d;
+    a.a_ld = d;
+    a.lb0 = w->lora_a[2];
+    a.lb_ld = f;
+    a.aux = const_cast<uint16_t*>(aux_gu);
+    a.out_ld = 2 * f;
+    a.n_valid = f;
+    bool ok = make_map(&maps[0], CU_TENSOR_MAP_DATA_TYPE_UINT8, w->wq[2], f / 2, uint64_t(w->E) * d, f / 2, 64, 64) &&
+              make_map(&maps[2], CU_TENSOR_MAP_DATA_TYPE_UINT16, w->wscale[2], d, uint64_t(w->E) * (f / w->group),
+                       uint64_t(d) * 2, 64, ngn);
+    maps[1] = maps[0];
+    maps[3] = maps[2];
+    if (!ok) return TQP_ERR_CUDA;
+    return run_gemm<DH>(a, maps, mb_upper * a.n_tiles, s);
+  }
+  // DX: K = 2f (gate rows then up rows of W), N = d
+  a.nkb_main = 2 * f / 64;
+  a.half_kb = f / 64;
+  a.nkb_lora = r > 0 ? (2 * r + 63) / 64 : 0;
+  a.lora_k = 2 * r;
+  a.lora_ld = 2 * r;
+  a.n_tiles = d / 128;
+  a.in_dim = d;
+  a.out_dim = f;
+  a.a_ld = 2 * f;
+  a.lb0 = w->lora_a[0];
+  a.lb1 = w->lora_a[1];
+  a.lb_ld = d;
+  a.out_ld = d;
+  a.n_valid = d;
+  bool ok = make_map(&maps[0], CU_TENSOR_MAP_DATA_TYPE_UINT8, w->wq[0], d / 2, uint64_t(w->E) * f, d / 2, 64, 64) &&
+            make_map(&maps[1], CU_TENSOR_MAP_DATA_TYPE_UINT8, w->wq[1], d / 2, uint64_t(w->E) * f, d / 2, 64, 64) &&
+            make_map(&maps[2], CU_TENSOR_MAP_DATA_TYPE_UINT16, w->wscale[0], f, uint64_t(w->E) * (d / w->group),
+                     uint64_t(f) * 2, 64, ngn) &&
+            make_map(&maps[3], CU_TENSOR_MAP_DATA_TYPE_UINT16, w->wscale[1], f, uint64_t(w->E) * (d / w->group),
+                     uint64_t(f) * 2, 64, ngn);
+  if (!ok) return TQP_ERR_CUDA;
+  return run_gemm<DX>(a, maps, mb_upper * a.n_tiles, s);
 }
 
 }  // namespace tqp

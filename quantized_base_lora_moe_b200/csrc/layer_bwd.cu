@@ -1,4 +1,16 @@
-// Backward of the TQP MoE layer (adapters only; base and router frozen).
+// Backward of the TQP MoE layer: adapters only, base and router frozen
+// ("Base expert weights: Quantized (fixed)", "Optimizer state only on adapters",
+// Principle 3 / Pattern 3 of "Reversible Sparse MoE Single Node").
+//
+// The dense dgrad contractions run on the tensor cores (launch_dgrad in
+// grouped_gemm.cu). This file holds the rest:
+//   bwd_combine  : dO = gamma * dy (fp16, permuted rows), dgamma = <dy, O>, the
+//                  softmax-over-chosen backward dl = gamma (dgamma - sum gamma dgamma)
+//                  and the frozen router's input gradient sum_j dl_j W_r[id_j]
+//   rowgemm      : small rank-space products dhA = s dO Bd^T and dxa = s [dG|dU] [Bg|Bu]^T
+//   outer        : per-expert adapter gradients, sums over the expert's routed rows
+//                  of outer products (dA^T, dB^T in the storage layouts)
+//   gather_add   : dx[t] += sum_j dX[row(t, j)]
 #include <cstdint>
 #include <cuda_runtime.h>
 
@@ -19,11 +31,350 @@ int launch_add_f32(const float* a, const float* b, float* out, size_t n, cudaStr
   return cudaGetLastError() == cudaSuccess ? TQP_OK : TQP_ERR_CUDA;
 }
 
-size_t layer_bwd_ws_bytes(int T, const tqp_moe_weights* w) { (void)T; (void)w; return 256; }
+// ----------------------------------------------------------------------------
+// combine backward + softmax-gate backward + router input gradient
+// ----------------------------------------------------------------------------
 
-int launch_layer_bwd(const uint16_t*, const float*, int, const tqp_moe_weights*, float*, const tqp_adapter_grads*,
-                     void*, int32_t*, cudaStream_t) {
-  return TQP_ERR_UNSUPPORTED;
+constexpr int kMaxK = 32;
+
+__global__ void __launch_bounds__(256) bwd_combine_kernel(const uint16_t* __restrict__ O, const int32_t* __restrict__ inv,
+                                                          const float* __restrict__ gates,
+                                                          const int32_t* __restrict__ ids,
+                                                          const float* __restrict__ router_w,
+                                                          const float* __restrict__ dy, int T, int k, int d,
+                                                          uint16_t* __restrict__ dO, float* __restrict__ dx) {
+  __shared__ float red[8][kMaxK];
+  __shared__ float dl_s[kMaxK];
+  const int t = blockIdx.x;
+  const int lane = threadIdx.x & 31, wid = threadIdx.x >> 5;
+  const int nwarps = blockDim.x >> 5;
+  float part[kMaxK];
+#pragma unroll
+  for (int j = 0; j < kMaxK; ++j) part[j] = 0.0f;
+  for (int c = threadIdx.x * 8; c < d; c += blockDim.x * 8) {
+    const float4* dp = reinterpret_cast<const float4*>(dy + size_t(t) * d + c);
+    const float4 a0 = dp[0], a1 = dp[1];
+    const float dv[8] = {a0.x, a0.y, a0.z, a0.w, a1.x, a1.y, a1.z, a1.w};
+#pragma unroll
+    for (int j = 0; j < kMaxK; ++j) {
+      if (j >= k) break;
+      const int row = inv[size_t(t) * k + j];
+      const float g = gates[size_t(t) * k + j];
+      const uint4 ov = *reinterpret_cast<const uint4*>(O + size_t(row) * d + c);
+      const uint32_t ow[4] = {ov.x, ov.y, ov.z, ov.w};
+      float acc = 0.0f;
+      uint32_t pk[4];
+#pragma unroll
+      for (int q = 0; q < 4; ++q) {
+        acc = fmaf(dv[2 * q], f16_to_f32(uint16_t(ow[q] & 0xFFFFu)), acc);
+        acc = fmaf(dv[2 * q + 1], f16_to_f32(uint16_t(ow[q] >> 16)), acc);
+        pk[q] = pack_f16x2(g * dv[2 * q], g * dv[2 * q + 1]);
+      }
+      part[j] += acc;
+      *reinterpret_cast<uint4*>(dO + size_t(row) * d + c) = make_uint4(pk[0], pk[1], pk[2], pk[3]);
+    }
+  }
+  // dgamma_j = sum over the row: warp then block reduction
+#pragma unroll
+  for (int j = 0; j < kMaxK; ++j) {
+    if (j >= k) break;
+    float v = part[j];
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) v += __shfl_xor_sync(0xFFFFFFFFu, v, o);
+    if (lane == 0) red[wid][j] = v;
+  }
+  __syncthreads();
+  if (threadIdx.x == 0) {
+    float dg[kMaxK], gs[kMaxK];
+    float sum = 0.0f;
+    for (int j = 0; j < k; ++j) {
+      float v = 0.0f;
+      for (int w = 0; w < nwarps; ++w) v += red[w][j];
+      dg[j] = v;
+      gs[j] = gates[size_t(t) * k + j];
+      sum += gs[j] * v;
+    }
+    for (int j = 0; j < k; ++j) dl_s[j] = gs[j] * (dg[j] - sum);
+  }
+  __syncthreads();
+  // dx[t] = sum_j dl_j W_r[id_j]  (through the frozen full-precision router)
+  for (int c = threadIdx.x * 8; c < d; c += blockDim.x * 8) {
+    float acc[8];
+#pragma unroll
+    for (int i = 0; i < 8; ++i) acc[i] = 0.0f;
+    for (int j = 0; j < k; ++j) {
+      const int e = ids[size_t(t) * k + j];
+      const float4* wp = reinterpret_cast<const float4*>(router_w + size_t(e) * d + c);
+      const float4 w0 = __ldg(wp), w1 = __ldg(wp + 1);
+      const float wv[8] = {w0.x, w0.y, w0.z, w0.w, w1.x, w1.y, w1.z, w1.w};
+      const float l = dl_s[j];
+#pragma unroll
+      for (int i = 0; i < 8; ++i) acc[i] = fmaf(l, wv[i], acc[i]);
+    }
+    float4* xp = reinterpret_cast<float4*>(dx + size_t(t) * d + c);
+    xp[0] = make_float4(acc[0], acc[1], acc[2], acc[3]);
+    xp[1] = make_float4(acc[4], acc[5], acc[6], acc[7]);
+  }
+}
+
+// dx[t] += sum_j dX[inv[t*k + j]]  (fp16 rows, fp32 accumulation, fixed j order)
+__global__ void __launch_bounds__(256) gather_add_kernel(const uint16_t* __restrict__ dX, const int32_t* __restrict__ inv,
+                                                         int T, int k, int d, float* __restrict__ dx) {
+  const int t = blockIdx.x;
+  for (int c = threadIdx.x * 8; c < d; c += blockDim.x * 8) {
+    float4* xp = reinterpret_cast<float4*>(dx + size_t(t) * d + c);
+    const float4 b0 = xp[0], b1 = xp[1];
+    float acc[8] = {b0.x, b0.y, b0.z, b0.w, b1.x, b1.y, b1.z, b1.w};
+    for (int j = 0; j < k; ++j) {
+      const int row = inv[size_t(t) * k + j];
+      const uint4 v = *reinterpret_cast<const uint4*>(dX + size_t(row) * d + c);
+      const uint32_t w[4] = {v.x, v.y, v.z, v.w};
+#pragma unroll
+      for (int q = 0; q < 4; ++q) {
+        acc[2 * q] += f16_to_f32(uint16_t(w[q] & 0xFFFFu));
+        acc[2 * q + 1] += f16_to_f32(uint16_t(w[q] >> 16));
+      }
+    }
+    xp[0] = make_float4(acc[0], acc[1], acc[2], acc[3]);
+    xp[1] = make_float4(acc[4], acc[5], acc[6], acc[7]);
+  }
+}
+
+// ----------------------------------------------------------------------------
+// per-expert row blocks of 64 (prefix of ceil(count/64))
+// ----------------------------------------------------------------------------
+
+constexpr int kRB = 64;
+
+__global__ void block_prefix_kernel(const int32_t* __restrict__ offsets, int E, int32_t* __restrict__ pre) {
+  if (threadIdx.x != 0 || blockIdx.x != 0) return;
+  int run = 0;
+  for (int e = 0; e < E; ++e) {
+    pre[e] = run;
+    run += (offsets[e + 1] - offsets[e] + kRB - 1) / kRB;
+  }
+  pre[E] = run;
+}
+
+__device__ __forceinline__ int find_expert(const int32_t* __restrict__ pre, int E, int u) {
+  int lo = 0, hi = E;
+  while (hi - lo > 1) {
+    const int mid = (lo + hi) >> 1;
+    if (pre[mid] <= u) lo = mid;
+    else hi = mid;
+  }
+  return lo;
+}
+
+// ----------------------------------------------------------------------------
+// rank-space row GEMMs: C[row][n] = s * sum_k P[row][k] * B_e[k][n], n < N <= 64
+// ----------------------------------------------------------------------------
+
+struct RowGemmArgs {
+  int which;                 // 0: dhA (B = Bd^T [d][r]); 1: dxa (B = blockdiag(Bg^T, Bu^T) [2f][2r])
+  int E, K, N, r, f;
+  float scale;
+  const int32_t* offsets;
+  const int32_t* pre;
+  const uint16_t* P;         // fp16 [A][K]
+  const uint16_t* b0;        // bf16 B^T sources
+  const uint16_t* b1;
+  uint16_t* C;               // fp16 [A][N]
+};
+
+__device__ __forceinline__ float rowgemm_b(const RowGemmArgs& a, int e, int k, int n) {
+  if (a.which == 0) return n < a.r ? bf16_to_f32(__ldg(a.b0 + (size_t(e) * a.K + k) * a.r + n)) : 0.0f;
+  if (k < a.f) return n < a.r ? bf16_to_f32(__ldg(a.b0 + (size_t(e) * a.f + k) * a.r + n)) : 0.0f;
+  return (n >= a.r && n < 2 * a.r) ? bf16_to_f32(__ldg(a.b1 + (size_t(e) * a.f + (k - a.f)) * a.r + (n - a.r)))
+                                   : 0.0f;
+}
+
+__global__ void __launch_bounds__(256) rowgemm_kernel(const RowGemmArgs a) {
+  __shared__ float Ps[kRB][33];
+  __shared__ float Bs[32][65];
+  const int nunits = a.pre[a.E];
+  const int tx = threadIdx.x & 15, ty = threadIdx.x >> 4;    // 16 col groups x 16 row groups
+  for (int u = blockIdx.x; u < nunits; u += gridDim.x) {
+    const int e = find_expert(a.pre, a.E, u);
+    const int mb = u - a.pre[e];
+    const int base = a.offsets[e] + mb * kRB;
+    const int rows = min(kRB, a.offsets[e + 1] - base);
+    float acc[4][4];
+#pragma unroll
+    for (int i = 0; i < 4; ++i)
+#pragma unroll
+      for (int j = 0; j < 4; ++j) acc[i][j] = 0.0f;
+    for (int k0 = 0; k0 < a.K; k0 += 32) {
+      __syncthreads();
+      for (int i = threadIdx.x; i < kRB * 32; i += blockDim.x) {
+        const int rr = i >> 5, kk = i & 31;
+        Ps[rr][kk] = (rr < rows) ? f16_to_f32(a.P[size_t(base + rr) * a.K + k0 + kk]) : 0.0f;
+      }
+      for (int i = threadIdx.x; i < 32 * 64; i += blockDim.x) {
+        const int kk = i >> 6, n = i & 63;
+        Bs[kk][n] = (n < a.N) ? rowgemm_b(a, e, k0 + kk, n) : 0.0f;
+      }
+      __syncthreads();
+#pragma unroll 8
+      for (int kk = 0; kk < 32; ++kk) {
+        float pv[4], bv[4];
+#pragma unroll
+        for (int i = 0; i < 4; ++i) pv[i] = Ps[ty * 4 + i][kk];
+#pragma unroll
+        for (int j = 0; j < 4; ++j) bv[j] = Bs[kk][tx * 4 + j];
+#pragma unroll
+        for (int i = 0; i < 4; ++i)
+#pragma unroll
+          for (int j = 0; j < 4; ++j) acc[i][j] = fmaf(pv[i], bv[j], acc[i][j]);
+      }
+    }
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+      const int rr = ty * 4 + i;
+      if (rr >= rows) continue;
+#pragma unroll
+      for (int j = 0; j < 4; ++j) {
+        const int n = tx * 4 + j;
+        if (n < a.N) a.C[size_t(base + rr) * a.N + n] = __half_as_ushort(__float2half_rn(a.scale * acc[i][j]));
+      }
+    }
+  }
+}
+
+// ----------------------------------------------------------------------------
+// adapter gradients: C[e][m][n] = sum_{rows of e} P(row, m) * Q(row, n)
+// ----------------------------------------------------------------------------
+
+struct OuterArgs {
+  int E, M, N;
+  const int32_t* offsets;
+  const int32_t* perm;       // row gather for Q (token rows of x), or null
+  const uint16_t* P;         // fp16, row stride ldp, column offset offp
+  int ldp, offp;
+  const uint16_t* Q;
+  int ldq, offq;
+  float* C;                  // fp32 [E][M][N]
+};
+
+__global__ void __launch_bounds__(256) outer_kernel(const OuterArgs a) {
+  __shared__ float Ps[32][65];
+  __shared__ float Qs[32][65];
+  const int e = blockIdx.x;
+  const int m0 = blockIdx.y * 64, n0 = blockIdx.z * 64;
+  const int tx = threadIdx.x & 15, ty = threadIdx.x >> 4;
+  const int r0 = a.offsets[e], r1 = a.offsets[e + 1];
+  float acc[4][4];
+#pragma unroll
+  for (int i = 0; i < 4; ++i)
+#pragma unroll
+    for (int j = 0; j < 4; ++j) acc[i][j] = 0.0f;
+  for (int rb = r0; rb < r1; rb += 32) {
+    __syncthreads();
+    for (int i = threadIdx.x; i < 32 * 64; i += blockDim.x) {
+      const int rr = i >> 6, c = i & 63;
+      const int row = rb + rr;
+      const bool ok = row < r1;
+      Ps[rr][c] = (ok && m0 + c < a.M) ? f16_to_f32(a.P[size_t(row) * a.ldp + a.offp + m0 + c]) : 0.0f;
+      const int qrow = ok ? (a.perm ? a.perm[row] : row) : 0;
+      Qs[rr][c] = (ok && n0 + c < a.N) ? f16_to_f32(a.Q[size_t(qrow) * a.ldq + a.offq + n0 + c]) : 0.0f;
+    }
+    __syncthreads();
+#pragma unroll 8
+    for (int rr = 0; rr < 32; ++rr) {
+      float pv[4], qv[4];
+#pragma unroll
+      for (int i = 0; i < 4; ++i) pv[i] = Ps[rr][ty * 4 + i];
+#pragma unroll
+      for (int j = 0; j < 4; ++j) qv[j] = Qs[rr][tx * 4 + j];
+#pragma unroll
+      for (int i = 0; i < 4; ++i)
+#pragma unroll
+        for (int j = 0; j < 4; ++j) acc[i][j] = fmaf(pv[i], qv[j], acc[i][j]);
+    }
+  }
+#pragma unroll
+  for (int i = 0; i < 4; ++i) {
+    const int m = m0 + ty * 4 + i;
+    if (m >= a.M) continue;
+#pragma unroll
+    for (int j = 0; j < 4; ++j) {
+      const int n = n0 + tx * 4 + j;
+      if (n < a.N) a.C[(size_t(e) * a.M + m) * a.N + n] = acc[i][j];
+    }
+  }
+}
+
+// ----------------------------------------------------------------------------
+// host launchers
+// ----------------------------------------------------------------------------
+
+int launch_bwd_combine(const uint16_t* O, const int32_t* inv, const float* gates, const int32_t* ids,
+                       const float* router_w, const float* dy, int T, int k, int d, uint16_t* dO, float* dx,
+                       cudaStream_t s) {
+  if (T == 0) return TQP_OK;
+  // at least one full warp: the row reductions use full-mask warp shuffles
+  const int threads = d / 8 < 32 ? 32 : (d / 8 < 256 ? d / 8 : 256);
+  bwd_combine_kernel<<<T, threads, 0, s>>>(O, inv, gates, ids, router_w, dy, T, k, d, dO, dx);
+  return cudaGetLastError() == cudaSuccess ? TQP_OK : TQP_ERR_CUDA;
+}
+
+int launch_gather_add(const uint16_t* dX, const int32_t* inv, int T, int k, int d, float* dx, cudaStream_t s) {
+  if (T == 0) return TQP_OK;
+  const int threads = d / 8 < 256 ? d / 8 : 256;
+  gather_add_kernel<<<T, threads, 0, s>>>(dX, inv, T, k, d, dx);
+  return cudaGetLastError() == cudaSuccess ? TQP_OK : TQP_ERR_CUDA;
+}
+
+int launch_block_prefix(const int32_t* offsets, int E, int32_t* pre, cudaStream_t s) {
+  block_prefix_kernel<<<1, 32, 0, s>>>(offsets, E, pre);
+  return cudaGetLastError() == cudaSuccess ? TQP_OK : TQP_ERR_CUDA;
+}
+
+int launch_rowgemm(int which, const uint16_t* P, const int32_t* offsets, const int32_t* pre, int A_rows,
+                   const tqp_moe_weights* w, uint16_t* C, cudaStream_t s) {
+  RowGemmArgs a{};
+  a.which = which;
+  a.E = w->E;
+  a.r = w->rank;
+  a.f = w->ffn;
+  a.scale = w->lora_scale;
+  a.offsets = offsets;
+  a.pre = pre;
+  a.P = P;
+  a.C = C;
+  if (which == 0) {
+    a.K = w->d;
+    a.N = w->rank;
+    a.b0 = w->lora_b[2];
+  } else {
+    a.K = 2 * w->ffn;
+    a.N = 2 * w->rank;
+    a.b0 = w->lora_b[0];
+    a.b1 = w->lora_b[1];
+  }
+  const int blocks = (A_rows + kRB - 1) / kRB + w->E;
+  rowgemm_kernel<<<blocks < 4096 ? blocks : 4096, 256, 0, s>>>(a);
+  return cudaGetLastError() == cudaSuccess ? TQP_OK : TQP_ERR_CUDA;
+}
+
+int launch_outer(int E, int M, int N, const int32_t* offsets, const int32_t* perm, const uint16_t* P, int ldp,
+                 int offp, const uint16_t* Q, int ldq, int offq, float* C, cudaStream_t s) {
+  OuterArgs a{};
+  a.E = E;
+  a.M = M;
+  a.N = N;
+  a.offsets = offsets;
+  a.perm = perm;
+  a.P = P;
+  a.ldp = ldp;
+  a.offp = offp;
+  a.Q = Q;
+  a.ldq = ldq;
+  a.offq = offq;
+  a.C = C;
+  dim3 grid(E, (M + 63) / 64, (N + 63) / 64);
+  outer_kernel<<<grid, 256, 0, s>>>(a);
+  return cudaGetLastError() == cudaSuccess ? TQP_OK : TQP_ERR_CUDA;
 }
 
 }  // namespace tqp

@@ -94,13 +94,83 @@ LayerWs carve_layer_ws(void* ws, int T, const tqp_moe_weights* w) {
 
 // router -> route -> permute -> experts (leaves everything in the workspace)
 int layer_experts(const uint16_t* x, int T, const tqp_moe_weights* w, const LayerWs& L, int32_t* status,
-                  cudaStream_t s) {
+                  cudaStream_t s, uint16_t* aux_gu = nullptr) {
   int rc;
   if ((rc = launch_router_gemm(x, T, w, L.logits, L.router_ws, status, s)) != TQP_OK) return rc;
   if ((rc = launch_route(L.logits, T, w->E, w->top_k, L.ids, L.gates, status, s)) != TQP_OK) return rc;
   if ((rc = launch_permute(L.ids, T, w->E, w->top_k, L.offsets, L.perm, L.inv, L.permute_ws, status, s)) != TQP_OK)
     return rc;
-  return launch_grouped_ffn(x, T, L.offsets, L.perm, w, L.h, L.out_perm, L.ffn_ws, status, s);
+  return launch_grouped_ffn(x, T, L.offsets, L.perm, w, L.h, L.out_perm, L.ffn_ws, status, s, aux_gu);
+}
+
+// Extra workspace of the layer backward, after the forward recompute's.
+struct BwdWs {
+  uint16_t* gu;     // G | U pre-activations [A][2f] fp16
+  uint16_t* dO;     // gamma * dy [A][d] fp16 (reused for dX rows)
+  uint16_t* dha;    // s dO Bd^T [A][r] fp16
+  uint16_t* dgu;    // dG | dU [A][2f] fp16
+  uint16_t* dxa;    // s [dG|dU] [Bg|Bu]^T [A][2r] fp16
+  int32_t* pre64;   // per-expert 64-row block prefix [E+1]
+};
+
+size_t bwd_extra_bytes(int T, const tqp_moe_weights* w) {
+  const size_t A = size_t(T) * w->top_k;
+  return align_up(A * 2 * w->ffn * 2, 256) * 2 + align_up(A * w->d * 2, 256) + align_up(A * w->rank * 2, 256) +
+         align_up(A * 2 * w->rank * 2, 256) + align_up(size_t(w->E + 1) * 4, 256) + 256;
+}
+
+BwdWs carve_bwd(void* p0, int T, const tqp_moe_weights* w) {
+  const size_t A = size_t(T) * w->top_k;
+  char* p = reinterpret_cast<char*>(align_up(reinterpret_cast<uintptr_t>(p0), 256));
+  BwdWs b;
+  auto take = [&](size_t bytes) {
+    char* q = p;
+    p += align_up(bytes, 256);
+    return static_cast<void*>(q);
+  };
+  b.gu = static_cast<uint16_t*>(take(A * 2 * w->ffn * 2));
+  b.dO = static_cast<uint16_t*>(take(A * w->d * 2));
+  b.dha = static_cast<uint16_t*>(take(A * w->rank * 2));
+  b.dgu = static_cast<uint16_t*>(take(A * 2 * w->ffn * 2));
+  b.dxa = static_cast<uint16_t*>(take(A * 2 * w->rank * 2));
+  b.pre64 = static_cast<int32_t*>(take(size_t(w->E + 1) * 4));
+  return b;
+}
+
+// Backward of one layer: recompute the forward (keeping G, U), then
+// combine/gate/router backward, dH (+SwiGLU backward) and dX on the tensor
+// cores, rank-space products and adapter gradients, and the token gather.
+int layer_backward(const uint16_t* x, const float* dy, int T, const tqp_moe_weights* w, float* dx,
+                   const tqp_adapter_grads* g, void* ws, int32_t* status, cudaStream_t s) {
+  const LayerWs L = carve_layer_ws(ws, T, w);
+  const BwdWs B = carve_bwd(static_cast<char*>(ws) + layer_ws_size(T, w), T, w);
+  const int k = w->top_k, d = w->d, f = w->ffn, r = w->rank, E = w->E;
+  const int A = T * k;
+  int rc;
+  if ((rc = layer_experts(x, T, w, L, status, s, B.gu)) != TQP_OK) return rc;
+  const FfnBufs fb = ffn_carve(L.ffn_ws, T, w);
+  if ((rc = launch_bwd_combine(L.out_perm, L.inv, L.gates, L.ids, w->router_w, dy, T, k, d, B.dO, dx, s)) != TQP_OK)
+    return rc;
+  if ((rc = launch_block_prefix(L.offsets, E, B.pre64, s)) != TQP_OK) return rc;
+  if (r > 0 && (rc = launch_rowgemm(0, B.dO, L.offsets, B.pre64, A, w, B.dha, s)) != TQP_OK) return rc;
+  if ((rc = launch_dgrad(0, B.dO, B.dha, L.offsets, fb.mb_prefix, w, T, B.gu, B.dgu, status, s)) != TQP_OK) return rc;
+  if (r > 0) {
+    if ((rc = launch_rowgemm(1, B.dgu, L.offsets, B.pre64, A, w, B.dxa, s)) != TQP_OK) return rc;
+    // adapter gradients, in the storage layouts A^T [r][in], B^T [out][r]
+    if ((rc = launch_outer(E, d, r, L.offsets, nullptr, B.dO, d, 0, fb.ha, r, 0, g->dB[2], s)) != TQP_OK) return rc;
+    if ((rc = launch_outer(E, r, f, L.offsets, nullptr, B.dha, r, 0, L.h, f, 0, g->dA[2], s)) != TQP_OK) return rc;
+    if ((rc = launch_outer(E, f, r, L.offsets, nullptr, B.dgu, 2 * f, 0, fb.xa, 2 * r, 0, g->dB[0], s)) != TQP_OK)
+      return rc;
+    if ((rc = launch_outer(E, f, r, L.offsets, nullptr, B.dgu, 2 * f, f, fb.xa, 2 * r, r, g->dB[1], s)) != TQP_OK)
+      return rc;
+    if ((rc = launch_outer(E, r, d, L.offsets, L.perm, B.dxa, 2 * r, 0, fb.x16, d, 0, g->dA[0], s)) != TQP_OK)
+      return rc;
+    if ((rc = launch_outer(E, r, d, L.offsets, L.perm, B.dxa, 2 * r, r, fb.x16, d, 0, g->dA[1], s)) != TQP_OK)
+      return rc;
+  }
+  uint16_t* dX = B.dO;  // dO is no longer needed
+  if ((rc = launch_dgrad(1, B.dgu, B.dxa, L.offsets, fb.mb_prefix, w, T, nullptr, dX, status, s)) != TQP_OK) return rc;
+  return launch_gather_add(dX, L.inv, T, k, d, dx, s);
 }
 
 int layer_forward(const uint16_t* x, int T, const tqp_moe_weights* w, const void* residual, int res_f32,
@@ -281,7 +351,7 @@ int rev_couple_inv(const float* y1, const float* y2, int T, const tqp_moe_weight
 
 size_t tqp_moe_layer_bwd_workspace_size(int T, const tqp_moe_weights* w) {
   if (check_weights(w) != TQP_OK || T < 0) return 0;
-  return layer_ws_size(T, w) + layer_bwd_ws_bytes(T, w);
+  return layer_ws_size(T, w) + bwd_extra_bytes(T, w);
 }
 
 int tqp_moe_layer_bwd(const uint16_t* x, const float* dy, int T, const tqp_moe_weights* w, float* dx,
@@ -290,12 +360,14 @@ int tqp_moe_layer_bwd(const uint16_t* x, const float* dy, int T, const tqp_moe_w
   if (rc != TQP_OK) return rc;
   const bool n = T > 0;
   if (T < 0 || !ptr_ok(x, n) || !ptr_ok(dy, n) || !ptr_ok(dx, n) || !grads) return TQP_ERR_INVALID_ARG;
+  if (w->ffn % 128 != 0) return TQP_ERR_UNSUPPORTED;   // the dH tiles are 128 columns of ffn
   if (w->rank > 0)
     for (int p = 0; p < 3; ++p)
       if (!grads->dA[p] || !grads->dB[p] || !aligned16(grads->dA[p]) || !aligned16(grads->dB[p]))
         return TQP_ERR_INVALID_ARG;
   if (n && (!ws || ws_bytes < tqp_moe_layer_bwd_workspace_size(T, w))) return TQP_ERR_WORKSPACE;
-  return launch_layer_bwd(x, dy, T, w, dx, grads, ws, dev_status, static_cast<cudaStream_t>(stream));
+  if (!n) return TQP_OK;
+  return layer_backward(x, dy, T, w, dx, grads, ws, dev_status, static_cast<cudaStream_t>(stream));
 }
 
 size_t tqp_adapter_bwd_workspace_size(int T, const tqp_moe_weights* F, const tqp_moe_weights* G) {
@@ -314,6 +386,7 @@ int tqp_adapter_bwd(const float* y1, const float* y2, const float* dy1, const fl
   int rc;
   if ((rc = check_weights(F)) != TQP_OK || (rc = check_weights(G)) != TQP_OK) return rc;
   if (F->d != G->d || T < 0 || !gF || !gG) return TQP_ERR_INVALID_ARG;
+  if (F->ffn % 128 != 0 || G->ffn % 128 != 0) return TQP_ERR_UNSUPPORTED;
   const bool n = T > 0;
   if (!ptr_ok(y1, n) || !ptr_ok(y2, n) || !ptr_ok(dy1, n) || !ptr_ok(dy2, n) || !ptr_ok(x1, n) || !ptr_ok(x2, n) ||
       !ptr_ok(dx1, n) || !ptr_ok(dx2, n))

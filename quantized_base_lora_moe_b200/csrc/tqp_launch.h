@@ -26,14 +26,32 @@ size_t router_ws_bytes(int T, const tqp_moe_weights* w);
 int launch_router_gemm(const uint16_t* x, int T, const tqp_moe_weights* w, float* logits, void* ws,
                        int32_t* status, cudaStream_t s);
 size_t ffn_ws_bytes(int T, const tqp_moe_weights* w);
+// Buffers inside the grouped-FFN workspace (valid after launch_grouped_ffn):
+// per-expert m-block prefix, x in fp16, s*X[Ag|Au] [A][2r] and s*H*Ad [A][r] (fp16).
+struct FfnBufs {
+  int32_t* mb_prefix;
+  uint16_t* x16;
+  uint16_t* xa;
+  uint16_t* ha;
+};
+FfnBufs ffn_carve(void* ws, int T, const tqp_moe_weights* w);
 int launch_grouped_ffn(const uint16_t* x, int T, const int32_t* offsets, const int32_t* perm_token,
                        const tqp_moe_weights* w, uint16_t* h, uint16_t* out_perm, void* ws, int32_t* status,
-                       cudaStream_t s);
+                       cudaStream_t s, uint16_t* aux_gu = nullptr);
+int launch_dgrad(int which, const uint16_t* a_src, const uint16_t* a_lora, const int32_t* offsets,
+                 const int32_t* mb_prefix, const tqp_moe_weights* w, int T, const uint16_t* aux_gu, uint16_t* out,
+                 int32_t* status, cudaStream_t s);
 
-// backward
-size_t layer_bwd_ws_bytes(int T, const tqp_moe_weights* w);
-int launch_layer_bwd(const uint16_t* x, const float* dy, int T, const tqp_moe_weights* w, float* dx,
-                     const tqp_adapter_grads* grads, void* ws, int32_t* status, cudaStream_t s);
+// backward pieces (layer_bwd.cu)
+int launch_bwd_combine(const uint16_t* O, const int32_t* inv, const float* gates, const int32_t* ids,
+                       const float* router_w, const float* dy, int T, int k, int d, uint16_t* dO, float* dx,
+                       cudaStream_t s);
+int launch_gather_add(const uint16_t* dX, const int32_t* inv, int T, int k, int d, float* dx, cudaStream_t s);
+int launch_block_prefix(const int32_t* offsets, int E, int32_t* pre, cudaStream_t s);
+int launch_rowgemm(int which, const uint16_t* P, const int32_t* offsets, const int32_t* pre, int A_rows,
+                   const tqp_moe_weights* w, uint16_t* C, cudaStream_t s);
+int launch_outer(int E, int M, int N, const int32_t* offsets, const int32_t* perm, const uint16_t* P, int ldp,
+                 int offp, const uint16_t* Q, int ldq, int offq, float* C, cudaStream_t s);
 
 int num_sms();
 

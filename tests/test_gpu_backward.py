@@ -1,0 +1,237 @@
+"""GPU parity of the backward path (layer backward, reversible block backward
+with activation reconstruction) against the fp64 oracle.
+
+Bars: dx, dA, dB max|err|/RMS(ref) <= 2e-2 per tensor; reconstruction of x1,
+x2 from the block outputs max|x - rec|/RMS(x) <= 5e-3. Tokens whose routing is
+ambiguous at the arithmetic's precision are excluded from the elementwise
+comparison, and so are the experts they touch (their gradient sums would
+differ by that token's contribution either way).
+"""
+import dataclasses
+
+import numpy as np
+import pytest
+import torch
+
+import synth
+from oracle import tqp_oracle as O
+from tests.gpu_util import dev, dev_bf16, host_bf16, near_tie_tokens, rel_err
+
+pytestmark = pytest.mark.gpu
+
+if torch.cuda.is_available():
+    import quantized_base_lora_moe_b200 as Q
+
+TOL = 2e-2
+BW1 = synth.LayerConfig("bw1", T=300, d=256, E=10, k=3, f=256, g=64, r=16)
+BW_ONE = synth.LayerConfig("bw_one", T=37, d=128, E=1, k=1, f=128, g=32, r=8)
+BW_R0 = synth.LayerConfig("bw_r0", T=50, d=128, E=4, k=4, f=128, g=128, r=0)
+BW_SKEW = synth.LayerConfig("bw_skew", T=600, d=256, E=12, k=2, f=256, g=64, r=16, zipf_s=1.1)
+LAYER_CFGS = [synth.TINY, BW1, BW_ONE, BW_R0, BW_SKEW, synth.MID]
+
+
+@pytest.fixture(scope="module", autouse=True)
+def _cuda():
+    if not torch.cuda.is_available():
+        pytest.skip("needs a CUDA device")
+    Q.lib()
+
+
+def ambiguous_experts(logits, k, margin):
+    """Experts at the k-th / (k+1)-th place of tokens whose gap is below margin."""
+    tie = near_tie_tokens(logits, k, margin)
+    srt = np.argsort(-logits[tie], axis=1, kind="stable")
+    ex = set(srt[:, k - 1].tolist()) | set(srt[:, k].tolist()) if k < logits.shape[1] and tie.any() else set()
+    return tie, ex
+
+
+def gpu_layer_bwd(cfg, raw, xb, dy):
+    L = Q.DeviceLayer(raw)
+    dx = torch.empty(cfg.T, cfg.d, dtype=torch.float32, device="cuda")
+    dA, dB, g = L.grads()
+    st = Q.Status()
+    Q.tqp_moe_layer_bwd(dev_bf16(xb), dev(dy), L, dx, g, status=st)
+    torch.cuda.synchronize()
+    assert st.read() == 0
+    return dx.cpu().numpy(), [t.cpu().numpy() for t in dA], [t.cpu().numpy() for t in dB]
+
+
+@pytest.mark.parametrize("cfg", LAYER_CFGS, ids=lambda c: c.name)
+def test_layer_bwd_matches_oracle(cfg):
+    raw = synth.make_layer(cfg)
+    L = O.Layer(raw)
+    xb = synth.make_tokens(cfg.T, cfg.d, 31)
+    dy = synth.make_grad(cfg.T, cfg.d, 32, "dy1")
+    x = O.bf16_to_f64(xb)
+    dx, dA, dB = gpu_layer_bwd(cfg, raw, xb, dy)
+    rdx, rdA, rdB = O.layer_backward(x, dy.astype(np.float64), L)
+    tie, amb = ambiguous_experts(O.router_logits(x, L), cfg.k, 1e-4)
+    assert tie.mean() < 0.02
+    assert rel_err(dx[~tie], rdx[~tie]) <= TOL
+    keep = np.array([e not in amb for e in range(cfg.E)])
+    if cfg.r > 0:
+        for p in range(3):
+            assert rel_err(dA[p][keep], rdA[p][keep]) <= TOL, ("dA", p)
+            assert rel_err(dB[p][keep], rdB[p][keep]) <= TOL, ("dB", p)
+
+
+def test_layer_bwd_rejects_ffn_not_multiple_of_128():
+    cfg = synth.LayerConfig("f192", T=16, d=128, E=4, k=2, f=192, g=64, r=8)
+    raw = synth.make_layer(cfg)
+    with pytest.raises(Q.TQPError) as ei:
+        gpu_layer_bwd(cfg, raw, synth.make_tokens(16, 128, 1), synth.make_grad(16, 128, 1, "dy1"))
+    assert ei.value.code == -2
+
+
+def test_layer_bwd_deterministic():
+    cfg = BW1
+    raw = synth.make_layer(cfg)
+    xb = synth.make_tokens(cfg.T, cfg.d, 33)
+    dy = synth.make_grad(cfg.T, cfg.d, 34, "dy1")
+    a = gpu_layer_bwd(cfg, raw, xb, dy)
+    b = gpu_layer_bwd(cfg, raw, xb, dy)
+    assert np.array_equal(a[0], b[0])
+    for p in range(3):
+        assert np.array_equal(a[1][p], b[1][p]) and np.array_equal(a[2][p], b[2][p])
+
+
+# ---------------------------------------------------------------- reversible block
+
+
+REV_TINY = (synth.TINY, dataclasses.replace(synth.TINY, seed=1))
+REV_MID = (synth.LayerConfig("rb", T=512, d=256, E=16, k=4, f=256, g=64, r=16),
+           synth.LayerConfig("rb", T=512, d=256, E=16, k=4, f=256, g=64, r=16, seed=1))
+
+
+def gpu_block(cfgF, cfgG, rawF, rawG, x1b, x2b, dy1, dy2):
+    F, G = Q.DeviceLayer(rawF), Q.DeviceLayer(rawG)
+    T, d = x1b.shape
+    y1 = torch.empty(T, d, dtype=torch.float32, device="cuda")
+    y2 = torch.empty_like(y1)
+    st = Q.Status()
+    Q.rev_couple_fwd(dev_bf16(x1b), dev_bf16(x2b), F, G, y1, y2, status=st)
+    r1 = torch.empty(T, d, dtype=torch.int16, device="cuda")
+    r2 = torch.empty_like(r1)
+    dx1 = torch.empty(T, d, dtype=torch.float32, device="cuda")
+    dx2 = torch.empty_like(dx1)
+    dAF, dBF, gF = F.grads()
+    dAG, dBG, gG = G.grads()
+    Q.tqp_adapter_bwd(y1, y2, dev(dy1), dev(dy2), F, G, r1, r2, dx1, dx2, gF, gG, status=st)
+    torch.cuda.synchronize()
+    assert st.read() == 0
+    c = lambda ts: [t.cpu().numpy() for t in ts]
+    return {"x1": host_bf16(r1), "x2": host_bf16(r2), "dx1": dx1.cpu().numpy(), "dx2": dx2.cpu().numpy(),
+            "dA_F": c(dAF), "dB_F": c(dBF), "dA_G": c(dAG), "dB_G": c(dBG)}
+
+
+@pytest.mark.parametrize("cfgs", [REV_TINY, REV_MID], ids=["tiny", "mid"])
+def test_adapter_bwd_block_matches_oracle(cfgs):
+    cfgF, cfgG = cfgs
+    rawF, rawG = synth.make_layer(cfgF, cfgF.seed), synth.make_layer(cfgG, cfgG.seed)
+    T, d = cfgF.T, cfgF.d
+    x1b, x2b = synth.make_tokens(T, d, 2), synth.make_tokens(T, d, 3)
+    dy1, dy2 = synth.make_grad(T, d, 4, "dy1"), synth.make_grad(T, d, 4, "dy2")
+    got = gpu_block(cfgF, cfgG, rawF, rawG, x1b, x2b, dy1, dy2)
+    x1, x2 = O.bf16_to_f64(x1b), O.bf16_to_f64(x2b)
+    # reconstruction is exact: the backward recomputes bit-identical F and G
+    rms = np.sqrt(np.mean(np.concatenate([x1, x2]) ** 2))
+    assert max(np.max(np.abs(got["x1"] - x1)), np.max(np.abs(got["x2"] - x2))) / rms <= 5e-3
+    LF, LG = O.Layer(rawF), O.Layer(rawG)
+    y1, y2 = O.coupling_forward(x1, x2, LF, LG)
+    ref = O.block_backward(y1, y2, dy1.astype(np.float64), dy2.astype(np.float64), LF, LG)
+    # ambiguous routing: F near ties, and G tokens whose routing moves when F's
+    # output moves by its own rounding (see test_rev_couple_fwd_inverse)
+    tieF, ambF = ambiguous_experts(O.router_logits(x2, LF), cfgF.k, 1e-4)
+    f_ref = y1 - x1
+    rng = np.random.default_rng(7)
+    z = O.round_bf16(y1)
+    zp = O.round_bf16(x1 + f_ref * (1.0 + 2.0 ** -8 * rng.uniform(-1.0, 1.0, f_ref.shape)))
+    lz = O.router_logits(z, LG)
+    flip = np.any(O.topk(lz, cfgG.k) != O.topk(O.router_logits(zp, LG), cfgG.k), axis=1)
+    tieG, ambG = ambiguous_experts(lz, cfgG.k, 5e-3)
+    tieG |= flip
+    for t in np.nonzero(flip)[0]:
+        ambG |= set(O.topk(lz[t:t + 1], cfgG.k)[0].tolist()) | set(O.topk(O.router_logits(zp[t:t + 1], LG),
+                                                                            cfgG.k)[0].tolist())
+    # a G-ambiguous token also changes F's cotangent dz1 at that token, so F's experts of that token too
+    ambF_from_G = set(O.topk(O.router_logits(x2[tieG], LF), cfgF.k).ravel().tolist()) if tieG.any() else set()
+    keep_t = ~(tieF | tieG)
+    assert keep_t.mean() > 0.7
+    kF = np.array([e not in (ambF | ambF_from_G) for e in range(cfgF.E)])
+    kG = np.array([e not in ambG for e in range(cfgG.E)])
+    # G runs on bf16(y1), which carries F's rounding: the oracle measures how far
+    # each result moves when F's output moves by 2^-8 relative (zp above), and the
+    # bound is TOL plus twice that spread.
+    dy1_, dy2_ = dy1.astype(np.float64), dy2.astype(np.float64)
+    dxGp, dAGp, dBGp = O.layer_backward(zp, dy2_, LG)
+    dz1p = dy1_ + dxGp
+    dxFp, dAFp, dBFp = O.layer_backward(ref["x2"], dz1p, LF)
+    pert = {"dx1": dz1p, "dx2": dy2_ + dxFp, "dA_F": dAFp, "dB_F": dBFp, "dA_G": dAGp, "dB_G": dBGp}
+
+    def check(key, sel, p=None):
+        g = got[key] if p is None else got[key][p]
+        r = ref[key] if p is None else ref[key][p]
+        q = pert[key] if p is None else pert[key][p]
+        spread = rel_err(q[sel], r[sel])
+        err = rel_err(g[sel], r[sel])
+        assert err <= TOL + 2 * spread, (key, p, err, spread)
+
+    check("dx1", keep_t)
+    check("dx2", keep_t)
+    for p in range(3):
+        if kF.any():
+            check("dA_F", kF, p)
+            check("dB_F", kF, p)
+        if kG.any():
+            check("dA_G", kG, p)
+            check("dB_G", kG, p)
+
+
+def test_adapter_bwd_full_size_reconstruction_and_sampled_tokens():
+    """The 460-expert top-12 block (F, G independent instances) at T=8192:
+    reconstruction over all tokens, and dx1/dx2 on sampled tokens against the
+    oracle evaluated token by token."""
+    cfgF, cfgG = synth.REV_F, synth.REV_G
+    rawF, rawG = synth.make_layer(cfgF, cfgF.seed), synth.make_layer(cfgG, cfgG.seed)
+    T, d = cfgF.T, cfgF.d
+    x1b = synth.make_tokens(T, d, synth.REV_SEEDS["x1"])
+    x2b = synth.make_tokens(T, d, synth.REV_SEEDS["x2"])
+    dy1 = synth.make_grad(T, d, synth.REV_SEEDS["dy"], "dy1")
+    dy2 = synth.make_grad(T, d, synth.REV_SEEDS["dy"], "dy2")
+    got = gpu_block(cfgF, cfgG, rawF, rawG, x1b, x2b, dy1, dy2)
+    x1, x2 = O.bf16_to_f64(x1b), O.bf16_to_f64(x2b)
+    rms = np.sqrt(np.mean(np.concatenate([x1, x2]) ** 2))
+    assert max(np.max(np.abs(got["x1"] - x1)), np.max(np.abs(got["x2"] - x2))) / rms <= 5e-3
+    assert all(np.isfinite(got[k]).all() for k in ("dx1", "dx2"))
+    LF, LG = O.Layer(rawF), O.Layer(rawG)
+    toks = [0, T - 1, 1234, 4321, 777, 6000]
+    rng = np.random.default_rng(9)
+    ok_rows, g1, g2, r1s, r2s, p1s, p2s = [], [], [], [], [], [], []
+    for t in toks:
+        yF, idF, _, lF = O.token_forward(x2[t], LF)
+        y1t = x1[t] + yF
+        z = O.round_bf16(y1t)[None, :]
+        zp = O.round_bf16(x1[t] + yF * (1.0 + 2.0 ** -8 * rng.uniform(-1.0, 1.0, yF.shape)))[None, :]
+        lG = O.router_logits(z, LG)
+        amb = (O.routing_gap(lF[None, :], cfgF.k)[0] < 1e-4) or (O.routing_gap(lG, cfgG.k)[0] < 2e-2) or \
+            np.any(O.topk(lG, cfgG.k) != O.topk(O.router_logits(zp, LG), cfgG.k))
+        if amb:
+            continue
+        dy1t, dy2t = dy1[t:t + 1].astype(np.float64), dy2[t:t + 1].astype(np.float64)
+        dz1 = dy1t + O.layer_backward(z, dy2t, LG)[0]
+        dz1p = dy1t + O.layer_backward(zp, dy2t, LG)[0]
+        ok_rows.append(t)
+        g1.append(got["dx1"][t])
+        g2.append(got["dx2"][t])
+        r1s.append(dz1[0])
+        r2s.append(dy2t[0] + O.layer_backward(x2[t:t + 1], dz1, LF)[0][0])
+        p1s.append(dz1p[0])
+        p2s.append(dy2t[0] + O.layer_backward(x2[t:t + 1], dz1p, LF)[0][0])
+    assert len(ok_rows) >= 4
+    # tolerance: TOL plus twice the oracle's own spread when F's output moves by 2^-8 relative
+    s1 = rel_err(np.array(p1s), np.array(r1s))
+    s2 = rel_err(np.array(p2s), np.array(r2s))
+    e1 = rel_err(np.array(g1), np.array(r1s))
+    e2 = rel_err(np.array(g2), np.array(r2s))
+    assert e1 <= TOL + 2 * s1, (e1, s1)
+    assert e2 <= TOL + 2 * s2, (e2, s2)
