@@ -1,27 +1,32 @@
 // Grouped tensor-core GEMM engine for the TQP MoE layer (sm_100a, tcgen05).
 //
 // One persistent, warp-specialised kernel template serves every contraction of
-// the forward path:
-//   GATEUP  : [G|U] = X_e Wg/u^T (+ s (X Ag/u) Bg/u), H = bf16(silu(G) * U)
-//   DOWN    : O = bf16(H_e Wd^T + s (H Ad) Bd)
-//   LORA_XA : xa = bf16(s * X_e [Ag | Au])        (rank-space input of gate/up)
-//   LORA_HA : ha = bf16(s * H_e Ad)               (rank-space input of down)
+// the layer ("Train low-rank adapters per expert" over "Quantize base expert
+// weights", Pattern 3; "Router: Full precision", TQP Quantization):
+//   GATEUP  : [G|U] = X_e [Wg|Wu]^T + s (X [Ag|Au]) [Bg|Bu],  H = silu(G) * U   (fp16)
+//   DOWN    : O = H_e Wd^T + s (H Ad) Bd                                          (fp16)
+//   LORA_XA : xa = s * X_e [Ag | Au]            (bf16 operands, fp16 out)
+//   LORA_HA : ha = s * H_e Ad                   (fp16)
 //   ROUTER  : logits = x W_r^T (+ bias), W_r split exactly into 3 bf16 parts
-// ("Train low-rank adapters per expert" over "Quantize base expert weights",
-// Pattern 3; "Router: Full precision", TQP Quantization.)
+//   DH      : dH = dO Wd + dhA Ad^T, with the SwiGLU backward in the epilogue
+//   DX      : dX = [dG|dU] [Wg;Wu] + dxa [Ag;Au]^T
 //
-// Work unit = (expert e, n-tile, m-block of up to 256 routed rows). Per CTA (1
-// per SM, 576 threads):
-//   warps 0-3   epilogue: tcgen05.ld from TMEM, activation, bf16 stores
-//   warp  4     TMEM allocation + one thread issuing tcgen05.mma (M=128 per
-//               sub-tile, two sub-tiles share each B tile)
-//   warp  5     TMA producer: int4 code tiles + bf16 group scales
-//   warps 6-9   A producer: cp.async 16-byte row gathers into 128B-swizzled tiles
-//   warps 10-17 B producer: int4 -> bf16 dequant (or bf16 copies) into
-//               128B-swizzled K-major tiles
-// Accumulators are double-buffered in TMEM (2 x 2 x 128 fp32 columns), so the
-// epilogue of one unit overlaps the main loop of the next.
+// Work unit = (expert e, n-tile of up to 256 columns, m-block of up to 128
+// routed rows); one 128 x N x 64 tcgen05.mma step per K-block. Per CTA (1 per
+// SM, 576 threads):
+//   warps 0-3   epilogue: tcgen05.ld from TMEM, activation, stores
+//   warp  4     TMEM allocation + one thread issuing tcgen05.mma
+//   warp  5     TMA producer of the int4 code / bf16 scale ring
+//   warps 6-9   A producer: TMA 128B-swizzled tiles for contiguous rows, or
+//               cp.async 16-byte row gathers (rows picked by perm_token); the
+//               rank-space (LoRA) A tiles; TMA B tiles of the rank-space GEMMs
+//   warps 10-17 B producer: int4 -> fp16 dequantisation (transposed for the
+//               dgrads) into 128B-swizzled K-major tiles, LoRA B^T tiles
+// Accumulators are double-buffered in TMEM (2 x 256 fp32 columns), so the
+// epilogue of one unit overlaps the main loop of the next. Operand stages:
+// 4 x (16 KB A + 32 KB B); code ring: 3 x 9 KB. No TMA multicast is used.
 #include <cstdint>
+#include <cstring>
 #include <cuda.h>
 #include <cudaTypedefs.h>
 #include <cuda_runtime.h>
@@ -34,56 +39,54 @@ namespace tqp {
 enum Mode : int { GATEUP = 0, DOWN = 1, LORA_XA = 2, LORA_HA = 3, ROUTER = 4, DH = 5, DX = 6 };
 
 constexpr int kThreads = 576;
-constexpr int kStages = 4;          // operand ring (A: 2 x 16 KB, B: 16 KB)
-constexpr int kQStages = 4;         // int4 + scale ring
-constexpr int kAStageBytes = 32768;
-constexpr int kBStageBytes = 16384;
-constexpr int kOpStageBytes = kAStageBytes + kBStageBytes;
-constexpr int kQStageBytes = 5120;  // 4096 B codes + up to 1024 B scales
-constexpr int kMBlock = 256;
+constexpr int kAStages = 5;           // A tiles (TMA / cp.async from L2): deep, to cover L2 latency
+constexpr int kBStages = 2;           // dequantised B tiles, produced just ahead of the MMA
+constexpr int kQStages = 8;           // int4 codes + scales from DRAM: deepest prefetch
+constexpr int kAStageBytes = 16384;   // 128 rows x 64 K x 2 B
+constexpr int kBStageBytes = 32768;   // up to 256 rows x 64 K x 2 B
+constexpr int kQStageBytes = 9216;    // up to 8192 B of codes + 1024 B of scales
+constexpr int kMBlock = 128;
 
 struct GemmArgs {
   int E;
   int nkb_main;        // main K-blocks (64 wide)
-  int kb_per_piece;    // ROUTER: K-blocks per bf16 piece (A columns repeat)
-  int nkb_lora;        // extra K-blocks of the LoRA term
-  int lora_k;          // LoRA contraction extent (2r gate/up, r down)
+  int kb_per_piece;    // ROUTER: K-blocks per bf16 part (the A columns repeat)
+  int nkb_lora;        // rank-space K-blocks, issued first in each unit
+  int lora_k;          // rank-space contraction extent (2r gate/up and dX, r down and dH)
   int n_tiles;         // n-tiles per m-block
-  int ntile;           // MMA N
+  int ntile;           // MMA N (16..256)
   int g;               // quantisation group
   int r;               // LoRA rank
-  int in_dim;          // K of the int4 projection (for scale rows)
-  int out_dim;         // rows of one expert's int4 projection
+  int in_dim;          // input dim of the int4 projection (scale rows)
+  int out_dim;         // output dim of the int4 projection (code rows)
   float lora_scale;
   const int32_t* offsets;
   const int32_t* mb_prefix;
   const int32_t* perm_token;
-  const uint16_t* a_src;
+  const uint16_t* a_src;   // gathered A rows (GATEUP, LORA_XA)
   int a_ld;
-  const uint16_t* a_lora;
+  const uint16_t* a_lora;  // rank-space A rows [A][lora_ld]
   int lora_ld;
-  const uint16_t* b0;   // bf16 B source 0 (Ag^T / Ad^T / router parts) or lora B^T (gate / down)
-  const uint16_t* b1;   // bf16 B source 1 (Au^T) or lora Bu^T
-  const uint8_t* wq0;   // int4 codes (gate or down) and scales, for direct loads
-  const uint8_t* wq1;
-  const uint16_t* ws0;
-  const uint16_t* ws1;
+  const uint16_t* b0;      // rank-space B^T sources (GATEUP: Bg^T, DOWN: Bd^T)
+  const uint16_t* b1;      // GATEUP: Bu^T
   void* out;
   int out_ld;
-  int n_valid;          // valid output columns (ROUTER: E)
-  uint16_t* aux;        // GATEUP: optional G|U pre-activations out [A][2f]; DH: G|U in
-  int f_dim;            // ffn (GATEUP aux / DH epilogue)
-  int half_kb;          // DX: K-blocks of the gate part (then the up part)
-  const uint16_t* lb0;  // DH / DX LoRA step: A^T sources read transposed (Ad^T | Ag^T)
-  const uint16_t* lb1;  // DX: Au^T
-  int lb_ld;            // row length of lb0 / lb1
+  int n_valid;             // valid output columns
   const float* bias;
   int32_t* status;
+  uint16_t* aux;           // GATEUP: optional G|U pre-activations out [A][2f]; DH: G|U in
+  int f_dim;
+  int half_kb;             // DX: K-blocks of the gate part
+  const uint16_t* lb0;     // DH / DX rank-space step: A^T sources read transposed (Ad^T | Ag^T)
+  const uint16_t* lb1;     // DX: Au^T
+  int lb_ld;
 };
 
 struct SmemCtl {
-  uint64_t op_full[kStages];
-  uint64_t op_empty[kStages];
+  uint64_t a_full[kAStages];
+  uint64_t a_empty[kAStages];
+  uint64_t b_full[kBStages];
+  uint64_t b_empty[kBStages];
   uint64_t q_full[kQStages];
   uint64_t q_empty[kQStages];
   uint64_t acc_full[2];
@@ -93,8 +96,9 @@ struct SmemCtl {
   int abort_flag;
 };
 
-constexpr size_t kSmemBytes = 1024 /*align slack*/ + size_t(kStages) * kOpStageBytes +
-                              size_t(kQStages) * kQStageBytes + sizeof(SmemCtl);
+constexpr size_t kSmemBytes = 1024 /*align slack*/ + size_t(kAStages) * kAStageBytes +
+                              size_t(kBStages) * kBStageBytes + size_t(kQStages) * kQStageBytes + sizeof(SmemCtl);
+static_assert(kSmemBytes <= 232448, "shared memory budget");
 
 struct Unit {
   int e, nt, mb, rows, base;
@@ -102,8 +106,10 @@ struct Unit {
 
 __device__ __forceinline__ int total_units(const GemmArgs& a) { return __ldg(a.mb_prefix + a.E) * a.n_tiles; }
 
+// Units are ordered (expert, n-tile, m-block): m-blocks of one n-tile share a B
+// tile, n-tiles of one m-block share the A rows; neighbours run concurrently.
 __device__ __forceinline__ Unit decode_unit(const GemmArgs& a, int u) {
-  int lo = 0, hi = a.E;  // find e with mb_prefix[e]*nt <= u < mb_prefix[e+1]*nt
+  int lo = 0, hi = a.E;
   while (hi - lo > 1) {
     const int mid = (lo + hi) >> 1;
     if (__ldg(a.mb_prefix + mid) * a.n_tiles <= u) lo = mid;
@@ -132,6 +138,10 @@ struct Ring {
   }
 };
 
+__device__ __forceinline__ void mbar_expect_tx(uint64_t* bar, uint32_t bytes) {
+  asm volatile("mbarrier.expect_tx.shared::cta.b64 [%0], %1;" ::"r"(smem_u32(bar)), "r"(bytes) : "memory");
+}
+
 __device__ __forceinline__ uint32_t f16x2_sub(uint32_t a, uint32_t b) {
   uint32_t d;
   asm("sub.rn.f16x2 %0, %1, %2;" : "=r"(d) : "r"(a), "r"(b));
@@ -159,17 +169,48 @@ __device__ __forceinline__ uint4 dequant_word(uint32_t w, uint32_t s2) {
   return make_uint4(o[0], o[1], o[2], o[3]);
 }
 
+__device__ __forceinline__ uint32_t scale_pair(uint16_t sbits) {
+  const uint32_t sh = __half_as_ushort(__float2half_rn(bf16_to_f32(sbits)));
+  return sh | (sh << 16);
+}
+
+// One B-tile row (forward): NW int4 words (8 K values each) of row `brow`
+// starting at chunk part*NW, dequantised into the 128B-swizzled K-major tile.
+// s_lo / s_hi: fp16 scale pairs of the first / second 32-wide group (equal when g >= 64).
+template <int NW>
+__device__ __forceinline__ void dequant_row(const uint8_t* qs, uint8_t* bst, int brow, int part, uint32_t s_lo,
+                                            uint32_t s_hi) {
+  uint32_t w[NW];
+#pragma unroll
+  for (int i = 0; i < NW; i += 4) {
+    const uint4 v = *reinterpret_cast<const uint4*>(qs + brow * 32 + part * NW * 4 + i * 4);
+    w[i] = v.x; w[i + 1] = v.y; w[i + 2] = v.z; w[i + 3] = v.w;
+  }
+  uint8_t* rowp = bst + (brow >> 3) * 1024 + (brow & 7) * 128;
+  const int x = brow & 7;
+#pragma unroll
+  for (int i = 0; i < NW; ++i) {
+    const int c = part * NW + i;
+    *reinterpret_cast<uint4*>(rowp + ((c ^ x) << 4)) = dequant_word(w[i], c < 4 ? s_lo : s_hi);
+  }
+}
+
 template <int MODE>
 __global__ void __launch_bounds__(kThreads, 1)
     grouped_gemm_kernel(const GemmArgs a, const __grid_constant__ CUtensorMap tq0,
                         const __grid_constant__ CUtensorMap tq1, const __grid_constant__ CUtensorMap ts0,
-                        const __grid_constant__ CUtensorMap ts1) {
-  constexpr bool kTrans = (MODE == DH || MODE == DX);   // B = W^T: dequantised transposed
+                        const __grid_constant__ CUtensorMap ts1, const __grid_constant__ CUtensorMap ta,
+                        const __grid_constant__ CUtensorMap tb0, const __grid_constant__ CUtensorMap tb1) {
+  constexpr bool kTrans = (MODE == DH || MODE == DX);      // B = W^T: dequantised transposed
   constexpr bool kDequant = (MODE == GATEUP || MODE == DOWN || kTrans);
+  constexpr bool kATma = (MODE == DOWN || MODE == LORA_HA || MODE == ROUTER || kTrans);
+  constexpr bool kBTma = (MODE == LORA_XA || MODE == LORA_HA || MODE == ROUTER);
+  constexpr bool kBf16 = (MODE == LORA_XA || MODE == ROUTER);
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
-  uint8_t* op_base = smem;
-  uint8_t* q_base = smem + size_t(kStages) * kOpStageBytes;
+  uint8_t* a_base = smem;
+  uint8_t* b_base = a_base + size_t(kAStages) * kAStageBytes;
+  uint8_t* q_base = b_base + size_t(kBStages) * kBStageBytes;
   SmemCtl* ctl = reinterpret_cast<SmemCtl*>(q_base + size_t(kQStages) * kQStageBytes);
   volatile int* abort_flag = &ctl->abort_flag;
 
@@ -177,9 +218,13 @@ __global__ void __launch_bounds__(kThreads, 1)
   const int lane = threadIdx.x & 31;
 
   if (threadIdx.x == 0) {
-    for (int i = 0; i < kStages; ++i) {
-      mbar_init(&ctl->op_full[i], 128 + 256);
-      mbar_init(&ctl->op_empty[i], 1);
+    for (int i = 0; i < kAStages; ++i) {
+      mbar_init(&ctl->a_full[i], 128);
+      mbar_init(&ctl->a_empty[i], 1);
+    }
+    for (int i = 0; i < kBStages; ++i) {
+      mbar_init(&ctl->b_full[i], kBTma ? 257 : 256);   // + the TMA issuer's arrival
+      mbar_init(&ctl->b_empty[i], 1);
     }
     for (int i = 0; i < kQStages; ++i) {
       mbar_init(&ctl->q_full[i], 1);
@@ -197,13 +242,18 @@ __global__ void __launch_bounds__(kThreads, 1)
     tmem_alloc(&ctl->tmem_base, 512);
     tmem_relinquish();
   }
-  if (warp == 5 && lane == 0 && kDequant) {
+  if (threadIdx.x == 5 * 32 && kDequant) {
     prefetch_tmap(&tq0);
     prefetch_tmap(&ts0);
     if (MODE == GATEUP || MODE == DX) {
       prefetch_tmap(&tq1);
       prefetch_tmap(&ts1);
     }
+  }
+  if (threadIdx.x == 6 * 32) {
+    if (kATma) prefetch_tmap(&ta);
+    if (kBTma) prefetch_tmap(&tb0);
+    if (MODE == LORA_XA) prefetch_tmap(&tb1);
   }
   tc_fence_before();
   __syncthreads();
@@ -215,127 +265,122 @@ __global__ void __launch_bounds__(kThreads, 1)
 
   if (warp < 4) {
     // ------------------------------------------------------------ epilogue
-    const int row_in_sub = warp * 32 + lane;
+    const int row = warp * 32 + lane;
     int it = 0;
     for (int u = blockIdx.x; u < nunits; u += gridDim.x, ++it) {
       const Unit un = decode_unit(a, u);
       const int ab = it & 1;
       const uint32_t aph = uint32_t(it >> 1) & 1u;
-      if (!mbar_wait(&ctl->acc_full[ab], aph, abort_flag, a.status)) break;
+      if (!mbar_wait<128>(&ctl->acc_full[ab], aph, abort_flag, a.status)) break;
       tc_fence_after();
-      const int nsub = un.rows > 128 ? 2 : 1;
-      for (int sub = 0; sub < nsub; ++sub) {
-        const int row = sub * 128 + row_in_sub;
-        const bool valid = row < un.rows;
-        const size_t grow = size_t(un.base) + row;
-        const uint32_t tacc = tmem_base + (uint32_t(warp * 32) << 16) + uint32_t(ab * 256 + sub * 128);
-        if (MODE == GATEUP) {
-          uint16_t* hrow = static_cast<uint16_t*>(a.out) + grow * a.out_ld + un.nt * 64;
+      const bool valid = row < un.rows;
+      const size_t grow = size_t(un.base) + row;
+      const uint32_t tacc = tmem_base + (uint32_t(warp * 32) << 16) + uint32_t(ab * 256);
+      if (MODE == GATEUP) {
+        const int half = a.ntile >> 1;
+        uint16_t* hrow = static_cast<uint16_t*>(a.out) + grow * a.out_ld + un.nt * half;
 #pragma unroll 1
-          for (int c = 0; c < 64; c += 32) {
-            float gv[32], uv[32];
-            tmem_ld32(tacc + c, gv);
-            tmem_ld32(tacc + 64 + c, uv);
-            uint32_t pk[16];
+        for (int c = 0; c < half; c += 32) {
+          float gv[32], uv[32];
+          tmem_ld32(tacc + c, gv);
+          tmem_ld32(tacc + half + c, uv);
+          uint32_t pk[16];
 #pragma unroll
-            for (int i = 0; i < 16; ++i) {
-              const float g0 = gv[2 * i], g1 = gv[2 * i + 1];
-              const float h0 = g0 / (1.0f + __expf(-g0)) * uv[2 * i];
-              const float h1 = g1 / (1.0f + __expf(-g1)) * uv[2 * i + 1];
-              pk[i] = pack_f16x2(h0, h1);
+          for (int i = 0; i < 16; ++i) {
+            const float g0 = gv[2 * i], g1 = gv[2 * i + 1];
+            const float h0 = g0 / (1.0f + __expf(-g0)) * uv[2 * i];
+            const float h1 = g1 / (1.0f + __expf(-g1)) * uv[2 * i + 1];
+            pk[i] = pack_f16x2(h0, h1);
+          }
+          if (valid) {
+            uint4* dst = reinterpret_cast<uint4*>(hrow + c);
+#pragma unroll
+            for (int i = 0; i < 4; ++i) dst[i] = make_uint4(pk[4 * i], pk[4 * i + 1], pk[4 * i + 2], pk[4 * i + 3]);
+            if (a.aux) {  // keep the pre-activations for the backward
+              uint16_t* gr = a.aux + grow * (2 * size_t(a.f_dim)) + un.nt * half + c;
+              uint4* ga = reinterpret_cast<uint4*>(gr);
+              uint4* ua = reinterpret_cast<uint4*>(gr + a.f_dim);
+#pragma unroll
+              for (int i = 0; i < 4; ++i) {
+                ga[i] = make_uint4(pack_f16x2(gv[8 * i], gv[8 * i + 1]), pack_f16x2(gv[8 * i + 2], gv[8 * i + 3]),
+                                   pack_f16x2(gv[8 * i + 4], gv[8 * i + 5]), pack_f16x2(gv[8 * i + 6], gv[8 * i + 7]));
+                ua[i] = make_uint4(pack_f16x2(uv[8 * i], uv[8 * i + 1]), pack_f16x2(uv[8 * i + 2], uv[8 * i + 3]),
+                                   pack_f16x2(uv[8 * i + 4], uv[8 * i + 5]), pack_f16x2(uv[8 * i + 6], uv[8 * i + 7]));
+              }
             }
-            if (valid) {
-              uint4* dst = reinterpret_cast<uint4*>(hrow + c);
+          }
+        }
+      } else if (MODE == DH) {
+        // dH -> dG = dH * U * silu'(G), dU = dH * silu(G); G, U from the recompute
+        const size_t ld2 = 2 * size_t(a.f_dim);
+        const uint16_t* grow_gu = a.aux + grow * ld2 + un.nt * a.ntile;
+        uint16_t* drow = static_cast<uint16_t*>(a.out) + grow * ld2 + un.nt * a.ntile;
+#pragma unroll 1
+        for (int c = 0; c < a.ntile; c += 32) {
+          float v[32];
+          tmem_ld32(tacc + c, v);
+          if (valid) {
+#pragma unroll
+            for (int q = 0; q < 4; ++q) {
+              const uint4 gq = *reinterpret_cast<const uint4*>(grow_gu + c + 8 * q);
+              const uint4 uq = *reinterpret_cast<const uint4*>(grow_gu + a.f_dim + c + 8 * q);
+              const uint32_t gw[4] = {gq.x, gq.y, gq.z, gq.w};
+              const uint32_t uw[4] = {uq.x, uq.y, uq.z, uq.w};
+              uint32_t dg[4], du[4];
+#pragma unroll
+              for (int t = 0; t < 4; ++t) {
+                float res_g[2], res_u[2];
+#pragma unroll
+                for (int hh = 0; hh < 2; ++hh) {
+                  const float g = f16_to_f32(uint16_t(hh ? (gw[t] >> 16) : (gw[t] & 0xFFFFu)));
+                  const float u = f16_to_f32(uint16_t(hh ? (uw[t] >> 16) : (uw[t] & 0xFFFFu)));
+                  const float dh = v[8 * q + 2 * t + hh];
+                  const float sg = 1.0f / (1.0f + __expf(-g));
+                  res_g[hh] = dh * u * sg * (1.0f + g * (1.0f - sg));
+                  res_u[hh] = dh * g * sg;
+                }
+                dg[t] = pack_f16x2(res_g[0], res_g[1]);
+                du[t] = pack_f16x2(res_u[0], res_u[1]);
+              }
+              *reinterpret_cast<uint4*>(drow + c + 8 * q) = make_uint4(dg[0], dg[1], dg[2], dg[3]);
+              *reinterpret_cast<uint4*>(drow + a.f_dim + c + 8 * q) = make_uint4(du[0], du[1], du[2], du[3]);
+            }
+          }
+        }
+      } else if (MODE == ROUTER) {
+        float* lrow = static_cast<float*>(a.out) + grow * a.out_ld;
+#pragma unroll 1
+        for (int c = 0; c < a.ntile; c += 32) {
+          float v[32];
+          tmem_ld32(tacc + c, v);
+          const int n0 = un.nt * a.ntile + c;
+          if (valid) {
+#pragma unroll
+            for (int i = 0; i < 32; ++i) {
+              const int n = n0 + i;
+              if (n < a.n_valid) lrow[n] = v[i] + (a.bias ? __ldg(a.bias + n) : 0.0f);
+            }
+          }
+        }
+      } else {
+        // DOWN / DX / LORA_XA / LORA_HA: fp16 output, optional scale
+        const float sc = (MODE == DOWN || MODE == DX) ? 1.0f : a.lora_scale;
+        uint16_t* orow = static_cast<uint16_t*>(a.out) + grow * a.out_ld + un.nt * a.ntile;
+#pragma unroll 1
+        for (int c = 0; c < a.ntile; c += 32) {
+          float v[32];
+          tmem_ld32(tacc + c, v);
+          uint32_t pk[16];
+#pragma unroll
+          for (int i = 0; i < 16; ++i) pk[i] = pack_f16x2(sc * v[2 * i], sc * v[2 * i + 1]);
+          if (valid) {
+            const int ncol = min(32, a.n_valid - (un.nt * a.ntile + c));
+            uint4* dst = reinterpret_cast<uint4*>(orow + c);
+            if (ncol >= 32) {
 #pragma unroll
               for (int i = 0; i < 4; ++i) dst[i] = make_uint4(pk[4 * i], pk[4 * i + 1], pk[4 * i + 2], pk[4 * i + 3]);
-              if (a.aux) {  // keep the pre-activations for the backward
-                uint4* ga = reinterpret_cast<uint4*>(a.aux + grow * (2 * size_t(a.f_dim)) + un.nt * 64 + c);
-                uint4* ua = reinterpret_cast<uint4*>(a.aux + grow * (2 * size_t(a.f_dim)) + a.f_dim + un.nt * 64 + c);
-#pragma unroll
-                for (int i = 0; i < 4; ++i) {
-                  ga[i] = make_uint4(pack_f16x2(gv[8 * i], gv[8 * i + 1]), pack_f16x2(gv[8 * i + 2], gv[8 * i + 3]),
-                                     pack_f16x2(gv[8 * i + 4], gv[8 * i + 5]), pack_f16x2(gv[8 * i + 6], gv[8 * i + 7]));
-                  ua[i] = make_uint4(pack_f16x2(uv[8 * i], uv[8 * i + 1]), pack_f16x2(uv[8 * i + 2], uv[8 * i + 3]),
-                                     pack_f16x2(uv[8 * i + 4], uv[8 * i + 5]), pack_f16x2(uv[8 * i + 6], uv[8 * i + 7]));
-                }
-              }
-            }
-          }
-        } else if (MODE == DH) {
-          // dH -> dG = dH * U * silu'(G), dU = dH * silu(G); G, U from the recompute
-          const size_t ld2 = 2 * size_t(a.f_dim);
-          const uint16_t* grow_gu = a.aux + grow * ld2 + un.nt * 128;
-          uint16_t* drow = static_cast<uint16_t*>(a.out) + grow * ld2 + un.nt * 128;
-#pragma unroll 1
-          for (int c = 0; c < 128; c += 32) {
-            float v[32];
-            tmem_ld32(tacc + c, v);
-            if (valid) {
-#pragma unroll
-              for (int q = 0; q < 4; ++q) {
-                const uint4 gq = *reinterpret_cast<const uint4*>(grow_gu + c + 8 * q);
-                const uint4 uq = *reinterpret_cast<const uint4*>(grow_gu + a.f_dim + c + 8 * q);
-                const uint32_t gw[4] = {gq.x, gq.y, gq.z, gq.w};
-                const uint32_t uw[4] = {uq.x, uq.y, uq.z, uq.w};
-                uint32_t dg[4], du[4];
-#pragma unroll
-                for (int t = 0; t < 4; ++t) {
-                  float res_g[2], res_u[2];
-#pragma unroll
-                  for (int hh = 0; hh < 2; ++hh) {
-                    const float g = f16_to_f32(uint16_t(hh ? (gw[t] >> 16) : (gw[t] & 0xFFFFu)));
-                    const float u = f16_to_f32(uint16_t(hh ? (uw[t] >> 16) : (uw[t] & 0xFFFFu)));
-                    const float dh = v[8 * q + 2 * t + hh];
-                    const float sg = 1.0f / (1.0f + __expf(-g));
-                    res_g[hh] = dh * u * sg * (1.0f + g * (1.0f - sg));
-                    res_u[hh] = dh * g * sg;
-                  }
-                  dg[t] = pack_f16x2(res_g[0], res_g[1]);
-                  du[t] = pack_f16x2(res_u[0], res_u[1]);
-                }
-                *reinterpret_cast<uint4*>(drow + c + 8 * q) = make_uint4(dg[0], dg[1], dg[2], dg[3]);
-                *reinterpret_cast<uint4*>(drow + a.f_dim + c + 8 * q) = make_uint4(du[0], du[1], du[2], du[3]);
-              }
-            }
-          }
-        } else if (MODE == ROUTER) {
-          float* lrow = static_cast<float*>(a.out) + grow * a.out_ld;
-#pragma unroll 1
-          for (int c = 0; c < a.ntile; c += 32) {
-            float v[32];
-            tmem_ld32(tacc + c, v);
-            const int n0 = un.nt * a.ntile + c;
-            if (valid) {
-#pragma unroll
-              for (int i = 0; i < 32; ++i) {
-                const int n = n0 + i;
-                if (n < a.n_valid) lrow[n] = v[i] + (a.bias ? __ldg(a.bias + n) : 0.0f);
-              }
-            }
-          }
-        } else {
-          // DOWN / LORA_XA / LORA_HA: fp16 output, optional scale
-          const float sc = (MODE == DOWN || MODE == DX) ? 1.0f : a.lora_scale;
-          uint16_t* orow = static_cast<uint16_t*>(a.out) + grow * a.out_ld + un.nt * a.ntile;
-#pragma unroll 1
-          for (int c = 0; c < a.ntile; c += 32) {
-            float v[32];
-            tmem_ld32(tacc + c, v);
-            uint32_t pk[16];
-#pragma unroll
-            for (int i = 0; i < 16; ++i) pk[i] = pack_f16x2(sc * v[2 * i], sc * v[2 * i + 1]);
-            if (valid) {
-              const int ncol = min(32, a.n_valid - (un.nt * a.ntile + c));
-              if (ncol >= 32) {
-                uint4* dst = reinterpret_cast<uint4*>(orow + c);
-#pragma unroll
-                for (int i = 0; i < 4; ++i)
-                  dst[i] = make_uint4(pk[4 * i], pk[4 * i + 1], pk[4 * i + 2], pk[4 * i + 3]);
-              } else {
-                for (int i = 0; i < ncol / 8; ++i)
-                  reinterpret_cast<uint4*>(orow + c)[i] =
-                      make_uint4(pk[4 * i], pk[4 * i + 1], pk[4 * i + 2], pk[4 * i + 3]);
-              }
+            } else {
+              for (int i = 0; i < ncol / 8; ++i) dst[i] = make_uint4(pk[4 * i], pk[4 * i + 1], pk[4 * i + 2], pk[4 * i + 3]);
             }
           }
         }
@@ -346,34 +391,33 @@ __global__ void __launch_bounds__(kThreads, 1)
   } else if (warp == 4) {
     // ------------------------------------------------------------ MMA issuer
     if (lane == 0) {
-      Ring ring;
+      Ring ra, rb;
       int it = 0;
       bool ok = true;
-      const uint32_t idesc = (MODE == ROUTER) ? idesc_bf16(128, a.ntile) : idesc_f16(128, a.ntile);
+      const uint32_t idesc = kBf16 ? idesc_bf16(128, a.ntile) : idesc_f16(128, a.ntile);
       for (int u = blockIdx.x; u < nunits && ok; u += gridDim.x, ++it) {
-        const Unit un = decode_unit(a, u);
-        const int nsub = un.rows > 128 ? 2 : 1;
         const int ab = it & 1;
         const uint32_t aph = uint32_t(it >> 1) & 1u;
         if (!mbar_wait(&ctl->acc_empty[ab], aph ^ 1u, abort_flag, a.status)) { ok = false; break; }
         tc_fence_after();
+        const uint32_t dt = tmem_base + uint32_t(ab * 256);
         for (int kb = 0; kb < nkb; ++kb) {
-          if (!mbar_wait(&ctl->op_full[ring.stage], ring.phase, abort_flag, a.status)) { ok = false; break; }
+          if (!mbar_wait(&ctl->a_full[ra.stage], ra.phase, abort_flag, a.status) ||
+              !mbar_wait(&ctl->b_full[rb.stage], rb.phase, abort_flag, a.status)) {
+            ok = false;
+            break;
+          }
           fence_proxy_async_smem();
           tc_fence_after();
-          int ksteps = 4;
-          if (kb >= a.nkb_main) ksteps = (min(64, a.lora_k - (kb - a.nkb_main) * 64) + 15) / 16;
-          uint8_t* st = op_base + size_t(ring.stage) * kOpStageBytes;
-          const uint64_t bdesc = sdesc_k_sw128(smem_u32(st + kAStageBytes));
-          for (int sub = 0; sub < nsub; ++sub) {
-            const uint64_t adesc = sdesc_k_sw128(smem_u32(st + sub * 16384));
-            const uint32_t dt = tmem_base + uint32_t(ab * 256 + sub * 128);
-            for (int kk = 0; kk < ksteps; ++kk)
-              umma_bf16(dt, adesc + uint64_t(2 * kk), bdesc + uint64_t(2 * kk), idesc,
-                        (kb > 0 || kk > 0) ? 1u : 0u);
-          }
-          umma_commit(&ctl->op_empty[ring.stage]);
-          ring.next<kStages>();
+          const int ksteps = (kb < a.nkb_lora) ? (min(64, a.lora_k - kb * 64) + 15) / 16 : 4;
+          const uint64_t adesc = sdesc_k_sw128(smem_u32(a_base + size_t(ra.stage) * kAStageBytes));
+          const uint64_t bdesc = sdesc_k_sw128(smem_u32(b_base + size_t(rb.stage) * kBStageBytes));
+          for (int kk = 0; kk < ksteps; ++kk)
+            umma_bf16(dt, adesc + uint64_t(2 * kk), bdesc + uint64_t(2 * kk), idesc, (kb > 0 || kk > 0) ? 1u : 0u);
+          umma_commit(&ctl->a_empty[ra.stage]);
+          umma_commit(&ctl->b_empty[rb.stage]);
+          ra.next<kAStages>();
+          rb.next<kBStages>();
         }
         if (!ok) break;
         umma_commit(&ctl->acc_full[ab]);
@@ -387,42 +431,38 @@ __global__ void __launch_bounds__(kThreads, 1)
     // ------------------------------------------------------------ TMA producer (int4 + scales)
     if (kDequant && lane == 0) {
       Ring q;
-      const int ngrp = kTrans ? (a.g >= 128 ? 1 : 128 / a.g) : (a.g >= 64 ? 1 : 64 / a.g);
-      const int rows_box = (MODE == GATEUP) ? 64 : 128;
-      // codes 4096 B + scale boxes: forward {64|128 out cols x ngrp} twice or once (256*ngrp B),
-      // transposed {64 K x ngrp} once (128*ngrp B)
-      const uint32_t bytes = 4096u + uint32_t(ngrp * (kTrans ? 128 : 256));
+      // forward: per n-tile rows of W [rows][64 K]: codes rows*32 B, scales [ngrp][rows] bf16
+      // dgrad:   transposed tile [64 K][ntile N]: codes 64*ntile/2 B, scales [ngn][64] bf16
+      const int ngrp = kTrans ? (a.g >= a.ntile ? 1 : a.ntile / a.g) : (a.g >= 64 ? 1 : 64 / a.g);
+      const uint32_t bytes = uint32_t(a.ntile) * 32u + uint32_t(kTrans ? 128 * ngrp : a.ntile * ngrp * 2);
+      const int rows_box = (MODE == GATEUP) ? (a.ntile >> 1) : a.ntile;
       const int gpe = a.in_dim / a.g;  // scale rows per expert
       int issued = 0;
       uint32_t last_phase = 0;
       int last_stage = 0;
       for (int u = blockIdx.x; u < nunits; u += gridDim.x) {
         const Unit un = decode_unit(a, u);
-        const int nrow0 = un.e * a.out_dim + un.nt * rows_box;
         bool ok = true;
-        for (int kb = 0; kb < a.nkb_main; ++kb) {
-          if (!mbar_wait(&ctl->q_empty[q.stage], q.phase ^ 1u, abort_flag, a.status)) { ok = false; break; }
+        for (int km = 0; km < a.nkb_main; ++km) {
+          if (!mbar_wait<64>(&ctl->q_empty[q.stage], q.phase ^ 1u, abort_flag, a.status)) { ok = false; break; }
           uint8_t* qs = q_base + size_t(q.stage) * kQStageBytes;
           uint64_t* bar = &ctl->q_full[q.stage];
           mbar_arrive_expect_tx(bar, bytes);
           if (kTrans) {
-            // B = W^T: int4 rows = K (output index of W), bytes = N (input index)
-            const bool up = (MODE == DX) && kb >= a.half_kb;
-            const int kl = up ? kb - a.half_kb : kb;
-            tma_load_2d(smem_u32(qs), up ? &tq1 : &tq0, bar, un.nt * 64, un.e * a.out_dim + kl * 64);
-            tma_load_2d(smem_u32(qs + 4096), up ? &ts1 : &ts0, bar, kl * 64, un.e * gpe + (un.nt * 128) / a.g);
-            ++issued;
-            last_stage = q.stage;
-            last_phase = q.phase;
-            q.next<kQStages>();
-            continue;
-          }
-          const int srow = un.e * gpe + (kb * 64) / a.g;
-          tma_load_2d(smem_u32(qs), &tq0, bar, kb * 32, nrow0);
-          tma_load_2d(smem_u32(qs + 4096), &ts0, bar, un.nt * rows_box, srow);
-          if (MODE == GATEUP) {
-            tma_load_2d(smem_u32(qs + 2048), &tq1, bar, kb * 32, nrow0);
-            tma_load_2d(smem_u32(qs + 4096 + ngrp * 128), &ts1, bar, un.nt * rows_box, srow);
+            const bool up = (MODE == DX) && km >= a.half_kb;
+            const int kl = up ? km - a.half_kb : km;
+            tma_load_2d(smem_u32(qs), up ? &tq1 : &tq0, bar, un.nt * (a.ntile >> 1), un.e * a.out_dim + kl * 64);
+            tma_load_2d(smem_u32(qs + a.ntile * 32), up ? &ts1 : &ts0, bar, kl * 64,
+                        un.e * gpe + (un.nt * a.ntile) / a.g);
+          } else {
+            const int nrow0 = un.e * a.out_dim + un.nt * rows_box;
+            const int srow = un.e * gpe + (km * 64) / a.g;
+            tma_load_2d(smem_u32(qs), &tq0, bar, km * 32, nrow0);
+            tma_load_2d(smem_u32(qs + a.ntile * 32), &ts0, bar, un.nt * rows_box, srow);
+            if (MODE == GATEUP) {
+              tma_load_2d(smem_u32(qs + rows_box * 32), &tq1, bar, km * 32, nrow0);
+              tma_load_2d(smem_u32(qs + a.ntile * 32 + ngrp * rows_box * 2), &ts1, bar, un.nt * rows_box, srow);
+            }
           }
           ++issued;
           last_stage = q.stage;
@@ -435,220 +475,213 @@ __global__ void __launch_bounds__(kThreads, 1)
       if (issued > 0 && *abort_flag) mbar_wait(&ctl->q_full[last_stage], last_phase, abort_flag, a.status);
     }
   } else if (warp < 10) {
-    // ------------------------------------------------------------ A producer (cp.async)
-    const int tid = threadIdx.x - 6 * 32;  // 0..127
-    Ring ring;
-    CpAsyncLagArrive<2> lag;
+    // ------------------------------------------------------------ A producer
+    const int tid = threadIdx.x - 6 * 32;  // 0..127 = tile row
+    Ring ra, rb;
+    const uint32_t a_bytes = uint32_t(kAStageBytes);
+    uint32_t b_bytes = 0;
+    if (MODE == LORA_XA) b_bytes = uint32_t(2 * a.r * 128);
+    if (MODE == LORA_HA) b_bytes = uint32_t(a.r * 128);
+    if (MODE == ROUTER) b_bytes = uint32_t(a.ntile * 128);
+    int pend_stage = -1;
+    uint32_t pend_phase = 0;
     for (int u = blockIdx.x; u < nunits; u += gridDim.x) {
       const Unit un = decode_unit(a, u);
-      const uint16_t* src[2];
-      const uint16_t* lsrc[2];
-      bool valid[2];
-#pragma unroll
-      for (int sub = 0; sub < 2; ++sub) {
-        const int row = sub * 128 + tid;
-        valid[sub] = row < un.rows;
-        const int grow = un.base + (valid[sub] ? row : 0);
-        int srow = grow;
-        if (MODE == GATEUP || MODE == LORA_XA) srow = valid[sub] ? __ldg(a.perm_token + grow) : 0;
-        src[sub] = a.a_src + size_t(srow) * a.a_ld;
-        lsrc[sub] = a.a_lora ? a.a_lora + size_t(grow) * a.lora_ld : nullptr;
+      const bool valid = tid < un.rows;
+      const int grow = un.base + (valid ? tid : 0);
+      const uint16_t* src = nullptr;
+      if (!kATma) {
+        const int srow = valid ? __ldg(a.perm_token + grow) : 0;
+        src = a.a_src + size_t(srow) * a.a_ld;
       }
+      const uint16_t* lsrc = a.a_lora ? a.a_lora + size_t(grow) * a.lora_ld : nullptr;
       bool ok = true;
       for (int kb = 0; kb < nkb; ++kb) {
-        if (!mbar_wait(&ctl->op_empty[ring.stage], ring.phase ^ 1u, abort_flag, a.status)) { ok = false; break; }
-        const uint32_t st = smem_u32(op_base + size_t(ring.stage) * kOpStageBytes);
-        if (kb < a.nkb_main) {
-          const int kcol = (MODE == ROUTER ? (kb % a.kb_per_piece) : kb) * 64;
-#pragma unroll
-          for (int sub = 0; sub < 2; ++sub) {
-            if (!valid[sub]) continue;
-            const uint16_t* p = src[sub] + kcol;
-#pragma unroll
-            for (int c = 0; c < 8; ++c) cp_async16(st + sub * 16384 + sw128_offset(tid, c), p + c * 8, 16);
-          }
-        } else {
-          const int lb = kb - a.nkb_main;
-#pragma unroll
-          for (int sub = 0; sub < 2; ++sub) {
-            if (!valid[sub]) continue;
+        if (!mbar_wait<64>(&ctl->a_empty[ra.stage], ra.phase ^ 1u, abort_flag, a.status)) { ok = false; break; }
+        const uint32_t st_u = smem_u32(a_base + size_t(ra.stage) * kAStageBytes);
+        uint64_t* full = &ctl->a_full[ra.stage];
+        if (kb < a.nkb_lora) {
+          // rank-space A tile: s*xA / s*hA / dhA / dxa rows, zero-filled past lora_k
+          if (valid) {
 #pragma unroll
             for (int c = 0; c < 8; ++c) {
-              const int col = lb * 64 + c * 8;
+              const int col = kb * 64 + c * 8;
               const bool in = col < a.lora_k;
-              cp_async16(st + sub * 16384 + sw128_offset(tid, c), lsrc[sub] + (in ? col : 0), in ? 16u : 0u);
+              cp_async16(st_u + sw128_offset(tid, c), lsrc + (in ? col : 0), in ? 16u : 0u);
             }
           }
+          cp_async_arrive_noinc(full);
+        } else {
+          const int km = kb - a.nkb_lora;
+          const int kcol = (MODE == ROUTER) ? (km % a.kb_per_piece) * 64 : km * 64;
+          if (kBTma && tid == 0) {
+            // the B tile of a rank-space GEMM / the router comes by TMA as well
+            if (!mbar_wait<64>(&ctl->b_empty[rb.stage], rb.phase ^ 1u, abort_flag, a.status)) { ok = false; break; }
+            uint64_t* bfull = &ctl->b_full[rb.stage];
+            const uint32_t bst_u = smem_u32(b_base + size_t(rb.stage) * kBStageBytes);
+            mbar_arrive_expect_tx(bfull, b_bytes);
+            if (MODE == LORA_XA) {
+              tma_load_2d(bst_u, &tb0, bfull, kcol, un.e * a.r);
+              tma_load_2d(bst_u + a.r * 128, &tb1, bfull, kcol, un.e * a.r);
+            } else if (MODE == LORA_HA) {
+              tma_load_2d(bst_u, &tb0, bfull, kcol, un.e * a.r);
+            } else if (MODE == ROUTER) {
+              const int piece = km / a.kb_per_piece;
+              tma_load_2d(bst_u, &tb0, bfull, kcol, piece * a.n_valid + un.nt * a.ntile);
+            }
+          }
+          if (kATma) {
+            if (tid == 0) {
+              mbar_arrive_expect_tx(full, a_bytes);
+              tma_load_2d(st_u, &ta, full, kcol, un.base);
+              pend_stage = ra.stage;
+              pend_phase = ra.phase;
+            } else {
+              mbar_arrive(full);
+            }
+          } else {
+            if (valid) {
+              const uint16_t* p = src + km * 64;
+#pragma unroll
+              for (int c = 0; c < 8; ++c) cp_async16(st_u + sw128_offset(tid, c), p + c * 8, 16);
+            }
+            cp_async_arrive_noinc(full);
+          }
+          if (kBTma) rb.next<kBStages>();
         }
-        lag.stage_done(&ctl->op_full[ring.stage]);
-        ring.next<kStages>();
+        ra.next<kAStages>();
       }
       if (!ok) break;
     }
-    lag.flush();
+    cp_async_wait_all();
+    // on an abort, wait (bounded) for the last TMA fill issued by this thread
+    if (tid == 0 && *abort_flag && pend_stage >= 0)
+      mbar_wait(&ctl->a_full[pend_stage], pend_phase, abort_flag, a.status);
   } else {
     // ------------------------------------------------------------ B producer
     const int tid = threadIdx.x - 10 * 32;  // 0..255
-    const int row = tid >> 1;               // 0..127
-    const int half = tid & 1;
-    Ring ring, q;
-    CpAsyncLagArrive<2> lag;
+    const int tpr = a.ntile >= 256 ? 1 : 256 / a.ntile;   // threads per B row (forward tiles)
+    const int brow = tid / tpr;                              // B row (forward tiles)
+    const int part = tid % tpr;
+    const int nwords = tpr >= 8 ? 1 : 8 / tpr;               // int4 words (8 K values each) per thread
+    Ring rb, q;
     for (int u = blockIdx.x; u < nunits; u += gridDim.x) {
       const Unit un = decode_unit(a, u);
       bool ok = true;
       for (int kb = 0; kb < nkb; ++kb) {
-        if (!mbar_wait(&ctl->op_empty[ring.stage], ring.phase ^ 1u, abort_flag, a.status)) { ok = false; break; }
-        uint8_t* bst = op_base + size_t(ring.stage) * kOpStageBytes + kAStageBytes;
-        const uint32_t bst_u = smem_u32(bst);
-        if (kTrans && kb < a.nkb_main) {
-          // transposed dequant: thread = 4 K rows x 8 N columns of the int4 tile [64 K][128 N]
+        if (!mbar_wait(&ctl->b_empty[rb.stage], rb.phase ^ 1u, abort_flag, a.status)) { ok = false; break; }
+        uint8_t* bst = b_base + size_t(rb.stage) * kBStageBytes;
+        uint64_t* full = &ctl->b_full[rb.stage];
+        if (kb < a.nkb_lora) {
+          if (MODE == GATEUP || MODE == DOWN) {
+            // rank-space B^T rows as fp16, K' columns [kb*64, kb*64+64); gate rows hold
+            // Bg^T in [0, r), up rows hold Bu^T in [r, 2r) (block-diagonal)
+            if (brow < a.ntile) {
+              const int half = a.ntile >> 1;
+              for (int i = 0; i < nwords; ++i) {
+                const int c = part * nwords + i;
+                const int col = kb * 64 + c * 8;
+                uint4 v = make_uint4(0, 0, 0, 0);
+                if (MODE == GATEUP) {
+                  const bool gate = brow < half;
+                  const int n = un.nt * half + (gate ? brow : brow - half);
+                  const int cc = gate ? col : col - a.r;
+                  if (cc >= 0 && cc < a.r)
+                    v = __ldg(reinterpret_cast<const uint4*>((gate ? a.b0 : a.b1) + (size_t(un.e) * a.out_dim + n) * a.r +
+                                                             cc));
+                } else {
+                  const int n = un.nt * a.ntile + brow;
+                  if (col < a.r)
+                    v = __ldg(reinterpret_cast<const uint4*>(a.b0 + (size_t(un.e) * a.out_dim + n) * a.r + col));
+                }
+                *reinterpret_cast<uint4*>(bst + sw128_offset(brow, c)) = bf16x8_to_f16x8(v);
+              }
+            }
+          } else if (kTrans) {
+            // dgrad rank-space step: B[n][rr] = A^T[rr][n0 + n] (bf16, read transposed) as fp16
+            for (int nrow = tid; nrow < a.ntile; nrow += 256) {
+              const int n = un.nt * a.ntile + nrow;
+#pragma unroll 1
+              for (int c = 0; c < 8; ++c) {
+                uint32_t pk[4];
+#pragma unroll
+                for (int t = 0; t < 4; ++t) {
+                  float vv[2];
+#pragma unroll
+                  for (int hh = 0; hh < 2; ++hh) {
+                    const int rr = kb * 64 + c * 8 + 2 * t + hh;
+                    float val = 0.0f;
+                    if (rr < a.r) val = bf16_to_f32(__ldg(a.lb0 + (size_t(un.e) * a.r + rr) * a.lb_ld + n));
+                    else if (MODE == DX && rr < 2 * a.r)
+                      val = bf16_to_f32(__ldg(a.lb1 + (size_t(un.e) * a.r + (rr - a.r)) * a.lb_ld + n));
+                    vv[hh] = val;
+                  }
+                  pk[t] = pack_f16x2(vv[0], vv[1]);
+                }
+                *reinterpret_cast<uint4*>(bst + sw128_offset(nrow, c)) = make_uint4(pk[0], pk[1], pk[2], pk[3]);
+              }
+            }
+          }
+          fence_proxy_async_smem();
+          mbar_arrive(full);
+        } else if (kTrans) {
+          // transposed dequant: thread = 4 K rows x 8 N columns per 128-column half
           if (!mbar_wait(&ctl->q_full[q.stage], q.phase, abort_flag, a.status)) { ok = false; break; }
           const uint8_t* qs = q_base + size_t(q.stage) * kQStageBytes;
           const int kq = tid >> 4, no = tid & 15;
-          const int n0 = un.nt * 128;
-          const int gi = (n0 + no * 8) / a.g - n0 / a.g;
-          const uint16_t* sc = reinterpret_cast<const uint16_t*>(qs + 4096);
-          uint32_t hv[4][4];
+          const int n0 = un.nt * a.ntile;
+          const int rowb = a.ntile >> 1;                     // bytes per code row
+          const uint16_t* sc = reinterpret_cast<const uint16_t*>(qs + a.ntile * 32);
+          for (int hb = 0; hb < a.ntile; hb += 128) {
+            const int oct = (hb >> 3) + no;                  // N octet of this thread
+            const int gi = (n0 + oct * 8) / a.g - n0 / a.g;
+            uint32_t hv[4][4];
 #pragma unroll
-          for (int r = 0; r < 4; ++r) {
-            const int k = kq * 4 + r;
-            const uint32_t wv = *reinterpret_cast<const uint32_t*>(qs + k * 64 + no * 4);
-            const uint32_t sh = __half_as_ushort(__float2half_rn(bf16_to_f32(sc[gi * 64 + k])));
-            const uint4 d4 = dequant_word(wv, sh | (sh << 16));
-            hv[r][0] = d4.x; hv[r][1] = d4.y; hv[r][2] = d4.z; hv[r][3] = d4.w;
-          }
+            for (int r = 0; r < 4; ++r) {
+              const int k = kq * 4 + r;
+              const uint32_t wv = *reinterpret_cast<const uint32_t*>(qs + k * rowb + oct * 4);
+              const uint4 d4 = dequant_word(wv, scale_pair(sc[gi * 64 + k]));
+              hv[r][0] = d4.x; hv[r][1] = d4.y; hv[r][2] = d4.z; hv[r][3] = d4.w;
+            }
 #pragma unroll
-          for (int nn = 0; nn < 8; ++nn) {
-            const uint32_t sel = (nn & 1) ? 0x7632u : 0x5410u;
-            const uint32_t p01 = __byte_perm(hv[0][nn >> 1], hv[1][nn >> 1], sel);
-            const uint32_t p23 = __byte_perm(hv[2][nn >> 1], hv[3][nn >> 1], sel);
-            *reinterpret_cast<uint2*>(bst + sw128_offset(no * 8 + nn, kq >> 1) + (kq & 1) * 8) = make_uint2(p01, p23);
+            for (int nn = 0; nn < 8; ++nn) {
+              const uint32_t sel = (nn & 1) ? 0x7632u : 0x5410u;
+              const uint32_t p01 = __byte_perm(hv[0][nn >> 1], hv[1][nn >> 1], sel);
+              const uint32_t p23 = __byte_perm(hv[2][nn >> 1], hv[3][nn >> 1], sel);
+              *reinterpret_cast<uint2*>(bst + sw128_offset(oct * 8 + nn, kq >> 1) + (kq & 1) * 8) =
+                  make_uint2(p01, p23);
+            }
           }
+          // hand the code slot back only after its values were consumed, behind a
+          // proxy fence (its next TMA fill and the tensor-core reads are async-proxy)
           fence_proxy_async_smem();
           mbar_arrive(&ctl->q_empty[q.stage]);
           q.next<kQStages>();
-          mbar_arrive(&ctl->op_full[ring.stage]);
-        } else if (kTrans) {
-          // LoRA step of a dgrad: B[n][rr] = A^T[rr][n0 + n] (bf16, read transposed) as fp16
-          const int lb = kb - a.nkb_main;
-          const int n = un.nt * 128 + row;
-#pragma unroll 1
-          for (int i = 0; i < 4; ++i) {
-            const int c = half * 4 + i;
-            uint32_t pk[4];
-#pragma unroll
-            for (int t = 0; t < 4; ++t) {
-              float vv[2];
-#pragma unroll
-              for (int hh = 0; hh < 2; ++hh) {
-                const int rr = lb * 64 + c * 8 + 2 * t + hh;
-                float val = 0.0f;
-                if (rr < a.r) val = bf16_to_f32(__ldg(a.lb0 + (size_t(un.e) * a.r + rr) * a.lb_ld + n));
-                else if (MODE == DX && rr < 2 * a.r)
-                  val = bf16_to_f32(__ldg(a.lb1 + (size_t(un.e) * a.r + (rr - a.r)) * a.lb_ld + n));
-                vv[hh] = val;
-              }
-              pk[t] = pack_f16x2(vv[0], vv[1]);
-            }
-            *reinterpret_cast<uint4*>(bst + sw128_offset(row, c)) = make_uint4(pk[0], pk[1], pk[2], pk[3]);
-          }
-          fence_proxy_async_smem();
-          mbar_arrive(&ctl->op_full[ring.stage]);
-        } else if (kDequant && kb < a.nkb_main) {
+          mbar_arrive(full);
+        } else if (kDequant) {
           if (!mbar_wait(&ctl->q_full[q.stage], q.phase, abort_flag, a.status)) { ok = false; break; }
           const uint8_t* qs = q_base + size_t(q.stage) * kQStageBytes;
-          const uint4 words = *reinterpret_cast<const uint4*>(qs + row * 32 + half * 16);
+          const uint16_t* sc = reinterpret_cast<const uint16_t*>(qs + a.ntile * 32);
+          const int half = a.ntile >> 1;
+          // scale pairs of this row's group(s) in this K-block (two 32-wide groups when g == 32)
           const int ngrp = a.g >= 64 ? 1 : 64 / a.g;
-          const int gl = (a.g == 32) ? half : 0;
-          const uint16_t* sc = reinterpret_cast<const uint16_t*>(qs + 4096);
-          uint16_t sbits;
-          if (MODE == GATEUP) {
-            const int blk = row >> 6;
-            sbits = sc[blk * ngrp * 64 + gl * 64 + (row & 63)];
-          } else {
-            sbits = sc[gl * 128 + row];
-          }
-          const uint32_t sh = __half_as_ushort(__float2half_rn(bf16_to_f32(sbits)));
-          const uint32_t s2 = sh | (sh << 16);
-          const uint32_t wv[4] = {words.x, words.y, words.z, words.w};
-#pragma unroll
-          for (int i = 0; i < 4; ++i) {
-            const uint4 v = dequant_word(wv[i], s2);
-            *reinterpret_cast<uint4*>(bst + sw128_offset(row, half * 4 + i)) = v;
-          }
-          // The ring slot is handed back only after its values were consumed and
-          // a proxy fence ordered these generic-proxy reads (and the B-tile writes)
-          // before the async-proxy accesses that follow: the next TMA fill of the
-          // slot and the tensor-core reads of the B tile.
+          const int sidx = (MODE == GATEUP) ? (brow / half) * ngrp * half + (brow % half) : brow;
+          const int sstride = (MODE == GATEUP) ? half : a.ntile;
+          const uint32_t s_lo = scale_pair(sc[sidx]);
+          const uint32_t s_hi = (a.g == 32) ? scale_pair(sc[sidx + sstride]) : s_lo;
+          if (nwords == 8) dequant_row<8>(qs, bst, brow, part, s_lo, s_hi);
+          else dequant_row<4>(qs, bst, brow, part, s_lo, s_hi);
           fence_proxy_async_smem();
           mbar_arrive(&ctl->q_empty[q.stage]);
           q.next<kQStages>();
-          mbar_arrive(&ctl->op_full[ring.stage]);
-        } else if (kDequant) {
-          // LoRA B^T tile: K' columns [lb*64, lb*64 + 64) of the rank space
-          const int lb = kb - a.nkb_main;
-#pragma unroll
-          for (int i = 0; i < 4; ++i) {
-            const int c = half * 4 + i;
-            const int col = lb * 64 + c * 8;
-            uint4 v = make_uint4(0, 0, 0, 0);
-            if (MODE == GATEUP) {
-              const int n = un.nt * 64 + (row & 63);
-              if (row < 64) {
-                if (col < a.r) v = __ldg(reinterpret_cast<const uint4*>(a.b0 + (size_t(un.e) * a.out_dim + n) * a.r + col));
-              } else {
-                if (col >= a.r && col < 2 * a.r)
-                  v = __ldg(reinterpret_cast<const uint4*>(a.b1 + (size_t(un.e) * a.out_dim + n) * a.r + (col - a.r)));
-              }
-            } else {
-              const int n = un.nt * 128 + row;
-              if (col < a.r) v = __ldg(reinterpret_cast<const uint4*>(a.b0 + (size_t(un.e) * a.out_dim + n) * a.r + col));
-            }
-            *reinterpret_cast<uint4*>(bst + sw128_offset(row, c)) = bf16x8_to_f16x8(v);
-          }
-          fence_proxy_async_smem();
-          mbar_arrive(&ctl->op_full[ring.stage]);
-        } else if (MODE == LORA_XA || MODE == LORA_HA) {
-          // rank-space B^T = A^T rows (bf16 in memory) -> fp16 tile rows [0, ntile)
-          if (row < a.ntile) {
-            const uint16_t* p = nullptr;
-            if (MODE == LORA_XA) {
-              if (row < a.r) p = a.b0 + (size_t(un.e) * a.r + row) * a.a_ld;
-              else if (row < 2 * a.r) p = a.b1 + (size_t(un.e) * a.r + (row - a.r)) * a.a_ld;
-            } else if (row < a.r) {
-              p = a.b0 + (size_t(un.e) * a.r + row) * a.a_ld;
-            }
-#pragma unroll
-            for (int i = 0; i < 4; ++i) {
-              const int c = half * 4 + i;
-              uint4 v = make_uint4(0, 0, 0, 0);
-              if (p) v = bf16x8_to_f16x8(__ldg(reinterpret_cast<const uint4*>(p + kb * 64 + c * 8)));
-              *reinterpret_cast<uint4*>(bst + sw128_offset(row, c)) = v;
-            }
-          }
-          fence_proxy_async_smem();
-          mbar_arrive(&ctl->op_full[ring.stage]);
+          mbar_arrive(full);
         } else {
-          // ROUTER: bf16 parts of W_r, rows [0, ntile) x 64 K, via cp.async (zero-filled padding)
-          if (row < a.ntile) {
-            const uint16_t* p = nullptr;
-            const int n = un.nt * a.ntile + row;
-            const int piece = kb / a.kb_per_piece;
-            const int kcol = (kb % a.kb_per_piece) * 64;
-            if (n < a.n_valid) p = a.b0 + (size_t(piece) * a.n_valid + n) * a.a_ld;
-#pragma unroll
-            for (int i = 0; i < 4; ++i) {
-              const int c = half * 4 + i;
-              cp_async16(bst_u + sw128_offset(row, c), p ? p + kcol + c * 8 : a.a_src, p ? 16u : 0u);
-            }
-          }
-          lag.stage_done(&ctl->op_full[ring.stage]);
+          mbar_arrive(full);  // the B tile arrives by TMA (LORA_XA, LORA_HA, ROUTER)
         }
-        ring.next<kStages>();
+        rb.next<kBStages>();
       }
       if (!ok) break;
     }
-    lag.flush();
   }
 
   tc_fence_before();
@@ -663,7 +696,7 @@ __global__ void __launch_bounds__(kThreads, 1)
 // small helper kernels
 // ----------------------------------------------------------------------------
 
-// mb_prefix[e] = sum_{e' < e} ceil(count(e') / 256), one block.
+// mb_prefix[e] = sum_{e' < e} ceil(count(e') / kMBlock), one block.
 __global__ void schedule_kernel(const int32_t* __restrict__ offsets, int E, int32_t* __restrict__ mb_prefix) {
   __shared__ int32_t warp_sums[32];
   const int nt = blockDim.x;
@@ -699,10 +732,10 @@ __global__ void schedule_kernel(const int32_t* __restrict__ offsets, int E, int3
   if (threadIdx.x == nt - 1) mb_prefix[E] = run;
 }
 
-// Token activations bf16 -> fp16 (the operand type of the expert contractions);
-// values beyond the fp16 range raise TQP_STATUS_NONFINITE.
-__global__ void x_to_f16_kernel(const uint16_t* __restrict__ x, uint16_t* __restrict__ x16, size_t n8,
-                                int32_t* status) {
+// bf16 -> fp16, 8 values per thread; values beyond the fp16 range raise
+// TQP_STATUS_NONFINITE (status may be null).
+__global__ void to_f16_kernel(const uint16_t* __restrict__ x, uint16_t* __restrict__ x16, size_t n8,
+                              int32_t* status) {
   const size_t i = size_t(blockIdx.x) * blockDim.x + threadIdx.x;
   if (i >= n8) return;
   const uint4 v = __ldg(reinterpret_cast<const uint4*>(x) + i);
@@ -754,7 +787,7 @@ static PFN_cuTensorMapEncodeTiled_v12000 encode_fn() {
 }
 
 static bool make_map(CUtensorMap* m, CUtensorMapDataType dt, const void* ptr, uint64_t inner, uint64_t outer,
-                     uint64_t row_bytes, uint32_t box_inner, uint32_t box_outer) {
+                     uint64_t row_bytes, uint32_t box_inner, uint32_t box_outer, bool sw128 = false) {
   auto fn = encode_fn();
   if (!fn) return false;
   cuuint64_t dims[2] = {inner, outer};
@@ -762,8 +795,13 @@ static bool make_map(CUtensorMap* m, CUtensorMapDataType dt, const void* ptr, ui
   cuuint32_t box[2] = {box_inner, box_outer};
   cuuint32_t estr[2] = {1, 1};
   return fn(m, dt, 2, const_cast<void*>(ptr), dims, strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
-            CU_TENSOR_MAP_SWIZZLE_NONE, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+            sw128 ? CU_TENSOR_MAP_SWIZZLE_128B : CU_TENSOR_MAP_SWIZZLE_NONE, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
             CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+// 128B-swizzled K-major tile map of a row-major 16-bit matrix [rows][cols]: box {64, box_rows}.
+static bool make_tile_map(CUtensorMap* m, const void* ptr, uint64_t rows, uint64_t cols, uint32_t box_rows) {
+  return make_map(m, CU_TENSOR_MAP_DATA_TYPE_UINT16, ptr, cols, rows, cols * 2, 64, box_rows, true);
 }
 
 int num_sms() {
@@ -773,8 +811,14 @@ int num_sms() {
   return n;
 }
 
+struct Maps {
+  CUtensorMap m[7];
+  Maps() { memset(m, 0, sizeof(m)); }
+};
+enum { TQ0 = 0, TQ1 = 1, TS0 = 2, TS1 = 3, TA = 4, TB0 = 5, TB1 = 6 };
+
 template <int MODE>
-static int run_gemm(const GemmArgs& a, const CUtensorMap* maps, int units_upper, cudaStream_t s) {
+static int run_gemm(const GemmArgs& a, const Maps& mp, int units_upper, cudaStream_t s) {
   static bool attr_set = false;
   if (!attr_set) {
     if (cudaFuncSetAttribute(grouped_gemm_kernel<MODE>, cudaFuncAttributeMaxDynamicSharedMemorySize,
@@ -783,7 +827,8 @@ static int run_gemm(const GemmArgs& a, const CUtensorMap* maps, int units_upper,
     attr_set = true;
   }
   const int grid = units_upper < num_sms() ? (units_upper > 0 ? units_upper : 1) : num_sms();
-  grouped_gemm_kernel<MODE><<<grid, kThreads, kSmemBytes, s>>>(a, maps[0], maps[1], maps[2], maps[3]);
+  grouped_gemm_kernel<MODE><<<grid, kThreads, kSmemBytes, s>>>(a, mp.m[0], mp.m[1], mp.m[2], mp.m[3], mp.m[4],
+                                                                mp.m[5], mp.m[6]);
   return cudaGetLastError() == cudaSuccess ? TQP_OK : TQP_ERR_CUDA;
 }
 
@@ -803,26 +848,22 @@ int launch_router_gemm(const uint16_t* x, int T, const tqp_moe_weights* w, float
   a.E = 1;
   a.kb_per_piece = w->d / 64;
   a.nkb_main = 3 * a.kb_per_piece;
-  a.nkb_lora = 0;
-  a.lora_k = 0;
-  a.ntile = 128;
-  a.n_tiles = (w->E + 127) / 128;
+  a.ntile = w->E <= 128 ? ((w->E + 15) / 16) * 16 : 256;
+  a.n_tiles = (w->E + a.ntile - 1) / a.ntile;
   a.g = 64;
   a.offsets = ctl;
   a.mb_prefix = ctl + 2;
-  a.perm_token = nullptr;
-  a.a_src = x;
-  a.a_ld = w->d;
-  a.b0 = parts;
   a.out = logits;
   a.out_ld = w->E;
   a.n_valid = w->E;
   a.bias = w->router_bias;
   a.status = status;
-  CUtensorMap maps[4];
-  memset(maps, 0, sizeof(maps));
+  Maps mp;
+  if (!make_tile_map(&mp.m[TA], x, uint64_t(T), uint64_t(w->d), 128) ||
+      !make_tile_map(&mp.m[TB0], parts, 3 * uint64_t(w->E), uint64_t(w->d), uint32_t(a.ntile)))
+    return TQP_ERR_CUDA;
   const int units = ((T + kMBlock - 1) / kMBlock) * a.n_tiles;
-  return run_gemm<ROUTER>(a, maps, units, s);
+  return run_gemm<ROUTER>(a, mp, units, s);
 }
 
 size_t ffn_ws_bytes(int T, const tqp_moe_weights* w) {
@@ -832,6 +873,7 @@ size_t ffn_ws_bytes(int T, const tqp_moe_weights* w) {
   if (w->rank > 0) {
     b += align_up(A * 2 * w->rank * 2, 256);                    // xa [A][2r]
     b += align_up(A * w->rank * 2, 256);                        // ha [A][r]
+    b += align_up(size_t(w->E) * w->rank * w->ffn * 2, 256);   // Ad^T in fp16
   }
   return b + 256;
 }
@@ -848,8 +890,17 @@ FfnBufs ffn_carve(void* ws, int T, const tqp_moe_weights* w) {
     b.xa = reinterpret_cast<uint16_t*>(p);
     p += align_up(A * 2 * w->rank * 2, 256);
     b.ha = reinterpret_cast<uint16_t*>(p);
+    p += align_up(A * w->rank * 2, 256);
+    b.adT16 = reinterpret_cast<uint16_t*>(p);
   }
   return b;
+}
+
+static int to_f16(const uint16_t* src, uint16_t* dst, size_t n, int32_t* status, cudaStream_t s) {
+  const size_t n8 = n / 8;
+  if (n8 == 0) return TQP_OK;
+  to_f16_kernel<<<unsigned((n8 + 255) / 256), 256, 0, s>>>(src, dst, n8, status);
+  return cudaGetLastError() == cudaSuccess ? TQP_OK : TQP_ERR_CUDA;
 }
 
 int launch_grouped_ffn(const uint16_t* x, int T, const int32_t* offsets, const int32_t* perm_token,
@@ -858,19 +909,14 @@ int launch_grouped_ffn(const uint16_t* x, int T, const int32_t* offsets, const i
   if (T == 0) return TQP_OK;
   const size_t A = size_t(T) * w->top_k;
   const FfnBufs fb = ffn_carve(ws, T, w);
-  int32_t* mb_prefix = fb.mb_prefix;
-  uint16_t* x16 = fb.x16;
-  uint16_t* xa = fb.xa;
-  uint16_t* ha = fb.ha;
-  schedule_kernel<<<1, 1024, 0, s>>>(offsets, w->E, mb_prefix);
-  {
-    const size_t n8 = size_t(T) * w->d / 8;
-    x_to_f16_kernel<<<unsigned((n8 + 255) / 256), 256, 0, s>>>(x, x16, n8, status);
-  }
+  const int d = w->d, f = w->ffn, r = w->rank;
+  schedule_kernel<<<1, 1024, 0, s>>>(offsets, w->E, fb.mb_prefix);
   if (cudaGetLastError() != cudaSuccess) return TQP_ERR_CUDA;
+  int rc;
+  if ((rc = to_f16(x, fb.x16, size_t(T) * d, status, s)) != TQP_OK) return rc;
+  if (r > 0 && (rc = to_f16(w->lora_a[2], fb.adT16, size_t(w->E) * r * f, nullptr, s)) != TQP_OK) return rc;
   // an upper bound on the number of work units (grid sizing only)
   const int mb_upper = int((A + kMBlock - 1) / kMBlock) + w->E;
-  const int d = w->d, f = w->ffn, r = w->rank;
 
   GemmArgs base{};
   base.E = w->E;
@@ -878,103 +924,99 @@ int launch_grouped_ffn(const uint16_t* x, int T, const int32_t* offsets, const i
   base.r = r;
   base.lora_scale = w->lora_scale;
   base.offsets = offsets;
-  base.mb_prefix = mb_prefix;
+  base.mb_prefix = fb.mb_prefix;
   base.perm_token = perm_token;
   base.status = status;
   base.kb_per_piece = 1;
-  int rc;
-  CUtensorMap maps[4];
-  memset(maps, 0, sizeof(maps));
 
-  if (r > 0) {  // xa = s * X [Ag | Au]
+  if (r > 0) {  // xa = s * X [Ag | Au]   (bf16 operands)
     GemmArgs a = base;
     a.nkb_main = d / 64;
-    a.ntile = 2 * r;
+    a.ntile = 2 * r < 16 ? 16 : 2 * r;
     a.n_tiles = 1;
-    a.a_src = x16;
+    a.a_src = x;
     a.a_ld = d;
-    a.b0 = w->lora_a[0];
-    a.b1 = w->lora_a[1];
-    a.out = xa;
+    a.out = fb.xa;
     a.out_ld = 2 * r;
     a.n_valid = 2 * r;
-    if ((rc = run_gemm<LORA_XA>(a, maps, mb_upper, s)) != TQP_OK) return rc;
+    Maps mp;
+    if (!make_tile_map(&mp.m[TB0], w->lora_a[0], uint64_t(w->E) * r, uint64_t(d), uint32_t(r)) ||
+        !make_tile_map(&mp.m[TB1], w->lora_a[1], uint64_t(w->E) * r, uint64_t(d), uint32_t(r)))
+      return TQP_ERR_CUDA;
+    if ((rc = run_gemm<LORA_XA>(a, mp, mb_upper, s)) != TQP_OK) return rc;
   }
   {  // H = silu(G) * U
     GemmArgs a = base;
     a.nkb_main = d / 64;
     a.nkb_lora = r > 0 ? (2 * r + 63) / 64 : 0;
     a.lora_k = 2 * r;
-    a.ntile = 128;
-    a.n_tiles = f / 64;
+    a.ntile = (f % 128 == 0) ? 256 : 128;
+    a.n_tiles = f / (a.ntile / 2);
     a.in_dim = d;
     a.out_dim = f;
-    a.a_src = x16;
+    a.a_src = fb.x16;
     a.a_ld = d;
-    a.a_lora = xa;
+    a.a_lora = fb.xa;
     a.lora_ld = 2 * r;
     a.b0 = w->lora_b[0];
     a.b1 = w->lora_b[1];
-    a.wq0 = w->wq[0];
-    a.wq1 = w->wq[1];
-    a.ws0 = w->wscale[0];
-    a.ws1 = w->wscale[1];
     a.out = h;
     a.out_ld = f;
     a.n_valid = f;
     a.aux = aux_gu;
     a.f_dim = f;
     const int ngrp = w->group >= 64 ? 1 : 64 / w->group;
-    bool ok = make_map(&maps[0], CU_TENSOR_MAP_DATA_TYPE_UINT8, w->wq[0], d / 2, uint64_t(w->E) * f, d / 2, 32, 64) &&
-              make_map(&maps[1], CU_TENSOR_MAP_DATA_TYPE_UINT8, w->wq[1], d / 2, uint64_t(w->E) * f, d / 2, 32, 64) &&
-              make_map(&maps[2], CU_TENSOR_MAP_DATA_TYPE_UINT16, w->wscale[0], f, uint64_t(w->E) * (d / w->group),
-                       uint64_t(f) * 2, 64, ngrp) &&
-              make_map(&maps[3], CU_TENSOR_MAP_DATA_TYPE_UINT16, w->wscale[1], f, uint64_t(w->E) * (d / w->group),
-                       uint64_t(f) * 2, 64, ngrp);
+    const uint32_t rows_box = uint32_t(a.ntile / 2);
+    Maps mp;
+    bool ok = make_map(&mp.m[TQ0], CU_TENSOR_MAP_DATA_TYPE_UINT8, w->wq[0], d / 2, uint64_t(w->E) * f, d / 2, 32,
+                       rows_box) &&
+              make_map(&mp.m[TQ1], CU_TENSOR_MAP_DATA_TYPE_UINT8, w->wq[1], d / 2, uint64_t(w->E) * f, d / 2, 32,
+                       rows_box) &&
+              make_map(&mp.m[TS0], CU_TENSOR_MAP_DATA_TYPE_UINT16, w->wscale[0], f, uint64_t(w->E) * (d / w->group),
+                       uint64_t(f) * 2, rows_box, ngrp) &&
+              make_map(&mp.m[TS1], CU_TENSOR_MAP_DATA_TYPE_UINT16, w->wscale[1], f, uint64_t(w->E) * (d / w->group),
+                       uint64_t(f) * 2, rows_box, ngrp);
     if (!ok) return TQP_ERR_CUDA;
-    if ((rc = run_gemm<GATEUP>(a, maps, mb_upper * a.n_tiles, s)) != TQP_OK) return rc;
+    if ((rc = run_gemm<GATEUP>(a, mp, mb_upper * a.n_tiles, s)) != TQP_OK) return rc;
   }
   if (r > 0) {  // ha = s * H Ad
     GemmArgs a = base;
-    memset(maps, 0, sizeof(maps));
     a.nkb_main = f / 64;
     a.ntile = r < 16 ? 16 : r;
     a.n_tiles = 1;
-    a.a_src = h;
-    a.a_ld = f;
-    a.b0 = w->lora_a[2];
-    a.out = ha;
+    a.out = fb.ha;
     a.out_ld = r;
     a.n_valid = r;
-    if ((rc = run_gemm<LORA_HA>(a, maps, mb_upper, s)) != TQP_OK) return rc;
+    Maps mp;
+    if (!make_tile_map(&mp.m[TA], h, uint64_t(A), uint64_t(f), 128) ||
+        !make_tile_map(&mp.m[TB0], fb.adT16, uint64_t(w->E) * r, uint64_t(f), uint32_t(r)))
+      return TQP_ERR_CUDA;
+    if ((rc = run_gemm<LORA_HA>(a, mp, mb_upper, s)) != TQP_OK) return rc;
   }
   {  // O = H Wd^T + (s H Ad) Bd
     GemmArgs a = base;
     a.nkb_main = f / 64;
     a.nkb_lora = r > 0 ? (r + 63) / 64 : 0;
     a.lora_k = r;
-    a.ntile = 128;
-    a.n_tiles = d / 128;
+    a.ntile = (d % 256 == 0) ? 256 : 128;
+    a.n_tiles = d / a.ntile;
     a.in_dim = f;
     a.out_dim = d;
-    a.a_src = h;
-    a.a_ld = f;
-    a.a_lora = ha;
+    a.a_lora = fb.ha;
     a.lora_ld = r;
     a.b0 = w->lora_b[2];
-    a.wq0 = w->wq[2];
-    a.ws0 = w->wscale[2];
     a.out = out_perm;
     a.out_ld = d;
     a.n_valid = d;
     const int ngrp = w->group >= 64 ? 1 : 64 / w->group;
-    bool ok = make_map(&maps[0], CU_TENSOR_MAP_DATA_TYPE_UINT8, w->wq[2], f / 2, uint64_t(w->E) * d, f / 2, 32, 128) &&
-              make_map(&maps[2], CU_TENSOR_MAP_DATA_TYPE_UINT16, w->wscale[2], d, uint64_t(w->E) * (f / w->group),
-                       uint64_t(d) * 2, 128, ngrp);
-    maps[1] = maps[0];
-    maps[3] = maps[2];
+    Maps mp;
+    bool ok = make_tile_map(&mp.m[TA], h, uint64_t(A), uint64_t(f), 128) &&
+              make_map(&mp.m[TQ0], CU_TENSOR_MAP_DATA_TYPE_UINT8, w->wq[2], f / 2, uint64_t(w->E) * d, f / 2, 32,
+                       uint32_t(a.ntile)) &&
+              make_map(&mp.m[TS0], CU_TENSOR_MAP_DATA_TYPE_UINT16, w->wscale[2], d, uint64_t(w->E) * (f / w->group),
+                       uint64_t(d) * 2, uint32_t(a.ntile), ngrp);
     if (!ok) return TQP_ERR_CUDA;
-    if ((rc = run_gemm<DOWN>(a, maps, mb_upper * a.n_tiles, s)) != TQP_OK) return rc;
+    if ((rc = run_gemm<DOWN>(a, mp, mb_upper * a.n_tiles, s)) != TQP_OK) return rc;
   }
   return TQP_OK;
 }
@@ -998,59 +1040,60 @@ int launch_dgrad(int which, const uint16_t* a_src, const uint16_t* a_lora, const
   a.mb_prefix = mb_prefix;
   a.kb_per_piece = 1;
   a.status = status;
-  a.ntile = 128;
   a.f_dim = f;
-  a.a_src = a_src;
   a.a_lora = a_lora;
   a.out = out;
-  CUtensorMap maps[4];
-  memset(maps, 0, sizeof(maps));
-  const int ngn = w->group >= 128 ? 1 : 128 / w->group;
+  Maps mp;
   if (which == 0) {  // DH: K = d (rows of Wd), N = f
+    a.ntile = (f % 256 == 0) ? 256 : 128;
+    const int ngn = w->group >= a.ntile ? 1 : a.ntile / w->group;
     a.nkb_main = d / 64;
     a.nkb_lora = r > 0 ? (r + 63) / 64 : 0;
     a.lora_k = r;
     a.lora_ld = r;
-    a.n_tiles = f / 128;
+    a.n_tiles = f / a.ntile;
     a.in_dim = f;
     a.out_dim = d;
-    a.a_ld = d;
     a.lb0 = w->lora_a[2];
     a.lb_ld = f;
     a.aux = const_cast<uint16_t*>(aux_gu);
     a.out_ld = 2 * f;
     a.n_valid = f;
-    bool ok = make_map(&maps[0], CU_TENSOR_MAP_DATA_TYPE_UINT8, w->wq[2], f / 2, uint64_t(w->E) * d, f / 2, 64, 64) &&
-              make_map(&maps[2], CU_TENSOR_MAP_DATA_TYPE_UINT16, w->wscale[2], d, uint64_t(w->E) * (f / w->group),
+    bool ok = make_tile_map(&mp.m[TA], a_src, uint64_t(A), uint64_t(d), 128) &&
+              make_map(&mp.m[TQ0], CU_TENSOR_MAP_DATA_TYPE_UINT8, w->wq[2], f / 2, uint64_t(w->E) * d, f / 2,
+                       uint32_t(a.ntile / 2), 64) &&
+              make_map(&mp.m[TS0], CU_TENSOR_MAP_DATA_TYPE_UINT16, w->wscale[2], d, uint64_t(w->E) * (f / w->group),
                        uint64_t(d) * 2, 64, ngn);
-    maps[1] = maps[0];
-    maps[3] = maps[2];
     if (!ok) return TQP_ERR_CUDA;
-    return run_gemm<DH>(a, maps, mb_upper * a.n_tiles, s);
+    return run_gemm<DH>(a, mp, mb_upper * a.n_tiles, s);
   }
   // DX: K = 2f (gate rows then up rows of W), N = d
+  a.ntile = (d % 256 == 0) ? 256 : 128;
+  const int ngn = w->group >= a.ntile ? 1 : a.ntile / w->group;
   a.nkb_main = 2 * f / 64;
   a.half_kb = f / 64;
   a.nkb_lora = r > 0 ? (2 * r + 63) / 64 : 0;
   a.lora_k = 2 * r;
   a.lora_ld = 2 * r;
-  a.n_tiles = d / 128;
+  a.n_tiles = d / a.ntile;
   a.in_dim = d;
   a.out_dim = f;
-  a.a_ld = 2 * f;
   a.lb0 = w->lora_a[0];
   a.lb1 = w->lora_a[1];
   a.lb_ld = d;
   a.out_ld = d;
   a.n_valid = d;
-  bool ok = make_map(&maps[0], CU_TENSOR_MAP_DATA_TYPE_UINT8, w->wq[0], d / 2, uint64_t(w->E) * f, d / 2, 64, 64) &&
-            make_map(&maps[1], CU_TENSOR_MAP_DATA_TYPE_UINT8, w->wq[1], d / 2, uint64_t(w->E) * f, d / 2, 64, 64) &&
-            make_map(&maps[2], CU_TENSOR_MAP_DATA_TYPE_UINT16, w->wscale[0], f, uint64_t(w->E) * (d / w->group),
+  bool ok = make_tile_map(&mp.m[TA], a_src, uint64_t(A), uint64_t(2 * f), 128) &&
+            make_map(&mp.m[TQ0], CU_TENSOR_MAP_DATA_TYPE_UINT8, w->wq[0], d / 2, uint64_t(w->E) * f, d / 2,
+                     uint32_t(a.ntile / 2), 64) &&
+            make_map(&mp.m[TQ1], CU_TENSOR_MAP_DATA_TYPE_UINT8, w->wq[1], d / 2, uint64_t(w->E) * f, d / 2,
+                     uint32_t(a.ntile / 2), 64) &&
+            make_map(&mp.m[TS0], CU_TENSOR_MAP_DATA_TYPE_UINT16, w->wscale[0], f, uint64_t(w->E) * (d / w->group),
                      uint64_t(f) * 2, 64, ngn) &&
-            make_map(&maps[3], CU_TENSOR_MAP_DATA_TYPE_UINT16, w->wscale[1], f, uint64_t(w->E) * (d / w->group),
+            make_map(&mp.m[TS1], CU_TENSOR_MAP_DATA_TYPE_UINT16, w->wscale[1], f, uint64_t(w->E) * (d / w->group),
                      uint64_t(f) * 2, 64, ngn);
   if (!ok) return TQP_ERR_CUDA;
-  return run_gemm<DX>(a, maps, mb_upper * a.n_tiles, s);
+  return run_gemm<DX>(a, mp, mb_upper * a.n_tiles, s);
 }
 
 }  // namespace tqp

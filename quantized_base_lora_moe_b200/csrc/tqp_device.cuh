@@ -72,7 +72,10 @@ __device__ __forceinline__ bool mbar_try_wait(uint32_t addr, uint32_t parity) {
 
 // Bounded wait for the phase with the given parity. Returns false (and sets the
 // CTA abort flag and the timeout status bit) when the limit expires or another
-// role has already aborted.
+// role has already aborted. kSleep > 0 backs off with nanosleep between polls,
+// for waiters off the critical path (they then leave issue slots to the
+// dequantising warps).
+template <int kSleep = 0>
 __device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, volatile int* abort_flag,
                                           int32_t* status) {
   const uint32_t addr = smem_u32(bar);
@@ -81,6 +84,7 @@ __device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, volati
   uint32_t spins = 0;
   while (true) {
     if (mbar_try_wait(addr, parity)) return true;
+    if (kSleep > 0) __nanosleep(kSleep);
     if (((++spins) & 63u) == 0u) {
       if (*abort_flag) return false;
       if (globaltimer() - t0 > kWaitLimitNs) {

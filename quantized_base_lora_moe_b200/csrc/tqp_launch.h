@@ -27,12 +27,14 @@ int launch_router_gemm(const uint16_t* x, int T, const tqp_moe_weights* w, float
                        int32_t* status, cudaStream_t s);
 size_t ffn_ws_bytes(int T, const tqp_moe_weights* w);
 // Buffers inside the grouped-FFN workspace (valid after launch_grouped_ffn):
-// per-expert m-block prefix, x in fp16, s*X[Ag|Au] [A][2r] and s*H*Ad [A][r] (fp16).
+// per-expert m-block prefix, x in fp16, s*X[Ag|Au] [A][2r] and s*H*Ad [A][r] (fp16),
+// and Ad^T in fp16.
 struct FfnBufs {
   int32_t* mb_prefix;
   uint16_t* x16;
   uint16_t* xa;
   uint16_t* ha;
+  uint16_t* adT16;   // Ad^T converted to fp16 [E][r][f]
 };
 FfnBufs ffn_carve(void* ws, int T, const tqp_moe_weights* w);
 int launch_grouped_ffn(const uint16_t* x, int T, const int32_t* offsets, const int32_t* perm_token,

@@ -75,7 +75,11 @@ REV_F = FULL
 REV_G = dataclasses.replace(FULL, name="full_g", seed=1)
 REV_SEEDS = {"x1": 2, "x2": 3, "dy": 4}
 
-CONFIGS = {c.name: c for c in (TINY, MID, FULL, SKEWED)}
+# profiling case: the full layer's shapes with 64 experts (151 MB of int4 codes,
+# larger than L2, a few hundred MB on the device in total)
+PROF = LayerConfig("prof", T=4096, d=2048, E=64, k=8, f=768, g=64, r=32)
+
+CONFIGS = {c.name: c for c in (TINY, MID, FULL, SKEWED, PROF)}
 
 # stream tags
 _TAG = {"router": 1, "w0": 2, "w1": 3, "w2": 4, "a0": 5, "a1": 6, "a2": 7,
