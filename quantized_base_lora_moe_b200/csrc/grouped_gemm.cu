@@ -407,7 +407,9 @@ __global__ void __launch_bounds__(kThreads, 1)
             ok = false;
             break;
           }
-          fence_proxy_async_smem();
+          // no proxy fence here: TMA fills are async-proxy writes, the dequantising
+          // threads fence their own generic stores before arriving, and cp.async
+          // completion is tracked by the barrier itself
           tc_fence_after();
           const int ksteps = (kb < a.nkb_lora) ? (min(64, a.lora_k - kb * 64) + 15) / 16 : 4;
           const uint64_t adesc = sdesc_k_sw128(smem_u32(a_base + size_t(ra.stage) * kAStageBytes));
@@ -569,7 +571,9 @@ __global__ void __launch_bounds__(kThreads, 1)
       const Unit un = decode_unit(a, u);
       bool ok = true;
       for (int kb = 0; kb < nkb; ++kb) {
-        if (!mbar_wait(&ctl->b_empty[rb.stage], rb.phase ^ 1u, abort_flag, a.status)) { ok = false; break; }
+        const bool waited = kBTma ? mbar_wait<256>(&ctl->b_empty[rb.stage], rb.phase ^ 1u, abort_flag, a.status)
+                                  : mbar_wait(&ctl->b_empty[rb.stage], rb.phase ^ 1u, abort_flag, a.status);
+        if (!waited) { ok = false; break; }
         uint8_t* bst = b_base + size_t(rb.stage) * kBStageBytes;
         uint64_t* full = &ctl->b_full[rb.stage];
         if (kb < a.nkb_lora) {
