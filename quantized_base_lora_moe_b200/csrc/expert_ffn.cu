@@ -1,0 +1,513 @@
+// Forward expert projections of the TQP MoE layer with the dequantised base
+// weights held in tensor memory (sm_100a, tcgen05):
+//   GATEUP : [G|U] = X_e [Wg|Wu]^T + (s X [Ag|Au]) [Bg|Bu],  H = silu(G) * U
+//   DOWN   : O = H_e Wd^T + (s H Ad) Bd
+// ("Train low-rank adapters per expert" over "Quantize base expert weights",
+// Pattern 3; SwiGLU experts, TQP Quantization).
+//
+// The contraction runs transposed: D[feature][token] = W[feature][:] . X[token][:],
+// with W (M = 128 output features of one tile) as the tcgen05.mma A operand in
+// TMEM and the token rows (N = the unit's routed rows rounded up to 16) as the B
+// operand in 128B-swizzled shared memory. The int4 codes are dequantised by
+// registers -> tcgen05.st straight into TMEM, so the dequantised tile never
+// touches shared memory, and a ragged expert block costs at most 15 idle
+// columns instead of a padded 128-row tile.
+//
+// Work unit = (expert e, 128-feature tile, block of up to 128 routed rows);
+// units are ordered (expert, tile, block) over a persistent grid. Per CTA
+// (1 per SM, 576 threads):
+//   warps 0-3   epilogue (TMEM lanes 32w..32w+31 = features of the tile)
+//   warp  4     TMEM allocation + one thread issuing tcgen05.mma
+//   warp  5     TMA producer of the int4 code / bf16 scale ring
+//   warps 6-9   token producer: cp.async row gathers (rows picked by perm_token)
+//               or TMA tiles of contiguous rows, and the rank-space rows
+//   warps 10-17 weight producer: int4 -> fp16 into TMEM, LoRA B rows
+// TMEM (512 columns): accumulators in [0, 256), weight stages in [256, 512).
+//   GATEUP: one accumulator (gate cols [0,128), up [128,256)), 4 weight stages
+//           of 64 columns (gate 32 | up 32). The epilogue drains G and U as
+//           fp16 into [token][feature] shared-memory tiles, hands TMEM back, and
+//           finishes SwiGLU + 16-byte row stores while the next unit runs.
+//   DOWN:   two accumulators of 128 columns, 8 weight stages of 32 columns;
+//           32-token chunks go out through a double-buffered [token][feature]
+//           tile, so that every global store is a 16-byte piece of a row.
+// Every wait is bounded (tqp_device.cuh); no TMA multicast is used.
+#include <cstdint>
+#include <cuda.h>
+#include <cuda_fp16.h>
+#include <cuda_runtime.h>
+
+#include "gemm_common.cuh"
+#include "tqp_device.cuh"
+#include "tqp_launch.h"
+
+namespace tqp {
+namespace tmem_ffn {
+
+constexpr int kThreads = 576;
+constexpr int kXStageBytes = 16384;   // 128 token rows x 64 K x 2 B
+constexpr int kQStages = 8;
+constexpr int kQStageBytes = 9216;    // up to 2 x 4096 B of codes + 1024 B of scales
+constexpr int kTRow = 272;            // staging row: one token's 128 features in fp16, +16 B against bank conflicts
+constexpr uint32_t kWBase = 256;      // first TMEM column of the weight stages
+
+template <int MODE> struct Cfg;
+template <> struct Cfg<GATEUP> {
+  static constexpr int kXStages = 5, kWStages = 4, kWCols = 64, kStaging = 2 * 128 * kTRow;   // G and U tiles
+};
+template <> struct Cfg<DOWN> {
+  static constexpr int kXStages = 8, kWStages = 8, kWCols = 32, kStaging = 2 * 32 * kTRow;    // 2 chunk buffers
+};
+
+struct Ctl {
+  uint64_t x_full[8], x_empty[8];
+  uint64_t q_full[kQStages], q_empty[kQStages];
+  uint64_t w_full[8], w_empty[8];
+  uint64_t acc_full[2], acc_empty[2];
+  uint64_t drain;
+  uint64_t epi;
+  uint32_t tmem_base;
+  int abort_flag;
+};
+
+template <int MODE>
+constexpr size_t smem_bytes() {
+  return 1024 + size_t(Cfg<MODE>::kXStages) * kXStageBytes + size_t(kQStages) * kQStageBytes +
+         size_t(Cfg<MODE>::kStaging) + sizeof(Ctl);
+}
+static_assert(smem_bytes<GATEUP>() <= 232448 && smem_bytes<DOWN>() <= 232448, "shared memory budget");
+
+// Barrier among the 128 epilogue threads (warps 0-3) only, on an mbarrier so
+// that the wait is bounded: false once the CTA has aborted or the limit expired.
+struct EpiSync {
+  uint64_t* bar;
+  uint32_t phase = 0;
+  __device__ __forceinline__ bool sync(volatile int* abort_flag, int32_t* status) {
+    mbar_arrive(bar);
+    const bool ok = mbar_wait<32>(bar, phase, abort_flag, status);
+    phase ^= 1u;
+    return ok;
+  }
+};
+
+// 32 tokens x this lane's feature (16 words of fp16 pairs, word j = tokens 2j,
+// 2j+1) into a [token][feature] tile: lane pairs trade halves so that each lane
+// writes two adjacent features of one token as one 32-bit word.
+__device__ __forceinline__ void stage_tokens(uint8_t* tile, int t0, int row, const uint32_t* w) {
+  const bool odd = (threadIdx.x & 1) != 0;
+  uint8_t* colp = tile + (row & ~1) * 2;
+#pragma unroll
+  for (int j = 0; j < 16; ++j) {
+    const uint32_t other = __shfl_xor_sync(0xFFFFFFFFu, w[j], 1);
+    const uint32_t v = odd ? __byte_perm(other, w[j], 0x7632) : __byte_perm(w[j], other, 0x5410);
+    *reinterpret_cast<uint32_t*>(colp + (t0 + 2 * j + (odd ? 1 : 0)) * kTRow) = v;
+  }
+}
+
+__device__ __forceinline__ uint32_t f32x2_to_f16x2(float lo, float hi) {
+  const __half2 h = __floats2half2_rn(lo, hi);
+  return *reinterpret_cast<const uint32_t*>(&h);
+}
+
+// silu(g) * u for a pair of fp16 values each, as an fp16 pair
+__device__ __forceinline__ uint32_t swiglu_pair(uint32_t g2, uint32_t u2) {
+  const float2 g = __half22float2(*reinterpret_cast<const __half2*>(&g2));
+  const float2 u = __half22float2(*reinterpret_cast<const __half2*>(&u2));
+  const float h0 = __fdividef(g.x * u.x, 1.0f + __expf(-g.x));
+  const float h1 = __fdividef(g.y * u.y, 1.0f + __expf(-g.y));
+  return f32x2_to_f16x2(h0, h1);
+}
+
+template <int MODE>
+__global__ void __launch_bounds__(kThreads, 1)
+    expert_ffn_kernel(const GemmArgs a, const __grid_constant__ CUtensorMap tq0,
+                      const __grid_constant__ CUtensorMap tq1, const __grid_constant__ CUtensorMap ts0,
+                      const __grid_constant__ CUtensorMap ts1, const __grid_constant__ CUtensorMap th) {
+  constexpr bool kGU = (MODE == GATEUP);
+  constexpr int XS = Cfg<MODE>::kXStages;
+  constexpr int WS = Cfg<MODE>::kWStages;
+  constexpr uint32_t kWCols = Cfg<MODE>::kWCols;
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  uint8_t* x_base = smem;
+  uint8_t* q_base = x_base + size_t(XS) * kXStageBytes;
+  uint8_t* staging = q_base + size_t(kQStages) * kQStageBytes;
+  Ctl* ctl = reinterpret_cast<Ctl*>(staging + Cfg<MODE>::kStaging);
+  volatile int* abort_flag = &ctl->abort_flag;
+
+  const int warp = threadIdx.x >> 5;
+  const int lane = threadIdx.x & 31;
+
+  if (threadIdx.x == 0) {
+    for (int i = 0; i < XS; ++i) {
+      mbar_init(&ctl->x_full[i], 128);
+      mbar_init(&ctl->x_empty[i], 1);
+    }
+    for (int i = 0; i < kQStages; ++i) {
+      mbar_init(&ctl->q_full[i], 1);
+      mbar_init(&ctl->q_empty[i], 256);
+    }
+    for (int i = 0; i < WS; ++i) {
+      mbar_init(&ctl->w_full[i], 256);
+      mbar_init(&ctl->w_empty[i], 1);
+    }
+    for (int i = 0; i < 2; ++i) {
+      mbar_init(&ctl->acc_full[i], 1);
+      mbar_init(&ctl->acc_empty[i], 128);
+    }
+    mbar_init(&ctl->drain, 1);
+    mbar_init(&ctl->epi, 128);
+    ctl->abort_flag = 0;
+    fence_barrier_init();
+  }
+  if (warp == 4) {
+    tmem_alloc(&ctl->tmem_base, 512);
+    tmem_relinquish();
+  }
+  if (threadIdx.x == 5 * 32) {
+    prefetch_tmap(&tq0);
+    prefetch_tmap(&ts0);
+    if (kGU) {
+      prefetch_tmap(&tq1);
+      prefetch_tmap(&ts1);
+    }
+  }
+  if (threadIdx.x == 6 * 32 && !kGU) prefetch_tmap(&th);
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem_base = ctl->tmem_base;
+
+  const int nunits = total_units(a);
+  const int nkb = a.nkb_main + a.nkb_lora;
+  const int ngrp = a.g >= 64 ? 1 : 64 / a.g;   // scale rows per 64-wide K-block
+
+  if (warp < 4) {
+    // ------------------------------------------------------------ epilogue
+    const int row = warp * 32 + lane;   // feature within the tile = TMEM lane
+    const uint32_t tl = tmem_base + (uint32_t(warp * 32) << 16);
+    int it = 0;
+    int chunk = 0;   // DOWN: running chunk count (selects the staging tile)
+    EpiSync es{&ctl->epi};
+    for (int u = blockIdx.x; u < nunits; u += gridDim.x, ++it) {
+      const Unit un = decode_unit(a, u);
+      const int n16 = (un.rows + 15) & ~15;
+      if (kGU) {
+        if (!mbar_wait<128>(&ctl->acc_full[0], uint32_t(it) & 1u, abort_flag, a.status)) break;
+        tc_fence_after();
+        uint8_t* tg = staging;
+        uint8_t* tu = staging + 128 * kTRow;
+        // drain: G and U as fp16 into the [token][feature] tiles
+#pragma unroll 1
+        for (int c = 0; c < n16; c += 32) {
+          float gv[32], uv[32];
+          tmem_ld32(tl + c, gv);
+          tmem_ld32(tl + 128 + c, uv);
+          uint32_t gw[16], uw[16];
+#pragma unroll
+          for (int j = 0; j < 16; ++j) {
+            gw[j] = f32x2_to_f16x2(gv[2 * j], gv[2 * j + 1]);
+            uw[j] = f32x2_to_f16x2(uv[2 * j], uv[2 * j + 1]);
+          }
+          stage_tokens(tg, c, row, gw);
+          stage_tokens(tu, c, row, uw);
+        }
+        tc_fence_before();
+        mbar_arrive(&ctl->acc_empty[0]);
+        if (!es.sync(abort_flag, a.status)) break;
+        // SwiGLU on 8-feature pieces of the valid tokens, 16-byte row stores,
+        // overlapping the next unit's main loop
+        uint16_t* hout = static_cast<uint16_t*>(a.out) + un.nt * 128;
+        for (int p = threadIdx.x; p < un.rows * 16; p += 128) {
+          const int t = p >> 4, fg = p & 15;
+          const uint4 g = *reinterpret_cast<const uint4*>(tg + t * kTRow + fg * 16);
+          const uint4 uq = *reinterpret_cast<const uint4*>(tu + t * kTRow + fg * 16);
+          const uint4 h = make_uint4(swiglu_pair(g.x, uq.x), swiglu_pair(g.y, uq.y), swiglu_pair(g.z, uq.z),
+                                     swiglu_pair(g.w, uq.w));
+          const size_t grow = size_t(un.base + t);
+          *reinterpret_cast<uint4*>(hout + grow * a.out_ld + fg * 8) = h;
+          if (a.aux) {  // keep the pre-activations for the backward
+            uint16_t* ar = a.aux + grow * (2 * size_t(a.f_dim)) + un.nt * 128 + fg * 8;
+            *reinterpret_cast<uint4*>(ar) = g;
+            *reinterpret_cast<uint4*>(ar + a.f_dim) = uq;
+          }
+        }
+        if (!es.sync(abort_flag, a.status)) break;  // the tiles are free for the next unit's drain
+      } else {
+        const int ab = it & 1;
+        if (!mbar_wait<128>(&ctl->acc_full[ab], uint32_t(it >> 1) & 1u, abort_flag, a.status)) break;
+        tc_fence_after();
+        uint16_t* out = static_cast<uint16_t*>(a.out) + un.nt * 128;
+        bool stop = false;
+#pragma unroll 1
+        for (int c = 0; c < n16; c += 32, ++chunk) {
+          float v[32];
+          tmem_ld32(tl + uint32_t(ab * 128 + c), v);
+          if (c + 32 >= n16) {  // last read of this accumulator: hand it back before storing
+            tc_fence_before();
+            mbar_arrive(&ctl->acc_empty[ab]);
+          }
+          uint32_t pk[16];
+#pragma unroll
+          for (int j = 0; j < 16; ++j) pk[j] = f32x2_to_f16x2(v[2 * j], v[2 * j + 1]);
+          // consecutive chunks alternate between the two tiles; the barrier after a
+          // tile is written also orders every earlier read of the other tile
+          uint8_t* tile = staging + (chunk & 1) * (32 * kTRow);
+          stage_tokens(tile, 0, row, pk);
+          if (!es.sync(abort_flag, a.status)) { stop = true; break; }
+          const int nt = min(32, un.rows - c);
+          for (int p = threadIdx.x; p < nt * 16; p += 128) {
+            const int t = p >> 4, fg = p & 15;
+            *reinterpret_cast<uint4*>(out + size_t(un.base + c + t) * a.out_ld + fg * 8) =
+                *reinterpret_cast<const uint4*>(tile + t * kTRow + fg * 16);
+          }
+        }
+        if (stop) break;
+      }
+    }
+  } else if (warp == 4) {
+    // ------------------------------------------------------------ MMA issuer
+    if (lane == 0) {
+      Ring rx, rw;
+      int it = 0;
+      bool ok = true;
+      for (int u = blockIdx.x; u < nunits && ok; u += gridDim.x, ++it) {
+        const Unit un = decode_unit(a, u);
+        const int n16 = (un.rows + 15) & ~15;
+        const uint32_t idesc = idesc_f16(128, n16);
+        const int ab = kGU ? 0 : (it & 1);
+        const uint32_t eph = (kGU ? uint32_t(it) & 1u : uint32_t(it >> 1) & 1u) ^ 1u;
+        if (!mbar_wait(&ctl->acc_empty[ab], eph, abort_flag, a.status)) { ok = false; break; }
+        tc_fence_after();
+        const uint32_t dacc = tmem_base + uint32_t(ab * 128);
+        for (int kb = 0; kb < nkb; ++kb) {
+          if (!mbar_wait(&ctl->x_full[rx.stage], rx.phase, abort_flag, a.status) ||
+              !mbar_wait(&ctl->w_full[rw.stage], rw.phase, abort_flag, a.status)) {
+            ok = false;
+            break;
+          }
+          tc_fence_after();
+          const int ksteps = (kb < a.nkb_lora) ? (min(64, a.lora_k - kb * 64) + 15) / 16 : 4;
+          const uint64_t bdesc = sdesc_k_sw128(smem_u32(x_base + size_t(rx.stage) * kXStageBytes));
+          const uint32_t wa = tmem_base + kWBase + uint32_t(rw.stage) * kWCols;
+          if (ksteps == 4) {
+#pragma unroll
+            for (int kk = 0; kk < 4; ++kk) {
+              const uint32_t acc = (kb > 0 || kk > 0) ? 1u : 0u;
+              umma_f16_ts(dacc, wa + uint32_t(8 * kk), bdesc + uint64_t(2 * kk), idesc, acc);
+              if (kGU) umma_f16_ts(dacc + 128, wa + 32 + uint32_t(8 * kk), bdesc + uint64_t(2 * kk), idesc, acc);
+            }
+          } else {
+            for (int kk = 0; kk < ksteps; ++kk) {
+              const uint32_t acc = (kb > 0 || kk > 0) ? 1u : 0u;
+              umma_f16_ts(dacc, wa + uint32_t(8 * kk), bdesc + uint64_t(2 * kk), idesc, acc);
+              if (kGU) umma_f16_ts(dacc + 128, wa + 32 + uint32_t(8 * kk), bdesc + uint64_t(2 * kk), idesc, acc);
+            }
+          }
+          umma_commit(&ctl->x_empty[rx.stage]);
+          umma_commit(&ctl->w_empty[rw.stage]);
+          rx.next<XS>();
+          rw.next<WS>();
+        }
+        if (!ok) break;
+        umma_commit(&ctl->acc_full[ab]);
+      }
+      // make sure no MMA is still reading or writing TMEM before teardown
+      umma_commit(&ctl->drain);
+      mbar_wait(&ctl->drain, 0, abort_flag, a.status);
+    }
+    __syncwarp();
+  } else if (warp == 5) {
+    // ------------------------------------------------------------ TMA producer (int4 + scales)
+    if (lane == 0) {
+      Ring q;
+      const uint32_t bytes = kGU ? uint32_t(8192 + 512 * ngrp) : uint32_t(4096 + 256 * ngrp);
+      const int gpe = a.in_dim / a.g;  // scale rows per expert
+      int issued = 0;
+      uint32_t last_phase = 0;
+      int last_stage = 0;
+      for (int u = blockIdx.x; u < nunits; u += gridDim.x) {
+        const Unit un = decode_unit(a, u);
+        const int nrow0 = un.e * a.out_dim + un.nt * 128;
+        bool ok = true;
+        for (int km = 0; km < a.nkb_main; ++km) {
+          if (!mbar_wait<64>(&ctl->q_empty[q.stage], q.phase ^ 1u, abort_flag, a.status)) { ok = false; break; }
+          uint8_t* qs = q_base + size_t(q.stage) * kQStageBytes;
+          uint64_t* bar = &ctl->q_full[q.stage];
+          const int srow = un.e * gpe + (km * 64) / a.g;
+          mbar_arrive_expect_tx(bar, bytes);
+          tma_load_2d(smem_u32(qs), &tq0, bar, km * 32, nrow0);
+          if (kGU) {
+            tma_load_2d(smem_u32(qs + 4096), &tq1, bar, km * 32, nrow0);
+            tma_load_2d(smem_u32(qs + 8192), &ts0, bar, un.nt * 128, srow);
+            tma_load_2d(smem_u32(qs + 8192 + 256 * ngrp), &ts1, bar, un.nt * 128, srow);
+          } else {
+            tma_load_2d(smem_u32(qs + 4096), &ts0, bar, un.nt * 128, srow);
+          }
+          ++issued;
+          last_stage = q.stage;
+          last_phase = q.phase;
+          q.next<kQStages>();
+        }
+        if (!ok) break;
+      }
+      // on an abort, wait (bounded) until the last issued stage has landed
+      if (issued > 0 && *abort_flag) mbar_wait(&ctl->q_full[last_stage], last_phase, abort_flag, a.status);
+    }
+  } else if (warp < 10) {
+    // ------------------------------------------------------------ token producer
+    const int tid = threadIdx.x - 6 * 32;  // 0..127 = token row of the tile
+    Ring rx;
+    int pend_stage = -1;
+    uint32_t pend_phase = 0;
+    for (int u = blockIdx.x; u < nunits; u += gridDim.x) {
+      const Unit un = decode_unit(a, u);
+      const bool valid = tid < un.rows;
+      const int grow = un.base + (valid ? tid : 0);
+      const uint16_t* src = nullptr;
+      if (kGU) src = a.a_src + size_t(valid ? __ldg(a.perm_token + grow) : 0) * a.a_ld;
+      const uint16_t* lsrc = a.a_lora ? a.a_lora + size_t(grow) * a.lora_ld : nullptr;
+      bool ok = true;
+      for (int kb = 0; kb < nkb; ++kb) {
+        if (!mbar_wait<64>(&ctl->x_empty[rx.stage], rx.phase ^ 1u, abort_flag, a.status)) { ok = false; break; }
+        const uint32_t st_u = smem_u32(x_base + size_t(rx.stage) * kXStageBytes);
+        uint64_t* full = &ctl->x_full[rx.stage];
+        if (kb < a.nkb_lora) {
+          // rank-space rows (s X[Ag|Au] or s H Ad), zero-filled past lora_k
+          if (valid) {
+#pragma unroll
+            for (int c = 0; c < 8; ++c) {
+              const int colk = kb * 64 + c * 8;
+              const bool in = colk < a.lora_k;
+              cp_async16(st_u + sw128_offset(tid, c), lsrc + (in ? colk : 0), in ? 16u : 0u);
+            }
+          }
+          cp_async_arrive_noinc(full);
+        } else {
+          const int km = kb - a.nkb_lora;
+          if (kGU) {
+            if (valid) {
+              const uint16_t* p = src + km * 64;
+#pragma unroll
+              for (int c = 0; c < 8; ++c) cp_async16(st_u + sw128_offset(tid, c), p + c * 8, 16);
+            }
+            cp_async_arrive_noinc(full);
+          } else if (tid == 0) {
+            mbar_arrive_expect_tx(full, uint32_t(kXStageBytes));
+            tma_load_2d(st_u, &th, full, km * 64, un.base);
+            pend_stage = rx.stage;
+            pend_phase = rx.phase;
+          } else {
+            mbar_arrive(full);
+          }
+        }
+        rx.next<XS>();
+      }
+      if (!ok) break;
+    }
+    cp_async_wait_all();
+    if (tid == 0 && *abort_flag && pend_stage >= 0)
+      mbar_wait(&ctl->x_full[pend_stage], pend_phase, abort_flag, a.status);
+  } else {
+    // ------------------------------------------------------------ weight producer
+    const int wi = warp - 10;                 // 0..7
+    const int lrow = 32 * (warp & 3) + lane;  // TMEM lane = feature within the tile
+    const int part = wi >> 2;                 // GATEUP: 0 gate / 1 up rows; DOWN: K half
+    const uint32_t tw = tmem_base + (uint32_t(32 * (warp & 3)) << 16) + kWBase + uint32_t(part * (kGU ? 32 : 16));
+    Ring rw, q;
+    for (int u = blockIdx.x; u < nunits; u += gridDim.x) {
+      const Unit un = decode_unit(a, u);
+      const int n = un.nt * 128 + lrow;     // output feature
+      bool ok = true;
+      for (int kb = 0; kb < nkb; ++kb) {
+        if (!mbar_wait(&ctl->w_empty[rw.stage], rw.phase ^ 1u, abort_flag, a.status)) { ok = false; break; }
+        tc_fence_after();
+        uint32_t v[kGU ? 32 : 16];
+        constexpr int kChunks = kGU ? 8 : 4;   // 8 K values per chunk
+        if (kb < a.nkb_lora) {
+          // LoRA B rows as fp16: gate rows hold Bg in K' [0, r), up rows Bu in [r, 2r)
+#pragma unroll
+          for (int c = 0; c < kChunks; ++c) {
+            const int colk = kb * 64 + (kGU ? c : part * 4 + c) * 8;
+            const int src = (kGU && part == 1) ? colk - a.r : colk;
+            uint4 w4 = make_uint4(0, 0, 0, 0);
+            if (src >= 0 && src < a.r) {
+              const uint16_t* bsrc = (kGU && part == 1) ? a.b1 : a.b0;
+              w4 = bf16x8_to_f16x8(__ldg(reinterpret_cast<const uint4*>(bsrc + (size_t(un.e) * a.out_dim + n) * a.r + src)));
+            }
+            v[4 * c] = w4.x; v[4 * c + 1] = w4.y; v[4 * c + 2] = w4.z; v[4 * c + 3] = w4.w;
+          }
+        } else {
+          if (!mbar_wait(&ctl->q_full[q.stage], q.phase, abort_flag, a.status)) { ok = false; break; }
+          const uint8_t* qs = q_base + size_t(q.stage) * kQStageBytes;
+          uint32_t wd[kChunks];
+          uint32_t s_lo, s_hi;
+          if (kGU) {
+            const uint4 c0 = *reinterpret_cast<const uint4*>(qs + part * 4096 + lrow * 32);
+            const uint4 c1 = *reinterpret_cast<const uint4*>(qs + part * 4096 + lrow * 32 + 16);
+            wd[0] = c0.x; wd[1] = c0.y; wd[2] = c0.z; wd[3] = c0.w;
+            wd[4] = c1.x; wd[5] = c1.y; wd[6] = c1.z; wd[7] = c1.w;
+            const uint16_t* sc = reinterpret_cast<const uint16_t*>(qs + 8192 + part * 256 * ngrp);
+            s_lo = scale_pair(sc[lrow]);
+            s_hi = (ngrp == 2) ? scale_pair(sc[128 + lrow]) : s_lo;
+          } else {
+            const uint4 c0 = *reinterpret_cast<const uint4*>(qs + lrow * 32 + part * 16);
+            wd[0] = c0.x; wd[1] = c0.y; wd[2] = c0.z; wd[3] = c0.w;
+            const uint16_t* sc = reinterpret_cast<const uint16_t*>(qs + 4096);
+            s_lo = scale_pair(sc[(ngrp == 2 ? part : 0) * 128 + lrow]);
+            s_hi = s_lo;
+          }
+          // the code slot goes back once its values are in registers, behind a proxy
+          // fence (its next fill is an async-proxy TMA write)
+          fence_proxy_async_smem();
+          mbar_arrive(&ctl->q_empty[q.stage]);
+          q.next<kQStages>();
+#pragma unroll
+          for (int c = 0; c < kChunks; ++c) {
+            const uint4 d4 = dequant_word(wd[c], (kGU && c >= 4) ? s_hi : s_lo);
+            v[4 * c] = d4.x; v[4 * c + 1] = d4.y; v[4 * c + 2] = d4.z; v[4 * c + 3] = d4.w;
+          }
+        }
+        const uint32_t taddr = tw + uint32_t(rw.stage) * kWCols;
+        if (kGU) tmem_st32(taddr, v);
+        else tmem_st16(taddr, v);
+        tmem_wait_st();
+        tc_fence_before();
+        mbar_arrive(&ctl->w_full[rw.stage]);
+        rw.next<WS>();
+      }
+      if (!ok) break;
+    }
+  }
+
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 4) {
+    tc_fence_after();
+    tmem_dealloc(tmem_base, 512);
+  }
+}
+
+template <int MODE>
+static int launch(const GemmArgs& a, const Maps& mp, int units_upper, cudaStream_t s) {
+  static bool attr_set = false;
+  if (!attr_set) {
+    if (cudaFuncSetAttribute(expert_ffn_kernel<MODE>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                             int(smem_bytes<MODE>())) != cudaSuccess)
+      return TQP_ERR_CUDA;
+    attr_set = true;
+  }
+  const int grid = units_upper < num_sms() ? (units_upper > 0 ? units_upper : 1) : num_sms();
+  expert_ffn_kernel<MODE><<<grid, kThreads, smem_bytes<MODE>(), s>>>(a, mp.m[TQ0], mp.m[TQ1], mp.m[TS0],
+                                                                      mp.m[TS1], mp.m[TA]);
+  return cudaGetLastError() == cudaSuccess ? TQP_OK : TQP_ERR_CUDA;
+}
+
+}  // namespace tmem_ffn
+
+int run_expert_ffn(int mode, const GemmArgs& a, const Maps& mp, int units_upper, cudaStream_t s) {
+  if (mode == GATEUP) return tmem_ffn::launch<GATEUP>(a, mp, units_upper, s);
+  if (mode == DOWN) return tmem_ffn::launch<DOWN>(a, mp, units_upper, s);
+  return TQP_ERR_INVALID_ARG;
+}
+
+}  // namespace tqp

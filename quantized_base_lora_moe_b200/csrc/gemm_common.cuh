@@ -1,0 +1,139 @@
+// Device-side pieces shared by the grouped GEMM kernels: work-unit arguments and
+// decoding, pipeline ring counters, and the exact int4 -> fp16 dequantisation.
+#pragma once
+
+#include <cstdint>
+#include <cuda.h>
+#include <cuda_runtime.h>
+
+#include "tqp_device.cuh"
+
+namespace tqp {
+
+enum Mode : int { GATEUP = 0, DOWN = 1, LORA_XA = 2, LORA_HA = 3, ROUTER = 4, DH = 5, DX = 6 };
+
+constexpr int kMBlock = 128;
+
+struct GemmArgs {
+  int E;
+  int nkb_main;        // main K-blocks (64 wide)
+  int kb_per_piece;    // ROUTER: K-blocks per bf16 part (the A columns repeat)
+  int nkb_lora;        // rank-space K-blocks, issued first in each unit
+  int lora_k;          // rank-space contraction extent (2r gate/up and dX, r down and dH)
+  int n_tiles;         // n-tiles per m-block
+  int ntile;           // MMA N (16..256)
+  int g;               // quantisation group
+  int r;               // LoRA rank
+  int in_dim;          // input dim of the int4 projection (scale rows)
+  int out_dim;         // output dim of the int4 projection (code rows)
+  float lora_scale;
+  const int32_t* offsets;
+  const int32_t* mb_prefix;
+  const int32_t* perm_token;
+  const uint16_t* a_src;   // gathered A rows (GATEUP, LORA_XA)
+  int a_ld;
+  const uint16_t* a_lora;  // rank-space A rows [A][lora_ld]
+  int lora_ld;
+  const uint16_t* b0;      // rank-space B^T sources (GATEUP: Bg^T, DOWN: Bd^T)
+  const uint16_t* b1;      // GATEUP: Bu^T
+  void* out;
+  int out_ld;
+  int n_valid;             // valid output columns
+  const float* bias;
+  int32_t* status;
+  uint16_t* aux;           // GATEUP: optional G|U pre-activations out [A][2f]; DH: G|U in
+  int f_dim;
+  int half_kb;             // DX: K-blocks of the gate part
+  const uint16_t* lb0;     // DH / DX rank-space step: A^T sources read transposed (Ad^T | Ag^T)
+  const uint16_t* lb1;     // DX: Au^T
+  int lb_ld;
+};
+
+struct Unit {
+  int e, nt, mb, rows, base;
+};
+
+__device__ __forceinline__ int total_units(const GemmArgs& a) { return __ldg(a.mb_prefix + a.E) * a.n_tiles; }
+
+// Units are ordered (expert, n-tile, m-block): m-blocks of one n-tile share a B
+// tile, n-tiles of one m-block share the A rows; neighbours run concurrently.
+__device__ __forceinline__ Unit decode_unit(const GemmArgs& a, int u) {
+  int lo = 0, hi = a.E;
+  while (hi - lo > 1) {
+    const int mid = (lo + hi) >> 1;
+    if (__ldg(a.mb_prefix + mid) * a.n_tiles <= u) lo = mid;
+    else hi = mid;
+  }
+  Unit un;
+  un.e = lo;
+  const int p0 = __ldg(a.mb_prefix + lo);
+  const int nmb = __ldg(a.mb_prefix + lo + 1) - p0;
+  const int idx = u - p0 * a.n_tiles;
+  un.nt = idx / nmb;
+  un.mb = idx - un.nt * nmb;
+  const int o0 = __ldg(a.offsets + lo);
+  const int cnt = __ldg(a.offsets + lo + 1) - o0;
+  un.rows = min(kMBlock, cnt - un.mb * kMBlock);
+  un.base = o0 + un.mb * kMBlock;
+  return un;
+}
+
+struct Ring {
+  int stage = 0;
+  uint32_t phase = 0;
+  template <int N>
+  __device__ __forceinline__ void next() {
+    if (++stage == N) { stage = 0; phase ^= 1u; }
+  }
+};
+
+__device__ __forceinline__ void mbar_expect_tx(uint64_t* bar, uint32_t bytes) {
+  asm volatile("mbarrier.expect_tx.shared::cta.b64 [%0], %1;" ::"r"(smem_u32(bar)), "r"(bytes) : "memory");
+}
+
+__device__ __forceinline__ uint32_t f16x2_sub(uint32_t a, uint32_t b) {
+  uint32_t d;
+  asm("sub.rn.f16x2 %0, %1, %2;" : "=r"(d) : "r"(a), "r"(b));
+  return d;
+}
+
+__device__ __forceinline__ uint32_t f16x2_mul(uint32_t a, uint32_t b) {
+  uint32_t d;
+  asm("mul.rn.f16x2 %0, %1, %2;" : "=r"(d) : "r"(a), "r"(b));
+  return d;
+}
+
+// 8 int4 codes (one storage word) -> 8 fp16 values q * s as a 16-byte chunk.
+// (n & 0xF) ^ 8 = q + 8 for a two's-complement nibble n, and 0x6400 | m is the
+// fp16 value 1024 + m, so one AND/XOR gives the pair (1032 + q); subtracting
+// 1032 is exact and q * s (3-bit code times 8-bit scale) is exact in fp16.
+__device__ __forceinline__ uint4 dequant_word(uint32_t w, uint32_t s2) {
+  const uint32_t k1032 = 0x64086408u;  // fp16 pair (1032, 1032)
+  uint32_t o[4];
+#pragma unroll
+  for (int i = 0; i < 4; ++i) {
+    const uint32_t v = ((w >> (4 * i)) & 0x000F000Fu) ^ 0x64086408u;  // fp16 pair 1032 + q
+    o[i] = f16x2_mul(f16x2_sub(v, k1032), s2);
+  }
+  return make_uint4(o[0], o[1], o[2], o[3]);
+}
+
+__device__ __forceinline__ uint32_t scale_pair(uint16_t sbits) {
+  const uint32_t sh = bf16_to_f16_bits(sbits);
+  return sh | (sh << 16);
+}
+
+// One B-tile row (forward): NW int4 words (8 K values each) of row `brow`
+// starting at chunk part*NW, dequantised into the 128B-swizzled K-major tile.
+
+// Host side: the tensor maps handed to a grouped GEMM launch.
+struct Maps {
+  CUtensorMap m[7];
+};
+enum { TQ0 = 0, TQ1 = 1, TS0 = 2, TS1 = 3, TA = 4, TB0 = 5, TB1 = 6 };
+
+// Forward expert projections with the dequantised weights held in tensor memory
+// (expert_ffn.cu): mode GATEUP or DOWN.
+int run_expert_ffn(int mode, const GemmArgs& a, const Maps& mp, int units_upper, cudaStream_t s);
+
+}  // namespace tqp

@@ -31,12 +31,11 @@
 #include <cudaTypedefs.h>
 #include <cuda_runtime.h>
 
+#include "gemm_common.cuh"
 #include "tqp_device.cuh"
 #include "tqp_launch.h"
 
 namespace tqp {
-
-enum Mode : int { GATEUP = 0, DOWN = 1, LORA_XA = 2, LORA_HA = 3, ROUTER = 4, DH = 5, DX = 6 };
 
 constexpr int kThreads = 576;
 constexpr int kAStages = 5;           // A tiles (TMA / cp.async from L2): deep, to cover L2 latency
@@ -45,42 +44,6 @@ constexpr int kQStages = 8;           // int4 codes + scales from DRAM: deepest 
 constexpr int kAStageBytes = 16384;   // 128 rows x 64 K x 2 B
 constexpr int kBStageBytes = 32768;   // up to 256 rows x 64 K x 2 B
 constexpr int kQStageBytes = 9216;    // up to 8192 B of codes + 1024 B of scales
-constexpr int kMBlock = 128;
-
-struct GemmArgs {
-  int E;
-  int nkb_main;        // main K-blocks (64 wide)
-  int kb_per_piece;    // ROUTER: K-blocks per bf16 part (the A columns repeat)
-  int nkb_lora;        // rank-space K-blocks, issued first in each unit
-  int lora_k;          // rank-space contraction extent (2r gate/up and dX, r down and dH)
-  int n_tiles;         // n-tiles per m-block
-  int ntile;           // MMA N (16..256)
-  int g;               // quantisation group
-  int r;               // LoRA rank
-  int in_dim;          // input dim of the int4 projection (scale rows)
-  int out_dim;         // output dim of the int4 projection (code rows)
-  float lora_scale;
-  const int32_t* offsets;
-  const int32_t* mb_prefix;
-  const int32_t* perm_token;
-  const uint16_t* a_src;   // gathered A rows (GATEUP, LORA_XA)
-  int a_ld;
-  const uint16_t* a_lora;  // rank-space A rows [A][lora_ld]
-  int lora_ld;
-  const uint16_t* b0;      // rank-space B^T sources (GATEUP: Bg^T, DOWN: Bd^T)
-  const uint16_t* b1;      // GATEUP: Bu^T
-  void* out;
-  int out_ld;
-  int n_valid;             // valid output columns
-  const float* bias;
-  int32_t* status;
-  uint16_t* aux;           // GATEUP: optional G|U pre-activations out [A][2f]; DH: G|U in
-  int f_dim;
-  int half_kb;             // DX: K-blocks of the gate part
-  const uint16_t* lb0;     // DH / DX rank-space step: A^T sources read transposed (Ad^T | Ag^T)
-  const uint16_t* lb1;     // DX: Au^T
-  int lb_ld;
-};
 
 struct SmemCtl {
   uint64_t a_full[kAStages];
@@ -100,82 +63,7 @@ constexpr size_t kSmemBytes = 1024 /*align slack*/ + size_t(kAStages) * kAStageB
                               size_t(kBStages) * kBStageBytes + size_t(kQStages) * kQStageBytes + sizeof(SmemCtl);
 static_assert(kSmemBytes <= 232448, "shared memory budget");
 
-struct Unit {
-  int e, nt, mb, rows, base;
-};
 
-__device__ __forceinline__ int total_units(const GemmArgs& a) { return __ldg(a.mb_prefix + a.E) * a.n_tiles; }
-
-// Units are ordered (expert, n-tile, m-block): m-blocks of one n-tile share a B
-// tile, n-tiles of one m-block share the A rows; neighbours run concurrently.
-__device__ __forceinline__ Unit decode_unit(const GemmArgs& a, int u) {
-  int lo = 0, hi = a.E;
-  while (hi - lo > 1) {
-    const int mid = (lo + hi) >> 1;
-    if (__ldg(a.mb_prefix + mid) * a.n_tiles <= u) lo = mid;
-    else hi = mid;
-  }
-  Unit un;
-  un.e = lo;
-  const int p0 = __ldg(a.mb_prefix + lo);
-  const int nmb = __ldg(a.mb_prefix + lo + 1) - p0;
-  const int idx = u - p0 * a.n_tiles;
-  un.nt = idx / nmb;
-  un.mb = idx - un.nt * nmb;
-  const int o0 = __ldg(a.offsets + lo);
-  const int cnt = __ldg(a.offsets + lo + 1) - o0;
-  un.rows = min(kMBlock, cnt - un.mb * kMBlock);
-  un.base = o0 + un.mb * kMBlock;
-  return un;
-}
-
-struct Ring {
-  int stage = 0;
-  uint32_t phase = 0;
-  template <int N>
-  __device__ __forceinline__ void next() {
-    if (++stage == N) { stage = 0; phase ^= 1u; }
-  }
-};
-
-__device__ __forceinline__ void mbar_expect_tx(uint64_t* bar, uint32_t bytes) {
-  asm volatile("mbarrier.expect_tx.shared::cta.b64 [%0], %1;" ::"r"(smem_u32(bar)), "r"(bytes) : "memory");
-}
-
-__device__ __forceinline__ uint32_t f16x2_sub(uint32_t a, uint32_t b) {
-  uint32_t d;
-  asm("sub.rn.f16x2 %0, %1, %2;" : "=r"(d) : "r"(a), "r"(b));
-  return d;
-}
-
-__device__ __forceinline__ uint32_t f16x2_mul(uint32_t a, uint32_t b) {
-  uint32_t d;
-  asm("mul.rn.f16x2 %0, %1, %2;" : "=r"(d) : "r"(a), "r"(b));
-  return d;
-}
-
-// 8 int4 codes (one storage word) -> 8 fp16 values q * s as a 16-byte chunk.
-// (n & 0xF) ^ 8 = q + 8 for a two's-complement nibble n, and 0x6400 | m is the
-// fp16 value 1024 + m, so one AND/XOR gives the pair (1032 + q); subtracting
-// 1032 is exact and q * s (3-bit code times 8-bit scale) is exact in fp16.
-__device__ __forceinline__ uint4 dequant_word(uint32_t w, uint32_t s2) {
-  const uint32_t k1032 = 0x64086408u;  // fp16 pair (1032, 1032)
-  uint32_t o[4];
-#pragma unroll
-  for (int i = 0; i < 4; ++i) {
-    const uint32_t v = ((w >> (4 * i)) & 0x000F000Fu) ^ 0x64086408u;  // fp16 pair 1032 + q
-    o[i] = f16x2_mul(f16x2_sub(v, k1032), s2);
-  }
-  return make_uint4(o[0], o[1], o[2], o[3]);
-}
-
-__device__ __forceinline__ uint32_t scale_pair(uint16_t sbits) {
-  const uint32_t sh = __half_as_ushort(__float2half_rn(bf16_to_f32(sbits)));
-  return sh | (sh << 16);
-}
-
-// One B-tile row (forward): NW int4 words (8 K values each) of row `brow`
-// starting at chunk part*NW, dequantised into the 128B-swizzled K-major tile.
 // s_lo / s_hi: fp16 scale pairs of the first / second 32-wide group (equal when g >= 64).
 template <int NW>
 __device__ __forceinline__ void dequant_row(const uint8_t* qs, uint8_t* bst, int brow, int part, uint32_t s_lo,
@@ -815,11 +703,6 @@ int num_sms() {
   return n;
 }
 
-struct Maps {
-  CUtensorMap m[7];
-  Maps() { memset(m, 0, sizeof(m)); }
-};
-enum { TQ0 = 0, TQ1 = 1, TS0 = 2, TS1 = 3, TA = 4, TB0 = 5, TB1 = 6 };
 
 template <int MODE>
 static int run_gemm(const GemmArgs& a, const Maps& mp, int units_upper, cudaStream_t s) {
@@ -862,7 +745,7 @@ int launch_router_gemm(const uint16_t* x, int T, const tqp_moe_weights* w, float
   a.n_valid = w->E;
   a.bias = w->router_bias;
   a.status = status;
-  Maps mp;
+  Maps mp{};
   if (!make_tile_map(&mp.m[TA], x, uint64_t(T), uint64_t(w->d), 128) ||
       !make_tile_map(&mp.m[TB0], parts, 3 * uint64_t(w->E), uint64_t(w->d), uint32_t(a.ntile)))
     return TQP_ERR_CUDA;
@@ -943,7 +826,7 @@ int launch_grouped_ffn(const uint16_t* x, int T, const int32_t* offsets, const i
     a.out = fb.xa;
     a.out_ld = 2 * r;
     a.n_valid = 2 * r;
-    Maps mp;
+    Maps mp{};
     if (!make_tile_map(&mp.m[TB0], w->lora_a[0], uint64_t(w->E) * r, uint64_t(d), uint32_t(r)) ||
         !make_tile_map(&mp.m[TB1], w->lora_a[1], uint64_t(w->E) * r, uint64_t(d), uint32_t(r)))
       return TQP_ERR_CUDA;
@@ -971,7 +854,7 @@ int launch_grouped_ffn(const uint16_t* x, int T, const int32_t* offsets, const i
     a.f_dim = f;
     const int ngrp = w->group >= 64 ? 1 : 64 / w->group;
     const uint32_t rows_box = uint32_t(a.ntile / 2);
-    Maps mp;
+    Maps mp{};
     bool ok = make_map(&mp.m[TQ0], CU_TENSOR_MAP_DATA_TYPE_UINT8, w->wq[0], d / 2, uint64_t(w->E) * f, d / 2, 32,
                        rows_box) &&
               make_map(&mp.m[TQ1], CU_TENSOR_MAP_DATA_TYPE_UINT8, w->wq[1], d / 2, uint64_t(w->E) * f, d / 2, 32,
@@ -981,7 +864,10 @@ int launch_grouped_ffn(const uint16_t* x, int T, const int32_t* offsets, const i
               make_map(&mp.m[TS1], CU_TENSOR_MAP_DATA_TYPE_UINT16, w->wscale[1], f, uint64_t(w->E) * (d / w->group),
                        uint64_t(f) * 2, rows_box, ngrp);
     if (!ok) return TQP_ERR_CUDA;
-    if ((rc = run_gemm<GATEUP>(a, mp, mb_upper * a.n_tiles, s)) != TQP_OK) return rc;
+    // 128-feature tiles run with the weights in TMEM (expert_ffn.cu)
+    rc = (f % 128 == 0) ? run_expert_ffn(GATEUP, a, mp, mb_upper * a.n_tiles, s)
+                        : run_gemm<GATEUP>(a, mp, mb_upper * a.n_tiles, s);
+    if (rc != TQP_OK) return rc;
   }
   if (r > 0) {  // ha = s * H Ad
     GemmArgs a = base;
@@ -991,7 +877,7 @@ int launch_grouped_ffn(const uint16_t* x, int T, const int32_t* offsets, const i
     a.out = fb.ha;
     a.out_ld = r;
     a.n_valid = r;
-    Maps mp;
+    Maps mp{};
     if (!make_tile_map(&mp.m[TA], h, uint64_t(A), uint64_t(f), 128) ||
         !make_tile_map(&mp.m[TB0], fb.adT16, uint64_t(w->E) * r, uint64_t(f), uint32_t(r)))
       return TQP_ERR_CUDA;
@@ -1002,8 +888,8 @@ int launch_grouped_ffn(const uint16_t* x, int T, const int32_t* offsets, const i
     a.nkb_main = f / 64;
     a.nkb_lora = r > 0 ? (r + 63) / 64 : 0;
     a.lora_k = r;
-    a.ntile = (d % 256 == 0) ? 256 : 128;
-    a.n_tiles = d / a.ntile;
+    a.ntile = 128;
+    a.n_tiles = d / 128;
     a.in_dim = f;
     a.out_dim = d;
     a.a_lora = fb.ha;
@@ -1013,14 +899,14 @@ int launch_grouped_ffn(const uint16_t* x, int T, const int32_t* offsets, const i
     a.out_ld = d;
     a.n_valid = d;
     const int ngrp = w->group >= 64 ? 1 : 64 / w->group;
-    Maps mp;
+    Maps mp{};
     bool ok = make_tile_map(&mp.m[TA], h, uint64_t(A), uint64_t(f), 128) &&
               make_map(&mp.m[TQ0], CU_TENSOR_MAP_DATA_TYPE_UINT8, w->wq[2], f / 2, uint64_t(w->E) * d, f / 2, 32,
                        uint32_t(a.ntile)) &&
               make_map(&mp.m[TS0], CU_TENSOR_MAP_DATA_TYPE_UINT16, w->wscale[2], d, uint64_t(w->E) * (f / w->group),
                        uint64_t(d) * 2, uint32_t(a.ntile), ngrp);
     if (!ok) return TQP_ERR_CUDA;
-    if ((rc = run_gemm<DOWN>(a, mp, mb_upper * a.n_tiles, s)) != TQP_OK) return rc;
+    if ((rc = run_expert_ffn(DOWN, a, mp, mb_upper * a.n_tiles, s)) != TQP_OK) return rc;
   }
   return TQP_OK;
 }
@@ -1047,7 +933,7 @@ int launch_dgrad(int which, const uint16_t* a_src, const uint16_t* a_lora, const
   a.f_dim = f;
   a.a_lora = a_lora;
   a.out = out;
-  Maps mp;
+  Maps mp{};
   if (which == 0) {  // DH: K = d (rows of Wd), N = f
     a.ntile = (f % 256 == 0) ? 256 : 128;
     const int ngn = w->group >= a.ntile ? 1 : a.ntile / w->group;

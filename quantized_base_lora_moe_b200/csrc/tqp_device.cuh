@@ -205,6 +205,19 @@ __device__ __forceinline__ void umma_bf16(uint32_t d_tmem, uint64_t adesc, uint6
       : "memory");
 }
 
+// D[tmem] (+)= A[tmem] * B[smem]^T, fp16 inputs, fp32 accumulation, one CTA. A is
+// M=128 lanes x K: each 32-bit column holds two consecutive K elements (the lower
+// K index in the low half); a K step of 16 spans 8 columns.
+__device__ __forceinline__ void umma_f16_ts(uint32_t d_tmem, uint32_t a_tmem, uint64_t bdesc, uint32_t idesc,
+                                            uint32_t accumulate) {
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "setp.ne.b32 p, %4, 0;\n\t"
+      "tcgen05.mma.cta_group::1.kind::f16 [%0], [%1], %2, %3, p;\n\t}" ::"r"(d_tmem),
+      "r"(a_tmem), "l"(bdesc), "r"(idesc), "r"(accumulate)
+      : "memory");
+}
+
 // Arrive on the barrier when all previously issued tcgen05.mma of this thread completed.
 __device__ __forceinline__ void umma_commit(uint64_t* bar) {
   asm volatile("tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0];" ::"r"(
@@ -256,6 +269,31 @@ __device__ __forceinline__ void tmem_ld32(uint32_t taddr, float* v) {
   for (int i = 0; i < 32; ++i) v[i] = __uint_as_float(r[i]);
 }
 
+// 32 / 16 consecutive 32-bit columns of this thread's TMEM lane, from registers.
+// tmem_wait_st() must follow before the values are published to another thread.
+__device__ __forceinline__ void tmem_st32(uint32_t taddr, const uint32_t* v) {
+  asm volatile(
+      "tcgen05.st.sync.aligned.32x32b.x32.b32 [%0], "
+      "{%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15,%16,"
+      "%17,%18,%19,%20,%21,%22,%23,%24,%25,%26,%27,%28,%29,%30,%31,%32};" ::"r"(taddr),
+      "r"(v[0]), "r"(v[1]), "r"(v[2]), "r"(v[3]), "r"(v[4]), "r"(v[5]), "r"(v[6]), "r"(v[7]), "r"(v[8]),
+      "r"(v[9]), "r"(v[10]), "r"(v[11]), "r"(v[12]), "r"(v[13]), "r"(v[14]), "r"(v[15]), "r"(v[16]),
+      "r"(v[17]), "r"(v[18]), "r"(v[19]), "r"(v[20]), "r"(v[21]), "r"(v[22]), "r"(v[23]), "r"(v[24]),
+      "r"(v[25]), "r"(v[26]), "r"(v[27]), "r"(v[28]), "r"(v[29]), "r"(v[30]), "r"(v[31])
+      : "memory");
+}
+
+__device__ __forceinline__ void tmem_st16(uint32_t taddr, const uint32_t* v) {
+  asm volatile(
+      "tcgen05.st.sync.aligned.32x32b.x16.b32 [%0], "
+      "{%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15,%16};" ::"r"(taddr),
+      "r"(v[0]), "r"(v[1]), "r"(v[2]), "r"(v[3]), "r"(v[4]), "r"(v[5]), "r"(v[6]), "r"(v[7]), "r"(v[8]),
+      "r"(v[9]), "r"(v[10]), "r"(v[11]), "r"(v[12]), "r"(v[13]), "r"(v[14]), "r"(v[15])
+      : "memory");
+}
+
+__device__ __forceinline__ void tmem_wait_st() { asm volatile("tcgen05.wait::st.sync.aligned;" ::: "memory"); }
+
 // ----------------------------------------------------------------------------
 // bf16
 // ----------------------------------------------------------------------------
@@ -280,12 +318,25 @@ __device__ __forceinline__ uint32_t pack_f16x2(float lo, float hi) {
 
 __device__ __forceinline__ float f16_to_f32(uint16_t h) { return __half2float(__ushort_as_half(h)); }
 
+// bf16 bits -> fp16 bits, rounding to nearest even. Where the value is an fp16
+// normal number it is exact (8 significant bits fit in 11) and done with integer
+// arithmetic alone, by re-biasing the exponent from 127 to 15; zeros keep their
+// sign; everything else (fp16 subnormals, overflow, inf, nan) takes the
+// hardware conversion. Keeping the common case off the conversion pipe matters
+// where that pipe is busy with transcendentals in other warps.
+__device__ __forceinline__ uint32_t bf16_to_f16_bits(uint32_t b) {
+  const uint32_t mag = b & 0x7FFFu;
+  if ((mag >> 7) - 113u <= 29u) return (b & 0x8000u) | ((mag << 3) - (112u << 10));
+  if (mag == 0u) return b & 0x8000u;
+  return __half_as_ushort(__float2half_rn(__uint_as_float(b << 16)));
+}
+
 // 8 bf16 values (one 16-byte chunk) -> 8 fp16 values (exact within fp16 range).
 __device__ __forceinline__ uint4 bf16x8_to_f16x8(uint4 v) {
   const uint32_t w[4] = {v.x, v.y, v.z, v.w};
   uint32_t o[4];
 #pragma unroll
-  for (int i = 0; i < 4; ++i) o[i] = pack_f16x2(__uint_as_float(w[i] << 16), __uint_as_float(w[i] & 0xFFFF0000u));
+  for (int i = 0; i < 4; ++i) o[i] = bf16_to_f16_bits(w[i] & 0xFFFFu) | (bf16_to_f16_bits(w[i] >> 16) << 16);
   return make_uint4(o[0], o[1], o[2], o[3]);
 }
 
