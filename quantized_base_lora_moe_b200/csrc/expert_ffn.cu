@@ -14,22 +14,28 @@
 // columns instead of a padded 128-row tile.
 //
 // Work unit = (expert e, 128-feature tile, block of up to 128 routed rows);
-// units are ordered (expert, tile, block) over a persistent grid. Per CTA
-// (1 per SM, 576 threads):
+// units are ordered (expert, tile, block) over a persistent grid. One K stage
+// is 8 tcgen05.mma of 128 x N x 16 (GATEUP: 64 K for gate and for up; DOWN:
+// 128 K), so that one barrier round trip is amortised over 8 MMAs. Per CTA
+// (1 per SM, 832 threads):
 //   warps 0-3   epilogue (TMEM lanes 32w..32w+31 = features of the tile)
 //   warp  4     TMEM allocation + one thread issuing tcgen05.mma
-//   warp  5     TMA producer of the int4 code / bf16 scale ring
+//   warp  5     TMA producer of the int4 code / bf16 scale ring (the code tiles
+//               come 32B- / 64B-swizzled, so the row reads below are free of
+//               bank conflicts)
 //   warps 6-9   token producer: cp.async row gathers (rows picked by perm_token)
 //               or TMA tiles of contiguous rows, and the rank-space rows
-//   warps 10-17 weight producer: int4 -> fp16 into TMEM, LoRA B rows
-// TMEM (512 columns): accumulators in [0, 256), weight stages in [256, 512).
-//   GATEUP: one accumulator (gate cols [0,128), up [128,256)), 4 weight stages
-//           of 64 columns (gate 32 | up 32). The epilogue drains G and U as
-//           fp16 into [token][feature] shared-memory tiles, hands TMEM back, and
+//   warps 10-25 weight producer: each thread dequantises 32 K values of one
+//               weight row (int4 -> fp16) into TMEM; LoRA B rows
+// TMEM (512 columns): accumulators in [0, 256), 4 weight stages of 64 columns
+// in [256, 512).
+//   GATEUP: one accumulator (gate cols [0,128), up [128,256)); a weight stage
+//           holds gate 32 | up 32 columns. The epilogue drains G and U as fp16
+//           into [token][feature] shared-memory tiles, hands TMEM back, and
 //           finishes SwiGLU + 16-byte row stores while the next unit runs.
-//   DOWN:   two accumulators of 128 columns, 8 weight stages of 32 columns;
-//           32-token chunks go out through a double-buffered [token][feature]
-//           tile, so that every global store is a 16-byte piece of a row.
+//   DOWN:   two accumulators of 128 columns; 32-token chunks go out through a
+//           double-buffered [token][feature] tile, so that every global store is
+//           a 16-byte piece of a row.
 // Every wait is bounded (tqp_device.cuh); no TMA multicast is used.
 #include <cstdint>
 #include <cuda.h>
@@ -43,25 +49,28 @@
 namespace tqp {
 namespace tmem_ffn {
 
-constexpr int kThreads = 576;
-constexpr int kXStageBytes = 16384;   // 128 token rows x 64 K x 2 B
+constexpr int kWWarp0 = 10;           // first weight-producer warp
+constexpr int kWWarps = 16;
+constexpr int kThreads = (kWWarp0 + kWWarps) * 32;
 constexpr int kQStages = 8;
-constexpr int kQStageBytes = 9216;    // up to 2 x 4096 B of codes + 1024 B of scales
+constexpr int kQStageBytes = 9216;    // up to 8192 B of codes + 1024 B of scales
 constexpr int kTRow = 272;            // staging row: one token's 128 features in fp16, +16 B against bank conflicts
 constexpr uint32_t kWBase = 256;      // first TMEM column of the weight stages
+constexpr int kWStages = 4;
+constexpr uint32_t kWCols = 64;       // TMEM columns per weight stage
 
 template <int MODE> struct Cfg;
-template <> struct Cfg<GATEUP> {
-  static constexpr int kXStages = 5, kWStages = 4, kWCols = 64, kStaging = 2 * 128 * kTRow;   // G and U tiles
+template <> struct Cfg<GATEUP> {      // K stage 64: 128 token rows x 128 B
+  static constexpr int kK = 64, kXStageBytes = 16384, kXStages = 5, kStaging = 2 * 128 * kTRow;
 };
-template <> struct Cfg<DOWN> {
-  static constexpr int kXStages = 8, kWStages = 8, kWCols = 32, kStaging = 2 * 32 * kTRow;    // 2 chunk buffers
+template <> struct Cfg<DOWN> {        // K stage 128: two 64-wide swizzled sub-tiles
+  static constexpr int kK = 128, kXStageBytes = 32768, kXStages = 4, kStaging = 2 * 32 * kTRow;
 };
 
 struct Ctl {
   uint64_t x_full[8], x_empty[8];
   uint64_t q_full[kQStages], q_empty[kQStages];
-  uint64_t w_full[8], w_empty[8];
+  uint64_t w_full[kWStages], w_empty[kWStages];
   uint64_t acc_full[2], acc_empty[2];
   uint64_t drain;
   uint64_t epi;
@@ -71,7 +80,7 @@ struct Ctl {
 
 template <int MODE>
 constexpr size_t smem_bytes() {
-  return 1024 + size_t(Cfg<MODE>::kXStages) * kXStageBytes + size_t(kQStages) * kQStageBytes +
+  return 1024 + size_t(Cfg<MODE>::kXStages) * Cfg<MODE>::kXStageBytes + size_t(kQStages) * kQStageBytes +
          size_t(Cfg<MODE>::kStaging) + sizeof(Ctl);
 }
 static_assert(smem_bytes<GATEUP>() <= 232448 && smem_bytes<DOWN>() <= 232448, "shared memory budget");
@@ -89,14 +98,15 @@ struct EpiSync {
   }
 };
 
-// 32 tokens x this lane's feature (16 words of fp16 pairs, word j = tokens 2j,
-// 2j+1) into a [token][feature] tile: lane pairs trade halves so that each lane
-// writes two adjacent features of one token as one 32-bit word.
+// 2*NW tokens x this lane's feature (NW words of fp16 pairs, word j = tokens
+// t0+2j, t0+2j+1) into a [token][feature] tile: lane pairs trade halves so that
+// each lane writes two adjacent features of one token as one 32-bit word.
+template <int NW>
 __device__ __forceinline__ void stage_tokens(uint8_t* tile, int t0, int row, const uint32_t* w) {
   const bool odd = (threadIdx.x & 1) != 0;
   uint8_t* colp = tile + (row & ~1) * 2;
 #pragma unroll
-  for (int j = 0; j < 16; ++j) {
+  for (int j = 0; j < NW; ++j) {
     const uint32_t other = __shfl_xor_sync(0xFFFFFFFFu, w[j], 1);
     const uint32_t v = odd ? __byte_perm(other, w[j], 0x7632) : __byte_perm(w[j], other, 0x5410);
     *reinterpret_cast<uint32_t*>(colp + (t0 + 2 * j + (odd ? 1 : 0)) * kTRow) = v;
@@ -123,13 +133,13 @@ __global__ void __launch_bounds__(kThreads, 1)
                       const __grid_constant__ CUtensorMap tq1, const __grid_constant__ CUtensorMap ts0,
                       const __grid_constant__ CUtensorMap ts1, const __grid_constant__ CUtensorMap th) {
   constexpr bool kGU = (MODE == GATEUP);
+  constexpr int kK = Cfg<MODE>::kK;
   constexpr int XS = Cfg<MODE>::kXStages;
-  constexpr int WS = Cfg<MODE>::kWStages;
-  constexpr uint32_t kWCols = Cfg<MODE>::kWCols;
+  constexpr int kXBytes = Cfg<MODE>::kXStageBytes;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   uint8_t* x_base = smem;
-  uint8_t* q_base = x_base + size_t(XS) * kXStageBytes;
+  uint8_t* q_base = x_base + size_t(XS) * kXBytes;
   uint8_t* staging = q_base + size_t(kQStages) * kQStageBytes;
   Ctl* ctl = reinterpret_cast<Ctl*>(staging + Cfg<MODE>::kStaging);
   volatile int* abort_flag = &ctl->abort_flag;
@@ -144,10 +154,10 @@ __global__ void __launch_bounds__(kThreads, 1)
     }
     for (int i = 0; i < kQStages; ++i) {
       mbar_init(&ctl->q_full[i], 1);
-      mbar_init(&ctl->q_empty[i], 256);
+      mbar_init(&ctl->q_empty[i], kWWarps * 32);
     }
-    for (int i = 0; i < WS; ++i) {
-      mbar_init(&ctl->w_full[i], 256);
+    for (int i = 0; i < kWStages; ++i) {
+      mbar_init(&ctl->w_full[i], kWWarps * 32);
       mbar_init(&ctl->w_empty[i], 1);
     }
     for (int i = 0; i < 2; ++i) {
@@ -179,7 +189,8 @@ __global__ void __launch_bounds__(kThreads, 1)
 
   const int nunits = total_units(a);
   const int nkb = a.nkb_main + a.nkb_lora;
-  const int ngrp = a.g >= 64 ? 1 : 64 / a.g;   // scale rows per 64-wide K-block
+  // scale rows per K stage (one per quantisation group it spans)
+  const int ngrp = a.g >= kK ? 1 : kK / a.g;
 
   if (warp < 4) {
     // ------------------------------------------------------------ epilogue
@@ -198,18 +209,18 @@ __global__ void __launch_bounds__(kThreads, 1)
         uint8_t* tu = staging + 128 * kTRow;
         // drain: G and U as fp16 into the [token][feature] tiles
 #pragma unroll 1
-        for (int c = 0; c < n16; c += 32) {
-          float gv[32], uv[32];
-          tmem_ld32(tl + c, gv);
-          tmem_ld32(tl + 128 + c, uv);
-          uint32_t gw[16], uw[16];
+        for (int c = 0; c < n16; c += 16) {
+          float gv[16], uv[16];
+          tmem_ld16(tl + c, gv);
+          tmem_ld16(tl + 128 + c, uv);
+          uint32_t gw[8], uw[8];
 #pragma unroll
-          for (int j = 0; j < 16; ++j) {
+          for (int j = 0; j < 8; ++j) {
             gw[j] = f32x2_to_f16x2(gv[2 * j], gv[2 * j + 1]);
             uw[j] = f32x2_to_f16x2(uv[2 * j], uv[2 * j + 1]);
           }
-          stage_tokens(tg, c, row, gw);
-          stage_tokens(tu, c, row, uw);
+          stage_tokens<8>(tg, c, row, gw);
+          stage_tokens<8>(tu, c, row, uw);
         }
         tc_fence_before();
         mbar_arrive(&ctl->acc_empty[0]);
@@ -240,19 +251,24 @@ __global__ void __launch_bounds__(kThreads, 1)
         bool stop = false;
 #pragma unroll 1
         for (int c = 0; c < n16; c += 32, ++chunk) {
-          float v[32];
-          tmem_ld32(tl + uint32_t(ab * 128 + c), v);
+          // consecutive chunks alternate between the two tiles; the barrier after a
+          // tile is written also orders every earlier read of the other tile
+          uint8_t* tile = staging + (chunk & 1) * (32 * kTRow);
+#pragma unroll
+          for (int hh = 0; hh < 2; ++hh) {
+            if (c + 16 * hh < n16) {
+              float v[16];
+              tmem_ld16(tl + uint32_t(ab * 128 + c + 16 * hh), v);
+              uint32_t pk[8];
+#pragma unroll
+              for (int j = 0; j < 8; ++j) pk[j] = f32x2_to_f16x2(v[2 * j], v[2 * j + 1]);
+              stage_tokens<8>(tile, 16 * hh, row, pk);
+            }
+          }
           if (c + 32 >= n16) {  // last read of this accumulator: hand it back before storing
             tc_fence_before();
             mbar_arrive(&ctl->acc_empty[ab]);
           }
-          uint32_t pk[16];
-#pragma unroll
-          for (int j = 0; j < 16; ++j) pk[j] = f32x2_to_f16x2(v[2 * j], v[2 * j + 1]);
-          // consecutive chunks alternate between the two tiles; the barrier after a
-          // tile is written also orders every earlier read of the other tile
-          uint8_t* tile = staging + (chunk & 1) * (32 * kTRow);
-          stage_tokens(tile, 0, row, pk);
           if (!es.sync(abort_flag, a.status)) { stop = true; break; }
           const int nt = min(32, un.rows - c);
           for (int p = threadIdx.x; p < nt * 16; p += 128) {
@@ -286,17 +302,29 @@ __global__ void __launch_bounds__(kThreads, 1)
             break;
           }
           tc_fence_after();
-          const int ksteps = (kb < a.nkb_lora) ? (min(64, a.lora_k - kb * 64) + 15) / 16 : 4;
-          const uint64_t bdesc = sdesc_k_sw128(smem_u32(x_base + size_t(rx.stage) * kXStageBytes));
+          const uint32_t xs = smem_u32(x_base + size_t(rx.stage) * kXBytes);
+          const uint64_t bdesc = sdesc_k_sw128(xs);
           const uint32_t wa = tmem_base + kWBase + uint32_t(rw.stage) * kWCols;
-          if (ksteps == 4) {
+          if (kb >= a.nkb_lora) {
+            if (kGU) {
 #pragma unroll
-            for (int kk = 0; kk < 4; ++kk) {
-              const uint32_t acc = (kb > 0 || kk > 0) ? 1u : 0u;
-              umma_f16_ts(dacc, wa + uint32_t(8 * kk), bdesc + uint64_t(2 * kk), idesc, acc);
-              if (kGU) umma_f16_ts(dacc + 128, wa + 32 + uint32_t(8 * kk), bdesc + uint64_t(2 * kk), idesc, acc);
+              for (int kk = 0; kk < 4; ++kk) {
+                const uint32_t acc = (kb > 0 || kk > 0) ? 1u : 0u;
+                umma_f16_ts(dacc, wa + uint32_t(8 * kk), bdesc + uint64_t(2 * kk), idesc, acc);
+                umma_f16_ts(dacc + 128, wa + 32 + uint32_t(8 * kk), bdesc + uint64_t(2 * kk), idesc, acc);
+              }
+            } else {
+              const uint64_t bdesc1 = sdesc_k_sw128(xs + 16384);
+#pragma unroll
+              for (int kk = 0; kk < 8; ++kk) {
+                const uint32_t acc = (kb > 0 || kk > 0) ? 1u : 0u;
+                umma_f16_ts(dacc, wa + uint32_t(8 * kk), (kk < 4 ? bdesc : bdesc1) + uint64_t(2 * (kk & 3)), idesc,
+                            acc);
+              }
             }
           } else {
+            // rank-space stage: only the first lora_k columns are live (within the first 64)
+            const int ksteps = (min(kK, a.lora_k - kb * kK) + 15) / 16;
             for (int kk = 0; kk < ksteps; ++kk) {
               const uint32_t acc = (kb > 0 || kk > 0) ? 1u : 0u;
               umma_f16_ts(dacc, wa + uint32_t(8 * kk), bdesc + uint64_t(2 * kk), idesc, acc);
@@ -306,7 +334,7 @@ __global__ void __launch_bounds__(kThreads, 1)
           umma_commit(&ctl->x_empty[rx.stage]);
           umma_commit(&ctl->w_empty[rw.stage]);
           rx.next<XS>();
-          rw.next<WS>();
+          rw.next<kWStages>();
         }
         if (!ok) break;
         umma_commit(&ctl->acc_full[ab]);
@@ -320,7 +348,9 @@ __global__ void __launch_bounds__(kThreads, 1)
     // ------------------------------------------------------------ TMA producer (int4 + scales)
     if (lane == 0) {
       Ring q;
-      const uint32_t bytes = kGU ? uint32_t(8192 + 512 * ngrp) : uint32_t(4096 + 256 * ngrp);
+      // GATEUP: gate codes [128 rows][32 B] | up codes | gate scales [ngrp][128] | up scales
+      // DOWN:   codes [128 rows][64 B] | scales [ngrp][128]
+      const uint32_t bytes = kGU ? uint32_t(8192 + 512 * ngrp) : uint32_t(8192 + 256 * ngrp);
       const int gpe = a.in_dim / a.g;  // scale rows per expert
       int issued = 0;
       uint32_t last_phase = 0;
@@ -333,15 +363,15 @@ __global__ void __launch_bounds__(kThreads, 1)
           if (!mbar_wait<64>(&ctl->q_empty[q.stage], q.phase ^ 1u, abort_flag, a.status)) { ok = false; break; }
           uint8_t* qs = q_base + size_t(q.stage) * kQStageBytes;
           uint64_t* bar = &ctl->q_full[q.stage];
-          const int srow = un.e * gpe + (km * 64) / a.g;
+          const int srow = un.e * gpe + (km * kK) / a.g;
           mbar_arrive_expect_tx(bar, bytes);
-          tma_load_2d(smem_u32(qs), &tq0, bar, km * 32, nrow0);
+          tma_load_2d(smem_u32(qs), &tq0, bar, km * (kK / 2), nrow0);
           if (kGU) {
-            tma_load_2d(smem_u32(qs + 4096), &tq1, bar, km * 32, nrow0);
+            tma_load_2d(smem_u32(qs + 4096), &tq1, bar, km * (kK / 2), nrow0);
             tma_load_2d(smem_u32(qs + 8192), &ts0, bar, un.nt * 128, srow);
             tma_load_2d(smem_u32(qs + 8192 + 256 * ngrp), &ts1, bar, un.nt * 128, srow);
           } else {
-            tma_load_2d(smem_u32(qs + 4096), &ts0, bar, un.nt * 128, srow);
+            tma_load_2d(smem_u32(qs + 8192), &ts0, bar, un.nt * 128, srow);
           }
           ++issued;
           last_stage = q.stage;
@@ -353,7 +383,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       // on an abort, wait (bounded) until the last issued stage has landed
       if (issued > 0 && *abort_flag) mbar_wait(&ctl->q_full[last_stage], last_phase, abort_flag, a.status);
     }
-  } else if (warp < 10) {
+  } else if (warp < kWWarp0) {
     // ------------------------------------------------------------ token producer
     const int tid = threadIdx.x - 6 * 32;  // 0..127 = token row of the tile
     Ring rx;
@@ -369,14 +399,15 @@ __global__ void __launch_bounds__(kThreads, 1)
       bool ok = true;
       for (int kb = 0; kb < nkb; ++kb) {
         if (!mbar_wait<64>(&ctl->x_empty[rx.stage], rx.phase ^ 1u, abort_flag, a.status)) { ok = false; break; }
-        const uint32_t st_u = smem_u32(x_base + size_t(rx.stage) * kXStageBytes);
+        const uint32_t st_u = smem_u32(x_base + size_t(rx.stage) * kXBytes);
         uint64_t* full = &ctl->x_full[rx.stage];
         if (kb < a.nkb_lora) {
-          // rank-space rows (s X[Ag|Au] or s H Ad), zero-filled past lora_k
+          // rank-space rows (s X[Ag|Au] or s H Ad) in the first 64-wide sub-tile,
+          // zero-filled past lora_k (lora_k <= 128, and <= 64 for DOWN)
           if (valid) {
 #pragma unroll
             for (int c = 0; c < 8; ++c) {
-              const int colk = kb * 64 + c * 8;
+              const int colk = kb * kK + c * 8;
               const bool in = colk < a.lora_k;
               cp_async16(st_u + sw128_offset(tid, c), lsrc + (in ? colk : 0), in ? 16u : 0u);
             }
@@ -392,8 +423,9 @@ __global__ void __launch_bounds__(kThreads, 1)
             }
             cp_async_arrive_noinc(full);
           } else if (tid == 0) {
-            mbar_arrive_expect_tx(full, uint32_t(kXStageBytes));
-            tma_load_2d(st_u, &th, full, km * 64, un.base);
+            mbar_arrive_expect_tx(full, uint32_t(kXBytes));
+            tma_load_2d(st_u, &th, full, km * 128, un.base);
+            tma_load_2d(st_u + 16384, &th, full, km * 128 + 64, un.base);
             pend_stage = rx.stage;
             pend_phase = rx.phase;
           } else {
@@ -409,10 +441,17 @@ __global__ void __launch_bounds__(kThreads, 1)
       mbar_wait(&ctl->x_full[pend_stage], pend_phase, abort_flag, a.status);
   } else {
     // ------------------------------------------------------------ weight producer
-    const int wi = warp - 10;                 // 0..7
+    // thread = 32 consecutive K values (4 int4 words) of one weight row per stage
+    const int wi = warp - kWWarp0;            // 0..15
     const int lrow = 32 * (warp & 3) + lane;  // TMEM lane = feature within the tile
-    const int part = wi >> 2;                 // GATEUP: 0 gate / 1 up rows; DOWN: K half
-    const uint32_t tw = tmem_base + (uint32_t(32 * (warp & 3)) << 16) + kWBase + uint32_t(part * (kGU ? 32 : 16));
+    const int mat = kGU ? (wi >> 3) : 0;      // GATEUP: 0 gate / 1 up rows
+    const int kq = kGU ? ((wi >> 2) & 1) : (wi >> 2);   // 32-wide K slice within the stage
+    const uint32_t tw = tmem_base + (uint32_t(32 * (warp & 3)) << 16) + kWBase + uint32_t(mat * 32 + kq * 16);
+    // code slice inside a stage (rows of kK/2 bytes, TMA-swizzled at 32 B / 64 B)
+    const int code_off = kGU ? (mat * 4096 + lrow * 32 + ((kq ^ ((lrow >> 2) & 1)) << 4))
+                             : (lrow * 64 + ((kq ^ ((lrow >> 1) & 3)) << 4));
+    const int grp = (ngrp == 1) ? 0 : (32 * kq) / a.g;   // this slice's quantisation group
+    const int scale_off = 8192 + (kGU ? mat * 256 * ngrp : 0) + (grp * 128 + lrow) * 2;
     Ring rw, q;
     for (int u = blockIdx.x; u < nunits; u += gridDim.x) {
       const Unit un = decode_unit(a, u);
@@ -421,59 +460,43 @@ __global__ void __launch_bounds__(kThreads, 1)
       for (int kb = 0; kb < nkb; ++kb) {
         if (!mbar_wait(&ctl->w_empty[rw.stage], rw.phase ^ 1u, abort_flag, a.status)) { ok = false; break; }
         tc_fence_after();
-        uint32_t v[kGU ? 32 : 16];
-        constexpr int kChunks = kGU ? 8 : 4;   // 8 K values per chunk
+        uint32_t v[16];
         if (kb < a.nkb_lora) {
           // LoRA B rows as fp16: gate rows hold Bg in K' [0, r), up rows Bu in [r, 2r)
 #pragma unroll
-          for (int c = 0; c < kChunks; ++c) {
-            const int colk = kb * 64 + (kGU ? c : part * 4 + c) * 8;
-            const int src = (kGU && part == 1) ? colk - a.r : colk;
+          for (int c = 0; c < 4; ++c) {
+            const int colk = kb * kK + kq * 32 + c * 8;
+            const int src = (kGU && mat == 1) ? colk - a.r : colk;
             uint4 w4 = make_uint4(0, 0, 0, 0);
             if (src >= 0 && src < a.r) {
-              const uint16_t* bsrc = (kGU && part == 1) ? a.b1 : a.b0;
-              w4 = bf16x8_to_f16x8(__ldg(reinterpret_cast<const uint4*>(bsrc + (size_t(un.e) * a.out_dim + n) * a.r + src)));
+              const uint16_t* bsrc = (kGU && mat == 1) ? a.b1 : a.b0;
+              w4 = bf16x8_to_f16x8(
+                  __ldg(reinterpret_cast<const uint4*>(bsrc + (size_t(un.e) * a.out_dim + n) * a.r + src)));
             }
             v[4 * c] = w4.x; v[4 * c + 1] = w4.y; v[4 * c + 2] = w4.z; v[4 * c + 3] = w4.w;
           }
         } else {
           if (!mbar_wait(&ctl->q_full[q.stage], q.phase, abort_flag, a.status)) { ok = false; break; }
           const uint8_t* qs = q_base + size_t(q.stage) * kQStageBytes;
-          uint32_t wd[kChunks];
-          uint32_t s_lo, s_hi;
-          if (kGU) {
-            const uint4 c0 = *reinterpret_cast<const uint4*>(qs + part * 4096 + lrow * 32);
-            const uint4 c1 = *reinterpret_cast<const uint4*>(qs + part * 4096 + lrow * 32 + 16);
-            wd[0] = c0.x; wd[1] = c0.y; wd[2] = c0.z; wd[3] = c0.w;
-            wd[4] = c1.x; wd[5] = c1.y; wd[6] = c1.z; wd[7] = c1.w;
-            const uint16_t* sc = reinterpret_cast<const uint16_t*>(qs + 8192 + part * 256 * ngrp);
-            s_lo = scale_pair(sc[lrow]);
-            s_hi = (ngrp == 2) ? scale_pair(sc[128 + lrow]) : s_lo;
-          } else {
-            const uint4 c0 = *reinterpret_cast<const uint4*>(qs + lrow * 32 + part * 16);
-            wd[0] = c0.x; wd[1] = c0.y; wd[2] = c0.z; wd[3] = c0.w;
-            const uint16_t* sc = reinterpret_cast<const uint16_t*>(qs + 4096);
-            s_lo = scale_pair(sc[(ngrp == 2 ? part : 0) * 128 + lrow]);
-            s_hi = s_lo;
-          }
-          // the code slot goes back once its values are in registers, behind a proxy
-          // fence (its next fill is an async-proxy TMA write)
+          const uint4 wd = *reinterpret_cast<const uint4*>(qs + code_off);
+          const uint32_t s2 = scale_pair(*reinterpret_cast<const uint16_t*>(qs + scale_off));
+          const uint4 d0 = dequant_word(wd.x, s2), d1 = dequant_word(wd.y, s2);
+          const uint4 d2 = dequant_word(wd.z, s2), d3 = dequant_word(wd.w, s2);
+          // the code slot's values have been consumed; its next fill is an
+          // async-proxy TMA write, hence the proxy fence before handing it back
           fence_proxy_async_smem();
           mbar_arrive(&ctl->q_empty[q.stage]);
           q.next<kQStages>();
-#pragma unroll
-          for (int c = 0; c < kChunks; ++c) {
-            const uint4 d4 = dequant_word(wd[c], (kGU && c >= 4) ? s_hi : s_lo);
-            v[4 * c] = d4.x; v[4 * c + 1] = d4.y; v[4 * c + 2] = d4.z; v[4 * c + 3] = d4.w;
-          }
+          v[0] = d0.x; v[1] = d0.y; v[2] = d0.z; v[3] = d0.w;
+          v[4] = d1.x; v[5] = d1.y; v[6] = d1.z; v[7] = d1.w;
+          v[8] = d2.x; v[9] = d2.y; v[10] = d2.z; v[11] = d2.w;
+          v[12] = d3.x; v[13] = d3.y; v[14] = d3.z; v[15] = d3.w;
         }
-        const uint32_t taddr = tw + uint32_t(rw.stage) * kWCols;
-        if (kGU) tmem_st32(taddr, v);
-        else tmem_st16(taddr, v);
+        tmem_st16(tw + uint32_t(rw.stage) * kWCols, v);
         tmem_wait_st();
         tc_fence_before();
         mbar_arrive(&ctl->w_full[rw.stage]);
-        rw.next<WS>();
+        rw.next<kWStages>();
       }
       if (!ok) break;
     }

@@ -678,8 +678,9 @@ static PFN_cuTensorMapEncodeTiled_v12000 encode_fn() {
   return fn;
 }
 
+// 2-D tensor map; swizzle = 0 (none), 32, 64 or 128 bytes.
 static bool make_map(CUtensorMap* m, CUtensorMapDataType dt, const void* ptr, uint64_t inner, uint64_t outer,
-                     uint64_t row_bytes, uint32_t box_inner, uint32_t box_outer, bool sw128 = false) {
+                     uint64_t row_bytes, uint32_t box_inner, uint32_t box_outer, int swizzle = 0) {
   auto fn = encode_fn();
   if (!fn) return false;
   cuuint64_t dims[2] = {inner, outer};
@@ -687,13 +688,17 @@ static bool make_map(CUtensorMap* m, CUtensorMapDataType dt, const void* ptr, ui
   cuuint32_t box[2] = {box_inner, box_outer};
   cuuint32_t estr[2] = {1, 1};
   return fn(m, dt, 2, const_cast<void*>(ptr), dims, strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
-            sw128 ? CU_TENSOR_MAP_SWIZZLE_128B : CU_TENSOR_MAP_SWIZZLE_NONE, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+            swizzle == 128 ? CU_TENSOR_MAP_SWIZZLE_128B
+            : swizzle == 64 ? CU_TENSOR_MAP_SWIZZLE_64B
+            : swizzle == 32 ? CU_TENSOR_MAP_SWIZZLE_32B
+                            : CU_TENSOR_MAP_SWIZZLE_NONE,
+            CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
             CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
 // 128B-swizzled K-major tile map of a row-major 16-bit matrix [rows][cols]: box {64, box_rows}.
 static bool make_tile_map(CUtensorMap* m, const void* ptr, uint64_t rows, uint64_t cols, uint32_t box_rows) {
-  return make_map(m, CU_TENSOR_MAP_DATA_TYPE_UINT16, ptr, cols, rows, cols * 2, 64, box_rows, true);
+  return make_map(m, CU_TENSOR_MAP_DATA_TYPE_UINT16, ptr, cols, rows, cols * 2, 64, box_rows, 128);
 }
 
 int num_sms() {
@@ -832,12 +837,16 @@ int launch_grouped_ffn(const uint16_t* x, int T, const int32_t* offsets, const i
       return TQP_ERR_CUDA;
     if ((rc = run_gemm<LORA_XA>(a, mp, mb_upper, s)) != TQP_OK) return rc;
   }
+  // The forward projections run with the weights in TMEM (expert_ffn.cu) when the
+  // hidden width is a multiple of 128 (its K stages and feature tiles), else on
+  // the shared-memory engine above.
+  const bool tm = (f % 128 == 0);
   {  // H = silu(G) * U
     GemmArgs a = base;
     a.nkb_main = d / 64;
     a.nkb_lora = r > 0 ? (2 * r + 63) / 64 : 0;
     a.lora_k = 2 * r;
-    a.ntile = (f % 128 == 0) ? 256 : 128;
+    a.ntile = tm ? 256 : 128;
     a.n_tiles = f / (a.ntile / 2);
     a.in_dim = d;
     a.out_dim = f;
@@ -854,19 +863,19 @@ int launch_grouped_ffn(const uint16_t* x, int T, const int32_t* offsets, const i
     a.f_dim = f;
     const int ngrp = w->group >= 64 ? 1 : 64 / w->group;
     const uint32_t rows_box = uint32_t(a.ntile / 2);
+    const int csw = tm ? 32 : 0;   // 32-byte code rows, swizzled for conflict-free row reads
     Maps mp{};
     bool ok = make_map(&mp.m[TQ0], CU_TENSOR_MAP_DATA_TYPE_UINT8, w->wq[0], d / 2, uint64_t(w->E) * f, d / 2, 32,
-                       rows_box) &&
+                       rows_box, csw) &&
               make_map(&mp.m[TQ1], CU_TENSOR_MAP_DATA_TYPE_UINT8, w->wq[1], d / 2, uint64_t(w->E) * f, d / 2, 32,
-                       rows_box) &&
+                       rows_box, csw) &&
               make_map(&mp.m[TS0], CU_TENSOR_MAP_DATA_TYPE_UINT16, w->wscale[0], f, uint64_t(w->E) * (d / w->group),
                        uint64_t(f) * 2, rows_box, ngrp) &&
               make_map(&mp.m[TS1], CU_TENSOR_MAP_DATA_TYPE_UINT16, w->wscale[1], f, uint64_t(w->E) * (d / w->group),
                        uint64_t(f) * 2, rows_box, ngrp);
     if (!ok) return TQP_ERR_CUDA;
-    // 128-feature tiles run with the weights in TMEM (expert_ffn.cu)
-    rc = (f % 128 == 0) ? run_expert_ffn(GATEUP, a, mp, mb_upper * a.n_tiles, s)
-                        : run_gemm<GATEUP>(a, mp, mb_upper * a.n_tiles, s);
+    rc = tm ? run_expert_ffn(GATEUP, a, mp, mb_upper * a.n_tiles, s)
+            : run_gemm<GATEUP>(a, mp, mb_upper * a.n_tiles, s);
     if (rc != TQP_OK) return rc;
   }
   if (r > 0) {  // ha = s * H Ad
@@ -885,11 +894,12 @@ int launch_grouped_ffn(const uint16_t* x, int T, const int32_t* offsets, const i
   }
   {  // O = H Wd^T + (s H Ad) Bd
     GemmArgs a = base;
-    a.nkb_main = f / 64;
-    a.nkb_lora = r > 0 ? (r + 63) / 64 : 0;
+    const int kst = tm ? 128 : 64;   // K stage
+    a.nkb_main = f / kst;
+    a.nkb_lora = r > 0 ? (r + kst - 1) / kst : 0;
     a.lora_k = r;
-    a.ntile = 128;
-    a.n_tiles = d / 128;
+    a.ntile = tm ? 128 : ((d % 256 == 0) ? 256 : 128);
+    a.n_tiles = d / a.ntile;
     a.in_dim = f;
     a.out_dim = d;
     a.a_lora = fb.ha;
@@ -898,15 +908,16 @@ int launch_grouped_ffn(const uint16_t* x, int T, const int32_t* offsets, const i
     a.out = out_perm;
     a.out_ld = d;
     a.n_valid = d;
-    const int ngrp = w->group >= 64 ? 1 : 64 / w->group;
+    const int ngrp = w->group >= kst ? 1 : kst / w->group;
     Maps mp{};
     bool ok = make_tile_map(&mp.m[TA], h, uint64_t(A), uint64_t(f), 128) &&
-              make_map(&mp.m[TQ0], CU_TENSOR_MAP_DATA_TYPE_UINT8, w->wq[2], f / 2, uint64_t(w->E) * d, f / 2, 32,
-                       uint32_t(a.ntile)) &&
+              make_map(&mp.m[TQ0], CU_TENSOR_MAP_DATA_TYPE_UINT8, w->wq[2], f / 2, uint64_t(w->E) * d, f / 2,
+                       uint32_t(kst / 2), uint32_t(a.ntile), tm ? 64 : 0) &&
               make_map(&mp.m[TS0], CU_TENSOR_MAP_DATA_TYPE_UINT16, w->wscale[2], d, uint64_t(w->E) * (f / w->group),
                        uint64_t(d) * 2, uint32_t(a.ntile), ngrp);
     if (!ok) return TQP_ERR_CUDA;
-    if ((rc = run_expert_ffn(DOWN, a, mp, mb_upper * a.n_tiles, s)) != TQP_OK) return rc;
+    rc = tm ? run_expert_ffn(DOWN, a, mp, mb_upper * a.n_tiles, s) : run_gemm<DOWN>(a, mp, mb_upper * a.n_tiles, s);
+    if (rc != TQP_OK) return rc;
   }
   return TQP_OK;
 }

@@ -28,7 +28,11 @@ if torch.cuda.is_available():
 RAGGED = synth.LayerConfig("ragged", T=300, d=256, E=10, k=3, f=192, g=64, r=16)
 ONE = synth.LayerConfig("one", T=37, d=128, E=1, k=1, f=64, g=32, r=8)
 ALLK = synth.LayerConfig("allk", T=50, d=128, E=4, k=4, f=128, g=128, r=0)
-SMALL_CFGS = [synth.TINY, RAGGED, ONE, ALLK, synth.MID]
+# group 256 (one scale row spans two 128-wide K stages of the down projection) and
+# the largest rank (the gate/up rank-space contraction spans two 64-wide stages)
+G256 = synth.LayerConfig("g256", T=200, d=256, E=6, k=2, f=256, g=256, r=8)
+R64 = synth.LayerConfig("r64", T=150, d=256, E=5, k=2, f=256, g=64, r=64)
+SMALL_CFGS = [synth.TINY, RAGGED, ONE, ALLK, G256, R64, synth.MID]
 TOL = 2e-2
 # The router's products are exact (bf16 x times an exact 3-part bf16 split of
 # the fp32 weights); its error is the tensor cores' fp32 accumulation, at most
