@@ -385,17 +385,25 @@ __global__ void __launch_bounds__(kThreads, 1)
     }
   } else if (warp < kWWarp0) {
     // ------------------------------------------------------------ token producer
-    const int tid = threadIdx.x - 6 * 32;  // 0..127 = token row of the tile
+    // Row gathers are spread so that 8 consecutive lanes copy the 8 16-byte
+    // chunks of one 128-byte row piece (one coalesced request per row piece):
+    // thread tid covers chunk tid % 8 of rows tid / 8 + 16 j, j = 0..7.
+    const int tid = threadIdx.x - 6 * 32;  // 0..127
+    const int chunk = tid & 7;
+    const int row0 = tid >> 3;             // 0..15
     Ring rx;
     int pend_stage = -1;
     uint32_t pend_phase = 0;
     for (int u = blockIdx.x; u < nunits; u += gridDim.x) {
       const Unit un = decode_unit(a, u);
-      const bool valid = tid < un.rows;
-      const int grow = un.base + (valid ? tid : 0);
-      const uint16_t* src = nullptr;
-      if (kGU) src = a.a_src + size_t(valid ? __ldg(a.perm_token + grow) : 0) * a.a_ld;
-      const uint16_t* lsrc = a.a_lora ? a.a_lora + size_t(grow) * a.lora_ld : nullptr;
+      // source rows of this thread's 8 tile rows (token rows for the gathers,
+      // routed rows for the rank-space operand)
+      int tok[8];
+#pragma unroll
+      for (int j = 0; j < 8; ++j) {
+        const int r = row0 + 16 * j;
+        tok[j] = (kGU && r < un.rows) ? __ldg(a.perm_token + un.base + r) : 0;
+      }
       bool ok = true;
       for (int kb = 0; kb < nkb; ++kb) {
         if (!mbar_wait<64>(&ctl->x_empty[rx.stage], rx.phase ^ 1u, abort_flag, a.status)) { ok = false; break; }
@@ -404,22 +412,24 @@ __global__ void __launch_bounds__(kThreads, 1)
         if (kb < a.nkb_lora) {
           // rank-space rows (s X[Ag|Au] or s H Ad) in the first 64-wide sub-tile,
           // zero-filled past lora_k (lora_k <= 128, and <= 64 for DOWN)
-          if (valid) {
+          const int colk = kb * kK + chunk * 8;
+          const bool in = colk < a.lora_k;
 #pragma unroll
-            for (int c = 0; c < 8; ++c) {
-              const int colk = kb * kK + c * 8;
-              const bool in = colk < a.lora_k;
-              cp_async16(st_u + sw128_offset(tid, c), lsrc + (in ? colk : 0), in ? 16u : 0u);
-            }
+          for (int j = 0; j < 8; ++j) {
+            const int r = row0 + 16 * j;
+            if (r < un.rows)
+              cp_async16(st_u + sw128_offset(r, chunk), a.a_lora + size_t(un.base + r) * a.lora_ld + (in ? colk : 0),
+                         in ? 16u : 0u);
           }
           cp_async_arrive_noinc(full);
         } else {
           const int km = kb - a.nkb_lora;
           if (kGU) {
-            if (valid) {
-              const uint16_t* p = src + km * 64;
 #pragma unroll
-              for (int c = 0; c < 8; ++c) cp_async16(st_u + sw128_offset(tid, c), p + c * 8, 16);
+            for (int j = 0; j < 8; ++j) {
+              const int r = row0 + 16 * j;
+              if (r < un.rows)
+                cp_async16(st_u + sw128_offset(r, chunk), a.a_src + size_t(tok[j]) * a.a_ld + km * 64 + chunk * 8, 16);
             }
             cp_async_arrive_noinc(full);
           } else if (tid == 0) {
@@ -457,6 +467,13 @@ __global__ void __launch_bounds__(kThreads, 1)
       const Unit un = decode_unit(a, u);
       const int n = un.nt * 128 + lrow;     // output feature
       bool ok = true;
+      if (a.nkb_lora > 0 && kq == 0 && u + int(gridDim.x) < nunits) {
+        // the next unit's LoRA B row into L2 (its rank-space stage comes first)
+        const Unit nx = decode_unit(a, u + gridDim.x);
+        const uint16_t* bsrc = (kGU && mat == 1) ? a.b1 : a.b0;
+        const uint16_t* row = bsrc + (size_t(nx.e) * a.out_dim + nx.nt * 128 + lrow) * a.r;
+        for (int off = 0; off < a.r; off += 64) prefetch_l2(row + off);
+      }
       for (int kb = 0; kb < nkb; ++kb) {
         if (!mbar_wait(&ctl->w_empty[rw.stage], rw.phase ^ 1u, abort_flag, a.status)) { ok = false; break; }
         tc_fence_after();

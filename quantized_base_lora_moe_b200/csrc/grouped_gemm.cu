@@ -366,7 +366,12 @@ __global__ void __launch_bounds__(kThreads, 1)
     }
   } else if (warp < 10) {
     // ------------------------------------------------------------ A producer
-    const int tid = threadIdx.x - 6 * 32;  // 0..127 = tile row
+    // Row gathers are spread so that 8 consecutive lanes copy the 8 16-byte
+    // chunks of one 128-byte row piece: thread tid covers chunk tid % 8 of rows
+    // tid / 8 + 16 j, j = 0..7.
+    const int tid = threadIdx.x - 6 * 32;  // 0..127
+    const int chunk = tid & 7;
+    const int row0 = tid >> 3;
     Ring ra, rb;
     const uint32_t a_bytes = uint32_t(kAStageBytes);
     uint32_t b_bytes = 0;
@@ -377,14 +382,12 @@ __global__ void __launch_bounds__(kThreads, 1)
     uint32_t pend_phase = 0;
     for (int u = blockIdx.x; u < nunits; u += gridDim.x) {
       const Unit un = decode_unit(a, u);
-      const bool valid = tid < un.rows;
-      const int grow = un.base + (valid ? tid : 0);
-      const uint16_t* src = nullptr;
-      if (!kATma) {
-        const int srow = valid ? __ldg(a.perm_token + grow) : 0;
-        src = a.a_src + size_t(srow) * a.a_ld;
+      int srow[8];   // gathered source rows of this thread's 8 tile rows
+#pragma unroll
+      for (int j = 0; j < 8; ++j) {
+        const int r = row0 + 16 * j;
+        srow[j] = (!kATma && r < un.rows) ? __ldg(a.perm_token + un.base + r) : 0;
       }
-      const uint16_t* lsrc = a.a_lora ? a.a_lora + size_t(grow) * a.lora_ld : nullptr;
       bool ok = true;
       for (int kb = 0; kb < nkb; ++kb) {
         if (!mbar_wait<64>(&ctl->a_empty[ra.stage], ra.phase ^ 1u, abort_flag, a.status)) { ok = false; break; }
@@ -392,13 +395,14 @@ __global__ void __launch_bounds__(kThreads, 1)
         uint64_t* full = &ctl->a_full[ra.stage];
         if (kb < a.nkb_lora) {
           // rank-space A tile: s*xA / s*hA / dhA / dxa rows, zero-filled past lora_k
-          if (valid) {
+          const int col = kb * 64 + chunk * 8;
+          const bool in = col < a.lora_k;
 #pragma unroll
-            for (int c = 0; c < 8; ++c) {
-              const int col = kb * 64 + c * 8;
-              const bool in = col < a.lora_k;
-              cp_async16(st_u + sw128_offset(tid, c), lsrc + (in ? col : 0), in ? 16u : 0u);
-            }
+          for (int j = 0; j < 8; ++j) {
+            const int r = row0 + 16 * j;
+            if (r < un.rows)
+              cp_async16(st_u + sw128_offset(r, chunk), a.a_lora + size_t(un.base + r) * a.lora_ld + (in ? col : 0),
+                         in ? 16u : 0u);
           }
           cp_async_arrive_noinc(full);
         } else {
@@ -430,10 +434,11 @@ __global__ void __launch_bounds__(kThreads, 1)
               mbar_arrive(full);
             }
           } else {
-            if (valid) {
-              const uint16_t* p = src + km * 64;
 #pragma unroll
-              for (int c = 0; c < 8; ++c) cp_async16(st_u + sw128_offset(tid, c), p + c * 8, 16);
+            for (int j = 0; j < 8; ++j) {
+              const int r = row0 + 16 * j;
+              if (r < un.rows)
+                cp_async16(st_u + sw128_offset(r, chunk), a.a_src + size_t(srow[j]) * a.a_ld + kcol + chunk * 8, 16);
             }
             cp_async_arrive_noinc(full);
           }
