@@ -175,25 +175,46 @@ int moe_permute_noalloc(const int32_t* ids, int T, int E, int k, int32_t* offset
  * tqp_grouped_ffn: the routed experts ("Train low-rank adapters per expert"
  * over "Quantize base expert weights", Pattern 3). For each expert e and each
  * of its rows (row r holds token perm_token[r]):
- *   G = X Wg^T + s (X Ag) Bg ;  U = X Wu^T + s (X Au) Bu ;  H = bf16(silu(G) * U)
- *   O = bf16(H Wd^T + s (H Ad) Bd)
- * with the int4 base dequantised in shared memory and all contractions on the
- * tensor cores (bf16 x bf16 -> fp32). X A and H A are rounded to bf16.
+ *   G = X Wg^T + s (X Ag) Bg ;  U = X Wu^T + s (X Au) Bu ;  H = fp16(silu(G) * U)
+ *   O = fp16(H Wd^T + s (H Ad) Bd)
+ * The int4 base is dequantised exactly to fp16 (q * scale) and every
+ * contraction runs on the tensor cores (fp16 x fp16 -> fp32); the adapter
+ * products s X A and s H A are kept in fp16.
  *   x [T][d] bf16 (tokens, gathered through perm_token); offsets [E+1];
- *   h [T*k][ffn] bf16 output (permuted row order); out_perm [T*k][d] bf16 output.
- *   ws: tqp_grouped_ffn_workspace_size.
+ *   h [T*k][ffn] fp16 output (permuted row order; kept for the backward);
+ *   out_perm [T*k][d] fp16 output (permuted row order).
+ *   ws: tqp_grouped_ffn_workspace_size. Errors: as the conventions above;
+ *   x values outside the fp16 range raise TQP_STATUS_NONFINITE.
+ *
+ * tqp_grouped_ffn_part: the same computation issued one part at a time, for a
+ * caller that times or overlaps the parts. Parts must be issued in order
+ * TQP_FFN_PREPARE, TQP_FFN_GATE_UP, TQP_FFN_RANK, TQP_FFN_DOWN with the same
+ * arguments and workspace; together they equal one tqp_grouped_ffn call.
+ *   TQP_FFN_PREPARE : expert block schedule, x and Ad in fp16, s X [Ag|Au]
+ *   TQP_FFN_GATE_UP : h (one kernel: the gate/up expert contraction + SwiGLU)
+ *   TQP_FFN_RANK    : s H Ad
+ *   TQP_FFN_DOWN    : out_perm (one kernel: the down expert contraction)
+ * Returns TQP_ERR_INVALID_ARG for an unknown part.
  * ------------------------------------------------------------------------- */
+#define TQP_FFN_PREPARE 0
+#define TQP_FFN_GATE_UP 1
+#define TQP_FFN_RANK 2
+#define TQP_FFN_DOWN 3
 size_t tqp_grouped_ffn_workspace_size(int T, const tqp_moe_weights* w);
 int tqp_grouped_ffn(const uint16_t* x, int T, const int32_t* offsets, const int32_t* perm_token,
                     const tqp_moe_weights* w, uint16_t* h, uint16_t* out_perm, void* ws, size_t ws_bytes,
                     int32_t* dev_status, void* stream);
+int tqp_grouped_ffn_part(int part, const uint16_t* x, int T, const int32_t* offsets, const int32_t* perm_token,
+                         const tqp_moe_weights* w, uint16_t* h, uint16_t* out_perm, void* ws, size_t ws_bytes,
+                         int32_t* dev_status, void* stream);
 
 /* ---------------------------------------------------------------------------
  * moe_combine: gate-weighted un-permute (scatter back to tokens), plus the
  * additive coupling when a residual is given ("Pattern 1": addition and
  * subtraction are the invertible primitives).
- *   m[t] = bf16( sum_{j<k} gates[t][j] * out_perm[inv[t*k + j]] )  (fixed j order,
- *   fp32 accumulation, no atomics: deterministic)
+ *   m[t] = bf16( sum_{j<k} gates[t][j] * out_perm[inv[t*k + j]] )  (out_perm fp16 as
+ *   written by tqp_grouped_ffn; fixed j order, fp32 accumulation, no atomics:
+ *   deterministic)
  *   y[t] = m[t]                         if residual == NULL
  *   y[t] = residual[t] + sign * m[t]    otherwise (fp32 arithmetic)
  *   residual_dtype / y_dtype: TQP_DTYPE_BF16 or TQP_DTYPE_F32 (bf16 output is

@@ -15,7 +15,8 @@ import numpy as np
 
 __all__ = [
     "lib", "TQPError", "DeviceLayer", "Status", "workspace",
-    "moe_router_gemm", "moe_route", "moe_permute", "moe_permute_noalloc", "tqp_grouped_ffn", "moe_combine", "tqp_moe_layer_fwd",
+    "moe_router_gemm", "moe_route", "moe_permute", "moe_permute_noalloc", "tqp_grouped_ffn", "tqp_grouped_ffn_part",
+    "moe_combine", "tqp_moe_layer_fwd",
     "rev_couple_fwd", "rev_couple_inv", "tqp_moe_layer_bwd", "tqp_adapter_bwd",
     "header_functions",
 ]
@@ -29,6 +30,7 @@ TQP_OK = 0
 ERRORS = {-1: "invalid argument", -2: "unsupported configuration", -3: "workspace too small",
           -4: "CUDA launch or runtime error"}
 STATUS_NONFINITE, STATUS_BAD_ID, STATUS_TIMEOUT = 1, 2, 4
+FFN_PREPARE, FFN_GATE_UP, FFN_RANK, FFN_DOWN = 0, 1, 2, 3
 DTYPE_BF16, DTYPE_F32 = 0, 1
 
 
@@ -67,6 +69,7 @@ _SIGS = {
     "moe_permute_noalloc": (_I, [_VP, _I, _I, _I, _VP, _VP, _VP, _VP, _VP]),
     "tqp_grouped_ffn_workspace_size": (_SZ, [_I, _WP]),
     "tqp_grouped_ffn": (_I, [_VP, _I, _VP, _VP, _WP, _VP, _VP, _VP, _SZ, _VP, _VP]),
+    "tqp_grouped_ffn_part": (_I, [_I, _VP, _I, _VP, _VP, _WP, _VP, _VP, _VP, _SZ, _VP, _VP]),
     "moe_combine": (_I, [_VP, _VP, _VP, _I, _I, _I, _VP, _I, _F, _VP, _I, _VP, _VP]),
     "tqp_moe_layer_workspace_size": (_SZ, [_I, _WP]),
     "tqp_moe_layer_fwd": (_I, [_VP, _I, _WP, _VP, _VP, _SZ, _VP, _VP]),
@@ -258,6 +261,16 @@ def tqp_grouped_ffn(x, offsets, perm_token, layer: DeviceLayer, h, out_perm, ws=
     _check("tqp_grouped_ffn", lib().tqp_grouped_ffn(x.data_ptr(), T, offsets.data_ptr(), perm_token.data_ptr(),
                                                     layer.ref(), h.data_ptr(), out_perm.data_ptr(), ws.data_ptr(),
                                                     ws.numel(), status.ptr() if status else None, _stream(stream)))
+    return h, out_perm
+
+
+def tqp_grouped_ffn_part(part: int, x, offsets, perm_token, layer: DeviceLayer, h, out_perm, ws,
+                         status: Status | None = None, stream=None):
+    """One part of tqp_grouped_ffn (FFN_PREPARE, FFN_GATE_UP, FFN_RANK, FFN_DOWN, in order, same ws)."""
+    _require_cuda(x, offsets, perm_token, h, out_perm)
+    _check("tqp_grouped_ffn_part", lib().tqp_grouped_ffn_part(
+        int(part), x.data_ptr(), x.shape[0], offsets.data_ptr(), perm_token.data_ptr(), layer.ref(), h.data_ptr(),
+        out_perm.data_ptr(), ws.data_ptr(), ws.numel(), status.ptr() if status else None, _stream(stream)))
     return h, out_perm
 
 

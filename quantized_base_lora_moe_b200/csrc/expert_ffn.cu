@@ -28,7 +28,9 @@
 //   warps 10-25 weight producer: each thread dequantises 32 K values of one
 //               weight row (int4 -> fp16) into TMEM; LoRA B rows
 // TMEM (512 columns): accumulators in [0, 256), 4 weight stages of 64 columns
-// in [256, 512).
+// in [256, 512). A pipeline stage pairs one token tile (shared memory) with
+// one weight stage (TMEM): one "full" barrier collects both producers'
+// arrivals and one commit per stage frees both.
 //   GATEUP: one accumulator (gate cols [0,128), up [128,256)); a weight stage
 //           holds gate 32 | up 32 columns. The epilogue drains G and U as fp16
 //           into [token][feature] shared-memory tiles, hands TMEM back, and
@@ -61,16 +63,16 @@ constexpr uint32_t kWCols = 64;       // TMEM columns per weight stage
 
 template <int MODE> struct Cfg;
 template <> struct Cfg<GATEUP> {      // K stage 64: 128 token rows x 128 B
-  static constexpr int kK = 64, kXStageBytes = 16384, kXStages = 5, kStaging = 2 * 128 * kTRow;
+  static constexpr int kK = 64, kXStageBytes = 16384, kStaging = 2 * 128 * kTRow;
 };
 template <> struct Cfg<DOWN> {        // K stage 128: two 64-wide swizzled sub-tiles
-  static constexpr int kK = 128, kXStageBytes = 32768, kXStages = 4, kStaging = 2 * 32 * kTRow;
+  static constexpr int kK = 128, kXStageBytes = 32768, kStaging = 2 * 32 * kTRow;
 };
+constexpr int kStages = kWStages;     // pipeline stages (token tile + weight stage)
 
 struct Ctl {
-  uint64_t x_full[8], x_empty[8];
+  uint64_t full[kStages], empty[kStages];
   uint64_t q_full[kQStages], q_empty[kQStages];
-  uint64_t w_full[kWStages], w_empty[kWStages];
   uint64_t acc_full[2], acc_empty[2];
   uint64_t drain;
   uint64_t epi;
@@ -80,7 +82,7 @@ struct Ctl {
 
 template <int MODE>
 constexpr size_t smem_bytes() {
-  return 1024 + size_t(Cfg<MODE>::kXStages) * Cfg<MODE>::kXStageBytes + size_t(kQStages) * kQStageBytes +
+  return 1024 + size_t(kStages) * Cfg<MODE>::kXStageBytes + size_t(kQStages) * kQStageBytes +
          size_t(Cfg<MODE>::kStaging) + sizeof(Ctl);
 }
 static_assert(smem_bytes<GATEUP>() <= 232448 && smem_bytes<DOWN>() <= 232448, "shared memory budget");
@@ -134,12 +136,11 @@ __global__ void __launch_bounds__(kThreads, 1)
                       const __grid_constant__ CUtensorMap ts1, const __grid_constant__ CUtensorMap th) {
   constexpr bool kGU = (MODE == GATEUP);
   constexpr int kK = Cfg<MODE>::kK;
-  constexpr int XS = Cfg<MODE>::kXStages;
   constexpr int kXBytes = Cfg<MODE>::kXStageBytes;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   uint8_t* x_base = smem;
-  uint8_t* q_base = x_base + size_t(XS) * kXBytes;
+  uint8_t* q_base = x_base + size_t(kStages) * kXBytes;
   uint8_t* staging = q_base + size_t(kQStages) * kQStageBytes;
   Ctl* ctl = reinterpret_cast<Ctl*>(staging + Cfg<MODE>::kStaging);
   volatile int* abort_flag = &ctl->abort_flag;
@@ -148,17 +149,13 @@ __global__ void __launch_bounds__(kThreads, 1)
   const int lane = threadIdx.x & 31;
 
   if (threadIdx.x == 0) {
-    for (int i = 0; i < XS; ++i) {
-      mbar_init(&ctl->x_full[i], 128);
-      mbar_init(&ctl->x_empty[i], 1);
+    for (int i = 0; i < kStages; ++i) {
+      mbar_init(&ctl->full[i], 128 + kWWarps * 32);   // token producer + weight producer threads
+      mbar_init(&ctl->empty[i], 1);
     }
     for (int i = 0; i < kQStages; ++i) {
       mbar_init(&ctl->q_full[i], 1);
       mbar_init(&ctl->q_empty[i], kWWarps * 32);
-    }
-    for (int i = 0; i < kWStages; ++i) {
-      mbar_init(&ctl->w_full[i], kWWarps * 32);
-      mbar_init(&ctl->w_empty[i], 1);
     }
     for (int i = 0; i < 2; ++i) {
       mbar_init(&ctl->acc_full[i], 1);
@@ -283,7 +280,7 @@ __global__ void __launch_bounds__(kThreads, 1)
   } else if (warp == 4) {
     // ------------------------------------------------------------ MMA issuer
     if (lane == 0) {
-      Ring rx, rw;
+      Ring rs;
       int it = 0;
       bool ok = true;
       for (int u = blockIdx.x; u < nunits && ok; u += gridDim.x, ++it) {
@@ -296,15 +293,11 @@ __global__ void __launch_bounds__(kThreads, 1)
         tc_fence_after();
         const uint32_t dacc = tmem_base + uint32_t(ab * 128);
         for (int kb = 0; kb < nkb; ++kb) {
-          if (!mbar_wait(&ctl->x_full[rx.stage], rx.phase, abort_flag, a.status) ||
-              !mbar_wait(&ctl->w_full[rw.stage], rw.phase, abort_flag, a.status)) {
-            ok = false;
-            break;
-          }
+          if (!mbar_wait(&ctl->full[rs.stage], rs.phase, abort_flag, a.status)) { ok = false; break; }
           tc_fence_after();
-          const uint32_t xs = smem_u32(x_base + size_t(rx.stage) * kXBytes);
+          const uint32_t xs = smem_u32(x_base + size_t(rs.stage) * kXBytes);
           const uint64_t bdesc = sdesc_k_sw128(xs);
-          const uint32_t wa = tmem_base + kWBase + uint32_t(rw.stage) * kWCols;
+          const uint32_t wa = tmem_base + kWBase + uint32_t(rs.stage) * kWCols;
           if (kb >= a.nkb_lora) {
             if (kGU) {
 #pragma unroll
@@ -331,10 +324,8 @@ __global__ void __launch_bounds__(kThreads, 1)
               if (kGU) umma_f16_ts(dacc + 128, wa + 32 + uint32_t(8 * kk), bdesc + uint64_t(2 * kk), idesc, acc);
             }
           }
-          umma_commit(&ctl->x_empty[rx.stage]);
-          umma_commit(&ctl->w_empty[rw.stage]);
-          rx.next<XS>();
-          rw.next<kWStages>();
+          umma_commit(&ctl->empty[rs.stage]);
+          rs.next<kStages>();
         }
         if (!ok) break;
         umma_commit(&ctl->acc_full[ab]);
@@ -381,7 +372,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         if (!ok) break;
       }
       // on an abort, wait (bounded) until the last issued stage has landed
-      if (issued > 0 && *abort_flag) mbar_wait(&ctl->q_full[last_stage], last_phase, abort_flag, a.status);
+      if (issued > 0 && *abort_flag) mbar_drain(&ctl->q_full[last_stage], last_phase);
     }
   } else if (warp < kWWarp0) {
     // ------------------------------------------------------------ token producer
@@ -406,9 +397,9 @@ __global__ void __launch_bounds__(kThreads, 1)
       }
       bool ok = true;
       for (int kb = 0; kb < nkb; ++kb) {
-        if (!mbar_wait<64>(&ctl->x_empty[rx.stage], rx.phase ^ 1u, abort_flag, a.status)) { ok = false; break; }
+        if (!mbar_wait<64>(&ctl->empty[rx.stage], rx.phase ^ 1u, abort_flag, a.status)) { ok = false; break; }
         const uint32_t st_u = smem_u32(x_base + size_t(rx.stage) * kXBytes);
-        uint64_t* full = &ctl->x_full[rx.stage];
+        uint64_t* full = &ctl->full[rx.stage];
         if (kb < a.nkb_lora) {
           // rank-space rows (s X[Ag|Au] or s H Ad) in the first 64-wide sub-tile,
           // zero-filled past lora_k (lora_k <= 128, and <= 64 for DOWN)
@@ -442,13 +433,15 @@ __global__ void __launch_bounds__(kThreads, 1)
             mbar_arrive(full);
           }
         }
-        rx.next<XS>();
+        rx.next<kStages>();
       }
       if (!ok) break;
     }
     cp_async_wait_all();
+    // on an abort, wait (bounded) until the last TMA fill issued here has landed
+    // (the stage's other arrivals may never come; the wait then runs out)
     if (tid == 0 && *abort_flag && pend_stage >= 0)
-      mbar_wait(&ctl->x_full[pend_stage], pend_phase, abort_flag, a.status);
+      mbar_drain(&ctl->full[pend_stage], pend_phase);
   } else {
     // ------------------------------------------------------------ weight producer
     // thread = 32 consecutive K values (4 int4 words) of one weight row per stage
@@ -475,7 +468,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         for (int off = 0; off < a.r; off += 64) prefetch_l2(row + off);
       }
       for (int kb = 0; kb < nkb; ++kb) {
-        if (!mbar_wait(&ctl->w_empty[rw.stage], rw.phase ^ 1u, abort_flag, a.status)) { ok = false; break; }
+        if (!mbar_wait(&ctl->empty[rw.stage], rw.phase ^ 1u, abort_flag, a.status)) { ok = false; break; }
         tc_fence_after();
         uint32_t v[16];
         if (kb < a.nkb_lora) {
@@ -512,8 +505,8 @@ __global__ void __launch_bounds__(kThreads, 1)
         tmem_st16(tw + uint32_t(rw.stage) * kWCols, v);
         tmem_wait_st();
         tc_fence_before();
-        mbar_arrive(&ctl->w_full[rw.stage]);
-        rw.next<kWStages>();
+        mbar_arrive(&ctl->full[rw.stage]);
+        rw.next<kStages>();
       }
       if (!ok) break;
     }

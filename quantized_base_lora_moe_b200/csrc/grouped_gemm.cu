@@ -362,7 +362,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         if (!ok) break;
       }
       // drain: wait until the last issued stage has landed (bounded)
-      if (issued > 0 && *abort_flag) mbar_wait(&ctl->q_full[last_stage], last_phase, abort_flag, a.status);
+      if (issued > 0 && *abort_flag) mbar_drain(&ctl->q_full[last_stage], last_phase);
     }
   } else if (warp < 10) {
     // ------------------------------------------------------------ A producer
@@ -378,8 +378,8 @@ __global__ void __launch_bounds__(kThreads, 1)
     if (MODE == LORA_XA) b_bytes = uint32_t(2 * a.r * 128);
     if (MODE == LORA_HA) b_bytes = uint32_t(a.r * 128);
     if (MODE == ROUTER) b_bytes = uint32_t(a.ntile * 128);
-    int pend_stage = -1;
-    uint32_t pend_phase = 0;
+    int pend_stage = -1, pend_b_stage = -1;
+    uint32_t pend_phase = 0, pend_b_phase = 0;
     for (int u = blockIdx.x; u < nunits; u += gridDim.x) {
       const Unit un = decode_unit(a, u);
       int srow[8];   // gathered source rows of this thread's 8 tile rows
@@ -414,6 +414,8 @@ __global__ void __launch_bounds__(kThreads, 1)
             uint64_t* bfull = &ctl->b_full[rb.stage];
             const uint32_t bst_u = smem_u32(b_base + size_t(rb.stage) * kBStageBytes);
             mbar_arrive_expect_tx(bfull, b_bytes);
+            pend_b_stage = rb.stage;
+            pend_b_phase = rb.phase;
             if (MODE == LORA_XA) {
               tma_load_2d(bst_u, &tb0, bfull, kcol, un.e * a.r);
               tma_load_2d(bst_u + a.r * 128, &tb1, bfull, kcol, un.e * a.r);
@@ -450,8 +452,8 @@ __global__ void __launch_bounds__(kThreads, 1)
     }
     cp_async_wait_all();
     // on an abort, wait (bounded) for the last TMA fill issued by this thread
-    if (tid == 0 && *abort_flag && pend_stage >= 0)
-      mbar_wait(&ctl->a_full[pend_stage], pend_phase, abort_flag, a.status);
+    if (tid == 0 && *abort_flag && pend_stage >= 0) mbar_drain(&ctl->a_full[pend_stage], pend_phase);
+    if (tid == 0 && *abort_flag && pend_b_stage >= 0) mbar_drain(&ctl->b_full[pend_b_stage], pend_b_phase);
   } else {
     // ------------------------------------------------------------ B producer
     const int tid = threadIdx.x - 10 * 32;  // 0..255
@@ -800,18 +802,25 @@ static int to_f16(const uint16_t* src, uint16_t* dst, size_t n, int32_t* status,
   return cudaGetLastError() == cudaSuccess ? TQP_OK : TQP_ERR_CUDA;
 }
 
-int launch_grouped_ffn(const uint16_t* x, int T, const int32_t* offsets, const int32_t* perm_token,
-                       const tqp_moe_weights* w, uint16_t* h, uint16_t* out_perm, void* ws, int32_t* status,
-                       cudaStream_t s, uint16_t* aux_gu) {
+// One part of the grouped FFN (parts run in order on one workspace):
+//   0 prepare : m-block schedule, x and Ad^T in fp16, xa = s X [Ag | Au]
+//   1 gate/up : H = silu(G) * U
+//   2 rank    : ha = s H Ad
+//   3 down    : O = H Wd^T + ha Bd
+int launch_grouped_ffn_part(int part, const uint16_t* x, int T, const int32_t* offsets, const int32_t* perm_token,
+                            const tqp_moe_weights* w, uint16_t* h, uint16_t* out_perm, void* ws, int32_t* status,
+                            cudaStream_t s, uint16_t* aux_gu) {
   if (T == 0) return TQP_OK;
   const size_t A = size_t(T) * w->top_k;
   const FfnBufs fb = ffn_carve(ws, T, w);
   const int d = w->d, f = w->ffn, r = w->rank;
-  schedule_kernel<<<1, 1024, 0, s>>>(offsets, w->E, fb.mb_prefix);
-  if (cudaGetLastError() != cudaSuccess) return TQP_ERR_CUDA;
   int rc;
-  if ((rc = to_f16(x, fb.x16, size_t(T) * d, status, s)) != TQP_OK) return rc;
-  if (r > 0 && (rc = to_f16(w->lora_a[2], fb.adT16, size_t(w->E) * r * f, nullptr, s)) != TQP_OK) return rc;
+  if (part == 0) {
+    schedule_kernel<<<1, 1024, 0, s>>>(offsets, w->E, fb.mb_prefix);
+    if (cudaGetLastError() != cudaSuccess) return TQP_ERR_CUDA;
+    if ((rc = to_f16(x, fb.x16, size_t(T) * d, status, s)) != TQP_OK) return rc;
+    if (r > 0 && (rc = to_f16(w->lora_a[2], fb.adT16, size_t(w->E) * r * f, nullptr, s)) != TQP_OK) return rc;
+  }
   // an upper bound on the number of work units (grid sizing only)
   const int mb_upper = int((A + kMBlock - 1) / kMBlock) + w->E;
 
@@ -826,7 +835,7 @@ int launch_grouped_ffn(const uint16_t* x, int T, const int32_t* offsets, const i
   base.status = status;
   base.kb_per_piece = 1;
 
-  if (r > 0) {  // xa = s * X [Ag | Au]   (bf16 operands)
+  if (part == 0 && r > 0) {  // xa = s * X [Ag | Au]   (bf16 operands)
     GemmArgs a = base;
     a.nkb_main = d / 64;
     a.ntile = 2 * r < 16 ? 16 : 2 * r;
@@ -846,7 +855,7 @@ int launch_grouped_ffn(const uint16_t* x, int T, const int32_t* offsets, const i
   // hidden width is a multiple of 128 (its K stages and feature tiles), else on
   // the shared-memory engine above.
   const bool tm = (f % 128 == 0);
-  {  // H = silu(G) * U
+  if (part == 1) {  // H = silu(G) * U
     GemmArgs a = base;
     a.nkb_main = d / 64;
     a.nkb_lora = r > 0 ? (2 * r + 63) / 64 : 0;
@@ -883,7 +892,7 @@ int launch_grouped_ffn(const uint16_t* x, int T, const int32_t* offsets, const i
             : run_gemm<GATEUP>(a, mp, mb_upper * a.n_tiles, s);
     if (rc != TQP_OK) return rc;
   }
-  if (r > 0) {  // ha = s * H Ad
+  if (part == 2 && r > 0) {  // ha = s * H Ad
     GemmArgs a = base;
     a.nkb_main = f / 64;
     a.ntile = r < 16 ? 16 : r;
@@ -897,7 +906,7 @@ int launch_grouped_ffn(const uint16_t* x, int T, const int32_t* offsets, const i
       return TQP_ERR_CUDA;
     if ((rc = run_gemm<LORA_HA>(a, mp, mb_upper, s)) != TQP_OK) return rc;
   }
-  {  // O = H Wd^T + (s H Ad) Bd
+  if (part == 3) {  // O = H Wd^T + (s H Ad) Bd
     GemmArgs a = base;
     const int kst = tm ? 128 : 64;   // K stage
     a.nkb_main = f / kst;
@@ -922,6 +931,16 @@ int launch_grouped_ffn(const uint16_t* x, int T, const int32_t* offsets, const i
                        uint64_t(d) * 2, uint32_t(a.ntile), ngrp);
     if (!ok) return TQP_ERR_CUDA;
     rc = tm ? run_expert_ffn(DOWN, a, mp, mb_upper * a.n_tiles, s) : run_gemm<DOWN>(a, mp, mb_upper * a.n_tiles, s);
+    if (rc != TQP_OK) return rc;
+  }
+  return TQP_OK;
+}
+
+int launch_grouped_ffn(const uint16_t* x, int T, const int32_t* offsets, const int32_t* perm_token,
+                       const tqp_moe_weights* w, uint16_t* h, uint16_t* out_perm, void* ws, int32_t* status,
+                       cudaStream_t s, uint16_t* aux_gu) {
+  for (int part = 0; part < 4; ++part) {
+    const int rc = launch_grouped_ffn_part(part, x, T, offsets, perm_token, w, h, out_perm, ws, status, s, aux_gu);
     if (rc != TQP_OK) return rc;
   }
   return TQP_OK;

@@ -271,6 +271,21 @@ int tqp_grouped_ffn(const uint16_t* x, int T, const int32_t* offsets, const int3
                             static_cast<cudaStream_t>(stream));
 }
 
+int tqp_grouped_ffn_part(int part, const uint16_t* x, int T, const int32_t* offsets, const int32_t* perm_token,
+                         const tqp_moe_weights* w, uint16_t* h, uint16_t* out_perm, void* ws, size_t ws_bytes,
+                         int32_t* dev_status, void* stream) {
+  if (part < TQP_FFN_PREPARE || part > TQP_FFN_DOWN) return TQP_ERR_INVALID_ARG;
+  int rc = check_weights(w);
+  if (rc != TQP_OK) return rc;
+  const bool n = T > 0;
+  if (T < 0 || !ptr_ok(x, n) || !ptr_ok(offsets, n) || !ptr_ok(perm_token, n) || !ptr_ok(h, n) ||
+      !ptr_ok(out_perm, n) || !ptr_ok(ws, n))
+    return TQP_ERR_INVALID_ARG;
+  if (n && ws_bytes < ffn_ws_bytes(T, w)) return TQP_ERR_WORKSPACE;
+  return launch_grouped_ffn_part(part, x, T, offsets, perm_token, w, h, out_perm, ws, dev_status,
+                                 static_cast<cudaStream_t>(stream));
+}
+
 int moe_combine(const uint16_t* out_perm, const int32_t* inv, const float* gates, int T, int k, int d,
                 const void* residual, int residual_dtype, float sign, void* y, int y_dtype, uint16_t* y_bf16,
                 void* stream) {

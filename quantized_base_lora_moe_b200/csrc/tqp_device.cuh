@@ -96,6 +96,18 @@ __device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, volati
   }
 }
 
+// Drain wait on the abort path: waits for the phase regardless of the abort
+// flag, but no longer than limit_ns, so that a TMA fill issued before the abort
+// has landed before the CTA exits (its barrier may also never complete when
+// other arrivals are missing; the wait then just runs out).
+__device__ __forceinline__ void mbar_drain(uint64_t* bar, uint32_t parity, uint64_t limit_ns = 1000000ull) {
+  const uint32_t addr = smem_u32(bar);
+  const uint64_t t0 = globaltimer();
+  while (!mbar_try_wait(addr, parity)) {
+    if (globaltimer() - t0 > limit_ns) return;
+  }
+}
+
 // ----------------------------------------------------------------------------
 // async copies
 // ----------------------------------------------------------------------------

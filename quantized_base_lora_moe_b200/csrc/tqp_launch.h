@@ -40,6 +40,9 @@ FfnBufs ffn_carve(void* ws, int T, const tqp_moe_weights* w);
 int launch_grouped_ffn(const uint16_t* x, int T, const int32_t* offsets, const int32_t* perm_token,
                        const tqp_moe_weights* w, uint16_t* h, uint16_t* out_perm, void* ws, int32_t* status,
                        cudaStream_t s, uint16_t* aux_gu = nullptr);
+int launch_grouped_ffn_part(int part, const uint16_t* x, int T, const int32_t* offsets, const int32_t* perm_token,
+                            const tqp_moe_weights* w, uint16_t* h, uint16_t* out_perm, void* ws, int32_t* status,
+                            cudaStream_t s, uint16_t* aux_gu = nullptr);
 int launch_dgrad(int which, const uint16_t* a_src, const uint16_t* a_lora, const int32_t* offsets,
                  const int32_t* mb_prefix, const tqp_moe_weights* w, int T, const uint16_t* aux_gu, uint16_t* out,
                  int32_t* status, cudaStream_t s);

@@ -83,3 +83,14 @@ def test_mismatched_coupling_widths_rejected():
     assert L.rev_couple_workspace_size(64, ctypes.byref(F), ctypes.byref(G)) == 0
     assert L.rev_couple_fwd(0x1000, 0x1000, 64, ctypes.byref(F), ctypes.byref(G), 0x1000, 0x1000, 0x1000,
                             1 << 30, None, None) == -1
+
+
+def test_grouped_ffn_part_rejects_unknown_part():
+    L = Q.lib()
+    w = _struct(synth.TINY)
+    for part in (-1, 4):
+        rc = L.tqp_grouped_ffn_part(part, None, 0, None, None, ctypes.byref(w), None, None, None, 0, None, None)
+        assert rc == -1, (part, rc)
+    # a valid part with an empty batch is a no-op that enqueues nothing
+    rc = L.tqp_grouped_ffn_part(Q.FFN_GATE_UP, None, 0, None, None, ctypes.byref(w), None, None, None, 0, None, None)
+    assert rc == 0

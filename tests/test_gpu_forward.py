@@ -217,6 +217,29 @@ def _run_ffn(cfg, xb, offsets, perm):
     return h, o
 
 
+@pytest.mark.parametrize("cfg", [synth.TINY, RAGGED, synth.MID], ids=lambda c: c.name)
+def test_grouped_ffn_parts_equal_whole_call(cfg):
+    """The four parts issued in order give bit-identical h and out_perm."""
+    xb = synth.make_tokens(cfg.T, cfg.d, 14)
+    x = O.bf16_to_f64(xb)
+    L = O.Layer(host_layer(cfg))
+    ids = O.topk(O.router_logits(x, L), cfg.k)
+    offsets, perm, _ = _ffn_case(cfg, x, L, ids)
+    h1, o1 = _run_ffn(cfg, xb, offsets, perm)
+    A = cfg.T * cfg.k
+    h2 = torch.empty(A, cfg.f, dtype=torch.int16, device="cuda")
+    o2 = torch.empty(A, cfg.d, dtype=torch.int16, device="cuda")
+    layer = device_layer(cfg)
+    ws = Q.workspace(Q.lib().tqp_grouped_ffn_workspace_size(cfg.T, layer.ref()), h2.device)
+    st = Q.Status()
+    xd, od, pd = dev_bf16(xb), dev(offsets), dev(perm)
+    for part in (Q.FFN_PREPARE, Q.FFN_GATE_UP, Q.FFN_RANK, Q.FFN_DOWN):
+        Q.tqp_grouped_ffn_part(part, xd, od, pd, layer, h2, o2, ws, status=st)
+    torch.cuda.synchronize()
+    assert st.read() == 0
+    assert torch.equal(h1, h2) and torch.equal(o1, o2)
+
+
 @pytest.mark.parametrize("cfg", SMALL_CFGS, ids=lambda c: c.name)
 def test_grouped_ffn_matches_oracle(cfg):
     raw = host_layer(cfg)

@@ -1,0 +1,74 @@
+"""Multi-process host logic of the benchmark, on CPU (gloo, world size 2).
+
+The layer shards by tokens: every rank runs the whole hot path on its own batch
+with replicated weights, and the only cross-rank step is the timing reduction
+(max over ranks of the step time). That reduction, the per-rank batch choice and
+the whole-job metric are what these tests pin; the reference arm's N>1 behaviour
+(rank 0 alone runs and prints) is checked on a tiny workload.
+"""
+import json
+import os
+import subprocess
+import sys
+
+import numpy as np
+import pytest
+import torch
+import torch.distributed as dist
+import torch.multiprocessing as mp
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+sys.path.insert(0, ROOT)
+
+import bench  # noqa: E402
+import synth  # noqa: E402
+
+
+def _worker(rank, world, port, out):
+    os.environ["MASTER_ADDR"] = "127.0.0.1"
+    os.environ["MASTER_PORT"] = str(port)
+    import datetime
+    dist.init_process_group("gloo", rank=rank, world_size=world, timeout=datetime.timedelta(seconds=60))
+    try:
+        local_ms = 3.0 + 2.0 * rank                       # rank 1 is the slow one
+        got = bench.max_over_ranks(local_ms, torch.device("cpu"), True)
+        cfg = synth.TINY
+        seed = bench.rank_token_seed(cfg, rank)
+        xb = synth.make_tokens(cfg.T, cfg.d, seed)
+        digest = int(np.asarray(xb, dtype=np.uint64).sum())
+        out[rank] = (got, seed, digest)
+    finally:
+        dist.destroy_process_group()
+
+
+def test_two_rank_timing_reduction_and_batches():
+    port = 29500 + (os.getpid() % 2000)
+    manager = mp.Manager()
+    out = manager.dict()
+    mp.spawn(_worker, args=(2, port, out), nprocs=2, join=True)
+    (m0, s0, d0), (m1, s1, d1) = out[0], out[1]
+    assert m0 == m1 == 5.0                  # every rank reports the slowest rank's time
+    assert s0 != s1 and d0 != d1            # independent token batches per rank
+    # whole-job value: both ranks' tokens over the max-over-ranks time
+    assert bench.weak_scaling_value(2, 8192, 5.0) == pytest.approx(2 * 8192 / 5e-3)
+
+
+def test_single_rank_reduction_is_identity():
+    assert bench.max_over_ranks(1.25, torch.device("cpu"), False) == 1.25
+
+
+def _run_reference(rank, world):
+    env = dict(os.environ, RANK=str(rank), WORLD_SIZE=str(world), LOCAL_RANK=str(rank))
+    return subprocess.run([sys.executable, os.path.join(ROOT, "bench.py"), "--impl", "reference", "--config", "tiny",
+                           "--steps", "1", "--warmup", "0", "--ref-sample", "2"],
+                          capture_output=True, text=True, env=env, timeout=300)
+
+
+def test_reference_arm_runs_on_rank0_only():
+    r1 = _run_reference(1, 2)
+    assert r1.returncode == 0 and r1.stdout.strip() == ""
+    r0 = _run_reference(0, 2)
+    assert r0.returncode == 0, r0.stderr[-500:]
+    line = json.loads(r0.stdout.strip().splitlines()[-1])
+    assert line["impl"] == "reference" and line["value"] > 0
+    assert line["cpu_baseline"]["kind"] == "oracle" and line["e2e"]["h2d_bytes_per_step"] == 0
