@@ -74,6 +74,24 @@ def weak_scaling_value(world: int, tokens_per_rank: int, ms_per_step: float) -> 
     return world * tokens_per_rank / (ms_per_step * 1e-3)
 
 
+def measured_traffic(kernel: str) -> int | None:
+    """DRAM bytes per launch of `kernel` from the committed ncu capture, if the
+    expert-kernel sources are still the ones that were captured; else None."""
+    import hashlib
+    path = os.path.join(ROOT, "profiles", "expert_ffn_traffic_full.json")
+    if not os.path.exists(path):
+        return None
+    doc = json.load(open(path))
+    h = hashlib.sha256()
+    for f in ("expert_ffn.cu", "gemm_common.cuh", "tqp_device.cuh"):
+        with open(os.path.join(ROOT, "quantized_base_lora_moe_b200", "csrc", f), "rb") as fh:
+            h.update(fh.read())
+    if h.hexdigest()[:16] != doc.get("kernel_sources_sha256_16"):
+        return None
+    k = doc["kernels"].get(kernel)
+    return None if k is None else int(k["dram_read_bytes"] + k["dram_write_bytes"])
+
+
 def peaks() -> dict:
     p = os.path.join(ROOT, "MEASURED_PEAKS.json")
     if os.path.exists(p):
@@ -299,7 +317,9 @@ def run_tqp(args, rank: int, world: int, local_rank: int) -> dict | None:
         "roofline": {"bound": "tensor",
                      "kernel": "expert_ffn_kernel<GATEUP> (int4 -> fp16 weights in TMEM, tcgen05 gate/up + SwiGLU)",
                      "achieved": gu_tflops, "peak": pk["bf16_tflops"], "unit": "TFLOP/s",
-                     "frac": gu_tflops / pk["bf16_tflops"], "traffic": None,
+                     "frac": gu_tflops / pk["bf16_tflops"],
+                     "traffic": measured_traffic("expert_ffn_kernel<GATEUP>") if args.config == "full" else None,
+                     "traffic_source": "profiles/expert_ffn_traffic_full.md (ncu dram__bytes_read+write, one launch)",
                      "peak_source": f"{pk['source']} bf16 dense burst (fp16 has the same nominal rate)",
                      "flop_per_launch": fl["gate_up"], "ms_per_launch": gu_ms},
         "ffn_call": {"achieved_tflops": ffn_tflops, "frac": ffn_tflops / pk["bf16_tflops"], "ms": ffn_ms,
