@@ -35,9 +35,9 @@
 //           holds gate 32 | up 32 columns. The epilogue drains G and U as fp16
 //           into [token][feature] shared-memory tiles, hands TMEM back, and
 //           finishes SwiGLU + 16-byte row stores while the next unit runs.
-//   DOWN:   two accumulators of 128 columns; 32-token chunks go out through a
-//           double-buffered [token][feature] tile, so that every global store is
-//           a 16-byte piece of a row.
+//   DOWN:   two accumulators of 128 columns; the epilogue drains a whole
+//           accumulator as fp16 into a [token][feature] tile, hands TMEM back,
+//           and then stores 16-byte row pieces.
 // Every wait is bounded (tqp_device.cuh); no TMA multicast is used.
 #include <cstdint>
 #include <cuda.h>
@@ -54,7 +54,7 @@ namespace tmem_ffn {
 constexpr int kWWarp0 = 10;           // first weight-producer warp
 constexpr int kWWarps = 16;
 constexpr int kThreads = (kWWarp0 + kWWarps) * 32;
-constexpr int kQStages = 8;
+constexpr int kQStagesMax = 8;
 constexpr int kQStageBytes = 9216;    // up to 8192 B of codes + 1024 B of scales
 constexpr int kTRow = 272;            // staging row: one token's 128 features in fp16, +16 B against bank conflicts
 constexpr uint32_t kWBase = 256;      // first TMEM column of the weight stages
@@ -63,16 +63,16 @@ constexpr uint32_t kWCols = 64;       // TMEM columns per weight stage
 
 template <int MODE> struct Cfg;
 template <> struct Cfg<GATEUP> {      // K stage 64: 128 token rows x 128 B
-  static constexpr int kK = 64, kXStageBytes = 16384, kStaging = 2 * 128 * kTRow;
+  static constexpr int kK = 64, kXStageBytes = 16384, kStaging = 2 * 128 * kTRow, kQStages = 8;
 };
 template <> struct Cfg<DOWN> {        // K stage 128: two 64-wide swizzled sub-tiles
-  static constexpr int kK = 128, kXStageBytes = 32768, kStaging = 2 * 32 * kTRow;
+  static constexpr int kK = 128, kXStageBytes = 32768, kStaging = 128 * kTRow, kQStages = 6;
 };
 constexpr int kStages = kWStages;     // pipeline stages (token tile + weight stage)
 
 struct Ctl {
   uint64_t full[kStages], empty[kStages];
-  uint64_t q_full[kQStages], q_empty[kQStages];
+  uint64_t q_full[kQStagesMax], q_empty[kQStagesMax];
   uint64_t acc_full[2], acc_empty[2];
   uint64_t drain;
   uint64_t epi;
@@ -82,7 +82,7 @@ struct Ctl {
 
 template <int MODE>
 constexpr size_t smem_bytes() {
-  return 1024 + size_t(kStages) * Cfg<MODE>::kXStageBytes + size_t(kQStages) * kQStageBytes +
+  return 1024 + size_t(kStages) * Cfg<MODE>::kXStageBytes + size_t(Cfg<MODE>::kQStages) * kQStageBytes +
          size_t(Cfg<MODE>::kStaging) + sizeof(Ctl);
 }
 static_assert(smem_bytes<GATEUP>() <= 232448 && smem_bytes<DOWN>() <= 232448, "shared memory budget");
@@ -137,6 +137,7 @@ __global__ void __launch_bounds__(kThreads, 1)
   constexpr bool kGU = (MODE == GATEUP);
   constexpr int kK = Cfg<MODE>::kK;
   constexpr int kXBytes = Cfg<MODE>::kXStageBytes;
+  constexpr int kQStages = Cfg<MODE>::kQStages;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   uint8_t* x_base = smem;
@@ -147,6 +148,8 @@ __global__ void __launch_bounds__(kThreads, 1)
 
   const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
+  __shared__ int32_t s_sched[2 * (kSchedSmemE + 1)];
+  const Sched sc = load_sched(a, s_sched);
 
   if (threadIdx.x == 0) {
     for (int i = 0; i < kStages; ++i) {
@@ -184,7 +187,7 @@ __global__ void __launch_bounds__(kThreads, 1)
   tc_fence_after();
   const uint32_t tmem_base = ctl->tmem_base;
 
-  const int nunits = total_units(a);
+  const int nunits = total_units(a, sc);
   const int nkb = a.nkb_main + a.nkb_lora;
   // scale rows per K stage (one per quantisation group it spans)
   const int ngrp = a.g >= kK ? 1 : kK / a.g;
@@ -194,10 +197,9 @@ __global__ void __launch_bounds__(kThreads, 1)
     const int row = warp * 32 + lane;   // feature within the tile = TMEM lane
     const uint32_t tl = tmem_base + (uint32_t(warp * 32) << 16);
     int it = 0;
-    int chunk = 0;   // DOWN: running chunk count (selects the staging tile)
     EpiSync es{&ctl->epi};
     for (int u = blockIdx.x; u < nunits; u += gridDim.x, ++it) {
-      const Unit un = decode_unit(a, u);
+      const Unit un = decode_unit(a, sc, u);
       const int n16 = (un.rows + 15) & ~15;
       if (kGU) {
         if (!mbar_wait<128>(&ctl->acc_full[0], uint32_t(it) & 1u, abort_flag, a.status)) break;
@@ -244,37 +246,26 @@ __global__ void __launch_bounds__(kThreads, 1)
         const int ab = it & 1;
         if (!mbar_wait<128>(&ctl->acc_full[ab], uint32_t(it >> 1) & 1u, abort_flag, a.status)) break;
         tc_fence_after();
-        uint16_t* out = static_cast<uint16_t*>(a.out) + un.nt * 128;
-        bool stop = false;
+        // drain the whole accumulator as fp16 into the [token][feature] tile
 #pragma unroll 1
-        for (int c = 0; c < n16; c += 32, ++chunk) {
-          // consecutive chunks alternate between the two tiles; the barrier after a
-          // tile is written also orders every earlier read of the other tile
-          uint8_t* tile = staging + (chunk & 1) * (32 * kTRow);
+        for (int c = 0; c < n16; c += 16) {
+          float v[16];
+          tmem_ld16(tl + uint32_t(ab * 128 + c), v);
+          uint32_t pk[8];
 #pragma unroll
-          for (int hh = 0; hh < 2; ++hh) {
-            if (c + 16 * hh < n16) {
-              float v[16];
-              tmem_ld16(tl + uint32_t(ab * 128 + c + 16 * hh), v);
-              uint32_t pk[8];
-#pragma unroll
-              for (int j = 0; j < 8; ++j) pk[j] = f32x2_to_f16x2(v[2 * j], v[2 * j + 1]);
-              stage_tokens<8>(tile, 16 * hh, row, pk);
-            }
-          }
-          if (c + 32 >= n16) {  // last read of this accumulator: hand it back before storing
-            tc_fence_before();
-            mbar_arrive(&ctl->acc_empty[ab]);
-          }
-          if (!es.sync(abort_flag, a.status)) { stop = true; break; }
-          const int nt = min(32, un.rows - c);
-          for (int p = threadIdx.x; p < nt * 16; p += 128) {
-            const int t = p >> 4, fg = p & 15;
-            *reinterpret_cast<uint4*>(out + size_t(un.base + c + t) * a.out_ld + fg * 8) =
-                *reinterpret_cast<const uint4*>(tile + t * kTRow + fg * 16);
-          }
+          for (int j = 0; j < 8; ++j) pk[j] = f32x2_to_f16x2(v[2 * j], v[2 * j + 1]);
+          stage_tokens<8>(staging, c, row, pk);
         }
-        if (stop) break;
+        tc_fence_before();
+        mbar_arrive(&ctl->acc_empty[ab]);
+        if (!es.sync(abort_flag, a.status)) break;
+        uint16_t* out = static_cast<uint16_t*>(a.out) + un.nt * 128;
+        for (int p = threadIdx.x; p < un.rows * 16; p += 128) {
+          const int t = p >> 4, fg = p & 15;
+          *reinterpret_cast<uint4*>(out + size_t(un.base + t) * a.out_ld + fg * 8) =
+              *reinterpret_cast<const uint4*>(staging + t * kTRow + fg * 16);
+        }
+        if (!es.sync(abort_flag, a.status)) break;  // the tile is free for the next unit's drain
       }
     }
   } else if (warp == 4) {
@@ -284,7 +275,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       int it = 0;
       bool ok = true;
       for (int u = blockIdx.x; u < nunits && ok; u += gridDim.x, ++it) {
-        const Unit un = decode_unit(a, u);
+        const Unit un = decode_unit(a, sc, u);
         const int n16 = (un.rows + 15) & ~15;
         const uint32_t idesc = idesc_f16(128, n16);
         const int ab = kGU ? 0 : (it & 1);
@@ -347,7 +338,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       uint32_t last_phase = 0;
       int last_stage = 0;
       for (int u = blockIdx.x; u < nunits; u += gridDim.x) {
-        const Unit un = decode_unit(a, u);
+        const Unit un = decode_unit(a, sc, u);
         const int nrow0 = un.e * a.out_dim + un.nt * 128;
         bool ok = true;
         for (int km = 0; km < a.nkb_main; ++km) {
@@ -386,7 +377,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     int pend_stage = -1;
     uint32_t pend_phase = 0;
     for (int u = blockIdx.x; u < nunits; u += gridDim.x) {
-      const Unit un = decode_unit(a, u);
+      const Unit un = decode_unit(a, sc, u);
       // source rows of this thread's 8 tile rows (token rows for the gathers,
       // routed rows for the rank-space operand)
       int tok[8];
@@ -457,12 +448,12 @@ __global__ void __launch_bounds__(kThreads, 1)
     const int scale_off = 8192 + (kGU ? mat * 256 * ngrp : 0) + (grp * 128 + lrow) * 2;
     Ring rw, q;
     for (int u = blockIdx.x; u < nunits; u += gridDim.x) {
-      const Unit un = decode_unit(a, u);
+      const Unit un = decode_unit(a, sc, u);
       const int n = un.nt * 128 + lrow;     // output feature
       bool ok = true;
       if (a.nkb_lora > 0 && kq == 0 && u + int(gridDim.x) < nunits) {
         // the next unit's LoRA B row into L2 (its rank-space stage comes first)
-        const Unit nx = decode_unit(a, u + gridDim.x);
+        const Unit nx = decode_unit(a, sc, u + gridDim.x);
         const uint16_t* bsrc = (kGU && mat == 1) ? a.b1 : a.b0;
         const uint16_t* row = bsrc + (size_t(nx.e) * a.out_dim + nx.nt * 128 + lrow) * a.r;
         for (int off = 0; off < a.r; off += 64) prefetch_l2(row + off);

@@ -53,26 +53,46 @@ struct Unit {
   int e, nt, mb, rows, base;
 };
 
-__device__ __forceinline__ int total_units(const GemmArgs& a) { return __ldg(a.mb_prefix + a.E) * a.n_tiles; }
+// Expert schedule (m-block prefix and row offsets) as the kernels read it: a
+// copy in shared memory when E <= kSchedSmemE (a unit then decodes in a few
+// shared-memory loads instead of a chain of dependent global loads), else the
+// global arrays.
+constexpr int kSchedSmemE = 512;
+struct Sched {
+  const int32_t* mbp;
+  const int32_t* off;
+};
+
+// Called by every thread before the kernel's first __syncthreads().
+__device__ __forceinline__ Sched load_sched(const GemmArgs& a, int32_t* smem_sched) {
+  if (a.E > kSchedSmemE) return Sched{a.mb_prefix, a.offsets};
+  for (int i = threadIdx.x; i <= a.E; i += blockDim.x) {
+    smem_sched[i] = __ldg(a.mb_prefix + i);
+    smem_sched[kSchedSmemE + 1 + i] = __ldg(a.offsets + i);
+  }
+  return Sched{smem_sched, smem_sched + kSchedSmemE + 1};
+}
+
+__device__ __forceinline__ int total_units(const GemmArgs& a, const Sched& sc) { return sc.mbp[a.E] * a.n_tiles; }
 
 // Units are ordered (expert, n-tile, m-block): m-blocks of one n-tile share a B
 // tile, n-tiles of one m-block share the A rows; neighbours run concurrently.
-__device__ __forceinline__ Unit decode_unit(const GemmArgs& a, int u) {
+__device__ __forceinline__ Unit decode_unit(const GemmArgs& a, const Sched& sc, int u) {
   int lo = 0, hi = a.E;
   while (hi - lo > 1) {
     const int mid = (lo + hi) >> 1;
-    if (__ldg(a.mb_prefix + mid) * a.n_tiles <= u) lo = mid;
+    if (sc.mbp[mid] * a.n_tiles <= u) lo = mid;
     else hi = mid;
   }
   Unit un;
   un.e = lo;
-  const int p0 = __ldg(a.mb_prefix + lo);
-  const int nmb = __ldg(a.mb_prefix + lo + 1) - p0;
+  const int p0 = sc.mbp[lo];
+  const int nmb = sc.mbp[lo + 1] - p0;
   const int idx = u - p0 * a.n_tiles;
   un.nt = idx / nmb;
   un.mb = idx - un.nt * nmb;
-  const int o0 = __ldg(a.offsets + lo);
-  const int cnt = __ldg(a.offsets + lo + 1) - o0;
+  const int o0 = sc.off[lo];
+  const int cnt = sc.off[lo + 1] - o0;
   un.rows = min(kMBlock, cnt - un.mb * kMBlock);
   un.base = o0 + un.mb * kMBlock;
   return un;

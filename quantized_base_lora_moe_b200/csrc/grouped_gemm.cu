@@ -104,6 +104,8 @@ __global__ void __launch_bounds__(kThreads, 1)
 
   const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
+  __shared__ int32_t s_sched[2 * (kSchedSmemE + 1)];
+  const Sched sc = load_sched(a, s_sched);
 
   if (threadIdx.x == 0) {
     for (int i = 0; i < kAStages; ++i) {
@@ -148,7 +150,7 @@ __global__ void __launch_bounds__(kThreads, 1)
   tc_fence_after();
   const uint32_t tmem_base = ctl->tmem_base;
 
-  const int nunits = total_units(a);
+  const int nunits = total_units(a, sc);
   const int nkb = a.nkb_main + a.nkb_lora;
 
   if (warp < 4) {
@@ -156,7 +158,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     const int row = warp * 32 + lane;
     int it = 0;
     for (int u = blockIdx.x; u < nunits; u += gridDim.x, ++it) {
-      const Unit un = decode_unit(a, u);
+      const Unit un = decode_unit(a, sc, u);
       const int ab = it & 1;
       const uint32_t aph = uint32_t(it >> 1) & 1u;
       if (!mbar_wait<128>(&ctl->acc_full[ab], aph, abort_flag, a.status)) break;
@@ -331,7 +333,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       uint32_t last_phase = 0;
       int last_stage = 0;
       for (int u = blockIdx.x; u < nunits; u += gridDim.x) {
-        const Unit un = decode_unit(a, u);
+        const Unit un = decode_unit(a, sc, u);
         bool ok = true;
         for (int km = 0; km < a.nkb_main; ++km) {
           if (!mbar_wait<64>(&ctl->q_empty[q.stage], q.phase ^ 1u, abort_flag, a.status)) { ok = false; break; }
@@ -381,7 +383,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     int pend_stage = -1, pend_b_stage = -1;
     uint32_t pend_phase = 0, pend_b_phase = 0;
     for (int u = blockIdx.x; u < nunits; u += gridDim.x) {
-      const Unit un = decode_unit(a, u);
+      const Unit un = decode_unit(a, sc, u);
       int srow[8];   // gathered source rows of this thread's 8 tile rows
 #pragma unroll
       for (int j = 0; j < 8; ++j) {
@@ -463,7 +465,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     const int nwords = tpr >= 8 ? 1 : 8 / tpr;               // int4 words (8 K values each) per thread
     Ring rb, q;
     for (int u = blockIdx.x; u < nunits; u += gridDim.x) {
-      const Unit un = decode_unit(a, u);
+      const Unit un = decode_unit(a, sc, u);
       bool ok = true;
       for (int kb = 0; kb < nkb; ++kb) {
         const bool waited = kBTma ? mbar_wait<256>(&ctl->b_empty[rb.stage], rb.phase ^ 1u, abort_flag, a.status)
