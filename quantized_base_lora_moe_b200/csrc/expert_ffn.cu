@@ -25,8 +25,9 @@
 //               bank conflicts)
 //   warps 6-9   token producer: cp.async row gathers (rows picked by perm_token)
 //               or TMA tiles of contiguous rows, and the rank-space rows
-//   warps 10-25 weight producer: each thread dequantises 32 K values of one
-//               weight row (int4 -> fp16) into TMEM; LoRA B rows
+//   warps 10-25 weight producer, two groups of 8 warps on alternate stages:
+//               each thread dequantises 64 K values of one weight row
+//               (int4 -> fp16) into TMEM; LoRA B rows
 // TMEM (512 columns): accumulators in [0, 256), 4 weight stages of 64 columns
 // in [256, 512). A pipeline stage pairs one token tile (shared memory) with
 // one weight stage (TMEM): one "full" barrier collects both producers'
@@ -153,12 +154,12 @@ __global__ void __launch_bounds__(kThreads, 1)
 
   if (threadIdx.x == 0) {
     for (int i = 0; i < kStages; ++i) {
-      mbar_init(&ctl->full[i], 128 + kWWarps * 32);   // token producer + weight producer threads
+      mbar_init(&ctl->full[i], 128 + kWWarps * 16);   // token producer + one weight-producer group
       mbar_init(&ctl->empty[i], 1);
     }
     for (int i = 0; i < kQStages; ++i) {
       mbar_init(&ctl->q_full[i], 1);
-      mbar_init(&ctl->q_empty[i], kWWarps * 32);
+      mbar_init(&ctl->q_empty[i], kWWarps * 16);
     }
     for (int i = 0; i < 2; ++i) {
       mbar_init(&ctl->acc_full[i], 1);
@@ -435,69 +436,90 @@ __global__ void __launch_bounds__(kThreads, 1)
       mbar_drain(&ctl->full[pend_stage], pend_phase);
   } else {
     // ------------------------------------------------------------ weight producer
-    // thread = 32 consecutive K values (4 int4 words) of one weight row per stage
+    // Two groups of 8 warps take alternate pipeline stages, so that two stages
+    // are being dequantised at any time (one stage's chain of code read ->
+    // dequant -> TMEM store -> arrive is latency-bound). Within a group, a
+    // thread converts 64 consecutive K values (8 int4 words) of one weight row:
+    // GATEUP: row lrow of the gate (mat 0) or up (mat 1) tile; DOWN: row lrow,
+    // K half kh of the 128-wide stage.
     const int wi = warp - kWWarp0;            // 0..15
+    const int grp = wi >> 3;                  // stage parity handled by this group
+    const int gw = wi & 7;
     const int lrow = 32 * (warp & 3) + lane;  // TMEM lane = feature within the tile
-    const int mat = kGU ? (wi >> 3) : 0;      // GATEUP: 0 gate / 1 up rows
-    const int kq = kGU ? ((wi >> 2) & 1) : (wi >> 2);   // 32-wide K slice within the stage
-    const uint32_t tw = tmem_base + (uint32_t(32 * (warp & 3)) << 16) + kWBase + uint32_t(mat * 32 + kq * 16);
-    // code slice inside a stage (rows of kK/2 bytes, TMA-swizzled at 32 B / 64 B)
-    const int code_off = kGU ? (mat * 4096 + lrow * 32 + ((kq ^ ((lrow >> 2) & 1)) << 4))
-                             : (lrow * 64 + ((kq ^ ((lrow >> 1) & 3)) << 4));
-    const int grp = (ngrp == 1) ? 0 : (32 * kq) / a.g;   // this slice's quantisation group
-    const int scale_off = 8192 + (kGU ? mat * 256 * ngrp : 0) + (grp * 128 + lrow) * 2;
-    Ring rw, q;
+    const int half = gw >> 2;                 // GATEUP: mat; DOWN: K half
+    const uint32_t tw = tmem_base + (uint32_t(32 * (warp & 3)) << 16) + kWBase + uint32_t(half * 32);
+    // the two 16-byte code chunks of this thread inside a stage (TMA-swizzled rows)
+    const int c0_off = kGU ? (half * 4096 + lrow * 32 + ((0 ^ ((lrow >> 2) & 1)) << 4))
+                           : (lrow * 64 + (((2 * half) ^ ((lrow >> 1) & 3)) << 4));
+    const int c1_off = kGU ? (half * 4096 + lrow * 32 + ((1 ^ ((lrow >> 2) & 1)) << 4))
+                           : (lrow * 64 + (((2 * half + 1) ^ ((lrow >> 1) & 3)) << 4));
+    // scale rows of the two 32-wide K halves of this thread's slice
+    const int k0 = kGU ? 0 : 64 * half;
+    const int g_lo = (ngrp == 1) ? 0 : k0 / a.g, g_hi = (ngrp == 1) ? 0 : (k0 + 32) / a.g;
+    const int sbase = 8192 + (kGU ? half * 256 * ngrp : 0);
+    const int s_lo_off = sbase + (g_lo * 128 + lrow) * 2, s_hi_off = sbase + (g_hi * 128 + lrow) * 2;
+    const bool is_up = kGU && half == 1;
+    int n = 0;    // pipeline stage counter of this CTA
+    int m = 0;    // main (code-carrying) stage counter
     for (int u = blockIdx.x; u < nunits; u += gridDim.x) {
       const Unit un = decode_unit(a, sc, u);
-      const int n = un.nt * 128 + lrow;     // output feature
+      const int feat = un.nt * 128 + lrow;  // output feature
       bool ok = true;
-      if (a.nkb_lora > 0 && kq == 0 && u + int(gridDim.x) < nunits) {
+      if (a.nkb_lora > 0 && grp == 0 && (kGU || half == 0) && u + int(gridDim.x) < nunits) {
         // the next unit's LoRA B row into L2 (its rank-space stage comes first)
         const Unit nx = decode_unit(a, sc, u + gridDim.x);
-        const uint16_t* bsrc = (kGU && mat == 1) ? a.b1 : a.b0;
+        const uint16_t* bsrc = is_up ? a.b1 : a.b0;
         const uint16_t* row = bsrc + (size_t(nx.e) * a.out_dim + nx.nt * 128 + lrow) * a.r;
         for (int off = 0; off < a.r; off += 64) prefetch_l2(row + off);
       }
-      for (int kb = 0; kb < nkb; ++kb) {
-        if (!mbar_wait(&ctl->empty[rw.stage], rw.phase ^ 1u, abort_flag, a.status)) { ok = false; break; }
+      for (int kb = 0; kb < nkb; ++kb, ++n) {
+        const bool main_stage = kb >= a.nkb_lora;
+        const int mq = m;
+        if (main_stage) ++m;
+        if ((n & 1) != grp) continue;
+        const int st = n & (kStages - 1);
+        const uint32_t ph = uint32_t(n / kStages) & 1u;
+        if (!mbar_wait(&ctl->empty[st], ph ^ 1u, abort_flag, a.status)) { ok = false; break; }
         tc_fence_after();
-        uint32_t v[16];
-        if (kb < a.nkb_lora) {
+        uint32_t v[32];
+        if (!main_stage) {
           // LoRA B rows as fp16: gate rows hold Bg in K' [0, r), up rows Bu in [r, 2r)
 #pragma unroll
-          for (int c = 0; c < 4; ++c) {
-            const int colk = kb * kK + kq * 32 + c * 8;
-            const int src = (kGU && mat == 1) ? colk - a.r : colk;
+          for (int c = 0; c < 8; ++c) {
+            const int colk = kb * kK + k0 + c * 8;
+            const int src = is_up ? colk - a.r : colk;
             uint4 w4 = make_uint4(0, 0, 0, 0);
             if (src >= 0 && src < a.r) {
-              const uint16_t* bsrc = (kGU && mat == 1) ? a.b1 : a.b0;
+              const uint16_t* bsrc = is_up ? a.b1 : a.b0;
               w4 = bf16x8_to_f16x8(
-                  __ldg(reinterpret_cast<const uint4*>(bsrc + (size_t(un.e) * a.out_dim + n) * a.r + src)));
+                  __ldg(reinterpret_cast<const uint4*>(bsrc + (size_t(un.e) * a.out_dim + feat) * a.r + src)));
             }
             v[4 * c] = w4.x; v[4 * c + 1] = w4.y; v[4 * c + 2] = w4.z; v[4 * c + 3] = w4.w;
           }
         } else {
-          if (!mbar_wait(&ctl->q_full[q.stage], q.phase, abort_flag, a.status)) { ok = false; break; }
-          const uint8_t* qs = q_base + size_t(q.stage) * kQStageBytes;
-          const uint4 wd = *reinterpret_cast<const uint4*>(qs + code_off);
-          const uint32_t s2 = scale_pair(*reinterpret_cast<const uint16_t*>(qs + scale_off));
-          const uint4 d0 = dequant_word(wd.x, s2), d1 = dequant_word(wd.y, s2);
-          const uint4 d2 = dequant_word(wd.z, s2), d3 = dequant_word(wd.w, s2);
+          const int qst = mq % kQStages;
+          const uint32_t qph = uint32_t(mq / kQStages) & 1u;
+          if (!mbar_wait(&ctl->q_full[qst], qph, abort_flag, a.status)) { ok = false; break; }
+          const uint8_t* qs = q_base + size_t(qst) * kQStageBytes;
+          const uint4 wa = *reinterpret_cast<const uint4*>(qs + c0_off);
+          const uint4 wb = *reinterpret_cast<const uint4*>(qs + c1_off);
+          const uint32_t s_lo = scale_pair(*reinterpret_cast<const uint16_t*>(qs + s_lo_off));
+          const uint32_t s_hi = scale_pair(*reinterpret_cast<const uint16_t*>(qs + s_hi_off));
+          const uint32_t wd[8] = {wa.x, wa.y, wa.z, wa.w, wb.x, wb.y, wb.z, wb.w};
+#pragma unroll
+          for (int c = 0; c < 8; ++c) {
+            const uint4 d4 = dequant_word(wd[c], c < 4 ? s_lo : s_hi);
+            v[4 * c] = d4.x; v[4 * c + 1] = d4.y; v[4 * c + 2] = d4.z; v[4 * c + 3] = d4.w;
+          }
           // the code slot's values have been consumed; its next fill is an
           // async-proxy TMA write, hence the proxy fence before handing it back
           fence_proxy_async_smem();
-          mbar_arrive(&ctl->q_empty[q.stage]);
-          q.next<kQStages>();
-          v[0] = d0.x; v[1] = d0.y; v[2] = d0.z; v[3] = d0.w;
-          v[4] = d1.x; v[5] = d1.y; v[6] = d1.z; v[7] = d1.w;
-          v[8] = d2.x; v[9] = d2.y; v[10] = d2.z; v[11] = d2.w;
-          v[12] = d3.x; v[13] = d3.y; v[14] = d3.z; v[15] = d3.w;
+          mbar_arrive(&ctl->q_empty[qst]);
         }
-        tmem_st16(tw + uint32_t(rw.stage) * kWCols, v);
+        tmem_st32(tw + uint32_t(st) * kWCols, v);
         tmem_wait_st();
         tc_fence_before();
-        mbar_arrive(&ctl->full[rw.stage]);
-        rw.next<kStages>();
+        mbar_arrive(&ctl->full[st]);
       }
       if (!ok) break;
     }
