@@ -189,6 +189,8 @@ __global__ void __launch_bounds__(kThreads, 1)
   const uint32_t tmem_base = ctl->tmem_base;
 
   const int nunits = total_units(a, sc);
+  UnitStream us{a.unit_tab, nunits, int(gridDim.x)};
+  us.start(blockIdx.x);
   const int nkb = a.nkb_main + a.nkb_lora;
   // scale rows per K stage (one per quantisation group it spans)
   const int ngrp = a.g >= kK ? 1 : kK / a.g;
@@ -200,7 +202,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     int it = 0;
     EpiSync es{&ctl->epi};
     for (int u = blockIdx.x; u < nunits; u += gridDim.x, ++it) {
-      const Unit un = decode_unit(a, sc, u);
+      const Unit un = us.take(u);
       const int n16 = (un.rows + 15) & ~15;
       if (kGU) {
         if (!mbar_wait<128>(&ctl->acc_full[0], uint32_t(it) & 1u, abort_flag, a.status)) break;
@@ -276,7 +278,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       int it = 0;
       bool ok = true;
       for (int u = blockIdx.x; u < nunits && ok; u += gridDim.x, ++it) {
-        const Unit un = decode_unit(a, sc, u);
+        const Unit un = us.take(u);
         const int n16 = (un.rows + 15) & ~15;
         const uint32_t idesc = idesc_f16(128, n16);
         const int ab = kGU ? 0 : (it & 1);
@@ -339,7 +341,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       uint32_t last_phase = 0;
       int last_stage = 0;
       for (int u = blockIdx.x; u < nunits; u += gridDim.x) {
-        const Unit un = decode_unit(a, sc, u);
+        const Unit un = us.take(u);
         const int nrow0 = un.e * a.out_dim + un.nt * 128;
         bool ok = true;
         for (int km = 0; km < a.nkb_main; ++km) {
@@ -378,7 +380,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     int pend_stage = -1;
     uint32_t pend_phase = 0;
     for (int u = blockIdx.x; u < nunits; u += gridDim.x) {
-      const Unit un = decode_unit(a, sc, u);
+      const Unit un = us.take(u);
       // source rows of this thread's 8 tile rows (token rows for the gathers,
       // routed rows for the rank-space operand)
       int tok[8];
@@ -462,12 +464,12 @@ __global__ void __launch_bounds__(kThreads, 1)
     int n = 0;    // pipeline stage counter of this CTA
     int m = 0;    // main (code-carrying) stage counter
     for (int u = blockIdx.x; u < nunits; u += gridDim.x) {
-      const Unit un = decode_unit(a, sc, u);
+      const Unit un = us.take(u);
       const int feat = un.nt * 128 + lrow;  // output feature
       bool ok = true;
       if (a.nkb_lora > 0 && grp == 0 && (kGU || half == 0) && u + int(gridDim.x) < nunits) {
         // the next unit's LoRA B row into L2 (its rank-space stage comes first)
-        const Unit nx = decode_unit(a, sc, u + gridDim.x);
+        const Unit nx = us.peek();
         const uint16_t* bsrc = is_up ? a.b1 : a.b0;
         const uint16_t* row = bsrc + (size_t(nx.e) * a.out_dim + nx.nt * 128 + lrow) * a.r;
         for (int off = 0; off < a.r; off += 64) prefetch_l2(row + off);

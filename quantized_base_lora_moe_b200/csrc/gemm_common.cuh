@@ -47,6 +47,7 @@ struct GemmArgs {
   const uint16_t* lb0;     // DH / DX rank-space step: A^T sources read transposed (Ad^T | Ag^T)
   const uint16_t* lb1;     // DX: Au^T
   int lb_ld;
+  const int4* unit_tab;    // expert kernels: decoded units {e, n-tile, rows, base}, one per unit
 };
 
 struct Unit {
@@ -97,6 +98,38 @@ __device__ __forceinline__ Unit decode_unit(const GemmArgs& a, const Sched& sc, 
   un.base = o0 + un.mb * kMBlock;
   return un;
 }
+
+// Units read from a table decoded beforehand (unit_table_kernel): one 16-byte
+// load per unit, issued one unit ahead so that its latency stays off the
+// consumer's critical path.
+struct UnitStream {
+  const int4* tab;
+  int total, stride;
+  int4 nxt;
+  __device__ __forceinline__ void start(int u0) { nxt = u0 < total ? __ldg(tab + u0) : make_int4(0, 0, 0, 0); }
+  // unit u (the one loaded last), and the load of unit u + stride
+  __device__ __forceinline__ Unit take(int u) {
+    const int4 c = nxt;
+    if (u + stride < total) nxt = __ldg(tab + u + stride);
+    Unit un;
+    un.e = c.x;
+    un.nt = c.y;
+    un.mb = 0;
+    un.rows = c.z;
+    un.base = c.w;
+    return un;
+  }
+  // the unit after the one last taken (valid when u + stride < total)
+  __device__ __forceinline__ Unit peek() const {
+    Unit un;
+    un.e = nxt.x;
+    un.nt = nxt.y;
+    un.mb = 0;
+    un.rows = nxt.z;
+    un.base = nxt.w;
+    return un;
+  }
+};
 
 struct Ring {
   int stage = 0;

@@ -633,6 +633,28 @@ __global__ void schedule_kernel(const int32_t* __restrict__ offsets, int E, int3
   if (threadIdx.x == nt - 1) mb_prefix[E] = run;
 }
 
+// Decoded work units of one expert-kernel launch: tab[u] = {expert, n-tile,
+// rows, first row} for u < mb_prefix[E] * n_tiles (units ordered as decode_unit).
+__global__ void unit_table_kernel(const int32_t* __restrict__ offsets, const int32_t* __restrict__ mb_prefix, int E,
+                                  int n_tiles, int max_units, int4* __restrict__ tab) {
+  const int u = blockIdx.x * blockDim.x + threadIdx.x;
+  if (u >= max_units || u >= mb_prefix[E] * n_tiles) return;
+  int lo = 0, hi = E;
+  while (hi - lo > 1) {
+    const int mid = (lo + hi) >> 1;
+    if (mb_prefix[mid] * n_tiles <= u) lo = mid;
+    else hi = mid;
+  }
+  const int p0 = mb_prefix[lo];
+  const int nmb = mb_prefix[lo + 1] - p0;
+  const int idx = u - p0 * n_tiles;
+  const int nt = idx / nmb;
+  const int mb = idx - nt * nmb;
+  const int o0 = offsets[lo];
+  const int cnt = offsets[lo + 1] - o0;
+  tab[u] = make_int4(lo, nt, min(kMBlock, cnt - mb * kMBlock), o0 + mb * kMBlock);
+}
+
 // bf16 -> fp16, 8 values per thread; values beyond the fp16 range raise
 // TQP_STATUS_NONFINITE (status may be null).
 __global__ void to_f16_kernel(const uint16_t* __restrict__ x, uint16_t* __restrict__ x16, size_t n8,
@@ -767,6 +789,15 @@ int launch_router_gemm(const uint16_t* x, int T, const tqp_moe_weights* w, float
   return run_gemm<ROUTER>(a, mp, units, s);
 }
 
+// Upper bound on the work units of one expert-kernel launch (128-row blocks x
+// 128-feature tiles of the wider projection).
+static size_t ffn_unit_upper(int T, const tqp_moe_weights* w) {
+  const size_t A = size_t(T) * w->top_k;
+  const size_t mb_upper = (A + kMBlock - 1) / kMBlock + size_t(w->E);
+  const int wide = w->d > w->ffn ? w->d : w->ffn;
+  return mb_upper * size_t((wide + 127) / 128);
+}
+
 size_t ffn_ws_bytes(int T, const tqp_moe_weights* w) {
   const size_t A = size_t(T) * w->top_k;
   size_t b = align_up(size_t(w->E + 1) * 4, 256);              // mb_prefix
@@ -776,6 +807,7 @@ size_t ffn_ws_bytes(int T, const tqp_moe_weights* w) {
     b += align_up(A * w->rank * 2, 256);                        // ha [A][r]
     b += align_up(size_t(w->E) * w->rank * w->ffn * 2, 256);   // Ad^T in fp16
   }
+  b += align_up(ffn_unit_upper(T, w) * 16, 256);                 // decoded units of one expert launch
   return b + 256;
 }
 
@@ -793,8 +825,16 @@ FfnBufs ffn_carve(void* ws, int T, const tqp_moe_weights* w) {
     b.ha = reinterpret_cast<uint16_t*>(p);
     p += align_up(A * w->rank * 2, 256);
     b.adT16 = reinterpret_cast<uint16_t*>(p);
+    p += align_up(size_t(w->E) * w->rank * w->ffn * 2, 256);
   }
+  b.unit_tab = reinterpret_cast<int4*>(p);
   return b;
+}
+
+static int build_unit_table(const GemmArgs& a, int max_units, int4* tab, cudaStream_t s) {
+  if (max_units <= 0) return TQP_OK;
+  unit_table_kernel<<<(max_units + 255) / 256, 256, 0, s>>>(a.offsets, a.mb_prefix, a.E, a.n_tiles, max_units, tab);
+  return cudaGetLastError() == cudaSuccess ? TQP_OK : TQP_ERR_CUDA;
 }
 
 static int to_f16(const uint16_t* src, uint16_t* dst, size_t n, int32_t* status, cudaStream_t s) {
@@ -890,6 +930,10 @@ int launch_grouped_ffn_part(int part, const uint16_t* x, int T, const int32_t* o
               make_map(&mp.m[TS1], CU_TENSOR_MAP_DATA_TYPE_UINT16, w->wscale[1], f, uint64_t(w->E) * (d / w->group),
                        uint64_t(f) * 2, rows_box, ngrp);
     if (!ok) return TQP_ERR_CUDA;
+    if (tm) {
+      if ((rc = build_unit_table(a, mb_upper * a.n_tiles, fb.unit_tab, s)) != TQP_OK) return rc;
+      a.unit_tab = fb.unit_tab;
+    }
     rc = tm ? run_expert_ffn(GATEUP, a, mp, mb_upper * a.n_tiles, s)
             : run_gemm<GATEUP>(a, mp, mb_upper * a.n_tiles, s);
     if (rc != TQP_OK) return rc;
@@ -932,6 +976,10 @@ int launch_grouped_ffn_part(int part, const uint16_t* x, int T, const int32_t* o
               make_map(&mp.m[TS0], CU_TENSOR_MAP_DATA_TYPE_UINT16, w->wscale[2], d, uint64_t(w->E) * (f / w->group),
                        uint64_t(d) * 2, uint32_t(a.ntile), ngrp);
     if (!ok) return TQP_ERR_CUDA;
+    if (tm) {
+      if ((rc = build_unit_table(a, mb_upper * a.n_tiles, fb.unit_tab, s)) != TQP_OK) return rc;
+      a.unit_tab = fb.unit_tab;
+    }
     rc = tm ? run_expert_ffn(DOWN, a, mp, mb_upper * a.n_tiles, s) : run_gemm<DOWN>(a, mp, mb_upper * a.n_tiles, s);
     if (rc != TQP_OK) return rc;
   }

@@ -35,6 +35,7 @@ struct FfnBufs {
   uint16_t* xa;
   uint16_t* ha;
   uint16_t* adT16;   // Ad^T converted to fp16 [E][r][f]
+  int4* unit_tab;    // decoded work units of the current expert-kernel launch
 };
 FfnBufs ffn_carve(void* ws, int T, const tqp_moe_weights* w);
 int launch_grouped_ffn(const uint16_t* x, int T, const int32_t* offsets, const int32_t* perm_token,
