@@ -34,8 +34,10 @@
 // arrivals and one commit per stage frees both.
 //   GATEUP: one accumulator (gate cols [0,128), up [128,256)); a weight stage
 //           holds gate 32 | up 32 columns. The epilogue drains G and U as fp16
-//           into [token][feature] shared-memory tiles, hands TMEM back, and
-//           finishes SwiGLU + 16-byte row stores while the next unit runs.
+//           rows (one feature per thread, 16-byte stores) into shared memory,
+//           hands TMEM back, and then, while the next unit runs, computes
+//           SwiGLU in 32-token chunks transposed through a [token][feature]
+//           tile for 16-byte row stores.
 //   DOWN:   two accumulators of 128 columns; the epilogue drains a whole
 //           accumulator as fp16 into a [token][feature] tile, hands TMEM back,
 //           and then stores 16-byte row pieces.
@@ -64,7 +66,7 @@ constexpr uint32_t kWCols = 64;       // TMEM columns per weight stage
 
 template <int MODE> struct Cfg;
 template <> struct Cfg<GATEUP> {      // K stage 64: 128 token rows x 128 B
-  static constexpr int kK = 64, kXStageBytes = 16384, kStaging = 2 * 128 * kTRow, kQStages = 8;
+  static constexpr int kK = 64, kXStageBytes = 16384, kStaging = (2 * 128 + 32) * kTRow, kQStages = 8;
 };
 template <> struct Cfg<DOWN> {        // K stage 128: two 64-wide swizzled sub-tiles
   static constexpr int kK = 128, kXStageBytes = 32768, kStaging = 128 * kTRow, kQStages = 6;
@@ -207,44 +209,74 @@ __global__ void __launch_bounds__(kThreads, 1)
       if (kGU) {
         if (!mbar_wait<128>(&ctl->acc_full[0], uint32_t(it) & 1u, abort_flag, a.status)) break;
         tc_fence_after();
-        uint8_t* tg = staging;
-        uint8_t* tu = staging + 128 * kTRow;
-        // drain: G and U as fp16 into the [token][feature] tiles
+        // staging: G rows [feature][token] | U rows | chunk tile [32 tokens][feature]
+        uint8_t* grow_s = staging + row * kTRow;
+        uint8_t* urow_s = staging + (128 + row) * kTRow;
+        uint8_t* ht = staging + 256 * kTRow;
+        // drain: this thread's feature row of G and U as fp16 (16-byte stores)
 #pragma unroll 1
-        for (int c = 0; c < n16; c += 16) {
-          float gv[16], uv[16];
-          tmem_ld16(tl + c, gv);
-          tmem_ld16(tl + 128 + c, uv);
-          uint32_t gw[8], uw[8];
+        for (int c = 0; c < n16; c += 32) {
 #pragma unroll
-          for (int j = 0; j < 8; ++j) {
-            gw[j] = f32x2_to_f16x2(gv[2 * j], gv[2 * j + 1]);
-            uw[j] = f32x2_to_f16x2(uv[2 * j], uv[2 * j + 1]);
+          for (int m2 = 0; m2 < 2; ++m2) {
+            float v[32];
+            tmem_ld32(tl + uint32_t(128 * m2 + c), v);
+            uint4* dst = reinterpret_cast<uint4*>((m2 ? urow_s : grow_s) + 2 * c);
+#pragma unroll
+            for (int q4 = 0; q4 < 4; ++q4)
+              dst[q4] = make_uint4(f32x2_to_f16x2(v[8 * q4], v[8 * q4 + 1]), f32x2_to_f16x2(v[8 * q4 + 2], v[8 * q4 + 3]),
+                                   f32x2_to_f16x2(v[8 * q4 + 4], v[8 * q4 + 5]),
+                                   f32x2_to_f16x2(v[8 * q4 + 6], v[8 * q4 + 7]));
           }
-          stage_tokens<8>(tg, c, row, gw);
-          stage_tokens<8>(tu, c, row, uw);
         }
         tc_fence_before();
         mbar_arrive(&ctl->acc_empty[0]);
-        if (!es.sync(abort_flag, a.status)) break;
-        // SwiGLU on 8-feature pieces of the valid tokens, 16-byte row stores,
-        // overlapping the next unit's main loop
+        // SwiGLU per 32-token chunk (own feature row), transposed through the chunk
+        // tile, then 16-byte row stores; overlaps the next unit's main loop
         uint16_t* hout = static_cast<uint16_t*>(a.out) + un.nt * 128;
-        for (int p = threadIdx.x; p < un.rows * 16; p += 128) {
-          const int t = p >> 4, fg = p & 15;
-          const uint4 g = *reinterpret_cast<const uint4*>(tg + t * kTRow + fg * 16);
-          const uint4 uq = *reinterpret_cast<const uint4*>(tu + t * kTRow + fg * 16);
-          const uint4 h = make_uint4(swiglu_pair(g.x, uq.x), swiglu_pair(g.y, uq.y), swiglu_pair(g.z, uq.z),
-                                     swiglu_pair(g.w, uq.w));
-          const size_t grow = size_t(un.base + t);
-          *reinterpret_cast<uint4*>(hout + grow * a.out_ld + fg * 8) = h;
-          if (a.aux) {  // keep the pre-activations for the backward
-            uint16_t* ar = a.aux + grow * (2 * size_t(a.f_dim)) + un.nt * 128 + fg * 8;
-            *reinterpret_cast<uint4*>(ar) = g;
-            *reinterpret_cast<uint4*>(ar + a.f_dim) = uq;
+        bool stop = false;
+#pragma unroll 1
+        for (int c = 0; c < n16; c += 32) {
+          // 16 words (32 tokens) of this thread's staged row
+          auto row_words = [&](const uint8_t* src, uint32_t* w) {
+#pragma unroll
+            for (int q4 = 0; q4 < 4; ++q4) {
+              const uint4 v4 = *reinterpret_cast<const uint4*>(src + 2 * c + 16 * q4);
+              w[4 * q4] = v4.x; w[4 * q4 + 1] = v4.y; w[4 * q4 + 2] = v4.z; w[4 * q4 + 3] = v4.w;
+            }
+          };
+          uint32_t hw[16];
+          {
+            uint32_t gw[16], uw[16];
+            row_words(grow_s, gw);
+            row_words(urow_s, uw);
+#pragma unroll
+            for (int j = 0; j < 16; ++j) hw[j] = swiglu_pair(gw[j], uw[j]);
+          }
+          const int nt = min(32, un.rows - c);
+          // one [32 token][128 feature] chunk through the tile: wait until the tile
+          // is free, transpose into it, wait until complete, 16-byte row stores
+          auto emit = [&](const uint32_t* w, uint16_t* dst, size_t ld) -> bool {
+            if (!es.sync(abort_flag, a.status)) return false;
+            stage_tokens<16>(ht, 0, row, w);
+            if (!es.sync(abort_flag, a.status)) return false;
+            for (int p = threadIdx.x; p < nt * 16; p += 128) {
+              const int t = p >> 4, fg = p & 15;
+              *reinterpret_cast<uint4*>(dst + size_t(un.base + c + t) * ld + fg * 8) =
+                  *reinterpret_cast<const uint4*>(ht + t * kTRow + fg * 16);
+            }
+            return true;
+          };
+          if (!emit(hw, hout, size_t(a.out_ld))) { stop = true; break; }
+          if (a.aux) {  // keep the pre-activations for the backward (re-read from the staged rows)
+            uint16_t* aux = a.aux + un.nt * 128;
+            uint32_t w16[16];
+            row_words(grow_s, w16);
+            if (!emit(w16, aux, 2 * size_t(a.f_dim))) { stop = true; break; }
+            row_words(urow_s, w16);
+            if (!emit(w16, aux + a.f_dim, 2 * size_t(a.f_dim))) { stop = true; break; }
           }
         }
-        if (!es.sync(abort_flag, a.status)) break;  // the tiles are free for the next unit's drain
+        if (stop) break;
       } else {
         const int ab = it & 1;
         if (!mbar_wait<128>(&ctl->acc_full[ab], uint32_t(it >> 1) & 1u, abort_flag, a.status)) break;
