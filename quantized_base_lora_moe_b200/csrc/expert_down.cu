@@ -1,0 +1,390 @@
+// Down projection of the TQP MoE experts with wide token blocks (sm_100a):
+//   O = H_e Wd^T + (s H Ad) Bd
+// ("Train low-rank adapters per expert" over "Quantize base expert weights",
+// Pattern 3; SwiGLU experts, TQP Quantization).
+//
+// As in expert_ffn.cu the contraction runs transposed, D[feature][token] =
+// Wd[feature][:] . H[token][:], with the dequantised 128-feature weight tile as
+// the tcgen05.mma A operand in TMEM and the expert's routed rows as the B
+// operand in shared memory. Here a unit takes up to 256 rows of one expert, so
+// that an expert of the 460-expert configuration (about 214 rows on average)
+// is one block: every MMA is 128 x N x 16 with N up to 256 (half as many MMA
+// instructions per expert as 128-row blocks, each near the compute-bound
+// rate), and every weight tile is dequantised once per expert instead of once
+// per 128-row block.
+//
+// Work unit = (expert e, 128-feature tile, block of up to 256 routed rows),
+// ordered (expert, tile, block) over a persistent grid. Per CTA (1 per SM, 832
+// threads):
+//   warps 0-3   epilogue: drains the accumulator row by row (one feature per
+//               thread, 16-byte shared-memory stores), hands TMEM back, then
+//               sends 32-token chunks out through a [token][feature] tile as
+//               16-byte row pieces
+//   warp  4     TMEM allocation + one thread issuing tcgen05.mma
+//   warp  5     TMA producer of the int4 code / bf16 scale ring (32B-swizzled
+//               code rows, read without bank conflicts)
+//   warps 6-9   token producer: two TMA boxes of 128 rows per 64-wide K stage;
+//               the rank-space rows (s H Ad) by coalesced cp.async
+//   warps 10-25 weight producer, two groups of 8 warps on alternate stages:
+//               each thread dequantises 32 K values of one weight row
+//               (int4 -> fp16) into TMEM; LoRA B rows
+// TMEM (512 columns): one accumulator in [0, 256), 8 weight stages of 32
+// columns (64 K values) in [256, 512). Token ring: 3 stages of 32 KB.
+// Every wait is bounded (tqp_device.cuh); no TMA multicast is used.
+#include <cstdint>
+#include <cuda.h>
+#include <cuda_fp16.h>
+#include <cuda_runtime.h>
+
+#include "expert_common.cuh"
+#include "gemm_common.cuh"
+#include "tqp_device.cuh"
+#include "tqp_launch.h"
+
+namespace tqp {
+namespace down_wide {
+
+constexpr int kWWarp0 = 10;
+constexpr int kWWarps = 16;
+constexpr int kThreads = (kWWarp0 + kWWarps) * 32;
+constexpr int kRows = 256;             // routed rows per unit
+constexpr int kK = 64;                 // K per pipeline stage
+constexpr int kXStages = 3;
+constexpr int kXStageBytes = kRows * kK * 2;   // 256 rows x 128 B, 128B-swizzled
+constexpr int kWStages = 8;
+constexpr uint32_t kWCols = 32;        // TMEM columns per weight stage
+constexpr uint32_t kWBase = 256;
+constexpr int kQStages = 8;
+constexpr int kQStageBytes = 4608;     // 128 rows x 32 B of codes + up to 2 x 128 scales
+constexpr int kDRow = 528;             // drain row: 256 tokens in fp16 + 16 B against bank conflicts
+constexpr int kStaging = 128 * kDRow + 32 * kTRow;
+
+struct Ctl {
+  uint64_t x_full[kXStages], x_empty[kXStages];
+  uint64_t w_full[kWStages], w_empty[kWStages];
+  uint64_t q_full[kQStages], q_empty[kQStages];
+  uint64_t acc_full, acc_empty;
+  uint64_t drain;
+  uint64_t epi;
+  uint32_t tmem_base;
+  int abort_flag;
+};
+
+constexpr size_t kSmemBytes = 1024 + size_t(kXStages) * kXStageBytes + size_t(kQStages) * kQStageBytes +
+                              size_t(kStaging) + sizeof(Ctl);
+static_assert(kSmemBytes + 2 * (kSchedSmemE + 1) * 4 <= 232448, "shared memory budget");
+
+__global__ void __launch_bounds__(kThreads, 1)
+    down_wide_kernel(const GemmArgs a, const __grid_constant__ CUtensorMap tq, const __grid_constant__ CUtensorMap ts,
+                     const __grid_constant__ CUtensorMap th) {
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  uint8_t* x_base = smem;
+  uint8_t* q_base = x_base + size_t(kXStages) * kXStageBytes;
+  uint8_t* staging = q_base + size_t(kQStages) * kQStageBytes;
+  Ctl* ctl = reinterpret_cast<Ctl*>(staging + kStaging);
+  volatile int* abort_flag = &ctl->abort_flag;
+
+  const int warp = threadIdx.x >> 5;
+  const int lane = threadIdx.x & 31;
+  __shared__ int32_t s_sched[2 * (kSchedSmemE + 1)];
+  const Sched sc = load_sched(a, s_sched);
+
+  if (threadIdx.x == 0) {
+    for (int i = 0; i < kXStages; ++i) {
+      mbar_init(&ctl->x_full[i], 128);
+      mbar_init(&ctl->x_empty[i], 1);
+    }
+    for (int i = 0; i < kWStages; ++i) {
+      mbar_init(&ctl->w_full[i], kWWarps * 16);   // one weight-producer group
+      mbar_init(&ctl->w_empty[i], 1);
+    }
+    for (int i = 0; i < kQStages; ++i) {
+      mbar_init(&ctl->q_full[i], 1);
+      mbar_init(&ctl->q_empty[i], kWWarps * 16);
+    }
+    mbar_init(&ctl->acc_full, 1);
+    mbar_init(&ctl->acc_empty, 128);
+    mbar_init(&ctl->drain, 1);
+    mbar_init(&ctl->epi, 128);
+    ctl->abort_flag = 0;
+    fence_barrier_init();
+  }
+  if (warp == 4) {
+    tmem_alloc(&ctl->tmem_base, 512);
+    tmem_relinquish();
+  }
+  if (threadIdx.x == 5 * 32) {
+    prefetch_tmap(&tq);
+    prefetch_tmap(&ts);
+  }
+  if (threadIdx.x == 6 * 32) prefetch_tmap(&th);
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem_base = ctl->tmem_base;
+
+  const int nunits = total_units(a, sc);
+  UnitStream us{a.unit_tab, nunits, int(gridDim.x)};
+  us.start(blockIdx.x);
+  const int nkb = a.nkb_main + a.nkb_lora;
+  const int ngrp = a.g >= kK ? 1 : kK / a.g;   // scale rows per K stage
+
+  if (warp < 4) {
+    // ------------------------------------------------------------ epilogue
+    const int row = warp * 32 + lane;   // feature within the tile = TMEM lane
+    const uint32_t tl = tmem_base + (uint32_t(warp * 32) << 16);
+    uint8_t* drow = staging + row * kDRow;
+    uint8_t* ct = staging + 128 * kDRow;
+    EpiSync es{&ctl->epi};
+    int it = 0;
+    for (int u = blockIdx.x; u < nunits; u += gridDim.x, ++it) {
+      const Unit un = us.take(u);
+      const int n16 = (un.rows + 15) & ~15;
+      if (!mbar_wait<128>(&ctl->acc_full, uint32_t(it) & 1u, abort_flag, a.status)) break;
+      tc_fence_after();
+      // drain this thread's feature row as fp16
+#pragma unroll 1
+      for (int c = 0; c < n16; c += 32) {
+        float v[32];
+        tmem_ld32(tl + uint32_t(c), v);
+        uint4* dst = reinterpret_cast<uint4*>(drow + 2 * c);
+#pragma unroll
+        for (int q4 = 0; q4 < 4; ++q4)
+          dst[q4] = make_uint4(f32x2_to_f16x2(v[8 * q4], v[8 * q4 + 1]), f32x2_to_f16x2(v[8 * q4 + 2], v[8 * q4 + 3]),
+                               f32x2_to_f16x2(v[8 * q4 + 4], v[8 * q4 + 5]),
+                               f32x2_to_f16x2(v[8 * q4 + 6], v[8 * q4 + 7]));
+      }
+      tc_fence_before();
+      mbar_arrive(&ctl->acc_empty);
+      // 32-token chunks through the [token][feature] tile, 16-byte row stores
+      uint16_t* out = static_cast<uint16_t*>(a.out) + un.nt * 128;
+      bool stop = false;
+#pragma unroll 1
+      for (int c = 0; c < n16; c += 32) {
+        uint32_t w[16];
+#pragma unroll
+        for (int q4 = 0; q4 < 4; ++q4) {
+          const uint4 v4 = *reinterpret_cast<const uint4*>(drow + 2 * c + 16 * q4);
+          w[4 * q4] = v4.x; w[4 * q4 + 1] = v4.y; w[4 * q4 + 2] = v4.z; w[4 * q4 + 3] = v4.w;
+        }
+        if (!es.sync(abort_flag, a.status)) { stop = true; break; }   // the chunk tile is free
+        stage_tokens<16>(ct, 0, row, w);
+        if (!es.sync(abort_flag, a.status)) { stop = true; break; }   // the chunk tile is complete
+        const int nt = min(32, un.rows - c);
+        for (int p = threadIdx.x; p < nt * 16; p += 128) {
+          const int t = p >> 4, fg = p & 15;
+          *reinterpret_cast<uint4*>(out + size_t(un.base + c + t) * a.out_ld + fg * 8) =
+              *reinterpret_cast<const uint4*>(ct + t * kTRow + fg * 16);
+        }
+      }
+      if (stop) break;
+    }
+  } else if (warp == 4) {
+    // ------------------------------------------------------------ MMA issuer
+    if (lane == 0) {
+      Ring rx, rw;
+      int it = 0;
+      bool ok = true;
+      for (int u = blockIdx.x; u < nunits && ok; u += gridDim.x, ++it) {
+        const Unit un = us.take(u);
+        const int n16 = (un.rows + 15) & ~15;
+        const uint32_t idesc = idesc_f16(128, n16);
+        if (!mbar_wait(&ctl->acc_empty, (uint32_t(it) & 1u) ^ 1u, abort_flag, a.status)) { ok = false; break; }
+        tc_fence_after();
+        for (int kb = 0; kb < nkb; ++kb) {
+          if (!mbar_wait(&ctl->x_full[rx.stage], rx.phase, abort_flag, a.status) ||
+              !mbar_wait(&ctl->w_full[rw.stage], rw.phase, abort_flag, a.status)) {
+            ok = false;
+            break;
+          }
+          tc_fence_after();
+          const uint64_t bdesc = sdesc_k_sw128(smem_u32(x_base + size_t(rx.stage) * kXStageBytes));
+          const uint32_t wa = tmem_base + kWBase + uint32_t(rw.stage) * kWCols;
+          if (kb >= a.nkb_lora) {
+#pragma unroll
+            for (int kk = 0; kk < 4; ++kk)
+              umma_f16_ts(tmem_base, wa + uint32_t(8 * kk), bdesc + uint64_t(2 * kk), idesc, (kb > 0 || kk > 0) ? 1u : 0u);
+          } else {
+            const int ksteps = (min(kK, a.lora_k - kb * kK) + 15) / 16;
+            for (int kk = 0; kk < ksteps; ++kk)
+              umma_f16_ts(tmem_base, wa + uint32_t(8 * kk), bdesc + uint64_t(2 * kk), idesc, (kb > 0 || kk > 0) ? 1u : 0u);
+          }
+          umma_commit(&ctl->x_empty[rx.stage]);
+          umma_commit(&ctl->w_empty[rw.stage]);
+          rx.next<kXStages>();
+          rw.next<kWStages>();
+        }
+        if (!ok) break;
+        umma_commit(&ctl->acc_full);
+      }
+      umma_commit(&ctl->drain);
+      mbar_wait(&ctl->drain, 0, abort_flag, a.status);
+    }
+    __syncwarp();
+  } else if (warp == 5) {
+    // ------------------------------------------------------------ TMA producer (int4 + scales)
+    if (lane == 0) {
+      Ring q;
+      const uint32_t bytes = uint32_t(4096 + 256 * ngrp);
+      const int gpe = a.in_dim / a.g;
+      int issued = 0;
+      uint32_t last_phase = 0;
+      int last_stage = 0;
+      for (int u = blockIdx.x; u < nunits; u += gridDim.x) {
+        const Unit un = us.take(u);
+        const int nrow0 = un.e * a.out_dim + un.nt * 128;
+        bool ok = true;
+        for (int km = 0; km < a.nkb_main; ++km) {
+          if (!mbar_wait<64>(&ctl->q_empty[q.stage], q.phase ^ 1u, abort_flag, a.status)) { ok = false; break; }
+          uint8_t* qs = q_base + size_t(q.stage) * kQStageBytes;
+          uint64_t* bar = &ctl->q_full[q.stage];
+          mbar_arrive_expect_tx(bar, bytes);
+          tma_load_2d(smem_u32(qs), &tq, bar, km * (kK / 2), nrow0);
+          tma_load_2d(smem_u32(qs + 4096), &ts, bar, un.nt * 128, un.e * gpe + (km * kK) / a.g);
+          ++issued;
+          last_stage = q.stage;
+          last_phase = q.phase;
+          q.next<kQStages>();
+        }
+        if (!ok) break;
+      }
+      if (issued > 0 && *abort_flag) mbar_drain(&ctl->q_full[last_stage], last_phase);
+    }
+  } else if (warp < kWWarp0) {
+    // ------------------------------------------------------------ token producer
+    const int tid = threadIdx.x - 6 * 32;  // 0..127
+    const int chunk = tid & 7;
+    const int row0 = tid >> 3;             // rows row0 + 16 j, j = 0..15
+    Ring rx;
+    int pend_stage = -1;
+    uint32_t pend_phase = 0;
+    for (int u = blockIdx.x; u < nunits; u += gridDim.x) {
+      const Unit un = us.take(u);
+      bool ok = true;
+      for (int kb = 0; kb < nkb; ++kb) {
+        if (!mbar_wait<64>(&ctl->x_empty[rx.stage], rx.phase ^ 1u, abort_flag, a.status)) { ok = false; break; }
+        uint8_t* st = x_base + size_t(rx.stage) * kXStageBytes;
+        uint64_t* full = &ctl->x_full[rx.stage];
+        if (kb < a.nkb_lora) {
+          // rank-space rows s H Ad, zero-filled past lora_k
+          const int colk = kb * kK + chunk * 8;
+          const bool in = colk < a.lora_k;
+          const uint32_t st_u = smem_u32(st);
+#pragma unroll 4
+          for (int j = 0; j < kRows / 16; ++j) {
+            const int r = row0 + 16 * j;
+            if (r < un.rows)
+              cp_async16(st_u + sw128_offset(r, chunk), a.a_lora + size_t(un.base + r) * a.lora_ld + (in ? colk : 0),
+                         in ? 16u : 0u);
+          }
+          cp_async_arrive_noinc(full);
+        } else if (tid == 0) {
+          const int km = kb - a.nkb_lora;
+          mbar_arrive_expect_tx(full, uint32_t(kXStageBytes));
+          tma_load_2d(smem_u32(st), &th, full, km * kK, un.base);
+          tma_load_2d(smem_u32(st + kXStageBytes / 2), &th, full, km * kK, un.base + 128);
+          pend_stage = rx.stage;
+          pend_phase = rx.phase;
+        } else {
+          mbar_arrive(full);
+        }
+        rx.next<kXStages>();
+      }
+      if (!ok) break;
+    }
+    cp_async_wait_all();
+    if (tid == 0 && *abort_flag && pend_stage >= 0) mbar_drain(&ctl->x_full[pend_stage], pend_phase);
+  } else {
+    // ------------------------------------------------------------ weight producer
+    const int wi = warp - kWWarp0;            // 0..15
+    const int grp = wi >> 3;                  // stage parity handled by this group
+    const int kh = (wi >> 2) & 1;             // 32-wide K half of the 64-wide stage
+    const int lrow = 32 * (warp & 3) + lane;  // TMEM lane = feature within the tile
+    const uint32_t tw = tmem_base + (uint32_t(32 * (warp & 3)) << 16) + kWBase + uint32_t(kh * 16);
+    const int code_off = lrow * 32 + ((kh ^ ((lrow >> 2) & 1)) << 4);   // 32B-swizzled code rows
+    const int scale_off = 4096 + (((ngrp == 2) ? kh : 0) * 128 + lrow) * 2;
+    int n = 0;   // stage counter
+    int m = 0;   // main (code-carrying) stage counter
+    for (int u = blockIdx.x; u < nunits; u += gridDim.x) {
+      const Unit un = us.take(u);
+      const int feat = un.nt * 128 + lrow;
+      bool ok = true;
+      if (a.nkb_lora > 0 && grp == 0 && kh == 0 && u + int(gridDim.x) < nunits) {
+        // the next unit's LoRA B row into L2 (its rank-space stage comes first)
+        const Unit nx = us.peek();
+        const uint16_t* row = a.b0 + (size_t(nx.e) * a.out_dim + nx.nt * 128 + lrow) * a.r;
+        for (int off = 0; off < a.r; off += 64) prefetch_l2(row + off);
+      }
+      for (int kb = 0; kb < nkb; ++kb, ++n) {
+        const bool main_stage = kb >= a.nkb_lora;
+        const int mq = m;
+        if (main_stage) ++m;
+        if ((n & 1) != grp) continue;
+        const int st = n % kWStages;
+        const uint32_t ph = uint32_t(n / kWStages) & 1u;
+        if (!mbar_wait(&ctl->w_empty[st], ph ^ 1u, abort_flag, a.status)) { ok = false; break; }
+        tc_fence_after();
+        uint32_t v[16];
+        if (!main_stage) {
+#pragma unroll
+          for (int c = 0; c < 4; ++c) {
+            const int colk = kb * kK + kh * 32 + c * 8;
+            uint4 w4 = make_uint4(0, 0, 0, 0);
+            if (colk < a.r)
+              w4 = bf16x8_to_f16x8(
+                  __ldg(reinterpret_cast<const uint4*>(a.b0 + (size_t(un.e) * a.out_dim + feat) * a.r + colk)));
+            v[4 * c] = w4.x; v[4 * c + 1] = w4.y; v[4 * c + 2] = w4.z; v[4 * c + 3] = w4.w;
+          }
+        } else {
+          const int qst = mq % kQStages;
+          const uint32_t qph = uint32_t(mq / kQStages) & 1u;
+          if (!mbar_wait(&ctl->q_full[qst], qph, abort_flag, a.status)) { ok = false; break; }
+          const uint8_t* qs = q_base + size_t(qst) * kQStageBytes;
+          const uint4 wd = *reinterpret_cast<const uint4*>(qs + code_off);
+          const uint32_t s2 = scale_pair(*reinterpret_cast<const uint16_t*>(qs + scale_off));
+          const uint4 d0 = dequant_word(wd.x, s2), d1 = dequant_word(wd.y, s2);
+          const uint4 d2 = dequant_word(wd.z, s2), d3 = dequant_word(wd.w, s2);
+          // the code slot's values have been consumed; its next fill is an
+          // async-proxy TMA write, hence the proxy fence before handing it back
+          fence_proxy_async_smem();
+          mbar_arrive(&ctl->q_empty[qst]);
+          v[0] = d0.x; v[1] = d0.y; v[2] = d0.z; v[3] = d0.w;
+          v[4] = d1.x; v[5] = d1.y; v[6] = d1.z; v[7] = d1.w;
+          v[8] = d2.x; v[9] = d2.y; v[10] = d2.z; v[11] = d2.w;
+          v[12] = d3.x; v[13] = d3.y; v[14] = d3.z; v[15] = d3.w;
+        }
+        tmem_st16(tw + uint32_t(st) * kWCols, v);
+        tmem_wait_st();
+        tc_fence_before();
+        mbar_arrive(&ctl->w_full[st]);
+      }
+      if (!ok) break;
+    }
+  }
+
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 4) {
+    tc_fence_after();
+    tmem_dealloc(tmem_base, 512);
+  }
+}
+
+}  // namespace down_wide
+
+int run_expert_down_wide(const GemmArgs& a, const Maps& mp, int units_upper, cudaStream_t s) {
+  static bool attr_set = false;
+  if (!attr_set) {
+    if (cudaFuncSetAttribute(down_wide::down_wide_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                             int(down_wide::kSmemBytes)) != cudaSuccess)
+      return TQP_ERR_CUDA;
+    attr_set = true;
+  }
+  const int grid = units_upper < num_sms() ? (units_upper > 0 ? units_upper : 1) : num_sms();
+  down_wide::down_wide_kernel<<<grid, down_wide::kThreads, down_wide::kSmemBytes, s>>>(a, mp.m[TQ0], mp.m[TS0],
+                                                                                        mp.m[TA]);
+  return cudaGetLastError() == cudaSuccess ? TQP_OK : TQP_ERR_CUDA;
+}
+
+}  // namespace tqp

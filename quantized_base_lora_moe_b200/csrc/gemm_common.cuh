@@ -189,4 +189,7 @@ enum { TQ0 = 0, TQ1 = 1, TS0 = 2, TS1 = 3, TA = 4, TB0 = 5, TB1 = 6 };
 // (expert_ffn.cu): mode GATEUP or DOWN.
 int run_expert_ffn(int mode, const GemmArgs& a, const Maps& mp, int units_upper, cudaStream_t s);
 
+// Down projection with blocks of up to 256 routed rows (expert_down.cu).
+int run_expert_down_wide(const GemmArgs& a, const Maps& mp, int units_upper, cudaStream_t s);
+
 }  // namespace tqp

@@ -597,15 +597,16 @@ __global__ void __launch_bounds__(kThreads, 1)
 // small helper kernels
 // ----------------------------------------------------------------------------
 
-// mb_prefix[e] = sum_{e' < e} ceil(count(e') / kMBlock), one block.
-__global__ void schedule_kernel(const int32_t* __restrict__ offsets, int E, int32_t* __restrict__ mb_prefix) {
+// mb_prefix[e] = sum_{e' < e} ceil(count(e') / block), one thread block.
+__global__ void schedule_kernel(const int32_t* __restrict__ offsets, int E, int32_t* __restrict__ mb_prefix,
+                                int block) {
   __shared__ int32_t warp_sums[32];
   const int nt = blockDim.x;
   const int per = (E + nt - 1) / nt;
   const int lo = threadIdx.x * per;
   const int hi = min(E, lo + per);
   int local = 0;
-  for (int e = lo; e < hi; ++e) local += (offsets[e + 1] - offsets[e] + kMBlock - 1) / kMBlock;
+  for (int e = lo; e < hi; ++e) local += (offsets[e + 1] - offsets[e] + block - 1) / block;
   const int lane = threadIdx.x & 31, wid = threadIdx.x >> 5;
   int v = local;
 #pragma unroll
@@ -628,15 +629,16 @@ __global__ void schedule_kernel(const int32_t* __restrict__ offsets, int E, int3
   int run = v - local + (wid > 0 ? warp_sums[wid - 1] : 0);
   for (int e = lo; e < hi; ++e) {
     mb_prefix[e] = run;
-    run += (offsets[e + 1] - offsets[e] + kMBlock - 1) / kMBlock;
+    run += (offsets[e + 1] - offsets[e] + block - 1) / block;
   }
   if (threadIdx.x == nt - 1) mb_prefix[E] = run;
 }
 
 // Decoded work units of one expert-kernel launch: tab[u] = {expert, n-tile,
-// rows, first row} for u < mb_prefix[E] * n_tiles (units ordered as decode_unit).
+// rows, first row} for u < mb_prefix[E] * n_tiles, with blocks of `block` rows
+// (units ordered as decode_unit).
 __global__ void unit_table_kernel(const int32_t* __restrict__ offsets, const int32_t* __restrict__ mb_prefix, int E,
-                                  int n_tiles, int max_units, int4* __restrict__ tab) {
+                                  int n_tiles, int block, int max_units, int4* __restrict__ tab) {
   const int u = blockIdx.x * blockDim.x + threadIdx.x;
   if (u >= max_units || u >= mb_prefix[E] * n_tiles) return;
   int lo = 0, hi = E;
@@ -652,7 +654,7 @@ __global__ void unit_table_kernel(const int32_t* __restrict__ offsets, const int
   const int mb = idx - nt * nmb;
   const int o0 = offsets[lo];
   const int cnt = offsets[lo + 1] - o0;
-  tab[u] = make_int4(lo, nt, min(kMBlock, cnt - mb * kMBlock), o0 + mb * kMBlock);
+  tab[u] = make_int4(lo, nt, min(block, cnt - mb * block), o0 + mb * block);
 }
 
 // bf16 -> fp16, 8 values per thread; values beyond the fp16 range raise
@@ -800,7 +802,7 @@ static size_t ffn_unit_upper(int T, const tqp_moe_weights* w) {
 
 size_t ffn_ws_bytes(int T, const tqp_moe_weights* w) {
   const size_t A = size_t(T) * w->top_k;
-  size_t b = align_up(size_t(w->E + 1) * 4, 256);              // mb_prefix
+  size_t b = 2 * align_up(size_t(w->E + 1) * 4, 256);          // block prefixes (128- and 256-row blocks)
   b += align_up(size_t(T) * w->d * 2, 256);                    // x in fp16
   if (w->rank > 0) {
     b += align_up(A * 2 * w->rank * 2, 256);                    // xa [A][2r]
@@ -817,6 +819,8 @@ FfnBufs ffn_carve(void* ws, int T, const tqp_moe_weights* w) {
   FfnBufs b{};
   b.mb_prefix = reinterpret_cast<int32_t*>(p);
   p += align_up(size_t(w->E + 1) * 4, 256);
+  b.mb_prefix256 = reinterpret_cast<int32_t*>(p);
+  p += align_up(size_t(w->E + 1) * 4, 256);
   b.x16 = reinterpret_cast<uint16_t*>(p);
   p += align_up(size_t(T) * w->d * 2, 256);
   if (w->rank > 0) {
@@ -831,9 +835,10 @@ FfnBufs ffn_carve(void* ws, int T, const tqp_moe_weights* w) {
   return b;
 }
 
-static int build_unit_table(const GemmArgs& a, int max_units, int4* tab, cudaStream_t s) {
+static int build_unit_table(const GemmArgs& a, int block, int max_units, int4* tab, cudaStream_t s) {
   if (max_units <= 0) return TQP_OK;
-  unit_table_kernel<<<(max_units + 255) / 256, 256, 0, s>>>(a.offsets, a.mb_prefix, a.E, a.n_tiles, max_units, tab);
+  unit_table_kernel<<<(max_units + 255) / 256, 256, 0, s>>>(a.offsets, a.mb_prefix, a.E, a.n_tiles, block, max_units,
+                                                           tab);
   return cudaGetLastError() == cudaSuccess ? TQP_OK : TQP_ERR_CUDA;
 }
 
@@ -858,7 +863,8 @@ int launch_grouped_ffn_part(int part, const uint16_t* x, int T, const int32_t* o
   const int d = w->d, f = w->ffn, r = w->rank;
   int rc;
   if (part == 0) {
-    schedule_kernel<<<1, 1024, 0, s>>>(offsets, w->E, fb.mb_prefix);
+    schedule_kernel<<<1, 1024, 0, s>>>(offsets, w->E, fb.mb_prefix, kMBlock);
+    schedule_kernel<<<1, 1024, 0, s>>>(offsets, w->E, fb.mb_prefix256, 256);
     if (cudaGetLastError() != cudaSuccess) return TQP_ERR_CUDA;
     if ((rc = to_f16(x, fb.x16, size_t(T) * d, status, s)) != TQP_OK) return rc;
     if (r > 0 && (rc = to_f16(w->lora_a[2], fb.adT16, size_t(w->E) * r * f, nullptr, s)) != TQP_OK) return rc;
@@ -931,7 +937,7 @@ int launch_grouped_ffn_part(int part, const uint16_t* x, int T, const int32_t* o
                        uint64_t(f) * 2, rows_box, ngrp);
     if (!ok) return TQP_ERR_CUDA;
     if (tm) {
-      if ((rc = build_unit_table(a, mb_upper * a.n_tiles, fb.unit_tab, s)) != TQP_OK) return rc;
+      if ((rc = build_unit_table(a, kMBlock, mb_upper * a.n_tiles, fb.unit_tab, s)) != TQP_OK) return rc;
       a.unit_tab = fb.unit_tab;
     }
     rc = tm ? run_expert_ffn(GATEUP, a, mp, mb_upper * a.n_tiles, s)
@@ -952,14 +958,14 @@ int launch_grouped_ffn_part(int part, const uint16_t* x, int T, const int32_t* o
       return TQP_ERR_CUDA;
     if ((rc = run_gemm<LORA_HA>(a, mp, mb_upper, s)) != TQP_OK) return rc;
   }
-  if (part == 3) {  // O = H Wd^T + (s H Ad) Bd
+  if (part == 3) {  // O = H Wd^T + (s H Ad) Bd: blocks of up to 256 rows, weights in TMEM (expert_down.cu)
     GemmArgs a = base;
-    const int kst = tm ? 128 : 64;   // K stage
-    a.nkb_main = f / kst;
-    a.nkb_lora = r > 0 ? (r + kst - 1) / kst : 0;
+    a.mb_prefix = fb.mb_prefix256;
+    a.nkb_main = f / 64;
+    a.nkb_lora = r > 0 ? 1 : 0;   // r <= 64: one 64-wide rank-space stage
     a.lora_k = r;
-    a.ntile = tm ? 128 : ((d % 256 == 0) ? 256 : 128);
-    a.n_tiles = d / a.ntile;
+    a.ntile = 128;
+    a.n_tiles = d / 128;
     a.in_dim = f;
     a.out_dim = d;
     a.a_lora = fb.ha;
@@ -968,20 +974,18 @@ int launch_grouped_ffn_part(int part, const uint16_t* x, int T, const int32_t* o
     a.out = out_perm;
     a.out_ld = d;
     a.n_valid = d;
-    const int ngrp = w->group >= kst ? 1 : kst / w->group;
+    const int ngrp = w->group >= 64 ? 1 : 64 / w->group;
     Maps mp{};
     bool ok = make_tile_map(&mp.m[TA], h, uint64_t(A), uint64_t(f), 128) &&
-              make_map(&mp.m[TQ0], CU_TENSOR_MAP_DATA_TYPE_UINT8, w->wq[2], f / 2, uint64_t(w->E) * d, f / 2,
-                       uint32_t(kst / 2), uint32_t(a.ntile), tm ? 64 : 0) &&
+              make_map(&mp.m[TQ0], CU_TENSOR_MAP_DATA_TYPE_UINT8, w->wq[2], f / 2, uint64_t(w->E) * d, f / 2, 32, 128,
+                       32) &&
               make_map(&mp.m[TS0], CU_TENSOR_MAP_DATA_TYPE_UINT16, w->wscale[2], d, uint64_t(w->E) * (f / w->group),
-                       uint64_t(d) * 2, uint32_t(a.ntile), ngrp);
+                       uint64_t(d) * 2, 128, ngrp);
     if (!ok) return TQP_ERR_CUDA;
-    if (tm) {
-      if ((rc = build_unit_table(a, mb_upper * a.n_tiles, fb.unit_tab, s)) != TQP_OK) return rc;
-      a.unit_tab = fb.unit_tab;
-    }
-    rc = tm ? run_expert_ffn(DOWN, a, mp, mb_upper * a.n_tiles, s) : run_gemm<DOWN>(a, mp, mb_upper * a.n_tiles, s);
-    if (rc != TQP_OK) return rc;
+    const int units_upper = int((A + 255) / 256 + w->E) * a.n_tiles;
+    if ((rc = build_unit_table(a, 256, units_upper, fb.unit_tab, s)) != TQP_OK) return rc;
+    a.unit_tab = fb.unit_tab;
+    if ((rc = run_expert_down_wide(a, mp, units_upper, s)) != TQP_OK) return rc;
   }
   return TQP_OK;
 }

@@ -30,7 +30,8 @@ size_t ffn_ws_bytes(int T, const tqp_moe_weights* w);
 // per-expert m-block prefix, x in fp16, s*X[Ag|Au] [A][2r] and s*H*Ad [A][r] (fp16),
 // and Ad^T in fp16.
 struct FfnBufs {
-  int32_t* mb_prefix;
+  int32_t* mb_prefix;      // per-expert prefix of 128-row blocks
+  int32_t* mb_prefix256;   // per-expert prefix of 256-row blocks (the down projection)
   uint16_t* x16;
   uint16_t* xa;
   uint16_t* ha;
