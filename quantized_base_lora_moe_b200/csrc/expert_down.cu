@@ -14,12 +14,14 @@
 // per 128-row block.
 //
 // Work unit = (expert e, 128-feature tile, block of up to 256 routed rows),
-// ordered (expert, tile, block) over a persistent grid. Per CTA (1 per SM, 832
+// ordered (expert, tile, block) over a persistent grid. Per CTA (1 per SM, 960
 // threads):
-//   warps 0-3   epilogue: drains the accumulator row by row (one feature per
-//               thread, 16-byte shared-memory stores), hands TMEM back, then
-//               sends 32-token chunks out through a [token][feature] tile as
-//               16-byte row pieces
+//   warps 0-3, 26-29  epilogue, two groups taking alternate 32-token chunks:
+//               drain the accumulator row by row (one feature per thread,
+//               16-byte shared-memory stores), hand TMEM back, then send their
+//               chunks out through a [token][feature] tile per group as
+//               16-byte row pieces (the single accumulator is released after
+//               half the drain time)
 //   warp  4     TMEM allocation + one thread issuing tcgen05.mma
 //   warp  5     TMA producer of the int4 code / bf16 scale ring (32B-swizzled
 //               code rows, read without bank conflicts)
@@ -46,7 +48,8 @@ namespace down_wide {
 
 constexpr int kWWarp0 = 10;
 constexpr int kWWarps = 16;
-constexpr int kThreads = (kWWarp0 + kWWarps) * 32;
+constexpr int kEpi1Warp0 = kWWarp0 + kWWarps;   // second epilogue group (4 warps)
+constexpr int kThreads = (kEpi1Warp0 + 4) * 32;
 constexpr int kRows = 256;             // routed rows per unit
 constexpr int kK = 64;                 // K per pipeline stage
 constexpr int kXStages = 3;
@@ -57,7 +60,7 @@ constexpr uint32_t kWBase = 256;
 constexpr int kQStages = 8;
 constexpr int kQStageBytes = 4608;     // 128 rows x 32 B of codes + up to 2 x 128 scales
 constexpr int kDRow = 528;             // drain row: 256 tokens in fp16 + 16 B against bank conflicts
-constexpr int kStaging = 128 * kDRow + 32 * kTRow;
+constexpr int kStaging = 128 * kDRow + 2 * 32 * kTRow;   // drain rows + one chunk tile per epilogue group
 
 struct Ctl {
   uint64_t x_full[kXStages], x_empty[kXStages];
@@ -65,7 +68,7 @@ struct Ctl {
   uint64_t q_full[kQStages], q_empty[kQStages];
   uint64_t acc_full, acc_empty;
   uint64_t drain;
-  uint64_t epi;
+  uint64_t epi[2];
   uint32_t tmem_base;
   int abort_flag;
 };
@@ -104,9 +107,10 @@ __global__ void __launch_bounds__(kThreads, 1)
       mbar_init(&ctl->q_empty[i], kWWarps * 16);
     }
     mbar_init(&ctl->acc_full, 1);
-    mbar_init(&ctl->acc_empty, 128);
+    mbar_init(&ctl->acc_empty, 256);   // both epilogue groups
     mbar_init(&ctl->drain, 1);
-    mbar_init(&ctl->epi, 128);
+    mbar_init(&ctl->epi[0], 128);
+    mbar_init(&ctl->epi[1], 128);
     ctl->abort_flag = 0;
     fence_barrier_init();
   }
@@ -130,22 +134,24 @@ __global__ void __launch_bounds__(kThreads, 1)
   const int nkb = a.nkb_main + a.nkb_lora;
   const int ngrp = a.g >= kK ? 1 : kK / a.g;   // scale rows per K stage
 
-  if (warp < 4) {
+  if (warp < 4 || warp >= kEpi1Warp0) {
     // ------------------------------------------------------------ epilogue
-    const int row = warp * 32 + lane;   // feature within the tile = TMEM lane
-    const uint32_t tl = tmem_base + (uint32_t(warp * 32) << 16);
+    const int eg = warp < 4 ? 0 : 1;          // group: 32-token chunks with (c / 32) % 2 == eg
+    const int row = 32 * (warp & 3) + lane;   // feature within the tile = TMEM lane
+    const int etid = row;                     // thread index within the group
+    const uint32_t tl = tmem_base + (uint32_t(32 * (warp & 3)) << 16);
     uint8_t* drow = staging + row * kDRow;
-    uint8_t* ct = staging + 128 * kDRow;
-    EpiSync es{&ctl->epi};
+    uint8_t* ct = staging + 128 * kDRow + eg * 32 * kTRow;
+    EpiSync es{&ctl->epi[eg]};
     int it = 0;
     for (int u = blockIdx.x; u < nunits; u += gridDim.x, ++it) {
       const Unit un = us.take(u);
       const int n16 = (un.rows + 15) & ~15;
       if (!mbar_wait<128>(&ctl->acc_full, uint32_t(it) & 1u, abort_flag, a.status)) break;
       tc_fence_after();
-      // drain this thread's feature row as fp16
+      // drain this group's chunks of this thread's feature row as fp16
 #pragma unroll 1
-      for (int c = 0; c < n16; c += 32) {
+      for (int c = 32 * eg; c < n16; c += 64) {
         float v[32];
         tmem_ld32(tl + uint32_t(c), v);
         uint4* dst = reinterpret_cast<uint4*>(drow + 2 * c);
@@ -157,11 +163,11 @@ __global__ void __launch_bounds__(kThreads, 1)
       }
       tc_fence_before();
       mbar_arrive(&ctl->acc_empty);
-      // 32-token chunks through the [token][feature] tile, 16-byte row stores
+      // this group's 32-token chunks through its [token][feature] tile, 16-byte row stores
       uint16_t* out = static_cast<uint16_t*>(a.out) + un.nt * 128;
       bool stop = false;
 #pragma unroll 1
-      for (int c = 0; c < n16; c += 32) {
+      for (int c = 32 * eg; c < n16; c += 64) {
         uint32_t w[16];
 #pragma unroll
         for (int q4 = 0; q4 < 4; ++q4) {
@@ -172,7 +178,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         stage_tokens<16>(ct, 0, row, w);
         if (!es.sync(abort_flag, a.status)) { stop = true; break; }   // the chunk tile is complete
         const int nt = min(32, un.rows - c);
-        for (int p = threadIdx.x; p < nt * 16; p += 128) {
+        for (int p = etid; p < nt * 16; p += 128) {
           const int t = p >> 4, fg = p & 15;
           *reinterpret_cast<uint4*>(out + size_t(un.base + c + t) * a.out_ld + fg * 8) =
               *reinterpret_cast<const uint4*>(ct + t * kTRow + fg * 16);
