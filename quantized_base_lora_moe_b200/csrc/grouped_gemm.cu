@@ -44,12 +44,29 @@ constexpr int kQStages = 8;           // int4 codes + scales from DRAM: deepest 
 constexpr int kAStageBytes = 16384;   // 128 rows x 64 K x 2 B
 constexpr int kBStageBytes = 32768;   // up to 256 rows x 64 K x 2 B
 constexpr int kQStageBytes = 9216;    // up to 8192 B of codes + 1024 B of scales
+constexpr int kBStagesMax = 8;
+
+// B ring of one mode. The dequantising modes keep two slots of 32 KB. The modes
+// whose B tile comes by TMA (rank-space GEMMs, router) read no codes, so their
+// ring also takes the code region and runs deeper: two TMA fills in flight
+// cannot cover the L2/DRAM latency of a 4-MMA stage, and the A producer's TMA
+// issuer waits on the same ring.
+template <int MODE>
+struct BRing {
+  static constexpr bool kTma = (MODE == LORA_XA || MODE == LORA_HA || MODE == ROUTER);
+  static constexpr int kStages = !kTma ? kBStages : (MODE == ROUTER ? 4 : 8);
+  // LORA_XA: 2r rows (r <= 64), LORA_HA: r rows, ROUTER: up to 256 rows, x 128 B
+  static constexpr int kBytes = (kTma && MODE != ROUTER) ? 16384 : kBStageBytes;
+  static_assert(kStages <= kBStagesMax, "B ring barriers");
+  static_assert(size_t(kStages) * kBytes <= size_t(kBStages) * kBStageBytes + (kTma ? size_t(kQStages) * kQStageBytes : 0),
+                "B ring footprint");
+};
 
 struct SmemCtl {
   uint64_t a_full[kAStages];
   uint64_t a_empty[kAStages];
-  uint64_t b_full[kBStages];
-  uint64_t b_empty[kBStages];
+  uint64_t b_full[kBStagesMax];
+  uint64_t b_empty[kBStagesMax];
   uint64_t q_full[kQStages];
   uint64_t q_empty[kQStages];
   uint64_t acc_full[2];
@@ -94,6 +111,9 @@ __global__ void __launch_bounds__(kThreads, 1)
   constexpr bool kATma = (MODE == DOWN || MODE == LORA_HA || MODE == ROUTER || kTrans);
   constexpr bool kBTma = (MODE == LORA_XA || MODE == LORA_HA || MODE == ROUTER);
   constexpr bool kBf16 = (MODE == LORA_XA || MODE == ROUTER);
+  constexpr int kBSt = BRing<MODE>::kStages;
+  constexpr int kBStride = BRing<MODE>::kBytes;
+  static_assert(BRing<MODE>::kTma == kBTma, "B ring mode");
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   uint8_t* a_base = smem;
@@ -112,7 +132,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       mbar_init(&ctl->a_full[i], 128);
       mbar_init(&ctl->a_empty[i], 1);
     }
-    for (int i = 0; i < kBStages; ++i) {
+    for (int i = 0; i < kBSt; ++i) {
       mbar_init(&ctl->b_full[i], kBTma ? 257 : 256);   // + the TMA issuer's arrival
       mbar_init(&ctl->b_empty[i], 1);
     }
@@ -303,13 +323,13 @@ __global__ void __launch_bounds__(kThreads, 1)
           tc_fence_after();
           const int ksteps = (kb < a.nkb_lora) ? (min(64, a.lora_k - kb * 64) + 15) / 16 : 4;
           const uint64_t adesc = sdesc_k_sw128(smem_u32(a_base + size_t(ra.stage) * kAStageBytes));
-          const uint64_t bdesc = sdesc_k_sw128(smem_u32(b_base + size_t(rb.stage) * kBStageBytes));
+          const uint64_t bdesc = sdesc_k_sw128(smem_u32(b_base + size_t(rb.stage) * kBStride));
           for (int kk = 0; kk < ksteps; ++kk)
             umma_bf16(dt, adesc + uint64_t(2 * kk), bdesc + uint64_t(2 * kk), idesc, (kb > 0 || kk > 0) ? 1u : 0u);
           umma_commit(&ctl->a_empty[ra.stage]);
           umma_commit(&ctl->b_empty[rb.stage]);
           ra.next<kAStages>();
-          rb.next<kBStages>();
+          rb.next<kBSt>();
         }
         if (!ok) break;
         umma_commit(&ctl->acc_full[ab]);
@@ -414,7 +434,7 @@ __global__ void __launch_bounds__(kThreads, 1)
             // the B tile of a rank-space GEMM / the router comes by TMA as well
             if (!mbar_wait<64>(&ctl->b_empty[rb.stage], rb.phase ^ 1u, abort_flag, a.status)) { ok = false; break; }
             uint64_t* bfull = &ctl->b_full[rb.stage];
-            const uint32_t bst_u = smem_u32(b_base + size_t(rb.stage) * kBStageBytes);
+            const uint32_t bst_u = smem_u32(b_base + size_t(rb.stage) * kBStride);
             mbar_arrive_expect_tx(bfull, b_bytes);
             pend_b_stage = rb.stage;
             pend_b_phase = rb.phase;
@@ -446,7 +466,7 @@ __global__ void __launch_bounds__(kThreads, 1)
             }
             cp_async_arrive_noinc(full);
           }
-          if (kBTma) rb.next<kBStages>();
+          if (kBTma) rb.next<kBSt>();
         }
         ra.next<kAStages>();
       }
@@ -471,7 +491,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         const bool waited = kBTma ? mbar_wait<256>(&ctl->b_empty[rb.stage], rb.phase ^ 1u, abort_flag, a.status)
                                   : mbar_wait(&ctl->b_empty[rb.stage], rb.phase ^ 1u, abort_flag, a.status);
         if (!waited) { ok = false; break; }
-        uint8_t* bst = b_base + size_t(rb.stage) * kBStageBytes;
+        uint8_t* bst = b_base + size_t(rb.stage) * kBStride;
         uint64_t* full = &ctl->b_full[rb.stage];
         if (kb < a.nkb_lora) {
           if (MODE == GATEUP || MODE == DOWN) {
@@ -579,7 +599,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         } else {
           mbar_arrive(full);  // the B tile arrives by TMA (LORA_XA, LORA_HA, ROUTER)
         }
-        rb.next<kBStages>();
+        rb.next<kBSt>();
       }
       if (!ok) break;
     }
