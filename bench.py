@@ -17,6 +17,9 @@ batch copied from pinned host memory and the layer output copied back inside
 the timed region. `cpu_baseline` times the fp64 oracle on a bounded sample of
 the same workload on this host's cores. `--impl reference` times that oracle
 as the reference arm (there is no other implementation of this layer).
+On one GPU with the full config, `rev_block` adds the reversible block built
+from two such layers (coupling forward, its inverse, adapter backward), each
+call timed with CUDA events outside the headline region.
 """
 from __future__ import annotations
 
@@ -178,6 +181,65 @@ class ClockSampler:
 # ---------------------------------------------------------------- GPU arm
 
 
+def time_rev_block(L_F, dev, steps: int, warmup: int, flush) -> dict:
+    """The reversible block at full size, timed per call with CUDA events.
+
+    F is the bench's 460-expert layer, G a second independent instance (seed 1);
+    streams x1, x2 of T x d bf16 and upstream gradients dy1, dy2 ~ N(0, 1) fp32.
+    One block step is rev_couple_fwd then tqp_adapter_bwd, which reconstructs
+    x1, x2 with the inverse coupling before the adapter gradients; the inverse
+    alone (rev_couple_inv) is timed beside it. L2 is flushed before each call.
+    """
+    import torch
+    import quantized_base_lora_moe_b200 as Q
+    cfgF, cfgG = synth.REV_F, synth.REV_G
+    G = Q.DeviceLayer(synth.make_layer(cfgG, cfgG.seed), device=dev)
+    T, d = cfgF.T, cfgF.d
+    tok = lambda seed: torch.from_numpy(synth.make_tokens(T, d, seed).view(np.int16)).to(dev)
+    x1, x2 = tok(synth.REV_SEEDS["x1"]), tok(synth.REV_SEEDS["x2"])
+    dy1 = torch.from_numpy(synth.make_grad(T, d, synth.REV_SEEDS["dy"], "dy1")).to(dev)
+    dy2 = torch.from_numpy(synth.make_grad(T, d, synth.REV_SEEDS["dy"], "dy2")).to(dev)
+    y1 = torch.empty(T, d, dtype=torch.float32, device=dev)
+    y2 = torch.empty_like(y1)
+    r1, r2 = torch.empty_like(x1), torch.empty_like(x2)
+    dx1, dx2 = torch.empty_like(y1), torch.empty_like(y1)
+    _, _, gF = L_F.grads(dev)
+    _, _, gG = G.grads(dev)
+    lib = Q.lib()
+    ws = Q.workspace(max(lib.rev_couple_workspace_size(T, L_F.ref(), G.ref()),
+                         lib.tqp_adapter_bwd_workspace_size(T, L_F.ref(), G.ref())), dev)
+    st = Q.Status(dev)
+    stream = torch.cuda.current_stream(dev)
+    calls = [("fwd", lambda: Q.rev_couple_fwd(x1, x2, L_F, G, y1, y2, ws, st)),
+             ("inv", lambda: Q.rev_couple_inv(y1, y2, L_F, G, r1, r2, ws, st)),
+             ("adapter_bwd", lambda: Q.tqp_adapter_bwd(y1, y2, dy1, dy2, L_F, G, r1, r2, dx1, dx2, gF, gG, ws, st))]
+    for _ in range(warmup):
+        for _, c in calls:
+            flush.zero_()
+            c()
+    torch.cuda.synchronize(dev)
+    ms = {n: [] for n, _ in calls}
+    for _ in range(steps):
+        for n, c in calls:
+            flush.zero_()
+            e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            e0.record(stream)
+            c()
+            e1.record(stream)
+            e1.synchronize()
+            ms[n].append(e0.elapsed_time(e1))
+    if st.read() != 0:
+        raise RuntimeError(f"device status {st.read()} in the reversible block")
+    f = lambda t: t.view(torch.bfloat16).float()
+    rms = torch.sqrt(torch.mean(torch.cat([f(x1), f(x2)]) ** 2))
+    err = float(max((f(r1) - f(x1)).abs().max(), (f(r2) - f(x2)).abs().max()) / rms)
+    mean = {n: statistics.mean(v) for n, v in ms.items()}
+    step_ms = mean["fwd"] + mean["adapter_bwd"]
+    return {"workload": f"two {cfgF.name} layers F, G; streams 2 x {T}x{d}; forward, inverse, adapter backward",
+            "ms_per_step": step_ms, "tokens_per_s": T / (step_ms * 1e-3), "ms": mean, "steps": steps,
+            "reconstruction_max_err_rel_rms": err, "l2": "flushed before every call"}
+
+
 def run_tqp(args, rank: int, world: int, local_rank: int) -> dict | None:
     import torch
     import quantized_base_lora_moe_b200 as Q
@@ -329,6 +391,8 @@ def run_tqp(args, rank: int, world: int, local_rank: int) -> dict | None:
         "clocks": clk,
         "e2e": e2e,
     }
+    if world == 1 and args.config == "full" and not args.no_rev:
+        result["rev_block"] = time_rev_block(L, dev, min(args.steps, 5), 2, flush)
     if world == 1 and not args.no_cpu_baseline:
         sample = min(T, args.cpu_sample)
         result["cpu_baseline"] = time_oracle(cfg, host, x_bits, sample)
@@ -368,6 +432,8 @@ def main():
     ap.add_argument("--ref-sample", type=int, default=8, help="tokens per step of the reference arm")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-e2e", action="store_true")
+    ap.add_argument("--no-rev", action="store_true", help="skip timing the reversible block (forward, inverse, "
+                                                             "adapter backward)")
     args = ap.parse_args()
     rank = int(os.environ.get("RANK", 0))
     world = int(os.environ.get("WORLD_SIZE", 1))
