@@ -1023,6 +1023,64 @@ int launch_grouped_ffn(const uint16_t* x, int T, const int32_t* offsets, const i
 // dH = dO Wd + dhA Ad^T (SwiGLU backward fused: writes dG | dU) or
 // dX = [dG | dU] [Wg ; Wu] + dxa [Ag^T ; Au^T]^T, per expert, on the tensor cores
 // with the int4 base dequantised transposed in shared memory.
+// K-major fp16 copy of a backward rank-space B operand, [E][n][K], one block
+// per (64-wide K slice, expert):
+//   which 0: Bd, stored B^T [E][d][r]  ->  [E][r][d]             (n = r,  K = d)
+//   which 1: blockdiag(Bg, Bu), each stored B^T [E][f][r]  ->  [E][2r][2f], Bg in
+//            rows [0, r) x columns [0, f), Bu in rows [r, 2r) x columns [f, 2f)
+__global__ void __launch_bounds__(256) rank_b_kernel(const uint16_t* __restrict__ b0, const uint16_t* __restrict__ b1,
+                                                     int which, int r, int f, int K, uint16_t* __restrict__ out) {
+  __shared__ uint16_t tile[64][66];   // [k][j], j < r <= 64
+  const int e = blockIdx.y, k0 = blockIdx.x * 64;
+  const int n = which == 0 ? r : 2 * r;
+  const bool up = which == 1 && k0 >= f;   // f % 64 == 0: a slice lies in one half
+  const uint16_t* src = which == 0 ? b0 + (size_t(e) * K + k0) * r
+                                   : (up ? b1 + (size_t(e) * f + (k0 - f)) * r : b0 + (size_t(e) * f + k0) * r);
+  for (int i = threadIdx.x; i < 64 * r; i += blockDim.x) tile[i / r][i % r] = src[i];   // 64 source rows of r
+  __syncthreads();
+  for (int i = threadIdx.x; i < n * 64; i += blockDim.x) {
+    const int j = i >> 6, kk = i & 63;
+    uint16_t v = 0;
+    if (which == 0) v = uint16_t(bf16_to_f16_bits(tile[kk][j]));
+    else if ((j >= r) == up) v = uint16_t(bf16_to_f16_bits(tile[kk][up ? j - r : j]));
+    out[(size_t(e) * n + j) * K + k0 + kk] = v;
+  }
+}
+
+int launch_rank_bwd(int which, const uint16_t* P, const int32_t* offsets, const int32_t* mb_prefix,
+                    const tqp_moe_weights* w, int T, uint16_t* bk16, uint16_t* C, int32_t* status, cudaStream_t s) {
+  const int r = w->rank, d = w->d, f = w->ffn;
+  if (T == 0 || r == 0) return TQP_OK;
+  const size_t A = size_t(T) * w->top_k;
+  const int K = which == 0 ? d : 2 * f;
+  const int n = which == 0 ? r : 2 * r;
+  rank_b_kernel<<<dim3(unsigned(K / 64), unsigned(w->E)), 256, 0, s>>>(w->lora_b[which == 0 ? 2 : 0], w->lora_b[1],
+                                                                       which, r, f, K, bk16);
+  if (cudaGetLastError() != cudaSuccess) return TQP_ERR_CUDA;
+  // C = s * P B_e^T on the rank-space engine mode: A = P rows by TMA, B = n rows of bk16 per expert
+  GemmArgs a{};
+  a.E = w->E;
+  a.g = w->group;
+  a.r = n;
+  a.lora_scale = w->lora_scale;
+  a.offsets = offsets;
+  a.mb_prefix = mb_prefix;
+  a.status = status;
+  a.kb_per_piece = 1;
+  a.nkb_main = K / 64;
+  a.ntile = n < 16 ? 16 : n;
+  a.n_tiles = 1;
+  a.out = C;
+  a.out_ld = n;
+  a.n_valid = n;
+  Maps mp{};
+  if (!make_tile_map(&mp.m[TA], P, uint64_t(A), uint64_t(K), 128) ||
+      !make_tile_map(&mp.m[TB0], bk16, uint64_t(w->E) * n, uint64_t(K), uint32_t(n)))
+    return TQP_ERR_CUDA;
+  const int mb_upper = int((A + kMBlock - 1) / kMBlock) + w->E;
+  return run_gemm<LORA_HA>(a, mp, mb_upper, s);
+}
+
 int launch_dgrad(int which, const uint16_t* a_src, const uint16_t* a_lora, const int32_t* offsets,
                  const int32_t* mb_prefix, const tqp_moe_weights* w, int T, const uint16_t* aux_gu, uint16_t* out,
                  int32_t* status, cudaStream_t s) {

@@ -2,12 +2,12 @@
 // ("Base expert weights: Quantized (fixed)", "Optimizer state only on adapters",
 // Principle 3 / Pattern 3 of "Reversible Sparse MoE Single Node").
 //
-// The dense dgrad contractions run on the tensor cores (launch_dgrad in
-// grouped_gemm.cu). This file holds the rest:
+// The dense dgrad contractions and the rank-space products dhA = s dO Bd^T and
+// dxa = s [dG|dU] [Bg|Bu]^T run on the tensor cores (launch_dgrad and
+// launch_rank_bwd in grouped_gemm.cu). This file holds the rest:
 //   bwd_combine  : dO = gamma * dy (fp16, permuted rows), dgamma = <dy, O>, the
 //                  softmax-over-chosen backward dl = gamma (dgamma - sum gamma dgamma)
 //                  and the frozen router's input gradient sum_j dl_j W_r[id_j]
-//   rowgemm      : small rank-space products dhA = s dO Bd^T and dxa = s [dG|dU] [Bg|Bu]^T
 //   outer        : per-expert adapter gradients, sums over the expert's routed rows
 //                  of outer products (dA^T, dB^T in the storage layouts)
 //   gather_add   : dx[t] += sum_j dX[row(t, j)]
@@ -141,107 +141,6 @@ __global__ void __launch_bounds__(256) gather_add_kernel(const uint16_t* __restr
 }
 
 // ----------------------------------------------------------------------------
-// per-expert row blocks of 64 (prefix of ceil(count/64))
-// ----------------------------------------------------------------------------
-
-constexpr int kRB = 64;
-
-__global__ void block_prefix_kernel(const int32_t* __restrict__ offsets, int E, int32_t* __restrict__ pre) {
-  if (threadIdx.x != 0 || blockIdx.x != 0) return;
-  int run = 0;
-  for (int e = 0; e < E; ++e) {
-    pre[e] = run;
-    run += (offsets[e + 1] - offsets[e] + kRB - 1) / kRB;
-  }
-  pre[E] = run;
-}
-
-__device__ __forceinline__ int find_expert(const int32_t* __restrict__ pre, int E, int u) {
-  int lo = 0, hi = E;
-  while (hi - lo > 1) {
-    const int mid = (lo + hi) >> 1;
-    if (pre[mid] <= u) lo = mid;
-    else hi = mid;
-  }
-  return lo;
-}
-
-// ----------------------------------------------------------------------------
-// rank-space row GEMMs: C[row][n] = s * sum_k P[row][k] * B_e[k][n], n < N <= 64
-// ----------------------------------------------------------------------------
-
-struct RowGemmArgs {
-  int which;                 // 0: dhA (B = Bd^T [d][r]); 1: dxa (B = blockdiag(Bg^T, Bu^T) [2f][2r])
-  int E, K, N, r, f;
-  float scale;
-  const int32_t* offsets;
-  const int32_t* pre;
-  const uint16_t* P;         // fp16 [A][K]
-  const uint16_t* b0;        // bf16 B^T sources
-  const uint16_t* b1;
-  uint16_t* C;               // fp16 [A][N]
-};
-
-__device__ __forceinline__ float rowgemm_b(const RowGemmArgs& a, int e, int k, int n) {
-  if (a.which == 0) return n < a.r ? bf16_to_f32(__ldg(a.b0 + (size_t(e) * a.K + k) * a.r + n)) : 0.0f;
-  if (k < a.f) return n < a.r ? bf16_to_f32(__ldg(a.b0 + (size_t(e) * a.f + k) * a.r + n)) : 0.0f;
-  return (n >= a.r && n < 2 * a.r) ? bf16_to_f32(__ldg(a.b1 + (size_t(e) * a.f + (k - a.f)) * a.r + (n - a.r)))
-                                   : 0.0f;
-}
-
-__global__ void __launch_bounds__(256) rowgemm_kernel(const RowGemmArgs a) {
-  __shared__ float Ps[kRB][33];
-  __shared__ float Bs[32][65];
-  const int nunits = a.pre[a.E];
-  const int tx = threadIdx.x & 15, ty = threadIdx.x >> 4;    // 16 col groups x 16 row groups
-  for (int u = blockIdx.x; u < nunits; u += gridDim.x) {
-    const int e = find_expert(a.pre, a.E, u);
-    const int mb = u - a.pre[e];
-    const int base = a.offsets[e] + mb * kRB;
-    const int rows = min(kRB, a.offsets[e + 1] - base);
-    float acc[4][4];
-#pragma unroll
-    for (int i = 0; i < 4; ++i)
-#pragma unroll
-      for (int j = 0; j < 4; ++j) acc[i][j] = 0.0f;
-    for (int k0 = 0; k0 < a.K; k0 += 32) {
-      __syncthreads();
-      for (int i = threadIdx.x; i < kRB * 32; i += blockDim.x) {
-        const int rr = i >> 5, kk = i & 31;
-        Ps[rr][kk] = (rr < rows) ? f16_to_f32(a.P[size_t(base + rr) * a.K + k0 + kk]) : 0.0f;
-      }
-      for (int i = threadIdx.x; i < 32 * 64; i += blockDim.x) {
-        const int kk = i >> 6, n = i & 63;
-        Bs[kk][n] = (n < a.N) ? rowgemm_b(a, e, k0 + kk, n) : 0.0f;
-      }
-      __syncthreads();
-#pragma unroll 8
-      for (int kk = 0; kk < 32; ++kk) {
-        float pv[4], bv[4];
-#pragma unroll
-        for (int i = 0; i < 4; ++i) pv[i] = Ps[ty * 4 + i][kk];
-#pragma unroll
-        for (int j = 0; j < 4; ++j) bv[j] = Bs[kk][tx * 4 + j];
-#pragma unroll
-        for (int i = 0; i < 4; ++i)
-#pragma unroll
-          for (int j = 0; j < 4; ++j) acc[i][j] = fmaf(pv[i], bv[j], acc[i][j]);
-      }
-    }
-#pragma unroll
-    for (int i = 0; i < 4; ++i) {
-      const int rr = ty * 4 + i;
-      if (rr >= rows) continue;
-#pragma unroll
-      for (int j = 0; j < 4; ++j) {
-        const int n = tx * 4 + j;
-        if (n < a.N) a.C[size_t(base + rr) * a.N + n] = __half_as_ushort(__float2half_rn(a.scale * acc[i][j]));
-      }
-    }
-  }
-}
-
-// ----------------------------------------------------------------------------
 // adapter gradients: C[e][m][n] = sum_{rows of e} P(row, m) * Q(row, n)
 // ----------------------------------------------------------------------------
 
@@ -256,40 +155,66 @@ struct OuterArgs {
   float* C;                  // fp32 [E][M][N]
 };
 
+// One block computes a TM x TN tile of C[e] (TM x TN = 4096, 4 x 4 per thread)
+// over all routed rows of expert e, 32 rows at a time. Rows are read as 16-byte
+// pieces (8 fp16 values; M, N, the strides and the column offsets are multiples
+// of 8). The tile shape follows the operand widths: one of M, N is the rank r,
+// so a 64 x 64 tile would leave half its FMAs on zero padding when r = 32.
+template <int TM, int TN>
 __global__ void __launch_bounds__(256) outer_kernel(const OuterArgs a) {
-  __shared__ float Ps[32][65];
-  __shared__ float Qs[32][65];
+  static_assert(TM * TN == 4096, "4 x 4 outputs per thread");
+  __shared__ __align__(16) float Ps[32][TM + 4];
+  __shared__ __align__(16) float Qs[32][TN + 4];
   const int e = blockIdx.x;
-  const int m0 = blockIdx.y * 64, n0 = blockIdx.z * 64;
-  const int tx = threadIdx.x & 15, ty = threadIdx.x >> 4;
+  const int m0 = blockIdx.y * TM, n0 = blockIdx.z * TN;
+  const int tx = threadIdx.x % (TN / 4), ty = threadIdx.x / (TN / 4);
   const int r0 = a.offsets[e], r1 = a.offsets[e + 1];
   float acc[4][4];
 #pragma unroll
   for (int i = 0; i < 4; ++i)
 #pragma unroll
     for (int j = 0; j < 4; ++j) acc[i][j] = 0.0f;
+  auto stage8 = [](float* dst, uint4 v) {
+    const uint32_t w[4] = {v.x, v.y, v.z, v.w};
+    float f[8];
+#pragma unroll
+    for (int t = 0; t < 4; ++t) {
+      f[2 * t] = f16_to_f32(uint16_t(w[t] & 0xFFFFu));
+      f[2 * t + 1] = f16_to_f32(uint16_t(w[t] >> 16));
+    }
+    *reinterpret_cast<float4*>(dst) = make_float4(f[0], f[1], f[2], f[3]);
+    *reinterpret_cast<float4*>(dst + 4) = make_float4(f[4], f[5], f[6], f[7]);
+  };
   for (int rb = r0; rb < r1; rb += 32) {
     __syncthreads();
-    for (int i = threadIdx.x; i < 32 * 64; i += blockDim.x) {
-      const int rr = i >> 6, c = i & 63;
+    for (int i = threadIdx.x; i < 32 * (TM / 8); i += blockDim.x) {
+      const int rr = i / (TM / 8), c = (i % (TM / 8)) * 8;
       const int row = rb + rr;
-      const bool ok = row < r1;
-      Ps[rr][c] = (ok && m0 + c < a.M) ? f16_to_f32(a.P[size_t(row) * a.ldp + a.offp + m0 + c]) : 0.0f;
-      const int qrow = ok ? (a.perm ? a.perm[row] : row) : 0;
-      Qs[rr][c] = (ok && n0 + c < a.N) ? f16_to_f32(a.Q[size_t(qrow) * a.ldq + a.offq + n0 + c]) : 0.0f;
+      uint4 v = make_uint4(0, 0, 0, 0);
+      if (row < r1 && m0 + c < a.M)
+        v = __ldg(reinterpret_cast<const uint4*>(a.P + size_t(row) * a.ldp + a.offp + m0 + c));
+      stage8(&Ps[rr][c], v);
+    }
+    for (int i = threadIdx.x; i < 32 * (TN / 8); i += blockDim.x) {
+      const int rr = i / (TN / 8), c = (i % (TN / 8)) * 8;
+      const int row = rb + rr;
+      uint4 v = make_uint4(0, 0, 0, 0);
+      if (row < r1 && n0 + c < a.N) {
+        const int qrow = a.perm ? __ldg(a.perm + row) : row;
+        v = __ldg(reinterpret_cast<const uint4*>(a.Q + size_t(qrow) * a.ldq + a.offq + n0 + c));
+      }
+      stage8(&Qs[rr][c], v);
     }
     __syncthreads();
 #pragma unroll 8
     for (int rr = 0; rr < 32; ++rr) {
-      float pv[4], qv[4];
-#pragma unroll
-      for (int i = 0; i < 4; ++i) pv[i] = Ps[rr][ty * 4 + i];
-#pragma unroll
-      for (int j = 0; j < 4; ++j) qv[j] = Qs[rr][tx * 4 + j];
+      const float4 pv = *reinterpret_cast<const float4*>(&Ps[rr][ty * 4]);
+      const float4 qv = *reinterpret_cast<const float4*>(&Qs[rr][tx * 4]);
+      const float p4[4] = {pv.x, pv.y, pv.z, pv.w}, q4[4] = {qv.x, qv.y, qv.z, qv.w};
 #pragma unroll
       for (int i = 0; i < 4; ++i)
 #pragma unroll
-        for (int j = 0; j < 4; ++j) acc[i][j] = fmaf(pv[i], qv[j], acc[i][j]);
+        for (int j = 0; j < 4; ++j) acc[i][j] = fmaf(p4[i], q4[j], acc[i][j]);
     }
   }
 #pragma unroll
@@ -325,38 +250,6 @@ int launch_gather_add(const uint16_t* dX, const int32_t* inv, int T, int k, int 
   return cudaGetLastError() == cudaSuccess ? TQP_OK : TQP_ERR_CUDA;
 }
 
-int launch_block_prefix(const int32_t* offsets, int E, int32_t* pre, cudaStream_t s) {
-  block_prefix_kernel<<<1, 32, 0, s>>>(offsets, E, pre);
-  return cudaGetLastError() == cudaSuccess ? TQP_OK : TQP_ERR_CUDA;
-}
-
-int launch_rowgemm(int which, const uint16_t* P, const int32_t* offsets, const int32_t* pre, int A_rows,
-                   const tqp_moe_weights* w, uint16_t* C, cudaStream_t s) {
-  RowGemmArgs a{};
-  a.which = which;
-  a.E = w->E;
-  a.r = w->rank;
-  a.f = w->ffn;
-  a.scale = w->lora_scale;
-  a.offsets = offsets;
-  a.pre = pre;
-  a.P = P;
-  a.C = C;
-  if (which == 0) {
-    a.K = w->d;
-    a.N = w->rank;
-    a.b0 = w->lora_b[2];
-  } else {
-    a.K = 2 * w->ffn;
-    a.N = 2 * w->rank;
-    a.b0 = w->lora_b[0];
-    a.b1 = w->lora_b[1];
-  }
-  const int blocks = (A_rows + kRB - 1) / kRB + w->E;
-  rowgemm_kernel<<<blocks < 4096 ? blocks : 4096, 256, 0, s>>>(a);
-  return cudaGetLastError() == cudaSuccess ? TQP_OK : TQP_ERR_CUDA;
-}
-
 int launch_outer(int E, int M, int N, const int32_t* offsets, const int32_t* perm, const uint16_t* P, int ldp,
                  int offp, const uint16_t* Q, int ldq, int offq, float* C, cudaStream_t s) {
   OuterArgs a{};
@@ -372,8 +265,13 @@ int launch_outer(int E, int M, int N, const int32_t* offsets, const int32_t* per
   a.ldq = ldq;
   a.offq = offq;
   a.C = C;
-  dim3 grid(E, (M + 63) / 64, (N + 63) / 64);
-  outer_kernel<<<grid, 256, 0, s>>>(a);
+  if (N <= 32) {
+    outer_kernel<128, 32><<<dim3(E, (M + 127) / 128, (N + 31) / 32), 256, 0, s>>>(a);
+  } else if (M <= 32) {
+    outer_kernel<32, 128><<<dim3(E, (M + 31) / 32, (N + 127) / 128), 256, 0, s>>>(a);
+  } else {
+    outer_kernel<64, 64><<<dim3(E, (M + 63) / 64, (N + 63) / 64), 256, 0, s>>>(a);
+  }
   return cudaGetLastError() == cudaSuccess ? TQP_OK : TQP_ERR_CUDA;
 }
 

@@ -110,13 +110,18 @@ struct BwdWs {
   uint16_t* dha;    // s dO Bd^T [A][r] fp16
   uint16_t* dgu;    // dG | dU [A][2f] fp16
   uint16_t* dxa;    // s [dG|dU] [Bg|Bu]^T [A][2r] fp16
-  int32_t* pre64;   // per-expert 64-row block prefix [E+1]
+  uint16_t* bk16;   // K-major fp16 B operand of dha / dxa, E * max(r d, 4 r f) values
 };
+
+size_t rank_b_values(const tqp_moe_weights* w) {
+  const size_t rd = size_t(w->rank) * w->d, rf4 = size_t(4) * w->rank * w->ffn;
+  return size_t(w->E) * (rd > rf4 ? rd : rf4);
+}
 
 size_t bwd_extra_bytes(int T, const tqp_moe_weights* w) {
   const size_t A = size_t(T) * w->top_k;
   return align_up(A * 2 * w->ffn * 2, 256) * 2 + align_up(A * w->d * 2, 256) + align_up(A * w->rank * 2, 256) +
-         align_up(A * 2 * w->rank * 2, 256) + align_up(size_t(w->E + 1) * 4, 256) + 256;
+         align_up(A * 2 * w->rank * 2, 256) + align_up(rank_b_values(w) * 2, 256) + 256;
 }
 
 BwdWs carve_bwd(void* p0, int T, const tqp_moe_weights* w) {
@@ -133,7 +138,7 @@ BwdWs carve_bwd(void* p0, int T, const tqp_moe_weights* w) {
   b.dha = static_cast<uint16_t*>(take(A * w->rank * 2));
   b.dgu = static_cast<uint16_t*>(take(A * 2 * w->ffn * 2));
   b.dxa = static_cast<uint16_t*>(take(A * 2 * w->rank * 2));
-  b.pre64 = static_cast<int32_t*>(take(size_t(w->E + 1) * 4));
+  b.bk16 = static_cast<uint16_t*>(take(rank_b_values(w) * 2));
   return b;
 }
 
@@ -145,17 +150,17 @@ int layer_backward(const uint16_t* x, const float* dy, int T, const tqp_moe_weig
   const LayerWs L = carve_layer_ws(ws, T, w);
   const BwdWs B = carve_bwd(static_cast<char*>(ws) + layer_ws_size(T, w), T, w);
   const int k = w->top_k, d = w->d, f = w->ffn, r = w->rank, E = w->E;
-  const int A = T * k;
   int rc;
   if ((rc = layer_experts(x, T, w, L, status, s, B.gu)) != TQP_OK) return rc;
   const FfnBufs fb = ffn_carve(L.ffn_ws, T, w);
   if ((rc = launch_bwd_combine(L.out_perm, L.inv, L.gates, L.ids, w->router_w, dy, T, k, d, B.dO, dx, s)) != TQP_OK)
     return rc;
-  if ((rc = launch_block_prefix(L.offsets, E, B.pre64, s)) != TQP_OK) return rc;
-  if (r > 0 && (rc = launch_rowgemm(0, B.dO, L.offsets, B.pre64, A, w, B.dha, s)) != TQP_OK) return rc;
+  if (r > 0 && (rc = launch_rank_bwd(0, B.dO, L.offsets, fb.mb_prefix, w, T, B.bk16, B.dha, status, s)) != TQP_OK)
+    return rc;
   if ((rc = launch_dgrad(0, B.dO, B.dha, L.offsets, fb.mb_prefix, w, T, B.gu, B.dgu, status, s)) != TQP_OK) return rc;
   if (r > 0) {
-    if ((rc = launch_rowgemm(1, B.dgu, L.offsets, B.pre64, A, w, B.dxa, s)) != TQP_OK) return rc;
+    if ((rc = launch_rank_bwd(1, B.dgu, L.offsets, fb.mb_prefix, w, T, B.bk16, B.dxa, status, s)) != TQP_OK)
+      return rc;
     // adapter gradients, in the storage layouts A^T [r][in], B^T [out][r]
     if ((rc = launch_outer(E, d, r, L.offsets, nullptr, B.dO, d, 0, fb.ha, r, 0, g->dB[2], s)) != TQP_OK) return rc;
     if ((rc = launch_outer(E, r, f, L.offsets, nullptr, B.dha, r, 0, L.h, f, 0, g->dA[2], s)) != TQP_OK) return rc;

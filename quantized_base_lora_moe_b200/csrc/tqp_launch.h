@@ -48,15 +48,18 @@ int launch_grouped_ffn_part(int part, const uint16_t* x, int T, const int32_t* o
 int launch_dgrad(int which, const uint16_t* a_src, const uint16_t* a_lora, const int32_t* offsets,
                  const int32_t* mb_prefix, const tqp_moe_weights* w, int T, const uint16_t* aux_gu, uint16_t* out,
                  int32_t* status, cudaStream_t s);
+// rank-space products of the backward on the tensor cores (grouped_gemm.cu):
+//   which 0: dha = s dO Bd      (P = dO [A][d]      -> C [A][r])
+//   which 1: dxa = s [dG|dU] blockdiag(Bg, Bu)   (P = dgu [A][2f] -> C [A][2r])
+// bk16: scratch for the K-major fp16 B operand, E * max(r d, 4 r f) values.
+int launch_rank_bwd(int which, const uint16_t* P, const int32_t* offsets, const int32_t* mb_prefix,
+                    const tqp_moe_weights* w, int T, uint16_t* bk16, uint16_t* C, int32_t* status, cudaStream_t s);
 
 // backward pieces (layer_bwd.cu)
 int launch_bwd_combine(const uint16_t* O, const int32_t* inv, const float* gates, const int32_t* ids,
                        const float* router_w, const float* dy, int T, int k, int d, uint16_t* dO, float* dx,
                        cudaStream_t s);
 int launch_gather_add(const uint16_t* dX, const int32_t* inv, int T, int k, int d, float* dx, cudaStream_t s);
-int launch_block_prefix(const int32_t* offsets, int E, int32_t* pre, cudaStream_t s);
-int launch_rowgemm(int which, const uint16_t* P, const int32_t* offsets, const int32_t* pre, int A_rows,
-                   const tqp_moe_weights* w, uint16_t* C, cudaStream_t s);
 int launch_outer(int E, int M, int N, const int32_t* offsets, const int32_t* perm, const uint16_t* P, int ldp,
                  int offp, const uint16_t* Q, int ldq, int offq, float* C, cudaStream_t s);
 
