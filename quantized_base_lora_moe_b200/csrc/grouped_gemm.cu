@@ -23,8 +23,9 @@
 //   warps 10-17 B producer: int4 -> fp16 dequantisation (transposed for the
 //               dgrads) into 128B-swizzled K-major tiles, LoRA B^T tiles
 // Accumulators are double-buffered in TMEM (2 x 256 fp32 columns), so the
-// epilogue of one unit overlaps the main loop of the next. Operand stages:
-// 4 x (16 KB A + 32 KB B); code ring: 3 x 9 KB. No TMA multicast is used.
+// epilogue of one unit overlaps the main loop of the next. The operand rings
+// (16 KB A tiles, B tiles, 9 KB code stages) share one 216 KB region whose
+// split depends on the mode (Layout below). No TMA multicast is used.
 #include <cstdint>
 #include <cstring>
 #include <cuda.h>
@@ -46,20 +47,31 @@ constexpr int kBStageBytes = 32768;   // up to 256 rows x 64 K x 2 B
 constexpr int kQStageBytes = 9216;    // up to 8192 B of codes + 1024 B of scales
 constexpr int kBStagesMax = 8;
 
-// B ring of one mode. The dequantising modes keep two slots of 32 KB. The modes
-// whose B tile comes by TMA (rank-space GEMMs, router) read no codes, so their
-// ring also takes the code region and runs deeper: two TMA fills in flight
-// cannot cover the L2/DRAM latency of a 4-MMA stage, and the A producer's TMA
-// issuer waits on the same ring.
+constexpr size_t kOperandBytes = size_t(kAStages) * kAStageBytes + size_t(kBStages) * kBStageBytes +
+                                 size_t(kQStages) * kQStageBytes;
+
+// Split of the operand region for one mode.
+// - Dequantising forward modes: 5 A, 2 B and 8 code stages.
+// - Modes whose B tile comes by TMA (rank-space GEMMs, router) read no codes, so
+//   their B ring also takes the code region and runs deeper: two TMA fills in
+//   flight cannot cover the L2/DRAM latency of a 4-MMA stage, and the A
+//   producer's TMA issuer waits on the same ring.
+// - Transposed dequantisation (dgrads): two producer groups of 128 threads take
+//   alternate stages (one stage's chain of code reads, dequant, transpose and
+//   stores is latency-bound), which needs a third B slot: 4 A, 3 B, 6 code stages.
 template <int MODE>
-struct BRing {
+struct Layout {
   static constexpr bool kTma = (MODE == LORA_XA || MODE == LORA_HA || MODE == ROUTER);
-  static constexpr int kStages = !kTma ? kBStages : (MODE == ROUTER ? 4 : 8);
+  static constexpr bool kTrans = (MODE == DH || MODE == DX);
+  static constexpr int kA = kTrans ? 4 : kAStages;
+  static constexpr int kB = kTma ? (MODE == ROUTER ? 4 : 8) : (kTrans ? 3 : kBStages);
   // LORA_XA: 2r rows (r <= 64), LORA_HA: r rows, ROUTER: up to 256 rows, x 128 B
-  static constexpr int kBytes = (kTma && MODE != ROUTER) ? 16384 : kBStageBytes;
-  static_assert(kStages <= kBStagesMax, "B ring barriers");
-  static_assert(size_t(kStages) * kBytes <= size_t(kBStages) * kBStageBytes + (kTma ? size_t(kQStages) * kQStageBytes : 0),
-                "B ring footprint");
+  static constexpr int kBBytes = (kTma && MODE != ROUTER) ? 16384 : kBStageBytes;
+  static constexpr int kQ = kTma ? 0 : (kTrans ? 6 : kQStages);
+  static constexpr int kBGroups = kTrans ? 2 : 1;
+  static_assert(kB <= kBStagesMax && kQ <= kQStages && kA <= kAStages, "ring barriers");
+  static_assert(size_t(kA) * kAStageBytes + size_t(kB) * kBBytes + size_t(kQ) * kQStageBytes <= kOperandBytes,
+                "operand region");
 };
 
 struct SmemCtl {
@@ -76,8 +88,7 @@ struct SmemCtl {
   int abort_flag;
 };
 
-constexpr size_t kSmemBytes = 1024 /*align slack*/ + size_t(kAStages) * kAStageBytes +
-                              size_t(kBStages) * kBStageBytes + size_t(kQStages) * kQStageBytes + sizeof(SmemCtl);
+constexpr size_t kSmemBytes = 1024 /*align slack*/ + kOperandBytes + sizeof(SmemCtl);
 static_assert(kSmemBytes <= 232448, "shared memory budget");
 
 
@@ -111,15 +122,18 @@ __global__ void __launch_bounds__(kThreads, 1)
   constexpr bool kATma = (MODE == DOWN || MODE == LORA_HA || MODE == ROUTER || kTrans);
   constexpr bool kBTma = (MODE == LORA_XA || MODE == LORA_HA || MODE == ROUTER);
   constexpr bool kBf16 = (MODE == LORA_XA || MODE == ROUTER);
-  constexpr int kBSt = BRing<MODE>::kStages;
-  constexpr int kBStride = BRing<MODE>::kBytes;
-  static_assert(BRing<MODE>::kTma == kBTma, "B ring mode");
+  constexpr int kASt = Layout<MODE>::kA;
+  constexpr int kBSt = Layout<MODE>::kB;
+  constexpr int kBStride = Layout<MODE>::kBBytes;
+  constexpr int kQSt = Layout<MODE>::kQ > 0 ? Layout<MODE>::kQ : 1;
+  constexpr int kBGroups = Layout<MODE>::kBGroups;
+  static_assert(Layout<MODE>::kTma == kBTma && Layout<MODE>::kTrans == kTrans, "layout mode");
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   uint8_t* a_base = smem;
-  uint8_t* b_base = a_base + size_t(kAStages) * kAStageBytes;
-  uint8_t* q_base = b_base + size_t(kBStages) * kBStageBytes;
-  SmemCtl* ctl = reinterpret_cast<SmemCtl*>(q_base + size_t(kQStages) * kQStageBytes);
+  uint8_t* b_base = a_base + size_t(kASt) * kAStageBytes;
+  uint8_t* q_base = b_base + size_t(kBSt) * kBStride;
+  SmemCtl* ctl = reinterpret_cast<SmemCtl*>(smem + kOperandBytes);
   volatile int* abort_flag = &ctl->abort_flag;
 
   const int warp = threadIdx.x >> 5;
@@ -128,17 +142,18 @@ __global__ void __launch_bounds__(kThreads, 1)
   const Sched sc = load_sched(a, s_sched);
 
   if (threadIdx.x == 0) {
-    for (int i = 0; i < kAStages; ++i) {
+    for (int i = 0; i < kASt; ++i) {
       mbar_init(&ctl->a_full[i], 128);
       mbar_init(&ctl->a_empty[i], 1);
     }
     for (int i = 0; i < kBSt; ++i) {
-      mbar_init(&ctl->b_full[i], kBTma ? 257 : 256);   // + the TMA issuer's arrival
+      // one producer group's threads (+ the TMA issuer's arrival)
+      mbar_init(&ctl->b_full[i], kBTma ? 257 : 256 / kBGroups);
       mbar_init(&ctl->b_empty[i], 1);
     }
-    for (int i = 0; i < kQStages; ++i) {
+    for (int i = 0; i < kQSt; ++i) {
       mbar_init(&ctl->q_full[i], 1);
-      mbar_init(&ctl->q_empty[i], 256);
+      mbar_init(&ctl->q_empty[i], 256 / kBGroups);
     }
     for (int i = 0; i < 2; ++i) {
       mbar_init(&ctl->acc_full[i], 1);
@@ -328,7 +343,7 @@ __global__ void __launch_bounds__(kThreads, 1)
             umma_bf16(dt, adesc + uint64_t(2 * kk), bdesc + uint64_t(2 * kk), idesc, (kb > 0 || kk > 0) ? 1u : 0u);
           umma_commit(&ctl->a_empty[ra.stage]);
           umma_commit(&ctl->b_empty[rb.stage]);
-          ra.next<kAStages>();
+          ra.next<kASt>();
           rb.next<kBSt>();
         }
         if (!ok) break;
@@ -379,7 +394,7 @@ __global__ void __launch_bounds__(kThreads, 1)
           ++issued;
           last_stage = q.stage;
           last_phase = q.phase;
-          q.next<kQStages>();
+          q.next<kQSt>();
         }
         if (!ok) break;
       }
@@ -468,7 +483,7 @@ __global__ void __launch_bounds__(kThreads, 1)
           }
           if (kBTma) rb.next<kBSt>();
         }
-        ra.next<kAStages>();
+        ra.next<kASt>();
       }
       if (!ok) break;
     }
@@ -483,11 +498,21 @@ __global__ void __launch_bounds__(kThreads, 1)
     const int brow = tid / tpr;                              // B row (forward tiles)
     const int part = tid % tpr;
     const int nwords = tpr >= 8 ? 1 : 8 / tpr;               // int4 words (8 K values each) per thread
+    // transposed modes: two groups of 128 threads take alternate stages
+    const int grp = kBGroups > 1 ? tid >> 7 : 0;
+    const int gtid = kBGroups > 1 ? tid & 127 : tid;
+    constexpr int kGT = 256 / kBGroups;                      // threads per group
     Ring rb, q;
+    int n = 0;                                               // stage counter over all units
     for (int u = blockIdx.x; u < nunits; u += gridDim.x) {
       const Unit un = decode_unit(a, sc, u);
       bool ok = true;
-      for (int kb = 0; kb < nkb; ++kb) {
+      for (int kb = 0; kb < nkb; ++kb, ++n) {
+        if (kBGroups > 1 && (n & 1) != grp) {
+          if (kb >= a.nkb_lora) q.next<kQSt>();   // the other group consumes this stage's codes
+          rb.next<kBSt>();
+          continue;
+        }
         const bool waited = kBTma ? mbar_wait<256>(&ctl->b_empty[rb.stage], rb.phase ^ 1u, abort_flag, a.status)
                                   : mbar_wait(&ctl->b_empty[rb.stage], rb.phase ^ 1u, abort_flag, a.status);
         if (!waited) { ok = false; break; }
@@ -520,7 +545,7 @@ __global__ void __launch_bounds__(kThreads, 1)
             }
           } else if (kTrans) {
             // dgrad rank-space step: B[n][rr] = A^T[rr][n0 + n] (bf16, read transposed) as fp16
-            for (int nrow = tid; nrow < a.ntile; nrow += 256) {
+            for (int nrow = gtid; nrow < a.ntile; nrow += kGT) {
               const int n = un.nt * a.ntile + nrow;
 #pragma unroll 1
               for (int c = 0; c < 8; ++c) {
@@ -546,14 +571,14 @@ __global__ void __launch_bounds__(kThreads, 1)
           fence_proxy_async_smem();
           mbar_arrive(full);
         } else if (kTrans) {
-          // transposed dequant: thread = 4 K rows x 8 N columns per 128-column half
           if (!mbar_wait(&ctl->q_full[q.stage], q.phase, abort_flag, a.status)) { ok = false; break; }
           const uint8_t* qs = q_base + size_t(q.stage) * kQStageBytes;
-          const int kq = tid >> 4, no = tid & 15;
+          // thread = 4 K rows (kq) x 8-column octets no, no + 8, ... of the tile
+          const int kq = gtid >> 3, no = gtid & 7;
           const int n0 = un.nt * a.ntile;
           const int rowb = a.ntile >> 1;                     // bytes per code row
           const uint16_t* sc = reinterpret_cast<const uint16_t*>(qs + a.ntile * 32);
-          for (int hb = 0; hb < a.ntile; hb += 128) {
+          for (int hb = 0; hb < a.ntile; hb += 64) {
             const int oct = (hb >> 3) + no;                  // N octet of this thread
             const int gi = (n0 + oct * 8) / a.g - n0 / a.g;
             uint32_t hv[4][4];
@@ -577,7 +602,7 @@ __global__ void __launch_bounds__(kThreads, 1)
           // proxy fence (its next TMA fill and the tensor-core reads are async-proxy)
           fence_proxy_async_smem();
           mbar_arrive(&ctl->q_empty[q.stage]);
-          q.next<kQStages>();
+          q.next<kQSt>();
           mbar_arrive(full);
         } else if (kDequant) {
           if (!mbar_wait(&ctl->q_full[q.stage], q.phase, abort_flag, a.status)) { ok = false; break; }
@@ -594,7 +619,7 @@ __global__ void __launch_bounds__(kThreads, 1)
           else dequant_row<4>(qs, bst, brow, part, s_lo, s_hi);
           fence_proxy_async_smem();
           mbar_arrive(&ctl->q_empty[q.stage]);
-          q.next<kQStages>();
+          q.next<kQSt>();
           mbar_arrive(full);
         } else {
           mbar_arrive(full);  // the B tile arrives by TMA (LORA_XA, LORA_HA, ROUTER)
