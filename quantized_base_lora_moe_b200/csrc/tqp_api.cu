@@ -113,6 +113,15 @@ struct BwdWs {
   uint16_t* bk16;   // K-major fp16 B operand of dha / dxa, E * max(r d, 4 r f) values
 };
 
+// Adapter-gradient buffers: present and 16-byte aligned when the rank is nonzero.
+bool grads_ok(const tqp_moe_weights* w, const tqp_adapter_grads* g) {
+  if (!g) return false;
+  if (w->rank > 0)
+    for (int p = 0; p < 3; ++p)
+      if (!g->dA[p] || !g->dB[p] || !aligned16(g->dA[p]) || !aligned16(g->dB[p])) return false;
+  return true;
+}
+
 size_t rank_b_values(const tqp_moe_weights* w) {
   const size_t rd = size_t(w->rank) * w->d, rf4 = size_t(4) * w->rank * w->ffn;
   return size_t(w->E) * (rd > rf4 ? rd : rf4);
@@ -145,13 +154,16 @@ BwdWs carve_bwd(void* p0, int T, const tqp_moe_weights* w) {
 // Backward of one layer: recompute the forward (keeping G, U), then
 // combine/gate/router backward, dH (+SwiGLU backward) and dX on the tensor
 // cores, rank-space products and adapter gradients, and the token gather.
+// recompute = false: the forward of this x has just run on the same workspace
+// with the G|U pre-activations kept (layer_forward with aux_gu = the backward
+// scratch's gu), so its routing and intermediates are still in place.
 int layer_backward(const uint16_t* x, const float* dy, int T, const tqp_moe_weights* w, float* dx,
-                   const tqp_adapter_grads* g, void* ws, int32_t* status, cudaStream_t s) {
+                   const tqp_adapter_grads* g, void* ws, int32_t* status, cudaStream_t s, bool recompute = true) {
   const LayerWs L = carve_layer_ws(ws, T, w);
   const BwdWs B = carve_bwd(static_cast<char*>(ws) + layer_ws_size(T, w), T, w);
   const int k = w->top_k, d = w->d, f = w->ffn, r = w->rank, E = w->E;
   int rc;
-  if ((rc = layer_experts(x, T, w, L, status, s, B.gu)) != TQP_OK) return rc;
+  if (recompute && (rc = layer_experts(x, T, w, L, status, s, B.gu)) != TQP_OK) return rc;
   const FfnBufs fb = ffn_carve(L.ffn_ws, T, w);
   if ((rc = launch_bwd_combine(L.out_perm, L.inv, L.gates, L.ids, w->router_w, dy, T, k, d, B.dO, dx, s)) != TQP_OK)
     return rc;
@@ -179,9 +191,10 @@ int layer_backward(const uint16_t* x, const float* dy, int T, const tqp_moe_weig
 }
 
 int layer_forward(const uint16_t* x, int T, const tqp_moe_weights* w, const void* residual, int res_f32,
-                  float sign, void* y, int y_f32, uint16_t* y_bf16, void* ws, int32_t* status, cudaStream_t s) {
+                  float sign, void* y, int y_f32, uint16_t* y_bf16, void* ws, int32_t* status, cudaStream_t s,
+                  uint16_t* aux_gu = nullptr) {
   const LayerWs L = carve_layer_ws(ws, T, w);
-  int rc = layer_experts(x, T, w, L, status, s);
+  int rc = layer_experts(x, T, w, L, status, s, aux_gu);
   if (rc != TQP_OK) return rc;
   return launch_combine(L.out_perm, L.inv, L.gates, T, w->top_k, w->d, residual, res_f32, sign, y, y_f32, y_bf16, s);
 }
@@ -381,10 +394,7 @@ int tqp_moe_layer_bwd(const uint16_t* x, const float* dy, int T, const tqp_moe_w
   const bool n = T > 0;
   if (T < 0 || !ptr_ok(x, n) || !ptr_ok(dy, n) || !ptr_ok(dx, n) || !grads) return TQP_ERR_INVALID_ARG;
   if (w->ffn % 128 != 0) return TQP_ERR_UNSUPPORTED;   // the dH tiles are 128 columns of ffn
-  if (w->rank > 0)
-    for (int p = 0; p < 3; ++p)
-      if (!grads->dA[p] || !grads->dB[p] || !aligned16(grads->dA[p]) || !aligned16(grads->dB[p]))
-        return TQP_ERR_INVALID_ARG;
+  if (!grads_ok(w, grads)) return TQP_ERR_INVALID_ARG;
   if (n && (!ws || ws_bytes < tqp_moe_layer_bwd_workspace_size(T, w))) return TQP_ERR_WORKSPACE;
   if (!n) return TQP_OK;
   return layer_backward(x, dy, T, w, dx, grads, ws, dev_status, static_cast<cudaStream_t>(stream));
@@ -405,7 +415,7 @@ int tqp_adapter_bwd(const float* y1, const float* y2, const float* dy1, const fl
                     int32_t* dev_status, void* stream) {
   int rc;
   if ((rc = check_weights(F)) != TQP_OK || (rc = check_weights(G)) != TQP_OK) return rc;
-  if (F->d != G->d || T < 0 || !gF || !gG) return TQP_ERR_INVALID_ARG;
+  if (F->d != G->d || T < 0 || !grads_ok(F, gF) || !grads_ok(G, gG)) return TQP_ERR_INVALID_ARG;
   if (F->ffn % 128 != 0 || G->ffn % 128 != 0) return TQP_ERR_UNSUPPORTED;
   const bool n = T > 0;
   if (!ptr_ok(y1, n) || !ptr_ok(y2, n) || !ptr_ok(dy1, n) || !ptr_ok(dy2, n) || !ptr_ok(x1, n) || !ptr_ok(x2, n) ||
@@ -419,16 +429,19 @@ int tqp_adapter_bwd(const float* y1, const float* y2, const float* dy1, const fl
   uint16_t* zb = reinterpret_cast<uint16_t*>(base);                     // bf16(y1)
   float* dxG = reinterpret_cast<float*>(base + align_up(Td * 2, 256));  // J_G^T dy2
   void* lws = base + align_up(Td * 2, 256) + align_up(Td * 4, 256);
-  const size_t lws_bytes = ws_bytes - size_t((char*)lws - (char*)ws);
+  // Each layer's backward follows the inverse step that ran that layer's forward
+  // on the same workspace (keeping G|U), so it does not recompute the forward.
   // G-step: reconstruct x2 = y2 - G(bf16(y1)); G's grads for cotangent dy2
   if ((rc = to_bf16(y1, zb, Td, s)) != TQP_OK) return rc;
-  if ((rc = layer_forward(zb, T, G, y2, 1, -1.0f, x2, 0, nullptr, lws, dev_status, s)) != TQP_OK) return rc;
-  if ((rc = tqp_moe_layer_bwd(zb, dy2, T, G, dxG, gG, lws, lws_bytes, dev_status, stream)) != TQP_OK) return rc;
+  uint16_t* gu = carve_bwd(static_cast<char*>(lws) + layer_ws_size(T, G), T, G).gu;
+  if ((rc = layer_forward(zb, T, G, y2, 1, -1.0f, x2, 0, nullptr, lws, dev_status, s, gu)) != TQP_OK) return rc;
+  if ((rc = layer_backward(zb, dy2, T, G, dxG, gG, lws, dev_status, s, false)) != TQP_OK) return rc;
   // dz1 = dy1 + J_G^T dy2 -> dx1 (dx1 = dz1)
   if ((rc = launch_add_f32(dy1, dxG, dx1, Td, s)) != TQP_OK) return rc;
   // F-step: x1 = y1 - F(x2); F's grads for cotangent dz1; dx2 = dy2 + J_F^T dz1
-  if ((rc = layer_forward(x2, T, F, y1, 1, -1.0f, x1, 0, nullptr, lws, dev_status, s)) != TQP_OK) return rc;
-  if ((rc = tqp_moe_layer_bwd(x2, dx1, T, F, dxG, gF, lws, lws_bytes, dev_status, stream)) != TQP_OK) return rc;
+  gu = carve_bwd(static_cast<char*>(lws) + layer_ws_size(T, F), T, F).gu;
+  if ((rc = layer_forward(x2, T, F, y1, 1, -1.0f, x1, 0, nullptr, lws, dev_status, s, gu)) != TQP_OK) return rc;
+  if ((rc = layer_backward(x2, dx1, T, F, dxG, gF, lws, dev_status, s, false)) != TQP_OK) return rc;
   return launch_add_f32(dy2, dxG, dx2, Td, s);
 }
 
