@@ -94,3 +94,46 @@ def test_grouped_ffn_part_rejects_unknown_part():
     # a valid part with an empty batch is a no-op that enqueues nothing
     rc = L.tqp_grouped_ffn_part(Q.FFN_GATE_UP, None, 0, None, None, ctypes.byref(w), None, None, None, 0, None, None)
     assert rc == 0
+
+
+@pytest.mark.parametrize("cfg", [synth.TINY, synth.MID, synth.FULL], ids=lambda c: c.name)
+def test_backward_workspace_holds_its_scratch(cfg):
+    # the backward adds, per routed row, G|U and dG|dU (2f each), dO (d), dha (r) and
+    # dxa (2r) as fp16, plus the K-major fp16 B operand of the rank-space products:
+    # Bd as [E][r][d] or blockdiag(Bg, Bu) as [E][2r][2f], whichever is larger
+    L = Q.lib()
+    w = _struct(cfg)
+    A = cfg.T * cfg.k
+    extra = (L.tqp_moe_layer_bwd_workspace_size(cfg.T, ctypes.byref(w))
+             - L.tqp_moe_layer_workspace_size(cfg.T, ctypes.byref(w)))
+    need = A * (4 * cfg.f + cfg.d + 3 * cfg.r) * 2 + cfg.E * max(cfg.r * cfg.d, 4 * cfg.r * cfg.f) * 2
+    assert need <= extra <= need + 8 * 256 + 256
+
+
+def _grads(**bad):
+    g = Q.Grads()
+    for p in range(3):
+        g.dA[p] = 0x50000 + 0x1000 * p
+        g.dB[p] = 0x60000 + 0x1000 * p
+    for k_, (p, v) in bad.items():
+        getattr(g, k_)[p] = v
+    return g
+
+
+@pytest.mark.parametrize("bad", [dict(dA=(1, None)), dict(dB=(2, None)), dict(dA=(0, 0x50004)), dict(dB=(0, 0x60008))],
+                         ids=["dA1-null", "dB2-null", "dA0-misaligned", "dB0-misaligned"])
+def test_backward_rejects_bad_gradient_buffers_before_any_launch(bad):
+    # both layers' gradient buffers are checked on the host before the first launch
+    L = Q.lib()
+    F, G = _struct(synth.TINY), _struct(synth.TINY)
+    good, wrong = _grads(), _grads(**bad)
+    p = 0x70000
+    for gF, gG in ((wrong, good), (good, wrong)):
+        rc = L.tqp_adapter_bwd(p, p, p, p, 64, ctypes.byref(F), ctypes.byref(G), p, p, p, p, ctypes.byref(gF),
+                               ctypes.byref(gG), p, 1 << 30, None, None)
+        assert rc == -1, rc
+    assert L.tqp_moe_layer_bwd(p, p, 64, ctypes.byref(F), p, ctypes.byref(wrong), p, 1 << 30, None, None) == -1
+    # rank 0 has no adapters: null gradient buffers are fine (T = 0: nothing is enqueued)
+    F0 = _struct(synth.TINY, rank=0)
+    null = Q.Grads()
+    assert L.tqp_moe_layer_bwd(None, None, 0, ctypes.byref(F0), None, ctypes.byref(null), None, 0, None, None) == 0
