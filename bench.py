@@ -57,6 +57,13 @@ def layer_flops(cfg: synth.LayerConfig) -> dict:
             "ffn": expert + lora, "gate_up": gate_up}
 
 
+def workload_config(cfg: synth.LayerConfig) -> dict:
+    """The workload as both arms report it in `config`."""
+    return {"workload": f"{cfg.name}: T={cfg.T} d={cfg.d} E={cfg.E} top-{cfg.k} ffn={cfg.f} int4 g{cfg.g} LoRA r{cfg.r}"
+                        f"{' zipf-bias' if cfg.zipf_s else ''}, layer forward",
+            "T": cfg.T, "d": cfg.d, "E": cfg.E, "k": cfg.k, "ffn": cfg.f, "group": cfg.g, "rank": cfg.r}
+
+
 def rank_token_seed(cfg: synth.LayerConfig, rank: int) -> int:
     """Each rank draws its own token batch (data parallel, weak scaling)."""
     return cfg.seed + rank
@@ -368,11 +375,8 @@ def run_tqp(args, rank: int, world: int, local_rank: int) -> dict | None:
         "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms, "higher_is_better": True,
         "scaling": "weak", "vs_baseline": None, "dtype": "f16",
         "data": "synthetic (seeded N(0,1) tokens, N(0,1/d) weights int4-quantised, random-init LoRA)",
-        "config": {"workload": f"{cfg.name}: T={T} d={d} E={E} top-{k} ffn={f} int4 g{cfg.g} LoRA r{cfg.r}"
-                               f"{' zipf-bias' if cfg.zipf_s else ''}, layer forward",
-                   "T": T, "d": d, "E": E, "k": k, "ffn": f, "group": cfg.g, "rank": cfg.r,
-                   "l2": "flushed before every step (512 MB write); weights 1.4 GB > L2",
-                   "parallelism": f"dp{world} (independent token batches, replicated weights)"},
+        "config": dict(workload_config(cfg), l2="flushed before every step (512 MB write); weights 1.4 GB > L2",
+                       parallelism=f"dp{world} (independent token batches, replicated weights)"),
         "tflops": fl["total"] / (ms * 1e-3) / 1e12 * world,
         "assignments_per_s": world * A / (ms * 1e-3),
         "per_call_ms": dict(per_call_ms, grouped_ffn=ffn_ms),
@@ -416,7 +420,7 @@ def run_reference(args, rank: int) -> dict | None:
     return {"impl": "reference", "metric": METRIC, "value": v, "unit": UNIT, "n_gpus": 1,
             "steps": args.steps, "warmup": args.warmup, "ms_per_step": sample / v * 1e3,
             "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
-            "data": "synthetic", "config": {"workload": f"{cfg.name}, layer forward, oracle on a {sample}-token sample"},
+            "data": "synthetic", "config": dict(workload_config(cfg), sample=f"oracle on the first {sample} tokens per step"),
             "cpu_baseline": {"value": v, "unit": UNIT, "cores": cores(), "kind": "oracle", "sample": vals[0]["sample"]},
             "e2e": {"value": v, "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
 
