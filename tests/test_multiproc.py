@@ -72,3 +72,10 @@ def test_reference_arm_runs_on_rank0_only():
     line = json.loads(r0.stdout.strip().splitlines()[-1])
     assert line["impl"] == "reference" and line["value"] > 0
     assert line["cpu_baseline"]["kind"] == "oracle" and line["e2e"]["h2d_bytes_per_step"] == 0
+    # same metric and workload description as the GPU arm, so the two lines compare
+    sys.path.insert(0, ROOT)
+    import bench
+    import synth
+    want = bench.workload_config(synth.CONFIGS["tiny"])
+    assert line["metric"] == bench.METRIC and line["unit"] == bench.UNIT and line["higher_is_better"] is True
+    assert {k: line["config"][k] for k in want} == want
