@@ -57,6 +57,18 @@ def layer_flops(cfg: synth.LayerConfig) -> dict:
             "ffn": expert + lora, "gate_up": gate_up}
 
 
+def layer_bwd_flops(cfg: synth.LayerConfig) -> float:
+    """Algorithmic FLOPs of one layer's adapter-only backward (base and router frozen).
+
+    Expert dgrads dH = dO Wd and dX = dG Wg + dU Wu: 6 A d f. Adapter terms, each
+    a 2 A r n product (n = d or f): down dBd, dha, dAd and the rank term of dH;
+    gate/up dBg, dBu, dxa, dAg, dAu and the rank term of dX: 12 A r (d + f).
+    Gate dot products and the router's input gradient: 4 A d.
+    """
+    A = cfg.T * cfg.k
+    return 6.0 * A * cfg.d * cfg.f + 12.0 * A * cfg.r * (cfg.d + cfg.f) + 4.0 * A * cfg.d
+
+
 def workload_config(cfg: synth.LayerConfig) -> dict:
     """The workload as both arms report it in `config`."""
     return {"workload": f"{cfg.name}: T={cfg.T} d={cfg.d} E={cfg.E} top-{cfg.k} ffn={cfg.f} int4 g{cfg.g} LoRA r{cfg.r}"
@@ -242,8 +254,12 @@ def time_rev_block(L_F, dev, steps: int, warmup: int, flush) -> dict:
     err = float(max((f(r1) - f(x1)).abs().max(), (f(r2) - f(x2)).abs().max()) / rms)
     mean = {n: statistics.mean(v) for n, v in ms.items()}
     step_ms = mean["fwd"] + mean["adapter_bwd"]
+    # forward: F and G; adapter backward: the inverse (F and G again) and both layers' backward
+    fwd_flop = layer_flops(cfgF)["total"] + layer_flops(cfgG)["total"]
+    step_flop = 2.0 * fwd_flop + layer_bwd_flops(cfgF) + layer_bwd_flops(cfgG)
     return {"workload": f"two {cfgF.name} layers F, G; streams 2 x {T}x{d}; forward, inverse, adapter backward",
             "ms_per_step": step_ms, "tokens_per_s": T / (step_ms * 1e-3), "ms": mean, "steps": steps,
+            "flop_per_step": step_flop, "tflops": step_flop / (step_ms * 1e-3) / 1e12,
             "reconstruction_max_err_rel_rms": err, "l2": "flushed before every call"}
 
 

@@ -17,3 +17,20 @@ def test_excess_error_sees_real_errors():
     bad = y.copy()
     bad[17] += 0.1 * np.sqrt(np.mean(y * y))
     assert rel_err_bf16_out(O.round_bf16(bad), y) > 0.09
+
+
+def test_block_flop_counts_match_the_survey_estimates():
+    # one full-config layer: forward 996 GFLOP (router 15.4, experts 927.7, LoRA 53.2);
+    # adapter-only backward: dgrad ~928 + adapter gradients ~106 GFLOP
+    import bench
+    import synth
+    fl = bench.layer_flops(synth.FULL)
+    assert abs(fl["router"] / 1e9 - 15.4) < 0.1 and abs(fl["expert"] / 1e9 - 927.7) < 0.1
+    assert abs(fl["lora"] / 1e9 - 53.2) < 0.1
+    bwd = bench.layer_bwd_flops(synth.FULL) / 1e9
+    assert abs(bwd - (927.7 + 106.3 + 0.8)) < 0.2
+    # rank 0: only the expert dgrads and the small gate/router terms remain
+    import dataclasses
+    r0 = dataclasses.replace(synth.FULL, r=0)
+    A = r0.T * r0.k
+    assert bench.layer_bwd_flops(r0) == 6.0 * A * r0.d * r0.f + 4.0 * A * r0.d
