@@ -209,6 +209,12 @@ class DeviceLayer:
             g.dB[p] = dB[p].data_ptr()
         return dA, dB, g
 
+    def flat_grads(self, device="cuda"):
+        """The same buffers as views of one flat fp32 tensor (dp.FlatGrads), so a
+        data-parallel backward sums them over ranks in a single all-reduce."""
+        from .dp import FlatGrads
+        return FlatGrads(self.E, self.d, self.f, self.r, device)
+
 
 # ---------------------------------------------------------------- entry points (same names as the C ABI)
 

@@ -1,10 +1,12 @@
 """Multi-process host logic of the benchmark, on CPU (gloo, world size 2).
 
 The layer shards by tokens: every rank runs the whole hot path on its own batch
-with replicated weights, and the only cross-rank step is the timing reduction
-(max over ranks of the step time). That reduction, the per-rank batch choice and
-the whole-job metric are what these tests pin; the reference arm's N>1 behaviour
-(rank 0 alone runs and prints) is checked on a tiny workload.
+with replicated weights. The forward's only cross-rank step is the timing
+reduction (max over ranks of the step time); the backward's is the sum of the
+adapter gradients over ranks (dp.allreduce_adapter_grads, one all-reduce of a
+flat buffer per layer). These tests pin both reductions, the per-rank batch
+choice and the whole-job metric; the reference arm's N>1 behaviour (rank 0 alone
+runs and prints) is checked on a tiny workload.
 """
 import json
 import os
@@ -79,3 +81,57 @@ def test_reference_arm_runs_on_rank0_only():
     want = bench.workload_config(synth.CONFIGS["tiny"])
     assert line["metric"] == bench.METRIC and line["unit"] == bench.UNIT and line["higher_is_better"] is True
     assert {k: line["config"][k] for k in want} == want
+
+
+def _grad_worker(rank, world, port, out):
+    os.environ["MASTER_ADDR"] = "127.0.0.1"
+    os.environ["MASTER_PORT"] = str(port)
+    import datetime
+    from quantized_base_lora_moe_b200.dp import FlatGrads, allreduce_adapter_grads
+    dist.init_process_group("gloo", rank=rank, world_size=world, timeout=datetime.timedelta(seconds=60))
+    try:
+        g = FlatGrads(E=4, d=64, f=128, r=8, device="cpu")
+        # each rank's gradients: rank-dependent values, different per tensor
+        for p in range(3):
+            g.dA[p].fill_((rank + 1) * (p + 1))
+            g.dB[p].fill_((rank + 1) * 10.0 * (p + 1))
+        g.dA[2][1, 3, 5] = 1000.0 * (rank + 1)           # one distinct element, to catch offset mix-ups
+        assert allreduce_adapter_grads(g) is None
+        s = sum(i + 1 for i in range(world))
+        ok = all(bool(torch.all(g.dB[p] == s * 10.0 * (p + 1))) for p in range(3))
+        ok &= bool(torch.all(g.dA[0] == s)) and bool(torch.all(g.dA[1] == 2 * s))
+        ok &= float(g.dA[2][1, 3, 5]) == 1000.0 * s and float(g.dA[2][1, 3, 4]) == 3 * s
+        # asynchronous form: the handle completes the same sum
+        g.zero_()
+        g.dB[1].fill_(rank + 0.5)
+        work = allreduce_adapter_grads(g, async_op=True)
+        work.wait()
+        ok &= bool(torch.all(g.dB[1] == sum(i + 0.5 for i in range(world)))) and float(g.flat.abs().sum()) == \
+            float(g.dB[1].abs().sum())
+        out[rank] = ok
+    finally:
+        dist.destroy_process_group()
+
+
+def test_adapter_gradient_allreduce_two_ranks():
+    port = 31500 + (os.getpid() % 2000)
+    out = mp.Manager().dict()
+    mp.spawn(_grad_worker, args=(2, port, out), nprocs=2, join=True)
+    assert out[0] and out[1]
+
+
+def test_flat_gradient_views_alias_one_buffer():
+    from quantized_base_lora_moe_b200.dp import FlatGrads, allreduce_adapter_grads
+    g = FlatGrads(E=3, d=128, f=256, r=16, device="cpu")
+    n = 3 * 16 * (128 + 128 + 256) + 3 * 16 * (256 + 256 + 128)
+    assert g.flat.numel() == n
+    base = g.flat.data_ptr()
+    for t in g.dA + g.dB:
+        assert t.data_ptr() % 32 == 0 and base <= t.data_ptr() < base + 4 * n
+        t.fill_(1.0)
+    assert float(g.flat.sum()) == n                           # the views tile the buffer exactly
+    for p in range(3):
+        assert g.struct.dA[p] == g.dA[p].data_ptr() and g.struct.dB[p] == g.dB[p].data_ptr()
+    assert allreduce_adapter_grads(g) is None                 # no process group: nothing to exchange
+    r0 = FlatGrads(E=3, d=128, f=256, r=0, device="cpu")
+    assert r0.flat.numel() == 0 and allreduce_adapter_grads(r0) is None
