@@ -219,6 +219,11 @@ class DeviceLayer:
 # ---------------------------------------------------------------- entry points (same names as the C ABI)
 
 
+def _grads(g):
+    """A tqp_adapter_grads struct, or a dp.FlatGrads (its struct)."""
+    return g.struct if hasattr(g, "struct") and not isinstance(g, Grads) else g
+
+
 def moe_router_gemm(x, layer: DeviceLayer, logits, ws=None, status: Status | None = None, stream=None):
     _require_cuda(x, logits)
     T = x.shape[0]
@@ -334,7 +339,7 @@ def tqp_moe_layer_bwd(x, dy, layer: DeviceLayer, dx, grads, ws=None, status: Sta
     n = lib().tqp_moe_layer_bwd_workspace_size(T, layer.ref())
     ws = ws if ws is not None else workspace(n, x.device)
     _check("tqp_moe_layer_bwd", lib().tqp_moe_layer_bwd(x.data_ptr(), dy.data_ptr(), T, layer.ref(), dx.data_ptr(),
-                                                        ctypes.byref(grads), ws.data_ptr(), ws.numel(),
+                                                        ctypes.byref(_grads(grads)), ws.data_ptr(), ws.numel(),
                                                         status.ptr() if status else None, _stream(stream)))
     return dx
 
@@ -347,7 +352,7 @@ def tqp_adapter_bwd(y1, y2, dy1, dy2, F: DeviceLayer, G: DeviceLayer, x1, x2, dx
     ws = ws if ws is not None else workspace(n, y1.device)
     _check("tqp_adapter_bwd", lib().tqp_adapter_bwd(y1.data_ptr(), y2.data_ptr(), dy1.data_ptr(), dy2.data_ptr(), T,
                                                     F.ref(), G.ref(), x1.data_ptr(), x2.data_ptr(), dx1.data_ptr(),
-                                                    dx2.data_ptr(), ctypes.byref(gF), ctypes.byref(gG),
+                                                    dx2.data_ptr(), ctypes.byref(_grads(gF)), ctypes.byref(_grads(gG)),
                                                     ws.data_ptr(), ws.numel(), status.ptr() if status else None,
                                                     _stream(stream)))
     return x1, x2, dx1, dx2

@@ -133,5 +133,7 @@ def test_flat_gradient_views_alias_one_buffer():
     for p in range(3):
         assert g.struct.dA[p] == g.dA[p].data_ptr() and g.struct.dB[p] == g.dB[p].data_ptr()
     assert allreduce_adapter_grads(g) is None                 # no process group: nothing to exchange
+    import quantized_base_lora_moe_b200 as Q
+    assert Q._grads(g) is g.struct                            # the backward calls take a FlatGrads as well
     r0 = FlatGrads(E=3, d=128, f=256, r=0, device="cpu")
     assert r0.flat.numel() == 0 and allreduce_adapter_grads(r0) is None
