@@ -256,7 +256,12 @@ int rev_couple_inv(const float* y1, const float* y2, int T, const tqp_moe_weight
  *   x [T][d] bf16; dy [T][d] fp32 -> dx [T][d] fp32 (through the experts and,
  *   via the softmax over the chosen logits, through the frozen router), and the
  *   adapter gradients `grads`. Top-k selection is treated as constant.
- *   ws: tqp_moe_layer_bwd_workspace_size.
+ *   grads: dA[p] [E][r][in_p], dB[p] [E][out_p][r] fp32, caller-owned device
+ *   memory, overwritten (not accumulated). With rank > 0 each must be non-null
+ *   and 16-byte aligned, else TQP_ERR_INVALID_ARG before any launch; ffn must be
+ *   a multiple of 128, else TQP_ERR_UNSUPPORTED.
+ *   ws: tqp_moe_layer_bwd_workspace_size (the layer's forward workspace plus
+ *   G|U, dG|dU, dO, dha, dxa and the rank-space B operand in fp16).
  * ------------------------------------------------------------------------- */
 size_t tqp_moe_layer_bwd_workspace_size(int T, const tqp_moe_weights* w);
 int tqp_moe_layer_bwd(const uint16_t* x, const float* dy, int T, const tqp_moe_weights* w, float* dx,
@@ -272,7 +277,10 @@ int tqp_moe_layer_bwd(const uint16_t* x, const float* dy, int T, const tqp_moe_w
  *   F-step: x1 = y1 - F(x2); F's adapter grads for cotangent dz1;
  *           dx2 = dy2 + J_F(x2)^T dz1; dx1 = dz1.
  *   y1, y2, dy1, dy2 [T][d] fp32 in; x1, x2 [T][d] bf16 out (reconstructed);
- *   dx1, dx2 [T][d] fp32 out; gF, gG adapter gradients of F and G.
+ *   dx1, dx2 [T][d] fp32 out; gF, gG adapter gradients of F and G (both
+ *   checked on the host, as for tqp_moe_layer_bwd, before any launch).
+ *   Each layer's backward reuses the routing and intermediates of the inverse
+ *   step that ran that layer's forward, so no layer forward runs twice.
  *   ws: tqp_adapter_bwd_workspace_size.
  * ------------------------------------------------------------------------- */
 size_t tqp_adapter_bwd_workspace_size(int T, const tqp_moe_weights* F, const tqp_moe_weights* G);
