@@ -257,132 +257,236 @@ def time_rev_block(L_F, dev, steps: int, warmup: int, flush) -> dict:
     # forward: F and G; adapter backward: the inverse (F and G again) and both layers' backward
     fwd_flop = layer_flops(cfgF)["total"] + layer_flops(cfgG)["total"]
     step_flop = 2.0 * fwd_flop + layer_bwd_flops(cfgF) + layer_bwd_flops(cfgG)
+    pk = peaks()
+    tflops = step_flop / (step_ms * 1e-3) / 1e12
     return {"workload": f"two {cfgF.name} layers F, G; streams 2 x {T}x{d}; forward, inverse, adapter backward",
             "ms_per_step": step_ms, "tokens_per_s": T / (step_ms * 1e-3), "ms": mean, "steps": steps,
-            "flop_per_step": step_flop, "tflops": step_flop / (step_ms * 1e-3) / 1e12,
+            "flop_per_step": step_flop, "tflops": tflops,
+            "roofline_frac_measured": tflops / pk["bf16_tflops"], "roofline_frac_nominal": tflops / 2250.0,
             "reconstruction_max_err_rel_rms": err, "l2": "flushed before every call"}
+
+
+def layer_bytes(cfg: synth.LayerConfig, touched: int) -> float:
+    """Algorithmic bytes of one layer forward: int4 codes, bf16 group scales and
+    bf16 LoRA factors of the touched experts, fp32 router weights, x and y in
+    bf16, ids and gates. Intermediates (logits, H, O) are implementation traffic."""
+    d, f, g, r = cfg.d, cfg.f, cfg.g, cfg.r
+    per_expert = 3 * d * f / 2 + (2 * (d // g) * f + (f // g) * d) * 2 + 3 * r * (d + f) * 2
+    return touched * per_expert + cfg.E * d * 4 + 2 * cfg.T * d * 2 + cfg.T * cfg.k * 8
+
+
+def layer_roofline(cfg: synth.LayerConfig, touched: int, ms: float) -> dict:
+    """The layer against its roofline: the slower of its FLOPs at the tensor
+    peak and its algorithmic bytes at the HBM peak, for the nominal peaks
+    (2.25 PFLOP/s dense bf16, 8 TB/s) and for the measured ones."""
+    fl = layer_flops(cfg)["total"]
+    by = layer_bytes(cfg, touched)
+    pk = peaks()
+    t_nom = max(fl / 2.25e15, by / 8.0e12)
+    t_meas = max(fl / (pk["bf16_tflops"] * 1e12), by / (pk["hbm_gbs"] * 1e9))
+    return {"bound": "tensor" if fl / 2.25e15 >= by / 8.0e12 else "hbm", "flop": fl, "bytes": by,
+            "touched_experts": touched, "achieved_tflops": fl / (ms * 1e-3) / 1e12,
+            "roofline_ms_nominal": t_nom * 1e3, "frac_nominal": t_nom / (ms * 1e-3),
+            "roofline_ms_measured": t_meas * 1e3, "frac_measured": t_meas / (ms * 1e-3),
+            "peaks": {"nominal": "2.25 PFLOP/s dense bf16, 8 TB/s HBM",
+                      "measured": f"{pk['bf16_tflops']} TFLOP/s bf16 burst, {pk['hbm_gbs']} GB/s ({pk['source']})"}}
+
+
+CALLS = ["router_gemm", "route", "permute", "ffn_prepare", "ffn_gate_up", "ffn_rank", "ffn_down", "combine"]
+
+
+class LayerBench:
+    """One configuration's weights, batch and buffers on the device, and the
+    layer forward step issued as the public C-ABI calls (the grouped FFN as its
+    four parts, so that the gate/up expert kernel is timed on its own)."""
+
+    def __init__(self, cfg: synth.LayerConfig, dev, token_seed: int, host: dict | None = None):
+        import torch
+        import quantized_base_lora_moe_b200 as Q
+        self.Q, self.cfg, self.dev = Q, cfg, dev
+        self.host = host if host is not None else synth.make_layer(cfg)
+        self.x_bits = synth.make_tokens(cfg.T, cfg.d, token_seed)
+        self.L = Q.DeviceLayer(self.host, device=dev)
+        T, E, k, d, f = cfg.T, cfg.E, cfg.k, cfg.d, cfg.f
+        A = T * k
+        self.x = torch.from_numpy(self.x_bits.view(np.int16)).to(dev)
+        self.y = torch.empty(T, d, dtype=torch.int16, device=dev)
+        self.logits = torch.empty(T, E, dtype=torch.float32, device=dev)
+        self.ids = torch.empty(T, k, dtype=torch.int32, device=dev)
+        self.gates = torch.empty(T, k, dtype=torch.float32, device=dev)
+        self.offsets = torch.empty(E + 1, dtype=torch.int32, device=dev)
+        self.perm = torch.empty(A, dtype=torch.int32, device=dev)
+        self.inv = torch.empty(A, dtype=torch.int32, device=dev)
+        self.h = torch.empty(A, f, dtype=torch.int16, device=dev)
+        self.o = torch.empty(A, d, dtype=torch.int16, device=dev)
+        lib = Q.lib()
+        self.ws_r = Q.workspace(lib.moe_router_gemm_workspace_size(T, self.L.ref()), dev)
+        self.ws_p = Q.workspace(lib.moe_permute_workspace_size(T, E, k), dev)
+        self.ws_f = Q.workspace(lib.tqp_grouped_ffn_workspace_size(T, self.L.ref()), dev)
+        self.ws_l = Q.workspace(lib.tqp_moe_layer_workspace_size(T, self.L.ref()), dev)
+        self.st = Q.Status(dev)
+        self.stream = torch.cuda.current_stream(dev)
+        lora = cfg.r > 0
+        # kernels per call: router split + GEMM; route; permute count, column scan,
+        # scatter; prepare = two block schedules, x (and Ad) to fp16, s X [Ag|Au];
+        # gate/up and down = unit table + expert kernel; rank = s H Ad; combine
+        self.launches = {"router_gemm": 2, "route": 1, "permute": 3, "ffn_prepare": 5 if lora else 3,
+                         "ffn_gate_up": 2, "ffn_rank": 1 if lora else 0, "ffn_down": 2, "combine": 1}
+
+    def step(self, evs=None):
+        Q, c = self.Q, self.cfg
+
+        def mark(i):
+            if evs is not None:
+                evs[i].record(self.stream)
+        mark(0)
+        Q.moe_router_gemm(self.x, self.L, self.logits, self.ws_r, self.st)
+        mark(1)
+        Q.moe_route(self.logits, c.k, self.ids, self.gates, self.st)
+        mark(2)
+        Q.moe_permute(self.ids, c.E, self.offsets, self.perm, self.inv, self.ws_p, self.st)
+        mark(3)
+        for j, part in enumerate([Q.FFN_PREPARE, Q.FFN_GATE_UP, Q.FFN_RANK, Q.FFN_DOWN]):
+            Q.tqp_grouped_ffn_part(part, self.x, self.offsets, self.perm, self.L, self.h, self.o, self.ws_f, self.st)
+            mark(4 + j)
+        Q.moe_combine(self.o, self.inv, self.gates, self.y)
+        mark(8)
+
+    def run(self, steps: int, warmup: int, flush, before_timed=None) -> dict:
+        """Warm-up, then `steps` timed steps with an L2 flush before each (outside
+        the per-step events). Returns per-call mean ms and the per-step ms."""
+        import torch
+        for _ in range(warmup):
+            flush.zero_()
+            self.step()
+        torch.cuda.synchronize(self.dev)
+        if self.st.read() != 0:
+            raise RuntimeError(f"device status {self.st.read()} after warm-up ({self.cfg.name})")
+        evs = [[torch.cuda.Event(enable_timing=True) for _ in range(len(CALLS) + 1)] for _ in range(steps)]
+        if before_timed:
+            before_timed()
+        torch.cuda.synchronize(self.dev)
+        for i in range(steps):
+            flush.zero_()
+            self.step(evs[i])
+        torch.cuda.synchronize(self.dev)
+        if self.st.read() != 0:
+            raise RuntimeError(f"device status {self.st.read()} after the timed steps ({self.cfg.name})")
+        per_call = {n: statistics.mean(e[j].elapsed_time(e[j + 1]) for e in evs) for j, n in enumerate(CALLS)}
+        step_ms = [e[0].elapsed_time(e[len(CALLS)]) for e in evs]
+        return {"per_call_ms": per_call, "step_ms": step_ms}
+
+    def touched_experts(self) -> int:
+        off = self.offsets.cpu().numpy()
+        return int(np.count_nonzero(np.diff(off)))
+
+    def summary(self, timing: dict) -> dict:
+        """Throughput, per-call times and rooflines of one configuration."""
+        cfg = self.cfg
+        fl = layer_flops(cfg)
+        pk = peaks()
+        ms = statistics.mean(timing["step_ms"])
+        pc = timing["per_call_ms"]
+        gu_tflops = fl["gate_up"] / (pc["ffn_gate_up"] * 1e-3) / 1e12
+        return {"workload": workload_config(cfg)["workload"], "ms_per_step": ms,
+                "tokens_per_s": cfg.T / (ms * 1e-3), "assignments_per_s": cfg.T * cfg.k / (ms * 1e-3),
+                "tflops": fl["total"] / (ms * 1e-3) / 1e12, "per_call_ms": pc,
+                "gate_up_frac": gu_tflops / pk["bf16_tflops"],
+                "layer_roofline": layer_roofline(cfg, self.touched_experts(), ms)}
+
+
+def time_e2e(lb: LayerBench, steps: int, dev, dist: bool, world: int) -> dict:
+    """The metric through the public API from pinned host memory: each step
+    copies its token batch in, runs tqp_moe_layer_fwd and copies the layer
+    output back. Two device buffers alternate, so that the copies of one step
+    overlap the compute of the neighbouring steps (copy-in and copy-out streams,
+    ordered by events)."""
+    import torch
+    Q, cfg = lb.Q, lb.cfg
+    T, d = cfg.T, cfg.d
+    x_host = torch.from_numpy(lb.x_bits.view(np.int16)).pin_memory()
+    y_host = [torch.empty(T, d, dtype=torch.int16).pin_memory() for _ in range(2)]
+    x_dev = [torch.empty_like(lb.x) for _ in range(2)]
+    y_dev = [torch.empty_like(lb.y) for _ in range(2)]
+    comp = lb.stream
+    s_in, s_out = torch.cuda.Stream(dev), torch.cuda.Stream(dev)
+    ev = lambda: torch.cuda.Event()
+    in_done, comp_done, out_done = [ev(), ev()], [ev(), ev()], [ev(), ev()]
+    for b in range(2):
+        comp_done[b].record(comp)
+        out_done[b].record(comp)
+
+    def one(i):
+        b = i % 2
+        s_in.wait_event(comp_done[b])            # step i-2's layer has read x_dev[b]
+        with torch.cuda.stream(s_in):
+            x_dev[b].copy_(x_host, non_blocking=True)
+        in_done[b].record(s_in)
+        comp.wait_event(in_done[b])
+        comp.wait_event(out_done[b])             # step i-2's output has left y_dev[b]
+        Q.tqp_moe_layer_fwd(x_dev[b], lb.L, y_dev[b], lb.ws_l, lb.st)
+        comp_done[b].record(comp)
+        s_out.wait_event(comp_done[b])
+        with torch.cuda.stream(s_out):
+            y_host[b].copy_(y_dev[b], non_blocking=True)
+        out_done[b].record(s_out)
+
+    for i in range(2):
+        one(i)
+    torch.cuda.synchronize(dev)
+    if dist:
+        torch.distributed.barrier()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record(comp)
+    s_in.wait_event(e0)
+    for i in range(steps):
+        one(i)
+    comp.wait_event(out_done[(steps - 1) % 2])
+    comp.wait_event(out_done[steps % 2])
+    e1.record(comp)
+    torch.cuda.synchronize(dev)
+    e2e_ms = max_over_ranks(e0.elapsed_time(e1), dev, dist) / steps
+    return {"value": weak_scaling_value(world, T, e2e_ms), "unit": UNIT, "h2d_bytes_per_step": int(T * d * 2),
+            "d2h_bytes_per_step": int(T * d * 2), "ms_per_step": e2e_ms,
+            "note": "tqp_moe_layer_fwd per step; copy-in, compute and copy-out of neighbouring steps overlap "
+                    "(two device buffers, three streams)"}
 
 
 def run_tqp(args, rank: int, world: int, local_rank: int) -> dict | None:
     import torch
-    import quantized_base_lora_moe_b200 as Q
     torch.cuda.set_device(local_rank)
     dev = torch.device("cuda", local_rank)
     cfg = synth.CONFIGS[args.config]
-    host = synth.make_layer(cfg)
-    x_bits = synth.make_tokens(cfg.T, cfg.d, rank_token_seed(cfg, rank))
-    L = Q.DeviceLayer(host, device=dev)
-    T, E, k, d, f = cfg.T, cfg.E, cfg.k, cfg.d, cfg.f
-    A = T * k
-    x = torch.from_numpy(x_bits.view(np.int16)).to(dev)
-    y = torch.empty(T, d, dtype=torch.int16, device=dev)
-    logits = torch.empty(T, E, dtype=torch.float32, device=dev)
-    ids = torch.empty(T, k, dtype=torch.int32, device=dev)
-    gates = torch.empty(T, k, dtype=torch.float32, device=dev)
-    offsets = torch.empty(E + 1, dtype=torch.int32, device=dev)
-    perm = torch.empty(A, dtype=torch.int32, device=dev)
-    inv = torch.empty(A, dtype=torch.int32, device=dev)
-    h = torch.empty(A, f, dtype=torch.int16, device=dev)
-    o = torch.empty(A, d, dtype=torch.int16, device=dev)
-    lib = Q.lib()
-    ws_r = Q.workspace(lib.moe_router_gemm_workspace_size(T, L.ref()), dev)
-    ws_p = Q.workspace(lib.moe_permute_workspace_size(T, E, k), dev)
-    ws_f = Q.workspace(lib.tqp_grouped_ffn_workspace_size(T, L.ref()), dev)
-    ws_l = Q.workspace(lib.tqp_moe_layer_workspace_size(T, L.ref()), dev)
-    st = Q.Status(dev)
+    lb = LayerBench(cfg, dev, rank_token_seed(cfg, rank))
     flush = torch.empty(L2_FLUSH_BYTES, dtype=torch.uint8, device=dev)
-    stream = torch.cuda.current_stream(dev)
-    # the grouped FFN is issued as its four parts, so that the gate/up expert
-    # kernel (one launch, the dominant one) is timed on its own
-    names = ["router_gemm", "route", "permute", "ffn_prepare", "ffn_gate_up", "ffn_rank", "ffn_down", "combine"]
-    lora = cfg.r > 0
-    launches_per_step = {"router_gemm": 2, "route": 1, "permute": 3, "ffn_prepare": 4 if lora else 2,
-                         "ffn_gate_up": 1, "ffn_rank": 1 if lora else 0, "ffn_down": 1, "combine": 1}
-    ffn_parts = [Q.FFN_PREPARE, Q.FFN_GATE_UP, Q.FFN_RANK, Q.FFN_DOWN]
-
-    def step(evs=None):
-        def mark(i):
-            if evs is not None:
-                evs[i].record(stream)
-        mark(0)
-        Q.moe_router_gemm(x, L, logits, ws_r, st)
-        mark(1)
-        Q.moe_route(logits, k, ids, gates, st)
-        mark(2)
-        Q.moe_permute(ids, E, offsets, perm, inv, ws_p, st)
-        mark(3)
-        for j, part in enumerate(ffn_parts):
-            Q.tqp_grouped_ffn_part(part, x, offsets, perm, L, h, o, ws_f, st)
-            mark(4 + j)
-        Q.moe_combine(o, inv, gates, y)
-        mark(8)
-
     dist = world > 1
-    for _ in range(args.warmup):
-        flush.zero_()
-        step()
-    torch.cuda.synchronize(dev)
-    if st.read() != 0:
-        raise RuntimeError(f"device status {st.read()} after warm-up")
-    evs = [[torch.cuda.Event(enable_timing=True) for _ in range(len(names) + 1)] for _ in range(args.steps)]
     clocks = ClockSampler(int(os.environ.get("CUDA_VISIBLE_DEVICES", str(local_rank)).split(",")[0])
                           if "CUDA_VISIBLE_DEVICES" in os.environ else local_rank)
-    if rank == 0:
-        clocks.start()
-        time.sleep(0.4)
-    if dist:
-        torch.distributed.barrier()
-    torch.cuda.synchronize(dev)
-    for i in range(args.steps):
-        flush.zero_()                       # L2 flush, outside the per-step events
-        step(evs[i])
-    torch.cuda.synchronize(dev)
+
+    def before_timed():
+        if rank == 0:
+            clocks.start()
+            time.sleep(0.4)
+        if dist:
+            torch.distributed.barrier()
+
+    timing = lb.run(args.steps, args.warmup, flush, before_timed)
     if dist:
         torch.distributed.barrier()
     clk = clocks.stop() if rank == 0 else None
-    per_call = {n: [] for n in names}
-    step_ms = []
-    for e in evs:
-        for j, n in enumerate(names):
-            per_call[n].append(e[j].elapsed_time(e[j + 1]))
-        step_ms.append(e[0].elapsed_time(e[len(names)]))
-    max_ms = max_over_ranks(float(sum(step_ms)), dev, dist)
-
-    # e2e through the public API: pinned host tokens in, layer output back to host, each step
-    e2e = None
-    if not args.no_e2e:
-        x_host = torch.from_numpy(x_bits.view(np.int16)).pin_memory()
-        y_host = torch.empty(T, d, dtype=torch.int16).pin_memory()
-        x_dev = torch.empty_like(x)
-        for _ in range(2):
-            x_dev.copy_(x_host, non_blocking=True)
-            Q.tqp_moe_layer_fwd(x_dev, L, y, ws_l, st)
-            y_host.copy_(y, non_blocking=True)
-        torch.cuda.synchronize(dev)
-        if dist:
-            torch.distributed.barrier()
-        e0 = torch.cuda.Event(enable_timing=True)
-        e1 = torch.cuda.Event(enable_timing=True)
-        e0.record(stream)
-        for _ in range(args.steps):
-            x_dev.copy_(x_host, non_blocking=True)
-            Q.tqp_moe_layer_fwd(x_dev, L, y, ws_l, st)
-            y_host.copy_(y, non_blocking=True)
-        e1.record(stream)
-        torch.cuda.synchronize(dev)
-        e2e_ms = max_over_ranks(e0.elapsed_time(e1), dev, dist) / args.steps
-        e2e = {"value": weak_scaling_value(world, T, e2e_ms), "unit": UNIT, "h2d_bytes_per_step": int(T * d * 2),
-               "d2h_bytes_per_step": int(T * d * 2), "ms_per_step": e2e_ms}
-    if st.read() != 0:
-        raise RuntimeError(f"device status {st.read()} after the timed steps")
+    max_ms = max_over_ranks(float(sum(timing["step_ms"])), dev, dist)
+    e2e = None if args.no_e2e else time_e2e(lb, args.steps, dev, dist, world)
+    if lb.st.read() != 0:
+        raise RuntimeError(f"device status {lb.st.read()} after the e2e steps")
     if rank != 0:
         return None
 
+    T, A = cfg.T, cfg.T * cfg.k
     ms = max_ms / args.steps
     fl = layer_flops(cfg)
     pk = peaks()
-    per_call_ms = {n: statistics.mean(v) for n, v in per_call.items()}
-    ffn_ms = sum(per_call_ms[n] for n in names if n.startswith("ffn_"))
+    per_call_ms = timing["per_call_ms"]
+    ffn_ms = sum(per_call_ms[n] for n in CALLS if n.startswith("ffn_"))
     ffn_tflops = fl["ffn"] / (ffn_ms * 1e-3) / 1e12
     gu_ms = per_call_ms["ffn_gate_up"]
     gu_tflops = fl["gate_up"] / (gu_ms * 1e-3) / 1e12
@@ -397,25 +501,37 @@ def run_tqp(args, rank: int, world: int, local_rank: int) -> dict | None:
         "assignments_per_s": world * A / (ms * 1e-3),
         "per_call_ms": dict(per_call_ms, grouped_ffn=ffn_ms),
         "roofline": {"bound": "tensor",
-                     "kernel": "expert_ffn_kernel<GATEUP> (int4 -> fp16 weights in TMEM, tcgen05 gate/up + SwiGLU)",
+                     "kernel": "gateup_kernel (int4 -> fp16 weights in TMEM, tcgen05 gate/up + SwiGLU)",
                      "achieved": gu_tflops, "peak": pk["bf16_tflops"], "unit": "TFLOP/s",
                      "frac": gu_tflops / pk["bf16_tflops"],
-                     "traffic": measured_traffic("expert_ffn_kernel<GATEUP>") if args.config == "full" else None,
+                     "traffic": measured_traffic("gateup_kernel") if args.config == "full" else None,
                      "traffic_source": "profiles/expert_ffn_traffic_full.md (ncu dram__bytes_read+write, one launch)",
                      "peak_source": f"{pk['source']} bf16 dense burst (fp16 has the same nominal rate)",
                      "flop_per_launch": fl["gate_up"], "ms_per_launch": gu_ms},
+        "layer_roofline": layer_roofline(cfg, lb.touched_experts(), ms),
         "ffn_call": {"achieved_tflops": ffn_tflops, "frac": ffn_tflops / pk["bf16_tflops"], "ms": ffn_ms,
                      "flop": fl["ffn"]},
-        "layer_roofline_frac_nominal": (fl["total"] / 2.25e15) / (ms * 1e-3),
-        "gpu_launches": args.steps * sum(launches_per_step.values()),
+        "gpu_launches": args.steps * sum(lb.launches.values()),
         "clocks": clk,
         "e2e": e2e,
     }
+    if world == 1 and args.config == "full" and not args.no_extra_configs:
+        extra = {}
+        n = min(args.steps, 10)
+        mid = LayerBench(synth.MID, dev, synth.MID.seed)
+        extra["mid"] = mid.summary(mid.run(n, args.warmup, flush))
+        del mid
+        sk_host = dict(lb.host, cfg=synth.SKEWED, bias=synth.zipf_bias(synth.SKEWED.E, synth.SKEWED.zipf_s))
+        sk = LayerBench(synth.SKEWED, dev, synth.SKEWED.seed, host=sk_host)
+        extra["skewed"] = sk.summary(sk.run(n, args.warmup, flush))
+        del sk
+        torch.cuda.empty_cache()
+        result["configs"] = extra
     if world == 1 and args.config == "full" and not args.no_rev:
-        result["rev_block"] = time_rev_block(L, dev, min(args.steps, 5), 2, flush)
+        result["rev_block"] = time_rev_block(lb.L, dev, min(args.steps, 5), 2, flush)
     if world == 1 and not args.no_cpu_baseline:
         sample = min(T, args.cpu_sample)
-        result["cpu_baseline"] = time_oracle(cfg, host, x_bits, sample)
+        result["cpu_baseline"] = time_oracle(cfg, lb.host, lb.x_bits, sample)
     return result
 
 
@@ -454,6 +570,7 @@ def main():
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-rev", action="store_true", help="skip timing the reversible block (forward, inverse, "
                                                              "adapter backward)")
+    ap.add_argument("--no-extra-configs", action="store_true", help="skip the mid and skewed configurations")
     args = ap.parse_args()
     rank = int(os.environ.get("RANK", 0))
     world = int(os.environ.get("WORLD_SIZE", 1))

@@ -26,17 +26,32 @@
  *     are detected on the host before anything is enqueued.
  *   - Data-dependent errors are OR-ed asynchronously into `dev_status`, a
  *     caller-owned int32 in device memory that the caller zeroes and reads
- *     after synchronising: TQP_STATUS_NONFINITE (a NaN/Inf router logit),
- *     TQP_STATUS_BAD_ID (an expert id outside [0, E)), TQP_STATUS_TIMEOUT (a
- *     device-side wait hit its limit; outputs are then undefined). Nothing
- *     traps, prints or exits.
+ *     after synchronising (nullable: then they are not reported):
+ *       TQP_STATUS_NONFINITE  a NaN/Inf router logit or input; an x value
+ *                             outside the fp16 range; an fp16 intermediate of
+ *                             the expert path (H, the kept G|U, O, s X A,
+ *                             s H A, and in the backward dO, dG|dU, dX and the
+ *                             rank-space products) that overflowed; a LoRA
+ *                             factor outside the fp16 range. Outputs are then
+ *                             unreliable.
+ *       TQP_STATUS_BAD_ID     an expert id outside [0, E), or one token listing
+ *                             the same expert twice.
+ *       TQP_STATUS_TIMEOUT    a device-side wait hit its limit; outputs are then
+ *                             undefined.
+ *       TQP_STATUS_RANGE      a nonzero group scale outside [2^-17, 8192): the
+ *                             products q * scale are then not all exact in fp16
+ *                             (the expert contractions run on exact fp16 weights
+ *                             otherwise).
+ *     Nothing traps, prints or exits.
  *   - Every pointer argument is caller-owned DEVICE memory (unless stated),
  *     16-byte aligned, dense row-major. The library never allocates device
  *     memory: scratch comes from `ws` of at least the size returned by the
  *     matching *_workspace_size query (which needs no GPU).
  *   - Work is enqueued on `stream` (a cudaStream_t; NULL = legacy default
  *     stream) and the call returns at once. Calls hold no global state and may
- *     run concurrently on different streams with disjoint workspaces.
+ *     run concurrently on different streams with disjoint workspaces (the two
+ *     exceptions are named where they are declared: moe_permute_noalloc's fixed
+ *     scratch and the tqp_debug_set_wait_limit_ns test hook).
  *   - bf16 tensors are uint16_t bit patterns.
  *   - Outputs are overwritten (never accumulated into).
  *
@@ -78,6 +93,7 @@ extern "C" {
 #define TQP_STATUS_NONFINITE 1
 #define TQP_STATUS_BAD_ID 2
 #define TQP_STATUS_TIMEOUT 4
+#define TQP_STATUS_RANGE 8
 
 #define TQP_DTYPE_BF16 0
 #define TQP_DTYPE_F32 1
@@ -110,8 +126,8 @@ int tqp_version(void);
 const char* tqp_error_string(int code);
 
 /* ---------------------------------------------------------------------------
- * moe_router_gemm: full-precision router logits.
- * "Router: Full precision (critical for routing quality)" (TQP Quantization).
+ * moe_router_gemm: router logits at full precision (the TQP Quantization list
+ * keeps the router unquantised because routing quality depends on it).
  *   logits[t][e] = sum_i x[t][i] * router_w[e][i] (+ router_bias[e]), accurate to
  *   fp32 (the fp32 weights are split exactly into three bf16 parts and the
  *   products accumulated in fp32 on the tensor cores).
@@ -139,8 +155,9 @@ int moe_route(const float* logits, int T, int E, int k, int32_t* ids, float* gat
  *   offsets[e] = #assignments to experts < e, offsets[E] = T*k;
  *   rows of one expert are in increasing token order;
  *   perm_token[row] = token of that row; inv[t*k + j] = row of assignment (t, j).
- *   ids outside [0, E) raise TQP_STATUS_BAD_ID (those assignments are dropped
- *   and the outputs are then incomplete).
+ *   Precondition: each token's k ids are distinct (moe_route guarantees it).
+ *   ids outside [0, E), and a token that lists one expert twice, raise
+ *   TQP_STATUS_BAD_ID; the outputs are then not a valid permutation.
  *   ws: moe_permute_workspace_size.
  * ------------------------------------------------------------------------- */
 size_t moe_permute_workspace_size(int T, int E, int k);
@@ -160,9 +177,11 @@ int moe_permute(const int32_t* ids, int T, int E, int k, int32_t* offsets, int32
  *   Limits: T <= 16384 and E <= 512, else TQP_ERR_UNSUPPORTED (nothing is
  *   enqueued). Allocates nothing: no cudaMalloc, no cudaFree, no allocating
  *   library call.
- *   The first call on a device looks up the array's device address with that
- *   device current (cudaGetSymbolAddress); make that first call before any
- *   stream capture.
+ *   The first call under each CUDA context looks up the array's device address
+ *   in that context with the device current (cudaGetSymbolAddress) and caches
+ *   it under the context's unique id, so a context created after a device
+ *   reset, or a second context on the device, gets its own lookup; make the
+ *   first call in a context before any stream capture.
  *   All calls share the one array, and every call overwrites it before reading
  *   it; calls that overlap on the GPU (concurrent streams) race on it and must
  *   be serialised by the caller.
@@ -172,8 +191,8 @@ int moe_permute_noalloc(const int32_t* ids, int T, int E, int k, int32_t* offset
                         int32_t* inv, int32_t* dev_status, void* stream);
 
 /* ---------------------------------------------------------------------------
- * tqp_grouped_ffn: the routed experts ("Train low-rank adapters per expert"
- * over "Quantize base expert weights", Pattern 3). For each expert e and each
+ * tqp_grouped_ffn: the routed experts (Pattern 3: low-rank adapters trained per
+ * expert over frozen quantised base expert weights). For each expert e and each
  * of its rows (row r holds token perm_token[r]):
  *   G = X Wg^T + s (X Ag) Bg ;  U = X Wu^T + s (X Au) Bu ;  H = fp16(silu(G) * U)
  *   O = fp16(H Wd^T + s (H Ad) Bd)
@@ -183,8 +202,9 @@ int moe_permute_noalloc(const int32_t* ids, int T, int E, int k, int32_t* offset
  *   x [T][d] bf16 (tokens, gathered through perm_token); offsets [E+1];
  *   h [T*k][ffn] fp16 output (permuted row order; kept for the backward);
  *   out_perm [T*k][d] fp16 output (permuted row order).
- *   ws: tqp_grouped_ffn_workspace_size. Errors: as the conventions above;
- *   x values outside the fp16 range raise TQP_STATUS_NONFINITE.
+ *   ws: tqp_grouped_ffn_workspace_size. Errors: as the conventions above (x
+ *   values and fp16 intermediates outside the fp16 range raise
+ *   TQP_STATUS_NONFINITE, group scales outside the exact range TQP_STATUS_RANGE).
  *
  * tqp_grouped_ffn_part: the same computation issued one part at a time, for a
  * caller that times or overlaps the parts. Parts must be issued in order
@@ -250,9 +270,10 @@ int rev_couple_inv(const float* y1, const float* y2, int T, const tqp_moe_weight
                    uint16_t* x1, uint16_t* x2, void* ws, size_t ws_bytes, int32_t* dev_status, void* stream);
 
 /* ---------------------------------------------------------------------------
- * tqp_moe_layer_bwd: gradients of <dy, layer(x)> (base weights and router
- * frozen: "Base expert weights: Quantized (fixed)"; optimizer state on the
- * adapters only).
+ * tqp_moe_layer_bwd: gradients of <dy, layer(x)>. The base weights stay fixed
+ * in their quantised form and the router is frozen, so only the adapters get
+ * gradients (TQP Quantization; Principle 3 keeps optimizer state on the
+ * adapters alone).
  *   x [T][d] bf16; dy [T][d] fp32 -> dx [T][d] fp32 (through the experts and,
  *   via the softmax over the chosen logits, through the frozen router), and the
  *   adapter gradients `grads`. Top-k selection is treated as constant.
@@ -260,6 +281,11 @@ int rev_couple_inv(const float* y1, const float* y2, int T, const tqp_moe_weight
  *   memory, overwritten (not accumulated). With rank > 0 each must be non-null
  *   and 16-byte aligned, else TQP_ERR_INVALID_ARG before any launch; ffn must be
  *   a multiple of 128, else TQP_ERR_UNSUPPORTED.
+ *   The fp16 intermediates are computed for dy * 2^P, with the power of two P
+ *   chosen from max|dy| on the device so that dO = gate * dy * 2^P peaks near
+ *   2^8; the gradients are scaled back by 2^-P in fp32. The result therefore
+ *   does not depend on the magnitude of dy (no fp16 underflow or overflow for
+ *   small or large cotangents).
  *   ws: tqp_moe_layer_bwd_workspace_size (the layer's forward workspace plus
  *   G|U, dG|dU, dO, dha, dxa and the rank-space B operand in fp16).
  * ------------------------------------------------------------------------- */
@@ -270,8 +296,8 @@ int tqp_moe_layer_bwd(const uint16_t* x, const float* dy, int T, const tqp_moe_w
 
 /* ---------------------------------------------------------------------------
  * tqp_adapter_bwd: reversible block backward from the block outputs only
- * ("Backward: reconstruct from final state ... compute gradients locally",
- * Principle 1).
+ * (Principle 1: the backward pass rebuilds each block's inputs from its
+ * outputs and takes that block's gradients locally).
  *   G-step: z = bf16(y1); x2 = y2 - G(z); G's adapter grads for cotangent dy2;
  *           dz1 = dy1 + J_G(z)^T dy2.
  *   F-step: x1 = y1 - F(x2); F's adapter grads for cotangent dz1;
@@ -288,6 +314,82 @@ int tqp_adapter_bwd(const float* y1, const float* y2, const float* dy1, const fl
                     const tqp_moe_weights* F, const tqp_moe_weights* G, uint16_t* x1, uint16_t* x2, float* dx1,
                     float* dx2, const tqp_adapter_grads* gF, const tqp_adapter_grads* gG, void* ws,
                     size_t ws_bytes, int32_t* dev_status, void* stream);
+
+/* ---------------------------------------------------------------------------
+ * Reversible stack of L coupling blocks (Principle 1: Reversible Recurrence
+ * Stack; Key Innovation: activation memory stays flat as the model deepens).
+ * Block l maps streams (a1, a2) to
+ *   b1 = a1 + F_l(bf16(a2)),   b2 = a2 + G_l(bf16(b1)).
+ * Block 0's inputs are x1, x2 (bf16); the streams between blocks are carried
+ * in fp32 (each layer reads the bf16 rounding of its stream); the outputs of
+ * block L-1 are y1, y2 (fp32). With L = 1 this is rev_couple_fwd exactly.
+ *   F, G: arrays of L weight sets (all with the same d).
+ *   rev_stack_fwd: x1, x2 [T][d] bf16 -> y1, y2 [T][d] fp32.
+ *   rev_stack_inv: y1, y2 -> x1, x2 (bf16), walking the blocks from L-1 down
+ *     with a2 = b2 - G_l(bf16(b1)), a1 = b1 - F_l(bf16(a2)); routing is
+ *     recomputed (stateless).
+ *   rev_stack_bwd: the backward of the whole stack from its outputs alone: for
+ *     l = L-1 .. 0 it reconstructs block l's inputs from its outputs and takes
+ *     that block's gradients (each layer's backward reuses the routing and
+ *     intermediates of the inverse step that just ran its forward), so no
+ *     block's activations are stored. In: y1, y2, dy1, dy2 [T][d] fp32. Out:
+ *     x1, x2 (bf16, reconstructed inputs of block 0), dx1, dx2 [T][d] fp32, and
+ *     the adapter gradients of every layer: gF[l], gG[l] (arrays of L structs,
+ *     each checked as for tqp_moe_layer_bwd; overwritten). Every ffn must be a
+ *     multiple of 128 (else TQP_ERR_UNSUPPORTED).
+ *   ws: rev_stack_workspace_size (the same size serves all three calls). It
+ *   holds two sets of four fp32 stream buffers, two bf16 layer inputs, one
+ *   fp32 input gradient and one layer's forward + backward workspace: it does
+ *   not grow with L. 1 <= L <= 4096.
+ * ------------------------------------------------------------------------- */
+size_t rev_stack_workspace_size(int T, int L, const tqp_moe_weights* const* F, const tqp_moe_weights* const* G);
+int rev_stack_fwd(const uint16_t* x1, const uint16_t* x2, int T, int L, const tqp_moe_weights* const* F,
+                  const tqp_moe_weights* const* G, float* y1, float* y2, void* ws, size_t ws_bytes,
+                  int32_t* dev_status, void* stream);
+int rev_stack_inv(const float* y1, const float* y2, int T, int L, const tqp_moe_weights* const* F,
+                  const tqp_moe_weights* const* G, uint16_t* x1, uint16_t* x2, void* ws, size_t ws_bytes,
+                  int32_t* dev_status, void* stream);
+int rev_stack_bwd(const float* y1, const float* y2, const float* dy1, const float* dy2, int T, int L,
+                  const tqp_moe_weights* const* F, const tqp_moe_weights* const* G, uint16_t* x1, uint16_t* x2,
+                  float* dx1, float* dx2, const tqp_adapter_grads* const* gF, const tqp_adapter_grads* const* gG,
+                  void* ws, size_t ws_bytes, int32_t* dev_status, void* stream);
+
+/* ---------------------------------------------------------------------------
+ * tqp_adamw_step: one optimizer step over adapter parameters (Principle 3 and
+ * Pattern 3: optimizer state lives on the adapters only; the pages do not name
+ * the optimizer, this is AdamW with decoupled weight decay). Elementwise over
+ * n parameters, in one pass over memory:
+ *   g = grad * grad_scale
+ *   exp_avg    = beta1 exp_avg    + (1 - beta1) g
+ *   exp_avg_sq = beta2 exp_avg_sq + (1 - beta2) g^2
+ *   param     -= lr * ( exp_avg / (1 - beta1^step)
+ *                       / (sqrt(exp_avg_sq / (1 - beta2^step)) + eps)
+ *                       + weight_decay * param )
+ *   param_bf16 = bf16(param) (round to nearest even), when non-null.
+ * param, exp_avg, exp_avg_sq: fp32 [n], updated in place (caller-owned device
+ * memory, 16-byte aligned); grad fp32 [n] (16-byte aligned); param_bf16 [n]
+ * bf16 (8-byte aligned) or NULL. The layout is the caller's: the flat buffer of
+ * a layer's six adapter tensors in the order dA[0..2], dB[0..2] lets one call
+ * update a whole layer. step >= 1; 0 <= beta1, beta2 < 1; eps > 0; lr,
+ * weight_decay >= 0 (else TQP_ERR_INVALID_ARG). A non-finite gradient raises
+ * TQP_STATUS_NONFINITE.
+ * ------------------------------------------------------------------------- */
+int tqp_adamw_step(float* param, float* exp_avg, float* exp_avg_sq, const float* grad, uint16_t* param_bf16, size_t n,
+                   float lr, float beta1, float beta2, float eps, float weight_decay, int step, float grad_scale,
+                   int32_t* dev_status, void* stream);
+
+/* ---------------------------------------------------------------------------
+ * tqp_debug_set_wait_limit_ns: test hook for the failure path, not for normal
+ * use. Every device-side barrier wait in the library's kernels is bounded; this
+ * sets that bound for the launches that follow in this process (0 restores the
+ * default of 2 s). A wait that runs out sets TQP_STATUS_TIMEOUT, every role of
+ * the CTA leaves its loop, copies and MMAs in flight are drained, and the call
+ * returns with undefined outputs; the CUDA context stays usable. A limit far
+ * below the kernels' normal waits (say 1 ns) makes the next launch time out on
+ * purpose. Process-wide; not synchronised with launches on other threads.
+ * Returns TQP_OK.
+ * ------------------------------------------------------------------------- */
+int tqp_debug_set_wait_limit_ns(unsigned long long ns);
 
 #ifdef __cplusplus
 }

@@ -438,6 +438,134 @@ def block_backward_stored(x1, x2, dy1, dy2, F: Layer, G: Layer):
 
 
 # ----------------------------------------------------------------------------
+# reversible stack of coupling blocks
+# ----------------------------------------------------------------------------
+
+
+def stack_forward(x1, x2, blocks, round_inputs: bool = True):
+    """L coupling blocks applied in order ("Principle 1: Reversible Recurrence
+    Stack": the forward pass runs the blocks one after the other, keeping only
+    the final state).
+
+    blocks: list of (F, G) Layers. Block l maps the streams (a1, a2) to
+    b1 = a1 + F(bf16(a2)), b2 = a2 + G(bf16(b1)): the streams are carried
+    exactly (fp64 here) and each layer reads its stream rounded to bf16, its
+    input format. Block 0 reads the bf16 inputs x1, x2, so one block is
+    coupling_forward. round_inputs=False drops the roundings (smooth in every
+    input, for finite differences).
+    """
+    rb = round_bf16 if round_inputs else (lambda v: v)
+    a1 = np.asarray(x1, dtype=np.float64)
+    a2 = np.asarray(x2, dtype=np.float64)
+    for F, G in blocks:
+        b1 = a1 + layer_forward(rb(a2), F)
+        b2 = a2 + layer_forward(rb(b1), G)
+        a1, a2 = b1, b2
+    return a1, a2
+
+
+def stack_inverse(y1, y2, blocks, round_inputs: bool = True):
+    """Reconstruct the stack's inputs from its outputs, last block first:
+    a2 = b2 - G(bf16(b1)), a1 = b1 - F(bf16(a2)) ("Principle 1": the backward
+    pass walks the stack in reverse through each layer's inverse)."""
+    rb = round_bf16 if round_inputs else (lambda v: v)
+    b1 = np.asarray(y1, dtype=np.float64)
+    b2 = np.asarray(y2, dtype=np.float64)
+    for F, G in reversed(blocks):
+        a2 = b2 - layer_forward(rb(b1), G)
+        a1 = b1 - layer_forward(rb(a2), F)
+        b1, b2 = a1, a2
+    return b1, b2
+
+
+def stack_backward(y1, y2, dy1, dy2, blocks, round_inputs: bool = True):
+    """Gradients of <dy1, y1> + <dy2, y2> for the whole stack from its outputs
+    alone ("Principle 1": reconstruct each layer's input from its output, then
+    take that layer's gradients locally, last block first).
+
+    Per block, with outputs (b1, b2) and their cotangents (g1, g2):
+    z = bf16(b1); a2 = b2 - G(z); G's adapter gradients for cotangent g2 and
+    dz1 = g1 + J_G(z)^T g2; a1 = b1 - F(bf16(a2)); F's adapter gradients for
+    cotangent dz1; the block's input cotangents are (dz1, g2 + J_F^T dz1). The
+    bf16 roundings pass gradients unchanged. Returns x1, x2 (reconstructed),
+    dx1, dx2 and grads[l] = (dA_F, dB_F, dA_G, dB_G) for every block l.
+    """
+    rb = round_bf16 if round_inputs else (lambda v: v)
+    b1 = np.asarray(y1, dtype=np.float64)
+    b2 = np.asarray(y2, dtype=np.float64)
+    g1 = np.asarray(dy1, dtype=np.float64)
+    g2 = np.asarray(dy2, dtype=np.float64)
+    grads = []
+    for F, G in reversed(blocks):
+        z = rb(b1)
+        a2 = b2 - layer_forward(z, G)
+        dxG, dAG, dBG = layer_backward(z, g2, G)
+        dz1 = g1 + dxG
+        ab = rb(a2)
+        a1 = b1 - layer_forward(ab, F)
+        dxF, dAF, dBF = layer_backward(ab, dz1, F)
+        g1, g2 = dz1, g2 + dxF
+        b1, b2 = a1, a2
+        grads.append((dAF, dBF, dAG, dBG))
+    grads.reverse()
+    return {"x1": b1, "x2": b2, "dx1": g1, "dx2": g2, "grads": grads}
+
+
+def stack_backward_stored(x1, x2, dy1, dy2, blocks, round_inputs: bool = True):
+    """The same gradients with every block's inputs stored during the forward
+    (the non-reversible baseline that reversibility replaces)."""
+    rb = round_bf16 if round_inputs else (lambda v: v)
+    a1 = np.asarray(x1, dtype=np.float64)
+    a2 = np.asarray(x2, dtype=np.float64)
+    saved = []
+    for F, G in blocks:
+        saved.append((a1, a2))
+        b1 = a1 + layer_forward(rb(a2), F)
+        b2 = a2 + layer_forward(rb(b1), G)
+        a1, a2 = b1, b2
+    g1 = np.asarray(dy1, dtype=np.float64)
+    g2 = np.asarray(dy2, dtype=np.float64)
+    grads = []
+    for (a1, a2), (F, G) in zip(reversed(saved), reversed(blocks)):
+        b1 = a1 + layer_forward(rb(a2), F)
+        dxG, dAG, dBG = layer_backward(rb(b1), g2, G)
+        dz1 = g1 + dxG
+        dxF, dAF, dBF = layer_backward(rb(a2), dz1, F)
+        g1, g2 = dz1, g2 + dxF
+        grads.append((dAF, dBF, dAG, dBG))
+    grads.reverse()
+    return {"dx1": g1, "dx2": g2, "grads": grads}
+
+
+# ----------------------------------------------------------------------------
+# adapter optimizer step
+# ----------------------------------------------------------------------------
+
+
+def adamw_step(p, m, v, g, lr, beta1, beta2, eps, weight_decay, t, grad_scale=1.0):
+    """One AdamW step (Adam with decoupled weight decay, Loshchilov & Hutter)
+    over adapter parameters: the only trained, optimizer-carrying parameters
+    ("Principle 3: TQP Optimizer Strategy"; "Pattern 3"). The pages do not name
+    the optimizer; this is the reading used.
+
+    g' = grad_scale g; m <- beta1 m + (1 - beta1) g'; v <- beta2 v + (1 - beta2) g'^2;
+    m_hat = m / (1 - beta1^t); v_hat = v / (1 - beta2^t);
+    p <- p - lr (m_hat / (sqrt(v_hat) + eps) + weight_decay p).
+    Returns the new (p, m, v) as float64 arrays.
+    """
+    p = np.asarray(p, dtype=np.float64)
+    m = np.asarray(m, dtype=np.float64)
+    v = np.asarray(v, dtype=np.float64)
+    g = np.asarray(g, dtype=np.float64) * grad_scale
+    m = beta1 * m + (1.0 - beta1) * g
+    v = beta2 * v + (1.0 - beta2) * g * g
+    m_hat = m / (1.0 - beta1 ** t)
+    v_hat = v / (1.0 - beta2 ** t)
+    p = p - lr * (m_hat / (np.sqrt(v_hat) + eps) + weight_decay * p)
+    return p, m, v
+
+
+# ----------------------------------------------------------------------------
 # per-token evaluation (for sampled checks at full size)
 # ----------------------------------------------------------------------------
 

@@ -18,7 +18,9 @@ __all__ = [
     "moe_router_gemm", "moe_route", "moe_permute", "moe_permute_noalloc", "tqp_grouped_ffn", "tqp_grouped_ffn_part",
     "moe_combine", "tqp_moe_layer_fwd",
     "rev_couple_fwd", "rev_couple_inv", "tqp_moe_layer_bwd", "tqp_adapter_bwd",
-    "header_functions",
+    "header_functions", "tqp_debug_set_wait_limit_ns",
+    "ReversibleStack", "rev_stack_fwd", "rev_stack_inv", "rev_stack_bwd",
+    "tqp_adamw_step", "AdapterAdamW",
 ]
 
 HERE = os.path.dirname(os.path.abspath(__file__))
@@ -29,7 +31,7 @@ HEADER = os.path.join(ROOT, "include", "tqp_moe.h")
 TQP_OK = 0
 ERRORS = {-1: "invalid argument", -2: "unsupported configuration", -3: "workspace too small",
           -4: "CUDA launch or runtime error"}
-STATUS_NONFINITE, STATUS_BAD_ID, STATUS_TIMEOUT = 1, 2, 4
+STATUS_NONFINITE, STATUS_BAD_ID, STATUS_TIMEOUT, STATUS_RANGE = 1, 2, 4, 8
 FFN_PREPARE, FFN_GATE_UP, FFN_RANK, FFN_DOWN = 0, 1, 2, 3
 DTYPE_BF16, DTYPE_F32 = 0, 1
 
@@ -81,6 +83,13 @@ _SIGS = {
     "tqp_adapter_bwd_workspace_size": (_SZ, [_I, _WP, _WP]),
     "tqp_adapter_bwd": (_I, [_VP, _VP, _VP, _VP, _I, _WP, _WP, _VP, _VP, _VP, _VP, _GP, _GP, _VP, _SZ, _VP,
                              _VP]),
+    "tqp_debug_set_wait_limit_ns": (_I, [ctypes.c_ulonglong]),
+    "tqp_adamw_step": (_I, [_VP, _VP, _VP, _VP, _VP, _SZ, _F, _F, _F, _F, _F, _I, _F, _VP, _VP]),
+    "rev_stack_workspace_size": (_SZ, [_I, _I, _VP, _VP]),
+    "rev_stack_fwd": (_I, [_VP, _VP, _I, _I, _VP, _VP, _VP, _VP, _VP, _SZ, _VP, _VP]),
+    "rev_stack_inv": (_I, [_VP, _VP, _I, _I, _VP, _VP, _VP, _VP, _VP, _SZ, _VP, _VP]),
+    "rev_stack_bwd": (_I, [_VP, _VP, _VP, _VP, _I, _I, _VP, _VP, _VP, _VP, _VP, _VP, _VP, _VP, _VP, _SZ, _VP,
+                           _VP]),
 }
 
 _lib = None
@@ -126,6 +135,29 @@ def _require_cuda(*tensors) -> None:
     for t in tensors:
         if t is not None and not t.is_cuda:
             raise ValueError("tensors passed to the TQP library must live on a CUDA device")
+
+
+def _require_int32(name: str, t, min_numel: int, ndim: int | None = None) -> None:
+    """The C ABI reads int32 arrays through raw pointers: refuse anything else
+    (an int64 tensor would be read as pairs of int32, an undersized output
+    would be written past its end)."""
+    import torch
+    if t.dtype != torch.int32 or not t.is_contiguous():
+        raise ValueError(f"{name} must be a contiguous int32 tensor (got {t.dtype}, contiguous={t.is_contiguous()})")
+    if ndim is not None and t.dim() != ndim:
+        raise ValueError(f"{name} must have {ndim} dimensions (got {t.dim()})")
+    if t.numel() < min_numel:
+        raise ValueError(f"{name} needs at least {min_numel} elements (got {t.numel()})")
+
+
+def _permute_args(ids, E: int, offsets, perm_token, inv) -> tuple[int, int]:
+    _require_int32("ids", ids, 0, ndim=2)
+    T, k = ids.shape
+    _require_int32("offsets", offsets, E + 1)
+    _require_int32("perm_token", perm_token, T * k)
+    _require_int32("inv", inv, T * k)
+    _require_cuda(ids, offsets, perm_token, inv)
+    return T, k
 
 
 class Status:
@@ -174,8 +206,17 @@ class DeviceLayer:
             np.ascontiguousarray(host["bias"], np.float32)).to(device)
         self.wq = [torch.from_numpy(np.ascontiguousarray(host[f"wq{p}"])).to(device) for p in range(3)]
         self.ws = [_bf16_tensor(host[f"ws{p}"], device) for p in range(3)]
-        self.la = [_bf16_tensor(host[f"la{p}"], device) for p in range(3)]
-        self.lb = [_bf16_tensor(host[f"lb{p}"], device) for p in range(3)]
+        # the six adapter factors as views of one flat bf16 buffer, in the order of
+        # the flat gradient buffer (A_gate, A_up, A_down, B_gate, B_up, B_down), so
+        # that one optimizer call updates the whole layer
+        parts = [np.ascontiguousarray(host[f"la{p}"]) for p in range(3)] + \
+                [np.ascontiguousarray(host[f"lb{p}"]) for p in range(3)]
+        self.lora_flat = torch.from_numpy(np.concatenate([a.reshape(-1) for a in parts]).view(np.int16)).to(device)
+        views, off = [], 0
+        for a in parts:
+            views.append(self.lora_flat[off:off + a.size].view(a.shape))
+            off += a.size
+        self.la, self.lb = views[:3], views[3:]
         self._struct = None
 
     @property
@@ -243,8 +284,7 @@ def moe_route(logits, k: int, ids, gates, status: Status | None = None, stream=N
 
 
 def moe_permute(ids, E: int, offsets, perm_token, inv, ws=None, status: Status | None = None, stream=None):
-    _require_cuda(ids, offsets, perm_token, inv)
-    T, k = ids.shape
+    T, k = _permute_args(ids, E, offsets, perm_token, inv)
     n = lib().moe_permute_workspace_size(T, E, k)
     ws = ws if ws is not None else workspace(n, ids.device)
     _check("moe_permute", lib().moe_permute(ids.data_ptr(), T, E, k, offsets.data_ptr(), perm_token.data_ptr(),
@@ -255,8 +295,7 @@ def moe_permute(ids, E: int, offsets, perm_token, inv, ws=None, status: Status |
 
 def moe_permute_noalloc(ids, E: int, offsets, perm_token, inv, status: Status | None = None, stream=None):
     """moe_permute with its scratch in the library's fixed device array (no workspace)."""
-    _require_cuda(ids, offsets, perm_token, inv)
-    T, k = ids.shape
+    T, k = _permute_args(ids, E, offsets, perm_token, inv)
     _check("moe_permute_noalloc", lib().moe_permute_noalloc(ids.data_ptr(), T, E, k, offsets.data_ptr(),
                                                             perm_token.data_ptr(), inv.data_ptr(),
                                                             status.ptr() if status else None, _stream(stream)))
@@ -356,3 +395,123 @@ def tqp_adapter_bwd(y1, y2, dy1, dy2, F: DeviceLayer, G: DeviceLayer, x1, x2, dx
                                                     ws.data_ptr(), ws.numel(), status.ptr() if status else None,
                                                     _stream(stream)))
     return x1, x2, dx1, dx2
+
+
+def tqp_debug_set_wait_limit_ns(ns: int) -> None:
+    """Test hook: bound of every device-side barrier wait of the launches that
+    follow (0 restores the 2 s default). See include/tqp_moe.h."""
+    _check("tqp_debug_set_wait_limit_ns", lib().tqp_debug_set_wait_limit_ns(int(ns)))
+
+
+# ---------------------------------------------------------------- reversible stack
+
+
+class ReversibleStack:
+    """L coupling blocks (F[l], G[l]) as the C ABI takes them: arrays of
+    tqp_moe_weights pointers, kept alive with the layers."""
+
+    def __init__(self, F: list, G: list):
+        if len(F) != len(G) or not F:
+            raise ValueError("a stack needs L >= 1 pairs of layers")
+        self.F, self.G, self.L = list(F), list(G), len(F)
+        self._fw = (ctypes.POINTER(Weights) * self.L)(*[ctypes.pointer(l.struct) for l in self.F])
+        self._gw = (ctypes.POINTER(Weights) * self.L)(*[ctypes.pointer(l.struct) for l in self.G])
+
+    def ptrs(self):
+        return ctypes.cast(self._fw, ctypes.c_void_p), ctypes.cast(self._gw, ctypes.c_void_p)
+
+    def workspace_size(self, T: int) -> int:
+        f, g = self.ptrs()
+        return int(lib().rev_stack_workspace_size(T, self.L, f, g))
+
+    def grads(self, device="cuda"):
+        """Per-layer FlatGrads for F and G, and the two pointer arrays the C ABI takes."""
+        gF = [l.flat_grads(device) for l in self.F]
+        gG = [l.flat_grads(device) for l in self.G]
+        aF = (ctypes.POINTER(Grads) * self.L)(*[ctypes.pointer(g.struct) for g in gF])
+        aG = (ctypes.POINTER(Grads) * self.L)(*[ctypes.pointer(g.struct) for g in gG])
+        return gF, gG, (aF, aG)
+
+
+def rev_stack_fwd(x1, x2, stack: ReversibleStack, y1, y2, ws=None, status: Status | None = None, stream=None):
+    _require_cuda(x1, x2, y1, y2)
+    T = x1.shape[0]
+    ws = ws if ws is not None else workspace(stack.workspace_size(T), x1.device)
+    f, g = stack.ptrs()
+    _check("rev_stack_fwd", lib().rev_stack_fwd(x1.data_ptr(), x2.data_ptr(), T, stack.L, f, g, y1.data_ptr(),
+                                                y2.data_ptr(), ws.data_ptr(), ws.numel(),
+                                                status.ptr() if status else None, _stream(stream)))
+    return y1, y2
+
+
+def rev_stack_inv(y1, y2, stack: ReversibleStack, x1, x2, ws=None, status: Status | None = None, stream=None):
+    _require_cuda(x1, x2, y1, y2)
+    T = y1.shape[0]
+    ws = ws if ws is not None else workspace(stack.workspace_size(T), y1.device)
+    f, g = stack.ptrs()
+    _check("rev_stack_inv", lib().rev_stack_inv(y1.data_ptr(), y2.data_ptr(), T, stack.L, f, g, x1.data_ptr(),
+                                                x2.data_ptr(), ws.data_ptr(), ws.numel(),
+                                                status.ptr() if status else None, _stream(stream)))
+    return x1, x2
+
+
+def rev_stack_bwd(y1, y2, dy1, dy2, stack: ReversibleStack, x1, x2, dx1, dx2, grad_arrays, ws=None,
+                  status: Status | None = None, stream=None):
+    """grad_arrays: the pointer arrays from ReversibleStack.grads()."""
+    _require_cuda(y1, y2, dy1, dy2, x1, x2, dx1, dx2)
+    T = y1.shape[0]
+    ws = ws if ws is not None else workspace(stack.workspace_size(T), y1.device)
+    f, g = stack.ptrs()
+    aF, aG = grad_arrays
+    _check("rev_stack_bwd", lib().rev_stack_bwd(
+        y1.data_ptr(), y2.data_ptr(), dy1.data_ptr(), dy2.data_ptr(), T, stack.L, f, g, x1.data_ptr(),
+        x2.data_ptr(), dx1.data_ptr(), dx2.data_ptr(), ctypes.cast(aF, ctypes.c_void_p),
+        ctypes.cast(aG, ctypes.c_void_p), ws.data_ptr(), ws.numel(), status.ptr() if status else None,
+        _stream(stream)))
+    return x1, x2, dx1, dx2
+
+
+# ---------------------------------------------------------------- adapter optimizer
+
+
+def tqp_adamw_step(param, exp_avg, exp_avg_sq, grad, step: int, lr: float, beta1: float = 0.9, beta2: float = 0.999,
+                   eps: float = 1e-8, weight_decay: float = 0.0, grad_scale: float = 1.0, param_bf16=None,
+                   status: Status | None = None, stream=None):
+    """One fused AdamW step over flat fp32 buffers (see include/tqp_moe.h)."""
+    import torch
+    _require_cuda(param, exp_avg, exp_avg_sq, grad, param_bf16)
+    n = param.numel()
+    for name, t in (("exp_avg", exp_avg), ("exp_avg_sq", exp_avg_sq), ("grad", grad)):
+        if t.numel() != n or t.dtype != torch.float32 or not t.is_contiguous():
+            raise ValueError(f"{name} must be a contiguous fp32 tensor of {n} elements")
+    if param.dtype != torch.float32 or not param.is_contiguous():
+        raise ValueError("param must be a contiguous fp32 tensor")
+    if param_bf16 is not None and (param_bf16.numel() != n or param_bf16.element_size() != 2):
+        raise ValueError("param_bf16 must hold n 16-bit values")
+    _check("tqp_adamw_step", lib().tqp_adamw_step(param.data_ptr(), exp_avg.data_ptr(), exp_avg_sq.data_ptr(),
+                                                  grad.data_ptr(), _ptr(param_bf16), n, lr, beta1, beta2, eps,
+                                                  weight_decay, int(step), grad_scale,
+                                                  status.ptr() if status else None, _stream(stream)))
+
+
+class AdapterAdamW:
+    """AdamW over one layer's adapters: fp32 master copy and moments in the
+    flat gradient layout, and the layer's bf16 factors rewritten by each step.
+
+    step(grads) takes the layer's FlatGrads (summed over data-parallel ranks
+    already, if any)."""
+
+    def __init__(self, layer: DeviceLayer, lr: float, betas=(0.9, 0.999), eps: float = 1e-8,
+                 weight_decay: float = 0.0):
+        import torch
+        self.layer, self.lr, self.betas, self.eps, self.wd = layer, lr, betas, eps, weight_decay
+        self.master = layer.lora_flat.view(torch.bfloat16).float()
+        self.exp_avg = torch.zeros_like(self.master)
+        self.exp_avg_sq = torch.zeros_like(self.master)
+        self.t = 0
+
+    def step(self, grads, grad_scale: float = 1.0, status: Status | None = None, stream=None):
+        flat = grads.flat if hasattr(grads, "flat") else grads
+        self.t += 1
+        tqp_adamw_step(self.master, self.exp_avg, self.exp_avg_sq, flat, self.t, self.lr, self.betas[0],
+                       self.betas[1], self.eps, self.wd, grad_scale, self.layer.lora_flat, status, stream)

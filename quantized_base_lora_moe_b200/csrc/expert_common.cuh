@@ -15,9 +15,10 @@ constexpr int kTRow = 272;   // staging row: one token's 128 features in fp16, +
 struct EpiSync {
   uint64_t* bar;
   uint32_t phase = 0;
-  __device__ __forceinline__ bool sync(volatile int* abort_flag, int32_t* status) {
+  // The result is warp-uniform (the callers go on to warp-collective tcgen05 loads).
+  __device__ __forceinline__ bool sync(Abort* abort_flag, int32_t* status) {
     mbar_arrive(bar);
-    const bool ok = mbar_wait<32>(bar, phase, abort_flag, status);
+    const bool ok = __all_sync(0xFFFFFFFFu, mbar_wait<32>(bar, phase, abort_flag, status));
     phase ^= 1u;
     return ok;
   }

@@ -1,9 +1,10 @@
 // Down projection of the TQP MoE experts with wide token blocks (sm_100a):
 //   O = H_e Wd^T + (s H Ad) Bd
-// ("Train low-rank adapters per expert" over "Quantize base expert weights",
-// Pattern 3; SwiGLU experts, TQP Quantization).
+// (low-rank adapters trained per expert over frozen quantised base expert
+// weights: "Reversible Sparse MoE Single Node", Pattern 3; SwiGLU experts, TQP
+// Quantization).
 //
-// As in expert_ffn.cu the contraction runs transposed, D[feature][token] =
+// As in the gate/up kernel (expert_ffn.cu), the contraction runs transposed, D[feature][token] =
 // Wd[feature][:] . H[token][:], with the dequantised 128-feature weight tile as
 // the tcgen05.mma A operand in TMEM and the expert's routed rows as the B
 // operand in shared memory. Here a unit takes up to 256 rows of one expert, so
@@ -32,7 +33,11 @@
 //               (int4 -> fp16) into TMEM; LoRA B rows
 // TMEM (512 columns): one accumulator in [0, 256), 8 weight stages of 32
 // columns (64 K values) in [256, 512). Token ring: 3 stages of 32 KB.
-// Every wait is bounded (tqp_device.cuh); no TMA multicast is used.
+// An O value of a routed row or a LoRA B value beyond the fp16 range raises
+// TQP_STATUS_NONFINITE; a group scale whose dequantised products are not exact
+// in fp16 raises TQP_STATUS_RANGE. Every wait is bounded (tqp_device.cuh); on an abort every
+// asynchronous copy and MMA still in flight is drained before the CTA frees
+// its memory. No TMA multicast is used.
 #include <cstdint>
 #include <cuda.h>
 #include <cuda_fp16.h>
@@ -70,7 +75,7 @@ struct Ctl {
   uint64_t drain;
   uint64_t epi[2];
   uint32_t tmem_base;
-  int abort_flag;
+  Abort ab;
 };
 
 constexpr size_t kSmemBytes = 1024 + size_t(kXStages) * kXStageBytes + size_t(kQStages) * kQStageBytes +
@@ -86,7 +91,7 @@ __global__ void __launch_bounds__(kThreads, 1)
   uint8_t* q_base = x_base + size_t(kXStages) * kXStageBytes;
   uint8_t* staging = q_base + size_t(kQStages) * kQStageBytes;
   Ctl* ctl = reinterpret_cast<Ctl*>(staging + kStaging);
-  volatile int* abort_flag = &ctl->abort_flag;
+  Abort* abort_flag = &ctl->ab;
 
   const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
@@ -111,7 +116,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     mbar_init(&ctl->drain, 1);
     mbar_init(&ctl->epi[0], 128);
     mbar_init(&ctl->epi[1], 128);
-    ctl->abort_flag = 0;
+    abort_init(&ctl->ab, a.wait_ns);
     fence_barrier_init();
   }
   if (warp == 4) {
@@ -143,11 +148,12 @@ __global__ void __launch_bounds__(kThreads, 1)
     uint8_t* drow = staging + row * kDRow;
     uint8_t* ct = staging + 128 * kDRow + eg * 32 * kTRow;
     EpiSync es{&ctl->epi[eg]};
+    uint32_t bad = 0;   // nonzero once an fp16 output of a valid token overflowed
     int it = 0;
     for (int u = blockIdx.x; u < nunits; u += gridDim.x, ++it) {
       const Unit un = us.take(u);
       const int n16 = (un.rows + 15) & ~15;
-      if (!mbar_wait<128>(&ctl->acc_full, uint32_t(it) & 1u, abort_flag, a.status)) break;
+      if (!__all_sync(0xFFFFFFFFu, mbar_wait<128>(&ctl->acc_full, uint32_t(it) & 1u, abort_flag, a.status))) break;
       tc_fence_after();
       // drain this group's chunks of this thread's feature row as fp16
 #pragma unroll 1
@@ -178,14 +184,17 @@ __global__ void __launch_bounds__(kThreads, 1)
         stage_tokens<16>(ct, 0, row, w);
         if (!es.sync(abort_flag, a.status)) { stop = true; break; }   // the chunk tile is complete
         const int nt = min(32, un.rows - c);
+        // (only valid tokens are stored and checked: padding columns hold stale data)
         for (int p = etid; p < nt * 16; p += 128) {
           const int t = p >> 4, fg = p & 15;
-          *reinterpret_cast<uint4*>(out + size_t(un.base + c + t) * a.out_ld + fg * 8) =
-              *reinterpret_cast<const uint4*>(ct + t * kTRow + fg * 16);
+          const uint4 v = *reinterpret_cast<const uint4*>(ct + t * kTRow + fg * 16);
+          bad |= f16x2_nonfinite(v.x) | f16x2_nonfinite(v.y) | f16x2_nonfinite(v.z) | f16x2_nonfinite(v.w);
+          *reinterpret_cast<uint4*>(out + size_t(un.base + c + t) * a.out_ld + fg * 8) = v;
         }
       }
       if (stop) break;
     }
+    if (__any_sync(0xFFFFFFFFu, bad != 0) && lane == 0) raise_status(a.status, TQP_STATUS_NONFINITE);
   } else if (warp == 4) {
     // ------------------------------------------------------------ MMA issuer
     if (lane == 0) {
@@ -224,19 +233,19 @@ __global__ void __launch_bounds__(kThreads, 1)
         if (!ok) break;
         umma_commit(&ctl->acc_full);
       }
+      // no MMA may still read or write TMEM when it is freed: wait for all of
+      // them (they run to completion whether or not the CTA aborted)
       umma_commit(&ctl->drain);
-      mbar_wait(&ctl->drain, 0, abort_flag, a.status);
+      mbar_drain(&ctl->drain, 0, 100000000ull);
     }
     __syncwarp();
   } else if (warp == 5) {
     // ------------------------------------------------------------ TMA producer (int4 + scales)
     if (lane == 0) {
       Ring q;
+      PendingFills pend;
       const uint32_t bytes = uint32_t(4096 + 256 * ngrp);
       const int gpe = a.in_dim / a.g;
-      int issued = 0;
-      uint32_t last_phase = 0;
-      int last_stage = 0;
       for (int u = blockIdx.x; u < nunits; u += gridDim.x) {
         const Unit un = us.take(u);
         const int nrow0 = un.e * a.out_dim + un.nt * 128;
@@ -248,14 +257,13 @@ __global__ void __launch_bounds__(kThreads, 1)
           mbar_arrive_expect_tx(bar, bytes);
           tma_load_2d(smem_u32(qs), &tq, bar, km * (kK / 2), nrow0);
           tma_load_2d(smem_u32(qs + 4096), &ts, bar, un.nt * 128, un.e * gpe + (km * kK) / a.g);
-          ++issued;
-          last_stage = q.stage;
-          last_phase = q.phase;
+          pend.issued(q.stage, q.phase);
           q.next<kQStages>();
         }
         if (!ok) break;
       }
-      if (issued > 0 && *abort_flag) mbar_drain(&ctl->q_full[last_stage], last_phase);
+      // on an abort, wait (bounded) until every issued fill has landed
+      if (aborted(abort_flag)) pend.drain(ctl->q_full);
     }
   } else if (warp < kWWarp0) {
     // ------------------------------------------------------------ token producer
@@ -263,8 +271,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     const int chunk = tid & 7;
     const int row0 = tid >> 3;             // rows row0 + 16 j, j = 0..15
     Ring rx;
-    int pend_stage = -1;
-    uint32_t pend_phase = 0;
+    PendingFills pend;
     for (int u = blockIdx.x; u < nunits; u += gridDim.x) {
       const Unit un = us.take(u);
       bool ok = true;
@@ -290,8 +297,7 @@ __global__ void __launch_bounds__(kThreads, 1)
           mbar_arrive_expect_tx(full, uint32_t(kXStageBytes));
           tma_load_2d(smem_u32(st), &th, full, km * kK, un.base);
           tma_load_2d(smem_u32(st + kXStageBytes / 2), &th, full, km * kK, un.base + 128);
-          pend_stage = rx.stage;
-          pend_phase = rx.phase;
+          pend.issued(rx.stage, rx.phase);
         } else {
           mbar_arrive(full);
         }
@@ -300,7 +306,9 @@ __global__ void __launch_bounds__(kThreads, 1)
       if (!ok) break;
     }
     cp_async_wait_all();
-    if (tid == 0 && *abort_flag && pend_stage >= 0) mbar_drain(&ctl->x_full[pend_stage], pend_phase);
+    // on an abort, wait (bounded) until every TMA fill issued here has landed
+    // (a stage's other arrivals may never come; that wait then runs out)
+    if (tid == 0 && aborted(abort_flag)) pend.drain(ctl->x_full);
   } else {
     // ------------------------------------------------------------ weight producer
     const int wi = warp - kWWarp0;            // 0..15
@@ -310,6 +318,8 @@ __global__ void __launch_bounds__(kThreads, 1)
     const uint32_t tw = tmem_base + (uint32_t(32 * (warp & 3)) << 16) + kWBase + uint32_t(kh * 16);
     const int code_off = lrow * 32 + ((kh ^ ((lrow >> 2) & 1)) << 4);   // 32B-swizzled code rows
     const int scale_off = 4096 + (((ngrp == 2) ? kh : 0) * 128 + lrow) * 2;
+    bool inexact = false;   // a group scale whose products q * s are not exact in fp16
+    bool lora_inf = false;  // a LoRA B value beyond the fp16 range
     int n = 0;   // stage counter
     int m = 0;   // main (code-carrying) stage counter
     for (int u = blockIdx.x; u < nunits; u += gridDim.x) {
@@ -329,7 +339,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         if ((n & 1) != grp) continue;
         const int st = n % kWStages;
         const uint32_t ph = uint32_t(n / kWStages) & 1u;
-        if (!mbar_wait(&ctl->w_empty[st], ph ^ 1u, abort_flag, a.status)) { ok = false; break; }
+        if (!__all_sync(0xFFFFFFFFu, mbar_wait(&ctl->w_empty[st], ph ^ 1u, abort_flag, a.status))) { ok = false; break; }
         tc_fence_after();
         uint32_t v[16];
         if (!main_stage) {
@@ -338,17 +348,17 @@ __global__ void __launch_bounds__(kThreads, 1)
             const int colk = kb * kK + kh * 32 + c * 8;
             uint4 w4 = make_uint4(0, 0, 0, 0);
             if (colk < a.r)
-              w4 = bf16x8_to_f16x8(
-                  __ldg(reinterpret_cast<const uint4*>(a.b0 + (size_t(un.e) * a.out_dim + feat) * a.r + colk)));
+              w4 = bf16x8_to_f16x8_chk(
+                  __ldg(reinterpret_cast<const uint4*>(a.b0 + (size_t(un.e) * a.out_dim + feat) * a.r + colk)), lora_inf);
             v[4 * c] = w4.x; v[4 * c + 1] = w4.y; v[4 * c + 2] = w4.z; v[4 * c + 3] = w4.w;
           }
         } else {
           const int qst = mq % kQStages;
           const uint32_t qph = uint32_t(mq / kQStages) & 1u;
-          if (!mbar_wait(&ctl->q_full[qst], qph, abort_flag, a.status)) { ok = false; break; }
+          if (!__all_sync(0xFFFFFFFFu, mbar_wait(&ctl->q_full[qst], qph, abort_flag, a.status))) { ok = false; break; }
           const uint8_t* qs = q_base + size_t(qst) * kQStageBytes;
           const uint4 wd = *reinterpret_cast<const uint4*>(qs + code_off);
-          const uint32_t s2 = scale_pair(*reinterpret_cast<const uint16_t*>(qs + scale_off));
+          const uint32_t s2 = scale_pair_chk(*reinterpret_cast<const uint16_t*>(qs + scale_off), inexact);
           const uint4 d0 = dequant_word(wd.x, s2), d1 = dequant_word(wd.y, s2);
           const uint4 d2 = dequant_word(wd.z, s2), d3 = dequant_word(wd.w, s2);
           // the code slot's values have been consumed; its next fill is an
@@ -367,6 +377,8 @@ __global__ void __launch_bounds__(kThreads, 1)
       }
       if (!ok) break;
     }
+    if (__any_sync(0xFFFFFFFFu, inexact) && lane == 0) raise_status(a.status, TQP_STATUS_RANGE);
+    if (__any_sync(0xFFFFFFFFu, lora_inf) && lane == 0) raise_status(a.status, TQP_STATUS_NONFINITE);
   }
 
   tc_fence_before();
@@ -380,13 +392,8 @@ __global__ void __launch_bounds__(kThreads, 1)
 }  // namespace down_wide
 
 int run_expert_down_wide(const GemmArgs& a, const Maps& mp, int units_upper, cudaStream_t s) {
-  static bool attr_set = false;
-  if (!attr_set) {
-    if (cudaFuncSetAttribute(down_wide::down_wide_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                             int(down_wide::kSmemBytes)) != cudaSuccess)
-      return TQP_ERR_CUDA;
-    attr_set = true;
-  }
+  static DeviceFlags attr_done;
+  if (!attr_done.test_and_set_device(down_wide::down_wide_kernel, int(down_wide::kSmemBytes))) return TQP_ERR_CUDA;
   const int grid = units_upper < num_sms() ? (units_upper > 0 ? units_upper : 1) : num_sms();
   down_wide::down_wide_kernel<<<grid, down_wide::kThreads, down_wide::kSmemBytes, s>>>(a, mp.m[TQ0], mp.m[TS0],
                                                                                         mp.m[TA]);

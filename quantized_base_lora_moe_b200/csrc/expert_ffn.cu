@@ -1,9 +1,9 @@
-// Forward expert projections of the TQP MoE layer with the dequantised base
+// Gate/up expert projection of the TQP MoE layer with the dequantised base
 // weights held in tensor memory (sm_100a, tcgen05):
-//   GATEUP : [G|U] = X_e [Wg|Wu]^T + (s X [Ag|Au]) [Bg|Bu],  H = silu(G) * U
-//   DOWN   : O = H_e Wd^T + (s H Ad) Bd
-// ("Train low-rank adapters per expert" over "Quantize base expert weights",
-// Pattern 3; SwiGLU experts, TQP Quantization).
+//   [G|U] = X_e [Wg|Wu]^T + (s X [Ag|Au]) [Bg|Bu],  H = silu(G) * U
+// (low-rank adapters trained per expert over frozen quantised base expert
+// weights: "Reversible Sparse MoE Single Node", Pattern 3; SwiGLU experts, TQP
+// Quantization).
 //
 // The contraction runs transposed: D[feature][token] = W[feature][:] . X[token][:],
 // with W (M = 128 output features of one tile) as the tcgen05.mma A operand in
@@ -15,33 +15,32 @@
 //
 // Work unit = (expert e, 128-feature tile, block of up to 128 routed rows);
 // units are ordered (expert, tile, block) over a persistent grid. One K stage
-// is 8 tcgen05.mma of 128 x N x 16 (GATEUP: 64 K for gate and for up; DOWN:
-// 128 K), so that one barrier round trip is amortised over 8 MMAs. Per CTA
-// (1 per SM, 832 threads):
+// is 8 tcgen05.mma of 128 x N x 16 (64 K for gate and for up), so that one
+// barrier round trip is amortised over 8 MMAs. Per CTA (1 per SM, 832 threads):
 //   warps 0-3   epilogue (TMEM lanes 32w..32w+31 = features of the tile)
 //   warp  4     TMEM allocation + one thread issuing tcgen05.mma
 //   warp  5     TMA producer of the int4 code / bf16 scale ring (the code tiles
-//               come 32B- / 64B-swizzled, so the row reads below are free of
-//               bank conflicts)
+//               come 32B-swizzled, so the row reads below are free of bank
+//               conflicts)
 //   warps 6-9   token producer: cp.async row gathers (rows picked by perm_token)
-//               or TMA tiles of contiguous rows, and the rank-space rows
+//               and the rank-space rows
 //   warps 10-25 weight producer, two groups of 8 warps on alternate stages:
 //               each thread dequantises 64 K values of one weight row
 //               (int4 -> fp16) into TMEM; LoRA B rows
-// TMEM (512 columns): accumulators in [0, 256), 4 weight stages of 64 columns
-// in [256, 512). A pipeline stage pairs one token tile (shared memory) with
+// TMEM (512 columns): accumulators in [0, 256) (gate cols [0,128), up
+// [128,256)), 4 weight stages of 64 columns in [256, 512), each holding gate 32
+// | up 32 columns. A pipeline stage pairs one token tile (shared memory) with
 // one weight stage (TMEM): one "full" barrier collects both producers'
-// arrivals and one commit per stage frees both.
-//   GATEUP: one accumulator (gate cols [0,128), up [128,256)); a weight stage
-//           holds gate 32 | up 32 columns. The epilogue drains G and U as fp16
-//           rows (one feature per thread, 16-byte stores) into shared memory,
-//           hands TMEM back, and then, while the next unit runs, computes
-//           SwiGLU in 32-token chunks transposed through a [token][feature]
-//           tile for 16-byte row stores.
-//   DOWN:   two accumulators of 128 columns; the epilogue drains a whole
-//           accumulator as fp16 into a [token][feature] tile, hands TMEM back,
-//           and then stores 16-byte row pieces.
-// Every wait is bounded (tqp_device.cuh); no TMA multicast is used.
+// arrivals and one commit per stage frees both. The epilogue drains G and U as
+// fp16 rows (one feature per thread, 16-byte stores) into shared memory, hands
+// TMEM back, and then, while the next unit runs, computes SwiGLU in 32-token
+// chunks transposed through a [token][feature] tile for 16-byte row stores.
+//
+// Range: an H (or kept G|U) value or a LoRA B value beyond the fp16 range
+// raises TQP_STATUS_NONFINITE; a group scale whose dequantised products are not
+// exact in fp16 raises TQP_STATUS_RANGE. Every wait is bounded (tqp_device.cuh); on
+// an abort every asynchronous copy and MMA still in flight is drained before
+// the CTA frees its memory. No TMA multicast is used.
 #include <cstdint>
 #include <cuda.h>
 #include <cuda_fp16.h>
@@ -58,54 +57,39 @@ namespace tmem_ffn {
 constexpr int kWWarp0 = 10;           // first weight-producer warp
 constexpr int kWWarps = 16;
 constexpr int kThreads = (kWWarp0 + kWWarps) * 32;
-constexpr int kQStagesMax = 8;
-constexpr int kQStageBytes = 9216;    // up to 8192 B of codes + 1024 B of scales
+constexpr int kQStages = 8;
+constexpr int kQStageBytes = 9216;    // 8192 B of codes + up to 1024 B of scales
 constexpr uint32_t kWBase = 256;      // first TMEM column of the weight stages
-constexpr int kWStages = 4;
+constexpr int kStages = 4;            // pipeline stages (token tile + weight stage)
 constexpr uint32_t kWCols = 64;       // TMEM columns per weight stage
-
-template <int MODE> struct Cfg;
-template <> struct Cfg<GATEUP> {      // K stage 64: 128 token rows x 128 B
-  static constexpr int kK = 64, kXStageBytes = 16384, kStaging = (2 * 128 + 32) * kTRow, kQStages = 8;
-};
-template <> struct Cfg<DOWN> {        // K stage 128: two 64-wide swizzled sub-tiles
-  static constexpr int kK = 128, kXStageBytes = 32768, kStaging = 128 * kTRow, kQStages = 6;
-};
-constexpr int kStages = kWStages;     // pipeline stages (token tile + weight stage)
+constexpr int kK = 64;                // K per stage
+constexpr int kXBytes = 16384;        // 128 token rows x 128 B
+constexpr int kStaging = (2 * 128 + 32) * kTRow;   // G rows | U rows | chunk tile
 
 struct Ctl {
   uint64_t full[kStages], empty[kStages];
-  uint64_t q_full[kQStagesMax], q_empty[kQStagesMax];
-  uint64_t acc_full[2], acc_empty[2];
+  uint64_t q_full[kQStages], q_empty[kQStages];
+  uint64_t acc_full, acc_empty;
   uint64_t drain;
   uint64_t epi;
   uint32_t tmem_base;
-  int abort_flag;
+  Abort ab;
 };
 
-template <int MODE>
-constexpr size_t smem_bytes() {
-  return 1024 + size_t(kStages) * Cfg<MODE>::kXStageBytes + size_t(Cfg<MODE>::kQStages) * kQStageBytes +
-         size_t(Cfg<MODE>::kStaging) + sizeof(Ctl);
-}
-static_assert(smem_bytes<GATEUP>() <= 232448 && smem_bytes<DOWN>() <= 232448, "shared memory budget");
+constexpr size_t kSmemBytes =
+    1024 + size_t(kStages) * kXBytes + size_t(kQStages) * kQStageBytes + size_t(kStaging) + sizeof(Ctl);
+static_assert(kSmemBytes + 2 * (kSchedSmemE + 1) * 4 <= 232448, "shared memory budget");
 
-template <int MODE>
 __global__ void __launch_bounds__(kThreads, 1)
-    expert_ffn_kernel(const GemmArgs a, const __grid_constant__ CUtensorMap tq0,
-                      const __grid_constant__ CUtensorMap tq1, const __grid_constant__ CUtensorMap ts0,
-                      const __grid_constant__ CUtensorMap ts1, const __grid_constant__ CUtensorMap th) {
-  constexpr bool kGU = (MODE == GATEUP);
-  constexpr int kK = Cfg<MODE>::kK;
-  constexpr int kXBytes = Cfg<MODE>::kXStageBytes;
-  constexpr int kQStages = Cfg<MODE>::kQStages;
+    gateup_kernel(const GemmArgs a, const __grid_constant__ CUtensorMap tq0, const __grid_constant__ CUtensorMap tq1,
+                  const __grid_constant__ CUtensorMap ts0, const __grid_constant__ CUtensorMap ts1) {
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   uint8_t* x_base = smem;
   uint8_t* q_base = x_base + size_t(kStages) * kXBytes;
   uint8_t* staging = q_base + size_t(kQStages) * kQStageBytes;
-  Ctl* ctl = reinterpret_cast<Ctl*>(staging + Cfg<MODE>::kStaging);
-  volatile int* abort_flag = &ctl->abort_flag;
+  Ctl* ctl = reinterpret_cast<Ctl*>(staging + kStaging);
+  Abort* abort_flag = &ctl->ab;
 
   const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
@@ -121,13 +105,11 @@ __global__ void __launch_bounds__(kThreads, 1)
       mbar_init(&ctl->q_full[i], 1);
       mbar_init(&ctl->q_empty[i], kWWarps * 16);
     }
-    for (int i = 0; i < 2; ++i) {
-      mbar_init(&ctl->acc_full[i], 1);
-      mbar_init(&ctl->acc_empty[i], 128);
-    }
+    mbar_init(&ctl->acc_full, 1);
+    mbar_init(&ctl->acc_empty, 128);
     mbar_init(&ctl->drain, 1);
     mbar_init(&ctl->epi, 128);
-    ctl->abort_flag = 0;
+    abort_init(&ctl->ab, a.wait_ns);
     fence_barrier_init();
   }
   if (warp == 4) {
@@ -137,12 +119,9 @@ __global__ void __launch_bounds__(kThreads, 1)
   if (threadIdx.x == 5 * 32) {
     prefetch_tmap(&tq0);
     prefetch_tmap(&ts0);
-    if (kGU) {
-      prefetch_tmap(&tq1);
-      prefetch_tmap(&ts1);
-    }
+    prefetch_tmap(&tq1);
+    prefetch_tmap(&ts1);
   }
-  if (threadIdx.x == 6 * 32 && !kGU) prefetch_tmap(&th);
   tc_fence_before();
   __syncthreads();
   tc_fence_after();
@@ -164,102 +143,79 @@ __global__ void __launch_bounds__(kThreads, 1)
     for (int u = blockIdx.x; u < nunits; u += gridDim.x, ++it) {
       const Unit un = us.take(u);
       const int n16 = (un.rows + 15) & ~15;
-      if (kGU) {
-        if (!mbar_wait<128>(&ctl->acc_full[0], uint32_t(it) & 1u, abort_flag, a.status)) break;
-        tc_fence_after();
-        // staging: G rows [feature][token] | U rows | chunk tile [32 tokens][feature]
-        uint8_t* grow_s = staging + row * kTRow;
-        uint8_t* urow_s = staging + (128 + row) * kTRow;
-        uint8_t* ht = staging + 256 * kTRow;
-        // drain: this thread's feature row of G and U as fp16 (16-byte stores)
+      if (!__all_sync(0xFFFFFFFFu, mbar_wait<128>(&ctl->acc_full, uint32_t(it) & 1u, abort_flag, a.status))) break;
+      tc_fence_after();
+      // staging: G rows [feature][token] | U rows | chunk tile [32 tokens][feature]
+      uint8_t* grow_s = staging + row * kTRow;
+      uint8_t* urow_s = staging + (128 + row) * kTRow;
+      uint8_t* ht = staging + 256 * kTRow;
+      // drain: this thread's feature row of G and U as fp16 (16-byte stores)
 #pragma unroll 1
-        for (int c = 0; c < n16; c += 32) {
+      for (int c = 0; c < n16; c += 32) {
 #pragma unroll
-          for (int m2 = 0; m2 < 2; ++m2) {
-            float v[32];
-            tmem_ld32(tl + uint32_t(128 * m2 + c), v);
-            uint4* dst = reinterpret_cast<uint4*>((m2 ? urow_s : grow_s) + 2 * c);
+        for (int m2 = 0; m2 < 2; ++m2) {
+          float v[32];
+          tmem_ld32(tl + uint32_t(128 * m2 + c), v);
+          uint4* dst = reinterpret_cast<uint4*>((m2 ? urow_s : grow_s) + 2 * c);
 #pragma unroll
-            for (int q4 = 0; q4 < 4; ++q4)
-              dst[q4] = make_uint4(f32x2_to_f16x2(v[8 * q4], v[8 * q4 + 1]), f32x2_to_f16x2(v[8 * q4 + 2], v[8 * q4 + 3]),
-                                   f32x2_to_f16x2(v[8 * q4 + 4], v[8 * q4 + 5]),
-                                   f32x2_to_f16x2(v[8 * q4 + 6], v[8 * q4 + 7]));
-          }
+          for (int q4 = 0; q4 < 4; ++q4)
+            dst[q4] = make_uint4(f32x2_to_f16x2(v[8 * q4], v[8 * q4 + 1]), f32x2_to_f16x2(v[8 * q4 + 2], v[8 * q4 + 3]),
+                                 f32x2_to_f16x2(v[8 * q4 + 4], v[8 * q4 + 5]),
+                                 f32x2_to_f16x2(v[8 * q4 + 6], v[8 * q4 + 7]));
         }
-        tc_fence_before();
-        mbar_arrive(&ctl->acc_empty[0]);
-        // SwiGLU per 32-token chunk (own feature row), transposed through the chunk
-        // tile, then 16-byte row stores; overlaps the next unit's main loop
-        uint16_t* hout = static_cast<uint16_t*>(a.out) + un.nt * 128;
-        bool stop = false;
-#pragma unroll 1
-        for (int c = 0; c < n16; c += 32) {
-          // 16 words (32 tokens) of this thread's staged row
-          auto row_words = [&](const uint8_t* src, uint32_t* w) {
-#pragma unroll
-            for (int q4 = 0; q4 < 4; ++q4) {
-              const uint4 v4 = *reinterpret_cast<const uint4*>(src + 2 * c + 16 * q4);
-              w[4 * q4] = v4.x; w[4 * q4 + 1] = v4.y; w[4 * q4 + 2] = v4.z; w[4 * q4 + 3] = v4.w;
-            }
-          };
-          uint32_t hw[16];
-          {
-            uint32_t gw[16], uw[16];
-            row_words(grow_s, gw);
-            row_words(urow_s, uw);
-#pragma unroll
-            for (int j = 0; j < 16; ++j) hw[j] = swiglu_pair(gw[j], uw[j]);
-          }
-          const int nt = min(32, un.rows - c);
-          // one [32 token][128 feature] chunk through the tile: wait until the tile
-          // is free, transpose into it, wait until complete, 16-byte row stores
-          auto emit = [&](const uint32_t* w, uint16_t* dst, size_t ld) -> bool {
-            if (!es.sync(abort_flag, a.status)) return false;
-            stage_tokens<16>(ht, 0, row, w);
-            if (!es.sync(abort_flag, a.status)) return false;
-            for (int p = threadIdx.x; p < nt * 16; p += 128) {
-              const int t = p >> 4, fg = p & 15;
-              *reinterpret_cast<uint4*>(dst + size_t(un.base + c + t) * ld + fg * 8) =
-                  *reinterpret_cast<const uint4*>(ht + t * kTRow + fg * 16);
-            }
-            return true;
-          };
-          if (!emit(hw, hout, size_t(a.out_ld))) { stop = true; break; }
-          if (a.aux) {  // keep the pre-activations for the backward (re-read from the staged rows)
-            uint16_t* aux = a.aux + un.nt * 128;
-            uint32_t w16[16];
-            row_words(grow_s, w16);
-            if (!emit(w16, aux, 2 * size_t(a.f_dim))) { stop = true; break; }
-            row_words(urow_s, w16);
-            if (!emit(w16, aux + a.f_dim, 2 * size_t(a.f_dim))) { stop = true; break; }
-          }
-        }
-        if (stop) break;
-      } else {
-        const int ab = it & 1;
-        if (!mbar_wait<128>(&ctl->acc_full[ab], uint32_t(it >> 1) & 1u, abort_flag, a.status)) break;
-        tc_fence_after();
-        // drain the whole accumulator as fp16 into the [token][feature] tile
-#pragma unroll 1
-        for (int c = 0; c < n16; c += 16) {
-          float v[16];
-          tmem_ld16(tl + uint32_t(ab * 128 + c), v);
-          uint32_t pk[8];
-#pragma unroll
-          for (int j = 0; j < 8; ++j) pk[j] = f32x2_to_f16x2(v[2 * j], v[2 * j + 1]);
-          stage_tokens<8>(staging, c, row, pk);
-        }
-        tc_fence_before();
-        mbar_arrive(&ctl->acc_empty[ab]);
-        if (!es.sync(abort_flag, a.status)) break;
-        uint16_t* out = static_cast<uint16_t*>(a.out) + un.nt * 128;
-        for (int p = threadIdx.x; p < un.rows * 16; p += 128) {
-          const int t = p >> 4, fg = p & 15;
-          *reinterpret_cast<uint4*>(out + size_t(un.base + t) * a.out_ld + fg * 8) =
-              *reinterpret_cast<const uint4*>(staging + t * kTRow + fg * 16);
-        }
-        if (!es.sync(abort_flag, a.status)) break;  // the tile is free for the next unit's drain
       }
+      tc_fence_before();
+      mbar_arrive(&ctl->acc_empty);
+      // SwiGLU per 32-token chunk (own feature row), transposed through the chunk
+      // tile, then 16-byte row stores; overlaps the next unit's main loop
+      uint16_t* hout = static_cast<uint16_t*>(a.out) + un.nt * 128;
+      bool stop = false;
+#pragma unroll 1
+      for (int c = 0; c < n16; c += 32) {
+        // 16 words (32 tokens) of this thread's staged row
+        auto row_words = [&](const uint8_t* src, uint32_t* w) {
+#pragma unroll
+          for (int q4 = 0; q4 < 4; ++q4) {
+            const uint4 v4 = *reinterpret_cast<const uint4*>(src + 2 * c + 16 * q4);
+            w[4 * q4] = v4.x; w[4 * q4 + 1] = v4.y; w[4 * q4 + 2] = v4.z; w[4 * q4 + 3] = v4.w;
+          }
+        };
+        uint32_t hw[16];
+        {
+          uint32_t gw[16], uw[16];
+          row_words(grow_s, gw);
+          row_words(urow_s, uw);
+#pragma unroll
+          for (int j = 0; j < 16; ++j) hw[j] = swiglu_pair(gw[j], uw[j]);
+        }
+        const int nt = min(32, un.rows - c);
+        // one [32 token][128 feature] chunk through the tile: wait until the tile
+        // is free, transpose into it, wait until complete, 16-byte row stores
+        auto emit = [&](const uint32_t* w, uint16_t* dst, size_t ld) -> bool {
+          if (!es.sync(abort_flag, a.status)) return false;
+          stage_tokens<16>(ht, 0, row, w);
+          if (!es.sync(abort_flag, a.status)) return false;
+          // (only valid tokens are stored and checked: padding columns hold stale data)
+          for (int p = threadIdx.x; p < nt * 16; p += 128) {
+            const int t = p >> 4, fg = p & 15;
+            const uint4 v = *reinterpret_cast<const uint4*>(ht + t * kTRow + fg * 16);
+            if (f16x2_nonfinite(v.x) | f16x2_nonfinite(v.y) | f16x2_nonfinite(v.z) | f16x2_nonfinite(v.w))
+              raise_status(a.status, TQP_STATUS_NONFINITE);   // rare: reported where it happens
+            *reinterpret_cast<uint4*>(dst + size_t(un.base + c + t) * ld + fg * 8) = v;
+          }
+          return true;
+        };
+        if (!emit(hw, hout, size_t(a.out_ld))) { stop = true; break; }
+        if (a.aux) {  // keep the pre-activations for the backward (re-read from the staged rows)
+          uint16_t* aux = a.aux + un.nt * 128;
+          uint32_t w16[16];
+          row_words(grow_s, w16);
+          if (!emit(w16, aux, 2 * size_t(a.f_dim))) { stop = true; break; }
+          row_words(urow_s, w16);
+          if (!emit(w16, aux + a.f_dim, 2 * size_t(a.f_dim))) { stop = true; break; }
+        }
+      }
+      if (stop) break;
     }
   } else if (warp == 4) {
     // ------------------------------------------------------------ MMA issuer
@@ -271,65 +227,41 @@ __global__ void __launch_bounds__(kThreads, 1)
         const Unit un = us.take(u);
         const int n16 = (un.rows + 15) & ~15;
         const uint32_t idesc = idesc_f16(128, n16);
-        const int ab = kGU ? 0 : (it & 1);
-        const uint32_t eph = (kGU ? uint32_t(it) & 1u : uint32_t(it >> 1) & 1u) ^ 1u;
-        if (!mbar_wait(&ctl->acc_empty[ab], eph, abort_flag, a.status)) { ok = false; break; }
+        if (!mbar_wait(&ctl->acc_empty, (uint32_t(it) & 1u) ^ 1u, abort_flag, a.status)) { ok = false; break; }
         tc_fence_after();
-        const uint32_t dacc = tmem_base + uint32_t(ab * 128);
+        const uint32_t dacc = tmem_base;
         for (int kb = 0; kb < nkb; ++kb) {
           if (!mbar_wait(&ctl->full[rs.stage], rs.phase, abort_flag, a.status)) { ok = false; break; }
           tc_fence_after();
-          const uint32_t xs = smem_u32(x_base + size_t(rs.stage) * kXBytes);
-          const uint64_t bdesc = sdesc_k_sw128(xs);
+          const uint64_t bdesc = sdesc_k_sw128(smem_u32(x_base + size_t(rs.stage) * kXBytes));
           const uint32_t wa = tmem_base + kWBase + uint32_t(rs.stage) * kWCols;
-          if (kb >= a.nkb_lora) {
-            if (kGU) {
-#pragma unroll
-              for (int kk = 0; kk < 4; ++kk) {
-                const uint32_t acc = (kb > 0 || kk > 0) ? 1u : 0u;
-                umma_f16_ts(dacc, wa + uint32_t(8 * kk), bdesc + uint64_t(2 * kk), idesc, acc);
-                umma_f16_ts(dacc + 128, wa + 32 + uint32_t(8 * kk), bdesc + uint64_t(2 * kk), idesc, acc);
-              }
-            } else {
-              const uint64_t bdesc1 = sdesc_k_sw128(xs + 16384);
-#pragma unroll
-              for (int kk = 0; kk < 8; ++kk) {
-                const uint32_t acc = (kb > 0 || kk > 0) ? 1u : 0u;
-                umma_f16_ts(dacc, wa + uint32_t(8 * kk), (kk < 4 ? bdesc : bdesc1) + uint64_t(2 * (kk & 3)), idesc,
-                            acc);
-              }
-            }
-          } else {
-            // rank-space stage: only the first lora_k columns are live (within the first 64)
-            const int ksteps = (min(kK, a.lora_k - kb * kK) + 15) / 16;
-            for (int kk = 0; kk < ksteps; ++kk) {
-              const uint32_t acc = (kb > 0 || kk > 0) ? 1u : 0u;
-              umma_f16_ts(dacc, wa + uint32_t(8 * kk), bdesc + uint64_t(2 * kk), idesc, acc);
-              if (kGU) umma_f16_ts(dacc + 128, wa + 32 + uint32_t(8 * kk), bdesc + uint64_t(2 * kk), idesc, acc);
-            }
+          // the rank-space stage has only its first lora_k columns live (within the first 64)
+          const int ksteps = (kb >= a.nkb_lora) ? 4 : (min(kK, a.lora_k - kb * kK) + 15) / 16;
+          for (int kk = 0; kk < ksteps; ++kk) {
+            const uint32_t acc = (kb > 0 || kk > 0) ? 1u : 0u;
+            umma_f16_ts(dacc, wa + uint32_t(8 * kk), bdesc + uint64_t(2 * kk), idesc, acc);
+            umma_f16_ts(dacc + 128, wa + 32 + uint32_t(8 * kk), bdesc + uint64_t(2 * kk), idesc, acc);
           }
           umma_commit(&ctl->empty[rs.stage]);
           rs.next<kStages>();
         }
         if (!ok) break;
-        umma_commit(&ctl->acc_full[ab]);
+        umma_commit(&ctl->acc_full);
       }
-      // make sure no MMA is still reading or writing TMEM before teardown
+      // no MMA may still read or write TMEM when it is freed: wait for all of
+      // them (they run to completion whether or not the CTA aborted)
       umma_commit(&ctl->drain);
-      mbar_wait(&ctl->drain, 0, abort_flag, a.status);
+      mbar_drain(&ctl->drain, 0, 100000000ull);
     }
     __syncwarp();
   } else if (warp == 5) {
     // ------------------------------------------------------------ TMA producer (int4 + scales)
     if (lane == 0) {
       Ring q;
-      // GATEUP: gate codes [128 rows][32 B] | up codes | gate scales [ngrp][128] | up scales
-      // DOWN:   codes [128 rows][64 B] | scales [ngrp][128]
-      const uint32_t bytes = kGU ? uint32_t(8192 + 512 * ngrp) : uint32_t(8192 + 256 * ngrp);
+      PendingFills pend;
+      // gate codes [128 rows][32 B] | up codes | gate scales [ngrp][128] | up scales
+      const uint32_t bytes = uint32_t(8192 + 512 * ngrp);
       const int gpe = a.in_dim / a.g;  // scale rows per expert
-      int issued = 0;
-      uint32_t last_phase = 0;
-      int last_stage = 0;
       for (int u = blockIdx.x; u < nunits; u += gridDim.x) {
         const Unit un = us.take(u);
         const int nrow0 = un.e * a.out_dim + un.nt * 128;
@@ -341,22 +273,16 @@ __global__ void __launch_bounds__(kThreads, 1)
           const int srow = un.e * gpe + (km * kK) / a.g;
           mbar_arrive_expect_tx(bar, bytes);
           tma_load_2d(smem_u32(qs), &tq0, bar, km * (kK / 2), nrow0);
-          if (kGU) {
-            tma_load_2d(smem_u32(qs + 4096), &tq1, bar, km * (kK / 2), nrow0);
-            tma_load_2d(smem_u32(qs + 8192), &ts0, bar, un.nt * 128, srow);
-            tma_load_2d(smem_u32(qs + 8192 + 256 * ngrp), &ts1, bar, un.nt * 128, srow);
-          } else {
-            tma_load_2d(smem_u32(qs + 8192), &ts0, bar, un.nt * 128, srow);
-          }
-          ++issued;
-          last_stage = q.stage;
-          last_phase = q.phase;
+          tma_load_2d(smem_u32(qs + 4096), &tq1, bar, km * (kK / 2), nrow0);
+          tma_load_2d(smem_u32(qs + 8192), &ts0, bar, un.nt * 128, srow);
+          tma_load_2d(smem_u32(qs + 8192 + 256 * ngrp), &ts1, bar, un.nt * 128, srow);
+          pend.issued(q.stage, q.phase);
           q.next<kQStages>();
         }
         if (!ok) break;
       }
-      // on an abort, wait (bounded) until the last issued stage has landed
-      if (issued > 0 && *abort_flag) mbar_drain(&ctl->q_full[last_stage], last_phase);
+      // on an abort, wait (bounded) until every issued fill has landed
+      if (aborted(abort_flag)) pend.drain(ctl->q_full);
     }
   } else if (warp < kWWarp0) {
     // ------------------------------------------------------------ token producer
@@ -367,17 +293,14 @@ __global__ void __launch_bounds__(kThreads, 1)
     const int chunk = tid & 7;
     const int row0 = tid >> 3;             // 0..15
     Ring rx;
-    int pend_stage = -1;
-    uint32_t pend_phase = 0;
     for (int u = blockIdx.x; u < nunits; u += gridDim.x) {
       const Unit un = us.take(u);
-      // source rows of this thread's 8 tile rows (token rows for the gathers,
-      // routed rows for the rank-space operand)
+      // source token rows of this thread's 8 tile rows
       int tok[8];
 #pragma unroll
       for (int j = 0; j < 8; ++j) {
         const int r = row0 + 16 * j;
-        tok[j] = (kGU && r < un.rows) ? __ldg(a.perm_token + un.base + r) : 0;
+        tok[j] = r < un.rows ? __ldg(a.perm_token + un.base + r) : 0;
       }
       bool ok = true;
       for (int kb = 0; kb < nkb; ++kb) {
@@ -385,8 +308,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         const uint32_t st_u = smem_u32(x_base + size_t(rx.stage) * kXBytes);
         uint64_t* full = &ctl->full[rx.stage];
         if (kb < a.nkb_lora) {
-          // rank-space rows (s X[Ag|Au] or s H Ad) in the first 64-wide sub-tile,
-          // zero-filled past lora_k (lora_k <= 128, and <= 64 for DOWN)
+          // rank-space rows s X[Ag|Au], zero-filled past lora_k (lora_k <= 128)
           const int colk = kb * kK + chunk * 8;
           const bool in = colk < a.lora_k;
 #pragma unroll
@@ -396,73 +318,56 @@ __global__ void __launch_bounds__(kThreads, 1)
               cp_async16(st_u + sw128_offset(r, chunk), a.a_lora + size_t(un.base + r) * a.lora_ld + (in ? colk : 0),
                          in ? 16u : 0u);
           }
-          cp_async_arrive_noinc(full);
         } else {
           const int km = kb - a.nkb_lora;
-          if (kGU) {
 #pragma unroll
-            for (int j = 0; j < 8; ++j) {
-              const int r = row0 + 16 * j;
-              if (r < un.rows)
-                cp_async16(st_u + sw128_offset(r, chunk), a.a_src + size_t(tok[j]) * a.a_ld + km * 64 + chunk * 8, 16);
-            }
-            cp_async_arrive_noinc(full);
-          } else if (tid == 0) {
-            mbar_arrive_expect_tx(full, uint32_t(kXBytes));
-            tma_load_2d(st_u, &th, full, km * 128, un.base);
-            tma_load_2d(st_u + 16384, &th, full, km * 128 + 64, un.base);
-            pend_stage = rx.stage;
-            pend_phase = rx.phase;
-          } else {
-            mbar_arrive(full);
+          for (int j = 0; j < 8; ++j) {
+            const int r = row0 + 16 * j;
+            if (r < un.rows)
+              cp_async16(st_u + sw128_offset(r, chunk), a.a_src + size_t(tok[j]) * a.a_ld + km * 64 + chunk * 8, 16);
           }
         }
+        cp_async_arrive_noinc(full);
         rx.next<kStages>();
       }
       if (!ok) break;
     }
     cp_async_wait_all();
-    // on an abort, wait (bounded) until the last TMA fill issued here has landed
-    // (the stage's other arrivals may never come; the wait then runs out)
-    if (tid == 0 && *abort_flag && pend_stage >= 0)
-      mbar_drain(&ctl->full[pend_stage], pend_phase);
   } else {
     // ------------------------------------------------------------ weight producer
     // Two groups of 8 warps take alternate pipeline stages, so that two stages
     // are being dequantised at any time (one stage's chain of code read ->
     // dequant -> TMEM store -> arrive is latency-bound). Within a group, a
     // thread converts 64 consecutive K values (8 int4 words) of one weight row:
-    // GATEUP: row lrow of the gate (mat 0) or up (mat 1) tile; DOWN: row lrow,
-    // K half kh of the 128-wide stage.
+    // row lrow of the gate (mat 0) or up (mat 1) tile.
     const int wi = warp - kWWarp0;            // 0..15
     const int grp = wi >> 3;                  // stage parity handled by this group
     const int gw = wi & 7;
     const int lrow = 32 * (warp & 3) + lane;  // TMEM lane = feature within the tile
-    const int half = gw >> 2;                 // GATEUP: mat; DOWN: K half
-    const uint32_t tw = tmem_base + (uint32_t(32 * (warp & 3)) << 16) + kWBase + uint32_t(half * 32);
+    const int mat = gw >> 2;                  // 0 gate, 1 up
+    const uint32_t tw = tmem_base + (uint32_t(32 * (warp & 3)) << 16) + kWBase + uint32_t(mat * 32);
     // the two 16-byte code chunks of this thread inside a stage (TMA-swizzled rows)
-    const int c0_off = kGU ? (half * 4096 + lrow * 32 + ((0 ^ ((lrow >> 2) & 1)) << 4))
-                           : (lrow * 64 + (((2 * half) ^ ((lrow >> 1) & 3)) << 4));
-    const int c1_off = kGU ? (half * 4096 + lrow * 32 + ((1 ^ ((lrow >> 2) & 1)) << 4))
-                           : (lrow * 64 + (((2 * half + 1) ^ ((lrow >> 1) & 3)) << 4));
+    const int c0_off = mat * 4096 + lrow * 32 + ((0 ^ ((lrow >> 2) & 1)) << 4);
+    const int c1_off = mat * 4096 + lrow * 32 + ((1 ^ ((lrow >> 2) & 1)) << 4);
     // scale rows of the two 32-wide K halves of this thread's slice
-    const int k0 = kGU ? 0 : 64 * half;
-    const int g_lo = (ngrp == 1) ? 0 : k0 / a.g, g_hi = (ngrp == 1) ? 0 : (k0 + 32) / a.g;
-    const int sbase = 8192 + (kGU ? half * 256 * ngrp : 0);
+    const int g_lo = 0, g_hi = (ngrp == 1) ? 0 : 32 / a.g;
+    const int sbase = 8192 + mat * 256 * ngrp;
     const int s_lo_off = sbase + (g_lo * 128 + lrow) * 2, s_hi_off = sbase + (g_hi * 128 + lrow) * 2;
-    const bool is_up = kGU && half == 1;
+    const bool is_up = mat == 1;
+    bool inexact = false;   // a group scale whose products q * s are not exact in fp16
+    bool lora_inf = false;  // a LoRA B value beyond the fp16 range
     int n = 0;    // pipeline stage counter of this CTA
     int m = 0;    // main (code-carrying) stage counter
     for (int u = blockIdx.x; u < nunits; u += gridDim.x) {
       const Unit un = us.take(u);
       const int feat = un.nt * 128 + lrow;  // output feature
       bool ok = true;
-      if (a.nkb_lora > 0 && grp == 0 && (kGU || half == 0) && u + int(gridDim.x) < nunits) {
+      if (a.nkb_lora > 0 && grp == 0 && u + int(gridDim.x) < nunits) {
         // the next unit's LoRA B row into L2 (its rank-space stage comes first)
         const Unit nx = us.peek();
         const uint16_t* bsrc = is_up ? a.b1 : a.b0;
-        const uint16_t* row = bsrc + (size_t(nx.e) * a.out_dim + nx.nt * 128 + lrow) * a.r;
-        for (int off = 0; off < a.r; off += 64) prefetch_l2(row + off);
+        const uint16_t* rowp = bsrc + (size_t(nx.e) * a.out_dim + nx.nt * 128 + lrow) * a.r;
+        for (int off = 0; off < a.r; off += 64) prefetch_l2(rowp + off);
       }
       for (int kb = 0; kb < nkb; ++kb, ++n) {
         const bool main_stage = kb >= a.nkb_lora;
@@ -471,32 +376,32 @@ __global__ void __launch_bounds__(kThreads, 1)
         if ((n & 1) != grp) continue;
         const int st = n & (kStages - 1);
         const uint32_t ph = uint32_t(n / kStages) & 1u;
-        if (!mbar_wait(&ctl->empty[st], ph ^ 1u, abort_flag, a.status)) { ok = false; break; }
+        if (!__all_sync(0xFFFFFFFFu, mbar_wait(&ctl->empty[st], ph ^ 1u, abort_flag, a.status))) { ok = false; break; }
         tc_fence_after();
         uint32_t v[32];
         if (!main_stage) {
           // LoRA B rows as fp16: gate rows hold Bg in K' [0, r), up rows Bu in [r, 2r)
 #pragma unroll
           for (int c = 0; c < 8; ++c) {
-            const int colk = kb * kK + k0 + c * 8;
+            const int colk = kb * kK + c * 8;
             const int src = is_up ? colk - a.r : colk;
             uint4 w4 = make_uint4(0, 0, 0, 0);
             if (src >= 0 && src < a.r) {
               const uint16_t* bsrc = is_up ? a.b1 : a.b0;
-              w4 = bf16x8_to_f16x8(
-                  __ldg(reinterpret_cast<const uint4*>(bsrc + (size_t(un.e) * a.out_dim + feat) * a.r + src)));
+              w4 = bf16x8_to_f16x8_chk(
+                  __ldg(reinterpret_cast<const uint4*>(bsrc + (size_t(un.e) * a.out_dim + feat) * a.r + src)), lora_inf);
             }
             v[4 * c] = w4.x; v[4 * c + 1] = w4.y; v[4 * c + 2] = w4.z; v[4 * c + 3] = w4.w;
           }
         } else {
           const int qst = mq % kQStages;
           const uint32_t qph = uint32_t(mq / kQStages) & 1u;
-          if (!mbar_wait(&ctl->q_full[qst], qph, abort_flag, a.status)) { ok = false; break; }
+          if (!__all_sync(0xFFFFFFFFu, mbar_wait(&ctl->q_full[qst], qph, abort_flag, a.status))) { ok = false; break; }
           const uint8_t* qs = q_base + size_t(qst) * kQStageBytes;
           const uint4 wa = *reinterpret_cast<const uint4*>(qs + c0_off);
           const uint4 wb = *reinterpret_cast<const uint4*>(qs + c1_off);
-          const uint32_t s_lo = scale_pair(*reinterpret_cast<const uint16_t*>(qs + s_lo_off));
-          const uint32_t s_hi = scale_pair(*reinterpret_cast<const uint16_t*>(qs + s_hi_off));
+          const uint32_t s_lo = scale_pair_chk(*reinterpret_cast<const uint16_t*>(qs + s_lo_off), inexact);
+          const uint32_t s_hi = scale_pair_chk(*reinterpret_cast<const uint16_t*>(qs + s_hi_off), inexact);
           const uint32_t wd[8] = {wa.x, wa.y, wa.z, wa.w, wb.x, wb.y, wb.z, wb.w};
 #pragma unroll
           for (int c = 0; c < 8; ++c) {
@@ -515,6 +420,8 @@ __global__ void __launch_bounds__(kThreads, 1)
       }
       if (!ok) break;
     }
+    if (__any_sync(0xFFFFFFFFu, inexact) && lane == 0) raise_status(a.status, TQP_STATUS_RANGE);
+    if (__any_sync(0xFFFFFFFFu, lora_inf) && lane == 0) raise_status(a.status, TQP_STATUS_NONFINITE);
   }
 
   tc_fence_before();
@@ -525,27 +432,15 @@ __global__ void __launch_bounds__(kThreads, 1)
   }
 }
 
-template <int MODE>
-static int launch(const GemmArgs& a, const Maps& mp, int units_upper, cudaStream_t s) {
-  static bool attr_set = false;
-  if (!attr_set) {
-    if (cudaFuncSetAttribute(expert_ffn_kernel<MODE>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                             int(smem_bytes<MODE>())) != cudaSuccess)
-      return TQP_ERR_CUDA;
-    attr_set = true;
-  }
-  const int grid = units_upper < num_sms() ? (units_upper > 0 ? units_upper : 1) : num_sms();
-  expert_ffn_kernel<MODE><<<grid, kThreads, smem_bytes<MODE>(), s>>>(a, mp.m[TQ0], mp.m[TQ1], mp.m[TS0],
-                                                                      mp.m[TS1], mp.m[TA]);
-  return cudaGetLastError() == cudaSuccess ? TQP_OK : TQP_ERR_CUDA;
-}
-
 }  // namespace tmem_ffn
 
-int run_expert_ffn(int mode, const GemmArgs& a, const Maps& mp, int units_upper, cudaStream_t s) {
-  if (mode == GATEUP) return tmem_ffn::launch<GATEUP>(a, mp, units_upper, s);
-  if (mode == DOWN) return tmem_ffn::launch<DOWN>(a, mp, units_upper, s);
-  return TQP_ERR_INVALID_ARG;
+int run_expert_gateup(const GemmArgs& a, const Maps& mp, int units_upper, cudaStream_t s) {
+  static DeviceFlags attr_done;
+  if (!attr_done.test_and_set_device(tmem_ffn::gateup_kernel, int(tmem_ffn::kSmemBytes))) return TQP_ERR_CUDA;
+  const int grid = units_upper < num_sms() ? (units_upper > 0 ? units_upper : 1) : num_sms();
+  tmem_ffn::gateup_kernel<<<grid, tmem_ffn::kThreads, tmem_ffn::kSmemBytes, s>>>(a, mp.m[TQ0], mp.m[TQ1], mp.m[TS0],
+                                                                               mp.m[TS1]);
+  return cudaGetLastError() == cudaSuccess ? TQP_OK : TQP_ERR_CUDA;
 }
 
 }  // namespace tqp

@@ -10,7 +10,7 @@
 
 namespace tqp {
 
-enum Mode : int { GATEUP = 0, DOWN = 1, LORA_XA = 2, LORA_HA = 3, ROUTER = 4, DH = 5, DX = 6 };
+enum Mode : int { GATEUP = 0, LORA_XA = 2, LORA_HA = 3, ROUTER = 4, DH = 5, DX = 6 };
 
 constexpr int kMBlock = 128;
 
@@ -48,6 +48,7 @@ struct GemmArgs {
   const uint16_t* lb1;     // DX: Au^T
   int lb_ld;
   const int4* unit_tab;    // expert kernels: decoded units {e, n-tile, rows, base}, one per unit
+  unsigned long long wait_ns;   // limit of one barrier wait (0: the default kWaitLimitNs)
 };
 
 struct Unit {
@@ -176,8 +177,15 @@ __device__ __forceinline__ uint32_t scale_pair(uint16_t sbits) {
   return sh | (sh << 16);
 }
 
-// One B-tile row (forward): NW int4 words (8 K values each) of row `brow`
-// starting at chunk part*NW, dequantised into the 128B-swizzled K-major tile.
+// As scale_pair, setting `inexact` when q * s is not exact in fp16 for every
+// int4 code q: a scale whose bf16 exponent is below -17 (bits under fp16's
+// subnormal spacing) or whose magnitude reaches 8192 (8 * s overflows), or inf/nan.
+__device__ __forceinline__ uint32_t scale_pair_chk(uint16_t sbits, bool& inexact) {
+  const uint32_t mag = sbits & 0x7FFFu;
+  inexact |= (mag != 0u) && ((mag >> 7) < 127u - 17u || mag >= 0x4600u);   // 0x4600 = 8192 in bf16
+  const uint32_t sh = bf16_to_f16_bits(sbits);
+  return sh | (sh << 16);
+}
 
 // Host side: the tensor maps handed to a grouped GEMM launch.
 struct Maps {
@@ -185,9 +193,9 @@ struct Maps {
 };
 enum { TQ0 = 0, TQ1 = 1, TS0 = 2, TS1 = 3, TA = 4, TB0 = 5, TB1 = 6 };
 
-// Forward expert projections with the dequantised weights held in tensor memory
-// (expert_ffn.cu): mode GATEUP or DOWN.
-int run_expert_ffn(int mode, const GemmArgs& a, const Maps& mp, int units_upper, cudaStream_t s);
+// Gate/up expert projection with the dequantised weights held in tensor memory
+// (expert_ffn.cu).
+int run_expert_gateup(const GemmArgs& a, const Maps& mp, int units_upper, cudaStream_t s);
 
 // Down projection with blocks of up to 256 routed rows (expert_down.cu).
 int run_expert_down_wide(const GemmArgs& a, const Maps& mp, int units_upper, cudaStream_t s);

@@ -1,15 +1,19 @@
 // Grouped tensor-core GEMM engine for the TQP MoE layer (sm_100a, tcgen05).
 //
-// One persistent, warp-specialised kernel template serves every contraction of
-// the layer ("Train low-rank adapters per expert" over "Quantize base expert
-// weights", Pattern 3; "Router: Full precision", TQP Quantization):
-//   GATEUP  : [G|U] = X_e [Wg|Wu]^T + s (X [Ag|Au]) [Bg|Bu],  H = silu(G) * U   (fp16)
-//   DOWN    : O = H_e Wd^T + s (H Ad) Bd                                          (fp16)
+// One persistent, warp-specialised kernel template serves the contractions of
+// the layer that do not run on the tensor-memory expert kernels (low-rank
+// adapters per expert over frozen quantised base weights: "Reversible Sparse
+// MoE Single Node", Pattern 3; full-precision router: TQP Quantization):
+//   GATEUP  : [G|U] = X_e [Wg|Wu]^T + s (X [Ag|Au]) [Bg|Bu],  H = silu(G) * U   (fp16;
+//             for hidden widths that are not a multiple of 128)
 //   LORA_XA : xa = s * X_e [Ag | Au]            (bf16 operands, fp16 out)
 //   LORA_HA : ha = s * H_e Ad                   (fp16)
 //   ROUTER  : logits = x W_r^T (+ bias), W_r split exactly into 3 bf16 parts
 //   DH      : dH = dO Wd + dhA Ad^T, with the SwiGLU backward in the epilogue
 //   DX      : dX = [dG|dU] [Wg;Wu] + dxa [Ag;Au]^T
+//             (the dgrads read the weight tile as an MN-major B operand: W is
+//             stored with the contraction index as its row, so the int4 rows are
+//             dequantised straight into the tile, no transpose)
 //
 // Work unit = (expert e, n-tile of up to 256 columns, m-block of up to 128
 // routed rows); one 128 x N x 64 tcgen05.mma step per K-block. Per CTA (1 per
@@ -20,8 +24,9 @@
 //   warps 6-9   A producer: TMA 128B-swizzled tiles for contiguous rows, or
 //               cp.async 16-byte row gathers (rows picked by perm_token); the
 //               rank-space (LoRA) A tiles; TMA B tiles of the rank-space GEMMs
-//   warps 10-17 B producer: int4 -> fp16 dequantisation (transposed for the
-//               dgrads) into 128B-swizzled K-major tiles, LoRA B^T tiles
+//   warps 10-17 B producer: int4 -> fp16 dequantisation into 128B-swizzled
+//               tiles (K-major for the forward, MN-major for the dgrads), the
+//               adapter factors of the rank-space stage
 // Accumulators are double-buffered in TMEM (2 x 256 fp32 columns), so the
 // epilogue of one unit overlaps the main loop of the next. The operand rings
 // (16 KB A tiles, B tiles, 9 KB code stages) share one 216 KB region whose
@@ -56,8 +61,8 @@ constexpr size_t kOperandBytes = size_t(kAStages) * kAStageBytes + size_t(kBStag
 //   their B ring also takes the code region and runs deeper: two TMA fills in
 //   flight cannot cover the L2/DRAM latency of a 4-MMA stage, and the A
 //   producer's TMA issuer waits on the same ring.
-// - Transposed dequantisation (dgrads): two producer groups of 128 threads take
-//   alternate stages (one stage's chain of code reads, dequant, transpose and
+// - Dequantisation for the dgrads (MN-major B tiles): two producer groups of 128
+//   threads take alternate stages (one stage's chain of code reads, dequant and
 //   stores is latency-bound), which needs a third B slot: 4 A, 3 B, 6 code stages.
 template <int MODE>
 struct Layout {
@@ -85,11 +90,21 @@ struct SmemCtl {
   uint64_t acc_empty[2];
   uint64_t drain;
   uint32_t tmem_base;
-  int abort_flag;
+  Abort ab;
 };
 
 constexpr size_t kSmemBytes = 1024 /*align slack*/ + kOperandBytes + sizeof(SmemCtl);
 static_assert(kSmemBytes <= 232448, "shared memory budget");
+
+// MN-major B tiles of the dgrads: 64 K rows x up to 256 features, as 64-feature
+// (128-byte) columns of 8-row, 1024-byte swizzle atoms; the columns are
+// kMnAtomBytes apart.
+constexpr uint32_t kMnAtomBytes = 64 * 128;
+
+// Byte offset of the 16-byte chunk of features [8J, 8J+8) of K row k.
+__device__ __forceinline__ uint32_t mn_tile_offset(int k, int J) {
+  return uint32_t((J >> 3) * kMnAtomBytes + (k >> 3) * 1024 + (k & 7) * 128 + (((J & 7) ^ (k & 7)) << 4));
+}
 
 
 // s_lo / s_hi: fp16 scale pairs of the first / second 32-wide group (equal when g >= 64).
@@ -117,9 +132,9 @@ __global__ void __launch_bounds__(kThreads, 1)
                         const __grid_constant__ CUtensorMap tq1, const __grid_constant__ CUtensorMap ts0,
                         const __grid_constant__ CUtensorMap ts1, const __grid_constant__ CUtensorMap ta,
                         const __grid_constant__ CUtensorMap tb0, const __grid_constant__ CUtensorMap tb1) {
-  constexpr bool kTrans = (MODE == DH || MODE == DX);      // B = W^T: dequantised transposed
-  constexpr bool kDequant = (MODE == GATEUP || MODE == DOWN || kTrans);
-  constexpr bool kATma = (MODE == DOWN || MODE == LORA_HA || MODE == ROUTER || kTrans);
+  constexpr bool kTrans = (MODE == DH || MODE == DX);      // dgrads: B = the weight tile, MN-major
+  constexpr bool kDequant = (MODE == GATEUP || kTrans);
+  constexpr bool kATma = (MODE == LORA_HA || MODE == ROUTER || kTrans);
   constexpr bool kBTma = (MODE == LORA_XA || MODE == LORA_HA || MODE == ROUTER);
   constexpr bool kBf16 = (MODE == LORA_XA || MODE == ROUTER);
   constexpr int kASt = Layout<MODE>::kA;
@@ -134,7 +149,7 @@ __global__ void __launch_bounds__(kThreads, 1)
   uint8_t* b_base = a_base + size_t(kASt) * kAStageBytes;
   uint8_t* q_base = b_base + size_t(kBSt) * kBStride;
   SmemCtl* ctl = reinterpret_cast<SmemCtl*>(smem + kOperandBytes);
-  volatile int* abort_flag = &ctl->abort_flag;
+  Abort* abort_flag = &ctl->ab;
 
   const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
@@ -160,7 +175,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       mbar_init(&ctl->acc_empty[i], 128);
     }
     mbar_init(&ctl->drain, 1);
-    ctl->abort_flag = 0;
+    abort_init(&ctl->ab, a.wait_ns);
     fence_barrier_init();
   }
   if (warp == 4) {
@@ -191,12 +206,13 @@ __global__ void __launch_bounds__(kThreads, 1)
   if (warp < 4) {
     // ------------------------------------------------------------ epilogue
     const int row = warp * 32 + lane;
+    uint32_t bad = 0;   // nonzero once an fp16 output of a valid row overflowed
     int it = 0;
     for (int u = blockIdx.x; u < nunits; u += gridDim.x, ++it) {
       const Unit un = decode_unit(a, sc, u);
       const int ab = it & 1;
       const uint32_t aph = uint32_t(it >> 1) & 1u;
-      if (!mbar_wait<128>(&ctl->acc_full[ab], aph, abort_flag, a.status)) break;
+      if (!__all_sync(0xFFFFFFFFu, mbar_wait<128>(&ctl->acc_full[ab], aph, abort_flag, a.status))) break;
       tc_fence_after();
       const bool valid = row < un.rows;
       const size_t grow = size_t(un.base) + row;
@@ -216,6 +232,7 @@ __global__ void __launch_bounds__(kThreads, 1)
             const float h0 = g0 / (1.0f + __expf(-g0)) * uv[2 * i];
             const float h1 = g1 / (1.0f + __expf(-g1)) * uv[2 * i + 1];
             pk[i] = pack_f16x2(h0, h1);
+            if (valid) bad |= f16x2_nonfinite(pk[i]);
           }
           if (valid) {
             uint4* dst = reinterpret_cast<uint4*>(hrow + c);
@@ -227,10 +244,16 @@ __global__ void __launch_bounds__(kThreads, 1)
               uint4* ua = reinterpret_cast<uint4*>(gr + a.f_dim);
 #pragma unroll
               for (int i = 0; i < 4; ++i) {
-                ga[i] = make_uint4(pack_f16x2(gv[8 * i], gv[8 * i + 1]), pack_f16x2(gv[8 * i + 2], gv[8 * i + 3]),
-                                   pack_f16x2(gv[8 * i + 4], gv[8 * i + 5]), pack_f16x2(gv[8 * i + 6], gv[8 * i + 7]));
-                ua[i] = make_uint4(pack_f16x2(uv[8 * i], uv[8 * i + 1]), pack_f16x2(uv[8 * i + 2], uv[8 * i + 3]),
-                                   pack_f16x2(uv[8 * i + 4], uv[8 * i + 5]), pack_f16x2(uv[8 * i + 6], uv[8 * i + 7]));
+                const uint4 gq = make_uint4(pack_f16x2(gv[8 * i], gv[8 * i + 1]), pack_f16x2(gv[8 * i + 2], gv[8 * i + 3]),
+                                            pack_f16x2(gv[8 * i + 4], gv[8 * i + 5]),
+                                            pack_f16x2(gv[8 * i + 6], gv[8 * i + 7]));
+                const uint4 uq = make_uint4(pack_f16x2(uv[8 * i], uv[8 * i + 1]), pack_f16x2(uv[8 * i + 2], uv[8 * i + 3]),
+                                            pack_f16x2(uv[8 * i + 4], uv[8 * i + 5]),
+                                            pack_f16x2(uv[8 * i + 6], uv[8 * i + 7]));
+                bad |= f16x2_nonfinite(gq.x) | f16x2_nonfinite(gq.y) | f16x2_nonfinite(gq.z) | f16x2_nonfinite(gq.w) |
+                       f16x2_nonfinite(uq.x) | f16x2_nonfinite(uq.y) | f16x2_nonfinite(uq.z) | f16x2_nonfinite(uq.w);
+                ga[i] = gq;
+                ua[i] = uq;
               }
             }
           }
@@ -266,6 +289,7 @@ __global__ void __launch_bounds__(kThreads, 1)
                 }
                 dg[t] = pack_f16x2(res_g[0], res_g[1]);
                 du[t] = pack_f16x2(res_u[0], res_u[1]);
+                bad |= f16x2_nonfinite(dg[t]) | f16x2_nonfinite(du[t]);
               }
               *reinterpret_cast<uint4*>(drow + c + 8 * q) = make_uint4(dg[0], dg[1], dg[2], dg[3]);
               *reinterpret_cast<uint4*>(drow + a.f_dim + c + 8 * q) = make_uint4(du[0], du[1], du[2], du[3]);
@@ -288,8 +312,8 @@ __global__ void __launch_bounds__(kThreads, 1)
           }
         }
       } else {
-        // DOWN / DX / LORA_XA / LORA_HA: fp16 output, optional scale
-        const float sc = (MODE == DOWN || MODE == DX) ? 1.0f : a.lora_scale;
+        // DX / LORA_XA / LORA_HA: fp16 output, optional scale
+        const float sc = (MODE == DX) ? 1.0f : a.lora_scale;
         uint16_t* orow = static_cast<uint16_t*>(a.out) + grow * a.out_ld + un.nt * a.ntile;
 #pragma unroll 1
         for (int c = 0; c < a.ntile; c += 32) {
@@ -300,6 +324,7 @@ __global__ void __launch_bounds__(kThreads, 1)
           for (int i = 0; i < 16; ++i) pk[i] = pack_f16x2(sc * v[2 * i], sc * v[2 * i + 1]);
           if (valid) {
             const int ncol = min(32, a.n_valid - (un.nt * a.ntile + c));
+            for (int i = 0; i < 16 && 2 * i < ncol; ++i) bad |= f16x2_nonfinite(pk[i]);
             uint4* dst = reinterpret_cast<uint4*>(orow + c);
             if (ncol >= 32) {
 #pragma unroll
@@ -313,13 +338,15 @@ __global__ void __launch_bounds__(kThreads, 1)
       tc_fence_before();
       mbar_arrive(&ctl->acc_empty[ab]);
     }
+    if (__any_sync(0xFFFFFFFFu, bad != 0) && lane == 0) raise_status(a.status, TQP_STATUS_NONFINITE);
   } else if (warp == 4) {
     // ------------------------------------------------------------ MMA issuer
     if (lane == 0) {
       Ring ra, rb;
       int it = 0;
       bool ok = true;
-      const uint32_t idesc = kBf16 ? idesc_bf16(128, a.ntile) : idesc_f16(128, a.ntile);
+      // dgrads: B (the weight tile) is MN-major, features contiguous
+      const uint32_t idesc = kBf16 ? idesc_bf16(128, a.ntile) : (kTrans ? idesc_f16_bmn(128, a.ntile) : idesc_f16(128, a.ntile));
       for (int u = blockIdx.x; u < nunits && ok; u += gridDim.x, ++it) {
         const int ab = it & 1;
         const uint32_t aph = uint32_t(it >> 1) & 1u;
@@ -338,9 +365,12 @@ __global__ void __launch_bounds__(kThreads, 1)
           tc_fence_after();
           const int ksteps = (kb < a.nkb_lora) ? (min(64, a.lora_k - kb * 64) + 15) / 16 : 4;
           const uint64_t adesc = sdesc_k_sw128(smem_u32(a_base + size_t(ra.stage) * kAStageBytes));
-          const uint64_t bdesc = sdesc_k_sw128(smem_u32(b_base + size_t(rb.stage) * kBStride));
+          const uint32_t bs = smem_u32(b_base + size_t(rb.stage) * kBStride);
+          const uint64_t bdesc = kTrans ? sdesc_mn_sw128(bs, kMnAtomBytes) : sdesc_k_sw128(bs);
+          // a K step of 16 advances a K-major tile by 32 B and an MN-major one by two 1024-byte atoms
+          const uint64_t bstep = kTrans ? uint64_t(2048 >> 4) : uint64_t(2);
           for (int kk = 0; kk < ksteps; ++kk)
-            umma_bf16(dt, adesc + uint64_t(2 * kk), bdesc + uint64_t(2 * kk), idesc, (kb > 0 || kk > 0) ? 1u : 0u);
+            umma_bf16(dt, adesc + uint64_t(2 * kk), bdesc + bstep * uint64_t(kk), idesc, (kb > 0 || kk > 0) ? 1u : 0u);
           umma_commit(&ctl->a_empty[ra.stage]);
           umma_commit(&ctl->b_empty[rb.stage]);
           ra.next<kASt>();
@@ -349,9 +379,10 @@ __global__ void __launch_bounds__(kThreads, 1)
         if (!ok) break;
         umma_commit(&ctl->acc_full[ab]);
       }
-      // make sure no MMA is still writing TMEM before teardown
+      // no MMA may still read or write TMEM when it is freed: wait for all of
+      // them (they run to completion whether or not the CTA aborted)
       umma_commit(&ctl->drain);
-      mbar_wait(&ctl->drain, 0, abort_flag, a.status);
+      mbar_drain(&ctl->drain, 0, 100000000ull);
     }
     __syncwarp();
   } else if (warp == 5) {
@@ -359,14 +390,12 @@ __global__ void __launch_bounds__(kThreads, 1)
     if (kDequant && lane == 0) {
       Ring q;
       // forward: per n-tile rows of W [rows][64 K]: codes rows*32 B, scales [ngrp][rows] bf16
-      // dgrad:   transposed tile [64 K][ntile N]: codes 64*ntile/2 B, scales [ngn][64] bf16
+      // dgrad:   tile [64 K rows][ntile N]: codes 64*ntile/2 B, scales [ngn][64] bf16
       const int ngrp = kTrans ? (a.g >= a.ntile ? 1 : a.ntile / a.g) : (a.g >= 64 ? 1 : 64 / a.g);
       const uint32_t bytes = uint32_t(a.ntile) * 32u + uint32_t(kTrans ? 128 * ngrp : a.ntile * ngrp * 2);
       const int rows_box = (MODE == GATEUP) ? (a.ntile >> 1) : a.ntile;
       const int gpe = a.in_dim / a.g;  // scale rows per expert
-      int issued = 0;
-      uint32_t last_phase = 0;
-      int last_stage = 0;
+      PendingFills pend;
       for (int u = blockIdx.x; u < nunits; u += gridDim.x) {
         const Unit un = decode_unit(a, sc, u);
         bool ok = true;
@@ -391,15 +420,13 @@ __global__ void __launch_bounds__(kThreads, 1)
               tma_load_2d(smem_u32(qs + a.ntile * 32 + ngrp * rows_box * 2), &ts1, bar, un.nt * rows_box, srow);
             }
           }
-          ++issued;
-          last_stage = q.stage;
-          last_phase = q.phase;
+          pend.issued(q.stage, q.phase);
           q.next<kQSt>();
         }
         if (!ok) break;
       }
-      // drain: wait until the last issued stage has landed (bounded)
-      if (issued > 0 && *abort_flag) mbar_drain(&ctl->q_full[last_stage], last_phase);
+      // on an abort, wait (bounded) until every issued fill has landed
+      if (aborted(abort_flag)) pend.drain(ctl->q_full);
     }
   } else if (warp < 10) {
     // ------------------------------------------------------------ A producer
@@ -415,8 +442,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     if (MODE == LORA_XA) b_bytes = uint32_t(2 * a.r * 128);
     if (MODE == LORA_HA) b_bytes = uint32_t(a.r * 128);
     if (MODE == ROUTER) b_bytes = uint32_t(a.ntile * 128);
-    int pend_stage = -1, pend_b_stage = -1;
-    uint32_t pend_phase = 0, pend_b_phase = 0;
+    PendingFills pend_a, pend_b;
     for (int u = blockIdx.x; u < nunits; u += gridDim.x) {
       const Unit un = decode_unit(a, sc, u);
       int srow[8];   // gathered source rows of this thread's 8 tile rows
@@ -451,8 +477,7 @@ __global__ void __launch_bounds__(kThreads, 1)
             uint64_t* bfull = &ctl->b_full[rb.stage];
             const uint32_t bst_u = smem_u32(b_base + size_t(rb.stage) * kBStride);
             mbar_arrive_expect_tx(bfull, b_bytes);
-            pend_b_stage = rb.stage;
-            pend_b_phase = rb.phase;
+            pend_b.issued(rb.stage, rb.phase);
             if (MODE == LORA_XA) {
               tma_load_2d(bst_u, &tb0, bfull, kcol, un.e * a.r);
               tma_load_2d(bst_u + a.r * 128, &tb1, bfull, kcol, un.e * a.r);
@@ -467,8 +492,7 @@ __global__ void __launch_bounds__(kThreads, 1)
             if (tid == 0) {
               mbar_arrive_expect_tx(full, a_bytes);
               tma_load_2d(st_u, &ta, full, kcol, un.base);
-              pend_stage = ra.stage;
-              pend_phase = ra.phase;
+              pend_a.issued(ra.stage, ra.phase);
             } else {
               mbar_arrive(full);
             }
@@ -488,9 +512,11 @@ __global__ void __launch_bounds__(kThreads, 1)
       if (!ok) break;
     }
     cp_async_wait_all();
-    // on an abort, wait (bounded) for the last TMA fill issued by this thread
-    if (tid == 0 && *abort_flag && pend_stage >= 0) mbar_drain(&ctl->a_full[pend_stage], pend_phase);
-    if (tid == 0 && *abort_flag && pend_b_stage >= 0) mbar_drain(&ctl->b_full[pend_b_stage], pend_b_phase);
+    // on an abort, wait (bounded) for every TMA fill issued by this thread
+    if (tid == 0 && aborted(abort_flag)) {
+      pend_a.drain(ctl->a_full);
+      pend_b.drain(ctl->b_full);
+    }
   } else {
     // ------------------------------------------------------------ B producer
     const int tid = threadIdx.x - 10 * 32;  // 0..255
@@ -498,11 +524,13 @@ __global__ void __launch_bounds__(kThreads, 1)
     const int brow = tid / tpr;                              // B row (forward tiles)
     const int part = tid % tpr;
     const int nwords = tpr >= 8 ? 1 : 8 / tpr;               // int4 words (8 K values each) per thread
-    // transposed modes: two groups of 128 threads take alternate stages
+    // dgrad modes: two groups of 128 threads take alternate stages
     const int grp = kBGroups > 1 ? tid >> 7 : 0;
     const int gtid = kBGroups > 1 ? tid & 127 : tid;
     constexpr int kGT = 256 / kBGroups;                      // threads per group
     Ring rb, q;
+    bool inexact = false;   // a group scale whose products q * s are not exact in fp16
+    bool lora_inf = false;  // an adapter value beyond the fp16 range
     int n = 0;                                               // stage counter over all units
     for (int u = blockIdx.x; u < nunits; u += gridDim.x) {
       const Unit un = decode_unit(a, sc, u);
@@ -519,7 +547,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         uint8_t* bst = b_base + size_t(rb.stage) * kBStride;
         uint64_t* full = &ctl->b_full[rb.stage];
         if (kb < a.nkb_lora) {
-          if (MODE == GATEUP || MODE == DOWN) {
+          if (MODE == GATEUP) {
             // rank-space B^T rows as fp16, K' columns [kb*64, kb*64+64); gate rows hold
             // Bg^T in [0, r), up rows hold Bu^T in [r, 2r) (block-diagonal)
             if (brow < a.ntile) {
@@ -528,44 +556,31 @@ __global__ void __launch_bounds__(kThreads, 1)
                 const int c = part * nwords + i;
                 const int col = kb * 64 + c * 8;
                 uint4 v = make_uint4(0, 0, 0, 0);
-                if (MODE == GATEUP) {
-                  const bool gate = brow < half;
-                  const int n = un.nt * half + (gate ? brow : brow - half);
-                  const int cc = gate ? col : col - a.r;
-                  if (cc >= 0 && cc < a.r)
-                    v = __ldg(reinterpret_cast<const uint4*>((gate ? a.b0 : a.b1) + (size_t(un.e) * a.out_dim + n) * a.r +
-                                                             cc));
-                } else {
-                  const int n = un.nt * a.ntile + brow;
-                  if (col < a.r)
-                    v = __ldg(reinterpret_cast<const uint4*>(a.b0 + (size_t(un.e) * a.out_dim + n) * a.r + col));
-                }
-                *reinterpret_cast<uint4*>(bst + sw128_offset(brow, c)) = bf16x8_to_f16x8(v);
+                const bool gate = brow < half;
+                const int n = un.nt * half + (gate ? brow : brow - half);
+                const int cc = gate ? col : col - a.r;
+                if (cc >= 0 && cc < a.r)
+                  v = __ldg(reinterpret_cast<const uint4*>((gate ? a.b0 : a.b1) + (size_t(un.e) * a.out_dim + n) * a.r +
+                                                           cc));
+                *reinterpret_cast<uint4*>(bst + sw128_offset(brow, c)) = bf16x8_to_f16x8_chk(v, lora_inf);
               }
             }
           } else if (kTrans) {
-            // dgrad rank-space step: B[n][rr] = A^T[rr][n0 + n] (bf16, read transposed) as fp16
-            for (int nrow = gtid; nrow < a.ntile; nrow += kGT) {
-              const int n = un.nt * a.ntile + nrow;
-#pragma unroll 1
-              for (int c = 0; c < 8; ++c) {
-                uint32_t pk[4];
-#pragma unroll
-                for (int t = 0; t < 4; ++t) {
-                  float vv[2];
-#pragma unroll
-                  for (int hh = 0; hh < 2; ++hh) {
-                    const int rr = kb * 64 + c * 8 + 2 * t + hh;
-                    float val = 0.0f;
-                    if (rr < a.r) val = bf16_to_f32(__ldg(a.lb0 + (size_t(un.e) * a.r + rr) * a.lb_ld + n));
-                    else if (MODE == DX && rr < 2 * a.r)
-                      val = bf16_to_f32(__ldg(a.lb1 + (size_t(un.e) * a.r + (rr - a.r)) * a.lb_ld + n));
-                    vv[hh] = val;
-                  }
-                  pk[t] = pack_f16x2(vv[0], vv[1]);
-                }
-                *reinterpret_cast<uint4*>(bst + sw128_offset(nrow, c)) = make_uint4(pk[0], pk[1], pk[2], pk[3]);
-              }
+            // dgrad rank-space step, MN-major: B row rr (the K index) = A^T[rr][n0 ..
+            // n0 + ntile) of the adapter (stored [r][features], bf16 -> fp16); rows
+            // past lora_k are zero. Thread gtid: row gtid / 2, half gtid % 2 of the row.
+            const int rr = kb * 64 + (gtid >> 1);
+            const int half = gtid & 1;
+            const int cpt = a.ntile >> 4;                      // 16-byte chunks per half row
+            const uint16_t* src = nullptr;
+            if (rr < a.r) src = a.lb0 + (size_t(un.e) * a.r + rr) * a.lb_ld;
+            else if (MODE == DX && rr < 2 * a.r) src = a.lb1 + (size_t(un.e) * a.r + (rr - a.r)) * a.lb_ld;
+            for (int j = 0; j < cpt; ++j) {
+              const int J = half * cpt + j;                    // chunk of 8 features within the tile
+              uint4 v = make_uint4(0, 0, 0, 0);
+              if (src) v = bf16x8_to_f16x8_chk(__ldg(reinterpret_cast<const uint4*>(src + un.nt * a.ntile + J * 8)),
+                                               lora_inf);
+              *reinterpret_cast<uint4*>(bst + mn_tile_offset(gtid >> 1, J)) = v;
             }
           }
           fence_proxy_async_smem();
@@ -573,29 +588,28 @@ __global__ void __launch_bounds__(kThreads, 1)
         } else if (kTrans) {
           if (!mbar_wait(&ctl->q_full[q.stage], q.phase, abort_flag, a.status)) { ok = false; break; }
           const uint8_t* qs = q_base + size_t(q.stage) * kQStageBytes;
-          // thread = 4 K rows (kq) x 8-column octets no, no + 8, ... of the tile
-          const int kq = gtid >> 3, no = gtid & 7;
+          // The code tile holds W rows n (the K index) with the tile's ntile
+          // features contiguous: exactly the MN-major operand, so each thread
+          // dequantises half a row (8 features per int4 word) straight into it.
+          // Thread gtid: row gtid / 2, half gtid % 2.
+          const int k = gtid >> 1, half = gtid & 1;
           const int n0 = un.nt * a.ntile;
           const int rowb = a.ntile >> 1;                     // bytes per code row
+          const int wph = a.ntile >> 4;                      // words per half row (16 or 8)
           const uint16_t* sc = reinterpret_cast<const uint16_t*>(qs + a.ntile * 32);
-          for (int hb = 0; hb < a.ntile; hb += 64) {
-            const int oct = (hb >> 3) + no;                  // N octet of this thread
-            const int gi = (n0 + oct * 8) / a.g - n0 / a.g;
-            uint32_t hv[4][4];
+          for (int j4 = 0; j4 < wph; j4 += 4) {
+            const int J = half * wph + j4;                   // first word of this 16-byte code chunk
+            const int cc = J >> 2;                           // code chunk within the row
+            // 128-byte rows come 128B-swizzled (conflict-free reads); 64-byte rows plain
+            const int pos = (rowb == 128) ? (cc ^ (k & 7)) : cc;
+            const uint4 w4 = *reinterpret_cast<const uint4*>(qs + k * rowb + pos * 16);
+            const uint32_t wv[4] = {w4.x, w4.y, w4.z, w4.w};
 #pragma unroll
-            for (int r = 0; r < 4; ++r) {
-              const int k = kq * 4 + r;
-              const uint32_t wv = *reinterpret_cast<const uint32_t*>(qs + k * rowb + oct * 4);
-              const uint4 d4 = dequant_word(wv, scale_pair(sc[gi * 64 + k]));
-              hv[r][0] = d4.x; hv[r][1] = d4.y; hv[r][2] = d4.z; hv[r][3] = d4.w;
-            }
-#pragma unroll
-            for (int nn = 0; nn < 8; ++nn) {
-              const uint32_t sel = (nn & 1) ? 0x7632u : 0x5410u;
-              const uint32_t p01 = __byte_perm(hv[0][nn >> 1], hv[1][nn >> 1], sel);
-              const uint32_t p23 = __byte_perm(hv[2][nn >> 1], hv[3][nn >> 1], sel);
-              *reinterpret_cast<uint2*>(bst + sw128_offset(oct * 8 + nn, kq >> 1) + (kq & 1) * 8) =
-                  make_uint2(p01, p23);
+            for (int i = 0; i < 4; ++i) {
+              const int Jw = J + i;                          // word = features n0 + 8 Jw .. + 7
+              const int gi = (n0 + Jw * 8) / a.g - n0 / a.g;
+              *reinterpret_cast<uint4*>(bst + mn_tile_offset(k, Jw)) =
+                  dequant_word(wv[i], scale_pair_chk(sc[gi * 64 + k], inexact));
             }
           }
           // hand the code slot back only after its values were consumed, behind a
@@ -613,8 +627,8 @@ __global__ void __launch_bounds__(kThreads, 1)
           const int ngrp = a.g >= 64 ? 1 : 64 / a.g;
           const int sidx = (MODE == GATEUP) ? (brow / half) * ngrp * half + (brow % half) : brow;
           const int sstride = (MODE == GATEUP) ? half : a.ntile;
-          const uint32_t s_lo = scale_pair(sc[sidx]);
-          const uint32_t s_hi = (a.g == 32) ? scale_pair(sc[sidx + sstride]) : s_lo;
+          const uint32_t s_lo = scale_pair_chk(sc[sidx], inexact);
+          const uint32_t s_hi = (a.g == 32) ? scale_pair_chk(sc[sidx + sstride], inexact) : s_lo;
           if (nwords == 8) dequant_row<8>(qs, bst, brow, part, s_lo, s_hi);
           else dequant_row<4>(qs, bst, brow, part, s_lo, s_hi);
           fence_proxy_async_smem();
@@ -628,6 +642,8 @@ __global__ void __launch_bounds__(kThreads, 1)
       }
       if (!ok) break;
     }
+    if (__any_sync(0xFFFFFFFFu, inexact) && lane == 0) raise_status(a.status, TQP_STATUS_RANGE);
+    if (__any_sync(0xFFFFFFFFu, lora_inf) && lane == 0) raise_status(a.status, TQP_STATUS_NONFINITE);
   }
 
   tc_fence_before();
@@ -702,8 +718,8 @@ __global__ void unit_table_kernel(const int32_t* __restrict__ offsets, const int
   tab[u] = make_int4(lo, nt, min(block, cnt - mb * block), o0 + mb * block);
 }
 
-// bf16 -> fp16, 8 values per thread; values beyond the fp16 range raise
-// TQP_STATUS_NONFINITE (status may be null).
+// bf16 -> fp16, 8 values per thread; values beyond the fp16 range (x, or a
+// LoRA factor) raise TQP_STATUS_NONFINITE (status may be null).
 __global__ void to_f16_kernel(const uint16_t* __restrict__ x, uint16_t* __restrict__ x16, size_t n8,
                               int32_t* status) {
   const size_t i = size_t(blockIdx.x) * blockDim.x + threadIdx.x;
@@ -788,14 +804,10 @@ int num_sms() {
 
 
 template <int MODE>
-static int run_gemm(const GemmArgs& a, const Maps& mp, int units_upper, cudaStream_t s) {
-  static bool attr_set = false;
-  if (!attr_set) {
-    if (cudaFuncSetAttribute(grouped_gemm_kernel<MODE>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                             int(kSmemBytes)) != cudaSuccess)
-      return TQP_ERR_CUDA;
-    attr_set = true;
-  }
+static int run_gemm(GemmArgs a, const Maps& mp, int units_upper, cudaStream_t s) {
+  static DeviceFlags attr_done;
+  if (!attr_done.test_and_set_device(grouped_gemm_kernel<MODE>, int(kSmemBytes))) return TQP_ERR_CUDA;
+  a.wait_ns = wait_limit_ns();
   const int grid = units_upper < num_sms() ? (units_upper > 0 ? units_upper : 1) : num_sms();
   grouped_gemm_kernel<MODE><<<grid, kThreads, kSmemBytes, s>>>(a, mp.m[0], mp.m[1], mp.m[2], mp.m[3], mp.m[4],
                                                                 mp.m[5], mp.m[6]);
@@ -912,7 +924,7 @@ int launch_grouped_ffn_part(int part, const uint16_t* x, int T, const int32_t* o
     schedule_kernel<<<1, 1024, 0, s>>>(offsets, w->E, fb.mb_prefix256, 256);
     if (cudaGetLastError() != cudaSuccess) return TQP_ERR_CUDA;
     if ((rc = to_f16(x, fb.x16, size_t(T) * d, status, s)) != TQP_OK) return rc;
-    if (r > 0 && (rc = to_f16(w->lora_a[2], fb.adT16, size_t(w->E) * r * f, nullptr, s)) != TQP_OK) return rc;
+    if (r > 0 && (rc = to_f16(w->lora_a[2], fb.adT16, size_t(w->E) * r * f, status, s)) != TQP_OK) return rc;
   }
   // an upper bound on the number of work units (grid sizing only)
   const int mb_upper = int((A + kMBlock - 1) / kMBlock) + w->E;
@@ -985,8 +997,8 @@ int launch_grouped_ffn_part(int part, const uint16_t* x, int T, const int32_t* o
       if ((rc = build_unit_table(a, kMBlock, mb_upper * a.n_tiles, fb.unit_tab, s)) != TQP_OK) return rc;
       a.unit_tab = fb.unit_tab;
     }
-    rc = tm ? run_expert_ffn(GATEUP, a, mp, mb_upper * a.n_tiles, s)
-            : run_gemm<GATEUP>(a, mp, mb_upper * a.n_tiles, s);
+    a.wait_ns = wait_limit_ns();
+    rc = tm ? run_expert_gateup(a, mp, mb_upper * a.n_tiles, s) : run_gemm<GATEUP>(a, mp, mb_upper * a.n_tiles, s);
     if (rc != TQP_OK) return rc;
   }
   if (part == 2 && r > 0) {  // ha = s * H Ad
@@ -1030,6 +1042,7 @@ int launch_grouped_ffn_part(int part, const uint16_t* x, int T, const int32_t* o
     const int units_upper = int((A + 255) / 256 + w->E) * a.n_tiles;
     if ((rc = build_unit_table(a, 256, units_upper, fb.unit_tab, s)) != TQP_OK) return rc;
     a.unit_tab = fb.unit_tab;
+    a.wait_ns = wait_limit_ns();
     if ((rc = run_expert_down_wide(a, mp, units_upper, s)) != TQP_OK) return rc;
   }
   return TQP_OK;
@@ -1047,7 +1060,7 @@ int launch_grouped_ffn(const uint16_t* x, int T, const int32_t* offsets, const i
 
 // dH = dO Wd + dhA Ad^T (SwiGLU backward fused: writes dG | dU) or
 // dX = [dG | dU] [Wg ; Wu] + dxa [Ag^T ; Au^T]^T, per expert, on the tensor cores
-// with the int4 base dequantised transposed in shared memory.
+// with the int4 base dequantised into MN-major shared-memory tiles.
 // K-major fp16 copy of a backward rank-space B operand, [E][n][K], one block
 // per (64-wide K slice, expert):
 //   which 0: Bd, stored B^T [E][d][r]  ->  [E][r][d]             (n = r,  K = d)
@@ -1143,7 +1156,7 @@ int launch_dgrad(int which, const uint16_t* a_src, const uint16_t* a_lora, const
     a.n_valid = f;
     bool ok = make_tile_map(&mp.m[TA], a_src, uint64_t(A), uint64_t(d), 128) &&
               make_map(&mp.m[TQ0], CU_TENSOR_MAP_DATA_TYPE_UINT8, w->wq[2], f / 2, uint64_t(w->E) * d, f / 2,
-                       uint32_t(a.ntile / 2), 64) &&
+                       uint32_t(a.ntile / 2), 64, a.ntile == 256 ? 128 : 0) &&
               make_map(&mp.m[TS0], CU_TENSOR_MAP_DATA_TYPE_UINT16, w->wscale[2], d, uint64_t(w->E) * (f / w->group),
                        uint64_t(d) * 2, 64, ngn);
     if (!ok) return TQP_ERR_CUDA;
@@ -1167,9 +1180,9 @@ int launch_dgrad(int which, const uint16_t* a_src, const uint16_t* a_lora, const
   a.n_valid = d;
   bool ok = make_tile_map(&mp.m[TA], a_src, uint64_t(A), uint64_t(2 * f), 128) &&
             make_map(&mp.m[TQ0], CU_TENSOR_MAP_DATA_TYPE_UINT8, w->wq[0], d / 2, uint64_t(w->E) * f, d / 2,
-                     uint32_t(a.ntile / 2), 64) &&
+                     uint32_t(a.ntile / 2), 64, a.ntile == 256 ? 128 : 0) &&
             make_map(&mp.m[TQ1], CU_TENSOR_MAP_DATA_TYPE_UINT8, w->wq[1], d / 2, uint64_t(w->E) * f, d / 2,
-                     uint32_t(a.ntile / 2), 64) &&
+                     uint32_t(a.ntile / 2), 64, a.ntile == 256 ? 128 : 0) &&
             make_map(&mp.m[TS0], CU_TENSOR_MAP_DATA_TYPE_UINT16, w->wscale[0], f, uint64_t(w->E) * (d / w->group),
                      uint64_t(f) * 2, 64, ngn) &&
             make_map(&mp.m[TS1], CU_TENSOR_MAP_DATA_TYPE_UINT16, w->wscale[1], f, uint64_t(w->E) * (d / w->group),

@@ -1,11 +1,15 @@
-// Backward of the TQP MoE layer: adapters only, base and router frozen
-// ("Base expert weights: Quantized (fixed)", "Optimizer state only on adapters",
-// Principle 3 / Pattern 3 of "Reversible Sparse MoE Single Node").
+// Backward of the TQP MoE layer: adapters only, with the quantised base weights
+// and the router frozen (TQP Quantization; Principle 3 / Pattern 3 of
+// "Reversible Sparse MoE Single Node" keep optimizer state on the adapters).
 //
 // The dense dgrad contractions and the rank-space products dhA = s dO Bd^T and
 // dxa = s [dG|dU] [Bg|Bu]^T run on the tensor cores (launch_dgrad and
 // launch_rank_bwd in grouped_gemm.cu). This file holds the rest:
-//   bwd_combine  : dO = gamma * dy (fp16, permuted rows), dgamma = <dy, O>, the
+//   absmax       : max|dy|, from which every fp16 intermediate is computed for
+//                  dy * 2^P (P chosen so that dO peaks near 2^8) and the fp32
+//                  gradients are scaled back by 2^-P, so that the fp16 path
+//                  neither underflows nor overflows whatever the size of dy
+//   bwd_combine  : dO = gamma * dy * 2^P (fp16, permuted rows), dgamma = <dy, O>, the
 //                  softmax-over-chosen backward dl = gamma (dgamma - sum gamma dgamma)
 //                  and the frozen router's input gradient sum_j dl_j W_r[id_j]
 //   outer        : per-expert adapter gradients, sums over the expert's routed rows
@@ -32,6 +36,33 @@ int launch_add_f32(const float* a, const float* b, float* out, size_t n, cudaStr
 }
 
 // ----------------------------------------------------------------------------
+// cotangent scale
+// ----------------------------------------------------------------------------
+
+// dmax = max |dy| as the bits of a non-negative float (ordered like unsigned
+// integers), by atomicMax; dmax must be zeroed first.
+__global__ void __launch_bounds__(256) absmax_kernel(const float* __restrict__ x, size_t n4, uint32_t* dmax) {
+  uint32_t m = 0;
+  for (size_t i = size_t(blockIdx.x) * blockDim.x + threadIdx.x; i < n4; i += size_t(gridDim.x) * blockDim.x) {
+    const float4 v = __ldg(reinterpret_cast<const float4*>(x) + i);
+    m = max(m, max(max(__float_as_uint(fabsf(v.x)), __float_as_uint(fabsf(v.y))),
+                   max(__float_as_uint(fabsf(v.z)), __float_as_uint(fabsf(v.w)))));
+  }
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) m = max(m, __shfl_xor_sync(0xFFFFFFFFu, m, o));
+  if ((threadIdx.x & 31) == 0 && m) atomicMax(dmax, m);
+}
+
+// 2^P with max|dy| * 2^P in [2^7, 2^8); 1 when dy is all zeros or not finite.
+__device__ __forceinline__ float grad_scale(const uint32_t* dmax) {
+  const float m = __uint_as_float(*dmax);
+  if (!(m > 0.0f) || !isfinite(m)) return 1.0f;
+  int e;
+  frexpf(m, &e);   // m = f * 2^e, 0.5 <= f < 1
+  return ldexpf(1.0f, max(-120, min(120, 8 - e)));
+}
+
+// ----------------------------------------------------------------------------
 // combine backward + softmax-gate backward + router input gradient
 // ----------------------------------------------------------------------------
 
@@ -42,10 +73,13 @@ __global__ void __launch_bounds__(256) bwd_combine_kernel(const uint16_t* __rest
                                                           const int32_t* __restrict__ ids,
                                                           const float* __restrict__ router_w,
                                                           const float* __restrict__ dy, int T, int k, int d,
-                                                          uint16_t* __restrict__ dO, float* __restrict__ dx) {
+                                                          const uint32_t* __restrict__ dmax, uint16_t* __restrict__ dO,
+                                                          float* __restrict__ dx, int32_t* status) {
   __shared__ float red[8][kMaxK];
   __shared__ float dl_s[kMaxK];
   const int t = blockIdx.x;
+  const float gsc = grad_scale(dmax);
+  uint32_t bad = 0;
   const int lane = threadIdx.x & 31, wid = threadIdx.x >> 5;
   const int nwarps = blockDim.x >> 5;
   float part[kMaxK];
@@ -59,7 +93,7 @@ __global__ void __launch_bounds__(256) bwd_combine_kernel(const uint16_t* __rest
     for (int j = 0; j < kMaxK; ++j) {
       if (j >= k) break;
       const int row = inv[size_t(t) * k + j];
-      const float g = gates[size_t(t) * k + j];
+      const float g = gates[size_t(t) * k + j] * gsc;
       const uint4 ov = *reinterpret_cast<const uint4*>(O + size_t(row) * d + c);
       const uint32_t ow[4] = {ov.x, ov.y, ov.z, ov.w};
       float acc = 0.0f;
@@ -69,11 +103,13 @@ __global__ void __launch_bounds__(256) bwd_combine_kernel(const uint16_t* __rest
         acc = fmaf(dv[2 * q], f16_to_f32(uint16_t(ow[q] & 0xFFFFu)), acc);
         acc = fmaf(dv[2 * q + 1], f16_to_f32(uint16_t(ow[q] >> 16)), acc);
         pk[q] = pack_f16x2(g * dv[2 * q], g * dv[2 * q + 1]);
+        bad |= f16x2_nonfinite(pk[q]);
       }
       part[j] += acc;
       *reinterpret_cast<uint4*>(dO + size_t(row) * d + c) = make_uint4(pk[0], pk[1], pk[2], pk[3]);
     }
   }
+  if (__any_sync(0xFFFFFFFFu, bad != 0) && lane == 0) raise_status(status, TQP_STATUS_NONFINITE);
   // dgamma_j = sum over the row: warp then block reduction
 #pragma unroll
   for (int j = 0; j < kMaxK; ++j) {
@@ -117,14 +153,17 @@ __global__ void __launch_bounds__(256) bwd_combine_kernel(const uint16_t* __rest
   }
 }
 
-// dx[t] += sum_j dX[inv[t*k + j]]  (fp16 rows, fp32 accumulation, fixed j order)
+// dx[t] += 2^-P sum_j dX[inv[t*k + j]]  (fp16 rows computed for dy * 2^P, fp32
+// accumulation, fixed j order)
 __global__ void __launch_bounds__(256) gather_add_kernel(const uint16_t* __restrict__ dX, const int32_t* __restrict__ inv,
-                                                         int T, int k, int d, float* __restrict__ dx) {
+                                                         int T, int k, int d, const uint32_t* __restrict__ dmax,
+                                                         float* __restrict__ dx) {
   const int t = blockIdx.x;
+  const float inv_sc = 1.0f / grad_scale(dmax);   // a power of two: exact
   for (int c = threadIdx.x * 8; c < d; c += blockDim.x * 8) {
     float4* xp = reinterpret_cast<float4*>(dx + size_t(t) * d + c);
     const float4 b0 = xp[0], b1 = xp[1];
-    float acc[8] = {b0.x, b0.y, b0.z, b0.w, b1.x, b1.y, b1.z, b1.w};
+    float acc[8] = {0.0f, 0.0f, 0.0f, 0.0f, 0.0f, 0.0f, 0.0f, 0.0f};
     for (int j = 0; j < k; ++j) {
       const int row = inv[size_t(t) * k + j];
       const uint4 v = *reinterpret_cast<const uint4*>(dX + size_t(row) * d + c);
@@ -135,8 +174,10 @@ __global__ void __launch_bounds__(256) gather_add_kernel(const uint16_t* __restr
         acc[2 * q + 1] += f16_to_f32(uint16_t(w[q] >> 16));
       }
     }
-    xp[0] = make_float4(acc[0], acc[1], acc[2], acc[3]);
-    xp[1] = make_float4(acc[4], acc[5], acc[6], acc[7]);
+    xp[0] = make_float4(fmaf(acc[0], inv_sc, b0.x), fmaf(acc[1], inv_sc, b0.y), fmaf(acc[2], inv_sc, b0.z),
+                        fmaf(acc[3], inv_sc, b0.w));
+    xp[1] = make_float4(fmaf(acc[4], inv_sc, b1.x), fmaf(acc[5], inv_sc, b1.y), fmaf(acc[6], inv_sc, b1.z),
+                        fmaf(acc[7], inv_sc, b1.w));
   }
 }
 
@@ -153,6 +194,7 @@ struct OuterArgs {
   const uint16_t* Q;
   int ldq, offq;
   float* C;                  // fp32 [E][M][N]
+  const uint32_t* dmax;      // the cotangent's max |dy|: C is scaled back by 2^-P
 };
 
 // One block computes a TM x TN tile of C[e] (TM x TN = 4096, 4 x 4 per thread)
@@ -217,6 +259,7 @@ __global__ void __launch_bounds__(256) outer_kernel(const OuterArgs a) {
         for (int j = 0; j < 4; ++j) acc[i][j] = fmaf(p4[i], q4[j], acc[i][j]);
     }
   }
+  const float inv_sc = 1.0f / grad_scale(a.dmax);   // a power of two: exact
 #pragma unroll
   for (int i = 0; i < 4; ++i) {
     const int m = m0 + ty * 4 + i;
@@ -224,7 +267,7 @@ __global__ void __launch_bounds__(256) outer_kernel(const OuterArgs a) {
 #pragma unroll
     for (int j = 0; j < 4; ++j) {
       const int n = n0 + tx * 4 + j;
-      if (n < a.N) a.C[(size_t(e) * a.M + m) * a.N + n] = acc[i][j];
+      if (n < a.N) a.C[(size_t(e) * a.M + m) * a.N + n] = acc[i][j] * inv_sc;
     }
   }
 }
@@ -233,26 +276,38 @@ __global__ void __launch_bounds__(256) outer_kernel(const OuterArgs a) {
 // host launchers
 // ----------------------------------------------------------------------------
 
-int launch_bwd_combine(const uint16_t* O, const int32_t* inv, const float* gates, const int32_t* ids,
-                       const float* router_w, const float* dy, int T, int k, int d, uint16_t* dO, float* dx,
-                       cudaStream_t s) {
-  if (T == 0) return TQP_OK;
-  // at least one full warp: the row reductions use full-mask warp shuffles
-  const int threads = d / 8 < 32 ? 32 : (d / 8 < 256 ? d / 8 : 256);
-  bwd_combine_kernel<<<T, threads, 0, s>>>(O, inv, gates, ids, router_w, dy, T, k, d, dO, dx);
+int launch_grad_absmax(const float* dy, size_t n, uint32_t* dmax, cudaStream_t s) {
+  if (cudaMemsetAsync(dmax, 0, sizeof(uint32_t), s) != cudaSuccess) return TQP_ERR_CUDA;
+  const size_t n4 = n / 4;
+  if (n4 == 0) return TQP_OK;
+  const size_t blocks = (n4 + 255) / 256;
+  const int grid = int(blocks < size_t(4 * num_sms()) ? blocks : size_t(4 * num_sms()));
+  absmax_kernel<<<grid, 256, 0, s>>>(dy, n4, dmax);
   return cudaGetLastError() == cudaSuccess ? TQP_OK : TQP_ERR_CUDA;
 }
 
-int launch_gather_add(const uint16_t* dX, const int32_t* inv, int T, int k, int d, float* dx, cudaStream_t s) {
+int launch_bwd_combine(const uint16_t* O, const int32_t* inv, const float* gates, const int32_t* ids,
+                       const float* router_w, const float* dy, int T, int k, int d, const uint32_t* dmax, uint16_t* dO,
+                       float* dx, int32_t* status, cudaStream_t s) {
+  if (T == 0) return TQP_OK;
+  // whole warps only: the row reductions use full-mask warp shuffles
+  const int threads = d / 8 >= 256 ? 256 : ((d / 8 + 31) / 32) * 32;
+  bwd_combine_kernel<<<T, threads, 0, s>>>(O, inv, gates, ids, router_w, dy, T, k, d, dmax, dO, dx, status);
+  return cudaGetLastError() == cudaSuccess ? TQP_OK : TQP_ERR_CUDA;
+}
+
+int launch_gather_add(const uint16_t* dX, const int32_t* inv, int T, int k, int d, const uint32_t* dmax, float* dx,
+                      cudaStream_t s) {
   if (T == 0) return TQP_OK;
   const int threads = d / 8 < 256 ? d / 8 : 256;
-  gather_add_kernel<<<T, threads, 0, s>>>(dX, inv, T, k, d, dx);
+  gather_add_kernel<<<T, threads, 0, s>>>(dX, inv, T, k, d, dmax, dx);
   return cudaGetLastError() == cudaSuccess ? TQP_OK : TQP_ERR_CUDA;
 }
 
 int launch_outer(int E, int M, int N, const int32_t* offsets, const int32_t* perm, const uint16_t* P, int ldp,
-                 int offp, const uint16_t* Q, int ldq, int offq, float* C, cudaStream_t s) {
+                 int offp, const uint16_t* Q, int ldq, int offq, float* C, const uint32_t* dmax, cudaStream_t s) {
   OuterArgs a{};
+  a.dmax = dmax;
   a.E = E;
   a.M = M;
   a.N = N;

@@ -12,11 +12,14 @@
 //
 // Host code cannot use the array's name as a device address: on the host it
 // names a stand-in, not the GPU copy. The address of the GPU copy is looked up
-// once per device with cudaGetSymbolAddress, with that device current, during
-// the first call on the device.
-#include <atomic>
+// with cudaGetSymbolAddress, with the device current, on the first call made
+// under a given CUDA context, and cached per context: a context created after
+// a device reset, or another (non-primary) context, gets a fresh lookup instead
+// of a stale address.
 #include <cstdint>
+#include <cuda.h>
 #include <cuda_runtime.h>
+#include <mutex>
 
 #include "../../include/tqp_moe.h"
 #include "tqp_launch.h"
@@ -31,19 +34,64 @@ constexpr size_t kScratchBytes = (size_t(1) << 20) + 4096;
 
 static __device__ __align__(256) unsigned char g_permute_scratch[kScratchBytes];
 
-constexpr int kMaxDevices = 64;
-std::atomic<void*> g_scratch_ptr[kMaxDevices];
+// Cached device addresses of the array, one per (device, context) seen. A
+// context is identified by its process-unique id (cuCtxGetId), so that a
+// context created after a device reset never reuses the address looked up in
+// the one it replaced, even if the driver hands out the same handle again.
+constexpr int kCacheSlots = 64;
+struct Slot {
+  int dev;
+  unsigned long long ctx_id;
+  void* ptr;
+};
+std::mutex g_mu;
+Slot g_slots[kCacheSlots];
+int g_nslots = 0;
 
-// Device address of the scratch array on the current device (looked up once).
+using CtxGetCurrentFn = CUresult (*)(CUcontext*);
+using CtxGetIdFn = CUresult (*)(CUcontext, unsigned long long*);
+
+template <typename F>
+F driver_fn(const char* name) {
+  void* p = nullptr;
+  cudaDriverEntryPointQueryResult q;
+  if (cudaGetDriverEntryPoint(name, &p, cudaEnableDefault, &q) != cudaSuccess || q != cudaDriverEntryPointSuccess)
+    return nullptr;
+  return reinterpret_cast<F>(p);
+}
+
+// Process-unique id of the current context; false when none is current.
+bool current_context_id(unsigned long long* id) {
+  static CtxGetCurrentFn get_current = driver_fn<CtxGetCurrentFn>("cuCtxGetCurrent");
+  static CtxGetIdFn get_id = driver_fn<CtxGetIdFn>("cuCtxGetId");
+  if (!get_current || !get_id) return false;
+  CUcontext c = nullptr;
+  if (get_current(&c) != CUDA_SUCCESS || c == nullptr) return false;
+  return get_id(c, id) == CUDA_SUCCESS;
+}
+
+// Device address of the scratch array in the current context (looked up with
+// cudaGetSymbolAddress on the first call under each context).
 int scratch_address(void** out) {
   int dev = 0;
   if (cudaGetDevice(&dev) != cudaSuccess) return TQP_ERR_CUDA;
-  if (dev < 0 || dev >= kMaxDevices) return TQP_ERR_UNSUPPORTED;
-  void* p = g_scratch_ptr[dev].load(std::memory_order_acquire);
-  if (p == nullptr) {
+  unsigned long long id = 0;
+  void* p = nullptr;
+  if (!current_context_id(&id)) {
+    // no context yet: the lookup makes the runtime create the device's primary one
     if (cudaGetSymbolAddress(&p, g_permute_scratch) != cudaSuccess || p == nullptr) return TQP_ERR_CUDA;
-    g_scratch_ptr[dev].store(p, std::memory_order_release);
+    if (!current_context_id(&id)) return TQP_ERR_CUDA;
   }
+  std::lock_guard<std::mutex> lock(g_mu);
+  for (int i = 0; i < g_nslots; ++i)
+    if (g_slots[i].dev == dev && g_slots[i].ctx_id == id) {
+      *out = g_slots[i].ptr;
+      return TQP_OK;
+    }
+  if (p == nullptr && (cudaGetSymbolAddress(&p, g_permute_scratch) != cudaSuccess || p == nullptr))
+    return TQP_ERR_CUDA;
+  if (g_nslots == kCacheSlots) g_nslots = 0;   // start over rather than grow
+  g_slots[g_nslots++] = Slot{dev, id, p};
   *out = p;
   return TQP_OK;
 }

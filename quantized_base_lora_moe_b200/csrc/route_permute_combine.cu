@@ -1,13 +1,14 @@
 // Routing, permutation and combine kernels of the TQP MoE layer (sm_100a).
 //
-//  moe_route    : one warp per token; top-k by repeated warp arg-max on a 64-bit
-//                 key (orderable logit, then lower expert id), renormalised
-//                 softmax over the chosen logits ("Top-12 routing",
+//  moe_route    : one warp per token; top-k by k rounds of warp arg-max over an
+//                 orderable 32-bit logit key, exact ties broken by the lower
+//                 expert id; renormalised softmax over the chosen logits ("Top-12 routing",
 //                 Architecture Details; stateless routing, Reversibility
 //                 Implementation).
 //  moe_permute  : stable counting sort by expert in three passes: per 32-token
 //                 chunk expert bitmaps -> per-expert column prefix over chunks
-//                 -> scatter with rank = popcount of earlier tokens' bits.
+//                 (block-parallel) -> scatter with rank = popcount of earlier
+//                 tokens' bits.
 //  moe_combine  : gate-weighted gather back to token order (fixed j order, fp32,
 //                 no atomics) with the additive coupling fused in ("Pattern 1":
 //                 addition/subtraction are invertible).
@@ -31,58 +32,86 @@ __device__ __forceinline__ uint32_t logit_key(float v) {
   return (b & 0x80000000u) ? (~b) : (b | 0x80000000u);
 }
 
-__device__ __forceinline__ uint64_t pack_key(float v, int e) {
-  return (uint64_t(logit_key(v)) << 32) | uint64_t(0xFFFFFFFFu - uint32_t(e));
-}
-
-__device__ __forceinline__ uint64_t warp_max_u64(uint64_t v) {
+__device__ __forceinline__ uint32_t warp_max_u32(uint32_t v) {
 #pragma unroll
-  for (int o = 16; o > 0; o >>= 1) {
-    const uint64_t w = __shfl_xor_sync(0xFFFFFFFFu, v, o);
-    v = w > v ? w : v;
-  }
+  for (int o = 16; o > 0; o >>= 1) v = max(v, __shfl_xor_sync(0xFFFFFFFFu, v, o));
   return v;
 }
 
+__device__ __forceinline__ uint32_t warp_min_u32(uint32_t v) {
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) v = min(v, __shfl_xor_sync(0xFFFFFFFFu, v, o));
+  return v;
+}
+
+// One warp per token. Lane l holds the orderable keys of experts l, l+32, ...
+// Each of the k rounds takes every lane's best key not yet chosen (lowest
+// expert id among equal keys: the lane's elements are visited in increasing
+// id order), the warp maximum of those, and among the lanes that hold it the
+// lowest expert id (one ballot; a min-reduction only when several lanes tie).
+// The winner lane marks its element as chosen.
 template <int EPL>  // logits per lane kept in registers (E <= 32 * EPL)
 __global__ void __launch_bounds__(256) route_kernel(const float* __restrict__ logits, int T, int E, int k,
                                                     int32_t* __restrict__ ids, float* __restrict__ gates,
                                                     int32_t* status) {
+  constexpr int NW = (EPL + 31) / 32;   // exclusion mask words
   const int lane = threadIdx.x & 31;
   const int t = blockIdx.x * (blockDim.x >> 5) + (threadIdx.x >> 5);
   if (t >= T) return;
   const float* row = logits + size_t(t) * E;
-  uint64_t key[EPL];
+  uint32_t key[EPL];
   bool nonfinite = false;
+  uint32_t excl[NW];   // bit i: element lane + 32 i chosen already, or past E
+#pragma unroll
+  for (int w = 0; w < NW; ++w) excl[w] = 0u;
 #pragma unroll
   for (int i = 0; i < EPL; ++i) {
     const int e = lane + 32 * i;
     if (e < E) {
       const float v = __ldg(row + e);
       nonfinite |= !isfinite(v);
-      key[i] = pack_key(v, e);
+      key[i] = logit_key(v);
     } else {
-      key[i] = 0ull;  // below every real entry (a real key has a non-zero low word)
+      key[i] = 0u;
+      excl[i >> 5] |= 1u << (i & 31);
     }
   }
   if (__any_sync(0xFFFFFFFFu, nonfinite) && lane == 0) raise_status(status, TQP_STATUS_NONFINITE);
 
-  uint64_t bound = ~0ull;
   int my_id = 0;
   float my_val = 0.0f;
   for (int j = 0; j < k; ++j) {
-    uint64_t best = 0ull;
+    uint32_t best = 0u;
+    int bi = -1;
 #pragma unroll
-    for (int i = 0; i < EPL; ++i) best = (key[i] < bound && key[i] > best) ? key[i] : best;
-    best = warp_max_u64(best);
-    bound = best;
+    for (int i = 0; i < EPL; ++i) {
+      const bool take = !((excl[i >> 5] >> (i & 31)) & 1u) && (bi < 0 || key[i] > best);
+      best = take ? key[i] : best;
+      bi = take ? i : bi;
+    }
+    const uint32_t m = warp_max_u32(bi >= 0 ? best : 0u);
+    const uint32_t cand = __ballot_sync(0xFFFFFFFFu, bi >= 0 && best == m);
+    int winner = __ffs(cand) - 1;                  // lowest lane; its id is lowest unless elements differ in i
+    const uint32_t my = (bi >= 0 && ((cand >> lane) & 1u)) ? uint32_t(lane + 32 * bi) : 0xFFFFFFFFu;
+    uint32_t wid;
+    if (__popc(cand) == 1) {
+      wid = __shfl_sync(0xFFFFFFFFu, my, winner);
+    } else {
+      wid = warp_min_u32(my);                      // exact tie between lanes: the lowest expert id
+      winner = int(wid & 31u);
+    }
+    if (lane == winner) {
+#pragma unroll
+      for (int w = 0; w < NW; ++w)
+        if (w == (bi >> 5)) excl[w] |= 1u << (bi & 31);
+    }
     if (lane == j) {
-      my_id = int(0xFFFFFFFFu - uint32_t(best & 0xFFFFFFFFull));
+      my_id = int(wid);
       my_val = __ldg(row + my_id);
     }
   }
-  const float m = __shfl_sync(0xFFFFFFFFu, my_val, 0);
-  float ex = (lane < k) ? expf(my_val - m) : 0.0f;
+  const float mx = __shfl_sync(0xFFFFFFFFu, my_val, 0);
+  float ex = (lane < k) ? expf(my_val - mx) : 0.0f;
   float sum = ex;
 #pragma unroll
   for (int o = 16; o > 0; o >>= 1) sum += __shfl_xor_sync(0xFFFFFFFFu, sum, o);
@@ -116,6 +145,8 @@ int launch_route(const float* logits, int T, int E, int k, int32_t* ids, float* 
 // ----------------------------------------------------------------------------
 
 // Pass 1: per 32-token chunk w, count[w][e] = #tokens of the chunk routed to e.
+// An id outside [0, E), or a token that lists one expert twice (its bit is
+// already set when the second slot is recorded), raises TQP_STATUS_BAD_ID.
 __global__ void permute_count_kernel(const int32_t* __restrict__ ids, int T, int E, int k,
                                      int32_t* __restrict__ count, int32_t* status) {
   extern __shared__ uint32_t bits_all[];
@@ -132,7 +163,7 @@ __global__ void permute_count_kernel(const int32_t* __restrict__ ids, int T, int
   if (t < T) {
     for (int j = 0; j < k; ++j) {
       const int e = ids[size_t(t) * k + j];
-      if (e >= 0 && e < E) atomicOr(&bits[e], 1u << lane);
+      if (e >= 0 && e < E) bad |= (atomicOr(&bits[e], 1u << lane) & (1u << lane)) != 0u;
       else bad = true;
     }
   }
@@ -141,19 +172,34 @@ __global__ void permute_count_kernel(const int32_t* __restrict__ ids, int T, int
   for (int e = lane; e < E; e += 32) count[size_t(w) * E + e] = __popc(bits[e]);
 }
 
-// Pass 2: one thread per expert: exclusive prefix of count[.][e] over chunks
-// (in place) and the expert total.
-__global__ void permute_colscan_kernel(int32_t* __restrict__ count, int W, int E, int32_t* __restrict__ total) {
-  const int e = blockIdx.x * blockDim.x + threadIdx.x;
-  if (e >= E) return;
+// Pass 2: exclusive prefix of count[.][e] over the chunks (in place) and the
+// expert totals. A block takes 32 experts (lane = expert, so every row access
+// is one coalesced 128-byte piece); its warps split the chunks into slices,
+// sum their slices, take the prefix over the earlier slices from shared
+// memory, and rewrite their slices with the running prefix.
+__global__ void __launch_bounds__(1024) permute_colscan_kernel(int32_t* __restrict__ count, int W, int E,
+                                                               int32_t* __restrict__ total) {
+  __shared__ int32_t part[32][33];
+  const int lane = threadIdx.x & 31, wid = threadIdx.x >> 5, nw = blockDim.x >> 5;
+  const int e = blockIdx.x * 32 + lane;
+  const int per = (W + nw - 1) / nw;
+  const int w0 = min(W, wid * per), w1 = min(W, w0 + per);
+  int sum = 0;
+  if (e < E)
+    for (int w = w0; w < w1; ++w) sum += count[size_t(w) * E + e];
+  part[wid][lane] = sum;
+  __syncthreads();
   int run = 0;
-  for (int w = 0; w < W; ++w) {
-    const size_t i = size_t(w) * E + e;
-    const int c = count[i];
-    count[i] = run;
-    run += c;
+  for (int i = 0; i < wid; ++i) run += part[i][lane];
+  if (e < E) {
+    for (int w = w0; w < w1; ++w) {
+      const size_t i = size_t(w) * E + e;
+      const int c = count[i];
+      count[i] = run;
+      run += c;
+    }
+    if (wid == nw - 1) total[e] = run;
   }
-  total[e] = run;
 }
 
 // Block-wide exclusive scan of total[0..E) into off[0..E] (shared memory).
@@ -252,14 +298,17 @@ int launch_permute(const int32_t* ids, int T, int E, int k, int32_t* offsets, in
   int wpb = 8;
   while (wpb > 1 && size_t(wpb) * E * 4 > 64 * 1024) wpb >>= 1;
   const size_t smem1 = size_t(wpb) * E * 4;
-  if (smem1 > 48 * 1024) cudaFuncSetAttribute(permute_count_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, int(smem1));
+  // the largest dynamic shared memory either pass can ask for (E <= 4096), set
+  // once per device
+  static DeviceFlags count_attr, scatter_attr;
+  if (smem1 > 48 * 1024 && !count_attr.test_and_set_device(permute_count_kernel, 64 * 1024)) return TQP_ERR_CUDA;
   permute_count_kernel<<<(W + wpb - 1) / wpb, wpb * 32, smem1, s>>>(ids, T, E, k, count, status);
   // pass 2
-  permute_colscan_kernel<<<(E + 127) / 128, 128, 0, s>>>(count, W, E, total);
+  permute_colscan_kernel<<<(E + 31) / 32, W >= 1024 ? 1024 : ((W + 31) / 32) * 32, 0, s>>>(count, W, E, total);
   // pass 3
   const size_t smem3 = size_t(E + 1 + 32) * 4 + size_t(wpb) * E * 4;
-  if (smem3 > 48 * 1024)
-    cudaFuncSetAttribute(permute_scatter_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, int(smem3));
+  if (smem3 > 48 * 1024 && !scatter_attr.test_and_set_device(permute_scatter_kernel, (4096 + 1 + 32) * 4 + 64 * 1024))
+    return TQP_ERR_CUDA;
   permute_scatter_kernel<<<(W + wpb - 1) / wpb, wpb * 32, smem3, s>>>(ids, T, E, k, count, total, offsets,
                                                                       perm_token, inv, wpb);
   return cudaGetLastError() == cudaSuccess ? TQP_OK : TQP_ERR_CUDA;

@@ -1,6 +1,7 @@
 // C ABI of the TQP MoE library: argument validation, workspace layout and the
 // composition of the per-step kernels into the layer, the reversible coupling
 // and its backward. Declarations and contracts: include/tqp_moe.h.
+#include <atomic>
 #include <cstdint>
 #include <cstring>
 #include <cuda_runtime.h>
@@ -10,6 +11,12 @@
 #include "tqp_launch.h"
 
 using namespace tqp;
+
+namespace {
+std::atomic<unsigned long long> g_wait_limit_ns{0};
+}  // namespace
+
+unsigned long long tqp::wait_limit_ns() { return g_wait_limit_ns.load(std::memory_order_relaxed); }
 
 namespace {
 
@@ -111,6 +118,7 @@ struct BwdWs {
   uint16_t* dgu;    // dG | dU [A][2f] fp16
   uint16_t* dxa;    // s [dG|dU] [Bg|Bu]^T [A][2r] fp16
   uint16_t* bk16;   // K-major fp16 B operand of dha / dxa, E * max(r d, 4 r f) values
+  uint32_t* dmax;   // max |dy| (sets the power-of-two scale of the fp16 intermediates)
 };
 
 // Adapter-gradient buffers: present and 16-byte aligned when the rank is nonzero.
@@ -130,7 +138,7 @@ size_t rank_b_values(const tqp_moe_weights* w) {
 size_t bwd_extra_bytes(int T, const tqp_moe_weights* w) {
   const size_t A = size_t(T) * w->top_k;
   return align_up(A * 2 * w->ffn * 2, 256) * 2 + align_up(A * w->d * 2, 256) + align_up(A * w->rank * 2, 256) +
-         align_up(A * 2 * w->rank * 2, 256) + align_up(rank_b_values(w) * 2, 256) + 256;
+         align_up(A * 2 * w->rank * 2, 256) + align_up(rank_b_values(w) * 2, 256) + 256 + 256;
 }
 
 BwdWs carve_bwd(void* p0, int T, const tqp_moe_weights* w) {
@@ -148,6 +156,7 @@ BwdWs carve_bwd(void* p0, int T, const tqp_moe_weights* w) {
   b.dgu = static_cast<uint16_t*>(take(A * 2 * w->ffn * 2));
   b.dxa = static_cast<uint16_t*>(take(A * 2 * w->rank * 2));
   b.bk16 = static_cast<uint16_t*>(take(rank_b_values(w) * 2));
+  b.dmax = static_cast<uint32_t*>(take(sizeof(uint32_t)));
   return b;
 }
 
@@ -165,7 +174,9 @@ int layer_backward(const uint16_t* x, const float* dy, int T, const tqp_moe_weig
   int rc;
   if (recompute && (rc = layer_experts(x, T, w, L, status, s, B.gu)) != TQP_OK) return rc;
   const FfnBufs fb = ffn_carve(L.ffn_ws, T, w);
-  if ((rc = launch_bwd_combine(L.out_perm, L.inv, L.gates, L.ids, w->router_w, dy, T, k, d, B.dO, dx, s)) != TQP_OK)
+  if ((rc = launch_grad_absmax(dy, size_t(T) * d, B.dmax, s)) != TQP_OK) return rc;
+  if ((rc = launch_bwd_combine(L.out_perm, L.inv, L.gates, L.ids, w->router_w, dy, T, k, d, B.dmax, B.dO, dx, status,
+                               s)) != TQP_OK)
     return rc;
   if (r > 0 && (rc = launch_rank_bwd(0, B.dO, L.offsets, fb.mb_prefix, w, T, B.bk16, B.dha, status, s)) != TQP_OK)
     return rc;
@@ -173,21 +184,26 @@ int layer_backward(const uint16_t* x, const float* dy, int T, const tqp_moe_weig
   if (r > 0) {
     if ((rc = launch_rank_bwd(1, B.dgu, L.offsets, fb.mb_prefix, w, T, B.bk16, B.dxa, status, s)) != TQP_OK)
       return rc;
-    // adapter gradients, in the storage layouts A^T [r][in], B^T [out][r]
-    if ((rc = launch_outer(E, d, r, L.offsets, nullptr, B.dO, d, 0, fb.ha, r, 0, g->dB[2], s)) != TQP_OK) return rc;
-    if ((rc = launch_outer(E, r, f, L.offsets, nullptr, B.dha, r, 0, L.h, f, 0, g->dA[2], s)) != TQP_OK) return rc;
-    if ((rc = launch_outer(E, f, r, L.offsets, nullptr, B.dgu, 2 * f, 0, fb.xa, 2 * r, 0, g->dB[0], s)) != TQP_OK)
+    // adapter gradients, in the storage layouts A^T [r][in], B^T [out][r]: on the
+    // tensor cores for ranks up to 32, else as outer products on the CUDA cores
+    rc = launch_wgrad(w, L.offsets, L.perm, B.dO, L.h, B.dgu, fb.x16, fb.ha, B.dha, fb.xa, B.dxa, g, B.dmax, status, s);
+    if (rc != TQP_OK && rc != TQP_ERR_UNSUPPORTED) return rc;
+  }
+  if (r > 0 && rc == TQP_ERR_UNSUPPORTED) {
+    if ((rc = launch_outer(E, d, r, L.offsets, nullptr, B.dO, d, 0, fb.ha, r, 0, g->dB[2], B.dmax, s)) != TQP_OK) return rc;
+    if ((rc = launch_outer(E, r, f, L.offsets, nullptr, B.dha, r, 0, L.h, f, 0, g->dA[2], B.dmax, s)) != TQP_OK) return rc;
+    if ((rc = launch_outer(E, f, r, L.offsets, nullptr, B.dgu, 2 * f, 0, fb.xa, 2 * r, 0, g->dB[0], B.dmax, s)) != TQP_OK)
       return rc;
-    if ((rc = launch_outer(E, f, r, L.offsets, nullptr, B.dgu, 2 * f, f, fb.xa, 2 * r, r, g->dB[1], s)) != TQP_OK)
+    if ((rc = launch_outer(E, f, r, L.offsets, nullptr, B.dgu, 2 * f, f, fb.xa, 2 * r, r, g->dB[1], B.dmax, s)) != TQP_OK)
       return rc;
-    if ((rc = launch_outer(E, r, d, L.offsets, L.perm, B.dxa, 2 * r, 0, fb.x16, d, 0, g->dA[0], s)) != TQP_OK)
+    if ((rc = launch_outer(E, r, d, L.offsets, L.perm, B.dxa, 2 * r, 0, fb.x16, d, 0, g->dA[0], B.dmax, s)) != TQP_OK)
       return rc;
-    if ((rc = launch_outer(E, r, d, L.offsets, L.perm, B.dxa, 2 * r, r, fb.x16, d, 0, g->dA[1], s)) != TQP_OK)
+    if ((rc = launch_outer(E, r, d, L.offsets, L.perm, B.dxa, 2 * r, r, fb.x16, d, 0, g->dA[1], B.dmax, s)) != TQP_OK)
       return rc;
   }
   uint16_t* dX = B.dO;  // dO is no longer needed
   if ((rc = launch_dgrad(1, B.dgu, B.dxa, L.offsets, fb.mb_prefix, w, T, nullptr, dX, status, s)) != TQP_OK) return rc;
-  return launch_gather_add(dX, L.inv, T, k, d, dx, s);
+  return launch_gather_add(dX, L.inv, T, k, d, B.dmax, dx, s);
 }
 
 int layer_forward(const uint16_t* x, int T, const tqp_moe_weights* w, const void* residual, int res_f32,
@@ -219,11 +235,100 @@ int to_bf16(const float* in, uint16_t* out, size_t n, cudaStream_t s) {
   return cudaGetLastError() == cudaSuccess ? TQP_OK : TQP_ERR_CUDA;
 }
 
+// ----------------------------------------------------------------------------
+// reversible stack of L coupling blocks
+// ----------------------------------------------------------------------------
+// Block l maps fp32 streams (a1, a2) to (b1, b2):  b1 = a1 + F_l(bf16(a2)),
+// b2 = a2 + G_l(bf16(b1)). The streams stay fp32 between blocks; every layer
+// reads the bf16 rounding of its stream. For block 0 the inputs are the bf16
+// x1, x2 (exact in fp32), so one block is exactly rev_couple_fwd. The
+// workspace holds two sets of stream buffers that the blocks alternate
+// between, two bf16 layer inputs, one fp32 input gradient and one layer's
+// workspace: activation memory does not grow with L.
+
+constexpr int kMaxStack = 4096;
+
+int check_stack(int T, int L, const tqp_moe_weights* const* F, const tqp_moe_weights* const* G, bool bwd) {
+  if (T < 0 || L < 1 || L > kMaxStack || !F || !G) return TQP_ERR_INVALID_ARG;
+  int rc;
+  for (int l = 0; l < L; ++l) {
+    if ((rc = check_weights(F[l])) != TQP_OK || (rc = check_weights(G[l])) != TQP_OK) return rc;
+    if (F[l]->d != F[0]->d || G[l]->d != F[0]->d) return TQP_ERR_INVALID_ARG;
+    if (bwd && (F[l]->ffn % 128 != 0 || G[l]->ffn % 128 != 0)) return TQP_ERR_UNSUPPORTED;
+  }
+  return TQP_OK;
+}
+
+size_t stack_layer_ws(int T, int L, const tqp_moe_weights* const* F, const tqp_moe_weights* const* G) {
+  size_t m = 0;
+  for (int l = 0; l < L; ++l) {
+    const size_t a = layer_ws_size(T, F[l]) + bwd_extra_bytes(T, F[l]);
+    const size_t b = layer_ws_size(T, G[l]) + bwd_extra_bytes(T, G[l]);
+    m = a > m ? a : m;
+    m = b > m ? b : m;
+  }
+  return m;
+}
+
+struct StackWs {
+  float* s[2][4];     // two sets of (stream 1, stream 2, cotangent 1, cotangent 2), fp32 [T][d]
+  uint16_t* zb;       // bf16 layer input
+  uint16_t* ab;       // bf16 layer input
+  float* dxl;         // a layer's input gradient
+  void* lws;          // one layer's forward + backward workspace
+};
+
+StackWs carve_stack(void* ws, int T, int d) {
+  const size_t Td = size_t(T) * d;
+  char* p = reinterpret_cast<char*>(align_up(reinterpret_cast<uintptr_t>(ws), 256));
+  StackWs w;
+  for (int i = 0; i < 2; ++i)
+    for (int j = 0; j < 4; ++j) {
+      w.s[i][j] = reinterpret_cast<float*>(p);
+      p += align_up(Td * 4, 256);
+    }
+  w.zb = reinterpret_cast<uint16_t*>(p);
+  p += align_up(Td * 2, 256);
+  w.ab = reinterpret_cast<uint16_t*>(p);
+  p += align_up(Td * 2, 256);
+  w.dxl = reinterpret_cast<float*>(p);
+  p += align_up(Td * 4, 256);
+  w.lws = p;
+  return w;
+}
+
+size_t stack_ws_size(int T, int L, const tqp_moe_weights* const* F, const tqp_moe_weights* const* G) {
+  const size_t Td = size_t(T) * F[0]->d;
+  return 8 * align_up(Td * 4, 256) + 2 * align_up(Td * 2, 256) + align_up(Td * 4, 256) +
+         stack_layer_ws(T, L, F, G) + 512;
+}
+
+// Block backward on fp32 streams: from the block outputs (y1, y2) and their
+// cotangents, the block inputs (a1, a2) and their cotangents (da1, da2) plus
+// both layers' adapter gradients. Each layer's backward follows the inverse
+// step that ran its forward on the same workspace. a2b receives bf16(a2).
+int block_backward_f32(const float* y1, const float* y2, const float* dy1, const float* dy2, int T,
+                       const tqp_moe_weights* F, const tqp_moe_weights* G, float* a1, float* a2, float* da1,
+                       float* da2, const tqp_adapter_grads* gF, const tqp_adapter_grads* gG, const StackWs& w,
+                       int32_t* status, cudaStream_t s) {
+  const size_t Td = size_t(T) * F->d;
+  int rc;
+  if ((rc = to_bf16(y1, w.zb, Td, s)) != TQP_OK) return rc;
+  uint16_t* gu = carve_bwd(static_cast<char*>(w.lws) + layer_ws_size(T, G), T, G).gu;
+  if ((rc = layer_forward(w.zb, T, G, y2, 1, -1.0f, a2, 1, w.ab, w.lws, status, s, gu)) != TQP_OK) return rc;
+  if ((rc = layer_backward(w.zb, dy2, T, G, w.dxl, gG, w.lws, status, s, false)) != TQP_OK) return rc;
+  if ((rc = launch_add_f32(dy1, w.dxl, da1, Td, s)) != TQP_OK) return rc;
+  gu = carve_bwd(static_cast<char*>(w.lws) + layer_ws_size(T, F), T, F).gu;
+  if ((rc = layer_forward(w.ab, T, F, y1, 1, -1.0f, a1, 1, nullptr, w.lws, status, s, gu)) != TQP_OK) return rc;
+  if ((rc = layer_backward(w.ab, da1, T, F, w.dxl, gF, w.lws, status, s, false)) != TQP_OK) return rc;
+  return launch_add_f32(dy2, w.dxl, da2, Td, s);
+}
+
 }  // namespace
 
 extern "C" {
 
-int tqp_version(void) { return 100; }
+int tqp_version(void) { return 200; }
 
 const char* tqp_error_string(int code) {
   switch (code) {
@@ -443,6 +548,118 @@ int tqp_adapter_bwd(const float* y1, const float* y2, const float* dy1, const fl
   if ((rc = layer_forward(x2, T, F, y1, 1, -1.0f, x1, 0, nullptr, lws, dev_status, s, gu)) != TQP_OK) return rc;
   if ((rc = layer_backward(x2, dx1, T, F, dxG, gF, lws, dev_status, s, false)) != TQP_OK) return rc;
   return launch_add_f32(dy2, dxG, dx2, Td, s);
+}
+
+size_t rev_stack_workspace_size(int T, int L, const tqp_moe_weights* const* F, const tqp_moe_weights* const* G) {
+  if (check_stack(T, L, F, G, false) != TQP_OK) return 0;
+  return stack_ws_size(T, L, F, G);
+}
+
+int rev_stack_fwd(const uint16_t* x1, const uint16_t* x2, int T, int L, const tqp_moe_weights* const* F,
+                  const tqp_moe_weights* const* G, float* y1, float* y2, void* ws, size_t ws_bytes,
+                  int32_t* dev_status, void* stream) {
+  int rc;
+  if ((rc = check_stack(T, L, F, G, false)) != TQP_OK) return rc;
+  const bool n = T > 0;
+  if (!ptr_ok(x1, n) || !ptr_ok(x2, n) || !ptr_ok(y1, n) || !ptr_ok(y2, n) || !ptr_ok(ws, n))
+    return TQP_ERR_INVALID_ARG;
+  if (!n) return TQP_OK;
+  if (ws_bytes < stack_ws_size(T, L, F, G)) return TQP_ERR_WORKSPACE;
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  const StackWs w = carve_stack(ws, T, F[0]->d);
+  const size_t Td = size_t(T) * F[0]->d;
+  for (int l = 0; l < L; ++l) {
+    float* b1 = (l == L - 1) ? y1 : w.s[l & 1][0];
+    float* b2 = (l == L - 1) ? y2 : w.s[l & 1][1];
+    if (l == 0) {
+      // b1 = x1 + F(x2), with bf16(b1) for G; b2 = x2 + G(bf16(b1))
+      if ((rc = layer_forward(x2, T, F[0], x1, 0, 1.0f, b1, 1, w.zb, w.lws, dev_status, s)) != TQP_OK) return rc;
+      if ((rc = layer_forward(w.zb, T, G[0], x2, 0, 1.0f, b2, 1, nullptr, w.lws, dev_status, s)) != TQP_OK)
+        return rc;
+    } else {
+      const float* a1 = w.s[(l - 1) & 1][0];
+      const float* a2 = w.s[(l - 1) & 1][1];
+      if ((rc = to_bf16(a2, w.ab, Td, s)) != TQP_OK) return rc;
+      if ((rc = layer_forward(w.ab, T, F[l], a1, 1, 1.0f, b1, 1, w.zb, w.lws, dev_status, s)) != TQP_OK) return rc;
+      if ((rc = layer_forward(w.zb, T, G[l], a2, 1, 1.0f, b2, 1, nullptr, w.lws, dev_status, s)) != TQP_OK)
+        return rc;
+    }
+  }
+  return TQP_OK;
+}
+
+int rev_stack_inv(const float* y1, const float* y2, int T, int L, const tqp_moe_weights* const* F,
+                  const tqp_moe_weights* const* G, uint16_t* x1, uint16_t* x2, void* ws, size_t ws_bytes,
+                  int32_t* dev_status, void* stream) {
+  int rc;
+  if ((rc = check_stack(T, L, F, G, false)) != TQP_OK) return rc;
+  const bool n = T > 0;
+  if (!ptr_ok(x1, n) || !ptr_ok(x2, n) || !ptr_ok(y1, n) || !ptr_ok(y2, n) || !ptr_ok(ws, n))
+    return TQP_ERR_INVALID_ARG;
+  if (!n) return TQP_OK;
+  if (ws_bytes < stack_ws_size(T, L, F, G)) return TQP_ERR_WORKSPACE;
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  const StackWs w = carve_stack(ws, T, F[0]->d);
+  const size_t Td = size_t(T) * F[0]->d;
+  const float* c1 = y1;
+  const float* c2 = y2;
+  for (int l = L - 1; l >= 0; --l) {
+    if ((rc = to_bf16(c1, w.zb, Td, s)) != TQP_OK) return rc;
+    if (l == 0) {
+      // the block inputs are bf16: x2 = y2 - G(bf16(y1)), x1 = y1 - F(x2)
+      if ((rc = layer_forward(w.zb, T, G[0], c2, 1, -1.0f, x2, 0, nullptr, w.lws, dev_status, s)) != TQP_OK)
+        return rc;
+      return layer_forward(x2, T, F[0], c1, 1, -1.0f, x1, 0, nullptr, w.lws, dev_status, s);
+    }
+    float* a1 = w.s[l & 1][0];
+    float* a2 = w.s[l & 1][1];
+    if ((rc = layer_forward(w.zb, T, G[l], c2, 1, -1.0f, a2, 1, w.ab, w.lws, dev_status, s)) != TQP_OK) return rc;
+    if ((rc = layer_forward(w.ab, T, F[l], c1, 1, -1.0f, a1, 1, nullptr, w.lws, dev_status, s)) != TQP_OK) return rc;
+    c1 = a1;
+    c2 = a2;
+  }
+  return TQP_OK;
+}
+
+int rev_stack_bwd(const float* y1, const float* y2, const float* dy1, const float* dy2, int T, int L,
+                  const tqp_moe_weights* const* F, const tqp_moe_weights* const* G, uint16_t* x1, uint16_t* x2,
+                  float* dx1, float* dx2, const tqp_adapter_grads* const* gF, const tqp_adapter_grads* const* gG,
+                  void* ws, size_t ws_bytes, int32_t* dev_status, void* stream) {
+  int rc;
+  if ((rc = check_stack(T, L, F, G, true)) != TQP_OK) return rc;
+  if (!gF || !gG) return TQP_ERR_INVALID_ARG;
+  for (int l = 0; l < L; ++l)
+    if (!grads_ok(F[l], gF[l]) || !grads_ok(G[l], gG[l])) return TQP_ERR_INVALID_ARG;
+  const bool n = T > 0;
+  if (!ptr_ok(y1, n) || !ptr_ok(y2, n) || !ptr_ok(dy1, n) || !ptr_ok(dy2, n) || !ptr_ok(x1, n) || !ptr_ok(x2, n) ||
+      !ptr_ok(dx1, n) || !ptr_ok(dx2, n) || !ptr_ok(ws, n))
+    return TQP_ERR_INVALID_ARG;
+  if (!n) return TQP_OK;
+  if (ws_bytes < stack_ws_size(T, L, F, G)) return TQP_ERR_WORKSPACE;
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  const StackWs w = carve_stack(ws, T, F[0]->d);
+  const size_t Td = size_t(T) * F[0]->d;
+  const float *c1 = y1, *c2 = y2, *c3 = dy1, *c4 = dy2;
+  for (int l = L - 1; l >= 0; --l) {
+    float* const* o = w.s[l & 1];
+    // block 0's cotangents are the call's outputs; its inputs are rounded to bf16 below
+    float* da1 = (l == 0) ? dx1 : o[2];
+    float* da2 = (l == 0) ? dx2 : o[3];
+    if ((rc = block_backward_f32(c1, c2, c3, c4, T, F[l], G[l], o[0], o[1], da1, da2, gF[l], gG[l], w, dev_status,
+                                 s)) != TQP_OK)
+      return rc;
+    c1 = o[0];
+    c2 = o[1];
+    c3 = da1;
+    c4 = da2;
+  }
+  if ((rc = to_bf16(c1, x1, Td, s)) != TQP_OK) return rc;
+  return to_bf16(c2, x2, Td, s);
+}
+
+int tqp_debug_set_wait_limit_ns(unsigned long long ns) {
+  g_wait_limit_ns.store(ns, std::memory_order_relaxed);
+  return TQP_OK;
 }
 
 }  // extern "C"

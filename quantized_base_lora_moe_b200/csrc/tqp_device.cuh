@@ -21,7 +21,22 @@
 
 namespace tqp {
 
-constexpr uint64_t kWaitLimitNs = 2000000000ull;   // 2 s per barrier wait
+constexpr uint64_t kWaitLimitNs = 2000000000ull;   // 2 s per barrier wait (default)
+
+// CTA-wide abort state in shared memory: the flag every role polls, and the
+// limit of one barrier wait (kWaitLimitNs unless the launch asked for another).
+struct Abort {
+  int flag;
+  int pad;
+  unsigned long long limit_ns;
+};
+
+__device__ __forceinline__ void abort_init(Abort* ab, unsigned long long limit_ns) {
+  ab->flag = 0;
+  ab->limit_ns = limit_ns ? limit_ns : kWaitLimitNs;
+}
+
+__device__ __forceinline__ bool aborted(const Abort* ab) { return *reinterpret_cast<const volatile int*>(&ab->flag) != 0; }
 
 __device__ __forceinline__ uint32_t smem_u32(const void* p) {
   return static_cast<uint32_t>(__cvta_generic_to_shared(p));
@@ -71,24 +86,24 @@ __device__ __forceinline__ bool mbar_try_wait(uint32_t addr, uint32_t parity) {
 }
 
 // Bounded wait for the phase with the given parity. Returns false (and sets the
-// CTA abort flag and the timeout status bit) when the limit expires or another
-// role has already aborted. kSleep > 0 backs off with nanosleep between polls,
-// for waiters off the critical path (they then leave issue slots to the
-// dequantising warps).
+// CTA abort flag and the timeout status bit) when the CTA's wait limit expires
+// or another role has already aborted. kSleep > 0 backs off with nanosleep
+// between polls, for waiters off the critical path (they then leave issue
+// slots to the dequantising warps).
 template <int kSleep = 0>
-__device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, volatile int* abort_flag,
-                                          int32_t* status) {
+__device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, Abort* ab, int32_t* status) {
   const uint32_t addr = smem_u32(bar);
   if (mbar_try_wait(addr, parity)) return true;
   const uint64_t t0 = globaltimer();
+  const uint64_t limit = ab->limit_ns;
   uint32_t spins = 0;
   while (true) {
     if (mbar_try_wait(addr, parity)) return true;
     if (kSleep > 0) __nanosleep(kSleep);
     if (((++spins) & 63u) == 0u) {
-      if (*abort_flag) return false;
-      if (globaltimer() - t0 > kWaitLimitNs) {
-        *abort_flag = 1;
+      if (aborted(ab)) return false;
+      if (globaltimer() - t0 > limit) {
+        *reinterpret_cast<volatile int*>(&ab->flag) = 1;
         raise_status(status, TQP_STATUS_TIMEOUT);
         return false;
       }
@@ -97,9 +112,10 @@ __device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, volati
 }
 
 // Drain wait on the abort path: waits for the phase regardless of the abort
-// flag, but no longer than limit_ns, so that a TMA fill issued before the abort
-// has landed before the CTA exits (its barrier may also never complete when
-// other arrivals are missing; the wait then just runs out).
+// flag, but no longer than limit_ns, so that asynchronous work issued before
+// the abort (a TMA fill, committed MMAs) has finished before the CTA releases
+// its shared and tensor memory. A phase that also needs arrivals that will
+// never come (the other roles left their loops) just runs out.
 __device__ __forceinline__ void mbar_drain(uint64_t* bar, uint32_t parity, uint64_t limit_ns = 1000000ull) {
   const uint32_t addr = smem_u32(bar);
   const uint64_t t0 = globaltimer();
@@ -107,6 +123,23 @@ __device__ __forceinline__ void mbar_drain(uint64_t* bar, uint32_t parity, uint6
     if (globaltimer() - t0 > limit_ns) return;
   }
 }
+
+// The TMA fills one thread has issued into a ring of barriers bar[0..N), so
+// that on the abort path every fill still in flight is waited for, not only
+// the last one (a fill landing after the CTA exits would write shared memory
+// that the next CTA on the SM owns).
+struct PendingFills {
+  uint32_t mask = 0;     // stages with at least one issued fill
+  uint32_t parity = 0;   // bit s: phase parity of the last fill of stage s
+  __device__ __forceinline__ void issued(int stage, uint32_t ph) {
+    mask |= 1u << stage;
+    parity = (parity & ~(1u << stage)) | ((ph & 1u) << stage);
+  }
+  __device__ __forceinline__ void drain(uint64_t* bar0) const {
+    for (int s = 0; s < 32; ++s)
+      if (mask & (1u << s)) mbar_drain(bar0 + s, (parity >> s) & 1u);
+  }
+};
 
 // ----------------------------------------------------------------------------
 // async copies
@@ -252,6 +285,20 @@ __host__ __device__ constexpr uint32_t idesc_f16(int M, int N) {
   return (1u << 4) | (uint32_t(N >> 3) << 17) | (uint32_t(M >> 4) << 24);
 }
 
+// Instruction descriptor: kind::f16, A = B = fp16, D = f32, A K-major, B MN-major.
+__host__ __device__ constexpr uint32_t idesc_f16_bmn(int M, int N) {
+  return (1u << 4) | (1u << 16) | (uint32_t(N >> 3) << 17) | (uint32_t(M >> 4) << 24);
+}
+
+// Shared-memory descriptor of an MN-major, 128B-swizzled 16-bit tile: 64 MN
+// elements (128 B) per K row, 8 K rows per 1024-byte atom (SBO = 1024 B between
+// atoms along K), 64-element MN columns `lbo` bytes apart (LBO). A K step of 16
+// advances the start by 2048 B.
+__device__ __forceinline__ uint64_t sdesc_mn_sw128(uint32_t saddr, uint32_t lbo) {
+  return (uint64_t((saddr & 0x3FFFF) >> 4)) | (uint64_t(lbo >> 4) << 16) | (uint64_t(1024 >> 4) << 32) |
+         (uint64_t(1) << 46) | (uint64_t(2) << 61);
+}
+
 // Shared-memory descriptor for a K-major, 128-byte-swizzled bf16 tile: rows of
 // 64 elements (128 B), 8-row atoms of 1024 B stacked along M/N. The tile base
 // must be 1024-byte aligned; a K sub-step of 16 elements advances the start by 32 B.
@@ -366,6 +413,17 @@ __device__ __forceinline__ uint32_t bf16_to_f16_bits(uint32_t b) {
   return __half_as_ushort(__float2half_rn(__uint_as_float(b << 16)));
 }
 
+// As bf16_to_f16_bits, and sets `overflow` when the value does not fit fp16:
+// a magnitude of 2^16 or more (bf16 values below that fit, with their 8
+// significant bits), inf or nan. The check runs on the slow path only.
+__device__ __forceinline__ uint32_t bf16_to_f16_bits_chk(uint32_t b, bool& overflow) {
+  const uint32_t mag = b & 0x7FFFu;
+  if ((mag >> 7) - 113u <= 29u) return (b & 0x8000u) | ((mag << 3) - (112u << 10));
+  if (mag == 0u) return b & 0x8000u;
+  overflow |= (mag >> 7) > 127u + 15u;
+  return __half_as_ushort(__float2half_rn(__uint_as_float(b << 16)));
+}
+
 // 8 bf16 values (one 16-byte chunk) -> 8 fp16 values (exact within fp16 range).
 __device__ __forceinline__ uint4 bf16x8_to_f16x8(uint4 v) {
   const uint32_t w[4] = {v.x, v.y, v.z, v.w};
@@ -374,6 +432,19 @@ __device__ __forceinline__ uint4 bf16x8_to_f16x8(uint4 v) {
   for (int i = 0; i < 4; ++i) o[i] = bf16_to_f16_bits(w[i] & 0xFFFFu) | (bf16_to_f16_bits(w[i] >> 16) << 16);
   return make_uint4(o[0], o[1], o[2], o[3]);
 }
+
+// As bf16x8_to_f16x8, setting `overflow` for any value that does not fit fp16.
+__device__ __forceinline__ uint4 bf16x8_to_f16x8_chk(uint4 v, bool& overflow) {
+  const uint32_t w[4] = {v.x, v.y, v.z, v.w};
+  uint32_t o[4];
+#pragma unroll
+  for (int i = 0; i < 4; ++i)
+    o[i] = bf16_to_f16_bits_chk(w[i] & 0xFFFFu, overflow) | (bf16_to_f16_bits_chk(w[i] >> 16, overflow) << 16);
+  return make_uint4(o[0], o[1], o[2], o[3]);
+}
+
+// Nonzero when either fp16 half of the pair is inf or nan (exponent field all ones).
+__device__ __forceinline__ uint32_t f16x2_nonfinite(uint32_t w) { return __vcmpeq2(w & 0x7C007C00u, 0x7C007C00u); }
 
 // Byte offset of 16-byte chunk c (0..7) of row r inside a K-major SW128 tile.
 __device__ __forceinline__ uint32_t sw128_offset(uint32_t r, uint32_t c) {

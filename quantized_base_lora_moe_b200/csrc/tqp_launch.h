@@ -1,6 +1,7 @@
 // Internal launcher declarations shared by the kernel files and the C ABI.
 #pragma once
 
+#include <atomic>
 #include <cstddef>
 #include <cstdint>
 #include <cuda_runtime.h>
@@ -10,6 +11,30 @@
 namespace tqp {
 
 inline size_t align_up(size_t v, size_t a) { return (v + a - 1) / a * a; }
+
+// Per-device "done" bits of a one-time setting of a kernel (its dynamic
+// shared-memory limit): the attribute belongs to the kernel on the current
+// device, so a process that drives several GPUs sets it once on each.
+struct DeviceFlags {
+  std::atomic<unsigned long long> bits{0};
+  // Sets the kernel's dynamic shared-memory limit on the current device unless
+  // already done there; false if the runtime refused.
+  template <typename K>
+  bool test_and_set_device(K kernel, int smem_bytes) {
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess) return false;
+    const unsigned long long bit = dev < 64 ? (1ull << dev) : 0ull;
+    if (bit && (bits.load(std::memory_order_acquire) & bit)) return true;
+    if (cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, smem_bytes) != cudaSuccess)
+      return false;
+    bits.fetch_or(bit, std::memory_order_acq_rel);
+    return true;
+  }
+};
+
+// Limit of one device-side barrier wait for the next launches, in ns (0 = the
+// kernels' default). Set only through tqp_debug_set_wait_limit_ns.
+unsigned long long wait_limit_ns();
 
 // route / permute / combine
 int launch_route(const float* logits, int T, int E, int k, int32_t* ids, float* gates, int32_t* status,
@@ -55,13 +80,22 @@ int launch_dgrad(int which, const uint16_t* a_src, const uint16_t* a_lora, const
 int launch_rank_bwd(int which, const uint16_t* P, const int32_t* offsets, const int32_t* mb_prefix,
                     const tqp_moe_weights* w, int T, uint16_t* bk16, uint16_t* C, int32_t* status, cudaStream_t s);
 
-// backward pieces (layer_bwd.cu)
+// backward pieces (layer_bwd.cu). dmax holds max|dy| (launch_grad_absmax): the
+// fp16 intermediates are computed for dy * 2^P, and dx and the adapter
+// gradients are scaled back by 2^-P.
+int launch_grad_absmax(const float* dy, size_t n, uint32_t* dmax, cudaStream_t s);
 int launch_bwd_combine(const uint16_t* O, const int32_t* inv, const float* gates, const int32_t* ids,
-                       const float* router_w, const float* dy, int T, int k, int d, uint16_t* dO, float* dx,
-                       cudaStream_t s);
-int launch_gather_add(const uint16_t* dX, const int32_t* inv, int T, int k, int d, float* dx, cudaStream_t s);
+                       const float* router_w, const float* dy, int T, int k, int d, const uint32_t* dmax, uint16_t* dO,
+                       float* dx, int32_t* status, cudaStream_t s);
+int launch_gather_add(const uint16_t* dX, const int32_t* inv, int T, int k, int d, const uint32_t* dmax, float* dx,
+                      cudaStream_t s);
+// adapter gradients on the tensor cores (wgrad.cu); TQP_ERR_UNSUPPORTED for ranks above 32
+int launch_wgrad(const tqp_moe_weights* w, const int32_t* offsets, const int32_t* perm, const uint16_t* dO,
+                 const uint16_t* h, const uint16_t* dgu, const uint16_t* x16, const uint16_t* ha, const uint16_t* dha,
+                 const uint16_t* xa, const uint16_t* dxa, const tqp_adapter_grads* g, const uint32_t* dmax,
+                 int32_t* status, cudaStream_t s);
 int launch_outer(int E, int M, int N, const int32_t* offsets, const int32_t* perm, const uint16_t* P, int ldp,
-                 int offp, const uint16_t* Q, int ldq, int offq, float* C, cudaStream_t s);
+                 int offp, const uint16_t* Q, int ldq, int offq, float* C, const uint32_t* dmax, cudaStream_t s);
 
 int num_sms();
 

@@ -2,9 +2,9 @@
 
 The layer shards by tokens with replicated weights, so the forward has no
 exchange. The backward has one: every rank's adapter gradients dA, dB are
-summed over the ranks before the optimizer step. Only the adapters train
-("Optimizer state only on adapters", Principle 3 of "Reversible Sparse MoE
-Single Node"), so this is the only data that crosses GPUs.
+summed over the ranks before the optimizer step. Only the adapters train and
+only they carry optimizer state (Principle 3 of "Reversible Sparse MoE Single
+Node"), so this is the only data that crosses GPUs.
 
 FlatGrads keeps the six gradient tensors of one layer as views of a single
 fp32 buffer, so the exchange is one all-reduce per layer rather than six.
@@ -61,3 +61,33 @@ def allreduce_adapter_grads(grads, group=None, async_op: bool = False):
         return None
     work = dist.all_reduce(t, op=dist.ReduceOp.SUM, group=group, async_op=async_op)
     return work if async_op else None
+
+
+def adapter_dp_step(local_backward, grads, optimizer=None, group=None):
+    """One data-parallel training step of a layer's adapters.
+
+    local_backward(grads) fills `grads` with the gradients of this rank's token
+    shard (overwriting them); the buffer is then summed over the ranks with one
+    all-reduce, so every rank holds the gradient of the union of the shards
+    (each expert's adapter gradient is a sum over the rows routed to it, so the
+    shards' sums add up to the full batch's); finally optimizer.step(grads)
+    runs the same update on every rank, which keeps the replicas identical.
+    Every rank must call this with the same layer in the same order.
+    """
+    local_backward(grads)
+    allreduce_adapter_grads(grads, group)
+    if optimizer is not None:
+        optimizer.step(grads)
+    return grads
+
+
+def layer_dp_step(layer, x_shard, dy_shard, dx_shard, grads, optimizer=None, group=None, ws=None, status=None,
+                  stream=None):
+    """adapter_dp_step with the library's layer backward as the local step:
+    tqp_moe_layer_bwd on this rank's tokens (x_shard bf16, dy_shard fp32)."""
+    from . import tqp_moe_layer_bwd
+
+    def local(g):
+        tqp_moe_layer_bwd(x_shard, dy_shard, layer, dx_shard, g, ws=ws, status=status, stream=stream)
+
+    return adapter_dp_step(local, grads, optimizer, group)

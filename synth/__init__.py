@@ -58,6 +58,7 @@ class LayerConfig:
     lora_scale: float = 2.0   # alpha / r
     zipf_s: float = 0.0       # >0: additive router bias ln(p_e), p_e ~ (e+1)^-s
     seed: int = 0
+    w_mult: float = 1.0       # multiplies the base weights (before quantising) and LoRA B
 
     @property
     def A(self) -> int:
@@ -175,11 +176,12 @@ def proj_dims(cfg: LayerConfig, p: int) -> tuple[int, int]:
 def _expert_tensors(cfg: LayerConfig, seed: int, p: int, e: int):
     out, inn = proj_dims(cfg, p)
     std_w = np.float32(1.0 / np.sqrt(cfg.d))
-    w = _rng(seed, f"w{p}", e).standard_normal((out, inn), dtype=np.float32) * std_w
+    mult = np.float32(cfg.w_mult)
+    w = _rng(seed, f"w{p}", e).standard_normal((out, inn), dtype=np.float32) * std_w * mult
     codes, scales = quantise_int4(w, cfg.g)
     at = f32_to_bf16_bits(_rng(seed, f"a{p}", e).standard_normal((cfg.r, inn), dtype=np.float32) * std_w)
     bt = f32_to_bf16_bits(_rng(seed, f"b{p}", e).standard_normal((out, cfg.r), dtype=np.float32)
-                          * np.float32(0.1))
+                          * np.float32(0.1) * mult)
     return codes, scales, at, bt
 
 

@@ -174,6 +174,8 @@ def test_adapter_bwd_block_matches_oracle(cfgs):
         q = pert[key] if p is None else pert[key][p]
         spread = rel_err(q[sel], r[sel])
         err = rel_err(g[sel], r[sel])
+        print(f"SPREAD block-{cfgF.T}x{cfgF.d} {key}{'' if p is None else p}: err {err:.3e} spread {spread:.3e} "
+              f"bound {TOL + 2 * spread:.3e}")
         assert err <= TOL + 2 * spread, (key, p, err, spread)
 
     check("dx1", keep_t)
@@ -187,18 +189,32 @@ def test_adapter_bwd_block_matches_oracle(cfgs):
             check("dB_G", kG, p)
 
 
+_FULL_BLOCK = {}
+
+
+def full_block():
+    """The 460-expert top-12 block (F, G independent instances) at T=8192, run
+    once on the GPU (forward, then the adapter backward from its outputs)."""
+    if not _FULL_BLOCK:
+        cfgF, cfgG = synth.REV_F, synth.REV_G
+        rawF, rawG = synth.make_layer(cfgF, cfgF.seed), synth.make_layer(cfgG, cfgG.seed)
+        T, d = cfgF.T, cfgF.d
+        x1b = synth.make_tokens(T, d, synth.REV_SEEDS["x1"])
+        x2b = synth.make_tokens(T, d, synth.REV_SEEDS["x2"])
+        dy1 = synth.make_grad(T, d, synth.REV_SEEDS["dy"], "dy1")
+        dy2 = synth.make_grad(T, d, synth.REV_SEEDS["dy"], "dy2")
+        got = gpu_block(cfgF, cfgG, rawF, rawG, x1b, x2b, dy1, dy2)
+        _FULL_BLOCK.update(cfgF=cfgF, cfgG=cfgG, rawF=rawF, rawG=rawG, x1b=x1b, x2b=x2b, dy1=dy1, dy2=dy2, got=got)
+    return _FULL_BLOCK
+
+
 def test_adapter_bwd_full_size_reconstruction_and_sampled_tokens():
-    """The 460-expert top-12 block (F, G independent instances) at T=8192:
-    reconstruction over all tokens, and dx1/dx2 on sampled tokens against the
-    oracle evaluated token by token."""
-    cfgF, cfgG = synth.REV_F, synth.REV_G
-    rawF, rawG = synth.make_layer(cfgF, cfgF.seed), synth.make_layer(cfgG, cfgG.seed)
+    """The 460-expert top-12 block at T=8192: reconstruction over all tokens,
+    and dx1/dx2 on sampled tokens against the oracle evaluated token by token."""
+    fb = full_block()
+    cfgF, cfgG, rawF, rawG = fb["cfgF"], fb["cfgG"], fb["rawF"], fb["rawG"]
+    x1b, x2b, dy1, dy2, got = fb["x1b"], fb["x2b"], fb["dy1"], fb["dy2"], fb["got"]
     T, d = cfgF.T, cfgF.d
-    x1b = synth.make_tokens(T, d, synth.REV_SEEDS["x1"])
-    x2b = synth.make_tokens(T, d, synth.REV_SEEDS["x2"])
-    dy1 = synth.make_grad(T, d, synth.REV_SEEDS["dy"], "dy1")
-    dy2 = synth.make_grad(T, d, synth.REV_SEEDS["dy"], "dy2")
-    got = gpu_block(cfgF, cfgG, rawF, rawG, x1b, x2b, dy1, dy2)
     x1, x2 = O.bf16_to_f64(x1b), O.bf16_to_f64(x2b)
     rms = np.sqrt(np.mean(np.concatenate([x1, x2]) ** 2))
     assert max(np.max(np.abs(got["x1"] - x1)), np.max(np.abs(got["x2"] - x2))) / rms <= 5e-3
@@ -233,5 +249,106 @@ def test_adapter_bwd_full_size_reconstruction_and_sampled_tokens():
     s2 = rel_err(np.array(p2s), np.array(r2s))
     e1 = rel_err(np.array(g1), np.array(r1s))
     e2 = rel_err(np.array(g2), np.array(r2s))
+    print(f"SPREAD block-full sampled tokens {ok_rows}: dx1 err {e1:.3e} spread {s1:.3e}; "
+          f"dx2 err {e2:.3e} spread {s2:.3e}")
     assert e1 <= TOL + 2 * s1, (e1, s1)
     assert e2 <= TOL + 2 * s2, (e2, s2)
+
+
+def _pick_experts(counts, amb_per_expert, n_between=2):
+    """The busiest expert, the least-loaded non-empty one and n_between in
+    between, preferring among equals those that no ambiguous token touches."""
+    nz = np.nonzero(counts)[0]
+    order = nz[np.lexsort((amb_per_expert[nz], -counts[nz]))]     # busiest first, fewest ambiguous first
+    clean = [e for e in order if amb_per_expert[e] == 0] or list(order)
+    picks = [clean[0], clean[-1]]
+    for q in np.linspace(0, len(clean) - 1, n_between + 2)[1:-1]:
+        picks.append(clean[int(round(q))])
+    return list(dict.fromkeys(int(e) for e in picks))
+
+
+def _expert_grads(X, dO, L, e):
+    """The oracle's adapter gradients of expert e for its routed rows X and upstream dO."""
+    P = L.expert(e)
+    fwd = O.expert_forward(X, P, L.s)
+    res = O.expert_backward(X, dO, P, L.s, fwd)
+    return res["dA"], res["dB"]
+
+
+def _routed_rows(ids, gam, e):
+    t_idx, j_idx = np.nonzero(ids == e)
+    return t_idx, gam[t_idx, j_idx]
+
+
+def test_adapter_bwd_full_size_sampled_expert_gradients():
+    """dA and dB of F and G at full size, element by element, on sampled
+    experts (the busiest, the least-loaded non-empty one and two in between).
+
+    The oracle runs F's forward on every token in fp64, rounds y1 to bf16 for G
+    and routes G on it. An expert's gradient sums over the tokens routed to it,
+    so it is the oracle's expert backward over those tokens with dO = gate *
+    cotangent; for F the cotangent dz1 = dy1 + J_G^T dy2 is the oracle's layer
+    backward of G at those tokens. G reads bf16(y1), which carries the rounding
+    of F's output on either side: the bound is TOL plus twice the oracle's own
+    spread when F's output moves by 2^-8 relative (as in the mid-size block
+    test), printed beside every error."""
+    fb = full_block()
+    cfgF, cfgG, rawF, rawG = fb["cfgF"], fb["cfgG"], fb["rawF"], fb["rawG"]
+    x1, x2 = O.bf16_to_f64(fb["x1b"]), O.bf16_to_f64(fb["x2b"])
+    dy1, dy2 = fb["dy1"].astype(np.float64), fb["dy2"].astype(np.float64)
+    got = fb["got"]
+    LF, LG = O.Layer(rawF), O.Layer(rawG)
+    kF, kG = cfgF.k, cfgG.k
+    # F on every token (exact input x2), y1, G's input and routing
+    lF = O.router_logits(x2, LF)
+    idsF = O.topk(lF, kF)
+    gF = O.gates(lF, idsF)
+    f_out = O.layer_forward(x2, LF, ids=idsF)
+    y1 = x1 + f_out
+    z = O.round_bf16(y1)
+    rng = np.random.default_rng(11)
+    zp = O.round_bf16(x1 + f_out * (1.0 + 2.0 ** -8 * rng.uniform(-1.0, 1.0, f_out.shape)))
+    lG, lGp = O.router_logits(z, LG), O.router_logits(zp, LG)
+    idsG, idsGp = O.topk(lG, kG), O.topk(lGp, kG)
+    gG, gGp = O.gates(lG, idsG), O.gates(lGp, idsGp)
+    ambG_tok = np.any(idsG != idsGp, axis=1) | (O.routing_gap(lG, kG) < 1e-4)
+    ambF_tok = O.routing_gap(lF, kF) < 1e-4
+    E = cfgF.E
+    countsG = np.bincount(idsG.ravel(), minlength=E)
+    countsF = np.bincount(idsF.ravel(), minlength=E)
+    ambG_e = np.bincount(idsG[ambG_tok].ravel(), minlength=E)
+    ambF_e = np.bincount(idsF[ambF_tok | ambG_tok].ravel(), minlength=E)   # a G-ambiguous token moves dz1
+    picksG = _pick_experts(countsG, ambG_e)
+    picksF = _pick_experts(countsF, ambF_e)
+    assert len(picksG) >= 4 and len(picksF) >= 4
+
+    def check(name, g, r, q):
+        err, spread = rel_err(g, r), rel_err(q, r)
+        print(f"SPREAD block-full {name}: err {err:.3e} spread {spread:.3e} bound {TOL + 2 * spread:.3e}")
+        assert err <= TOL + 2 * spread, (name, err, spread)
+
+    # G: cotangent dy2, input z (perturbed: zp, with zp's own routing)
+    for e in picksG:
+        t, gam = _routed_rows(idsG, gG, e)
+        tp, gamp = _routed_rows(idsGp, gGp, e)
+        dA, dB = _expert_grads(z[t], gam[:, None] * dy2[t], LG, e)
+        dAp, dBp = _expert_grads(zp[tp], gamp[:, None] * dy2[tp], LG, e)
+        for p in range(3):
+            check(f"dA_G[{p}] expert {e} ({len(t)} rows)", got["dA_G"][p][e], dA[p], dAp[p])
+            check(f"dB_G[{p}] expert {e} ({len(t)} rows)", got["dB_G"][p][e], dB[p], dBp[p])
+    # F: cotangent dz1 = dy1 + J_G^T dy2 at the tokens of the picked experts
+    S = np.unique(np.concatenate([np.nonzero(np.any(idsF == e, axis=1))[0] for e in picksF]))
+    dz1 = np.zeros_like(dy1)
+    dz1p = np.zeros_like(dy1)
+    # one call over z and zp stacked (each row's input gradient is its own; every
+    # expert is decoded once)
+    dxG = O.layer_backward(np.concatenate([z[S], zp[S]]), np.concatenate([dy2[S], dy2[S]]), LG)[0]
+    dz1[S] = dy1[S] + dxG[:len(S)]
+    dz1p[S] = dy1[S] + dxG[len(S):]
+    for e in picksF:
+        t, gam = _routed_rows(idsF, gF, e)
+        dA, dB = _expert_grads(x2[t], gam[:, None] * dz1[t], LF, e)
+        dAp, dBp = _expert_grads(x2[t], gam[:, None] * dz1p[t], LF, e)
+        for p in range(3):
+            check(f"dA_F[{p}] expert {e} ({len(t)} rows)", got["dA_F"][p][e], dA[p], dAp[p])
+            check(f"dB_F[{p}] expert {e} ({len(t)} rows)", got["dB_F"][p][e], dB[p], dBp[p])

@@ -286,6 +286,9 @@ def test_grouped_ffn_skewed_and_empty_experts():
 
 @pytest.mark.parametrize("cfg", [synth.FULL, synth.SKEWED], ids=lambda c: c.name)
 def test_grouped_ffn_full_size_sampled_experts(cfg):
+    """Every row of at least 16 experts at full size: the busiest, the
+    least-loaded non-empty one, one whose rows span three or more of the down
+    kernel's 256-row blocks (when the load has one) and random others."""
     raw = host_layer(cfg)
     L = O.Layer(raw)
     xb = synth.make_tokens(cfg.T, cfg.d, cfg.seed)
@@ -293,17 +296,22 @@ def test_grouped_ffn_full_size_sampled_experts(cfg):
     ids = O.topk(O.router_logits(x, L), cfg.k)
     offsets, perm, _ = _ffn_case(cfg, x, L, ids)
     h, o = _run_ffn(cfg, xb, offsets, perm)
+    hg_all, og_all = host_f16(h), host_f16(o)
     counts = np.diff(offsets)
-    busiest = int(np.argmax(counts))
-    picks = [busiest, int(np.argmin(np.where(counts > 0, counts, 1 << 30))), 1, cfg.E - 1]
+    nz = np.nonzero(counts)[0]
+    picks = [int(np.argmax(counts)), int(nz[np.argmin(counts[nz])])]
+    wide = np.nonzero((counts > 512) & (counts <= 4096))[0]
+    if len(wide):
+        picks.append(int(wide[0]))
+    rng = np.random.default_rng(1)
+    picks += [int(e) for e in rng.choice(nz, 16, replace=False)]
+    picks = list(dict.fromkeys(picks))
+    assert len(picks) >= 16
     for e in picks:
         rows = np.arange(offsets[e], offsets[e + 1])
-        if len(rows) == 0:
-            continue
-        rows = rows[:600]
         out = O.expert_forward(x[perm[rows]], L.expert(e), L.s)
-        assert rel_err(host_f16(o[rows[0]:rows[-1] + 1]), out["o"]) <= TOL, e
-        assert rel_err(host_f16(h[rows[0]:rows[-1] + 1]), out["h"]) <= TOL, e
+        assert rel_err(og_all[rows], out["o"]) <= TOL, (e, len(rows))
+        assert rel_err(hg_all[rows], out["h"]) <= TOL, (e, len(rows))
 
 
 # ---------------------------------------------------------------- combine
@@ -374,6 +382,8 @@ def test_layer_fwd_deterministic():
 
 @pytest.mark.parametrize("cfg", [synth.FULL, synth.SKEWED], ids=lambda c: c.name)
 def test_layer_fwd_full_size_sampled_tokens(cfg):
+    """The whole layer at full size on 98 sampled tokens (the first, the last
+    and 96 random ones), the oracle run on that subset of rows."""
     raw = host_layer(cfg)
     L = O.Layer(raw)
     xb = synth.make_tokens(cfg.T, cfg.d, cfg.seed)
@@ -385,17 +395,12 @@ def test_layer_fwd_full_size_sampled_tokens(cfg):
     got = host_bf16(y)
     x = O.bf16_to_f64(xb)
     rng = np.random.default_rng(0)
-    toks = np.concatenate([[0, cfg.T - 1], rng.choice(cfg.T, 30, replace=False)])
-    ref = np.zeros((len(toks), cfg.d))
-    ok = np.ones(len(toks), bool)
-    for i, t in enumerate(toks):
-        yt, _, _, lt = O.token_forward(x[t], L)
-        ref[i] = yt
-        ok[i] = O.routing_gap(lt[None, :], cfg.k)[0] >= 1e-4
+    toks = np.unique(np.concatenate([[0, cfg.T - 1], rng.choice(np.arange(1, cfg.T - 1), 96, replace=False)]))
+    ref = O.layer_forward(x[toks], L)
+    ok = O.routing_gap(O.router_logits(x[toks], L), cfg.k) >= 1e-4
     assert ok.sum() >= len(toks) - 2
-    per_tok = [rel_err(got[t][None], ref[i][None]) for i, t in enumerate(toks)]
     err = rel_err_bf16_out(got[toks][ok], ref[ok])
-    assert err <= TOL, (err, np.round(per_tok, 4).tolist())
+    assert err <= TOL, err
     # every output row is finite and the whole batch was written
     assert np.isfinite(got).all()
 
@@ -454,6 +459,7 @@ def test_rev_couple_fwd_inverse(cfgs):
     spread = rel_err(gzp[keep], gz[keep])
     e1 = rel_err_bf16_out(y1.cpu().numpy()[keep] - x1[keep], f_ref[keep])
     e2 = rel_err_bf16_out(y2.cpu().numpy()[keep] - x2[keep], (o2 - x2)[keep])
+    print(f"SPREAD coupling-{T}x{d} y2: err {e2:.3e} spread {spread:.3e} bound {TOL + 2 * spread:.3e}")
     assert e1 <= TOL, e1
     assert e2 <= TOL + 2 * spread, (e2, spread)
 

@@ -137,3 +137,71 @@ def test_flat_gradient_views_alias_one_buffer():
     assert Q._grads(g) is g.struct                            # the backward calls take a FlatGrads as well
     r0 = FlatGrads(E=3, d=128, f=256, r=0, device="cpu")
     assert r0.flat.numel() == 0 and allreduce_adapter_grads(r0) is None
+
+
+class _OracleAdamW:
+    """CPU stand-in for AdapterAdamW in the gloo test: the oracle's AdamW on a
+    master copy in the flat gradient layout."""
+
+    def __init__(self, flat_init):
+        self.p = flat_init.astype(np.float64)
+        self.m = np.zeros_like(self.p)
+        self.v = np.zeros_like(self.p)
+        self.t = 0
+
+    def step(self, grads):
+        from oracle import tqp_oracle as O
+        self.t += 1
+        self.p, self.m, self.v = O.adamw_step(self.p, self.m, self.v, grads.flat.numpy().astype(np.float64), 1e-3,
+                                              0.9, 0.999, 1e-8, 0.01, self.t)
+
+
+def _dp_step_worker(rank, world, port, out):
+    """Each rank: the oracle's layer backward on its own token shard as the local
+    step, one all-reduce, the optimizer step; reports the summed gradient and
+    the updated parameters."""
+    os.environ["MASTER_ADDR"] = "127.0.0.1"
+    os.environ["MASTER_PORT"] = str(port)
+    import datetime
+    from oracle import tqp_oracle as O
+    from quantized_base_lora_moe_b200.dp import FlatGrads, adapter_dp_step
+    dist.init_process_group("gloo", rank=rank, world_size=world, timeout=datetime.timedelta(seconds=60))
+    try:
+        cfg = synth.LayerConfig("dp", T=96, d=64, E=6, k=2, f=64, g=32, r=8)
+        raw = synth.make_layer(cfg)
+        L = O.Layer(raw)
+        x = O.bf16_to_f64(synth.make_tokens(cfg.T, cfg.d, 7))
+        dy = synth.make_grad(cfg.T, cfg.d, 8, "dy1").astype(np.float64)
+        shard = slice(rank * cfg.T // world, (rank + 1) * cfg.T // world)
+        g = FlatGrads(cfg.E, cfg.d, cfg.f, cfg.r, device="cpu")
+
+        def local_backward(grads):
+            _, dA, dB = O.layer_backward(x[shard], dy[shard], L)
+            for p in range(3):
+                grads.dA[p].copy_(torch.from_numpy(dA[p]))
+                grads.dB[p].copy_(torch.from_numpy(dB[p]))
+
+        lora = np.concatenate([O.bf16_to_f64(raw[f"la{p}"]).ravel() for p in range(3)] +
+                              [O.bf16_to_f64(raw[f"lb{p}"]).ravel() for p in range(3)])
+        opt = _OracleAdamW(lora)
+        adapter_dp_step(local_backward, g, opt)
+        out[rank] = (g.flat.numpy().copy(), opt.p.copy())
+    finally:
+        dist.destroy_process_group()
+
+
+def test_data_parallel_step_sums_shards_to_the_full_batch_gradient():
+    from oracle import tqp_oracle as O
+    port = 33500 + (os.getpid() % 2000)
+    out = mp.Manager().dict()
+    mp.spawn(_dp_step_worker, args=(2, port, out), nprocs=2, join=True)
+    (g0, p0), (g1, p1) = out[0], out[1]
+    assert np.array_equal(g0, g1) and np.array_equal(p0, p1)     # identical replicas after the step
+    # the summed gradient is the gradient over the union of the shards
+    cfg = synth.LayerConfig("dp", T=96, d=64, E=6, k=2, f=64, g=32, r=8)
+    L = O.Layer(synth.make_layer(cfg))
+    x = O.bf16_to_f64(synth.make_tokens(cfg.T, cfg.d, 7))
+    dy = synth.make_grad(cfg.T, cfg.d, 8, "dy1").astype(np.float64)
+    _, dA, dB = O.layer_backward(x, dy, L)
+    full = np.concatenate([a.ravel() for a in dA] + [b.ravel() for b in dB])
+    assert np.max(np.abs(g0 - full)) <= 1e-5 * np.max(np.abs(full))   # fp32 buffer of fp64 sums

@@ -69,6 +69,28 @@ def _unscaled_lora_grad(X, dO, P, s, fwd):
     return res
 
 
+def _stack_grads_in_walk_order(y1, y2, dy1, dy2, blocks, round_inputs=True):
+    # the per-block gradients left in the order the backward walks the blocks
+    res = _orig_stack_backward(y1, y2, dy1, dy2, blocks, round_inputs)
+    res["grads"] = res["grads"][::-1]
+    return res
+
+
+def _stack_inverse_forward_order(y1, y2, blocks, round_inputs=True):
+    # undoes the blocks first to last instead of last to first
+    return _orig_stack_inverse(y1, y2, blocks[::-1], round_inputs)
+
+
+def _adamw_coupled_decay(p, m, v, g, lr, beta1, beta2, eps, weight_decay, t, grad_scale=1.0):
+    # L2-regularised Adam (decay folded into the gradient) instead of decoupled decay
+    p = np.asarray(p, dtype=np.float64)
+    return _orig_adamw_step(p, m, v, np.asarray(g, dtype=np.float64) + weight_decay * p, lr, beta1, beta2, eps, 0.0,
+                            t, grad_scale)
+
+
+_orig_adamw_step = O.adamw_step
+_orig_stack_backward = O.stack_backward
+_orig_stack_inverse = O.stack_inverse
 _orig_expert_forward = O.expert_forward
 _orig_topk = O.topk
 _orig_layer_backward = O.layer_backward
@@ -82,6 +104,9 @@ CASES = [
     ("coupling_inverse", _inverse_adds, pins.test_coupling_inverse_reconstructs_inputs),
     ("expert_backward", _skip_down_adapter_grad, pins.test_layer_backward_finite_differences),
     ("expert_backward", _unscaled_lora_grad, pins.test_layer_backward_finite_differences),
+    ("stack_backward", _stack_grads_in_walk_order, pins.test_stack_backward_finite_differences),
+    ("stack_inverse", _stack_inverse_forward_order, pins.test_stack_inverse_reconstructs_inputs),
+    ("adamw_step", _adamw_coupled_decay, pins.test_adamw_matches_torch_adamw_over_several_steps),
 ]
 
 

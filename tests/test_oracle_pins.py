@@ -431,3 +431,153 @@ def test_block_backward_finite_differences():
                 j = int(rng.integers(P[bn].shape[1]))
                 ref = fd(P[bn], (i, j))
                 assert abs(res[f"dB_{tag}"][p][e][j, i] - ref) <= 1e-6 * max(1.0, abs(ref))
+
+
+# ---------------------------------------------------------------- reversible stack
+
+
+def _stack_blocks(L, cfg=SMALL):
+    """L blocks of independent small layers (seeds 0, 1, ..., 2L-1)."""
+    return [(O.Layer(synth.make_layer(dataclasses.replace(cfg, seed=2 * l), 2 * l)),
+             O.Layer(synth.make_layer(dataclasses.replace(cfg, seed=2 * l + 1), 2 * l + 1))) for l in range(L)]
+
+
+def test_stack_of_one_block_is_the_coupling():
+    # with one block the stack is the (separately pinned) coupling and its backward
+    blocks = _stack_blocks(1)
+    F, G = blocks[0]
+    x1, x2 = tokens(SMALL, 2), tokens(SMALL, 3)
+    rng = np.random.default_rng(21)
+    dy1, dy2 = rng.standard_normal(x1.shape), rng.standard_normal(x1.shape)
+    s1, s2 = O.stack_forward(x1, x2, blocks)
+    c1, c2 = O.coupling_forward(x1, x2, F, G)
+    assert rel(s1, c1) <= 1e-14 and rel(s2, c2) <= 1e-14
+    st = O.stack_backward(s1, s2, dy1, dy2, blocks)
+    bl = O.block_backward(c1, c2, dy1, dy2, F, G)
+    for key in ("x1", "x2", "dx1", "dx2"):
+        assert rel(st[key], bl[key]) <= 1e-12, key
+    for i, key in enumerate(("dA_F", "dB_F", "dA_G", "dB_G")):
+        for p in range(3):
+            assert rel(st["grads"][0][i][p], bl[key][p]) <= 1e-12, (key, p)
+
+
+def test_stack_inverse_reconstructs_inputs():
+    blocks = _stack_blocks(3)
+    x1, x2 = tokens(SMALL, 2), tokens(SMALL, 3)
+    y1, y2 = O.stack_forward(x1, x2, blocks)
+    assert rel(y1, x1) > 1e-3                     # the stack does change the streams
+    r1, r2 = O.stack_inverse(y1, y2, blocks)
+    # exact up to fp64 rounding: each subtraction loses at most half an ulp of
+    # the larger stream, and these small random layers let the streams grow
+    bound = 8 * 3 * 2.0 ** -52 * max(np.abs(y1).max(), np.abs(y2).max())
+    assert np.abs(r1 - x1).max() <= bound and np.abs(r2 - x2).max() <= bound
+
+
+def test_stack_reversible_backward_equals_stored():
+    blocks = _stack_blocks(3)
+    x1, x2 = tokens(SMALL, 2), tokens(SMALL, 3)
+    rng = np.random.default_rng(22)
+    dy1, dy2 = rng.standard_normal(x1.shape), rng.standard_normal(x1.shape)
+    y1, y2 = O.stack_forward(x1, x2, blocks)
+    rev = O.stack_backward(y1, y2, dy1, dy2, blocks)
+    sto = O.stack_backward_stored(x1, x2, dy1, dy2, blocks)
+    bound = 8 * 3 * 2.0 ** -52 * max(np.abs(y1).max(), np.abs(y2).max())
+    assert np.abs(rev["x1"] - x1).max() <= bound and np.abs(rev["x2"] - x2).max() <= bound
+    for key in ("dx1", "dx2"):
+        assert rel(rev[key], sto[key]) <= 1e-9, key
+    for l in range(3):
+        for i in range(4):
+            for p in range(3):
+                assert rel(rev["grads"][l][i][p], sto["grads"][l][i][p]) <= 1e-9, (l, i, p)
+
+
+def test_stack_backward_finite_differences():
+    # central differences of <dy1, y1> + <dy2, y2> through two blocks (bf16
+    # roundings of the layer inputs off, so that the loss is smooth)
+    blocks = _stack_blocks(2)
+    x1, x2 = tokens(SMALL, 2), tokens(SMALL, 3)
+    rng = np.random.default_rng(23)
+    dy1, dy2 = rng.standard_normal(x1.shape), rng.standard_normal(x1.shape)
+    y1, y2 = O.stack_forward(x1, x2, blocks, round_inputs=False)
+    res = O.stack_backward(y1, y2, dy1, dy2, blocks, round_inputs=False)
+    eps = 1e-6
+
+    def loss():
+        u1, u2 = O.stack_forward(x1, x2, blocks, round_inputs=False)
+        return float(np.sum(dy1 * u1) + np.sum(dy2 * u2))
+
+    def fd(arr, idx):
+        old = arr[idx]
+        arr[idx] = old + eps
+        lp = loss()
+        arr[idx] = old - eps
+        lm = loss()
+        arr[idx] = old
+        return (lp - lm) / (2 * eps)
+
+    for _ in range(6):
+        t = int(rng.integers(SMALL.T))
+        i = int(rng.integers(SMALL.d))
+        for arr, key in ((x1, "dx1"), (x2, "dx2")):
+            ref = fd(arr, (t, i))
+            assert abs(res[key][t, i] - ref) <= 1e-6 * max(1.0, abs(ref)), (key, t, i)
+    for l, (F, G) in enumerate(blocks):
+        for Lyr, gi in ((F, 0), (G, 2)):
+            e = int(rng.integers(SMALL.E))
+            P = Lyr.expert(e)
+            for p, (an, bn) in enumerate((("Ag", "Bg"), ("Au", "Bu"), ("Ad", "Bd"))):
+                i = int(rng.integers(P[an].shape[0]))
+                j = int(rng.integers(P[an].shape[1]))
+                ref = fd(P[an], (i, j))
+                assert abs(res["grads"][l][gi][p][e][j, i] - ref) <= 1e-6 * max(1.0, abs(ref)), (l, gi, p)
+                i = int(rng.integers(P[bn].shape[0]))
+                j = int(rng.integers(P[bn].shape[1]))
+                ref = fd(P[bn], (i, j))
+                assert abs(res["grads"][l][gi + 1][p][e][j, i] - ref) <= 1e-6 * max(1.0, abs(ref)), (l, gi + 1, p)
+
+
+# ---------------------------------------------------------------- adapter optimizer
+
+
+def test_adamw_matches_torch_adamw_over_several_steps():
+    # torch.optim.AdamW implements the same update (decoupled weight decay,
+    # bias-corrected moments); run both in fp64 on the same gradient sequence
+    import torch
+    rng = np.random.default_rng(41)
+    n = 257
+    p0 = rng.standard_normal(n) * 0.05
+    lr, b1, b2, eps, wd = 3e-3, 0.9, 0.999, 1e-8, 0.01
+    tp = torch.nn.Parameter(torch.tensor(p0, dtype=torch.float64))
+    opt = torch.optim.AdamW([tp], lr=lr, betas=(b1, b2), eps=eps, weight_decay=wd)
+    p, m, v = p0.copy(), np.zeros(n), np.zeros(n)
+    for t in range(1, 7):
+        g = rng.standard_normal(n) * (0.1 if t % 2 else 3.0)
+        tp.grad = torch.tensor(g, dtype=torch.float64)
+        opt.step()
+        p, m, v = O.adamw_step(p, m, v, g, lr, b1, b2, eps, wd, t)
+        st = opt.state[tp]
+        assert np.max(np.abs(p - tp.detach().numpy())) <= 1e-14
+        assert np.max(np.abs(m - st["exp_avg"].numpy())) <= 1e-15
+        assert np.max(np.abs(v - st["exp_avg_sq"].numpy())) <= 1e-15
+
+
+def test_adamw_first_step_and_weight_decay_closed_forms():
+    rng = np.random.default_rng(42)
+    n = 64
+    p0 = rng.standard_normal(n)
+    g = rng.standard_normal(n)
+    lr, b1, b2, eps, wd = 1e-2, 0.8, 0.95, 1e-6, 0.1
+    # step 1: the bias-corrected moments are g and g^2
+    p, m, v = O.adamw_step(p0, np.zeros(n), np.zeros(n), g, lr, b1, b2, eps, wd, 1)
+    assert np.allclose(p, p0 - lr * (g / (np.abs(g) + eps) + wd * p0), rtol=0, atol=1e-15)
+    assert np.allclose(m, (1 - b1) * g, rtol=0, atol=1e-16) and np.allclose(v, (1 - b2) * g * g, rtol=0, atol=1e-16)
+    # no gradient: only the decoupled decay acts, p <- p (1 - lr wd) each step
+    q, mq, vq = p0.copy(), np.zeros(n), np.zeros(n)
+    for t in range(1, 5):
+        q, mq, vq = O.adamw_step(q, mq, vq, np.zeros(n), lr, b1, b2, eps, wd, t)
+    assert np.allclose(q, p0 * (1 - lr * wd) ** 4, rtol=1e-15, atol=0)
+    # grad_scale multiplies the gradient before anything else
+    a = O.adamw_step(p0, np.zeros(n), np.zeros(n), g, lr, b1, b2, eps, wd, 1, grad_scale=0.5)
+    b = O.adamw_step(p0, np.zeros(n), np.zeros(n), 0.5 * g, lr, b1, b2, eps, wd, 1)
+    for x, y in zip(a, b):
+        assert np.array_equal(x, y)
