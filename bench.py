@@ -24,6 +24,7 @@ call timed with CUDA events outside the headline region.
 from __future__ import annotations
 
 import argparse
+import dataclasses
 import json
 import os
 import statistics
@@ -71,7 +72,7 @@ def layer_bwd_flops(cfg: synth.LayerConfig) -> float:
 
 def workload_config(cfg: synth.LayerConfig) -> dict:
     """The workload as both arms report it in `config`."""
-    return {"workload": f"{cfg.name}: T={cfg.T} d={cfg.d} E={cfg.E} top-{cfg.k} ffn={cfg.f} int4 g{cfg.g} LoRA r{cfg.r}"
+    return {"workload": f"{cfg.name}: T={cfg.T} d={cfg.d} E={cfg.E} top-{cfg.k} ffn={cfg.f} int{cfg.bits} g{cfg.g} LoRA r{cfg.r}"
                         f"{' zipf-bias' if cfg.zipf_s else ''}, layer forward",
             "T": cfg.T, "d": cfg.d, "E": cfg.E, "k": cfg.k, "ffn": cfg.f, "group": cfg.g, "rank": cfg.r}
 
@@ -200,18 +201,18 @@ class ClockSampler:
 # ---------------------------------------------------------------- GPU arm
 
 
-def time_rev_block(L_F, dev, steps: int, warmup: int, flush) -> dict:
-    """The reversible block at full size, timed per call with CUDA events.
+def time_rev_block(L_F, cfgF: synth.LayerConfig, dev, steps: int, warmup: int, flush) -> dict:
+    """The reversible block, timed per call with CUDA events.
 
-    F is the bench's 460-expert layer, G a second independent instance (seed 1);
-    streams x1, x2 of T x d bf16 and upstream gradients dy1, dy2 ~ N(0, 1) fp32.
+    F is the bench's layer, G a second independent instance (seed 1); streams
+    x1, x2 of T x d bf16 and upstream gradients dy1, dy2 ~ N(0, 1) fp32.
     One block step is rev_couple_fwd then tqp_adapter_bwd, which reconstructs
     x1, x2 with the inverse coupling before the adapter gradients; the inverse
     alone (rev_couple_inv) is timed beside it. L2 is flushed before each call.
     """
     import torch
     import quantized_base_lora_moe_b200 as Q
-    cfgF, cfgG = synth.REV_F, synth.REV_G
+    cfgG = synth.REV_G if cfgF == synth.FULL else dataclasses.replace(cfgF, name=cfgF.name + "_g", seed=1)
     G = Q.DeviceLayer(synth.make_layer(cfgG, cfgG.seed), device=dev)
     T, d = cfgF.T, cfgF.d
     tok = lambda seed: torch.from_numpy(synth.make_tokens(T, d, seed).view(np.int16)).to(dev)
@@ -266,12 +267,84 @@ def time_rev_block(L_F, dev, steps: int, warmup: int, flush) -> dict:
             "reconstruction_max_err_rel_rms": err, "l2": "flushed before every call"}
 
 
+def time_stack(dev, flush, depths=(1, 2, 4, 8)) -> dict:
+    """The reversible stack against its depth L at full size: peak device
+    memory, workspace, time of the forward and of the backward from the outputs
+    alone, and the reconstruction error of the inputs.
+
+    The blocks are built from two full-size layers F, G (460 experts, top-12,
+    T = 8192, d = 2048) whose base weights and LoRA B are scaled by 1/2, so
+    that the un-normalised SwiGLU branches stay small against the streams over
+    8 blocks (at scale 1 they grow quadratically from block to block). Every
+    block uses the same two weight sets; each layer of each block has its own
+    adapter-gradient buffers. The activation memory is measured with torch's
+    allocator statistics over one forward + backward, beyond the weights, the
+    gradient buffers and the call's inputs and outputs (so: the workspace and
+    anything transient); a store-everything backward would instead keep every
+    block's input streams and every layer's saved intermediates.
+    """
+    import torch
+    import quantized_base_lora_moe_b200 as Q
+    cfgF = dataclasses.replace(synth.FULL, name="stack_f", w_mult=0.5)
+    cfgG = dataclasses.replace(synth.FULL, name="stack_g", seed=1, w_mult=0.5)
+    F = Q.DeviceLayer(synth.make_layer(cfgF, cfgF.seed), device=dev)
+    G = Q.DeviceLayer(synth.make_layer(cfgG, cfgG.seed), device=dev)
+    T, d = cfgF.T, cfgF.d
+    tok = lambda seed: torch.from_numpy(synth.make_tokens(T, d, seed).view(np.int16)).to(dev)
+    x1, x2 = tok(synth.REV_SEEDS["x1"]), tok(synth.REV_SEEDS["x2"])
+    dy1 = torch.from_numpy(synth.make_grad(T, d, synth.REV_SEEDS["dy"], "dy1")).to(dev)
+    dy2 = torch.from_numpy(synth.make_grad(T, d, synth.REV_SEEDS["dy"], "dy2")).to(dev)
+    f32 = lambda: torch.empty(T, d, dtype=torch.float32, device=dev)
+    y1, y2, dx1, dx2 = f32(), f32(), f32(), f32()
+    r1, r2 = torch.empty_like(x1), torch.empty_like(x2)
+    st = Q.Status(dev)
+    stream = torch.cuda.current_stream(dev)
+    lib = Q.lib()
+    per_layer_bwd_ws = max(lib.tqp_moe_layer_bwd_workspace_size(T, F.ref()), lib.tqp_moe_layer_bwd_workspace_size(T, G.ref()))
+    out = {"workload": "L blocks of two full-size layers (460 experts, top-12, T=8192, d=2048; base weights and "
+                       "LoRA B x 1/2), fp32 streams between blocks", "depths": {}}
+    bf = lambda t: t.view(torch.bfloat16).float()
+    rms = float(torch.sqrt(torch.mean(torch.cat([bf(x1), bf(x2)]) ** 2)))
+    for L in depths:
+        stack = Q.ReversibleStack([F] * L, [G] * L)
+        gF, gG, arrays = stack.grads(dev)
+        torch.cuda.synchronize(dev)
+        base = torch.cuda.memory_allocated(dev)      # weights, gradient buffers, inputs and outputs
+        torch.cuda.reset_peak_memory_stats(dev)
+        ws = Q.workspace(stack.workspace_size(T), dev)
+        ms = {"fwd": [], "bwd": []}
+        for i in range(2):                     # the first pass is the warm-up
+            for name, call in (("fwd", lambda: Q.rev_stack_fwd(x1, x2, stack, y1, y2, ws, st)),
+                               ("bwd", lambda: Q.rev_stack_bwd(y1, y2, dy1, dy2, stack, r1, r2, dx1, dx2, arrays,
+                                                              ws, st))):
+                flush.zero_()
+                e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+                e0.record(stream)
+                call()
+                e1.record(stream)
+                e1.synchronize()
+                if i:
+                    ms[name].append(e0.elapsed_time(e1))
+        peak = torch.cuda.max_memory_allocated(dev) - base
+        if st.read() != 0:
+            raise RuntimeError(f"device status {st.read()} in the reversible stack (L={L})")
+        err = float(max((bf(r1) - bf(x1)).abs().max(), (bf(r2) - bf(x2)).abs().max())) / rms
+        store_all = L * (2 * T * d * 4 + 2 * per_layer_bwd_ws)
+        out["depths"][str(L)] = {"fwd_ms": ms["fwd"][0], "bwd_ms": ms["bwd"][0],
+                                 "workspace_bytes": ws.numel(), "peak_activation_bytes": peak,
+                                 "store_all_estimate_bytes": store_all,
+                                 "reconstruction_max_err_rel_rms": err}
+        del stack, gF, gG, arrays, ws
+        torch.cuda.empty_cache()
+    return out
+
+
 def layer_bytes(cfg: synth.LayerConfig, touched: int) -> float:
-    """Algorithmic bytes of one layer forward: int4 codes, bf16 group scales and
+    """Algorithmic bytes of one layer forward: int4 (or int8) codes, bf16 group scales and
     bf16 LoRA factors of the touched experts, fp32 router weights, x and y in
     bf16, ids and gates. Intermediates (logits, H, O) are implementation traffic."""
     d, f, g, r = cfg.d, cfg.f, cfg.g, cfg.r
-    per_expert = 3 * d * f / 2 + (2 * (d // g) * f + (f // g) * d) * 2 + 3 * r * (d + f) * 2
+    per_expert = 3 * d * f * cfg.bits / 8 + (2 * (d // g) * f + (f // g) * d) * 2 + 3 * r * (d + f) * 2
     return touched * per_expert + cfg.E * d * 4 + 2 * cfg.T * d * 2 + cfg.T * cfg.k * 8
 
 
@@ -526,9 +599,18 @@ def run_tqp(args, rank: int, world: int, local_rank: int) -> dict | None:
         extra["skewed"] = sk.summary(sk.run(n, args.warmup, flush))
         del sk
         torch.cuda.empty_cache()
+        i8cfg = dataclasses.replace(synth.FULL, name="full_int8", bits=8)
+        i8 = LayerBench(i8cfg, dev, i8cfg.seed)
+        extra["full_int8"] = i8.summary(i8.run(n, args.warmup, flush))
+        del i8
+        torch.cuda.empty_cache()
         result["configs"] = extra
-    if world == 1 and args.config == "full" and not args.no_rev:
-        result["rev_block"] = time_rev_block(lb.L, dev, min(args.steps, 5), 2, flush)
+    if world == 1 and not args.no_rev:
+        result["rev_block"] = time_rev_block(lb.L, cfg, dev, min(args.steps, 5), 2, flush)
+    if world == 1 and args.config == "full" and not args.no_stack:
+        del lb
+        torch.cuda.empty_cache()
+        result["rev_stack"] = time_stack(dev, flush)
     if world == 1 and not args.no_cpu_baseline:
         sample = min(T, args.cpu_sample)
         result["cpu_baseline"] = time_oracle(cfg, lb.host, lb.x_bits, sample)
@@ -571,6 +653,7 @@ def main():
     ap.add_argument("--no-rev", action="store_true", help="skip timing the reversible block (forward, inverse, "
                                                              "adapter backward)")
     ap.add_argument("--no-extra-configs", action="store_true", help="skip the mid and skewed configurations")
+    ap.add_argument("--no-stack", action="store_true", help="skip the reversible stack's memory and time against depth")
     args = ap.parse_args()
     rank = int(os.environ.get("RANK", 0))
     world = int(os.environ.get("WORLD_SIZE", 1))

@@ -60,16 +60,25 @@
  *   router_w   [E][d] fp32.
  *   router_bias[E] fp32 or NULL: additive per-expert bias, added to the logits
  *              before top-k and gates.
- *   wq[p]      [E][out_p][in_p/2] uint8: int4 codes of the frozen base weight
- *              W_p[out][in]. Each little-endian 32-bit word holds 8 consecutive
- *              input positions k0..k7 of one output row as two's-complement
- *              nibbles: k(2i) in bits [4i,4i+4), k(2i+1) in bits [16+4i,16+4i+4).
+ *   wq[p]      bits = 4: [E][out_p][in_p/2] uint8: int4 codes of the frozen base
+ *              weight W_p[out][in]. Each little-endian 32-bit word holds 8
+ *              consecutive input positions k0..k7 of one output row as
+ *              two's-complement nibbles: k(2i) in bits [4i,4i+4), k(2i+1) in bits
+ *              [16+4i,16+4i+4).
+ *              bits = 8: [E][out_p][in_p] int8 codes (two's complement), one per
+ *              input position (TQP Quantization: base weights int8 or int4).
  *   wscale[p]  [E][in_p/group][out_p] bf16: W_p[n][k] = q[n][k] * wscale[k/group][n].
  *   lora_a[p]  [E][rank][in_p] bf16: A_p^T.
  *   lora_b[p]  [E][out_p][rank] bf16: B_p^T.
  *   The projection is  x -> x W_p^T + lora_scale * (x A_p) B_p.
  *
+ * Exactness: int4 codes times bf16 scales are exact in fp16, so the expert
+ * contractions run on the exact dequantised weights; int8 codes times bf16
+ * scales (up to 15 significant bits) are rounded once to fp16 (relative error
+ * at most 2^-11 per weight).
+ *
  * Validity (host-checked, else TQP_ERR_INVALID_ARG / TQP_ERR_UNSUPPORTED):
+ *   bits in {0, 4, 8}, and ffn % 128 == 0 for bits = 8;
  *   1 <= top_k <= E <= 4096; d % 128 == 0; ffn % 64 == 0; 64 <= d, ffn <= 16384;
  *   group in {32, 64, 128, 256} dividing d and ffn; rank % 8 == 0 and
  *   0 <= rank <= 64 (rank 0 skips the adapter path); T >= 0 (T == 0 is a no-op).
@@ -112,6 +121,7 @@ typedef struct tqp_moe_weights {
   const uint16_t* wscale[3];
   const uint16_t* lora_a[3];
   const uint16_t* lora_b[3];
+  int bits;         /* base-weight code width: 4 (0 also means 4) or 8 */
 } tqp_moe_weights;
 
 /* Adapter gradients of one layer, fp32, same layouts as lora_a / lora_b:

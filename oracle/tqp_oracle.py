@@ -82,12 +82,19 @@ def unpack_int4(codes) -> np.ndarray:
     return out.reshape(c.shape[:-1] + (K,))
 
 
-def dequant(codes, scales, g: int) -> np.ndarray:
+def unpack_int8(codes) -> np.ndarray:
+    """int8 codes [..., K] (two's-complement bytes) -> signed integers [..., K]."""
+    return np.ascontiguousarray(codes, dtype=np.uint8).view(np.int8).astype(np.int64)
+
+
+def dequant(codes, scales, g: int, bits: int = 4) -> np.ndarray:
     """Dequantised weight W[n, k] = q[n, k] * scale[k // g, n], exact in fp64.
 
-    codes [out][in/2] (packed), scales [in/g][out] bf16 bits.
+    codes [out][in/2] (packed int4) or [out][in] (int8, bits = 8), scales
+    [in/g][out] bf16 bits. Base expert weights are stored as int8 or int4
+    ("TQP Quantization").
     """
-    q = unpack_int4(codes).astype(np.float64)
+    q = (unpack_int4(codes) if bits == 4 else unpack_int8(codes)).astype(np.float64)
     s = bf16_to_f64(scales)                      # [in/g][out]
     return q * np.repeat(s.T, g, axis=1)
 
@@ -109,6 +116,7 @@ class Layer:
         cfg = raw["cfg"]
         self.raw = raw
         self.E, self.d, self.f, self.g, self.r = cfg.E, cfg.d, cfg.f, cfg.g, cfg.r
+        self.bits = getattr(cfg, "bits", 4)
         self.k = cfg.k
         self.s = float(cfg.lora_scale)
         self.router_w = np.asarray(raw["router_w"], dtype=np.float64)   # [E][d]
@@ -125,7 +133,7 @@ class Layer:
         raw = self.raw
         p_ = {}
         for p, name in enumerate(("g", "u", "d")):
-            p_[f"W{name}"] = dequant(raw[f"wq{p}"][e], raw[f"ws{p}"][e], self.g)
+            p_[f"W{name}"] = dequant(raw[f"wq{p}"][e], raw[f"ws{p}"][e], self.g, self.bits)
             p_[f"A{name}"] = bf16_to_f64(raw[f"la{p}"][e]).T          # [in][r]
             p_[f"B{name}"] = bf16_to_f64(raw[f"lb{p}"][e]).T          # [r][out]
         p_.update(self.overrides.get(e, {}))

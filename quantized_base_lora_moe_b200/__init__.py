@@ -48,7 +48,7 @@ class Weights(ctypes.Structure):
         ("rank", ctypes.c_int), ("top_k", ctypes.c_int), ("lora_scale", ctypes.c_float),
         ("router_w", ctypes.c_void_p), ("router_bias", ctypes.c_void_p),
         ("wq", ctypes.c_void_p * 3), ("wscale", ctypes.c_void_p * 3),
-        ("lora_a", ctypes.c_void_p * 3), ("lora_b", ctypes.c_void_p * 3),
+        ("lora_a", ctypes.c_void_p * 3), ("lora_b", ctypes.c_void_p * 3), ("bits", ctypes.c_int),
     ]
 
 
@@ -201,6 +201,7 @@ class DeviceLayer:
         self.E, self.d, self.f, self.g, self.r = cfg.E, cfg.d, cfg.f, cfg.g, cfg.r
         self.k = top_k or cfg.k
         self.s = float(cfg.lora_scale)
+        self.bits = int(getattr(cfg, "bits", 4))
         self.router_w = torch.from_numpy(np.ascontiguousarray(host["router_w"], np.float32)).to(device)
         self.bias = None if host.get("bias") is None else torch.from_numpy(
             np.ascontiguousarray(host["bias"], np.float32)).to(device)
@@ -225,6 +226,7 @@ class DeviceLayer:
             w = Weights()
             w.E, w.d, w.ffn, w.group, w.rank, w.top_k = self.E, self.d, self.f, self.g, self.r, self.k
             w.lora_scale = self.s
+            w.bits = self.bits
             w.router_w = self.router_w.data_ptr()
             w.router_bias = _ptr(self.bias)
             for p in range(3):

@@ -24,13 +24,13 @@
 //               16-byte row pieces (the single accumulator is released after
 //               half the drain time)
 //   warp  4     TMEM allocation + one thread issuing tcgen05.mma
-//   warp  5     TMA producer of the int4 code / bf16 scale ring (32B-swizzled
-//               code rows, read without bank conflicts)
+//   warp  5     TMA producer of the code / bf16 scale ring (int4 rows
+//               32B-swizzled, int8 rows 64B-swizzled, read without bank conflicts)
 //   warps 6-9   token producer: two TMA boxes of 128 rows per 64-wide K stage;
 //               the rank-space rows (s H Ad) by coalesced cp.async
 //   warps 10-25 weight producer, two groups of 8 warps on alternate stages:
 //               each thread dequantises 32 K values of one weight row
-//               (int4 -> fp16) into TMEM; LoRA B rows
+//               (int4 or int8 -> fp16) into TMEM; LoRA B rows
 // TMEM (512 columns): one accumulator in [0, 256), 8 weight stages of 32
 // columns (64 K values) in [256, 512). Token ring: 3 stages of 32 KB.
 // An O value of a routed row or a LoRA B value beyond the fp16 range raises
@@ -62,15 +62,14 @@ constexpr int kXStageBytes = kRows * kK * 2;   // 256 rows x 128 B, 128B-swizzle
 constexpr int kWStages = 8;
 constexpr uint32_t kWCols = 32;        // TMEM columns per weight stage
 constexpr uint32_t kWBase = 256;
-constexpr int kQStages = 8;
-constexpr int kQStageBytes = 4608;     // 128 rows x 32 B of codes + up to 2 x 128 scales
+constexpr int kQStagesMax = 8;
 constexpr int kDRow = 528;             // drain row: 256 tokens in fp16 + 16 B against bank conflicts
 constexpr int kStaging = 128 * kDRow + 2 * 32 * kTRow;   // drain rows + one chunk tile per epilogue group
 
 struct Ctl {
   uint64_t x_full[kXStages], x_empty[kXStages];
   uint64_t w_full[kWStages], w_empty[kWStages];
-  uint64_t q_full[kQStages], q_empty[kQStages];
+  uint64_t q_full[kQStagesMax], q_empty[kQStagesMax];
   uint64_t acc_full, acc_empty;
   uint64_t drain;
   uint64_t epi[2];
@@ -78,13 +77,35 @@ struct Ctl {
   Abort ab;
 };
 
-constexpr size_t kSmemBytes = 1024 + size_t(kXStages) * kXStageBytes + size_t(kQStages) * kQStageBytes +
-                              size_t(kStaging) + sizeof(Ctl);
-static_assert(kSmemBytes + 2 * (kSchedSmemE + 1) * 4 <= 232448, "shared memory budget");
+// Code ring per code width: a stage holds 64 K values of 128 weight rows (32 B
+// per row for int4, 64 B for int8; TMA 32B / 64B swizzle) and up to 2 x 128 scales.
+template <int BITS>
+struct QCfg {
+  static constexpr int kCB = 8 * BITS;                 // code bytes per row and stage
+  static constexpr int kStages = BITS == 4 ? 8 : 4;
+  static constexpr int kStageBytes = 128 * kCB + 512;
+  // 16-byte chunk c of row r, as the TMA swizzle placed it
+  __device__ static __forceinline__ int chunk_offset(int r, int c) {
+    return r * kCB + ((BITS == 4 ? (c ^ ((r >> 2) & 1)) : (c ^ ((r >> 1) & 3))) << 4);
+  }
+};
 
+template <int BITS>
+constexpr size_t smem_bytes() {
+  return 1024 + size_t(kXStages) * kXStageBytes + size_t(QCfg<BITS>::kStages) * QCfg<BITS>::kStageBytes +
+         size_t(kStaging) + sizeof(Ctl);
+}
+static_assert(smem_bytes<4>() + 2 * (kSchedSmemE + 1) * 4 <= 232448, "shared memory budget");
+static_assert(smem_bytes<8>() + 2 * (kSchedSmemE + 1) * 4 <= 232448, "shared memory budget");
+
+template <int BITS>
 __global__ void __launch_bounds__(kThreads, 1)
     down_wide_kernel(const GemmArgs a, const __grid_constant__ CUtensorMap tq, const __grid_constant__ CUtensorMap ts,
                      const __grid_constant__ CUtensorMap th) {
+  using QC = QCfg<BITS>;
+  constexpr int kQStages = QC::kStages;
+  constexpr int kQStageBytes = QC::kStageBytes;
+  constexpr int kCB = QC::kCB;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   uint8_t* x_base = smem;
@@ -244,7 +265,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     if (lane == 0) {
       Ring q;
       PendingFills pend;
-      const uint32_t bytes = uint32_t(4096 + 256 * ngrp);
+      const uint32_t bytes = uint32_t(128 * kCB + 256 * ngrp);
       const int gpe = a.in_dim / a.g;
       for (int u = blockIdx.x; u < nunits; u += gridDim.x) {
         const Unit un = us.take(u);
@@ -255,8 +276,8 @@ __global__ void __launch_bounds__(kThreads, 1)
           uint8_t* qs = q_base + size_t(q.stage) * kQStageBytes;
           uint64_t* bar = &ctl->q_full[q.stage];
           mbar_arrive_expect_tx(bar, bytes);
-          tma_load_2d(smem_u32(qs), &tq, bar, km * (kK / 2), nrow0);
-          tma_load_2d(smem_u32(qs + 4096), &ts, bar, un.nt * 128, un.e * gpe + (km * kK) / a.g);
+          tma_load_2d(smem_u32(qs), &tq, bar, km * kCB, nrow0);
+          tma_load_2d(smem_u32(qs + 128 * kCB), &ts, bar, un.nt * 128, un.e * gpe + (km * kK) / a.g);
           pend.issued(q.stage, q.phase);
           q.next<kQStages>();
         }
@@ -316,8 +337,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     const int kh = (wi >> 2) & 1;             // 32-wide K half of the 64-wide stage
     const int lrow = 32 * (warp & 3) + lane;  // TMEM lane = feature within the tile
     const uint32_t tw = tmem_base + (uint32_t(32 * (warp & 3)) << 16) + kWBase + uint32_t(kh * 16);
-    const int code_off = lrow * 32 + ((kh ^ ((lrow >> 2) & 1)) << 4);   // 32B-swizzled code rows
-    const int scale_off = 4096 + (((ngrp == 2) ? kh : 0) * 128 + lrow) * 2;
+    const int scale_off = 128 * kCB + (((ngrp == 2) ? kh : 0) * 128 + lrow) * 2;
     bool inexact = false;   // a group scale whose products q * s are not exact in fp16
     bool lora_inf = false;  // a LoRA B value beyond the fp16 range
     int n = 0;   // stage counter
@@ -357,18 +377,34 @@ __global__ void __launch_bounds__(kThreads, 1)
           const uint32_t qph = uint32_t(mq / kQStages) & 1u;
           if (!__all_sync(0xFFFFFFFFu, mbar_wait(&ctl->q_full[qst], qph, abort_flag, a.status))) { ok = false; break; }
           const uint8_t* qs = q_base + size_t(qst) * kQStageBytes;
-          const uint4 wd = *reinterpret_cast<const uint4*>(qs + code_off);
           const uint32_t s2 = scale_pair_chk(*reinterpret_cast<const uint16_t*>(qs + scale_off), inexact);
-          const uint4 d0 = dequant_word(wd.x, s2), d1 = dequant_word(wd.y, s2);
-          const uint4 d2 = dequant_word(wd.z, s2), d3 = dequant_word(wd.w, s2);
+          if (BITS == 4) {
+            // this thread's 32 K values: one 16-byte chunk (4 words of 8 codes)
+            const uint4 wd = *reinterpret_cast<const uint4*>(qs + QC::chunk_offset(lrow, kh));
+            const uint4 d0 = dequant_word(wd.x, s2), d1 = dequant_word(wd.y, s2);
+            const uint4 d2 = dequant_word(wd.z, s2), d3 = dequant_word(wd.w, s2);
+            v[0] = d0.x; v[1] = d0.y; v[2] = d0.z; v[3] = d0.w;
+            v[4] = d1.x; v[5] = d1.y; v[6] = d1.z; v[7] = d1.w;
+            v[8] = d2.x; v[9] = d2.y; v[10] = d2.z; v[11] = d2.w;
+            v[12] = d3.x; v[13] = d3.y; v[14] = d3.z; v[15] = d3.w;
+          } else {
+            // two 16-byte chunks (8 words of 4 codes)
+#pragma unroll
+            for (int ch = 0; ch < 2; ++ch) {
+              const uint4 w4 = *reinterpret_cast<const uint4*>(qs + QC::chunk_offset(lrow, 2 * kh + ch));
+              const uint32_t wd[4] = {w4.x, w4.y, w4.z, w4.w};
+#pragma unroll
+              for (int i = 0; i < 4; ++i) {
+                const uint2 d2 = dequant_word8(wd[i], s2);
+                v[8 * ch + 2 * i] = d2.x;
+                v[8 * ch + 2 * i + 1] = d2.y;
+              }
+            }
+          }
           // the code slot's values have been consumed; its next fill is an
           // async-proxy TMA write, hence the proxy fence before handing it back
           fence_proxy_async_smem();
           mbar_arrive(&ctl->q_empty[qst]);
-          v[0] = d0.x; v[1] = d0.y; v[2] = d0.z; v[3] = d0.w;
-          v[4] = d1.x; v[5] = d1.y; v[6] = d1.z; v[7] = d1.w;
-          v[8] = d2.x; v[9] = d2.y; v[10] = d2.z; v[11] = d2.w;
-          v[12] = d3.x; v[13] = d3.y; v[14] = d3.z; v[15] = d3.w;
         }
         tmem_st16(tw + uint32_t(st) * kWCols, v);
         tmem_wait_st();
@@ -391,13 +427,18 @@ __global__ void __launch_bounds__(kThreads, 1)
 
 }  // namespace down_wide
 
-int run_expert_down_wide(const GemmArgs& a, const Maps& mp, int units_upper, cudaStream_t s) {
+template <int BITS>
+static int launch_down(const GemmArgs& a, const Maps& mp, int units_upper, cudaStream_t s) {
   static DeviceFlags attr_done;
-  if (!attr_done.test_and_set_device(down_wide::down_wide_kernel, int(down_wide::kSmemBytes))) return TQP_ERR_CUDA;
+  constexpr size_t smem = down_wide::smem_bytes<BITS>();
+  if (!attr_done.test_and_set_device(down_wide::down_wide_kernel<BITS>, int(smem))) return TQP_ERR_CUDA;
   const int grid = units_upper < num_sms() ? (units_upper > 0 ? units_upper : 1) : num_sms();
-  down_wide::down_wide_kernel<<<grid, down_wide::kThreads, down_wide::kSmemBytes, s>>>(a, mp.m[TQ0], mp.m[TS0],
-                                                                                        mp.m[TA]);
+  down_wide::down_wide_kernel<BITS><<<grid, down_wide::kThreads, smem, s>>>(a, mp.m[TQ0], mp.m[TS0], mp.m[TA]);
   return cudaGetLastError() == cudaSuccess ? TQP_OK : TQP_ERR_CUDA;
+}
+
+int run_expert_down_wide(const GemmArgs& a, const Maps& mp, int units_upper, cudaStream_t s) {
+  return a.bits == 8 ? launch_down<8>(a, mp, units_upper, s) : launch_down<4>(a, mp, units_upper, s);
 }
 
 }  // namespace tqp

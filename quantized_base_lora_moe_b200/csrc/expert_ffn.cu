@@ -19,14 +19,14 @@
 // barrier round trip is amortised over 8 MMAs. Per CTA (1 per SM, 832 threads):
 //   warps 0-3   epilogue (TMEM lanes 32w..32w+31 = features of the tile)
 //   warp  4     TMEM allocation + one thread issuing tcgen05.mma
-//   warp  5     TMA producer of the int4 code / bf16 scale ring (the code tiles
-//               come 32B-swizzled, so the row reads below are free of bank
-//               conflicts)
+//   warp  5     TMA producer of the code / bf16 scale ring (int4 code rows come
+//               32B-swizzled, int8 rows 64B-swizzled, so the row reads below
+//               are free of bank conflicts)
 //   warps 6-9   token producer: cp.async row gathers (rows picked by perm_token)
 //               and the rank-space rows
 //   warps 10-25 weight producer, two groups of 8 warps on alternate stages:
-//               each thread dequantises 64 K values of one weight row
-//               (int4 -> fp16) into TMEM; LoRA B rows
+//               each thread dequantises 64 K values of one weight row (int4 or
+//               int8 -> fp16) into TMEM; LoRA B rows
 // TMEM (512 columns): accumulators in [0, 256) (gate cols [0,128), up
 // [128,256)), 4 weight stages of 64 columns in [256, 512), each holding gate 32
 // | up 32 columns. A pipeline stage pairs one token tile (shared memory) with
@@ -57,8 +57,7 @@ namespace tmem_ffn {
 constexpr int kWWarp0 = 10;           // first weight-producer warp
 constexpr int kWWarps = 16;
 constexpr int kThreads = (kWWarp0 + kWWarps) * 32;
-constexpr int kQStages = 8;
-constexpr int kQStageBytes = 9216;    // 8192 B of codes + up to 1024 B of scales
+constexpr int kQStagesMax = 8;
 constexpr uint32_t kWBase = 256;      // first TMEM column of the weight stages
 constexpr int kStages = 4;            // pipeline stages (token tile + weight stage)
 constexpr uint32_t kWCols = 64;       // TMEM columns per weight stage
@@ -66,9 +65,23 @@ constexpr int kK = 64;                // K per stage
 constexpr int kXBytes = 16384;        // 128 token rows x 128 B
 constexpr int kStaging = (2 * 128 + 32) * kTRow;   // G rows | U rows | chunk tile
 
+// Code ring per code width: a stage holds 64 K values of 128 gate rows and 128
+// up rows (32 B per row for int4, 64 B for int8; TMA 32B / 64B swizzle) and up
+// to 2 x 2 x 128 scales.
+template <int BITS>
+struct QCfg {
+  static constexpr int kCB = 8 * BITS;                 // code bytes per row and stage
+  static constexpr int kStages = BITS == 4 ? 8 : 4;
+  static constexpr int kStageBytes = 256 * kCB + 1024;
+  // 16-byte chunk c of row r, as the TMA swizzle placed it
+  __device__ static __forceinline__ int chunk_offset(int r, int c) {
+    return r * kCB + ((BITS == 4 ? (c ^ ((r >> 2) & 1)) : (c ^ ((r >> 1) & 3))) << 4);
+  }
+};
+
 struct Ctl {
   uint64_t full[kStages], empty[kStages];
-  uint64_t q_full[kQStages], q_empty[kQStages];
+  uint64_t q_full[kQStagesMax], q_empty[kQStagesMax];
   uint64_t acc_full, acc_empty;
   uint64_t drain;
   uint64_t epi;
@@ -76,13 +89,22 @@ struct Ctl {
   Abort ab;
 };
 
-constexpr size_t kSmemBytes =
-    1024 + size_t(kStages) * kXBytes + size_t(kQStages) * kQStageBytes + size_t(kStaging) + sizeof(Ctl);
-static_assert(kSmemBytes + 2 * (kSchedSmemE + 1) * 4 <= 232448, "shared memory budget");
+template <int BITS>
+constexpr size_t smem_bytes() {
+  return 1024 + size_t(kStages) * kXBytes + size_t(QCfg<BITS>::kStages) * QCfg<BITS>::kStageBytes + size_t(kStaging) +
+         sizeof(Ctl);
+}
+static_assert(smem_bytes<4>() + 2 * (kSchedSmemE + 1) * 4 <= 232448, "shared memory budget");
+static_assert(smem_bytes<8>() + 2 * (kSchedSmemE + 1) * 4 <= 232448, "shared memory budget");
 
+template <int BITS>
 __global__ void __launch_bounds__(kThreads, 1)
     gateup_kernel(const GemmArgs a, const __grid_constant__ CUtensorMap tq0, const __grid_constant__ CUtensorMap tq1,
                   const __grid_constant__ CUtensorMap ts0, const __grid_constant__ CUtensorMap ts1) {
+  using QC = QCfg<BITS>;
+  constexpr int kQStages = QC::kStages;
+  constexpr int kQStageBytes = QC::kStageBytes;
+  constexpr int kCB = QC::kCB;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   uint8_t* x_base = smem;
@@ -259,8 +281,8 @@ __global__ void __launch_bounds__(kThreads, 1)
     if (lane == 0) {
       Ring q;
       PendingFills pend;
-      // gate codes [128 rows][32 B] | up codes | gate scales [ngrp][128] | up scales
-      const uint32_t bytes = uint32_t(8192 + 512 * ngrp);
+      // gate codes [128 rows][kCB B] | up codes | gate scales [ngrp][128] | up scales
+      const uint32_t bytes = uint32_t(256 * kCB + 512 * ngrp);
       const int gpe = a.in_dim / a.g;  // scale rows per expert
       for (int u = blockIdx.x; u < nunits; u += gridDim.x) {
         const Unit un = us.take(u);
@@ -272,10 +294,10 @@ __global__ void __launch_bounds__(kThreads, 1)
           uint64_t* bar = &ctl->q_full[q.stage];
           const int srow = un.e * gpe + (km * kK) / a.g;
           mbar_arrive_expect_tx(bar, bytes);
-          tma_load_2d(smem_u32(qs), &tq0, bar, km * (kK / 2), nrow0);
-          tma_load_2d(smem_u32(qs + 4096), &tq1, bar, km * (kK / 2), nrow0);
-          tma_load_2d(smem_u32(qs + 8192), &ts0, bar, un.nt * 128, srow);
-          tma_load_2d(smem_u32(qs + 8192 + 256 * ngrp), &ts1, bar, un.nt * 128, srow);
+          tma_load_2d(smem_u32(qs), &tq0, bar, km * kCB, nrow0);
+          tma_load_2d(smem_u32(qs + 128 * kCB), &tq1, bar, km * kCB, nrow0);
+          tma_load_2d(smem_u32(qs + 256 * kCB), &ts0, bar, un.nt * 128, srow);
+          tma_load_2d(smem_u32(qs + 256 * kCB + 256 * ngrp), &ts1, bar, un.nt * 128, srow);
           pend.issued(q.stage, q.phase);
           q.next<kQStages>();
         }
@@ -346,12 +368,11 @@ __global__ void __launch_bounds__(kThreads, 1)
     const int lrow = 32 * (warp & 3) + lane;  // TMEM lane = feature within the tile
     const int mat = gw >> 2;                  // 0 gate, 1 up
     const uint32_t tw = tmem_base + (uint32_t(32 * (warp & 3)) << 16) + kWBase + uint32_t(mat * 32);
-    // the two 16-byte code chunks of this thread inside a stage (TMA-swizzled rows)
-    const int c0_off = mat * 4096 + lrow * 32 + ((0 ^ ((lrow >> 2) & 1)) << 4);
-    const int c1_off = mat * 4096 + lrow * 32 + ((1 ^ ((lrow >> 2) & 1)) << 4);
+    // this thread's code row inside a stage (TMA-swizzled rows of kCB bytes)
+    const int row_off = mat * 128 * kCB;
     // scale rows of the two 32-wide K halves of this thread's slice
     const int g_lo = 0, g_hi = (ngrp == 1) ? 0 : 32 / a.g;
-    const int sbase = 8192 + mat * 256 * ngrp;
+    const int sbase = 256 * kCB + mat * 256 * ngrp;
     const int s_lo_off = sbase + (g_lo * 128 + lrow) * 2, s_hi_off = sbase + (g_hi * 128 + lrow) * 2;
     const bool is_up = mat == 1;
     bool inexact = false;   // a group scale whose products q * s are not exact in fp16
@@ -398,15 +419,31 @@ __global__ void __launch_bounds__(kThreads, 1)
           const uint32_t qph = uint32_t(mq / kQStages) & 1u;
           if (!__all_sync(0xFFFFFFFFu, mbar_wait(&ctl->q_full[qst], qph, abort_flag, a.status))) { ok = false; break; }
           const uint8_t* qs = q_base + size_t(qst) * kQStageBytes;
-          const uint4 wa = *reinterpret_cast<const uint4*>(qs + c0_off);
-          const uint4 wb = *reinterpret_cast<const uint4*>(qs + c1_off);
           const uint32_t s_lo = scale_pair_chk(*reinterpret_cast<const uint16_t*>(qs + s_lo_off), inexact);
           const uint32_t s_hi = scale_pair_chk(*reinterpret_cast<const uint16_t*>(qs + s_hi_off), inexact);
-          const uint32_t wd[8] = {wa.x, wa.y, wa.z, wa.w, wb.x, wb.y, wb.z, wb.w};
+          if (BITS == 4) {
+            // 64 K values = 8 words of 8 codes
+            const uint4 wa = *reinterpret_cast<const uint4*>(qs + row_off + QC::chunk_offset(lrow, 0));
+            const uint4 wb = *reinterpret_cast<const uint4*>(qs + row_off + QC::chunk_offset(lrow, 1));
+            const uint32_t wd[8] = {wa.x, wa.y, wa.z, wa.w, wb.x, wb.y, wb.z, wb.w};
 #pragma unroll
-          for (int c = 0; c < 8; ++c) {
-            const uint4 d4 = dequant_word(wd[c], c < 4 ? s_lo : s_hi);
-            v[4 * c] = d4.x; v[4 * c + 1] = d4.y; v[4 * c + 2] = d4.z; v[4 * c + 3] = d4.w;
+            for (int c = 0; c < 8; ++c) {
+              const uint4 d4 = dequant_word(wd[c], c < 4 ? s_lo : s_hi);
+              v[4 * c] = d4.x; v[4 * c + 1] = d4.y; v[4 * c + 2] = d4.z; v[4 * c + 3] = d4.w;
+            }
+          } else {
+            // 64 K values = 16 words of 4 codes
+#pragma unroll
+            for (int ch = 0; ch < 4; ++ch) {
+              const uint4 w4 = *reinterpret_cast<const uint4*>(qs + row_off + QC::chunk_offset(lrow, ch));
+              const uint32_t wd[4] = {w4.x, w4.y, w4.z, w4.w};
+#pragma unroll
+              for (int i = 0; i < 4; ++i) {
+                const uint2 d2 = dequant_word8(wd[i], ch < 2 ? s_lo : s_hi);
+                v[8 * ch + 2 * i] = d2.x;
+                v[8 * ch + 2 * i + 1] = d2.y;
+              }
+            }
           }
           // the code slot's values have been consumed; its next fill is an
           // async-proxy TMA write, hence the proxy fence before handing it back
@@ -434,13 +471,18 @@ __global__ void __launch_bounds__(kThreads, 1)
 
 }  // namespace tmem_ffn
 
-int run_expert_gateup(const GemmArgs& a, const Maps& mp, int units_upper, cudaStream_t s) {
+template <int BITS>
+static int launch_gateup(const GemmArgs& a, const Maps& mp, int units_upper, cudaStream_t s) {
   static DeviceFlags attr_done;
-  if (!attr_done.test_and_set_device(tmem_ffn::gateup_kernel, int(tmem_ffn::kSmemBytes))) return TQP_ERR_CUDA;
+  constexpr size_t smem = tmem_ffn::smem_bytes<BITS>();
+  if (!attr_done.test_and_set_device(tmem_ffn::gateup_kernel<BITS>, int(smem))) return TQP_ERR_CUDA;
   const int grid = units_upper < num_sms() ? (units_upper > 0 ? units_upper : 1) : num_sms();
-  tmem_ffn::gateup_kernel<<<grid, tmem_ffn::kThreads, tmem_ffn::kSmemBytes, s>>>(a, mp.m[TQ0], mp.m[TQ1], mp.m[TS0],
-                                                                               mp.m[TS1]);
+  tmem_ffn::gateup_kernel<BITS><<<grid, tmem_ffn::kThreads, smem, s>>>(a, mp.m[TQ0], mp.m[TQ1], mp.m[TS0], mp.m[TS1]);
   return cudaGetLastError() == cudaSuccess ? TQP_OK : TQP_ERR_CUDA;
+}
+
+int run_expert_gateup(const GemmArgs& a, const Maps& mp, int units_upper, cudaStream_t s) {
+  return a.bits == 8 ? launch_gateup<8>(a, mp, units_upper, s) : launch_gateup<4>(a, mp, units_upper, s);
 }
 
 }  // namespace tqp

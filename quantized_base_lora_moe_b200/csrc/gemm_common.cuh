@@ -48,6 +48,7 @@ struct GemmArgs {
   const uint16_t* lb1;     // DX: Au^T
   int lb_ld;
   const int4* unit_tab;    // expert kernels: decoded units {e, n-tile, rows, base}, one per unit
+  int bits;                // base-weight code width: 4 (packed int4) or 8 (int8)
   unsigned long long wait_ns;   // limit of one barrier wait (0: the default kWaitLimitNs)
 };
 
@@ -172,6 +173,19 @@ __device__ __forceinline__ uint4 dequant_word(uint32_t w, uint32_t s2) {
   return make_uint4(o[0], o[1], o[2], o[3]);
 }
 
+// 4 int8 codes (one storage word, code j in byte j) -> 4 fp16 values q * s as
+// two pairs (codes 0,1 | codes 2,3). (b ^ 0x80) = q + 128 for a two's-complement
+// byte b, and 0x6400 | m is the fp16 value 1024 + m, so one byte permute gives
+// 1152 + q exactly; subtracting 1152 is exact, and q * s (7-bit code times 8-bit
+// scale) is rounded once to fp16.
+__device__ __forceinline__ uint2 dequant_word8(uint32_t w, uint32_t s2) {
+  const uint32_t k1152 = 0x64806480u;   // fp16 pair (1152, 1152)
+  const uint32_t b = w ^ 0x80808080u;
+  const uint32_t lo = __byte_perm(b, 0x64646464u, 0x4140);
+  const uint32_t hi = __byte_perm(b, 0x64646464u, 0x4342);
+  return make_uint2(f16x2_mul(f16x2_sub(lo, k1152), s2), f16x2_mul(f16x2_sub(hi, k1152), s2));
+}
+
 __device__ __forceinline__ uint32_t scale_pair(uint16_t sbits) {
   const uint32_t sh = bf16_to_f16_bits(sbits);
   return sh | (sh << 16);
@@ -194,7 +208,7 @@ struct Maps {
 enum { TQ0 = 0, TQ1 = 1, TS0 = 2, TS1 = 3, TA = 4, TB0 = 5, TB1 = 6 };
 
 // Gate/up expert projection with the dequantised weights held in tensor memory
-// (expert_ffn.cu).
+// (expert_ffn.cu); a.bits selects int4 or int8 codes.
 int run_expert_gateup(const GemmArgs& a, const Maps& mp, int units_upper, cudaStream_t s);
 
 // Down projection with blocks of up to 256 routed rows (expert_down.cu).

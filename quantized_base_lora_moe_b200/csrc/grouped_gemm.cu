@@ -392,7 +392,9 @@ __global__ void __launch_bounds__(kThreads, 1)
       // forward: per n-tile rows of W [rows][64 K]: codes rows*32 B, scales [ngrp][rows] bf16
       // dgrad:   tile [64 K rows][ntile N]: codes 64*ntile/2 B, scales [ngn][64] bf16
       const int ngrp = kTrans ? (a.g >= a.ntile ? 1 : a.ntile / a.g) : (a.g >= 64 ? 1 : 64 / a.g);
-      const uint32_t bytes = uint32_t(a.ntile) * 32u + uint32_t(kTrans ? 128 * ngrp : a.ntile * ngrp * 2);
+      // dgrad code rows: ntile features at bits/8 bytes each (int4 or int8)
+      const int code_bytes = kTrans ? 64 * (a.ntile * a.bits / 8) : a.ntile * 32;
+      const uint32_t bytes = uint32_t(code_bytes) + uint32_t(kTrans ? 128 * ngrp : a.ntile * ngrp * 2);
       const int rows_box = (MODE == GATEUP) ? (a.ntile >> 1) : a.ntile;
       const int gpe = a.in_dim / a.g;  // scale rows per expert
       PendingFills pend;
@@ -407,9 +409,8 @@ __global__ void __launch_bounds__(kThreads, 1)
           if (kTrans) {
             const bool up = (MODE == DX) && km >= a.half_kb;
             const int kl = up ? km - a.half_kb : km;
-            tma_load_2d(smem_u32(qs), up ? &tq1 : &tq0, bar, un.nt * (a.ntile >> 1), un.e * a.out_dim + kl * 64);
-            tma_load_2d(smem_u32(qs + a.ntile * 32), up ? &ts1 : &ts0, bar, kl * 64,
-                        un.e * gpe + (un.nt * a.ntile) / a.g);
+            tma_load_2d(smem_u32(qs), up ? &tq1 : &tq0, bar, un.nt * (a.ntile * a.bits / 8), un.e * a.out_dim + kl * 64);
+            tma_load_2d(smem_u32(qs + code_bytes), up ? &ts1 : &ts0, bar, kl * 64, un.e * gpe + (un.nt * a.ntile) / a.g);
           } else {
             const int nrow0 = un.e * a.out_dim + un.nt * rows_box;
             const int srow = un.e * gpe + (km * 64) / a.g;
@@ -594,22 +595,33 @@ __global__ void __launch_bounds__(kThreads, 1)
           // Thread gtid: row gtid / 2, half gtid % 2.
           const int k = gtid >> 1, half = gtid & 1;
           const int n0 = un.nt * a.ntile;
-          const int rowb = a.ntile >> 1;                     // bytes per code row
-          const int wph = a.ntile >> 4;                      // words per half row (16 or 8)
-          const uint16_t* sc = reinterpret_cast<const uint16_t*>(qs + a.ntile * 32);
-          for (int j4 = 0; j4 < wph; j4 += 4) {
-            const int J = half * wph + j4;                   // first word of this 16-byte code chunk
-            const int cc = J >> 2;                           // code chunk within the row
-            // 128-byte rows come 128B-swizzled (conflict-free reads); 64-byte rows plain
+          const int rowb = a.ntile * a.bits / 8;            // bytes per code row (128 for the wide tiles)
+          const uint16_t* sc = reinterpret_cast<const uint16_t*>(qs + 64 * rowb);
+          // 16-byte code chunks of this thread's half row: 128-byte rows come
+          // 128B-swizzled (conflict-free reads), 64-byte rows plain
+          const int cph = rowb >> 5;
+          for (int j = 0; j < cph; ++j) {
+            const int cc = half * cph + j;                   // code chunk within the row
             const int pos = (rowb == 128) ? (cc ^ (k & 7)) : cc;
             const uint4 w4 = *reinterpret_cast<const uint4*>(qs + k * rowb + pos * 16);
             const uint32_t wv[4] = {w4.x, w4.y, w4.z, w4.w};
+            if (a.bits == 4) {
 #pragma unroll
-            for (int i = 0; i < 4; ++i) {
-              const int Jw = J + i;                          // word = features n0 + 8 Jw .. + 7
-              const int gi = (n0 + Jw * 8) / a.g - n0 / a.g;
-              *reinterpret_cast<uint4*>(bst + mn_tile_offset(k, Jw)) =
-                  dequant_word(wv[i], scale_pair_chk(sc[gi * 64 + k], inexact));
+              for (int i = 0; i < 4; ++i) {
+                const int Jw = cc * 4 + i;                   // word = features n0 + 8 Jw .. + 7
+                const int gi = (n0 + Jw * 8) / a.g - n0 / a.g;
+                *reinterpret_cast<uint4*>(bst + mn_tile_offset(k, Jw)) =
+                    dequant_word(wv[i], scale_pair_chk(sc[gi * 64 + k], inexact));
+              }
+            } else {
+              // int8: a chunk is 16 features = two 8-feature output chunks
+#pragma unroll
+              for (int i = 0; i < 2; ++i) {
+                const int Jo = cc * 2 + i;                   // output chunk = features n0 + 8 Jo .. + 7
+                const uint32_t s2 = scale_pair_chk(sc[((n0 + Jo * 8) / a.g - n0 / a.g) * 64 + k], inexact);
+                const uint2 lo = dequant_word8(wv[2 * i], s2), hi = dequant_word8(wv[2 * i + 1], s2);
+                *reinterpret_cast<uint4*>(bst + mn_tile_offset(k, Jo)) = make_uint4(lo.x, lo.y, hi.x, hi.y);
+              }
             }
           }
           // hand the code slot back only after its values were consumed, behind a
@@ -939,6 +951,8 @@ int launch_grouped_ffn_part(int part, const uint16_t* x, int T, const int32_t* o
   base.perm_token = perm_token;
   base.status = status;
   base.kb_per_piece = 1;
+  base.bits = w->bits == 8 ? 8 : 4;
+  const int bB = base.bits;
 
   if (part == 0 && r > 0) {  // xa = s * X [Ag | Au]   (bf16 operands)
     GemmArgs a = base;
@@ -982,11 +996,15 @@ int launch_grouped_ffn_part(int part, const uint16_t* x, int T, const int32_t* o
     a.f_dim = f;
     const int ngrp = w->group >= 64 ? 1 : 64 / w->group;
     const uint32_t rows_box = uint32_t(a.ntile / 2);
-    const int csw = tm ? 32 : 0;   // 32-byte code rows, swizzled for conflict-free row reads
+    // 64 K values per stage: 32-byte int4 / 64-byte int8 code rows, swizzled for
+    // conflict-free row reads in the tensor-memory kernel
+    const uint32_t cbox = uint32_t(8 * bB);
+    const int csw = tm ? int(cbox) : 0;
+    const uint64_t crow = uint64_t(d) * bB / 8;
     Maps mp{};
-    bool ok = make_map(&mp.m[TQ0], CU_TENSOR_MAP_DATA_TYPE_UINT8, w->wq[0], d / 2, uint64_t(w->E) * f, d / 2, 32,
+    bool ok = make_map(&mp.m[TQ0], CU_TENSOR_MAP_DATA_TYPE_UINT8, w->wq[0], crow, uint64_t(w->E) * f, crow, cbox,
                        rows_box, csw) &&
-              make_map(&mp.m[TQ1], CU_TENSOR_MAP_DATA_TYPE_UINT8, w->wq[1], d / 2, uint64_t(w->E) * f, d / 2, 32,
+              make_map(&mp.m[TQ1], CU_TENSOR_MAP_DATA_TYPE_UINT8, w->wq[1], crow, uint64_t(w->E) * f, crow, cbox,
                        rows_box, csw) &&
               make_map(&mp.m[TS0], CU_TENSOR_MAP_DATA_TYPE_UINT16, w->wscale[0], f, uint64_t(w->E) * (d / w->group),
                        uint64_t(f) * 2, rows_box, ngrp) &&
@@ -1034,8 +1052,8 @@ int launch_grouped_ffn_part(int part, const uint16_t* x, int T, const int32_t* o
     const int ngrp = w->group >= 64 ? 1 : 64 / w->group;
     Maps mp{};
     bool ok = make_tile_map(&mp.m[TA], h, uint64_t(A), uint64_t(f), 128) &&
-              make_map(&mp.m[TQ0], CU_TENSOR_MAP_DATA_TYPE_UINT8, w->wq[2], f / 2, uint64_t(w->E) * d, f / 2, 32, 128,
-                       32) &&
+              make_map(&mp.m[TQ0], CU_TENSOR_MAP_DATA_TYPE_UINT8, w->wq[2], uint64_t(f) * bB / 8, uint64_t(w->E) * d,
+                       uint64_t(f) * bB / 8, uint32_t(8 * bB), 128, 8 * bB) &&
               make_map(&mp.m[TS0], CU_TENSOR_MAP_DATA_TYPE_UINT16, w->wscale[2], d, uint64_t(w->E) * (f / w->group),
                        uint64_t(d) * 2, 128, ngrp);
     if (!ok) return TQP_ERR_CUDA;
@@ -1138,9 +1156,11 @@ int launch_dgrad(int which, const uint16_t* a_src, const uint16_t* a_lora, const
   a.f_dim = f;
   a.a_lora = a_lora;
   a.out = out;
+  a.bits = w->bits == 8 ? 8 : 4;
+  const int bB = a.bits;   // code bits: a tile row of ntile features is ntile * bits / 8 bytes
   Maps mp{};
   if (which == 0) {  // DH: K = d (rows of Wd), N = f
-    a.ntile = (f % 256 == 0) ? 256 : 128;
+    a.ntile = (f % 256 == 0 && bB == 4) ? 256 : 128;
     const int ngn = w->group >= a.ntile ? 1 : a.ntile / w->group;
     a.nkb_main = d / 64;
     a.nkb_lora = r > 0 ? (r + 63) / 64 : 0;
@@ -1155,15 +1175,15 @@ int launch_dgrad(int which, const uint16_t* a_src, const uint16_t* a_lora, const
     a.out_ld = 2 * f;
     a.n_valid = f;
     bool ok = make_tile_map(&mp.m[TA], a_src, uint64_t(A), uint64_t(d), 128) &&
-              make_map(&mp.m[TQ0], CU_TENSOR_MAP_DATA_TYPE_UINT8, w->wq[2], f / 2, uint64_t(w->E) * d, f / 2,
-                       uint32_t(a.ntile / 2), 64, a.ntile == 256 ? 128 : 0) &&
+              make_map(&mp.m[TQ0], CU_TENSOR_MAP_DATA_TYPE_UINT8, w->wq[2], uint64_t(f) * bB / 8, uint64_t(w->E) * d,
+                       uint64_t(f) * bB / 8, uint32_t(a.ntile * bB / 8), 64, a.ntile * bB / 8 == 128 ? 128 : 0) &&
               make_map(&mp.m[TS0], CU_TENSOR_MAP_DATA_TYPE_UINT16, w->wscale[2], d, uint64_t(w->E) * (f / w->group),
                        uint64_t(d) * 2, 64, ngn);
     if (!ok) return TQP_ERR_CUDA;
     return run_gemm<DH>(a, mp, mb_upper * a.n_tiles, s);
   }
   // DX: K = 2f (gate rows then up rows of W), N = d
-  a.ntile = (d % 256 == 0) ? 256 : 128;
+  a.ntile = (d % 256 == 0 && bB == 4) ? 256 : 128;
   const int ngn = w->group >= a.ntile ? 1 : a.ntile / w->group;
   a.nkb_main = 2 * f / 64;
   a.half_kb = f / 64;
@@ -1179,10 +1199,10 @@ int launch_dgrad(int which, const uint16_t* a_src, const uint16_t* a_lora, const
   a.out_ld = d;
   a.n_valid = d;
   bool ok = make_tile_map(&mp.m[TA], a_src, uint64_t(A), uint64_t(2 * f), 128) &&
-            make_map(&mp.m[TQ0], CU_TENSOR_MAP_DATA_TYPE_UINT8, w->wq[0], d / 2, uint64_t(w->E) * f, d / 2,
-                     uint32_t(a.ntile / 2), 64, a.ntile == 256 ? 128 : 0) &&
-            make_map(&mp.m[TQ1], CU_TENSOR_MAP_DATA_TYPE_UINT8, w->wq[1], d / 2, uint64_t(w->E) * f, d / 2,
-                     uint32_t(a.ntile / 2), 64, a.ntile == 256 ? 128 : 0) &&
+            make_map(&mp.m[TQ0], CU_TENSOR_MAP_DATA_TYPE_UINT8, w->wq[0], uint64_t(d) * bB / 8, uint64_t(w->E) * f,
+                     uint64_t(d) * bB / 8, uint32_t(a.ntile * bB / 8), 64, a.ntile * bB / 8 == 128 ? 128 : 0) &&
+            make_map(&mp.m[TQ1], CU_TENSOR_MAP_DATA_TYPE_UINT8, w->wq[1], uint64_t(d) * bB / 8, uint64_t(w->E) * f,
+                     uint64_t(d) * bB / 8, uint32_t(a.ntile * bB / 8), 64, a.ntile * bB / 8 == 128 ? 128 : 0) &&
             make_map(&mp.m[TS0], CU_TENSOR_MAP_DATA_TYPE_UINT16, w->wscale[0], f, uint64_t(w->E) * (d / w->group),
                      uint64_t(f) * 2, 64, ngn) &&
             make_map(&mp.m[TS1], CU_TENSOR_MAP_DATA_TYPE_UINT16, w->wscale[1], f, uint64_t(w->E) * (d / w->group),

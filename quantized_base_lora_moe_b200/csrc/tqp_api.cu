@@ -34,6 +34,8 @@ int check_weights(const tqp_moe_weights* w) {
   if (!(w->group == 32 || w->group == 64 || w->group == 128 || w->group == 256)) return TQP_ERR_UNSUPPORTED;
   if (w->d % w->group != 0 || w->ffn % w->group != 0) return TQP_ERR_INVALID_ARG;
   if (w->rank < 0 || w->rank > 64 || w->rank % 8 != 0) return TQP_ERR_UNSUPPORTED;
+  if (!(w->bits == 0 || w->bits == 4 || w->bits == 8)) return TQP_ERR_INVALID_ARG;
+  if (w->bits == 8 && w->ffn % 128 != 0) return TQP_ERR_UNSUPPORTED;   // int8 runs on the tensor-memory kernels only
   if (!w->router_w || !aligned16(w->router_w)) return TQP_ERR_INVALID_ARG;
   if (w->router_bias && !aligned16(w->router_bias)) return TQP_ERR_INVALID_ARG;
   for (int p = 0; p < 3; ++p) {

@@ -16,6 +16,8 @@ Storage formats (shared contract with the C-ABI, see include/tqp_moe.h):
 
 * bf16 values are carried as uint16 bit patterns (round-to-nearest-even from
   fp32).
+* int8 codes (bits = 8) of one projection, per expert, are an [out][in] array of
+  two's-complement bytes.
 * int4 codes of one projection, per expert, are a [out][in/2] uint8 array made of
   little-endian 32-bit words. Each word holds 8 consecutive input-dimension
   values k0..k7 of one output row as two's-complement nibbles: k(2i) sits in bits
@@ -59,6 +61,7 @@ class LayerConfig:
     zipf_s: float = 0.0       # >0: additive router bias ln(p_e), p_e ~ (e+1)^-s
     seed: int = 0
     w_mult: float = 1.0       # multiplies the base weights (before quantising) and LoRA B
+    bits: int = 4             # base-weight code width: 4 (packed int4) or 8 (int8)
 
     @property
     def A(self) -> int:
@@ -155,6 +158,28 @@ def quantise_int4(w: np.ndarray, g: int) -> tuple[np.ndarray, np.ndarray]:
     return pack_int4(q), np.ascontiguousarray(sbits.T)
 
 
+def quantise_int8(w: np.ndarray, g: int) -> tuple[np.ndarray, np.ndarray]:
+    """Symmetric group-wise int8 quantiser for one expert's [out][in] fp32 weight.
+
+    scale = bf16(absmax / 127) per group of g consecutive inputs; q = clamp(rint(w /
+    scale), -127, 127); an all-zero group gets scale 0 and codes 0. Returns the
+    codes [out][in] as int8 bytes (two's complement, stored uint8) and the scale
+    bits laid out [in/g][out].
+    """
+    w = np.asarray(w, dtype=np.float32)
+    out, inn = w.shape
+    wg = w.reshape(out, inn // g, g)
+    amax = np.abs(wg).max(axis=2)
+    sbits = f32_to_bf16_bits(amax / np.float32(127.0))
+    s = bf16_bits_to_f32(sbits)
+    safe = np.where(s == 0, np.float32(1.0), s)
+    q = np.rint(wg / safe[:, :, None])
+    q = np.clip(q, -127, 127)
+    q[s == 0] = 0
+    q = q.astype(np.int8).reshape(out, inn)
+    return np.ascontiguousarray(q.view(np.uint8)), np.ascontiguousarray(sbits.T)
+
+
 # ----------------------------------------------------------------------------
 # layer weights and activations
 # ----------------------------------------------------------------------------
@@ -178,7 +203,7 @@ def _expert_tensors(cfg: LayerConfig, seed: int, p: int, e: int):
     std_w = np.float32(1.0 / np.sqrt(cfg.d))
     mult = np.float32(cfg.w_mult)
     w = _rng(seed, f"w{p}", e).standard_normal((out, inn), dtype=np.float32) * std_w * mult
-    codes, scales = quantise_int4(w, cfg.g)
+    codes, scales = quantise_int4(w, cfg.g) if cfg.bits == 4 else quantise_int8(w, cfg.g)
     at = f32_to_bf16_bits(_rng(seed, f"a{p}", e).standard_normal((cfg.r, inn), dtype=np.float32) * std_w)
     bt = f32_to_bf16_bits(_rng(seed, f"b{p}", e).standard_normal((out, cfg.r), dtype=np.float32)
                           * np.float32(0.1) * mult)
@@ -200,7 +225,7 @@ def make_layer(cfg: LayerConfig, seed: int | None = None, threads: int | None = 
     layer["bias"] = zipf_bias(E, cfg.zipf_s) if cfg.zipf_s > 0 else None
     for p in range(3):
         out, inn = proj_dims(cfg, p)
-        layer[f"wq{p}"] = np.empty((E, out, inn // 2), np.uint8)
+        layer[f"wq{p}"] = np.empty((E, out, inn * cfg.bits // 8), np.uint8)
         layer[f"ws{p}"] = np.empty((E, inn // cfg.g, out), np.uint16)
         layer[f"la{p}"] = np.empty((E, cfg.r, inn), np.uint16)
         layer[f"lb{p}"] = np.empty((E, out, cfg.r), np.uint16)

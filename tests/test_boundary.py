@@ -2,6 +2,7 @@
 header declares, answers workspace queries, and rejects bad arguments before
 touching the GPU. No compute call is made."""
 import ctypes
+import dataclasses
 
 import pytest
 
@@ -50,7 +51,7 @@ def test_workspace_queries(cfg):
 
 BAD = [
     dict(E=0), dict(top_k=0), dict(top_k=33), dict(d=100), dict(d=192), dict(ffn=96), dict(group=48),
-    dict(rank=12), dict(rank=72), dict(router_w=None), dict(router_w=0x10004),
+    dict(rank=12), dict(rank=72), dict(router_w=None), dict(router_w=0x10004), dict(bits=3), dict(bits=16),
 ]
 
 
@@ -137,3 +138,48 @@ def test_backward_rejects_bad_gradient_buffers_before_any_launch(bad):
     F0 = _struct(synth.TINY, rank=0)
     null = Q.Grads()
     assert L.tqp_moe_layer_bwd(None, None, 0, ctypes.byref(F0), None, ctypes.byref(null), None, 0, None, None) == 0
+
+
+def test_int8_needs_ffn_multiple_of_128():
+    L = Q.lib()
+    cfg = synth.LayerConfig("i8", T=64, d=128, E=4, k=2, f=192, g=64, r=8)
+    assert L.tqp_moe_layer_workspace_size(64, ctypes.byref(_struct(cfg, bits=8))) == 0
+    assert L.tqp_moe_layer_fwd(0x20000, 64, ctypes.byref(_struct(cfg, bits=8)), 0x30000, 0x40000, 1 << 30, None,
+                               None) == -2
+    assert L.tqp_moe_layer_workspace_size(64, ctypes.byref(_struct(cfg, bits=4))) > 0
+    assert L.tqp_moe_layer_workspace_size(64, ctypes.byref(_struct(synth.TINY, bits=8))) > 0
+
+
+def _stack_arrays(ws_list):
+    arr = (ctypes.POINTER(Q.Weights) * len(ws_list))(*[ctypes.pointer(w) for w in ws_list])
+    return ctypes.cast(arr, ctypes.c_void_p), arr
+
+
+def test_stack_workspace_is_flat_in_depth_and_bad_stacks_are_rejected():
+    L = Q.lib()
+    w = _struct(synth.MID)
+    sizes = []
+    for depth in (1, 2, 16, 256):
+        p, keep = _stack_arrays([w] * depth)
+        sizes.append(L.rev_stack_workspace_size(synth.MID.T, depth, p, p))
+    assert sizes[0] > 0 and len(set(sizes)) == 1
+    p, keep = _stack_arrays([w] * 2)
+    assert L.rev_stack_workspace_size(synth.MID.T, 0, p, p) == 0                 # L = 0
+    other = _struct(dataclasses.replace(synth.MID, d=512))
+    q, keep2 = _stack_arrays([w, other])
+    assert L.rev_stack_workspace_size(synth.MID.T, 2, q, q) == 0                  # mixed widths
+    # the backward needs gradient arrays: refused before anything is enqueued
+    rc = L.rev_stack_bwd(0x20000, 0x20000, 0x20000, 0x20000, synth.MID.T, 2, p, p, 0x20000, 0x20000, 0x20000,
+                         0x20000, None, None, 0x30000, 1 << 40, None, None)
+    assert rc == -1
+
+
+def test_adamw_rejects_bad_hyperparameters_on_host():
+    L = Q.lib()
+    f = ctypes.c_void_p(0x10000)
+    assert L.tqp_adamw_step(f, f, f, f, None, 16, 1e-3, 0.9, 0.999, 1e-8, 0.0, 0, 1.0, None, None) == -1  # step 0
+    assert L.tqp_adamw_step(f, f, f, f, None, 16, 1e-3, 1.0, 0.999, 1e-8, 0.0, 1, 1.0, None, None) == -1  # beta1 = 1
+    assert L.tqp_adamw_step(f, f, f, f, None, 16, 1e-3, 0.9, 0.999, 0.0, 0.0, 1, 1.0, None, None) == -1   # eps = 0
+    assert L.tqp_adamw_step(ctypes.c_void_p(0x10004), f, f, f, None, 16, 1e-3, 0.9, 0.999, 1e-8, 0.0, 1, 1.0, None,
+                            None) == -1                                                                   # misaligned
+    assert L.tqp_adamw_step(f, f, f, f, None, 0, 1e-3, 0.9, 0.999, 1e-8, 0.0, 1, 1.0, None, None) == 0    # n = 0: no-op

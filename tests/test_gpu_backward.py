@@ -27,7 +27,8 @@ BW1 = synth.LayerConfig("bw1", T=300, d=256, E=10, k=3, f=256, g=64, r=16)
 BW_ONE = synth.LayerConfig("bw_one", T=37, d=128, E=1, k=1, f=128, g=32, r=8)
 BW_R0 = synth.LayerConfig("bw_r0", T=50, d=128, E=4, k=4, f=128, g=128, r=0)
 BW_SKEW = synth.LayerConfig("bw_skew", T=600, d=256, E=12, k=2, f=256, g=64, r=16, zipf_s=1.1)
-LAYER_CFGS = [synth.TINY, BW1, BW_ONE, BW_R0, BW_SKEW, synth.MID]
+BW_I8 = synth.LayerConfig("bw_i8", T=300, d=256, E=10, k=3, f=256, g=64, r=16, bits=8)
+LAYER_CFGS = [synth.TINY, BW1, BW_ONE, BW_R0, BW_SKEW, synth.MID, BW_I8]
 
 
 @pytest.fixture(scope="module", autouse=True)

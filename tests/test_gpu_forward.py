@@ -33,6 +33,11 @@ ALLK = synth.LayerConfig("allk", T=50, d=128, E=4, k=4, f=128, g=128, r=0)
 G256 = synth.LayerConfig("g256", T=200, d=256, E=6, k=2, f=256, g=256, r=8)
 R64 = synth.LayerConfig("r64", T=150, d=256, E=5, k=2, f=256, g=64, r=64)
 SMALL_CFGS = [synth.TINY, RAGGED, ONE, ALLK, G256, R64, synth.MID]
+# int8 base weights (TQP Quantization: int8 or int4): codes one byte each, q * s
+# rounded once to fp16; group 32 (two scale groups per 64-wide K stage), rank 0
+INT8_CFGS = [synth.LayerConfig("i8", T=300, d=256, E=10, k=3, f=256, g=64, r=16, bits=8),
+             synth.LayerConfig("i8g32", T=200, d=128, E=6, k=2, f=128, g=32, r=0, bits=8),
+             dataclasses.replace(synth.MID, name="mid_i8", bits=8)]
 TOL = 2e-2
 # The router's products are exact (bf16 x times an exact 3-part bf16 split of
 # the fp32 weights); its error is the tensor cores' fp32 accumulation, at most
@@ -240,7 +245,7 @@ def test_grouped_ffn_parts_equal_whole_call(cfg):
     assert torch.equal(h1, h2) and torch.equal(o1, o2)
 
 
-@pytest.mark.parametrize("cfg", SMALL_CFGS, ids=lambda c: c.name)
+@pytest.mark.parametrize("cfg", SMALL_CFGS + INT8_CFGS, ids=lambda c: c.name)
 def test_grouped_ffn_matches_oracle(cfg):
     raw = host_layer(cfg)
     L = O.Layer(raw)
@@ -356,7 +361,7 @@ def _layer_check(cfg, raw, xb, y_dev, margin=1e-4):
     return ties
 
 
-@pytest.mark.parametrize("cfg", SMALL_CFGS, ids=lambda c: c.name)
+@pytest.mark.parametrize("cfg", SMALL_CFGS + INT8_CFGS, ids=lambda c: c.name)
 def test_layer_fwd_matches_oracle(cfg):
     raw = host_layer(cfg)
     xb = synth.make_tokens(cfg.T, cfg.d, 21)

@@ -92,6 +92,30 @@ def test_dequant_roundtrip_bound_and_on_grid_exact():
     assert np.array_equal(O.unpack_int4(c2), q)
 
 
+def test_int8_decode_golden_bytes_and_dequant_roundtrip():
+    # two's-complement bytes, hand-decoded
+    raw = np.array([[0x00, 0x01, 0x7F, 0x80, 0x81, 0xFF, 0xF9, 0x07]], dtype=np.uint8)
+    assert O.unpack_int8(raw).tolist() == [[0, 1, 127, -128, -127, -1, -7, 7]]
+    g = 64
+    rng = np.random.default_rng(5)
+    w = (rng.standard_normal((16, 256)) / 8).astype(np.float32)
+    w[2, 64:128] = 0.0
+    codes, scales = synth.quantise_int8(w, g)
+    assert codes.shape == (16, 256)
+    what = O.dequant(codes, scales, g, bits=8)
+    s = np.repeat(O.bf16_to_f64(scales).T, g, axis=1)
+    assert np.all(np.abs(what - w) <= s / 2 + 1e-12)
+    assert np.all(what[2, 64:128] == 0)
+    # on-grid weights with a group reaching |q| = 127 round-trip exactly
+    q = rng.integers(-127, 128, size=(16, 256))
+    q[:, ::g] = 127
+    sc = O.bf16_to_f64(synth.f32_to_bf16_bits(rng.uniform(1e-4, 1e-3, size=(16, 256 // g)).astype(np.float32)))
+    w2 = (q * np.repeat(sc, g, axis=1)).astype(np.float32)
+    c2, s2 = synth.quantise_int8(w2, g)
+    assert np.array_equal(O.unpack_int8(c2), q)
+    assert np.array_equal(O.dequant(c2, s2, g, bits=8), w2.astype(np.float64))
+
+
 # ---------------------------------------------------------------- router, top-k, gates
 
 
