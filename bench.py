@@ -607,13 +607,14 @@ def run_tqp(args, rank: int, world: int, local_rank: int) -> dict | None:
         result["configs"] = extra
     if world == 1 and not args.no_rev:
         result["rev_block"] = time_rev_block(lb.L, cfg, dev, min(args.steps, 5), 2, flush)
+    host, x_bits = lb.host, lb.x_bits
     if world == 1 and args.config == "full" and not args.no_stack:
         del lb
         torch.cuda.empty_cache()
         result["rev_stack"] = time_stack(dev, flush)
     if world == 1 and not args.no_cpu_baseline:
         sample = min(T, args.cpu_sample)
-        result["cpu_baseline"] = time_oracle(cfg, lb.host, lb.x_bits, sample)
+        result["cpu_baseline"] = time_oracle(cfg, host, x_bits, sample)
     return result
 
 

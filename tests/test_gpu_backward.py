@@ -6,6 +6,11 @@ x2 from the block outputs max|x - rec|/RMS(x) <= 5e-3. Tokens whose routing is
 ambiguous at the arithmetic's precision are excluded from the elementwise
 comparison, and so are the experts they touch (their gradient sums would
 differ by that token's contribution either way).
+
+In the block tests G's input is bf16(y1) of the GPU's own forward output: the
+backward reads exactly that, so both sides route G on the same bf16 values and
+the comparison isolates the backward's arithmetic. (How far y1 itself is from
+the oracle's forward is the forward tests' concern.)
 """
 import dataclasses
 
@@ -28,7 +33,8 @@ BW_ONE = synth.LayerConfig("bw_one", T=37, d=128, E=1, k=1, f=128, g=32, r=8)
 BW_R0 = synth.LayerConfig("bw_r0", T=50, d=128, E=4, k=4, f=128, g=128, r=0)
 BW_SKEW = synth.LayerConfig("bw_skew", T=600, d=256, E=12, k=2, f=256, g=64, r=16, zipf_s=1.1)
 BW_I8 = synth.LayerConfig("bw_i8", T=300, d=256, E=10, k=3, f=256, g=64, r=16, bits=8)
-LAYER_CFGS = [synth.TINY, BW1, BW_ONE, BW_R0, BW_SKEW, synth.MID, BW_I8]
+BW_R32 = synth.LayerConfig("bw_r32", T=300, d=256, E=10, k=3, f=256, g=64, r=32)   # the full config's rank
+LAYER_CFGS = [synth.TINY, BW1, BW_ONE, BW_R0, BW_SKEW, synth.MID, BW_I8, BW_R32]
 
 
 @pytest.fixture(scope="module", autouse=True)
@@ -121,8 +127,13 @@ def gpu_block(cfgF, cfgG, rawF, rawG, x1b, x2b, dy1, dy2):
     torch.cuda.synchronize()
     assert st.read() == 0
     c = lambda ts: [t.cpu().numpy() for t in ts]
-    return {"x1": host_bf16(r1), "x2": host_bf16(r2), "dx1": dx1.cpu().numpy(), "dx2": dx2.cpu().numpy(),
-            "dA_F": c(dAF), "dB_F": c(dBF), "dA_G": c(dAG), "dB_G": c(dBG)}
+    return {"y1": y1.cpu().numpy(), "x1": host_bf16(r1), "x2": host_bf16(r2), "dx1": dx1.cpu().numpy(),
+            "dx2": dx2.cpu().numpy(), "dA_F": c(dAF), "dB_F": c(dBF), "dA_G": c(dAG), "dB_G": c(dBG)}
+
+
+def g_input(y1_gpu):
+    """bf16(y1) of the GPU's fp32 y1: the input the block backward gives G."""
+    return O.round_bf16(y1_gpu.astype(np.float64))
 
 
 @pytest.mark.parametrize("cfgs", [REV_TINY, REV_MID], ids=["tiny", "mid"])
@@ -138,56 +149,35 @@ def test_adapter_bwd_block_matches_oracle(cfgs):
     rms = np.sqrt(np.mean(np.concatenate([x1, x2]) ** 2))
     assert max(np.max(np.abs(got["x1"] - x1)), np.max(np.abs(got["x2"] - x2))) / rms <= 5e-3
     LF, LG = O.Layer(rawF), O.Layer(rawG)
-    y1, y2 = O.coupling_forward(x1, x2, LF, LG)
-    ref = O.block_backward(y1, y2, dy1.astype(np.float64), dy2.astype(np.float64), LF, LG)
-    # ambiguous routing: F near ties, and G tokens whose routing moves when F's
-    # output moves by its own rounding (see test_rev_couple_fwd_inverse)
-    tieF, ambF = ambiguous_experts(O.router_logits(x2, LF), cfgF.k, 1e-4)
-    f_ref = y1 - x1
-    rng = np.random.default_rng(7)
-    z = O.round_bf16(y1)
-    zp = O.round_bf16(x1 + f_ref * (1.0 + 2.0 ** -8 * rng.uniform(-1.0, 1.0, f_ref.shape)))
-    lz = O.router_logits(z, LG)
-    flip = np.any(O.topk(lz, cfgG.k) != O.topk(O.router_logits(zp, LG), cfgG.k), axis=1)
-    tieG, ambG = ambiguous_experts(lz, cfgG.k, 5e-3)
-    tieG |= flip
-    for t in np.nonzero(flip)[0]:
-        ambG |= set(O.topk(lz[t:t + 1], cfgG.k)[0].tolist()) | set(O.topk(O.router_logits(zp[t:t + 1], LG),
-                                                                            cfgG.k)[0].tolist())
-    # a G-ambiguous token also changes F's cotangent dz1 at that token, so F's experts of that token too
-    ambF_from_G = set(O.topk(O.router_logits(x2[tieG], LF), cfgF.k).ravel().tolist()) if tieG.any() else set()
-    keep_t = ~(tieF | tieG)
-    assert keep_t.mean() > 0.7
-    kF = np.array([e not in (ambF | ambF_from_G) for e in range(cfgF.E)])
-    kG = np.array([e not in ambG for e in range(cfgG.E)])
-    # G runs on bf16(y1), which carries F's rounding: the oracle measures how far
-    # each result moves when F's output moves by 2^-8 relative (zp above), and the
-    # bound is TOL plus twice that spread.
+    z = g_input(got["y1"])
     dy1_, dy2_ = dy1.astype(np.float64), dy2.astype(np.float64)
-    dxGp, dAGp, dBGp = O.layer_backward(zp, dy2_, LG)
-    dz1p = dy1_ + dxGp
-    dxFp, dAFp, dBFp = O.layer_backward(ref["x2"], dz1p, LF)
-    pert = {"dx1": dz1p, "dx2": dy2_ + dxFp, "dA_F": dAFp, "dB_F": dBFp, "dA_G": dAGp, "dB_G": dBGp}
+    dxG, dAG, dBG = O.layer_backward(z, dy2_, LG)
+    dz1 = dy1_ + dxG
+    dxF, dAF, dBF = O.layer_backward(x2, dz1, LF)
+    ref = {"dx1": dz1, "dx2": dy2_ + dxF, "dA_F": dAF, "dB_F": dBF, "dA_G": dAG, "dB_G": dBG}
+    tieF, ambF = ambiguous_experts(O.router_logits(x2, LF), cfgF.k, 1e-4)
+    tieG, ambG = ambiguous_experts(O.router_logits(z, LG), cfgG.k, 1e-4)
+    # a G-ambiguous token also changes F's cotangent dz1 at that token, so F's experts of that token too
+    if tieG.any():
+        ambF |= set(O.topk(O.router_logits(x2[tieG], LF), cfgF.k).ravel().tolist())
+    keep_t = ~(tieF | tieG)
+    assert keep_t.mean() > 0.95
+    kF = np.array([e not in ambF for e in range(cfgF.E)])
+    kG = np.array([e not in ambG for e in range(cfgG.E)])
+    assert kF.mean() >= 0.5 and kG.mean() >= 0.5, (kF.sum(), kG.sum())
 
     def check(key, sel, p=None):
         g = got[key] if p is None else got[key][p]
         r = ref[key] if p is None else ref[key][p]
-        q = pert[key] if p is None else pert[key][p]
-        spread = rel_err(q[sel], r[sel])
         err = rel_err(g[sel], r[sel])
-        print(f"SPREAD block-{cfgF.T}x{cfgF.d} {key}{'' if p is None else p}: err {err:.3e} spread {spread:.3e} "
-              f"bound {TOL + 2 * spread:.3e}")
-        assert err <= TOL + 2 * spread, (key, p, err, spread)
+        print(f"BLOCK {cfgF.T}x{cfgF.d} {key}{'' if p is None else p}: err {err:.3e}")
+        assert err <= TOL, (key, p, err)
 
     check("dx1", keep_t)
     check("dx2", keep_t)
     for p in range(3):
-        if kF.any():
-            check("dA_F", kF, p)
-            check("dB_F", kF, p)
-        if kG.any():
-            check("dA_G", kG, p)
-            check("dB_G", kG, p)
+        for key, keep in (("dA_F", kF), ("dB_F", kF), ("dA_G", kG), ("dB_G", kG)):
+            check(key, keep, p)
 
 
 _FULL_BLOCK = {}
@@ -221,44 +211,31 @@ def test_adapter_bwd_full_size_reconstruction_and_sampled_tokens():
     assert max(np.max(np.abs(got["x1"] - x1)), np.max(np.abs(got["x2"] - x2))) / rms <= 5e-3
     assert all(np.isfinite(got[k]).all() for k in ("dx1", "dx2"))
     LF, LG = O.Layer(rawF), O.Layer(rawG)
-    toks = [0, T - 1, 1234, 4321, 777, 6000]
-    rng = np.random.default_rng(9)
-    ok_rows, g1, g2, r1s, r2s, p1s, p2s = [], [], [], [], [], [], []
+    toks = [0, T - 1, 1234, 4321, 777, 6000, 100, 8000]
+    ok_rows, g1, g2, r1s, r2s = [], [], [], [], []
     for t in toks:
-        yF, idF, _, lF = O.token_forward(x2[t], LF)
-        y1t = x1[t] + yF
-        z = O.round_bf16(y1t)[None, :]
-        zp = O.round_bf16(x1[t] + yF * (1.0 + 2.0 ** -8 * rng.uniform(-1.0, 1.0, yF.shape)))[None, :]
-        lG = O.router_logits(z, LG)
-        amb = (O.routing_gap(lF[None, :], cfgF.k)[0] < 1e-4) or (O.routing_gap(lG, cfgG.k)[0] < 2e-2) or \
-            np.any(O.topk(lG, cfgG.k) != O.topk(O.router_logits(zp, LG), cfgG.k))
+        z = g_input(got["y1"][t:t + 1])
+        amb = (O.routing_gap(O.router_logits(x2[t:t + 1], LF), cfgF.k)[0] < 1e-4) or \
+            (O.routing_gap(O.router_logits(z, LG), cfgG.k)[0] < 1e-4)
         if amb:
             continue
         dy1t, dy2t = dy1[t:t + 1].astype(np.float64), dy2[t:t + 1].astype(np.float64)
         dz1 = dy1t + O.layer_backward(z, dy2t, LG)[0]
-        dz1p = dy1t + O.layer_backward(zp, dy2t, LG)[0]
         ok_rows.append(t)
         g1.append(got["dx1"][t])
         g2.append(got["dx2"][t])
         r1s.append(dz1[0])
         r2s.append(dy2t[0] + O.layer_backward(x2[t:t + 1], dz1, LF)[0][0])
-        p1s.append(dz1p[0])
-        p2s.append(dy2t[0] + O.layer_backward(x2[t:t + 1], dz1p, LF)[0][0])
-    assert len(ok_rows) >= 4
-    # tolerance: TOL plus twice the oracle's own spread when F's output moves by 2^-8 relative
-    s1 = rel_err(np.array(p1s), np.array(r1s))
-    s2 = rel_err(np.array(p2s), np.array(r2s))
+    assert len(ok_rows) >= 6
     e1 = rel_err(np.array(g1), np.array(r1s))
     e2 = rel_err(np.array(g2), np.array(r2s))
-    print(f"SPREAD block-full sampled tokens {ok_rows}: dx1 err {e1:.3e} spread {s1:.3e}; "
-          f"dx2 err {e2:.3e} spread {s2:.3e}")
-    assert e1 <= TOL + 2 * s1, (e1, s1)
-    assert e2 <= TOL + 2 * s2, (e2, s2)
+    print(f"BLOCK full sampled tokens {ok_rows}: dx1 err {e1:.3e}; dx2 err {e2:.3e}")
+    assert e1 <= TOL and e2 <= TOL, (e1, e2)
 
 
 def _pick_experts(counts, amb_per_expert, n_between=2):
     """The busiest expert, the least-loaded non-empty one and n_between in
-    between, preferring among equals those that no ambiguous token touches."""
+    between, among those that no ambiguous token touches."""
     nz = np.nonzero(counts)[0]
     order = nz[np.lexsort((amb_per_expert[nz], -counts[nz]))]     # busiest first, fewest ambiguous first
     clean = [e for e in order if amb_per_expert[e] == 0] or list(order)
@@ -283,36 +260,25 @@ def _routed_rows(ids, gam, e):
 
 def test_adapter_bwd_full_size_sampled_expert_gradients():
     """dA and dB of F and G at full size, element by element, on sampled
-    experts (the busiest, the least-loaded non-empty one and two in between).
+    experts (the busiest, the least-loaded non-empty one and two in between,
+    none touched by a token whose routing is a near tie).
 
-    The oracle runs F's forward on every token in fp64, rounds y1 to bf16 for G
-    and routes G on it. An expert's gradient sums over the tokens routed to it,
-    so it is the oracle's expert backward over those tokens with dO = gate *
-    cotangent; for F the cotangent dz1 = dy1 + J_G^T dy2 is the oracle's layer
-    backward of G at those tokens. G reads bf16(y1), which carries the rounding
-    of F's output on either side: the bound is TOL plus twice the oracle's own
-    spread when F's output moves by 2^-8 relative (as in the mid-size block
-    test), printed beside every error."""
+    An expert's gradient sums over the tokens routed to it, so it is the
+    oracle's expert backward over those tokens with dO = gate * cotangent. G's
+    input is bf16 of the GPU's y1; F's cotangent dz1 = dy1 + J_G^T dy2 is the
+    oracle's layer backward of G at the tokens of F's picked experts."""
     fb = full_block()
     cfgF, cfgG, rawF, rawG = fb["cfgF"], fb["cfgG"], fb["rawF"], fb["rawG"]
-    x1, x2 = O.bf16_to_f64(fb["x1b"]), O.bf16_to_f64(fb["x2b"])
+    x2 = O.bf16_to_f64(fb["x2b"])
     dy1, dy2 = fb["dy1"].astype(np.float64), fb["dy2"].astype(np.float64)
     got = fb["got"]
     LF, LG = O.Layer(rawF), O.Layer(rawG)
     kF, kG = cfgF.k, cfgG.k
-    # F on every token (exact input x2), y1, G's input and routing
-    lF = O.router_logits(x2, LF)
-    idsF = O.topk(lF, kF)
-    gF = O.gates(lF, idsF)
-    f_out = O.layer_forward(x2, LF, ids=idsF)
-    y1 = x1 + f_out
-    z = O.round_bf16(y1)
-    rng = np.random.default_rng(11)
-    zp = O.round_bf16(x1 + f_out * (1.0 + 2.0 ** -8 * rng.uniform(-1.0, 1.0, f_out.shape)))
-    lG, lGp = O.router_logits(z, LG), O.router_logits(zp, LG)
-    idsG, idsGp = O.topk(lG, kG), O.topk(lGp, kG)
-    gG, gGp = O.gates(lG, idsG), O.gates(lGp, idsGp)
-    ambG_tok = np.any(idsG != idsGp, axis=1) | (O.routing_gap(lG, kG) < 1e-4)
+    z = g_input(got["y1"])
+    lF, lG = O.router_logits(x2, LF), O.router_logits(z, LG)
+    idsF, idsG = O.topk(lF, kF), O.topk(lG, kG)
+    gF, gG = O.gates(lF, idsF), O.gates(lG, idsG)
+    ambG_tok = O.routing_gap(lG, kG) < 1e-4
     ambF_tok = O.routing_gap(lF, kF) < 1e-4
     E = cfgF.E
     countsG = np.bincount(idsG.ravel(), minlength=E)
@@ -322,34 +288,25 @@ def test_adapter_bwd_full_size_sampled_expert_gradients():
     picksG = _pick_experts(countsG, ambG_e)
     picksF = _pick_experts(countsF, ambF_e)
     assert len(picksG) >= 4 and len(picksF) >= 4
+    assert all(ambG_e[e] == 0 for e in picksG) and all(ambF_e[e] == 0 for e in picksF)
 
-    def check(name, g, r, q):
-        err, spread = rel_err(g, r), rel_err(q, r)
-        print(f"SPREAD block-full {name}: err {err:.3e} spread {spread:.3e} bound {TOL + 2 * spread:.3e}")
-        assert err <= TOL + 2 * spread, (name, err, spread)
+    def check(name, g, r):
+        err = rel_err(g, r)
+        print(f"BLOCK full {name}: err {err:.3e}")
+        assert err <= TOL, (name, err)
 
-    # G: cotangent dy2, input z (perturbed: zp, with zp's own routing)
     for e in picksG:
         t, gam = _routed_rows(idsG, gG, e)
-        tp, gamp = _routed_rows(idsGp, gGp, e)
         dA, dB = _expert_grads(z[t], gam[:, None] * dy2[t], LG, e)
-        dAp, dBp = _expert_grads(zp[tp], gamp[:, None] * dy2[tp], LG, e)
         for p in range(3):
-            check(f"dA_G[{p}] expert {e} ({len(t)} rows)", got["dA_G"][p][e], dA[p], dAp[p])
-            check(f"dB_G[{p}] expert {e} ({len(t)} rows)", got["dB_G"][p][e], dB[p], dBp[p])
-    # F: cotangent dz1 = dy1 + J_G^T dy2 at the tokens of the picked experts
+            check(f"dA_G[{p}] expert {e} ({len(t)} rows)", got["dA_G"][p][e], dA[p])
+            check(f"dB_G[{p}] expert {e} ({len(t)} rows)", got["dB_G"][p][e], dB[p])
     S = np.unique(np.concatenate([np.nonzero(np.any(idsF == e, axis=1))[0] for e in picksF]))
     dz1 = np.zeros_like(dy1)
-    dz1p = np.zeros_like(dy1)
-    # one call over z and zp stacked (each row's input gradient is its own; every
-    # expert is decoded once)
-    dxG = O.layer_backward(np.concatenate([z[S], zp[S]]), np.concatenate([dy2[S], dy2[S]]), LG)[0]
-    dz1[S] = dy1[S] + dxG[:len(S)]
-    dz1p[S] = dy1[S] + dxG[len(S):]
+    dz1[S] = dy1[S] + O.layer_backward(z[S], dy2[S], LG)[0]
     for e in picksF:
         t, gam = _routed_rows(idsF, gF, e)
         dA, dB = _expert_grads(x2[t], gam[:, None] * dz1[t], LF, e)
-        dAp, dBp = _expert_grads(x2[t], gam[:, None] * dz1p[t], LF, e)
         for p in range(3):
-            check(f"dA_F[{p}] expert {e} ({len(t)} rows)", got["dA_F"][p][e], dA[p], dAp[p])
-            check(f"dB_F[{p}] expert {e} ({len(t)} rows)", got["dB_F"][p][e], dB[p], dBp[p])
+            check(f"dA_F[{p}] expert {e} ({len(t)} rows)", got["dA_F"][p][e], dA[p])
+            check(f"dB_F[{p}] expert {e} ({len(t)} rows)", got["dB_F"][p][e], dB[p])

@@ -445,28 +445,21 @@ def test_rev_couple_fwd_inverse(cfgs):
     assert err <= 5e-3
     # forward values against the oracle (tokens away from routing ties in both layers)
     LF, LG = O.Layer(rawF), O.Layer(rawG)
-    o1, o2 = O.coupling_forward(x1, x2, LF, LG)
+    o1, _ = O.coupling_forward(x1, x2, LF, LG)
     f_ref = o1 - x1
     tieF = near_tie_tokens(O.router_logits(x2, LF), cfgF.k, 1e-4)
-    # G reads bf16(y1): an error in F within its own bound flips the bf16 rounding
-    # of some y1 elements by one ulp. The oracle measures how far G moves under
-    # such a perturbation of F's output (2^-8 relative, twice bf16's rounding
-    # error) and which tokens change their G routing; those are ambiguous.
-    rng = np.random.default_rng(7)
-    z = O.round_bf16(o1)
-    zp = O.round_bf16(x1 + f_ref * (1.0 + 2.0 ** -8 * rng.uniform(-1.0, 1.0, f_ref.shape)))
-    lz, lzp = O.router_logits(z, LG), O.router_logits(zp, LG)
-    flip = np.any(O.topk(lz, cfgG.k) != O.topk(lzp, cfgG.k), axis=1)
-    tieG = near_tie_tokens(lz, cfgG.k, 5e-3) | flip
-    keep = ~(tieF | tieG)
-    assert keep.mean() > 0.8
-    gz, gzp = O.layer_forward(z, LG), O.layer_forward(zp, LG)
-    spread = rel_err(gzp[keep], gz[keep])
-    e1 = rel_err_bf16_out(y1.cpu().numpy()[keep] - x1[keep], f_ref[keep])
-    e2 = rel_err_bf16_out(y2.cpu().numpy()[keep] - x2[keep], (o2 - x2)[keep])
-    print(f"SPREAD coupling-{T}x{d} y2: err {e2:.3e} spread {spread:.3e} bound {TOL + 2 * spread:.3e}")
+    # G reads bf16(y1) of the GPU's own y1: the oracle's G runs on exactly that
+    # input, so G's branch is compared without F's rounding in between.
+    z = O.round_bf16(y1.cpu().numpy().astype(np.float64))
+    tieG = near_tie_tokens(O.router_logits(z, LG), cfgG.k, 1e-4)
+    g_ref = O.layer_forward(z, LG)
+    e1 = rel_err_bf16_out(y1.cpu().numpy()[~tieF] - x1[~tieF], f_ref[~tieF])
+    e2 = rel_err_bf16_out(y2.cpu().numpy()[~tieG] - x2[~tieG], g_ref[~tieG])
+    print(f"COUPLING {T}x{d}: y1 - x1 err {e1:.3e}, y2 - x2 err {e2:.3e} (tokens kept {np.mean(~tieF):.3f}, "
+          f"{np.mean(~tieG):.3f})")
+    assert np.mean(~tieF) > 0.95 and np.mean(~tieG) > 0.95
     assert e1 <= TOL, e1
-    assert e2 <= TOL + 2 * spread, (e2, spread)
+    assert e2 <= TOL, e2
 
 
 def test_rev_couple_full_size_reconstruction():

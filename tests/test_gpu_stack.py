@@ -3,12 +3,18 @@ fp64 oracle.
 
 * One block is the coupling: rev_stack_* at L = 1 equals rev_couple_fwd,
   rev_couple_inv and tqp_adapter_bwd bit for bit.
-* Three blocks of mid-size layers: the forward's residual branches (y - x),
-  the reconstruction after the inverse at every depth (max|x - inv(fwd(x))| /
-  RMS(x) <= 5e-3), and dx1, dx2 and the adapter gradients of all six layers
-  from the backward. The GPU carries bf16-rounded layer outputs through its
-  own trajectory; the bound is TOL plus twice the oracle's own spread when
-  every layer output moves by 2^-8 relative (as for the single block).
+* Reconstruction of the inputs after the inverse at every depth 1..3 of a
+  sparse (16 experts, top-4) stack: max|x - inv(fwd(x))| / RMS(x) <= 5e-3.
+* Three blocks against the oracle: the forward's residual branches (y - x) and
+  dx1, dx2 and the adapter gradients of all six layers from the backward. The
+  GPU carries bf16-rounded layer outputs through its own trajectory, so the
+  layers after the first see inputs that differ from the oracle's by that
+  rounding. With sparse routing a handful of those differences flip a token's
+  expert set and move whole expert sums; this comparison therefore uses layers
+  whose every token reaches every expert (top-4 of 4, gates still a softmax of
+  the logits), where the outputs are smooth in the inputs. The bound is TOL;
+  the oracle's own spread when every layer output moves by 2^-8 relative is
+  printed beside each error for scale.
 
 The layers' base weights and LoRA B are scaled by 1/2 (synth's w_mult): with
 unscaled random weights the un-normalised SwiGLU branches grow quadratically
@@ -32,6 +38,7 @@ if torch.cuda.is_available():
 
 TOL = 2e-2
 STK = synth.LayerConfig("stk", T=384, d=256, E=16, k=4, f=256, g=64, r=16, w_mult=0.5)
+STK_DENSE = synth.LayerConfig("stkd", T=384, d=256, E=4, k=4, f=256, g=64, r=16, w_mult=0.5)
 
 
 @pytest.fixture(scope="module", autouse=True)
@@ -99,9 +106,33 @@ def _perturbed_forward(x1, x2, blocks, rng):
     return a1, a2
 
 
-def test_stack_of_three_blocks_matches_oracle():
+def test_stack_reconstruction_at_every_depth():
     cfg, L = STK, 3
     rawF, rawG = layers(L)
+    F, G, _ = gpu_stack(rawF, rawG)
+    T, d = cfg.T, cfg.d
+    x1b, x2b = synth.make_tokens(T, d, 2), synth.make_tokens(T, d, 3)
+    x1, x2 = O.bf16_to_f64(x1b), O.bf16_to_f64(x2b)
+    rms = np.sqrt(np.mean(np.concatenate([x1, x2]) ** 2))
+    st = Q.Status()
+    for depth in range(1, L + 1):
+        sub = Q.ReversibleStack(F[:depth], G[:depth])
+        y1 = torch.empty(T, d, dtype=torch.float32, device="cuda")
+        y2 = torch.empty_like(y1)
+        Q.rev_stack_fwd(dev_bf16(x1b), dev_bf16(x2b), sub, y1, y2, status=st)
+        r1 = torch.empty(T, d, dtype=torch.int16, device="cuda")
+        r2 = torch.empty_like(r1)
+        Q.rev_stack_inv(y1, y2, sub, r1, r2, status=st)
+        torch.cuda.synchronize()
+        assert st.read() == 0
+        err = max(np.max(np.abs(host_bf16(r1) - x1)), np.max(np.abs(host_bf16(r2) - x2))) / rms
+        print(f"STACK depth {depth}: reconstruction max|x - inv(fwd(x))| / RMS(x) = {err:.3e}")
+        assert err <= 5e-3, (depth, err)
+
+
+def test_stack_of_three_blocks_matches_oracle():
+    cfg, L = STK_DENSE, 3
+    rawF, rawG = layers(L, cfg)
     F, G, stack = gpu_stack(rawF, rawG)
     blocks = [(O.Layer(f), O.Layer(g)) for f, g in zip(rawF, rawG)]
     T, d = cfg.T, cfg.d
@@ -112,18 +143,6 @@ def test_stack_of_three_blocks_matches_oracle():
     st = Q.Status()
     f32 = lambda: torch.empty(T, d, dtype=torch.float32, device="cuda")
     b16 = lambda: torch.empty(T, d, dtype=torch.int16, device="cuda")
-    # reconstruction at every depth 1..L (prefix stacks)
-    for depth in range(1, L + 1):
-        sub = Q.ReversibleStack(F[:depth], G[:depth])
-        y1, y2 = f32(), f32()
-        Q.rev_stack_fwd(dev_bf16(x1b), dev_bf16(x2b), sub, y1, y2, status=st)
-        r1, r2 = b16(), b16()
-        Q.rev_stack_inv(y1, y2, sub, r1, r2, status=st)
-        torch.cuda.synchronize()
-        assert st.read() == 0
-        err = max(np.max(np.abs(host_bf16(r1) - x1)), np.max(np.abs(host_bf16(r2) - x2))) / rms
-        print(f"STACK depth {depth}: reconstruction max|x - inv(fwd(x))| / RMS(x) = {err:.3e}")
-        assert err <= 5e-3, (depth, err)
     # forward values (the residual branches) against the oracle
     y1, y2 = f32(), f32()
     Q.rev_stack_fwd(dev_bf16(x1b), dev_bf16(x2b), stack, y1, y2, status=st)
@@ -132,8 +151,8 @@ def test_stack_of_three_blocks_matches_oracle():
     g1, g2 = y1.cpu().numpy().astype(np.float64), y2.cpu().numpy().astype(np.float64)
     for name, g, o, p, x in (("y1", g1, o1, p1, x1), ("y2", g2, o2, p2, x2)):
         err, spread = rel_err(g - x, o - x), rel_err(p - x, o - x)
-        print(f"SPREAD stack-3 {name} - x: err {err:.3e} spread {spread:.3e} bound {TOL + 2 * spread:.3e}")
-        assert err <= TOL + 2 * spread, (name, err, spread)
+        print(f"SPREAD stack-3 {name} - x: err {err:.3e} spread {spread:.3e} bound {TOL:.1e}")
+        assert err <= TOL, (name, err, spread)
     # backward from the GPU's outputs
     gF, gG, arrays = stack.grads()
     r1, r2, dx1, dx2 = b16(), b16(), f32(), f32()
@@ -148,8 +167,8 @@ def test_stack_of_three_blocks_matches_oracle():
 
     def check(name, g, r, q):
         err, spread = rel_err(g, r), rel_err(q, r)
-        print(f"SPREAD stack-3 {name}: err {err:.3e} spread {spread:.3e} bound {TOL + 2 * spread:.3e}")
-        assert err <= TOL + 2 * spread, (name, err, spread)
+        print(f"SPREAD stack-3 {name}: err {err:.3e} spread {spread:.3e} bound {TOL:.1e}")
+        assert err <= TOL, (name, err, spread)
 
     check("dx1", dx1.cpu().numpy(), ref["dx1"], pert["dx1"])
     check("dx2", dx2.cpu().numpy(), ref["dx2"], pert["dx2"])
