@@ -106,7 +106,7 @@ def measured_traffic(kernel: str) -> int | None:
         return None
     doc = json.load(open(path))
     h = hashlib.sha256()
-    for f in ("expert_ffn.cu", "expert_down.cu", "expert_common.cuh", "gemm_common.cuh", "tqp_device.cuh"):
+    for f in ("expert_gateup.cu", "expert_down.cu", "expert_common.cuh", "gemm_common.cuh", "tqp_device.cuh"):
         with open(os.path.join(ROOT, "quantized_base_lora_moe_b200", "csrc", f), "rb") as fh:
             h.update(fh.read())
     if h.hexdigest()[:16] != doc.get("kernel_sources_sha256_16"):

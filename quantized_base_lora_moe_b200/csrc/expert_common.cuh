@@ -1,4 +1,4 @@
-// Epilogue helpers shared by the expert kernels (expert_ffn.cu, expert_down.cu).
+// Epilogue helpers shared by the expert kernels (expert_gateup.cu, expert_down.cu).
 #pragma once
 
 #include <cstdint>

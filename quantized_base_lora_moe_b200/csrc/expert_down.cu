@@ -4,7 +4,7 @@
 // weights: "Reversible Sparse MoE Single Node", Pattern 3; SwiGLU experts, TQP
 // Quantization).
 //
-// As in the gate/up kernel (expert_ffn.cu), the contraction runs transposed, D[feature][token] =
+// As in the gate/up kernel (expert_gateup.cu), the contraction runs transposed, D[feature][token] =
 // Wd[feature][:] . H[token][:], with the dequantised 128-feature weight tile as
 // the tcgen05.mma A operand in TMEM and the expert's routed rows as the B
 // operand in shared memory. Here a unit takes up to 256 rows of one expert, so

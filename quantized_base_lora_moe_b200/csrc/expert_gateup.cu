@@ -1,0 +1,489 @@
+// Gate/up expert projection of the TQP MoE layer with wide token blocks and the
+// dequantised base weights in tensor memory (sm_100a, tcgen05):
+//   [G|U] = X_e [Wg|Wu]^T + (s X [Ag|Au]) [Bg|Bu],  H = silu(G) * U
+// (low-rank adapters trained per expert over frozen quantised base expert
+// weights: "Reversible Sparse MoE Single Node", Pattern 3; SwiGLU experts, TQP
+// Quantization).
+//
+// The contraction runs transposed, D[feature][token] = W[feature][:] . X[token][:].
+// One work unit is (expert e, 64-feature tile, block of up to 256 routed rows):
+// the A operand (M = 128, in TMEM) stacks the tile's 64 gate rows on its 64 up
+// rows, so a single tcgen05.mma of 128 x N x 16 (N = the block's rows rounded
+// up to 16, up to 256) serves both projections, and each weight tile is
+// dequantised once per 256-row block (once per expert for all but the largest
+// experts). The token rows come expert-sorted (X_perm, written by the prepare
+// step) as TMA boxes of 128 rows, so no thread gathers rows.
+//
+// Per CTA (1 per SM, 896 threads):
+//   warps 0-3, 24-27  epilogue, two groups taking alternate 32-token chunks:
+//               drain the accumulator lane by lane (TMEM lane = one gate or up
+//               feature), hand TMEM back, then SwiGLU and 16-byte row stores
+//               through a [token][feature] tile per group
+//   warp  4     TMEM allocation + one thread issuing tcgen05.mma
+//   warp  5     TMA producer of the code / bf16 scale ring (int4 rows
+//               32B-swizzled, int8 rows 64B-swizzled: conflict-free row reads)
+//   warp  6     TMA producer of the token ring: X_perm boxes, and the rank-space
+//               rows s X [Ag|Au] for the adapter stage
+//   warps 8-23  weight producer, four groups of 4 warps on stages n % 4: each
+//               thread dequantises 64 K values of one weight row (int4 or int8
+//               -> fp16) into TMEM; LoRA B rows for the adapter stage
+// TMEM (512 columns): one accumulator in [0, 256) (lanes 0-63 gate, 64-127 up),
+// 8 weight stages of 32 columns (64 K values) in [256, 512). Token ring: 3
+// stages of 32 KB. Range: an H (or kept G|U) value or a LoRA B value beyond the
+// fp16 range raises TQP_STATUS_NONFINITE; a group scale whose dequantised
+// products are not exact in fp16 raises TQP_STATUS_RANGE. Every wait is bounded
+// (tqp_device.cuh); on an abort every asynchronous copy and MMA still in flight
+// is drained before the CTA frees its memory. No TMA multicast is used.
+#include <cstdint>
+#include <cuda.h>
+#include <cuda_fp16.h>
+#include <cuda_runtime.h>
+
+#include "expert_common.cuh"
+#include "gemm_common.cuh"
+#include "tqp_device.cuh"
+#include "tqp_launch.h"
+
+namespace tqp {
+namespace gu_wide {
+
+constexpr int kRows = 256;            // routed rows per unit
+constexpr int kF = 64;                // features per unit, of gate and of up each
+constexpr int kK = 64;                // K per pipeline stage
+constexpr int kXStages = 3;
+constexpr int kXStageBytes = kRows * kK * 2;   // 256 rows x 128 B, 128B-swizzled
+constexpr int kWStages = 8;
+constexpr uint32_t kWCols = 32;       // TMEM columns per weight stage (64 fp16 K values)
+constexpr uint32_t kWBase = 256;
+constexpr int kQStagesMax = 8;
+constexpr int kGroups = 4;            // weight-producer groups
+constexpr int kWWarp0 = 8;            // first weight-producer warp (a multiple of 4)
+constexpr int kWWarps = 16;
+constexpr int kEpi1Warp0 = kWWarp0 + kWWarps;   // second epilogue group (4 warps)
+constexpr int kThreads = (kEpi1Warp0 + 4) * 32;
+constexpr int kDRow = 528;            // drain row: 256 tokens in fp16 + 16 B against bank conflicts
+constexpr int kHRow = 144;            // chunk tile row: one token's 64 features in fp16 + 16 B
+constexpr int kStaging = 128 * kDRow + 2 * 32 * kHRow;
+
+struct Ctl {
+  uint64_t x_full[kXStages], x_empty[kXStages];
+  uint64_t w_full[kWStages], w_empty[kWStages];
+  uint64_t q_full[kQStagesMax], q_empty[kQStagesMax];
+  uint64_t acc_full, acc_empty;
+  uint64_t drain;
+  uint64_t epi[2];
+  uint32_t tmem_base;
+  Abort ab;
+};
+
+// Code ring per code width: a stage holds 64 K values of the tile's 64 gate
+// rows and 64 up rows (32 B per row for int4, 64 B for int8; TMA 32B / 64B
+// swizzle) and up to 2 x 2 x 64 scales.
+template <int BITS>
+struct QCfg {
+  static constexpr int kCB = 8 * BITS;                 // code bytes per row and stage
+  static constexpr int kStages = BITS == 4 ? 8 : 5;
+  static constexpr int kStageBytes = 128 * kCB + 512;
+  // 16-byte chunk c of row r of one 64-row box, as the TMA swizzle placed it
+  __device__ static __forceinline__ int chunk_offset(int r, int c) {
+    return r * kCB + ((BITS == 4 ? (c ^ ((r >> 2) & 1)) : (c ^ ((r >> 1) & 3))) << 4);
+  }
+};
+
+template <int BITS>
+constexpr size_t smem_bytes() {
+  return 1024 + size_t(kXStages) * kXStageBytes + size_t(QCfg<BITS>::kStages) * QCfg<BITS>::kStageBytes +
+         size_t(kStaging) + sizeof(Ctl);
+}
+static_assert(smem_bytes<4>() + 2 * (kSchedSmemE + 1) * 4 <= 232448, "shared memory budget");
+static_assert(smem_bytes<8>() + 2 * (kSchedSmemE + 1) * 4 <= 232448, "shared memory budget");
+
+// 16 tokens x this lane's feature (8 words of fp16 pairs, word j = tokens
+// t0+2j, t0+2j+1) into the [token][64 feature] chunk tile: lane pairs trade
+// halves so that each lane writes two adjacent features of one token as one
+// 32-bit word.
+__device__ __forceinline__ void stage16(uint8_t* tile, int t0, int feat, const uint32_t* w) {
+  const bool odd = (threadIdx.x & 1) != 0;
+  uint8_t* colp = tile + (feat & ~1) * 2;
+#pragma unroll
+  for (int j = 0; j < 8; ++j) {
+    const uint32_t other = __shfl_xor_sync(0xFFFFFFFFu, w[j], 1);
+    const uint32_t v = odd ? __byte_perm(other, w[j], 0x7632) : __byte_perm(w[j], other, 0x5410);
+    *reinterpret_cast<uint32_t*>(colp + (t0 + 2 * j + (odd ? 1 : 0)) * kHRow) = v;
+  }
+}
+
+template <int BITS>
+__global__ void __launch_bounds__(kThreads, 1)
+    gateup_wide_kernel(const GemmArgs a, const __grid_constant__ CUtensorMap tq0, const __grid_constant__ CUtensorMap tq1,
+                       const __grid_constant__ CUtensorMap ts0, const __grid_constant__ CUtensorMap ts1,
+                       const __grid_constant__ CUtensorMap tx, const __grid_constant__ CUtensorMap txa) {
+  using QC = QCfg<BITS>;
+  constexpr int kQStages = QC::kStages;
+  constexpr int kQStageBytes = QC::kStageBytes;
+  constexpr int kCB = QC::kCB;
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  uint8_t* x_base = smem;
+  uint8_t* q_base = x_base + size_t(kXStages) * kXStageBytes;
+  uint8_t* staging = q_base + size_t(kQStages) * kQStageBytes;
+  Ctl* ctl = reinterpret_cast<Ctl*>(staging + kStaging);
+  Abort* abort_flag = &ctl->ab;
+
+  const int warp = threadIdx.x >> 5;
+  const int lane = threadIdx.x & 31;
+  __shared__ int32_t s_sched[2 * (kSchedSmemE + 1)];
+  const Sched sc = load_sched(a, s_sched);
+
+  if (threadIdx.x == 0) {
+    for (int i = 0; i < kXStages; ++i) {
+      mbar_init(&ctl->x_full[i], 1);
+      mbar_init(&ctl->x_empty[i], 1);
+    }
+    for (int i = 0; i < kWStages; ++i) {
+      mbar_init(&ctl->w_full[i], 128);   // one weight-producer group
+      mbar_init(&ctl->w_empty[i], 1);
+    }
+    for (int i = 0; i < kQStages; ++i) {
+      mbar_init(&ctl->q_full[i], 1);
+      mbar_init(&ctl->q_empty[i], 128);
+    }
+    mbar_init(&ctl->acc_full, 1);
+    mbar_init(&ctl->acc_empty, 256);   // both epilogue groups
+    mbar_init(&ctl->drain, 1);
+    mbar_init(&ctl->epi[0], 128);
+    mbar_init(&ctl->epi[1], 128);
+    abort_init(&ctl->ab, a.wait_ns);
+    fence_barrier_init();
+  }
+  if (warp == 4) {
+    tmem_alloc(&ctl->tmem_base, 512);
+    tmem_relinquish();
+  }
+  if (threadIdx.x == 5 * 32) {
+    prefetch_tmap(&tq0);
+    prefetch_tmap(&tq1);
+    prefetch_tmap(&ts0);
+    prefetch_tmap(&ts1);
+  }
+  if (threadIdx.x == 6 * 32) {
+    prefetch_tmap(&tx);
+    if (a.nkb_lora > 0) prefetch_tmap(&txa);
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem_base = ctl->tmem_base;
+
+  const int nunits = total_units(a, sc);
+  UnitStream us{a.unit_tab, nunits, int(gridDim.x)};
+  us.start(blockIdx.x);
+  const int nkb = a.nkb_main + a.nkb_lora;
+  const int ngrp = a.g >= kK ? 1 : kK / a.g;   // scale rows per K stage
+
+  if (warp < 4 || warp >= kEpi1Warp0) {
+    // ------------------------------------------------------------ epilogue
+    const int eg = warp < 4 ? 0 : 1;           // group: 32-token chunks with (c / 32) % 2 == eg
+    const int lrow = 32 * (warp & 3) + lane;   // TMEM lane: gate feature lrow (< 64) or up feature lrow - 64
+    const int etid = lrow;                     // thread index within the group
+    const uint32_t tl = tmem_base + (uint32_t(32 * (warp & 3)) << 16);
+    uint8_t* drow = staging + lrow * kDRow;
+    uint8_t* ct = staging + 128 * kDRow + eg * 32 * kHRow;
+    // SwiGLU assignment: feature j of the tile, tokens [16 hh, 16 hh + 16) of each chunk
+    const int j = etid & 63, hh = etid >> 6;
+    const uint8_t* grow = staging + j * kDRow;
+    const uint8_t* urow = staging + (64 + j) * kDRow;
+    EpiSync es{&ctl->epi[eg]};
+    uint32_t bad = 0;   // nonzero once an fp16 output of a valid token overflowed
+    int it = 0;
+    for (int u = blockIdx.x; u < nunits; u += gridDim.x, ++it) {
+      const Unit un = us.take(u);
+      const int n16 = (un.rows + 15) & ~15;
+      if (!__all_sync(0xFFFFFFFFu, mbar_wait<128>(&ctl->acc_full, uint32_t(it) & 1u, abort_flag, a.status))) break;
+      tc_fence_after();
+      // drain this group's chunks of this lane's row as fp16
+#pragma unroll 1
+      for (int c = 32 * eg; c < n16; c += 64) {
+        float v[32];
+        tmem_ld32(tl + uint32_t(c), v);
+        uint4* dst = reinterpret_cast<uint4*>(drow + 2 * c);
+#pragma unroll
+        for (int q4 = 0; q4 < 4; ++q4)
+          dst[q4] = make_uint4(f32x2_to_f16x2(v[8 * q4], v[8 * q4 + 1]), f32x2_to_f16x2(v[8 * q4 + 2], v[8 * q4 + 3]),
+                               f32x2_to_f16x2(v[8 * q4 + 4], v[8 * q4 + 5]),
+                               f32x2_to_f16x2(v[8 * q4 + 6], v[8 * q4 + 7]));
+      }
+      tc_fence_before();
+      mbar_arrive(&ctl->acc_empty);
+      // the group's gate and up rows of its chunks are complete
+      if (!es.sync(abort_flag, a.status)) break;
+      uint16_t* hout = static_cast<uint16_t*>(a.out) + un.nt * kF;
+      bool stop = false;
+#pragma unroll 1
+      for (int c = 32 * eg; c < n16; c += 64) {
+        const int nt = min(32, un.rows - c);
+        auto words8 = [&](const uint8_t* src, uint32_t* w) {
+          const uint4 v0 = *reinterpret_cast<const uint4*>(src + 2 * (c + 16 * hh));
+          const uint4 v1 = *reinterpret_cast<const uint4*>(src + 2 * (c + 16 * hh) + 16);
+          w[0] = v0.x; w[1] = v0.y; w[2] = v0.z; w[3] = v0.w;
+          w[4] = v1.x; w[5] = v1.y; w[6] = v1.z; w[7] = v1.w;
+        };
+        // one [32 token][64 feature] chunk through the tile: wait until the tile
+        // is free, transpose into it, wait until complete, 16-byte row stores
+        auto emit = [&](const uint32_t* w, uint16_t* dst, size_t ld) -> bool {
+          if (!es.sync(abort_flag, a.status)) return false;
+          stage16(ct, 16 * hh, j, w);
+          if (!es.sync(abort_flag, a.status)) return false;
+          // (only valid tokens are stored and checked: padding columns hold stale data)
+          for (int p = etid; p < nt * 8; p += 128) {
+            const int t = p >> 3, fg = p & 7;
+            const uint4 v = *reinterpret_cast<const uint4*>(ct + t * kHRow + fg * 16);
+            bad |= f16x2_nonfinite(v.x) | f16x2_nonfinite(v.y) | f16x2_nonfinite(v.z) | f16x2_nonfinite(v.w);
+            *reinterpret_cast<uint4*>(dst + size_t(un.base + c + t) * ld + fg * 8) = v;
+          }
+          return true;
+        };
+        uint32_t hw[8];
+        {
+          uint32_t gw[8], uw[8];
+          words8(grow, gw);
+          words8(urow, uw);
+#pragma unroll
+          for (int q = 0; q < 8; ++q) hw[q] = swiglu_pair(gw[q], uw[q]);
+        }
+        if (!emit(hw, hout, size_t(a.out_ld))) { stop = true; break; }
+        if (a.aux) {  // keep the pre-activations for the backward: G in [0, f), U in [f, 2f)
+          uint16_t* aux = a.aux + un.nt * kF;
+          uint32_t w8[8];
+          words8(grow, w8);
+          if (!emit(w8, aux, 2 * size_t(a.f_dim))) { stop = true; break; }
+          words8(urow, w8);
+          if (!emit(w8, aux + a.f_dim, 2 * size_t(a.f_dim))) { stop = true; break; }
+        }
+      }
+      if (stop) break;
+    }
+    if (__any_sync(0xFFFFFFFFu, bad != 0) && lane == 0) raise_status(a.status, TQP_STATUS_NONFINITE);
+  } else if (warp == 4) {
+    // ------------------------------------------------------------ MMA issuer
+    if (lane == 0) {
+      Ring rx, rw;
+      int it = 0;
+      bool ok = true;
+      for (int u = blockIdx.x; u < nunits && ok; u += gridDim.x, ++it) {
+        const Unit un = us.take(u);
+        const int n16 = (un.rows + 15) & ~15;
+        const uint32_t idesc = idesc_f16(128, n16);
+        if (!mbar_wait(&ctl->acc_empty, (uint32_t(it) & 1u) ^ 1u, abort_flag, a.status)) { ok = false; break; }
+        tc_fence_after();
+        for (int kb = 0; kb < nkb; ++kb) {
+          if (!mbar_wait(&ctl->x_full[rx.stage], rx.phase, abort_flag, a.status) ||
+              !mbar_wait(&ctl->w_full[rw.stage], rw.phase, abort_flag, a.status)) {
+            ok = false;
+            break;
+          }
+          tc_fence_after();
+          const uint64_t bdesc = sdesc_k_sw128(smem_u32(x_base + size_t(rx.stage) * kXStageBytes));
+          const uint32_t wa = tmem_base + kWBase + uint32_t(rw.stage) * kWCols;
+          // the rank-space stage has only its first lora_k columns live (within the first 64)
+          const int ksteps = (kb >= a.nkb_lora) ? 4 : (min(kK, a.lora_k - kb * kK) + 15) / 16;
+          for (int kk = 0; kk < ksteps; ++kk)
+            umma_f16_ts(tmem_base, wa + uint32_t(8 * kk), bdesc + uint64_t(2 * kk), idesc, (kb > 0 || kk > 0) ? 1u : 0u);
+          umma_commit(&ctl->x_empty[rx.stage]);
+          umma_commit(&ctl->w_empty[rw.stage]);
+          rx.next<kXStages>();
+          rw.next<kWStages>();
+        }
+        if (!ok) break;
+        umma_commit(&ctl->acc_full);
+      }
+      // no MMA may still read or write TMEM when it is freed: wait for all of
+      // them (they run to completion whether or not the CTA aborted)
+      umma_commit(&ctl->drain);
+      mbar_drain(&ctl->drain, 0, 100000000ull);
+    }
+    __syncwarp();
+  } else if (warp == 5) {
+    // ------------------------------------------------------------ TMA producer (codes + scales)
+    if (lane == 0) {
+      Ring q;
+      PendingFills pend;
+      // gate codes [64 rows][kCB B] | up codes | gate scales [ngrp][64] | up scales
+      const uint32_t bytes = uint32_t(128 * kCB + 256 * ngrp);
+      const int gpe = a.in_dim / a.g;  // scale rows per expert
+      for (int u = blockIdx.x; u < nunits; u += gridDim.x) {
+        const Unit un = us.take(u);
+        const int nrow0 = un.e * a.out_dim + un.nt * kF;
+        bool ok = true;
+        for (int km = 0; km < a.nkb_main; ++km) {
+          if (!mbar_wait<64>(&ctl->q_empty[q.stage], q.phase ^ 1u, abort_flag, a.status)) { ok = false; break; }
+          uint8_t* qs = q_base + size_t(q.stage) * kQStageBytes;
+          uint64_t* bar = &ctl->q_full[q.stage];
+          const int srow = un.e * gpe + (km * kK) / a.g;
+          mbar_arrive_expect_tx(bar, bytes);
+          tma_load_2d(smem_u32(qs), &tq0, bar, km * kCB, nrow0);
+          tma_load_2d(smem_u32(qs + 64 * kCB), &tq1, bar, km * kCB, nrow0);
+          tma_load_2d(smem_u32(qs + 128 * kCB), &ts0, bar, un.nt * kF, srow);
+          tma_load_2d(smem_u32(qs + 128 * kCB + 128 * ngrp), &ts1, bar, un.nt * kF, srow);
+          pend.issued(q.stage, q.phase);
+          q.next<kQStages>();
+        }
+        if (!ok) break;
+      }
+      // on an abort, wait (bounded) until every issued fill has landed
+      if (aborted(abort_flag)) pend.drain(ctl->q_full);
+    }
+  } else if (warp == 6) {
+    // ------------------------------------------------------------ TMA producer (token rows)
+    if (lane == 0) {
+      Ring rx;
+      PendingFills pend;
+      for (int u = blockIdx.x; u < nunits; u += gridDim.x) {
+        const Unit un = us.take(u);
+        const int nbox = un.rows > 128 ? 2 : 1;   // a second 128-row box only when the MMA reads it
+        bool ok = true;
+        for (int kb = 0; kb < nkb; ++kb) {
+          if (!mbar_wait<64>(&ctl->x_empty[rx.stage], rx.phase ^ 1u, abort_flag, a.status)) { ok = false; break; }
+          uint8_t* st = x_base + size_t(rx.stage) * kXStageBytes;
+          uint64_t* bar = &ctl->x_full[rx.stage];
+          // the adapter stage reads s X [Ag|Au] (zero-filled past its 2r columns), the rest X_perm
+          const CUtensorMap* map = kb < a.nkb_lora ? &txa : &tx;
+          const int col = (kb < a.nkb_lora ? kb : kb - a.nkb_lora) * kK;
+          mbar_arrive_expect_tx(bar, uint32_t(nbox * (kXStageBytes / 2)));
+          tma_load_2d(smem_u32(st), map, bar, col, un.base);
+          if (nbox == 2) tma_load_2d(smem_u32(st + kXStageBytes / 2), map, bar, col, un.base + 128);
+          pend.issued(rx.stage, rx.phase);
+          rx.next<kXStages>();
+        }
+        if (!ok) break;
+      }
+      if (aborted(abort_flag)) pend.drain(ctl->x_full);
+    }
+  } else if (warp >= kWWarp0) {
+    // ------------------------------------------------------------ weight producer
+    // Four groups of 4 warps take stages n % 4, so that four stages are being
+    // dequantised at any time (one stage's chain of code read -> dequant ->
+    // TMEM store -> arrive is latency-bound). A thread converts 64 consecutive
+    // K values (8 int4 words) of one weight row: TMEM lane lrow, the gate row
+    // of feature lrow (lrow < 64) or the up row of feature lrow - 64.
+    const int wi = warp - kWWarp0;            // 0..15
+    const int grp = wi >> 2;                  // stages n with n % 4 == grp
+    const int lrow = 32 * (warp & 3) + lane;  // TMEM lane
+    const int mat = lrow >> 6;                // 0 gate, 1 up
+    const int r64 = lrow & 63;                // row within the tile's gate / up box
+    const uint32_t tw = tmem_base + (uint32_t(32 * (warp & 3)) << 16) + kWBase;
+    const int row_off = mat * 64 * kCB;
+    // scale rows of the two 32-wide K halves of this thread's slice
+    const int g_hi = (ngrp == 1) ? 0 : 32 / a.g;
+    const int sbase = 128 * kCB + mat * 128 * ngrp;
+    const int s_lo_off = sbase + r64 * 2, s_hi_off = sbase + (g_hi * 64 + r64) * 2;
+    const uint16_t* bsrc = mat ? a.b1 : a.b0;
+    bool inexact = false;   // a group scale whose products q * s are not exact in fp16
+    bool lora_inf = false;  // a LoRA B value beyond the fp16 range
+    int n = 0;    // pipeline stage counter of this CTA
+    int m = 0;    // main (code-carrying) stage counter
+    for (int u = blockIdx.x; u < nunits; u += gridDim.x) {
+      const Unit un = us.take(u);
+      const int feat = un.nt * kF + r64;   // output feature of this row
+      bool ok = true;
+      if (a.nkb_lora > 0 && grp == 0 && u + int(gridDim.x) < nunits) {
+        // the next unit's LoRA B row into L2 (its rank-space stage comes first)
+        const Unit nx = us.peek();
+        const uint16_t* rowp = bsrc + (size_t(nx.e) * a.out_dim + nx.nt * kF + r64) * a.r;
+        for (int off = 0; off < a.r; off += 64) prefetch_l2(rowp + off);
+      }
+      for (int kb = 0; kb < nkb; ++kb, ++n) {
+        const bool main_stage = kb >= a.nkb_lora;
+        const int mq = m;
+        if (main_stage) ++m;
+        if ((n & (kGroups - 1)) != grp) continue;
+        const int st = n & (kWStages - 1);
+        const uint32_t ph = uint32_t(n / kWStages) & 1u;
+        if (!__all_sync(0xFFFFFFFFu, mbar_wait(&ctl->w_empty[st], ph ^ 1u, abort_flag, a.status))) { ok = false; break; }
+        tc_fence_after();
+        uint32_t v[32];
+        if (!main_stage) {
+          // LoRA B rows as fp16: gate rows hold Bg in K' [0, r), up rows Bu in [r, 2r)
+#pragma unroll
+          for (int c = 0; c < 8; ++c) {
+            const int colk = kb * kK + c * 8;
+            const int src = mat ? colk - a.r : colk;
+            uint4 w4 = make_uint4(0, 0, 0, 0);
+            if (src >= 0 && src < a.r)
+              w4 = bf16x8_to_f16x8_chk(
+                  __ldg(reinterpret_cast<const uint4*>(bsrc + (size_t(un.e) * a.out_dim + feat) * a.r + src)), lora_inf);
+            v[4 * c] = w4.x; v[4 * c + 1] = w4.y; v[4 * c + 2] = w4.z; v[4 * c + 3] = w4.w;
+          }
+        } else {
+          const int qst = mq % kQStages;
+          const uint32_t qph = uint32_t(mq / kQStages) & 1u;
+          if (!__all_sync(0xFFFFFFFFu, mbar_wait(&ctl->q_full[qst], qph, abort_flag, a.status))) { ok = false; break; }
+          const uint8_t* qs = q_base + size_t(qst) * kQStageBytes;
+          const uint32_t s_lo = scale_pair_chk(*reinterpret_cast<const uint16_t*>(qs + s_lo_off), inexact);
+          const uint32_t s_hi = scale_pair_chk(*reinterpret_cast<const uint16_t*>(qs + s_hi_off), inexact);
+          if (BITS == 4) {
+            // 64 K values = 8 words of 8 codes
+            const uint4 wa = *reinterpret_cast<const uint4*>(qs + row_off + QC::chunk_offset(r64, 0));
+            const uint4 wb = *reinterpret_cast<const uint4*>(qs + row_off + QC::chunk_offset(r64, 1));
+            const uint32_t wd[8] = {wa.x, wa.y, wa.z, wa.w, wb.x, wb.y, wb.z, wb.w};
+#pragma unroll
+            for (int c = 0; c < 8; ++c) {
+              const uint4 d4 = dequant_word(wd[c], c < 4 ? s_lo : s_hi);
+              v[4 * c] = d4.x; v[4 * c + 1] = d4.y; v[4 * c + 2] = d4.z; v[4 * c + 3] = d4.w;
+            }
+          } else {
+            // 64 K values = 16 words of 4 codes
+#pragma unroll
+            for (int ch = 0; ch < 4; ++ch) {
+              const uint4 w4 = *reinterpret_cast<const uint4*>(qs + row_off + QC::chunk_offset(r64, ch));
+              const uint32_t wd[4] = {w4.x, w4.y, w4.z, w4.w};
+#pragma unroll
+              for (int i = 0; i < 4; ++i) {
+                const uint2 d2 = dequant_word8(wd[i], ch < 2 ? s_lo : s_hi);
+                v[8 * ch + 2 * i] = d2.x;
+                v[8 * ch + 2 * i + 1] = d2.y;
+              }
+            }
+          }
+          // the code slot's values have been consumed; its next fill is an
+          // async-proxy TMA write, hence the proxy fence before handing it back
+          fence_proxy_async_smem();
+          mbar_arrive(&ctl->q_empty[qst]);
+        }
+        tmem_st32(tw + uint32_t(st) * kWCols, v);
+        tmem_wait_st();
+        tc_fence_before();
+        mbar_arrive(&ctl->w_full[st]);
+      }
+      if (!ok) break;
+    }
+    if (__any_sync(0xFFFFFFFFu, inexact) && lane == 0) raise_status(a.status, TQP_STATUS_RANGE);
+    if (__any_sync(0xFFFFFFFFu, lora_inf) && lane == 0) raise_status(a.status, TQP_STATUS_NONFINITE);
+  }
+
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 4) {
+    tc_fence_after();
+    tmem_dealloc(tmem_base, 512);
+  }
+}
+
+}  // namespace gu_wide
+
+template <int BITS>
+static int launch_gateup_wide(const GemmArgs& a, const Maps& mp, int units_upper, cudaStream_t s) {
+  static DeviceFlags attr_done;
+  constexpr size_t smem = gu_wide::smem_bytes<BITS>();
+  if (!attr_done.test_and_set_device(gu_wide::gateup_wide_kernel<BITS>, int(smem))) return TQP_ERR_CUDA;
+  const int grid = units_upper < num_sms() ? (units_upper > 0 ? units_upper : 1) : num_sms();
+  gu_wide::gateup_wide_kernel<BITS><<<grid, gu_wide::kThreads, smem, s>>>(a, mp.m[TQ0], mp.m[TQ1], mp.m[TS0], mp.m[TS1],
+                                                                            mp.m[TA], mp.m[TB0]);
+  return cudaGetLastError() == cudaSuccess ? TQP_OK : TQP_ERR_CUDA;
+}
+
+int run_expert_gateup_wide(const GemmArgs& a, const Maps& mp, int units_upper, cudaStream_t s) {
+  return a.bits == 8 ? launch_gateup_wide<8>(a, mp, units_upper, s) : launch_gateup_wide<4>(a, mp, units_upper, s);
+}
+
+}  // namespace tqp

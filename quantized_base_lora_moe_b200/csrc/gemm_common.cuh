@@ -207,9 +207,11 @@ struct Maps {
 };
 enum { TQ0 = 0, TQ1 = 1, TS0 = 2, TS1 = 3, TA = 4, TB0 = 5, TB1 = 6 };
 
-// Gate/up expert projection with the dequantised weights held in tensor memory
-// (expert_ffn.cu); a.bits selects int4 or int8 codes.
-int run_expert_gateup(const GemmArgs& a, const Maps& mp, int units_upper, cudaStream_t s);
+// Gate/up expert projection with the dequantised weights held in tensor memory,
+// 64 gate + 64 up features per unit over blocks of up to 256 expert-sorted rows
+// (expert_gateup.cu): TA = X_perm [A][d], TB0 = s X [Ag|Au] [A][2r] (box {64, 128}
+// each); a.bits selects int4 or int8 codes.
+int run_expert_gateup_wide(const GemmArgs& a, const Maps& mp, int units_upper, cudaStream_t s);
 
 // Down projection with blocks of up to 256 routed rows (expert_down.cu).
 int run_expert_down_wide(const GemmArgs& a, const Maps& mp, int units_upper, cudaStream_t s);

@@ -746,6 +746,25 @@ __global__ void to_f16_kernel(const uint16_t* __restrict__ x, uint16_t* __restri
   if (bad) raise_status(status, TQP_STATUS_NONFINITE);
 }
 
+// Expert-sorted token rows in fp16, X_perm[i] = x[perm_token[i]], one warp per
+// row; values beyond the fp16 range raise TQP_STATUS_NONFINITE.
+__global__ void __launch_bounds__(256) gather_rows_f16_kernel(const uint16_t* __restrict__ x,
+                                                              const int32_t* __restrict__ perm, int A, int d,
+                                                              uint16_t* __restrict__ out, int32_t* status) {
+  const int row = blockIdx.x * 8 + (threadIdx.x >> 5);
+  if (row >= A) return;
+  const int lane = threadIdx.x & 31;
+  const uint4* src = reinterpret_cast<const uint4*>(x + size_t(__ldg(perm + row)) * d);
+  uint4* dst = reinterpret_cast<uint4*>(out + size_t(row) * d);
+  uint32_t bad = 0;
+  for (int c = lane; c < d / 8; c += 32) {
+    const uint4 o = bf16x8_to_f16x8(__ldg(src + c));
+    dst[c] = o;
+    bad |= f16x2_nonfinite(o.x) | f16x2_nonfinite(o.y) | f16x2_nonfinite(o.z) | f16x2_nonfinite(o.w);
+  }
+  if (__any_sync(0xFFFFFFFFu, bad != 0) && lane == 0) raise_status(status, TQP_STATUS_NONFINITE);
+}
+
 // Router: one group covering all T tokens; split W_r into three exact bf16 parts.
 __global__ void router_prep_kernel(const float* __restrict__ wr, int n, int T, uint16_t* __restrict__ parts,
                                    int32_t* __restrict__ offsets2, int32_t* __restrict__ mbp2) {
@@ -872,7 +891,7 @@ static size_t ffn_unit_upper(int T, const tqp_moe_weights* w) {
 size_t ffn_ws_bytes(int T, const tqp_moe_weights* w) {
   const size_t A = size_t(T) * w->top_k;
   size_t b = 2 * align_up(size_t(w->E + 1) * 4, 256);          // block prefixes (128- and 256-row blocks)
-  b += align_up(size_t(T) * w->d * 2, 256);                    // x in fp16
+  b += align_up(A * w->d * 2, 256);                            // X_perm (or x) in fp16
   if (w->rank > 0) {
     b += align_up(A * 2 * w->rank * 2, 256);                    // xa [A][2r]
     b += align_up(A * w->rank * 2, 256);                        // ha [A][r]
@@ -891,7 +910,8 @@ FfnBufs ffn_carve(void* ws, int T, const tqp_moe_weights* w) {
   b.mb_prefix256 = reinterpret_cast<int32_t*>(p);
   p += align_up(size_t(w->E + 1) * 4, 256);
   b.x16 = reinterpret_cast<uint16_t*>(p);
-  p += align_up(size_t(T) * w->d * 2, 256);
+  b.xperm = b.x16;
+  p += align_up(A * w->d * 2, 256);
   if (w->rank > 0) {
     b.xa = reinterpret_cast<uint16_t*>(p);
     p += align_up(A * 2 * w->rank * 2, 256);
@@ -935,7 +955,12 @@ int launch_grouped_ffn_part(int part, const uint16_t* x, int T, const int32_t* o
     schedule_kernel<<<1, 1024, 0, s>>>(offsets, w->E, fb.mb_prefix, kMBlock);
     schedule_kernel<<<1, 1024, 0, s>>>(offsets, w->E, fb.mb_prefix256, 256);
     if (cudaGetLastError() != cudaSuccess) return TQP_ERR_CUDA;
-    if ((rc = to_f16(x, fb.x16, size_t(T) * d, status, s)) != TQP_OK) return rc;
+    if (f % 128 == 0) {   // the wide gate/up kernel reads expert-sorted rows by TMA
+      gather_rows_f16_kernel<<<unsigned((A + 7) / 8), 256, 0, s>>>(x, perm_token, int(A), d, fb.xperm, status);
+      if (cudaGetLastError() != cudaSuccess) return TQP_ERR_CUDA;
+    } else if ((rc = to_f16(x, fb.x16, size_t(T) * d, status, s)) != TQP_OK) {
+      return rc;
+    }
     if (r > 0 && (rc = to_f16(w->lora_a[2], fb.adT16, size_t(w->E) * r * f, status, s)) != TQP_OK) return rc;
   }
   // an upper bound on the number of work units (grid sizing only)
@@ -970,16 +995,54 @@ int launch_grouped_ffn_part(int part, const uint16_t* x, int T, const int32_t* o
       return TQP_ERR_CUDA;
     if ((rc = run_gemm<LORA_XA>(a, mp, mb_upper, s)) != TQP_OK) return rc;
   }
-  // The forward projections run with the weights in TMEM (expert_ffn.cu) when the
-  // hidden width is a multiple of 128 (its K stages and feature tiles), else on
-  // the shared-memory engine above.
+  // The forward projections run with the weights in TMEM (expert_gateup.cu,
+  // expert_down.cu) when the hidden width is a multiple of 128, else on the
+  // shared-memory engine.
   const bool tm = (f % 128 == 0);
-  if (part == 1) {  // H = silu(G) * U
+  if (part == 1 && tm) {  // H = silu(G) * U: 64 gate + 64 up features x up to 256 rows per unit
+    GemmArgs a = base;
+    a.mb_prefix = fb.mb_prefix256;
+    a.nkb_main = d / 64;
+    a.nkb_lora = r > 0 ? (2 * r + 63) / 64 : 0;
+    a.lora_k = 2 * r;
+    a.n_tiles = f / 64;
+    a.in_dim = d;
+    a.out_dim = f;
+    a.b0 = w->lora_b[0];
+    a.b1 = w->lora_b[1];
+    a.out = h;
+    a.out_ld = f;
+    a.n_valid = f;
+    a.aux = aux_gu;
+    a.f_dim = f;
+    const int ngrp = w->group >= 64 ? 1 : 64 / w->group;
+    const uint32_t cbox = uint32_t(8 * bB);   // 64 K values: 32-byte int4 / 64-byte int8 code rows
+    const uint64_t crow = uint64_t(d) * bB / 8;
+    Maps mp{};
+    bool ok = make_map(&mp.m[TQ0], CU_TENSOR_MAP_DATA_TYPE_UINT8, w->wq[0], crow, uint64_t(w->E) * f, crow, cbox, 64,
+                       int(cbox)) &&
+              make_map(&mp.m[TQ1], CU_TENSOR_MAP_DATA_TYPE_UINT8, w->wq[1], crow, uint64_t(w->E) * f, crow, cbox, 64,
+                       int(cbox)) &&
+              make_map(&mp.m[TS0], CU_TENSOR_MAP_DATA_TYPE_UINT16, w->wscale[0], f, uint64_t(w->E) * (d / w->group),
+                       uint64_t(f) * 2, 64, ngrp) &&
+              make_map(&mp.m[TS1], CU_TENSOR_MAP_DATA_TYPE_UINT16, w->wscale[1], f, uint64_t(w->E) * (d / w->group),
+                       uint64_t(f) * 2, 64, ngrp) &&
+              make_tile_map(&mp.m[TA], fb.xperm, uint64_t(A), uint64_t(d), 128);
+    // the rank-space rows: 2r columns, the rest of each 64-wide box zero-filled
+    if (ok && r > 0) ok = make_tile_map(&mp.m[TB0], fb.xa, uint64_t(A), uint64_t(2 * r), 128);
+    if (!ok) return TQP_ERR_CUDA;
+    const int units_upper = int((A + 255) / 256 + w->E) * a.n_tiles;
+    if ((rc = build_unit_table(a, 256, units_upper, fb.unit_tab, s)) != TQP_OK) return rc;
+    a.unit_tab = fb.unit_tab;
+    a.wait_ns = wait_limit_ns();
+    if ((rc = run_expert_gateup_wide(a, mp, units_upper, s)) != TQP_OK) return rc;
+  }
+  if (part == 1 && !tm) {  // H = silu(G) * U on the shared-memory engine
     GemmArgs a = base;
     a.nkb_main = d / 64;
     a.nkb_lora = r > 0 ? (2 * r + 63) / 64 : 0;
     a.lora_k = 2 * r;
-    a.ntile = tm ? 256 : 128;
+    a.ntile = 128;
     a.n_tiles = f / (a.ntile / 2);
     a.in_dim = d;
     a.out_dim = f;
@@ -996,28 +1059,20 @@ int launch_grouped_ffn_part(int part, const uint16_t* x, int T, const int32_t* o
     a.f_dim = f;
     const int ngrp = w->group >= 64 ? 1 : 64 / w->group;
     const uint32_t rows_box = uint32_t(a.ntile / 2);
-    // 64 K values per stage: 32-byte int4 / 64-byte int8 code rows, swizzled for
-    // conflict-free row reads in the tensor-memory kernel
     const uint32_t cbox = uint32_t(8 * bB);
-    const int csw = tm ? int(cbox) : 0;
     const uint64_t crow = uint64_t(d) * bB / 8;
     Maps mp{};
     bool ok = make_map(&mp.m[TQ0], CU_TENSOR_MAP_DATA_TYPE_UINT8, w->wq[0], crow, uint64_t(w->E) * f, crow, cbox,
-                       rows_box, csw) &&
+                       rows_box) &&
               make_map(&mp.m[TQ1], CU_TENSOR_MAP_DATA_TYPE_UINT8, w->wq[1], crow, uint64_t(w->E) * f, crow, cbox,
-                       rows_box, csw) &&
+                       rows_box) &&
               make_map(&mp.m[TS0], CU_TENSOR_MAP_DATA_TYPE_UINT16, w->wscale[0], f, uint64_t(w->E) * (d / w->group),
                        uint64_t(f) * 2, rows_box, ngrp) &&
               make_map(&mp.m[TS1], CU_TENSOR_MAP_DATA_TYPE_UINT16, w->wscale[1], f, uint64_t(w->E) * (d / w->group),
                        uint64_t(f) * 2, rows_box, ngrp);
     if (!ok) return TQP_ERR_CUDA;
-    if (tm) {
-      if ((rc = build_unit_table(a, kMBlock, mb_upper * a.n_tiles, fb.unit_tab, s)) != TQP_OK) return rc;
-      a.unit_tab = fb.unit_tab;
-    }
     a.wait_ns = wait_limit_ns();
-    rc = tm ? run_expert_gateup(a, mp, mb_upper * a.n_tiles, s) : run_gemm<GATEUP>(a, mp, mb_upper * a.n_tiles, s);
-    if (rc != TQP_OK) return rc;
+    if ((rc = run_gemm<GATEUP>(a, mp, mb_upper * a.n_tiles, s)) != TQP_OK) return rc;
   }
   if (part == 2 && r > 0) {  // ha = s * H Ad
     GemmArgs a = base;

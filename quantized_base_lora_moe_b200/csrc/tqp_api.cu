@@ -188,7 +188,7 @@ int layer_backward(const uint16_t* x, const float* dy, int T, const tqp_moe_weig
       return rc;
     // adapter gradients, in the storage layouts A^T [r][in], B^T [out][r]: on the
     // tensor cores for ranks up to 32, else as outer products on the CUDA cores
-    rc = launch_wgrad(w, L.offsets, L.perm, B.dO, L.h, B.dgu, fb.x16, fb.ha, B.dha, fb.xa, B.dxa, g, B.dmax, status, s);
+    rc = launch_wgrad(w, L.offsets, nullptr, B.dO, L.h, B.dgu, fb.xperm, fb.ha, B.dha, fb.xa, B.dxa, g, B.dmax, status, s);
     if (rc != TQP_OK && rc != TQP_ERR_UNSUPPORTED) return rc;
   }
   if (r > 0 && rc == TQP_ERR_UNSUPPORTED) {
@@ -198,9 +198,9 @@ int layer_backward(const uint16_t* x, const float* dy, int T, const tqp_moe_weig
       return rc;
     if ((rc = launch_outer(E, f, r, L.offsets, nullptr, B.dgu, 2 * f, f, fb.xa, 2 * r, r, g->dB[1], B.dmax, s)) != TQP_OK)
       return rc;
-    if ((rc = launch_outer(E, r, d, L.offsets, L.perm, B.dxa, 2 * r, 0, fb.x16, d, 0, g->dA[0], B.dmax, s)) != TQP_OK)
+    if ((rc = launch_outer(E, r, d, L.offsets, nullptr, B.dxa, 2 * r, 0, fb.xperm, d, 0, g->dA[0], B.dmax, s)) != TQP_OK)
       return rc;
-    if ((rc = launch_outer(E, r, d, L.offsets, L.perm, B.dxa, 2 * r, r, fb.x16, d, 0, g->dA[1], B.dmax, s)) != TQP_OK)
+    if ((rc = launch_outer(E, r, d, L.offsets, nullptr, B.dxa, 2 * r, r, fb.xperm, d, 0, g->dA[1], B.dmax, s)) != TQP_OK)
       return rc;
   }
   uint16_t* dX = B.dO;  // dO is no longer needed

@@ -57,7 +57,8 @@ size_t ffn_ws_bytes(int T, const tqp_moe_weights* w);
 struct FfnBufs {
   int32_t* mb_prefix;      // per-expert prefix of 128-row blocks
   int32_t* mb_prefix256;   // per-expert prefix of 256-row blocks (the down projection)
-  uint16_t* x16;
+  uint16_t* x16;     // x in fp16 [T][d] (the shared-memory engine's gate/up fallback)
+  uint16_t* xperm;   // expert-sorted token rows in fp16 [A][d] (same region as x16)
   uint16_t* xa;
   uint16_t* ha;
   uint16_t* adT16;   // Ad^T converted to fp16 [E][r][f]

@@ -10,7 +10,8 @@
 //   kind 1  dA_down[e][j][m]  = sum h[row][m]   * dha[row][j]      (m < f,  j < r)
 //   kind 2  dB_gate[e][m][j]  = sum dG[row][m]  * xa[row][j]       (m < f,  j < r)
 //           dB_up[e][m][j]    = sum dU[row][m]  * xa[row][r + j]   (dG|dU rows are [2f], xa rows [2r])
-//   kind 3  dA_gate[e][j][m]  = sum x[tok][m]   * dxa[row][j]      (m < d,  j < r; tok = perm[row])
+//   kind 3  dA_gate[e][j][m]  = sum x[tok][m]   * dxa[row][j]      (m < d,  j < r; x[tok] = X_perm[row],
+//                                                                     or x[perm[row]] when perm is given)
 //           dA_up[e][j][m]    = sum x[tok][m]   * dxa[row][r + j]  (one unit computes both: N = 2r)
 // The operands hold the fp16 intermediates of the backward, computed for the
 // cotangent dy * 2^P; the fp32 results are scaled back by 2^-P.
@@ -78,7 +79,7 @@ struct Args {
   const uint16_t* dO;    // [A][d]
   const uint16_t* h;     // [A][f]
   const uint16_t* dgu;   // [A][2f]
-  const uint16_t* x16;   // [T][d]
+  const uint16_t* x16;   // X_perm [A][d] (perm null), or x [T][d] gathered by perm
   const uint16_t* ha;    // [A][r]
   const uint16_t* dha;   // [A][r]
   const uint16_t* xa;    // [A][2r]
@@ -276,7 +277,7 @@ __global__ void __launch_bounds__(kThreads, 1) wgrad_kernel(const Args a) {
           const int kk = c >> 4, ch = c & 15;
           const bool in = k0 + kk < w.rows;
           int prow = w.base + k0 + kk;
-          if (w.kind == 3 && in) prow = __ldg(a.perm + prow);
+          if (w.kind == 3 && in && a.perm) prow = __ldg(a.perm + prow);
           const uint16_t* src = P + size_t(in ? prow : 0) * ldp + pcol + ch * 8;
           cp_async16(as + mn_offset(kk, ch), src, in ? 16u : 0u);
         }
