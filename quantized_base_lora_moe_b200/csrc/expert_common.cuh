@@ -10,19 +10,28 @@ namespace tqp {
 
 constexpr int kTRow = 272;   // staging row: one token's 128 features in fp16, +16 B against bank conflicts
 
-// Barrier among the 128 epilogue threads (warps 0-3) only, on an mbarrier so
+// Barrier among the 4 warps of one epilogue group only, on an mbarrier so
 // that the wait is bounded: false once the CTA has aborted or the limit expired.
-struct EpiSync {
+// The barrier expects one arrival per warp when kPerWarp (else one per thread).
+template <bool kPerWarp = false>
+struct EpiSyncT {
   uint64_t* bar;
   uint32_t phase = 0;
   // The result is warp-uniform (the callers go on to warp-collective tcgen05 loads).
   __device__ __forceinline__ bool sync(Abort* abort_flag, int32_t* status) {
-    mbar_arrive(bar);
-    const bool ok = __all_sync(0xFFFFFFFFu, mbar_wait<32>(bar, phase, abort_flag, status));
+    bool ok;
+    if (kPerWarp) {
+      mbar_arrive_warp(bar);
+      ok = mbar_wait_warp<32>(bar, phase, abort_flag, status);
+    } else {
+      mbar_arrive(bar);
+      ok = __all_sync(0xFFFFFFFFu, mbar_wait<32>(bar, phase, abort_flag, status));
+    }
     phase ^= 1u;
     return ok;
   }
 };
+using EpiSync = EpiSyncT<false>;
 
 // 2*NW tokens x this lane's feature (NW words of fp16 pairs, word j = tokens
 // t0+2j, t0+2j+1) into a [token][feature] tile: lane pairs trade halves so that

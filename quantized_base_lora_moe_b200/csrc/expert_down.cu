@@ -26,13 +26,18 @@
 //   warp  4     TMEM allocation + one thread issuing tcgen05.mma
 //   warp  5     TMA producer of the code / bf16 scale ring (int4 rows
 //               32B-swizzled, int8 rows 64B-swizzled, read without bank conflicts)
-//   warps 6-9   token producer: two TMA boxes of 128 rows per 64-wide K stage;
-//               the rank-space rows (s H Ad) by coalesced cp.async
-//   warps 10-25 weight producer, two groups of 8 warps on alternate stages:
-//               each thread dequantises 32 K values of one weight row
+//   warp  6     TMA producer of the token ring: two boxes of 128 H rows per
+//               64-wide K stage, and the rank-space rows s H Ad (zero-filled
+//               past their r columns) for the adapter stage
+//   warps 7-9   idle
+//   warps 10-25 weight producer, four groups of 4 warps on stages n % 4: each
+//               thread dequantises the 64 K values of one weight row per stage
 //               (int4 or int8 -> fp16) into TMEM; LoRA B rows
 // TMEM (512 columns): one accumulator in [0, 256), 8 weight stages of 32
-// columns (64 K values) in [256, 512). Token ring: 3 stages of 32 KB.
+// columns (64 K values) in [256, 512). Token ring: 3 stages of 32 KB. Stage n is
+// ready when full[n % 8] completes (the weight group's 4 warps and the token
+// tile's TMA bytes), so the MMA thread waits once per stage; every role arrives
+// once per warp.
 // An O value of a routed row or a LoRA B value beyond the fp16 range raises
 // TQP_STATUS_NONFINITE; a group scale whose dequantised products are not exact
 // in fp16 raises TQP_STATUS_RANGE. Every wait is bounded (tqp_device.cuh); on an abort every
@@ -67,7 +72,7 @@ constexpr int kDRow = 528;             // drain row: 256 tokens in fp16 + 16 B a
 constexpr int kStaging = 128 * kDRow + 2 * 32 * kTRow;   // drain rows + one chunk tile per epilogue group
 
 struct Ctl {
-  uint64_t x_full[kXStages], x_empty[kXStages];
+  uint64_t x_empty[kXStages];
   uint64_t w_full[kWStages], w_empty[kWStages];
   uint64_t q_full[kQStagesMax], q_empty[kQStagesMax];
   uint64_t acc_full, acc_empty;
@@ -101,7 +106,7 @@ static_assert(smem_bytes<8>() + 2 * (kSchedSmemE + 1) * 4 <= 232448, "shared mem
 template <int BITS>
 __global__ void __launch_bounds__(kThreads, 1)
     down_wide_kernel(const GemmArgs a, const __grid_constant__ CUtensorMap tq, const __grid_constant__ CUtensorMap ts,
-                     const __grid_constant__ CUtensorMap th) {
+                     const __grid_constant__ CUtensorMap th, const __grid_constant__ CUtensorMap tha) {
   using QC = QCfg<BITS>;
   constexpr int kQStages = QC::kStages;
   constexpr int kQStageBytes = QC::kStageBytes;
@@ -120,23 +125,20 @@ __global__ void __launch_bounds__(kThreads, 1)
   const Sched sc = load_sched(a, s_sched);
 
   if (threadIdx.x == 0) {
-    for (int i = 0; i < kXStages; ++i) {
-      mbar_init(&ctl->x_full[i], 128);
-      mbar_init(&ctl->x_empty[i], 1);
-    }
+    for (int i = 0; i < kXStages; ++i) mbar_init(&ctl->x_empty[i], 1);
     for (int i = 0; i < kWStages; ++i) {
-      mbar_init(&ctl->w_full[i], kWWarps * 16);   // one weight-producer group
+      mbar_init(&ctl->w_full[i], 4 + 1);   // one weight-producer group (4 warps) + the token TMA thread
       mbar_init(&ctl->w_empty[i], 1);
     }
     for (int i = 0; i < kQStages; ++i) {
       mbar_init(&ctl->q_full[i], 1);
-      mbar_init(&ctl->q_empty[i], kWWarps * 16);
+      mbar_init(&ctl->q_empty[i], 4);
     }
     mbar_init(&ctl->acc_full, 1);
-    mbar_init(&ctl->acc_empty, 256);   // both epilogue groups
+    mbar_init(&ctl->acc_empty, 8);   // one arrival per epilogue warp, both groups
     mbar_init(&ctl->drain, 1);
-    mbar_init(&ctl->epi[0], 128);
-    mbar_init(&ctl->epi[1], 128);
+    mbar_init(&ctl->epi[0], 4);
+    mbar_init(&ctl->epi[1], 4);
     abort_init(&ctl->ab, a.wait_ns);
     fence_barrier_init();
   }
@@ -148,7 +150,10 @@ __global__ void __launch_bounds__(kThreads, 1)
     prefetch_tmap(&tq);
     prefetch_tmap(&ts);
   }
-  if (threadIdx.x == 6 * 32) prefetch_tmap(&th);
+  if (threadIdx.x == 6 * 32) {
+    prefetch_tmap(&th);
+    if (a.nkb_lora > 0) prefetch_tmap(&tha);
+  }
   tc_fence_before();
   __syncthreads();
   tc_fence_after();
@@ -168,7 +173,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     const uint32_t tl = tmem_base + (uint32_t(32 * (warp & 3)) << 16);
     uint8_t* drow = staging + row * kDRow;
     uint8_t* ct = staging + 128 * kDRow + eg * 32 * kTRow;
-    EpiSync es{&ctl->epi[eg]};
+    EpiSyncT<true> es{&ctl->epi[eg]};
     uint32_t bad = 0;   // nonzero once an fp16 output of a valid token overflowed
     int it = 0;
     for (int u = blockIdx.x; u < nunits; u += gridDim.x, ++it) {
@@ -189,7 +194,7 @@ __global__ void __launch_bounds__(kThreads, 1)
                                f32x2_to_f16x2(v[8 * q4 + 6], v[8 * q4 + 7]));
       }
       tc_fence_before();
-      mbar_arrive(&ctl->acc_empty);
+      mbar_arrive_warp(&ctl->acc_empty);
       // this group's 32-token chunks through its [token][feature] tile, 16-byte row stores
       uint16_t* out = static_cast<uint16_t*>(a.out) + un.nt * 128;
       bool stop = false;
@@ -222,29 +227,36 @@ __global__ void __launch_bounds__(kThreads, 1)
       Ring rx, rw;
       int it = 0;
       bool ok = true;
+      // descriptors of ring stage 0; a stage's are these plus a fixed offset
+      const uint64_t xdesc0 = sdesc_k_sw128(smem_u32(x_base));
+      const uint32_t wa0 = tmem_base + kWBase;
       for (int u = blockIdx.x; u < nunits && ok; u += gridDim.x, ++it) {
         const Unit un = us.take(u);
         const int n16 = (un.rows + 15) & ~15;
         const uint32_t idesc = idesc_f16(128, n16);
         if (!mbar_wait(&ctl->acc_empty, (uint32_t(it) & 1u) ^ 1u, abort_flag, a.status)) { ok = false; break; }
         tc_fence_after();
+        uint32_t accf = 0u;   // the unit's first MMA overwrites the accumulator
         for (int kb = 0; kb < nkb; ++kb) {
-          if (!mbar_wait(&ctl->x_full[rx.stage], rx.phase, abort_flag, a.status) ||
-              !mbar_wait(&ctl->w_full[rw.stage], rw.phase, abort_flag, a.status)) {
+          if (!mbar_wait(&ctl->w_full[rw.stage], rw.phase, abort_flag, a.status)) {
             ok = false;
             break;
           }
           tc_fence_after();
-          const uint64_t bdesc = sdesc_k_sw128(smem_u32(x_base + size_t(rx.stage) * kXStageBytes));
-          const uint32_t wa = tmem_base + kWBase + uint32_t(rw.stage) * kWCols;
+          const uint64_t bdesc = xdesc0 + uint64_t(rx.stage) * uint64_t(kXStageBytes >> 4);
+          const uint32_t wa = wa0 + uint32_t(rw.stage) * kWCols;
           if (kb >= a.nkb_lora) {
 #pragma unroll
-            for (int kk = 0; kk < 4; ++kk)
-              umma_f16_ts(tmem_base, wa + uint32_t(8 * kk), bdesc + uint64_t(2 * kk), idesc, (kb > 0 || kk > 0) ? 1u : 0u);
+            for (int kk = 0; kk < 4; ++kk) {
+              umma_f16_ts(tmem_base, wa + uint32_t(8 * kk), bdesc + uint64_t(2 * kk), idesc, accf);
+              accf = 1u;
+            }
           } else {
             const int ksteps = (min(kK, a.lora_k - kb * kK) + 15) / 16;
-            for (int kk = 0; kk < ksteps; ++kk)
-              umma_f16_ts(tmem_base, wa + uint32_t(8 * kk), bdesc + uint64_t(2 * kk), idesc, (kb > 0 || kk > 0) ? 1u : 0u);
+            for (int kk = 0; kk < ksteps; ++kk) {
+              umma_f16_ts(tmem_base, wa + uint32_t(8 * kk), bdesc + uint64_t(2 * kk), idesc, accf);
+              accf = 1u;
+            }
           }
           umma_commit(&ctl->x_empty[rx.stage]);
           umma_commit(&ctl->w_empty[rw.stage]);
@@ -286,58 +298,46 @@ __global__ void __launch_bounds__(kThreads, 1)
       // on an abort, wait (bounded) until every issued fill has landed
       if (aborted(abort_flag)) pend.drain(ctl->q_full);
     }
-  } else if (warp < kWWarp0) {
-    // ------------------------------------------------------------ token producer
-    const int tid = threadIdx.x - 6 * 32;  // 0..127
-    const int chunk = tid & 7;
-    const int row0 = tid >> 3;             // rows row0 + 16 j, j = 0..15
-    Ring rx;
-    PendingFills pend;
-    for (int u = blockIdx.x; u < nunits; u += gridDim.x) {
-      const Unit un = us.take(u);
-      bool ok = true;
-      for (int kb = 0; kb < nkb; ++kb) {
-        if (!mbar_wait<64>(&ctl->x_empty[rx.stage], rx.phase ^ 1u, abort_flag, a.status)) { ok = false; break; }
-        uint8_t* st = x_base + size_t(rx.stage) * kXStageBytes;
-        uint64_t* full = &ctl->x_full[rx.stage];
-        if (kb < a.nkb_lora) {
-          // rank-space rows s H Ad, zero-filled past lora_k
-          const int colk = kb * kK + chunk * 8;
-          const bool in = colk < a.lora_k;
-          const uint32_t st_u = smem_u32(st);
-#pragma unroll 4
-          for (int j = 0; j < kRows / 16; ++j) {
-            const int r = row0 + 16 * j;
-            if (r < un.rows)
-              cp_async16(st_u + sw128_offset(r, chunk), a.a_lora + size_t(un.base + r) * a.lora_ld + (in ? colk : 0),
-                         in ? 16u : 0u);
-          }
-          cp_async_arrive_noinc(full);
-        } else if (tid == 0) {
-          const int km = kb - a.nkb_lora;
-          mbar_arrive_expect_tx(full, uint32_t(kXStageBytes));
-          tma_load_2d(smem_u32(st), &th, full, km * kK, un.base);
-          tma_load_2d(smem_u32(st + kXStageBytes / 2), &th, full, km * kK, un.base + 128);
-          pend.issued(rx.stage, rx.phase);
-        } else {
-          mbar_arrive(full);
+  } else if (warp == 6) {
+    // ------------------------------------------------------------ TMA producer (token rows)
+    if (lane == 0) {
+      Ring rx, rw;
+      PendingFills pend;
+      for (int u = blockIdx.x; u < nunits; u += gridDim.x) {
+        const Unit un = us.take(u);
+        const int nbox = un.rows > 128 ? 2 : 1;   // a second 128-row box only when the MMA reads it
+        bool ok = true;
+        for (int kb = 0; kb < nkb; ++kb) {
+          if (!mbar_wait<64>(&ctl->x_empty[rx.stage], rx.phase ^ 1u, abort_flag, a.status)) { ok = false; break; }
+          uint8_t* st = x_base + size_t(rx.stage) * kXStageBytes;
+          uint64_t* bar = &ctl->w_full[rw.stage];
+          // the adapter stage reads s H Ad (zero-filled past its r columns), the rest H
+          const CUtensorMap* map = kb < a.nkb_lora ? &tha : &th;
+          const int col = (kb < a.nkb_lora ? kb : kb - a.nkb_lora) * kK;
+          mbar_arrive_expect_tx(bar, uint32_t(nbox * (kXStageBytes / 2)));
+          tma_load_2d(smem_u32(st), map, bar, col, un.base);
+          if (nbox == 2) tma_load_2d(smem_u32(st + kXStageBytes / 2), map, bar, col, un.base + 128);
+          pend.issued(rw.stage, rw.phase);
+          rx.next<kXStages>();
+          rw.next<kWStages>();
         }
-        rx.next<kXStages>();
+        if (!ok) break;
       }
-      if (!ok) break;
+      if (aborted(abort_flag)) pend.drain(ctl->w_full);
     }
-    cp_async_wait_all();
-    // on an abort, wait (bounded) until every TMA fill issued here has landed
-    // (a stage's other arrivals may never come; that wait then runs out)
-    if (tid == 0 && aborted(abort_flag)) pend.drain(ctl->x_full);
-  } else {
+  } else if (warp >= kWWarp0) {
     // ------------------------------------------------------------ weight producer
+    // Four groups of 4 warps take stages n % 4, so that four stages are being
+    // dequantised at any time (one stage's chain of code read -> dequant ->
+    // TMEM store -> arrive is latency-bound). A thread converts the 64 K
+    // values of one weight row (TMEM lane lrow) per stage.
     const int wi = warp - kWWarp0;            // 0..15
-    const int grp = wi >> 3;                  // stage parity handled by this group
-    const int kh = (wi >> 2) & 1;             // 32-wide K half of the 64-wide stage
+    const int grp = wi >> 2;                  // stages n with n % 4 == grp
     const int lrow = 32 * (warp & 3) + lane;  // TMEM lane = feature within the tile
-    const uint32_t tw = tmem_base + (uint32_t(32 * (warp & 3)) << 16) + kWBase + uint32_t(kh * 16);
-    const int scale_off = 128 * kCB + (((ngrp == 2) ? kh : 0) * 128 + lrow) * 2;
+    const uint32_t tw = tmem_base + (uint32_t(32 * (warp & 3)) << 16) + kWBase;
+    // scale rows of the two 32-wide K halves of this thread's slice
+    const int g_hi = (ngrp == 1) ? 0 : 32 / a.g;
+    const int s_lo_off = 128 * kCB + lrow * 2, s_hi_off = 128 * kCB + (g_hi * 128 + lrow) * 2;
     bool inexact = false;   // a group scale whose products q * s are not exact in fp16
     bool lora_inf = false;  // a LoRA B value beyond the fp16 range
     int n = 0;   // stage counter
@@ -346,7 +346,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       const Unit un = us.take(u);
       const int feat = un.nt * 128 + lrow;
       bool ok = true;
-      if (a.nkb_lora > 0 && grp == 0 && kh == 0 && u + int(gridDim.x) < nunits) {
+      if (a.nkb_lora > 0 && grp == 0 && u + int(gridDim.x) < nunits) {
         // the next unit's LoRA B row into L2 (its rank-space stage comes first)
         const Unit nx = us.peek();
         const uint16_t* row = a.b0 + (size_t(nx.e) * a.out_dim + nx.nt * 128 + lrow) * a.r;
@@ -356,16 +356,16 @@ __global__ void __launch_bounds__(kThreads, 1)
         const bool main_stage = kb >= a.nkb_lora;
         const int mq = m;
         if (main_stage) ++m;
-        if ((n & 1) != grp) continue;
+        if ((n & 3) != grp) continue;
         const int st = n % kWStages;
         const uint32_t ph = uint32_t(n / kWStages) & 1u;
-        if (!__all_sync(0xFFFFFFFFu, mbar_wait(&ctl->w_empty[st], ph ^ 1u, abort_flag, a.status))) { ok = false; break; }
+        if (!mbar_wait_warp(&ctl->w_empty[st], ph ^ 1u, abort_flag, a.status)) { ok = false; break; }
         tc_fence_after();
-        uint32_t v[16];
+        uint32_t v[32];
         if (!main_stage) {
 #pragma unroll
-          for (int c = 0; c < 4; ++c) {
-            const int colk = kb * kK + kh * 32 + c * 8;
+          for (int c = 0; c < 8; ++c) {
+            const int colk = kb * kK + c * 8;
             uint4 w4 = make_uint4(0, 0, 0, 0);
             if (colk < a.r)
               w4 = bf16x8_to_f16x8_chk(
@@ -375,27 +375,29 @@ __global__ void __launch_bounds__(kThreads, 1)
         } else {
           const int qst = mq % kQStages;
           const uint32_t qph = uint32_t(mq / kQStages) & 1u;
-          if (!__all_sync(0xFFFFFFFFu, mbar_wait(&ctl->q_full[qst], qph, abort_flag, a.status))) { ok = false; break; }
+          if (!mbar_wait_warp(&ctl->q_full[qst], qph, abort_flag, a.status)) { ok = false; break; }
           const uint8_t* qs = q_base + size_t(qst) * kQStageBytes;
-          const uint32_t s2 = scale_pair_chk(*reinterpret_cast<const uint16_t*>(qs + scale_off), inexact);
+          const uint32_t s_lo = scale_pair_chk(*reinterpret_cast<const uint16_t*>(qs + s_lo_off), inexact);
+          const uint32_t s_hi = scale_pair_chk(*reinterpret_cast<const uint16_t*>(qs + s_hi_off), inexact);
           if (BITS == 4) {
-            // this thread's 32 K values: one 16-byte chunk (4 words of 8 codes)
-            const uint4 wd = *reinterpret_cast<const uint4*>(qs + QC::chunk_offset(lrow, kh));
-            const uint4 d0 = dequant_word(wd.x, s2), d1 = dequant_word(wd.y, s2);
-            const uint4 d2 = dequant_word(wd.z, s2), d3 = dequant_word(wd.w, s2);
-            v[0] = d0.x; v[1] = d0.y; v[2] = d0.z; v[3] = d0.w;
-            v[4] = d1.x; v[5] = d1.y; v[6] = d1.z; v[7] = d1.w;
-            v[8] = d2.x; v[9] = d2.y; v[10] = d2.z; v[11] = d2.w;
-            v[12] = d3.x; v[13] = d3.y; v[14] = d3.z; v[15] = d3.w;
-          } else {
-            // two 16-byte chunks (8 words of 4 codes)
+            // 64 K values = 8 words of 8 codes
+            const uint4 wa = *reinterpret_cast<const uint4*>(qs + QC::chunk_offset(lrow, 0));
+            const uint4 wb = *reinterpret_cast<const uint4*>(qs + QC::chunk_offset(lrow, 1));
+            const uint32_t wd[8] = {wa.x, wa.y, wa.z, wa.w, wb.x, wb.y, wb.z, wb.w};
 #pragma unroll
-            for (int ch = 0; ch < 2; ++ch) {
-              const uint4 w4 = *reinterpret_cast<const uint4*>(qs + QC::chunk_offset(lrow, 2 * kh + ch));
+            for (int c = 0; c < 8; ++c) {
+              const uint4 d4 = dequant_word(wd[c], c < 4 ? s_lo : s_hi);
+              v[4 * c] = d4.x; v[4 * c + 1] = d4.y; v[4 * c + 2] = d4.z; v[4 * c + 3] = d4.w;
+            }
+          } else {
+            // 64 K values = 16 words of 4 codes
+#pragma unroll
+            for (int ch = 0; ch < 4; ++ch) {
+              const uint4 w4 = *reinterpret_cast<const uint4*>(qs + QC::chunk_offset(lrow, ch));
               const uint32_t wd[4] = {w4.x, w4.y, w4.z, w4.w};
 #pragma unroll
               for (int i = 0; i < 4; ++i) {
-                const uint2 d2 = dequant_word8(wd[i], s2);
+                const uint2 d2 = dequant_word8(wd[i], ch < 2 ? s_lo : s_hi);
                 v[8 * ch + 2 * i] = d2.x;
                 v[8 * ch + 2 * i + 1] = d2.y;
               }
@@ -404,12 +406,12 @@ __global__ void __launch_bounds__(kThreads, 1)
           // the code slot's values have been consumed; its next fill is an
           // async-proxy TMA write, hence the proxy fence before handing it back
           fence_proxy_async_smem();
-          mbar_arrive(&ctl->q_empty[qst]);
+          mbar_arrive_warp(&ctl->q_empty[qst]);
         }
-        tmem_st16(tw + uint32_t(st) * kWCols, v);
+        tmem_st32(tw + uint32_t(st) * kWCols, v);
         tmem_wait_st();
         tc_fence_before();
-        mbar_arrive(&ctl->w_full[st]);
+        mbar_arrive_warp(&ctl->w_full[st]);
       }
       if (!ok) break;
     }
@@ -433,7 +435,8 @@ static int launch_down(const GemmArgs& a, const Maps& mp, int units_upper, cudaS
   constexpr size_t smem = down_wide::smem_bytes<BITS>();
   if (!attr_done.test_and_set_device(down_wide::down_wide_kernel<BITS>, int(smem))) return TQP_ERR_CUDA;
   const int grid = units_upper < num_sms() ? (units_upper > 0 ? units_upper : 1) : num_sms();
-  down_wide::down_wide_kernel<BITS><<<grid, down_wide::kThreads, smem, s>>>(a, mp.m[TQ0], mp.m[TS0], mp.m[TA]);
+  down_wide::down_wide_kernel<BITS><<<grid, down_wide::kThreads, smem, s>>>(a, mp.m[TQ0], mp.m[TS0], mp.m[TA],
+                                                                             mp.m[TB0]);
   return cudaGetLastError() == cudaSuccess ? TQP_OK : TQP_ERR_CUDA;
 }
 

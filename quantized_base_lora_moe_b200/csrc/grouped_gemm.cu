@@ -747,20 +747,34 @@ __global__ void to_f16_kernel(const uint16_t* __restrict__ x, uint16_t* __restri
 }
 
 // Expert-sorted token rows in fp16, X_perm[i] = x[perm_token[i]], one warp per
-// row; values beyond the fp16 range raise TQP_STATUS_NONFINITE.
+// row, 8 16-byte loads in flight per lane; values beyond the fp16 range raise
+// TQP_STATUS_NONFINITE.
 __global__ void __launch_bounds__(256) gather_rows_f16_kernel(const uint16_t* __restrict__ x,
                                                               const int32_t* __restrict__ perm, int A, int d,
                                                               uint16_t* __restrict__ out, int32_t* status) {
   const int row = blockIdx.x * 8 + (threadIdx.x >> 5);
   if (row >= A) return;
   const int lane = threadIdx.x & 31;
+  const int n16 = d / 8;   // 16-byte pieces per row
   const uint4* src = reinterpret_cast<const uint4*>(x + size_t(__ldg(perm + row)) * d);
   uint4* dst = reinterpret_cast<uint4*>(out + size_t(row) * d);
   uint32_t bad = 0;
-  for (int c = lane; c < d / 8; c += 32) {
-    const uint4 o = bf16x8_to_f16x8(__ldg(src + c));
-    dst[c] = o;
-    bad |= f16x2_nonfinite(o.x) | f16x2_nonfinite(o.y) | f16x2_nonfinite(o.z) | f16x2_nonfinite(o.w);
+  for (int c0 = 0; c0 < n16; c0 += 256) {
+    uint4 v[8];
+#pragma unroll
+    for (int i = 0; i < 8; ++i) {
+      const int c = c0 + 32 * i + lane;
+      v[i] = c < n16 ? __ldg(src + c) : make_uint4(0, 0, 0, 0);
+    }
+#pragma unroll
+    for (int i = 0; i < 8; ++i) {
+      const int c = c0 + 32 * i + lane;
+      if (c < n16) {
+        const uint4 o = bf16x8_to_f16x8(v[i]);
+        dst[c] = o;
+        bad |= f16x2_nonfinite(o.x) | f16x2_nonfinite(o.y) | f16x2_nonfinite(o.z) | f16x2_nonfinite(o.w);
+      }
+    }
   }
   if (__any_sync(0xFFFFFFFFu, bad != 0) && lane == 0) raise_status(status, TQP_STATUS_NONFINITE);
 }
@@ -999,13 +1013,13 @@ int launch_grouped_ffn_part(int part, const uint16_t* x, int T, const int32_t* o
   // expert_down.cu) when the hidden width is a multiple of 128, else on the
   // shared-memory engine.
   const bool tm = (f % 128 == 0);
-  if (part == 1 && tm) {  // H = silu(G) * U: 64 gate + 64 up features x up to 256 rows per unit
+  if (part == 1 && tm) {  // H = silu(G) * U: wide units of up to 256 rows (expert_gateup.cu)
     GemmArgs a = base;
     a.mb_prefix = fb.mb_prefix256;
     a.nkb_main = d / 64;
     a.nkb_lora = r > 0 ? (2 * r + 63) / 64 : 0;
     a.lora_k = 2 * r;
-    a.n_tiles = f / 64;
+    a.n_tiles = f / kGateUpUnitFeatures;
     a.in_dim = d;
     a.out_dim = f;
     a.b0 = w->lora_b[0];
@@ -1111,6 +1125,8 @@ int launch_grouped_ffn_part(int part, const uint16_t* x, int T, const int32_t* o
                        uint64_t(f) * bB / 8, uint32_t(8 * bB), 128, 8 * bB) &&
               make_map(&mp.m[TS0], CU_TENSOR_MAP_DATA_TYPE_UINT16, w->wscale[2], d, uint64_t(w->E) * (f / w->group),
                        uint64_t(d) * 2, 128, ngrp);
+    // the rank-space rows s H Ad: r columns, the rest of each 64-wide box zero-filled
+    if (ok && r > 0) ok = make_tile_map(&mp.m[TB0], fb.ha, uint64_t(A), uint64_t(r), 128);
     if (!ok) return TQP_ERR_CUDA;
     const int units_upper = int((A + 255) / 256 + w->E) * a.n_tiles;
     if ((rc = build_unit_table(a, 256, units_upper, fb.unit_tab, s)) != TQP_OK) return rc;

@@ -85,22 +85,37 @@ __device__ __forceinline__ bool mbar_try_wait(uint32_t addr, uint32_t parity) {
   return ok != 0;
 }
 
+// As mbar_try_wait, with acquire at cluster scope: for barriers that also take
+// arrivals from the other CTA of a pair.
+__device__ __forceinline__ bool mbar_try_wait_cluster(uint32_t addr, uint32_t parity) {
+  uint32_t ok;
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "mbarrier.try_wait.parity.acquire.cluster.shared::cta.b64 p, [%1], %2;\n\t"
+      "selp.u32 %0, 1, 0, p;\n\t}"
+      : "=r"(ok)
+      : "r"(addr), "r"(parity)
+      : "memory");
+  return ok != 0;
+}
+
 // Bounded wait for the phase with the given parity. Returns false (and sets the
 // CTA abort flag and the timeout status bit) when the CTA's wait limit expires
 // or another role has already aborted. kSleep > 0 backs off with nanosleep
 // between polls, for waiters off the critical path (they then leave issue
 // slots to the dequantising warps).
-template <int kSleep = 0>
+template <int kSleep = 0, bool kCluster = false>
 __device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, Abort* ab, int32_t* status) {
   const uint32_t addr = smem_u32(bar);
-  if (mbar_try_wait(addr, parity)) return true;
+  auto try_wait = [&]() { return kCluster ? mbar_try_wait_cluster(addr, parity) : mbar_try_wait(addr, parity); };
+  if (try_wait()) return true;
   const uint64_t t0 = globaltimer();
   const uint64_t limit = ab->limit_ns;
   // the clock is read every 64 polls, or every poll under a short test limit
   const uint32_t every = limit < 1000000ull ? 0u : 63u;
   uint32_t spins = 0;
   while (true) {
-    if (mbar_try_wait(addr, parity)) return true;
+    if (try_wait()) return true;
     if (kSleep > 0) __nanosleep(kSleep);
     if (((++spins) & every) == 0u) {
       if (aborted(ab)) return false;
@@ -111,6 +126,19 @@ __device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, Abort*
       }
     }
   }
+}
+
+// Warp-uniform bounded wait: every lane polls (measured faster than one polling
+// lane with a broadcast), and the result is the same for the whole warp.
+template <int kSleep = 0, bool kCluster = false>
+__device__ __forceinline__ bool mbar_wait_warp(uint64_t* bar, uint32_t parity, Abort* ab, int32_t* status) {
+  return __all_sync(0xFFFFFFFFu, mbar_wait<kSleep, kCluster>(bar, parity, ab, status));
+}
+
+// One arrival for the whole warp, after every lane's preceding accesses.
+__device__ __forceinline__ void mbar_arrive_warp(uint64_t* bar) {
+  __syncwarp();
+  if ((threadIdx.x & 31) == 0) mbar_arrive(bar);
 }
 
 // Drain wait on the abort path: waits for the phase regardless of the abort
@@ -267,6 +295,72 @@ __device__ __forceinline__ void umma_f16_ts(uint32_t d_tmem, uint32_t a_tmem, ui
       "setp.ne.b32 p, %4, 0;\n\t"
       "tcgen05.mma.cta_group::1.kind::f16 [%0], [%1], %2, %3, p;\n\t}" ::"r"(d_tmem),
       "r"(a_tmem), "l"(bdesc), "r"(idesc), "r"(accumulate)
+      : "memory");
+}
+
+// ----------------------------------------------------------------------------
+// CTA pairs (a cluster of two CTAs sharing one tcgen05.mma of M = 256)
+// ----------------------------------------------------------------------------
+
+__device__ __forceinline__ uint32_t cluster_ctarank() {
+  uint32_t r;
+  asm volatile("mov.u32 %0, %%cluster_ctarank;" : "=r"(r));
+  return r;
+}
+
+// Shared::cluster address of this CTA's shared variable at `saddr` in CTA `rank`.
+__device__ __forceinline__ uint32_t mapa_shared(uint32_t saddr, uint32_t rank) {
+  uint32_t r;
+  asm volatile("mapa.shared::cluster.u32 %0, %1, %2;" : "=r"(r) : "r"(saddr), "r"(rank));
+  return r;
+}
+
+// Arrive on a barrier of a CTA of this cluster (release at cluster scope).
+__device__ __forceinline__ void mbar_arrive_cluster(uint32_t cluster_addr) {
+  asm volatile("mbarrier.arrive.release.cluster.shared::cluster.b64 _, [%0];" ::"r"(cluster_addr) : "memory");
+}
+
+// Every thread of both CTAs of the cluster (release / acquire at cluster scope).
+__device__ __forceinline__ void cluster_sync() {
+  asm volatile("barrier.cluster.arrive.release;\n\tbarrier.cluster.wait.acquire;" ::: "memory");
+}
+
+// Tensor memory of a CTA pair: both CTAs' allocating warps (the same warp index)
+// allocate, relinquish and free together.
+__device__ __forceinline__ void tmem_alloc2(uint32_t* dst_smem, uint32_t ncols) {
+  asm volatile("tcgen05.alloc.cta_group::2.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(smem_u32(dst_smem)),
+               "r"(ncols)
+               : "memory");
+}
+
+__device__ __forceinline__ void tmem_relinquish2() {
+  asm volatile("tcgen05.relinquish_alloc_permit.cta_group::2.sync.aligned;" ::: "memory");
+}
+
+__device__ __forceinline__ void tmem_dealloc2(uint32_t taddr, uint32_t ncols) {
+  asm volatile("tcgen05.dealloc.cta_group::2.sync.aligned.b32 %0, %1;" ::"r"(taddr), "r"(ncols) : "memory");
+}
+
+// D[tmem] (+)= A[tmem] * B[smem]^T across a CTA pair (M = 256): issued by one
+// thread of the even CTA; each CTA holds 128 rows of A (TMEM, same address),
+// half of B's N rows (shared memory, same offset) and its 128 x N quarter of D.
+__device__ __forceinline__ void umma2_f16_ts(uint32_t d_tmem, uint32_t a_tmem, uint64_t bdesc, uint32_t idesc,
+                                             uint32_t accumulate) {
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "setp.ne.b32 p, %4, 0;\n\t"
+      "tcgen05.mma.cta_group::2.kind::f16 [%0], [%1], %2, %3, p;\n\t}" ::"r"(d_tmem),
+      "r"(a_tmem), "l"(bdesc), "r"(idesc), "r"(accumulate)
+      : "memory");
+}
+
+// Arrive on the barrier at this offset in both CTAs of the pair once all
+// previously issued pair MMAs of this thread completed.
+__device__ __forceinline__ void umma2_commit_both(uint64_t* bar) {
+  asm volatile(
+      "tcgen05.commit.cta_group::2.mbarrier::arrive::one.shared::cluster.multicast::cluster.b64 [%0], %1;" ::"r"(
+          smem_u32(bar)),
+      "h"(uint16_t(3))
       : "memory");
 }
 
