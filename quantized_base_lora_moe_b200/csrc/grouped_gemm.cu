@@ -26,7 +26,8 @@
 //               rank-space (LoRA) A tiles; TMA B tiles of the rank-space GEMMs
 //   warps 10-17 B producer: int4 -> fp16 dequantisation into 128B-swizzled
 //               tiles (K-major for the forward, MN-major for the dgrads), the
-//               adapter factors of the rank-space stage
+//               adapter factors of the rank-space stage (idle where B comes by
+//               TMA); one arrival per warp
 // Accumulators are double-buffered in TMEM (2 x 256 fp32 columns), so the
 // epilogue of one unit overlaps the main loop of the next. The operand rings
 // (16 KB A tiles, B tiles, 9 KB code stages) share one 216 KB region whose
@@ -162,17 +163,17 @@ __global__ void __launch_bounds__(kThreads, 1)
       mbar_init(&ctl->a_empty[i], 1);
     }
     for (int i = 0; i < kBSt; ++i) {
-      // one producer group's threads (+ the TMA issuer's arrival)
-      mbar_init(&ctl->b_full[i], kBTma ? 257 : 256 / kBGroups);
+      // one arrival per warp of a dequantising group, or the TMA issuer alone
+      mbar_init(&ctl->b_full[i], kBTma ? 1 : 8 / kBGroups);
       mbar_init(&ctl->b_empty[i], 1);
     }
     for (int i = 0; i < kQSt; ++i) {
       mbar_init(&ctl->q_full[i], 1);
-      mbar_init(&ctl->q_empty[i], 256 / kBGroups);
+      mbar_init(&ctl->q_empty[i], 8 / kBGroups);
     }
     for (int i = 0; i < 2; ++i) {
       mbar_init(&ctl->acc_full[i], 1);
-      mbar_init(&ctl->acc_empty[i], 128);
+      mbar_init(&ctl->acc_empty[i], 4);   // one arrival per epilogue warp
     }
     mbar_init(&ctl->drain, 1);
     abort_init(&ctl->ab, a.wait_ns);
@@ -336,7 +337,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         }
       }
       tc_fence_before();
-      mbar_arrive(&ctl->acc_empty[ab]);
+      mbar_arrive_warp(&ctl->acc_empty[ab]);
     }
     if (__any_sync(0xFFFFFFFFu, bad != 0) && lane == 0) raise_status(a.status, TQP_STATUS_NONFINITE);
   } else if (warp == 4) {
@@ -347,12 +348,18 @@ __global__ void __launch_bounds__(kThreads, 1)
       bool ok = true;
       // dgrads: B (the weight tile) is MN-major, features contiguous
       const uint32_t idesc = kBf16 ? idesc_bf16(128, a.ntile) : (kTrans ? idesc_f16_bmn(128, a.ntile) : idesc_f16(128, a.ntile));
+      // descriptors of ring stage 0; a stage's are these plus a fixed offset
+      const uint64_t adesc0 = sdesc_k_sw128(smem_u32(a_base));
+      const uint64_t bdesc0 = kTrans ? sdesc_mn_sw128(smem_u32(b_base), kMnAtomBytes) : sdesc_k_sw128(smem_u32(b_base));
+      // a K step of 16 advances a K-major tile by 32 B and an MN-major one by two 1024-byte atoms
+      constexpr uint64_t kBStep = kTrans ? uint64_t(2048 >> 4) : uint64_t(2);
       for (int u = blockIdx.x; u < nunits && ok; u += gridDim.x, ++it) {
         const int ab = it & 1;
         const uint32_t aph = uint32_t(it >> 1) & 1u;
         if (!mbar_wait(&ctl->acc_empty[ab], aph ^ 1u, abort_flag, a.status)) { ok = false; break; }
         tc_fence_after();
         const uint32_t dt = tmem_base + uint32_t(ab * 256);
+        uint32_t accf = 0u;   // the unit's first MMA overwrites the accumulator
         for (int kb = 0; kb < nkb; ++kb) {
           if (!mbar_wait(&ctl->a_full[ra.stage], ra.phase, abort_flag, a.status) ||
               !mbar_wait(&ctl->b_full[rb.stage], rb.phase, abort_flag, a.status)) {
@@ -363,14 +370,21 @@ __global__ void __launch_bounds__(kThreads, 1)
           // threads fence their own generic stores before arriving, and cp.async
           // completion is tracked by the barrier itself
           tc_fence_after();
-          const int ksteps = (kb < a.nkb_lora) ? (min(64, a.lora_k - kb * 64) + 15) / 16 : 4;
-          const uint64_t adesc = sdesc_k_sw128(smem_u32(a_base + size_t(ra.stage) * kAStageBytes));
-          const uint32_t bs = smem_u32(b_base + size_t(rb.stage) * kBStride);
-          const uint64_t bdesc = kTrans ? sdesc_mn_sw128(bs, kMnAtomBytes) : sdesc_k_sw128(bs);
-          // a K step of 16 advances a K-major tile by 32 B and an MN-major one by two 1024-byte atoms
-          const uint64_t bstep = kTrans ? uint64_t(2048 >> 4) : uint64_t(2);
-          for (int kk = 0; kk < ksteps; ++kk)
-            umma_bf16(dt, adesc + uint64_t(2 * kk), bdesc + bstep * uint64_t(kk), idesc, (kb > 0 || kk > 0) ? 1u : 0u);
+          const uint64_t adesc = adesc0 + uint64_t(ra.stage) * uint64_t(kAStageBytes >> 4);
+          const uint64_t bdesc = bdesc0 + uint64_t(rb.stage) * uint64_t(kBStride >> 4);
+          if (kb >= a.nkb_lora) {
+#pragma unroll
+            for (int kk = 0; kk < 4; ++kk) {
+              umma_bf16(dt, adesc + uint64_t(2 * kk), bdesc + kBStep * uint64_t(kk), idesc, accf);
+              accf = 1u;
+            }
+          } else {
+            const int ksteps = (min(64, a.lora_k - kb * 64) + 15) / 16;
+            for (int kk = 0; kk < ksteps; ++kk) {
+              umma_bf16(dt, adesc + uint64_t(2 * kk), bdesc + kBStep * uint64_t(kk), idesc, accf);
+              accf = 1u;
+            }
+          }
           umma_commit(&ctl->a_empty[ra.stage]);
           umma_commit(&ctl->b_empty[rb.stage]);
           ra.next<kASt>();
@@ -518,8 +532,10 @@ __global__ void __launch_bounds__(kThreads, 1)
       pend_a.drain(ctl->a_full);
       pend_b.drain(ctl->b_full);
     }
-  } else {
+  } else if (!kBTma) {
     // ------------------------------------------------------------ B producer
+    // (the modes whose B tile arrives by TMA have none: the A producer's TMA
+    // issuer is the B stage's only arrival)
     const int tid = threadIdx.x - 10 * 32;  // 0..255
     const int tpr = a.ntile >= 256 ? 1 : 256 / a.ntile;   // threads per B row (forward tiles)
     const int brow = tid / tpr;                              // B row (forward tiles)
@@ -542,9 +558,7 @@ __global__ void __launch_bounds__(kThreads, 1)
           rb.next<kBSt>();
           continue;
         }
-        const bool waited = kBTma ? mbar_wait<256>(&ctl->b_empty[rb.stage], rb.phase ^ 1u, abort_flag, a.status)
-                                  : mbar_wait(&ctl->b_empty[rb.stage], rb.phase ^ 1u, abort_flag, a.status);
-        if (!waited) { ok = false; break; }
+        if (!mbar_wait_warp(&ctl->b_empty[rb.stage], rb.phase ^ 1u, abort_flag, a.status)) { ok = false; break; }
         uint8_t* bst = b_base + size_t(rb.stage) * kBStride;
         uint64_t* full = &ctl->b_full[rb.stage];
         if (kb < a.nkb_lora) {
@@ -585,9 +599,9 @@ __global__ void __launch_bounds__(kThreads, 1)
             }
           }
           fence_proxy_async_smem();
-          mbar_arrive(full);
+          mbar_arrive_warp(full);
         } else if (kTrans) {
-          if (!mbar_wait(&ctl->q_full[q.stage], q.phase, abort_flag, a.status)) { ok = false; break; }
+          if (!mbar_wait_warp(&ctl->q_full[q.stage], q.phase, abort_flag, a.status)) { ok = false; break; }
           const uint8_t* qs = q_base + size_t(q.stage) * kQStageBytes;
           // The code tile holds W rows n (the K index) with the tile's ntile
           // features contiguous: exactly the MN-major operand, so each thread
@@ -627,11 +641,11 @@ __global__ void __launch_bounds__(kThreads, 1)
           // hand the code slot back only after its values were consumed, behind a
           // proxy fence (its next TMA fill and the tensor-core reads are async-proxy)
           fence_proxy_async_smem();
-          mbar_arrive(&ctl->q_empty[q.stage]);
+          mbar_arrive_warp(&ctl->q_empty[q.stage]);
           q.next<kQSt>();
-          mbar_arrive(full);
+          mbar_arrive_warp(full);
         } else if (kDequant) {
-          if (!mbar_wait(&ctl->q_full[q.stage], q.phase, abort_flag, a.status)) { ok = false; break; }
+          if (!mbar_wait_warp(&ctl->q_full[q.stage], q.phase, abort_flag, a.status)) { ok = false; break; }
           const uint8_t* qs = q_base + size_t(q.stage) * kQStageBytes;
           const uint16_t* sc = reinterpret_cast<const uint16_t*>(qs + a.ntile * 32);
           const int half = a.ntile >> 1;
@@ -644,11 +658,9 @@ __global__ void __launch_bounds__(kThreads, 1)
           if (nwords == 8) dequant_row<8>(qs, bst, brow, part, s_lo, s_hi);
           else dequant_row<4>(qs, bst, brow, part, s_lo, s_hi);
           fence_proxy_async_smem();
-          mbar_arrive(&ctl->q_empty[q.stage]);
+          mbar_arrive_warp(&ctl->q_empty[q.stage]);
           q.next<kQSt>();
-          mbar_arrive(full);
-        } else {
-          mbar_arrive(full);  // the B tile arrives by TMA (LORA_XA, LORA_HA, ROUTER)
+          mbar_arrive_warp(full);
         }
         rb.next<kBSt>();
       }
