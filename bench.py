@@ -101,7 +101,7 @@ def measured_traffic(kernel: str) -> int | None:
     """DRAM bytes per launch of `kernel` from the committed ncu capture, if the
     expert-kernel sources are still the ones that were captured; else None."""
     import hashlib
-    path = os.path.join(ROOT, "profiles", "expert_ffn_traffic_full.json")
+    path = os.path.join(ROOT, "profiles", "expert_traffic_full.json")
     if not os.path.exists(path):
         return None
     doc = json.load(open(path))
@@ -574,11 +574,11 @@ def run_tqp(args, rank: int, world: int, local_rank: int) -> dict | None:
         "assignments_per_s": world * A / (ms * 1e-3),
         "per_call_ms": dict(per_call_ms, grouped_ffn=ffn_ms),
         "roofline": {"bound": "tensor",
-                     "kernel": "gateup_kernel (int4 -> fp16 weights in TMEM, tcgen05 gate/up + SwiGLU)",
+                     "kernel": "gateup_wide_kernel (int4 -> fp16 weights in TMEM, 64 gate + 64 up features x up to 256 rows per unit, tcgen05 + SwiGLU)",
                      "achieved": gu_tflops, "peak": pk["bf16_tflops"], "unit": "TFLOP/s",
                      "frac": gu_tflops / pk["bf16_tflops"],
-                     "traffic": measured_traffic("gateup_kernel") if args.config == "full" else None,
-                     "traffic_source": "profiles/expert_ffn_traffic_full.md (ncu dram__bytes_read+write, one launch)",
+                     "traffic": measured_traffic("gateup_wide_kernel") if args.config == "full" else None,
+                     "traffic_source": "profiles/expert_traffic_full.md (ncu dram__bytes_read+write, one launch)",
                      "peak_source": f"{pk['source']} bf16 dense burst (fp16 has the same nominal rate)",
                      "flop_per_launch": fl["gate_up"], "ms_per_launch": gu_ms},
         "layer_roofline": layer_roofline(cfg, lb.touched_experts(), ms),
