@@ -15,7 +15,7 @@ CSRC = os.path.join(HERE, "csrc")
 ROOT = os.path.dirname(HERE)
 LIB = os.path.join(HERE, "libtqpmoe.so")
 SOURCES = ["tqp_api.cu", "route_permute_combine.cu", "grouped_gemm.cu", "expert_gateup.cu", "expert_down.cu", "layer_bwd.cu",
-           "permute_noalloc.cu", "optim.cu", "wgrad.cu"]
+           "permute_noalloc.cu", "optim.cu", "wgrad.cu", "expert_dgrad.cu"]
 ARCH = ["-gencode", "arch=compute_100a,code=sm_100a"]
 
 

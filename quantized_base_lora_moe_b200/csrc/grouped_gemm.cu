@@ -1222,7 +1222,7 @@ int launch_rank_bwd(int which, const uint16_t* P, const int32_t* offsets, const 
 
 int launch_dgrad(int which, const uint16_t* a_src, const uint16_t* a_lora, const int32_t* offsets,
                  const int32_t* mb_prefix, const tqp_moe_weights* w, int T, const uint16_t* aux_gu, uint16_t* out,
-                 int32_t* status, cudaStream_t s) {
+                 int32_t* status, cudaStream_t s, const int32_t* mb_prefix256, int4* unit_tab) {
   if (T == 0) return TQP_OK;
   const size_t A = size_t(T) * w->top_k;
   const int d = w->d, f = w->ffn, r = w->rank;
@@ -1265,7 +1265,44 @@ int launch_dgrad(int which, const uint16_t* a_src, const uint16_t* a_lora, const
     if (!ok) return TQP_ERR_CUDA;
     return run_gemm<DH>(a, mp, mb_upper * a.n_tiles, s);
   }
-  // DX: K = 2f (gate rows then up rows of W), N = d
+  if (mb_prefix256 && unit_tab && d % 128 == 0) {
+    // DX with W^T in tensor memory (expert_dgrad.cu): units of 128 input features x
+    // up to 256 rows; K = 2r rank-space columns, then the f gate and f up rows of W
+    a.mb_prefix = mb_prefix256;
+    a.nkb_main = 2 * f / 64;
+    a.half_kb = f / 64;
+    a.nkb_lora = r > 0 ? (2 * r + 63) / 64 : 0;
+    a.lora_k = 2 * r;
+    a.n_tiles = d / 128;
+    a.in_dim = d;
+    a.out_dim = f;
+    a.lb0 = w->lora_a[0];
+    a.lb1 = w->lora_a[1];
+    a.lb_ld = d;
+    a.out_ld = d;
+    a.n_valid = d;
+    const uint32_t cbox = uint32_t(128 * bB / 8);   // one tile's 128 features of a code row
+    const uint32_t srows = uint32_t(w->group >= 128 ? 1 : 128 / w->group);
+    const uint64_t crow = uint64_t(d) * bB / 8;
+    bool ok = make_map(&mp.m[TQ0], CU_TENSOR_MAP_DATA_TYPE_UINT8, w->wq[0], crow, uint64_t(w->E) * f, crow, cbox, 64,
+                       int(cbox)) &&
+              make_map(&mp.m[TQ1], CU_TENSOR_MAP_DATA_TYPE_UINT8, w->wq[1], crow, uint64_t(w->E) * f, crow, cbox, 64,
+                       int(cbox)) &&
+              make_map(&mp.m[TS0], CU_TENSOR_MAP_DATA_TYPE_UINT16, w->wscale[0], f, uint64_t(w->E) * (d / w->group),
+                       uint64_t(f) * 2, 64, srows) &&
+              make_map(&mp.m[TS1], CU_TENSOR_MAP_DATA_TYPE_UINT16, w->wscale[1], f, uint64_t(w->E) * (d / w->group),
+                       uint64_t(f) * 2, 64, srows) &&
+              make_tile_map(&mp.m[TA], a_src, uint64_t(A), uint64_t(2 * f), 128);
+    if (ok && r > 0) ok = make_tile_map(&mp.m[TB0], a_lora, uint64_t(A), uint64_t(2 * r), 128);
+    if (!ok) return TQP_ERR_CUDA;
+    const int units_upper = int((A + 255) / 256 + w->E) * a.n_tiles;
+    int rc = build_unit_table(a, 256, units_upper, unit_tab, s);
+    if (rc != TQP_OK) return rc;
+    a.unit_tab = unit_tab;
+    a.wait_ns = wait_limit_ns();
+    return run_expert_dx(a, mp, units_upper, s);
+  }
+  // DX on the shared-memory engine: K = 2f (gate rows then up rows of W), N = d
   a.ntile = (d % 256 == 0 && bB == 4) ? 256 : 128;
   const int ngn = w->group >= a.ntile ? 1 : a.ntile / w->group;
   a.nkb_main = 2 * f / 64;

@@ -204,7 +204,9 @@ int layer_backward(const uint16_t* x, const float* dy, int T, const tqp_moe_weig
       return rc;
   }
   uint16_t* dX = B.dO;  // dO is no longer needed
-  if ((rc = launch_dgrad(1, B.dgu, B.dxa, L.offsets, fb.mb_prefix, w, T, nullptr, dX, status, s)) != TQP_OK) return rc;
+  if ((rc = launch_dgrad(1, B.dgu, B.dxa, L.offsets, fb.mb_prefix, w, T, nullptr, dX, status, s, fb.mb_prefix256,
+                         fb.unit_tab)) != TQP_OK)
+    return rc;
   return launch_gather_add(dX, L.inv, T, k, d, B.dmax, dx, s);
 }
 

@@ -71,9 +71,12 @@ int launch_grouped_ffn(const uint16_t* x, int T, const int32_t* offsets, const i
 int launch_grouped_ffn_part(int part, const uint16_t* x, int T, const int32_t* offsets, const int32_t* perm_token,
                             const tqp_moe_weights* w, uint16_t* h, uint16_t* out_perm, void* ws, int32_t* status,
                             cudaStream_t s, uint16_t* aux_gu = nullptr);
+// dgrads: which 0 dH (+ SwiGLU backward into dG|dU), 1 dX. mb_prefix256 and
+// unit_tab (the FFN workspace's 256-row schedule and unit table) select the
+// tensor-memory dX kernel; null keeps the shared-memory engine.
 int launch_dgrad(int which, const uint16_t* a_src, const uint16_t* a_lora, const int32_t* offsets,
                  const int32_t* mb_prefix, const tqp_moe_weights* w, int T, const uint16_t* aux_gu, uint16_t* out,
-                 int32_t* status, cudaStream_t s);
+                 int32_t* status, cudaStream_t s, const int32_t* mb_prefix256 = nullptr, int4* unit_tab = nullptr);
 // rank-space products of the backward on the tensor cores (grouped_gemm.cu):
 //   which 0: dha = s dO Bd      (P = dO [A][d]      -> C [A][r])
 //   which 1: dxa = s [dG|dU] blockdiag(Bg, Bu)   (P = dgu [A][2f] -> C [A][2r])
