@@ -1,40 +1,44 @@
-// Input gradient of the gate/up projection of the TQP MoE experts with the
-// dequantised base weights in tensor memory (sm_100a, tcgen05):
-//   dX = dG Wg + dU Wu + dxa [Ag ; Au]^T      (per expert, expert-sorted rows)
+// Input gradients of the TQP MoE expert projections with the dequantised base
+// weights in tensor memory (sm_100a, tcgen05), per expert over expert-sorted rows:
+//   dX : dX = dG Wg + dU Wu + dxa [Ag ; Au]^T
+//   dH : dH = dO Wd + dha Ad^T, then the SwiGLU backward
+//        dG = dH U silu'(G), dU = dH silu(G) (G, U kept by the forward)
 // (the base weights are frozen and only the adapters train, but the input
-// gradient still flows through W + s A B: "Reversible Sparse MoE Single Node",
-// Principle 3 and Pattern 3; the rank-space row products dxa = s [dG|dU]
-// blockdiag(Bg, Bu) come from the engine's rank-space mode).
+// gradients still flow through W + s A B: "Reversible Sparse MoE Single Node",
+// Principle 3 and Pattern 3; the rank-space row products dxa, dha come from
+// the engine's rank-space mode).
 //
-// The contraction runs transposed, D[m][row] = W^T[m][:] . dGU[row][:], as in
-// the forward expert kernels: one unit is (expert e, 128 input features m of one
+// The contraction runs transposed, D[m][row] = W^T[m][:] . P[row][:], as in the
+// forward expert kernels: one unit is (expert e, 128 output features m of one
 // tile, block of up to 256 routed rows). A = W^T (M = 128 TMEM lanes = features
-// m, K = the hidden index n) is dequantised into TMEM; B = the [dG | dU] rows
-// (N = rows, K-major) come by TMA from the expert-sorted gradient buffer; the
-// K loop runs over the rank-space stage, then the f gate rows of W, then the f
-// up rows. Each weight tile is dequantised once per 256-row block.
+// m, K = the contraction index n) is dequantised into TMEM; B = the rows P
+// ([dG | dU] for dX, dO for dH; N = rows, K-major) come by TMA from the
+// expert-sorted buffers; the K loop runs over the rank-space stage, then the
+// weight rows (for dX the f gate rows, then the f up rows). Each weight tile is
+// dequantised once per 256-row block.
 //
-// W is stored with n as its row ([E][f][d] codes): a lane (one m) needs one code
-// from each of 64 code rows per stage. Eight lanes load one 32-bit word each
-// (8 int4 codes of 8 consecutive m, from 8 different rows) and transpose the
-// 8 x 8 nibble block with three shuffle stages, so that each lane holds the 8
-// codes of its m along n. The rows are loaded in the order 0,2,4,6,1,3,5,7, which
-// leaves the codes in the storage order of an int4 word (even positions in the
-// low half-word), so the exact fp16 dequantisation of the forward kernels
-// applies with one scale pair per pair of positions (the group scale varies
-// along n here: scale[m / g][n]). The lanes then hold the word's features in
-// its storage order, so TMEM lane L carries feature lane_feature(L) and the
-// epilogue writes each lane's output column there. int8 codes use a 4 x 4
-// byte transpose and keep lane = feature.
-// One warp converts each stage's bf16 scale tile to fp16 in place first.
+// W is stored with n as its row (the codes of the contraction index are rows):
+// a lane (one m) needs one code from each of 64 code rows per stage. Eight lanes
+// load one 32-bit word each (8 int4 codes of 8 consecutive m, from 8 different
+// rows) and transpose the 8 x 8 nibble block with three shuffle stages, so that
+// each lane holds the 8 codes of its m along n. The rows are loaded in the order
+// 0,2,4,6,1,3,5,7, which leaves the codes in the storage order of an int4 word
+// (even positions in the low half-word), so the exact fp16 dequantisation of
+// the forward kernels applies with one scale pair per pair of positions (the
+// group scale varies along n here: scale[m / g][n]). The lanes then hold the
+// word's features in its storage order, so TMEM lane L carries feature
+// lane_feature(L) and the epilogue writes each lane's output column there. int8
+// codes use a 4 x 4 byte transpose and keep lane = feature. One warp converts
+// each stage's bf16 scale tile to fp16 in place first.
 //
 // Per CTA (1 per SM, 896 threads):
 //   warps 0-3, 24-27  epilogue (two groups on alternate 32-row chunks): the
-//               down kernel's transposing 16-byte row stores of dX
+//               down kernel's transposing 16-byte row stores (dX), or the
+//               SwiGLU backward on the [row][feature] chunk tile (dH)
 //   warp  4     TMEM allocation + one thread issuing tcgen05.mma
 //   warp  5     TMA producer of the code / scale ring
-//   warp  6     TMA producer of the row ring ([dG | dU] rows; dxa rows for the
-//               rank-space stage, zero-filled past 2r)
+//   warp  6     TMA producer of the row ring (P rows; the rank-space rows for
+//               the rank-space stage, zero-filled past their width)
 //   warp  7     scale converter (bf16 -> fp16 in place; range status)
 //   warps 8-23  weight producer, four groups of 4 warps on stages n % 4
 // TMEM: one 256-column accumulator and 8 weight stages of 32 columns. Every
@@ -141,9 +145,10 @@ __device__ __forceinline__ void stage_tokens_pair(uint8_t* tile, int feat, const
   }
 }
 
-template <int BITS>
+// MODE: DX or DH (gemm_common.cuh).
+template <int MODE, int BITS>
 __global__ void __launch_bounds__(kThreads, 1)
-    dx_kernel(const GemmArgs a, const __grid_constant__ CUtensorMap tq0, const __grid_constant__ CUtensorMap tq1,
+    dgrad_kernel(const GemmArgs a, const __grid_constant__ CUtensorMap tq0, const __grid_constant__ CUtensorMap tq1,
               const __grid_constant__ CUtensorMap ts0, const __grid_constant__ CUtensorMap ts1,
               const __grid_constant__ CUtensorMap tx, const __grid_constant__ CUtensorMap txa) {
   using QC = QCfg<BITS>;
@@ -188,9 +193,11 @@ __global__ void __launch_bounds__(kThreads, 1)
   }
   if (threadIdx.x == 5 * 32) {
     prefetch_tmap(&tq0);
-    prefetch_tmap(&tq1);
     prefetch_tmap(&ts0);
-    prefetch_tmap(&ts1);
+    if (MODE == DX) {
+      prefetch_tmap(&tq1);
+      prefetch_tmap(&ts1);
+    }
   }
   if (threadIdx.x == 6 * 32) {
     prefetch_tmap(&tx);
@@ -254,8 +261,34 @@ __global__ void __launch_bounds__(kThreads, 1)
         for (int p = etid; p < nt * 16; p += 128) {
           const int t = p >> 4, fg = p & 15;
           const uint4 v = *reinterpret_cast<const uint4*>(ct + t * kTRow + fg * 16);
-          bad |= f16x2_nonfinite(v.x) | f16x2_nonfinite(v.y) | f16x2_nonfinite(v.z) | f16x2_nonfinite(v.w);
-          *reinterpret_cast<uint4*>(out + size_t(un.base + c + t) * a.out_ld + fg * 8) = v;
+          const size_t orow = size_t(un.base + c + t) * a.out_ld;
+          if (MODE == DX) {
+            bad |= f16x2_nonfinite(v.x) | f16x2_nonfinite(v.y) | f16x2_nonfinite(v.z) | f16x2_nonfinite(v.w);
+            *reinterpret_cast<uint4*>(out + orow + fg * 8) = v;
+          } else {
+            // SwiGLU backward of 8 features: dG = dH U s (1 + G (1 - s)), dU = dH G s, s = sigmoid(G)
+            const uint16_t* gu = a.aux + orow + un.nt * 128 + fg * 8;
+            const uint4 g4 = *reinterpret_cast<const uint4*>(gu);
+            const uint4 u4 = *reinterpret_cast<const uint4*>(gu + a.f_dim);
+            const uint32_t hw[4] = {v.x, v.y, v.z, v.w};
+            const uint32_t gw[4] = {g4.x, g4.y, g4.z, g4.w};
+            const uint32_t uw[4] = {u4.x, u4.y, u4.z, u4.w};
+            uint32_t dg[4], du[4];
+#pragma unroll
+            for (int q = 0; q < 4; ++q) {
+              const float2 dh = __half22float2(*reinterpret_cast<const __half2*>(&hw[q]));
+              const float2 g = __half22float2(*reinterpret_cast<const __half2*>(&gw[q]));
+              const float2 uu = __half22float2(*reinterpret_cast<const __half2*>(&uw[q]));
+              const float s0 = 1.0f / (1.0f + __expf(-g.x)), s1 = 1.0f / (1.0f + __expf(-g.y));
+              dg[q] = f32x2_to_f16x2(dh.x * uu.x * s0 * (1.0f + g.x * (1.0f - s0)),
+                                     dh.y * uu.y * s1 * (1.0f + g.y * (1.0f - s1)));
+              du[q] = f32x2_to_f16x2(dh.x * g.x * s0, dh.y * g.y * s1);
+              bad |= f16x2_nonfinite(dg[q]) | f16x2_nonfinite(du[q]);
+            }
+            uint16_t* dgu = static_cast<uint16_t*>(a.out) + orow + un.nt * 128 + fg * 8;
+            *reinterpret_cast<uint4*>(dgu) = make_uint4(dg[0], dg[1], dg[2], dg[3]);
+            *reinterpret_cast<uint4*>(dgu + a.f_dim) = make_uint4(du[0], du[1], du[2], du[3]);
+          }
         }
       }
       if (stop) break;
@@ -416,8 +449,9 @@ __global__ void __launch_bounds__(kThreads, 1)
         if (!main_stage) {
           // rank-space stage: A[m][j] = Ag^T[j][m] (j < r), Au^T[j - r][m] (r <= j < 2r), else 0,
           // written to TMEM in two halves of 16 columns (32 K values each)
+          // dX: Ag^T then Au^T (lora_k = 2r); dH: Ad^T (lora_k = r)
           const uint16_t* pg = a.lb0 + size_t(un.e) * a.r * a.lb_ld + feat;
-          const uint16_t* pu = a.lb1 + size_t(un.e) * a.r * a.lb_ld + feat;
+          const uint16_t* pu = MODE == DX ? a.lb1 + size_t(un.e) * a.r * a.lb_ld + feat : pg;
 #pragma unroll 1
           for (int hv = 0; hv < 2; ++hv) {
             uint32_t w16[16];
@@ -429,7 +463,7 @@ __global__ void __launch_bounds__(kThreads, 1)
                 const int j = kb * kK + 32 * hv + 2 * c + h;
                 uint32_t bits = 0;
                 if (j < a.r) bits = __ldg(pg + size_t(j) * a.lb_ld);
-                else if (j < 2 * a.r) bits = __ldg(pu + size_t(j - a.r) * a.lb_ld);
+                else if (j < a.lora_k) bits = __ldg(pu + size_t(j - a.r) * a.lb_ld);
                 pr |= bf16_to_f16_bits_chk(bits, lora_inf) << (16 * h);
               }
               w16[c] = pr;
@@ -502,19 +536,20 @@ __global__ void __launch_bounds__(kThreads, 1)
 
 }  // namespace dgrad_tm
 
-template <int BITS>
-static int launch_dx_tm(const GemmArgs& a, const Maps& mp, int units_upper, cudaStream_t s) {
+template <int MODE, int BITS>
+static int launch_dgrad_tm(const GemmArgs& a, const Maps& mp, int units_upper, cudaStream_t s) {
   static DeviceFlags attr_done;
   constexpr size_t smem = dgrad_tm::smem_bytes<BITS>();
-  if (!attr_done.test_and_set_device(dgrad_tm::dx_kernel<BITS>, int(smem))) return TQP_ERR_CUDA;
+  auto kern = dgrad_tm::dgrad_kernel<MODE, BITS>;
+  if (!attr_done.test_and_set_device(kern, int(smem))) return TQP_ERR_CUDA;
   const int grid = units_upper < num_sms() ? (units_upper > 0 ? units_upper : 1) : num_sms();
-  dgrad_tm::dx_kernel<BITS><<<grid, dgrad_tm::kThreads, smem, s>>>(a, mp.m[TQ0], mp.m[TQ1], mp.m[TS0], mp.m[TS1],
-                                                                     mp.m[TA], mp.m[TB0]);
+  kern<<<grid, dgrad_tm::kThreads, smem, s>>>(a, mp.m[TQ0], mp.m[TQ1], mp.m[TS0], mp.m[TS1], mp.m[TA], mp.m[TB0]);
   return cudaGetLastError() == cudaSuccess ? TQP_OK : TQP_ERR_CUDA;
 }
 
-int run_expert_dx(const GemmArgs& a, const Maps& mp, int units_upper, cudaStream_t s) {
-  return a.bits == 8 ? launch_dx_tm<8>(a, mp, units_upper, s) : launch_dx_tm<4>(a, mp, units_upper, s);
+int run_expert_dgrad(int mode, const GemmArgs& a, const Maps& mp, int units_upper, cudaStream_t s) {
+  if (mode == DX) return a.bits == 8 ? launch_dgrad_tm<DX, 8>(a, mp, units_upper, s) : launch_dgrad_tm<DX, 4>(a, mp, units_upper, s);
+  return a.bits == 8 ? launch_dgrad_tm<DH, 8>(a, mp, units_upper, s) : launch_dgrad_tm<DH, 4>(a, mp, units_upper, s);
 }
 
 }  // namespace tqp

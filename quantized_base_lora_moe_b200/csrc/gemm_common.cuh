@@ -212,9 +212,10 @@ enum { TQ0 = 0, TQ1 = 1, TS0 = 2, TS1 = 3, TA = 4, TB0 = 5, TB1 = 6 };
 // (expert_gateup.cu): TA = X_perm [A][d], TB0 = s X [Ag|Au] [A][2r] (box {64, 128}
 // each); a.bits selects int4 or int8 codes.
 int run_expert_gateup_wide(const GemmArgs& a, const Maps& mp, int units_upper, cudaStream_t s);
-// Input gradient of gate/up, dX = [dG|dU][Wg;Wu] + dxa [Ag;Au]^T, with W^T in TMEM
-// (expert_dgrad.cu): TA = [dG|dU] rows [A][2f], TB0 = dxa [A][2r] (box {64, 128}).
-int run_expert_dx(const GemmArgs& a, const Maps& mp, int units_upper, cudaStream_t s);
+// Input gradients with W^T in TMEM (expert_dgrad.cu), mode DX: dX = [dG|dU][Wg;Wu]
+// + dxa [Ag;Au]^T (TA = [dG|dU] rows [A][2f], TB0 = dxa [A][2r]); mode DH: dH = dO Wd
+// + dha Ad^T and the SwiGLU backward into [dG|dU] (TA = dO [A][d], TB0 = dha [A][r]).
+int run_expert_dgrad(int mode, const GemmArgs& a, const Maps& mp, int units_upper, cudaStream_t s);
 // The wide gate/up kernel runs on CTA pairs (cta_group::2, M = 256 per MMA): a
 // unit then covers 128 features of gate and of up (64 per CTA), else 64.
 constexpr bool kGateUpPair = false;

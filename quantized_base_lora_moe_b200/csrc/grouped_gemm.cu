@@ -1242,7 +1242,43 @@ int launch_dgrad(int which, const uint16_t* a_src, const uint16_t* a_lora, const
   a.bits = w->bits == 8 ? 8 : 4;
   const int bB = a.bits;   // code bits: a tile row of ntile features is ntile * bits / 8 bytes
   Maps mp{};
-  if (which == 0) {  // DH: K = d (rows of Wd), N = f
+  if (which == 0 && mb_prefix256 && unit_tab && f % 128 == 0) {
+    // dH with Wd^T in tensor memory (expert_dgrad.cu): units of 128 hidden features
+    // x up to 256 rows; K = r rank-space columns, then the d rows of Wd; the
+    // SwiGLU backward writes [dG | dU]
+    a.mb_prefix = mb_prefix256;
+    a.nkb_main = d / 64;
+    a.half_kb = d / 64;   // one weight matrix
+    a.nkb_lora = r > 0 ? (r + 63) / 64 : 0;
+    a.lora_k = r;
+    a.n_tiles = f / 128;
+    a.in_dim = f;
+    a.out_dim = d;
+    a.lb0 = w->lora_a[2];
+    a.lb_ld = f;
+    a.aux = const_cast<uint16_t*>(aux_gu);
+    a.out_ld = 2 * f;
+    a.n_valid = f;
+    const uint32_t cbox = uint32_t(128 * bB / 8);   // one tile's 128 features of a code row
+    const uint32_t srows = uint32_t(w->group >= 128 ? 1 : 128 / w->group);
+    const uint64_t crow = uint64_t(f) * bB / 8;
+    bool ok = make_map(&mp.m[TQ0], CU_TENSOR_MAP_DATA_TYPE_UINT8, w->wq[2], crow, uint64_t(w->E) * d, crow, cbox, 64,
+                       int(cbox)) &&
+              make_map(&mp.m[TS0], CU_TENSOR_MAP_DATA_TYPE_UINT16, w->wscale[2], d, uint64_t(w->E) * (f / w->group),
+                       uint64_t(d) * 2, 64, srows) &&
+              make_tile_map(&mp.m[TA], a_src, uint64_t(A), uint64_t(d), 128);
+    if (ok && r > 0) ok = make_tile_map(&mp.m[TB0], a_lora, uint64_t(A), uint64_t(r), 128);
+    if (!ok) return TQP_ERR_CUDA;
+    mp.m[TQ1] = mp.m[TQ0];   // one weight matrix: the second map slot repeats the first
+    mp.m[TS1] = mp.m[TS0];
+    const int units_upper = int((A + 255) / 256 + w->E) * a.n_tiles;
+    int rc = build_unit_table(a, 256, units_upper, unit_tab, s);
+    if (rc != TQP_OK) return rc;
+    a.unit_tab = unit_tab;
+    a.wait_ns = wait_limit_ns();
+    return run_expert_dgrad(DH, a, mp, units_upper, s);
+  }
+  if (which == 0) {  // DH on the shared-memory engine: K = d (rows of Wd), N = f
     a.ntile = (f % 256 == 0 && bB == 4) ? 256 : 128;
     const int ngn = w->group >= a.ntile ? 1 : a.ntile / w->group;
     a.nkb_main = d / 64;
@@ -1300,7 +1336,7 @@ int launch_dgrad(int which, const uint16_t* a_src, const uint16_t* a_lora, const
     if (rc != TQP_OK) return rc;
     a.unit_tab = unit_tab;
     a.wait_ns = wait_limit_ns();
-    return run_expert_dx(a, mp, units_upper, s);
+    return run_expert_dgrad(DX, a, mp, units_upper, s);
   }
   // DX on the shared-memory engine: K = 2f (gate rows then up rows of W), N = d
   a.ntile = (d % 256 == 0 && bB == 4) ? 256 : 128;

@@ -182,7 +182,9 @@ int layer_backward(const uint16_t* x, const float* dy, int T, const tqp_moe_weig
     return rc;
   if (r > 0 && (rc = launch_rank_bwd(0, B.dO, L.offsets, fb.mb_prefix, w, T, B.bk16, B.dha, status, s)) != TQP_OK)
     return rc;
-  if ((rc = launch_dgrad(0, B.dO, B.dha, L.offsets, fb.mb_prefix, w, T, B.gu, B.dgu, status, s)) != TQP_OK) return rc;
+  if ((rc = launch_dgrad(0, B.dO, B.dha, L.offsets, fb.mb_prefix, w, T, B.gu, B.dgu, status, s, fb.mb_prefix256,
+                         fb.unit_tab)) != TQP_OK)
+    return rc;
   if (r > 0) {
     if ((rc = launch_rank_bwd(1, B.dgu, L.offsets, fb.mb_prefix, w, T, B.bk16, B.dxa, status, s)) != TQP_OK)
       return rc;
