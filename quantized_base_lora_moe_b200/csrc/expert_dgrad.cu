@@ -437,6 +437,17 @@ __global__ void __launch_bounds__(kThreads, 1)
       const Unit un = us.take(u);
       const int feat = un.nt * 128 + lane_feature<BITS>(lrow);   // input feature m of this lane
       bool ok = true;
+      if (a.nkb_lora > 0 && grp == 0 && u + int(gridDim.x) < nunits) {
+        // the next unit's rank-space columns into L2: for each j, this warp's 32
+        // features are one 64-byte piece of row j of Ag^T / Au^T (Ad^T)
+        const Unit nx = us.peek();
+        const size_t col = size_t(nx.nt) * 128 + 32 * q4;
+        for (int j = lane; j < a.lora_k; j += 32) {
+          const uint16_t* src = j < a.r ? a.lb0 + (size_t(nx.e) * a.r + j) * a.lb_ld
+                                        : a.lb1 + (size_t(nx.e) * a.r + (j - a.r)) * a.lb_ld;
+          prefetch_l2(src + col);
+        }
+      }
       for (int kb = 0; kb < nkb; ++kb, ++n) {
         const bool main_stage = kb >= a.nkb_lora;
         const int mq = m;
@@ -448,27 +459,30 @@ __global__ void __launch_bounds__(kThreads, 1)
         tc_fence_after();
         if (!main_stage) {
           // rank-space stage: A[m][j] = Ag^T[j][m] (j < r), Au^T[j - r][m] (r <= j < 2r), else 0,
-          // written to TMEM in two halves of 16 columns (32 K values each)
+          // written to TMEM in eight pieces of 4 columns (8 K values each)
           // dX: Ag^T then Au^T (lora_k = 2r); dH: Ad^T (lora_k = r)
           const uint16_t* pg = a.lb0 + size_t(un.e) * a.r * a.lb_ld + feat;
           const uint16_t* pu = MODE == DX ? a.lb1 + size_t(un.e) * a.r * a.lb_ld + feat : pg;
 #pragma unroll 1
-          for (int hv = 0; hv < 2; ++hv) {
-            uint32_t w16[16];
+          for (int qv = 0; qv < 8; ++qv) {
+            // 8 loads are issued together (addresses selected, invalid columns read
+            // a valid element and are zeroed), then converted into 4 columns
+            uint16_t raw[8];
 #pragma unroll
-            for (int c = 0; c < 16; ++c) {
-              uint32_t pr = 0;
-#pragma unroll
-              for (int h = 0; h < 2; ++h) {
-                const int j = kb * kK + 32 * hv + 2 * c + h;
-                uint32_t bits = 0;
-                if (j < a.r) bits = __ldg(pg + size_t(j) * a.lb_ld);
-                else if (j < a.lora_k) bits = __ldg(pu + size_t(j - a.r) * a.lb_ld);
-                pr |= bf16_to_f16_bits_chk(bits, lora_inf) << (16 * h);
-              }
-              w16[c] = pr;
+            for (int t = 0; t < 8; ++t) {
+              const int j = kb * kK + 8 * qv + t;
+              const uint16_t* ptr = (j < a.r) ? pg + size_t(j) * a.lb_ld : pu + size_t(j - a.r) * a.lb_ld;
+              raw[t] = __ldg(j < a.lora_k ? ptr : pg);
             }
-            tmem_st16(tw + uint32_t(st) * kWCols + uint32_t(16 * hv), w16);
+            uint32_t w4[4];
+#pragma unroll
+            for (int c = 0; c < 4; ++c) {
+              const int j = kb * kK + 8 * qv + 2 * c;
+              const uint32_t lo = j < a.lora_k ? bf16_to_f16_bits_chk(raw[2 * c], lora_inf) : 0u;
+              const uint32_t hi = j + 1 < a.lora_k ? bf16_to_f16_bits_chk(raw[2 * c + 1], lora_inf) : 0u;
+              w4[c] = lo | (hi << 16);
+            }
+            tmem_st4(tw + uint32_t(st) * kWCols + uint32_t(4 * qv), w4);
           }
         } else {
           uint32_t v[32];
