@@ -9,11 +9,10 @@
 //   LORA_XA : xa = s * X_e [Ag | Au]            (bf16 operands, fp16 out)
 //   LORA_HA : ha = s * H_e Ad                   (fp16)
 //   ROUTER  : logits = x W_r^T (+ bias), W_r split exactly into 3 bf16 parts
-//   DH      : dH = dO Wd + dhA Ad^T, with the SwiGLU backward in the epilogue
-//   DX      : dX = [dG|dU] [Wg;Wu] + dxa [Ag;Au]^T
-//             (the dgrads read the weight tile as an MN-major B operand: W is
-//             stored with the contraction index as its row, so the int4 rows are
-//             dequantised straight into the tile, no transpose)
+//   DX      : dX = [dG|dU] [Wg;Wu] + dxa [Ag;Au]^T, for model widths that are not
+//             a multiple of 128 (else expert_dgrad.cu); the weight tile is an
+//             MN-major B operand: W is stored with the contraction index as its
+//             row, so the int4 rows are dequantised straight into the tile)
 //
 // Work unit = (expert e, n-tile of up to 256 columns, m-block of up to 128
 // routed rows); one 128 x N x 64 tcgen05.mma step per K-block. Per CTA (1 per
@@ -68,7 +67,7 @@ constexpr size_t kOperandBytes = size_t(kAStages) * kAStageBytes + size_t(kBStag
 template <int MODE>
 struct Layout {
   static constexpr bool kTma = (MODE == LORA_XA || MODE == LORA_HA || MODE == ROUTER);
-  static constexpr bool kTrans = (MODE == DH || MODE == DX);
+  static constexpr bool kTrans = (MODE == DX);
   static constexpr int kA = kTrans ? 4 : kAStages;
   static constexpr int kB = kTma ? (MODE == ROUTER ? 4 : 8) : (kTrans ? 3 : kBStages);
   // LORA_XA: 2r rows (r <= 64), LORA_HA: r rows, ROUTER: up to 256 rows, x 128 B
@@ -133,7 +132,7 @@ __global__ void __launch_bounds__(kThreads, 1)
                         const __grid_constant__ CUtensorMap tq1, const __grid_constant__ CUtensorMap ts0,
                         const __grid_constant__ CUtensorMap ts1, const __grid_constant__ CUtensorMap ta,
                         const __grid_constant__ CUtensorMap tb0, const __grid_constant__ CUtensorMap tb1) {
-  constexpr bool kTrans = (MODE == DH || MODE == DX);      // dgrads: B = the weight tile, MN-major
+  constexpr bool kTrans = (MODE == DX);      // dgrad: B = the weight tile, MN-major
   constexpr bool kDequant = (MODE == GATEUP || kTrans);
   constexpr bool kATma = (MODE == LORA_HA || MODE == ROUTER || kTrans);
   constexpr bool kBTma = (MODE == LORA_XA || MODE == LORA_HA || MODE == ROUTER);
@@ -256,44 +255,6 @@ __global__ void __launch_bounds__(kThreads, 1)
                 ga[i] = gq;
                 ua[i] = uq;
               }
-            }
-          }
-        }
-      } else if (MODE == DH) {
-        // dH -> dG = dH * U * silu'(G), dU = dH * silu(G); G, U from the recompute
-        const size_t ld2 = 2 * size_t(a.f_dim);
-        const uint16_t* grow_gu = a.aux + grow * ld2 + un.nt * a.ntile;
-        uint16_t* drow = static_cast<uint16_t*>(a.out) + grow * ld2 + un.nt * a.ntile;
-#pragma unroll 1
-        for (int c = 0; c < a.ntile; c += 32) {
-          float v[32];
-          tmem_ld32(tacc + c, v);
-          if (valid) {
-#pragma unroll
-            for (int q = 0; q < 4; ++q) {
-              const uint4 gq = *reinterpret_cast<const uint4*>(grow_gu + c + 8 * q);
-              const uint4 uq = *reinterpret_cast<const uint4*>(grow_gu + a.f_dim + c + 8 * q);
-              const uint32_t gw[4] = {gq.x, gq.y, gq.z, gq.w};
-              const uint32_t uw[4] = {uq.x, uq.y, uq.z, uq.w};
-              uint32_t dg[4], du[4];
-#pragma unroll
-              for (int t = 0; t < 4; ++t) {
-                float res_g[2], res_u[2];
-#pragma unroll
-                for (int hh = 0; hh < 2; ++hh) {
-                  const float g = f16_to_f32(uint16_t(hh ? (gw[t] >> 16) : (gw[t] & 0xFFFFu)));
-                  const float u = f16_to_f32(uint16_t(hh ? (uw[t] >> 16) : (uw[t] & 0xFFFFu)));
-                  const float dh = v[8 * q + 2 * t + hh];
-                  const float sg = 1.0f / (1.0f + __expf(-g));
-                  res_g[hh] = dh * u * sg * (1.0f + g * (1.0f - sg));
-                  res_u[hh] = dh * g * sg;
-                }
-                dg[t] = pack_f16x2(res_g[0], res_g[1]);
-                du[t] = pack_f16x2(res_u[0], res_u[1]);
-                bad |= f16x2_nonfinite(dg[t]) | f16x2_nonfinite(du[t]);
-              }
-              *reinterpret_cast<uint4*>(drow + c + 8 * q) = make_uint4(dg[0], dg[1], dg[2], dg[3]);
-              *reinterpret_cast<uint4*>(drow + a.f_dim + c + 8 * q) = make_uint4(du[0], du[1], du[2], du[3]);
             }
           }
         }
@@ -544,7 +505,6 @@ __global__ void __launch_bounds__(kThreads, 1)
     // dgrad modes: two groups of 128 threads take alternate stages
     const int grp = kBGroups > 1 ? tid >> 7 : 0;
     const int gtid = kBGroups > 1 ? tid & 127 : tid;
-    constexpr int kGT = 256 / kBGroups;                      // threads per group
     Ring rb, q;
     bool inexact = false;   // a group scale whose products q * s are not exact in fp16
     bool lora_inf = false;  // an adapter value beyond the fp16 range
@@ -1278,29 +1238,8 @@ int launch_dgrad(int which, const uint16_t* a_src, const uint16_t* a_lora, const
     a.wait_ns = wait_limit_ns();
     return run_expert_dgrad(DH, a, mp, units_upper, s);
   }
-  if (which == 0) {  // DH on the shared-memory engine: K = d (rows of Wd), N = f
-    a.ntile = (f % 256 == 0 && bB == 4) ? 256 : 128;
-    const int ngn = w->group >= a.ntile ? 1 : a.ntile / w->group;
-    a.nkb_main = d / 64;
-    a.nkb_lora = r > 0 ? (r + 63) / 64 : 0;
-    a.lora_k = r;
-    a.lora_ld = r;
-    a.n_tiles = f / a.ntile;
-    a.in_dim = f;
-    a.out_dim = d;
-    a.lb0 = w->lora_a[2];
-    a.lb_ld = f;
-    a.aux = const_cast<uint16_t*>(aux_gu);
-    a.out_ld = 2 * f;
-    a.n_valid = f;
-    bool ok = make_tile_map(&mp.m[TA], a_src, uint64_t(A), uint64_t(d), 128) &&
-              make_map(&mp.m[TQ0], CU_TENSOR_MAP_DATA_TYPE_UINT8, w->wq[2], uint64_t(f) * bB / 8, uint64_t(w->E) * d,
-                       uint64_t(f) * bB / 8, uint32_t(a.ntile * bB / 8), 64, a.ntile * bB / 8 == 128 ? 128 : 0) &&
-              make_map(&mp.m[TS0], CU_TENSOR_MAP_DATA_TYPE_UINT16, w->wscale[2], d, uint64_t(w->E) * (f / w->group),
-                       uint64_t(d) * 2, 64, ngn);
-    if (!ok) return TQP_ERR_CUDA;
-    return run_gemm<DH>(a, mp, mb_upper * a.n_tiles, s);
-  }
+  // dH runs only on the tensor-memory kernel (the backward requires ffn % 128 == 0)
+  if (which == 0) return TQP_ERR_UNSUPPORTED;
   if (mb_prefix256 && unit_tab && d % 128 == 0) {
     // DX with W^T in tensor memory (expert_dgrad.cu): units of 128 input features x
     // up to 256 rows; K = 2r rank-space columns, then the f gate and f up rows of W
