@@ -1127,22 +1127,37 @@ int launch_grouped_ffn(const uint16_t* x, int T, const int32_t* offsets, const i
 //   which 0: Bd, stored B^T [E][d][r]  ->  [E][r][d]             (n = r,  K = d)
 //   which 1: blockdiag(Bg, Bu), each stored B^T [E][f][r]  ->  [E][2r][2f], Bg in
 //            rows [0, r) x columns [0, f), Bu in rows [r, 2r) x columns [f, 2f)
+// The r values of a source row arrive as 16-byte pieces and land transposed in
+// shared memory as fp16; each output row's 64 K values leave as 16-byte pieces.
 __global__ void __launch_bounds__(256) rank_b_kernel(const uint16_t* __restrict__ b0, const uint16_t* __restrict__ b1,
                                                      int which, int r, int f, int K, uint16_t* __restrict__ out) {
-  __shared__ uint16_t tile[64][66];   // [k][j], j < r <= 64
+  __shared__ __align__(16) uint16_t tile[64][72];   // [j][k], fp16; j < r <= 64, row pitch 144 B
   const int e = blockIdx.y, k0 = blockIdx.x * 64;
   const int n = which == 0 ? r : 2 * r;
   const bool up = which == 1 && k0 >= f;   // f % 64 == 0: a slice lies in one half
   const uint16_t* src = which == 0 ? b0 + (size_t(e) * K + k0) * r
                                    : (up ? b1 + (size_t(e) * f + (k0 - f)) * r : b0 + (size_t(e) * f + k0) * r);
-  for (int i = threadIdx.x; i < 64 * r; i += blockDim.x) tile[i / r][i % r] = src[i];   // 64 source rows of r
+  const int r8 = r >> 3;   // r % 8 == 0
+  for (int i = threadIdx.x; i < 64 * r8; i += blockDim.x) {   // 64 source rows of r
+    const int kk = i / r8, j8 = i - kk * r8;
+    const uint4 v = __ldg(reinterpret_cast<const uint4*>(src) + i);
+    const uint32_t wv[4] = {v.x, v.y, v.z, v.w};
+#pragma unroll
+    for (int q = 0; q < 4; ++q) {
+      tile[j8 * 8 + 2 * q][kk] = uint16_t(bf16_to_f16_bits(uint16_t(wv[q] & 0xFFFFu)));
+      tile[j8 * 8 + 2 * q + 1][kk] = uint16_t(bf16_to_f16_bits(uint16_t(wv[q] >> 16)));
+    }
+  }
   __syncthreads();
-  for (int i = threadIdx.x; i < n * 64; i += blockDim.x) {
-    const int j = i >> 6, kk = i & 63;
-    uint16_t v = 0;
-    if (which == 0) v = uint16_t(bf16_to_f16_bits(tile[kk][j]));
-    else if ((j >= r) == up) v = uint16_t(bf16_to_f16_bits(tile[kk][up ? j - r : j]));
-    out[(size_t(e) * n + j) * K + k0 + kk] = v;
+  for (int i = threadIdx.x; i < n * 8; i += blockDim.x) {
+    const int j = i >> 3, c = i & 7;
+    uint4 o = make_uint4(0, 0, 0, 0);
+    if (which == 0) {
+      o = *reinterpret_cast<const uint4*>(&tile[j][c * 8]);
+    } else if ((j >= r) == up) {
+      o = *reinterpret_cast<const uint4*>(&tile[up ? j - r : j][c * 8]);
+    }
+    *reinterpret_cast<uint4*>(out + (size_t(e) * n + j) * K + k0 + c * 8) = o;
   }
 }
 

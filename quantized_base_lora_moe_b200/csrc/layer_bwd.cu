@@ -23,18 +23,6 @@
 
 namespace tqp {
 
-__global__ void add_f32_kernel(const float* __restrict__ a, const float* __restrict__ b, float* __restrict__ out,
-                               size_t n) {
-  const size_t i = size_t(blockIdx.x) * blockDim.x + threadIdx.x;
-  if (i < n) out[i] = a[i] + b[i];
-}
-
-int launch_add_f32(const float* a, const float* b, float* out, size_t n, cudaStream_t s) {
-  if (n == 0) return TQP_OK;
-  add_f32_kernel<<<unsigned((n + 255) / 256), 256, 0, s>>>(a, b, out, n);
-  return cudaGetLastError() == cudaSuccess ? TQP_OK : TQP_ERR_CUDA;
-}
-
 // ----------------------------------------------------------------------------
 // cotangent scale
 // ----------------------------------------------------------------------------
@@ -68,84 +56,119 @@ __device__ __forceinline__ float grad_scale(const uint32_t* dmax) {
 
 constexpr int kMaxK = 32;
 
+// One block per token. The token's slots (row, gate, expert) go to shared memory
+// first; the O and router rows are then loaded four slots at a time, so that
+// their latencies overlap, and each slot's dot product <dy, O> is reduced per
+// warp straight into shared memory.
 __global__ void __launch_bounds__(256) bwd_combine_kernel(const uint16_t* __restrict__ O, const int32_t* __restrict__ inv,
                                                           const float* __restrict__ gates,
                                                           const int32_t* __restrict__ ids,
                                                           const float* __restrict__ router_w,
                                                           const float* __restrict__ dy, int T, int k, int d,
                                                           const uint32_t* __restrict__ dmax, uint16_t* __restrict__ dO,
-                                                          float* __restrict__ dx, int32_t* status) {
+                                                          const float* __restrict__ addend, float* __restrict__ dx,
+                                                          int32_t* status) {
   __shared__ float red[8][kMaxK];
   __shared__ float dl_s[kMaxK];
+  __shared__ int row_s[kMaxK], id_s[kMaxK];
+  __shared__ float g_s[kMaxK];
   const int t = blockIdx.x;
   const float gsc = grad_scale(dmax);
   uint32_t bad = 0;
   const int lane = threadIdx.x & 31, wid = threadIdx.x >> 5;
   const int nwarps = blockDim.x >> 5;
-  float part[kMaxK];
-#pragma unroll
-  for (int j = 0; j < kMaxK; ++j) part[j] = 0.0f;
-  for (int c = threadIdx.x * 8; c < d; c += blockDim.x * 8) {
-    const float4* dp = reinterpret_cast<const float4*>(dy + size_t(t) * d + c);
-    const float4 a0 = dp[0], a1 = dp[1];
+  if (threadIdx.x < k) {
+    row_s[threadIdx.x] = inv[size_t(t) * k + threadIdx.x];
+    id_s[threadIdx.x] = ids[size_t(t) * k + threadIdx.x];
+    g_s[threadIdx.x] = gates[size_t(t) * k + threadIdx.x];
+  }
+  for (int i = threadIdx.x; i < 8 * kMaxK; i += blockDim.x) (&red[0][0])[i] = 0.0f;
+  __syncthreads();
+  // the column loop runs whole warps (lanes past d idle inside it), so the
+  // full-mask shuffles below always see all 32 lanes
+  for (int cw = (threadIdx.x & ~31) * 8; cw < d; cw += blockDim.x * 8) {
+    const int c = cw + lane * 8;
+    const bool act = c < d;
+    float4 a0 = make_float4(0.0f, 0.0f, 0.0f, 0.0f), a1 = a0;
+    if (act) {
+      const float4* dp = reinterpret_cast<const float4*>(dy + size_t(t) * d + c);
+      a0 = __ldg(dp);
+      a1 = __ldg(dp + 1);
+    }
     const float dv[8] = {a0.x, a0.y, a0.z, a0.w, a1.x, a1.y, a1.z, a1.w};
+    for (int j0 = 0; j0 < k; j0 += 4) {
+      uint4 ov[4];
 #pragma unroll
-    for (int j = 0; j < kMaxK; ++j) {
-      if (j >= k) break;
-      const int row = inv[size_t(t) * k + j];
-      const float g = gates[size_t(t) * k + j] * gsc;
-      const uint4 ov = *reinterpret_cast<const uint4*>(O + size_t(row) * d + c);
-      const uint32_t ow[4] = {ov.x, ov.y, ov.z, ov.w};
-      float acc = 0.0f;
-      uint32_t pk[4];
+      for (int b = 0; b < 4; ++b)
+        ov[b] = (act && j0 + b < k) ? __ldg(reinterpret_cast<const uint4*>(O + size_t(row_s[j0 + b]) * d + c))
+                                    : make_uint4(0, 0, 0, 0);
 #pragma unroll
-      for (int q = 0; q < 4; ++q) {
-        acc = fmaf(dv[2 * q], f16_to_f32(uint16_t(ow[q] & 0xFFFFu)), acc);
-        acc = fmaf(dv[2 * q + 1], f16_to_f32(uint16_t(ow[q] >> 16)), acc);
-        pk[q] = pack_f16x2(g * dv[2 * q], g * dv[2 * q + 1]);
-        bad |= f16x2_nonfinite(pk[q]);
+      for (int b = 0; b < 4; ++b) {
+        const int j = j0 + b;
+        if (j >= k) break;
+        const float g = g_s[j] * gsc;
+        const uint32_t ow[4] = {ov[b].x, ov[b].y, ov[b].z, ov[b].w};
+        float acc = 0.0f;
+        uint32_t pk[4];
+#pragma unroll
+        for (int q = 0; q < 4; ++q) {
+          acc = fmaf(dv[2 * q], f16_to_f32(uint16_t(ow[q] & 0xFFFFu)), acc);
+          acc = fmaf(dv[2 * q + 1], f16_to_f32(uint16_t(ow[q] >> 16)), acc);
+          pk[q] = pack_f16x2(g * dv[2 * q], g * dv[2 * q + 1]);
+          bad |= f16x2_nonfinite(pk[q]);
+        }
+        if (act) *reinterpret_cast<uint4*>(dO + size_t(row_s[j]) * d + c) = make_uint4(pk[0], pk[1], pk[2], pk[3]);
+        // dgamma_j partial of this warp's columns
+#pragma unroll
+        for (int o = 16; o > 0; o >>= 1) acc += __shfl_xor_sync(0xFFFFFFFFu, acc, o);
+        if (lane == 0) red[wid][j] += acc;
       }
-      part[j] += acc;
-      *reinterpret_cast<uint4*>(dO + size_t(row) * d + c) = make_uint4(pk[0], pk[1], pk[2], pk[3]);
     }
   }
   if (__any_sync(0xFFFFFFFFu, bad != 0) && lane == 0) raise_status(status, TQP_STATUS_NONFINITE);
-  // dgamma_j = sum over the row: warp then block reduction
-#pragma unroll
-  for (int j = 0; j < kMaxK; ++j) {
-    if (j >= k) break;
-    float v = part[j];
-#pragma unroll
-    for (int o = 16; o > 0; o >>= 1) v += __shfl_xor_sync(0xFFFFFFFFu, v, o);
-    if (lane == 0) red[wid][j] = v;
-  }
   __syncthreads();
   if (threadIdx.x == 0) {
-    float dg[kMaxK], gs[kMaxK];
     float sum = 0.0f;
     for (int j = 0; j < k; ++j) {
       float v = 0.0f;
       for (int w = 0; w < nwarps; ++w) v += red[w][j];
-      dg[j] = v;
-      gs[j] = gates[size_t(t) * k + j];
-      sum += gs[j] * v;
+      dl_s[j] = v;
+      sum += g_s[j] * v;
     }
-    for (int j = 0; j < k; ++j) dl_s[j] = gs[j] * (dg[j] - sum);
+    for (int j = 0; j < k; ++j) dl_s[j] = g_s[j] * (dl_s[j] - sum);
   }
   __syncthreads();
-  // dx[t] = sum_j dl_j W_r[id_j]  (through the frozen full-precision router)
+  // dx[t] = addend[t] + sum_j dl_j W_r[id_j]  (through the frozen full-precision router)
   for (int c = threadIdx.x * 8; c < d; c += blockDim.x * 8) {
     float acc[8];
+    if (addend) {
+      const float4* ap = reinterpret_cast<const float4*>(addend + size_t(t) * d + c);
+      const float4 b0 = __ldg(ap), b1 = __ldg(ap + 1);
+      acc[0] = b0.x; acc[1] = b0.y; acc[2] = b0.z; acc[3] = b0.w;
+      acc[4] = b1.x; acc[5] = b1.y; acc[6] = b1.z; acc[7] = b1.w;
+    } else {
 #pragma unroll
-    for (int i = 0; i < 8; ++i) acc[i] = 0.0f;
-    for (int j = 0; j < k; ++j) {
-      const int e = ids[size_t(t) * k + j];
-      const float4* wp = reinterpret_cast<const float4*>(router_w + size_t(e) * d + c);
-      const float4 w0 = __ldg(wp), w1 = __ldg(wp + 1);
-      const float wv[8] = {w0.x, w0.y, w0.z, w0.w, w1.x, w1.y, w1.z, w1.w};
-      const float l = dl_s[j];
+      for (int i = 0; i < 8; ++i) acc[i] = 0.0f;
+    }
+    for (int j0 = 0; j0 < k; j0 += 4) {
+      float4 w[4][2];
 #pragma unroll
-      for (int i = 0; i < 8; ++i) acc[i] = fmaf(l, wv[i], acc[i]);
+      for (int b = 0; b < 4; ++b) {
+        if (j0 + b < k) {
+          const float4* wp = reinterpret_cast<const float4*>(router_w + size_t(id_s[j0 + b]) * d + c);
+          w[b][0] = __ldg(wp);
+          w[b][1] = __ldg(wp + 1);
+        } else {
+          w[b][0] = w[b][1] = make_float4(0.0f, 0.0f, 0.0f, 0.0f);
+        }
+      }
+#pragma unroll
+      for (int b = 0; b < 4; ++b) {
+        const float l = (j0 + b < k) ? dl_s[j0 + b] : 0.0f;
+        const float wv[8] = {w[b][0].x, w[b][0].y, w[b][0].z, w[b][0].w, w[b][1].x, w[b][1].y, w[b][1].z, w[b][1].w};
+#pragma unroll
+        for (int i = 0; i < 8; ++i) acc[i] = fmaf(l, wv[i], acc[i]);
+      }
     }
     float4* xp = reinterpret_cast<float4*>(dx + size_t(t) * d + c);
     xp[0] = make_float4(acc[0], acc[1], acc[2], acc[3]);
@@ -164,14 +187,22 @@ __global__ void __launch_bounds__(256) gather_add_kernel(const uint16_t* __restr
     float4* xp = reinterpret_cast<float4*>(dx + size_t(t) * d + c);
     const float4 b0 = xp[0], b1 = xp[1];
     float acc[8] = {0.0f, 0.0f, 0.0f, 0.0f, 0.0f, 0.0f, 0.0f, 0.0f};
-    for (int j = 0; j < k; ++j) {
-      const int row = inv[size_t(t) * k + j];
-      const uint4 v = *reinterpret_cast<const uint4*>(dX + size_t(row) * d + c);
-      const uint32_t w[4] = {v.x, v.y, v.z, v.w};
+    // four slots' rows in flight at a time; the sum keeps the fixed j order
+    for (int j0 = 0; j0 < k; j0 += 4) {
+      uint4 v[4];
 #pragma unroll
-      for (int q = 0; q < 4; ++q) {
-        acc[2 * q] += f16_to_f32(uint16_t(w[q] & 0xFFFFu));
-        acc[2 * q + 1] += f16_to_f32(uint16_t(w[q] >> 16));
+      for (int b = 0; b < 4; ++b)
+        v[b] = (j0 + b < k) ? __ldg(reinterpret_cast<const uint4*>(dX + size_t(__ldg(inv + size_t(t) * k + j0 + b)) * d + c))
+                            : make_uint4(0, 0, 0, 0);
+#pragma unroll
+      for (int b = 0; b < 4; ++b) {
+        if (j0 + b >= k) break;
+        const uint32_t w[4] = {v[b].x, v[b].y, v[b].z, v[b].w};
+#pragma unroll
+        for (int q = 0; q < 4; ++q) {
+          acc[2 * q] += f16_to_f32(uint16_t(w[q] & 0xFFFFu));
+          acc[2 * q + 1] += f16_to_f32(uint16_t(w[q] >> 16));
+        }
       }
     }
     xp[0] = make_float4(fmaf(acc[0], inv_sc, b0.x), fmaf(acc[1], inv_sc, b0.y), fmaf(acc[2], inv_sc, b0.z),
@@ -288,11 +319,11 @@ int launch_grad_absmax(const float* dy, size_t n, uint32_t* dmax, cudaStream_t s
 
 int launch_bwd_combine(const uint16_t* O, const int32_t* inv, const float* gates, const int32_t* ids,
                        const float* router_w, const float* dy, int T, int k, int d, const uint32_t* dmax, uint16_t* dO,
-                       float* dx, int32_t* status, cudaStream_t s) {
+                       const float* addend, float* dx, int32_t* status, cudaStream_t s) {
   if (T == 0) return TQP_OK;
   // whole warps only: the row reductions use full-mask warp shuffles
   const int threads = d / 8 >= 256 ? 256 : ((d / 8 + 31) / 32) * 32;
-  bwd_combine_kernel<<<T, threads, 0, s>>>(O, inv, gates, ids, router_w, dy, T, k, d, dmax, dO, dx, status);
+  bwd_combine_kernel<<<T, threads, 0, s>>>(O, inv, gates, ids, router_w, dy, T, k, d, dmax, dO, addend, dx, status);
   return cudaGetLastError() == cudaSuccess ? TQP_OK : TQP_ERR_CUDA;
 }
 

@@ -169,7 +169,8 @@ BwdWs carve_bwd(void* p0, int T, const tqp_moe_weights* w) {
 // with the G|U pre-activations kept (layer_forward with aux_gu = the backward
 // scratch's gu), so its routing and intermediates are still in place.
 int layer_backward(const uint16_t* x, const float* dy, int T, const tqp_moe_weights* w, float* dx,
-                   const tqp_adapter_grads* g, void* ws, int32_t* status, cudaStream_t s, bool recompute = true) {
+                   const tqp_adapter_grads* g, void* ws, int32_t* status, cudaStream_t s, bool recompute = true,
+                   const float* dx_addend = nullptr) {
   const LayerWs L = carve_layer_ws(ws, T, w);
   const BwdWs B = carve_bwd(static_cast<char*>(ws) + layer_ws_size(T, w), T, w);
   const int k = w->top_k, d = w->d, f = w->ffn, r = w->rank, E = w->E;
@@ -177,8 +178,8 @@ int layer_backward(const uint16_t* x, const float* dy, int T, const tqp_moe_weig
   if (recompute && (rc = layer_experts(x, T, w, L, status, s, B.gu)) != TQP_OK) return rc;
   const FfnBufs fb = ffn_carve(L.ffn_ws, T, w);
   if ((rc = launch_grad_absmax(dy, size_t(T) * d, B.dmax, s)) != TQP_OK) return rc;
-  if ((rc = launch_bwd_combine(L.out_perm, L.inv, L.gates, L.ids, w->router_w, dy, T, k, d, B.dmax, B.dO, dx, status,
-                               s)) != TQP_OK)
+  if ((rc = launch_bwd_combine(L.out_perm, L.inv, L.gates, L.ids, w->router_w, dy, T, k, d, B.dmax, B.dO, dx_addend,
+                               dx, status, s)) != TQP_OK)
     return rc;
   if (r > 0 && (rc = launch_rank_bwd(0, B.dO, L.offsets, fb.mb_prefix, w, T, B.bk16, B.dha, status, s)) != TQP_OK)
     return rc;
@@ -280,7 +281,6 @@ struct StackWs {
   float* s[2][4];     // two sets of (stream 1, stream 2, cotangent 1, cotangent 2), fp32 [T][d]
   uint16_t* zb;       // bf16 layer input
   uint16_t* ab;       // bf16 layer input
-  float* dxl;         // a layer's input gradient
   void* lws;          // one layer's forward + backward workspace
 };
 
@@ -297,16 +297,13 @@ StackWs carve_stack(void* ws, int T, int d) {
   p += align_up(Td * 2, 256);
   w.ab = reinterpret_cast<uint16_t*>(p);
   p += align_up(Td * 2, 256);
-  w.dxl = reinterpret_cast<float*>(p);
-  p += align_up(Td * 4, 256);
   w.lws = p;
   return w;
 }
 
 size_t stack_ws_size(int T, int L, const tqp_moe_weights* const* F, const tqp_moe_weights* const* G) {
   const size_t Td = size_t(T) * F[0]->d;
-  return 8 * align_up(Td * 4, 256) + 2 * align_up(Td * 2, 256) + align_up(Td * 4, 256) +
-         stack_layer_ws(T, L, F, G) + 512;
+  return 8 * align_up(Td * 4, 256) + 2 * align_up(Td * 2, 256) + stack_layer_ws(T, L, F, G) + 512;
 }
 
 // Block backward on fp32 streams: from the block outputs (y1, y2) and their
@@ -322,12 +319,12 @@ int block_backward_f32(const float* y1, const float* y2, const float* dy1, const
   if ((rc = to_bf16(y1, w.zb, Td, s)) != TQP_OK) return rc;
   uint16_t* gu = carve_bwd(static_cast<char*>(w.lws) + layer_ws_size(T, G), T, G).gu;
   if ((rc = layer_forward(w.zb, T, G, y2, 1, -1.0f, a2, 1, w.ab, w.lws, status, s, gu)) != TQP_OK) return rc;
-  if ((rc = layer_backward(w.zb, dy2, T, G, w.dxl, gG, w.lws, status, s, false)) != TQP_OK) return rc;
-  if ((rc = launch_add_f32(dy1, w.dxl, da1, Td, s)) != TQP_OK) return rc;
+  // da1 = dy1 + J_G^T dy2, the sum taken inside G's backward
+  if ((rc = layer_backward(w.zb, dy2, T, G, da1, gG, w.lws, status, s, false, dy1)) != TQP_OK) return rc;
   gu = carve_bwd(static_cast<char*>(w.lws) + layer_ws_size(T, F), T, F).gu;
   if ((rc = layer_forward(w.ab, T, F, y1, 1, -1.0f, a1, 1, nullptr, w.lws, status, s, gu)) != TQP_OK) return rc;
-  if ((rc = layer_backward(w.ab, da1, T, F, w.dxl, gF, w.lws, status, s, false)) != TQP_OK) return rc;
-  return launch_add_f32(dy2, w.dxl, da2, Td, s);
+  // da2 = dy2 + J_F^T da1
+  return layer_backward(w.ab, da1, T, F, da2, gF, w.lws, status, s, false, dy2);
 }
 
 }  // namespace
@@ -517,7 +514,7 @@ size_t tqp_adapter_bwd_workspace_size(int T, const tqp_moe_weights* F, const tqp
   const size_t fw = rev_couple_workspace_size(T, F, G);
   size_t m = a > b ? a : b;
   m = m > fw ? m : fw;
-  return m + align_up(size_t(T) * F->d * 2, 256) + align_up(size_t(T) * F->d * 4, 256) + 512;
+  return m + align_up(size_t(T) * F->d * 2, 256) + 512;
 }
 
 int tqp_adapter_bwd(const float* y1, const float* y2, const float* dy1, const float* dy2, int T,
@@ -538,22 +535,19 @@ int tqp_adapter_bwd(const float* y1, const float* y2, const float* dy1, const fl
   const size_t Td = size_t(T) * F->d;
   char* base = reinterpret_cast<char*>(align_up(reinterpret_cast<uintptr_t>(ws), 256));
   uint16_t* zb = reinterpret_cast<uint16_t*>(base);                     // bf16(y1)
-  float* dxG = reinterpret_cast<float*>(base + align_up(Td * 2, 256));  // J_G^T dy2
-  void* lws = base + align_up(Td * 2, 256) + align_up(Td * 4, 256);
+  void* lws = base + align_up(Td * 2, 256);
   // Each layer's backward follows the inverse step that ran that layer's forward
   // on the same workspace (keeping G|U), so it does not recompute the forward.
   // G-step: reconstruct x2 = y2 - G(bf16(y1)); G's grads for cotangent dy2
   if ((rc = to_bf16(y1, zb, Td, s)) != TQP_OK) return rc;
   uint16_t* gu = carve_bwd(static_cast<char*>(lws) + layer_ws_size(T, G), T, G).gu;
   if ((rc = layer_forward(zb, T, G, y2, 1, -1.0f, x2, 0, nullptr, lws, dev_status, s, gu)) != TQP_OK) return rc;
-  if ((rc = layer_backward(zb, dy2, T, G, dxG, gG, lws, dev_status, s, false)) != TQP_OK) return rc;
-  // dz1 = dy1 + J_G^T dy2 -> dx1 (dx1 = dz1)
-  if ((rc = launch_add_f32(dy1, dxG, dx1, Td, s)) != TQP_OK) return rc;
+  // dz1 = dy1 + J_G^T dy2 -> dx1 (dx1 = dz1), the sum taken inside G's backward
+  if ((rc = layer_backward(zb, dy2, T, G, dx1, gG, lws, dev_status, s, false, dy1)) != TQP_OK) return rc;
   // F-step: x1 = y1 - F(x2); F's grads for cotangent dz1; dx2 = dy2 + J_F^T dz1
   gu = carve_bwd(static_cast<char*>(lws) + layer_ws_size(T, F), T, F).gu;
   if ((rc = layer_forward(x2, T, F, y1, 1, -1.0f, x1, 0, nullptr, lws, dev_status, s, gu)) != TQP_OK) return rc;
-  if ((rc = layer_backward(x2, dx1, T, F, dxG, gF, lws, dev_status, s, false)) != TQP_OK) return rc;
-  return launch_add_f32(dy2, dxG, dx2, Td, s);
+  return layer_backward(x2, dx1, T, F, dx2, gF, lws, dev_status, s, false, dy2);
 }
 
 size_t rev_stack_workspace_size(int T, int L, const tqp_moe_weights* const* F, const tqp_moe_weights* const* G) {

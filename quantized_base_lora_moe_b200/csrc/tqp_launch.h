@@ -90,7 +90,7 @@ int launch_rank_bwd(int which, const uint16_t* P, const int32_t* offsets, const 
 int launch_grad_absmax(const float* dy, size_t n, uint32_t* dmax, cudaStream_t s);
 int launch_bwd_combine(const uint16_t* O, const int32_t* inv, const float* gates, const int32_t* ids,
                        const float* router_w, const float* dy, int T, int k, int d, const uint32_t* dmax, uint16_t* dO,
-                       float* dx, int32_t* status, cudaStream_t s);
+                       const float* addend, float* dx, int32_t* status, cudaStream_t s);   // dx = addend (or 0) + router term
 int launch_gather_add(const uint16_t* dX, const int32_t* inv, int T, int k, int d, const uint32_t* dmax, float* dx,
                       cudaStream_t s);
 // adapter gradients on the tensor cores (wgrad.cu); TQP_ERR_UNSUPPORTED for ranks above 32
@@ -103,8 +103,4 @@ int launch_outer(int E, int M, int N, const int32_t* offsets, const int32_t* per
 
 int num_sms();
 
-}  // namespace tqp
-
-namespace tqp {
-int launch_add_f32(const float* a, const float* b, float* out, size_t n, cudaStream_t s);
 }  // namespace tqp
