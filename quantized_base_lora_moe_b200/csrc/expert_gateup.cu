@@ -140,9 +140,11 @@ __device__ __forceinline__ void stage16(uint8_t* tile, int t0, int feat, const u
 // the 64 gate and 64 up rows of its 64 features in its own TMEM, half of the
 // unit's token rows in its shared memory, and receives its 128 x N quarter of
 // the accumulator (all N tokens of its features), so SwiGLU stays in the CTA.
-// The odd CTA's readiness reaches the MMA thread through a relay thread that
-// forwards each completed stage to the even CTA's full barrier of that stage;
-// the MMA completions are multicast to both CTAs.
+// Stage n is ready when the even CTA's full barrier completes: both CTAs' weight
+// groups arrive on it (the odd CTA's remotely, release at cluster scope), and
+// both CTAs' token loads complete their bytes on it (the odd CTA's through the
+// cta_group::2 form of the TMA load); the even CTA's token thread expects the
+// bytes of both halves. The MMA completions are multicast to both CTAs.
 //
 // Every role arrives once per warp (after __syncwarp), and the MMA thread waits
 // on one barrier per stage (weights, token bytes and the pair relay together).
@@ -176,8 +178,9 @@ __global__ void __launch_bounds__(kThreads, 1)
   if (threadIdx.x == 0) {
     for (int i = 0; i < kXStages; ++i) mbar_init(&ctl->x_empty[i], 1);
     for (int i = 0; i < kWStages; ++i) {
-      // one weight group (4 warps) + the token TMA thread (+ the odd CTA's relay)
-      mbar_init(&ctl->w_full[i], 4 + 1 + ((PAIR && rank == 0) ? 1 : 0));
+      // one weight group (4 warps) + the token TMA thread; pair (even CTA): the
+      // odd CTA's weight group as well (its token bytes need no arrival)
+      mbar_init(&ctl->w_full[i], PAIR ? 4 + 4 + 1 : 4 + 1);
       mbar_init(&ctl->w_empty[i], 1);
     }
     for (int i = 0; i < kQStages; ++i) {
@@ -373,23 +376,6 @@ __global__ void __launch_bounds__(kThreads, 1)
       if (PAIR) umma2_commit_both(&ctl->drain);
       else umma_commit(&ctl->drain);
       mbar_drain(&ctl->drain, 0, 100000000ull);
-    } else if (lane == 0) {
-      // ------------------------------------------------------------ relay (odd CTA of a pair)
-      // Each stage whose token tile has landed and whose weight stage is in
-      // TMEM here is reported to the even CTA's MMA thread, in stage order.
-      const uint32_t full0 = mapa_shared(smem_u32(&ctl->w_full[0]), 0);
-      Ring rw;
-      bool ok = true;
-      for (int u = u0; u < nunits && ok; u += ustride) {
-        for (int kb = 0; kb < nkb; ++kb) {
-          if (!mbar_wait(&ctl->w_full[rw.stage], rw.phase, abort_flag, a.status)) {
-            ok = false;
-            break;
-          }
-          mbar_arrive_cluster(full0 + uint32_t(rw.stage) * 8u);
-          rw.next<kWStages>();
-        }
-      }
     }
     __syncwarp();
   } else if (warp == 5) {
@@ -442,16 +428,25 @@ __global__ void __launch_bounds__(kThreads, 1)
           // the adapter stage reads s X [Ag|Au] (zero-filled past its 2r columns), the rest X_perm
           const CUtensorMap* map = kb < a.nkb_lora ? &txa : &tx;
           const int col = (kb < a.nkb_lora ? kb : kb - a.nkb_lora) * kK;
-          mbar_arrive_expect_tx(bar, uint32_t(nbox * 16384));
-          tma_load_2d(smem_u32(st), map, bar, col, row0);
-          if (nbox == 2) tma_load_2d(smem_u32(st + 16384), map, bar, col, row0 + 128);
+          if (!PAIR) {
+            mbar_arrive_expect_tx(bar, uint32_t(nbox * 16384));
+            tma_load_2d(smem_u32(st), map, bar, col, row0);
+            if (nbox == 2) tma_load_2d(smem_u32(st + 16384), map, bar, col, row0 + 128);
+          } else if (rank == 0) {
+            mbar_arrive_expect_tx(bar, uint32_t(2 * 16384));   // both CTAs' halves
+            tma_load_2d(smem_u32(st), map, bar, col, row0);
+          } else {
+            tma_load_2d_pair(smem_u32(st), map, mapa_shared(smem_u32(bar), 0), col, row0);
+          }
           pend.issued(rw.stage, rw.phase);
           rx.next<kXStages>();
           rw.next<kWStages>();
         }
         if (!ok) break;
       }
-      if (aborted(abort_flag)) pend.drain(ctl->w_full);
+      // (the odd CTA's fills complete on the even CTA's barriers, which the even
+      // CTA drains before the pair's final cluster barrier)
+      if (aborted(abort_flag) && (!PAIR || rank == 0)) pend.drain(ctl->w_full);
     }
   } else if (warp >= kWWarp0) {
     // ------------------------------------------------------------ weight producer
@@ -547,7 +542,12 @@ __global__ void __launch_bounds__(kThreads, 1)
         tmem_st32(tw + uint32_t(st) * kWCols, v);
         tmem_wait_st();
         tc_fence_before();
-        mbar_arrive_warp(&ctl->w_full[st]);
+        if (PAIR) {   // both CTAs' groups arrive on the even CTA's barrier
+          __syncwarp();
+          if (lane == 0) mbar_arrive_cluster(mapa_shared(smem_u32(&ctl->w_full[st]), 0));
+        } else {
+          mbar_arrive_warp(&ctl->w_full[st]);
+        }
       }
       if (!ok) break;
     }
