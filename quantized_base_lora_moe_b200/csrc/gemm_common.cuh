@@ -202,6 +202,10 @@ __device__ __forceinline__ uint32_t scale_pair_chk(uint16_t sbits, bool& inexact
 }
 
 // Host side: the tensor maps handed to a grouped GEMM launch.
+// 128B-swizzled tile map of a row-major 16-bit matrix [rows][cols]: box {64, box_rows}
+// (grouped_gemm.cu).
+bool make_tile_map(CUtensorMap* m, const void* ptr, uint64_t rows, uint64_t cols, uint32_t box_rows);
+
 struct Maps {
   CUtensorMap m[7];
 };

@@ -808,7 +808,7 @@ static bool make_map(CUtensorMap* m, CUtensorMapDataType dt, const void* ptr, ui
 }
 
 // 128B-swizzled K-major tile map of a row-major 16-bit matrix [rows][cols]: box {64, box_rows}.
-static bool make_tile_map(CUtensorMap* m, const void* ptr, uint64_t rows, uint64_t cols, uint32_t box_rows) {
+bool make_tile_map(CUtensorMap* m, const void* ptr, uint64_t rows, uint64_t cols, uint32_t box_rows) {
   return make_map(m, CU_TENSOR_MAP_DATA_TYPE_UINT16, ptr, cols, rows, cols * 2, 64, box_rows, 128);
 }
 

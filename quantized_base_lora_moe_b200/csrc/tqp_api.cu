@@ -191,7 +191,7 @@ int layer_backward(const uint16_t* x, const float* dy, int T, const tqp_moe_weig
       return rc;
     // adapter gradients, in the storage layouts A^T [r][in], B^T [out][r]: on the
     // tensor cores for ranks up to 32, else as outer products on the CUDA cores
-    rc = launch_wgrad(w, L.offsets, nullptr, B.dO, L.h, B.dgu, fb.xperm, fb.ha, B.dha, fb.xa, B.dxa, g, B.dmax, status, s);
+    rc = launch_wgrad(w, size_t(T) * k, L.offsets, nullptr, B.dO, L.h, B.dgu, fb.xperm, fb.ha, B.dha, fb.xa, B.dxa, g, B.dmax, status, s);
     if (rc != TQP_OK && rc != TQP_ERR_UNSUPPORTED) return rc;
   }
   if (r > 0 && rc == TQP_ERR_UNSUPPORTED) {

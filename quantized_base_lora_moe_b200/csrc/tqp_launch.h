@@ -94,7 +94,8 @@ int launch_bwd_combine(const uint16_t* O, const int32_t* inv, const float* gates
 int launch_gather_add(const uint16_t* dX, const int32_t* inv, int T, int k, int d, const uint32_t* dmax, float* dx,
                       cudaStream_t s);
 // adapter gradients on the tensor cores (wgrad.cu); TQP_ERR_UNSUPPORTED for ranks above 32
-int launch_wgrad(const tqp_moe_weights* w, const int32_t* offsets, const int32_t* perm, const uint16_t* dO,
+// A: the routed rows of the expert-sorted operands (T * top_k)
+int launch_wgrad(const tqp_moe_weights* w, size_t A, const int32_t* offsets, const int32_t* perm, const uint16_t* dO,
                  const uint16_t* h, const uint16_t* dgu, const uint16_t* x16, const uint16_t* ha, const uint16_t* dha,
                  const uint16_t* xa, const uint16_t* dxa, const tqp_adapter_grads* g, const uint32_t* dmax,
                  int32_t* status, cudaStream_t s);

@@ -25,11 +25,16 @@
 // Per CTA (persistent, 1 per SM, 288 threads):
 //   warps 0-3  epilogue: TMEM -> registers -> fp32 stores (one m per thread)
 //   warp  4    TMEM allocation + one thread issuing tcgen05.mma
-//   warps 5-8  producers: cp.async of 64-row stages of P (128 m) and Q (r or 2r)
+//   warps 5-8  producers of 64-row stages: P (128 m) by two TMA boxes of
+//              64 x 64 (128B swizzle, the MN-major atom layout), issued by one
+//              thread; Q (r or 2r) by cp.async, zero-filled past the expert's
+//              rows, so that the P rows a box reads past them contribute nothing.
+//              (X gathered through perm: P by cp.async as well.)
 // Accumulators are double-buffered in TMEM (2 x 64 columns), so ranks up to 32
 // (kind 3 needs 2r columns); the MMA's N is the width rounded up to 16. Every
-// wait is bounded (tqp_device.cuh); no TMA is used.
+// wait is bounded (tqp_device.cuh); no TMA multicast is used.
 #include <cstdint>
+#include <cstring>
 #include <cuda_runtime.h>
 
 #include "../../include/tqp_moe.h"
@@ -41,7 +46,7 @@ namespace tqp {
 namespace wgrad {
 
 constexpr int kThreads = 288;
-constexpr int kStages = 6;
+constexpr int kStages = 8;
 constexpr int kRowsPerStage = 64;                 // k rows (routed rows) per stage: 4 MMA K-steps
 constexpr int kABytes = 2 * kRowsPerStage * 128;  // 128 m: two 64-wide MN atoms of 64 rows x 128 B
 constexpr int kBBytes = kRowsPerStage * 128;      // up to 64 j: one MN atom
@@ -124,7 +129,10 @@ __device__ __forceinline__ float inv_grad_scale(const uint32_t* dmax) {
   return ldexpf(1.0f, -max(-120, min(120, 8 - e)));
 }
 
-__global__ void __launch_bounds__(kThreads, 1) wgrad_kernel(const Args a) {
+// tp[kind]: the P matrix of each kind as a box {64 m, 64 rows} map (unused when perm is set)
+__global__ void __launch_bounds__(kThreads, 1)
+    wgrad_kernel(const Args a, const __grid_constant__ CUtensorMap tp0, const __grid_constant__ CUtensorMap tp1,
+                 const __grid_constant__ CUtensorMap tp2, const __grid_constant__ CUtensorMap tp3) {
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   uint8_t* a_base = smem;
@@ -136,7 +144,7 @@ __global__ void __launch_bounds__(kThreads, 1) wgrad_kernel(const Args a) {
 
   if (threadIdx.x == 0) {
     for (int i = 0; i < kStages; ++i) {
-      mbar_init(&ctl->full[i], 128);
+      mbar_init(&ctl->full[i], 128);   // the producers' cp.async arrivals (the P boxes add their bytes)
       mbar_init(&ctl->empty[i], 1);
     }
     for (int i = 0; i < 2; ++i) {
@@ -244,9 +252,17 @@ __global__ void __launch_bounds__(kThreads, 1) wgrad_kernel(const Args a) {
     }
     __syncwarp();
   } else {
-    // ------------------------------------------------------------ producers (cp.async)
+    // ------------------------------------------------------------ producers
     const int tid = threadIdx.x - 5 * 32;   // 0..127
+    const bool ptma = a.perm == nullptr;    // P rows are contiguous: TMA boxes
     Ring rs;
+    PendingFills pend;
+    if (tid == 0 && ptma) {
+      prefetch_tmap(&tp0);
+      prefetch_tmap(&tp1);
+      prefetch_tmap(&tp2);
+      prefetch_tmap(&tp3);
+    }
     for (int u = blockIdx.x; u < nunits; u += gridDim.x) {
       const WUnit w = decode(a, u);
       if (w.rows <= 0) continue;
@@ -270,16 +286,28 @@ __global__ void __launch_bounds__(kThreads, 1) wgrad_kernel(const Args a) {
         const uint32_t as = smem_u32(a_base + size_t(rs.stage) * kABytes);
         const uint32_t bs = smem_u32(b_base + size_t(rs.stage) * kBBytes);
         const int k0 = s * kRowsPerStage;
-        // P: 64 rows x 16 chunks (128 m); 16 consecutive threads read one row
+        if (ptma) {
+          // P: two boxes of 64 m x 64 rows (rows past the expert are read, and
+          // meet Q's zero rows; rows past the matrix are zero-filled)
+          if (tid == 0) {
+            const CUtensorMap* map = w.kind == 0 ? &tp0 : w.kind == 1 ? &tp1 : w.kind == 2 ? &tp2 : &tp3;
+            mbar_expect_tx(&ctl->full[rs.stage], uint32_t(2 * 64 * 128));
+            tma_load_2d(as, map, &ctl->full[rs.stage], pcol, w.base + k0);
+            tma_load_2d(as + kAtomCol, map, &ctl->full[rs.stage], pcol + 64, w.base + k0);
+            pend.issued(rs.stage, rs.phase);
+          }
+        } else {
+          // P: 64 rows x 16 chunks (128 m); 16 consecutive threads read one row
 #pragma unroll
-        for (int i = 0; i < 8; ++i) {
-          const int c = tid + 128 * i;
-          const int kk = c >> 4, ch = c & 15;
-          const bool in = k0 + kk < w.rows;
-          int prow = w.base + k0 + kk;
-          if (w.kind == 3 && in && a.perm) prow = __ldg(a.perm + prow);
-          const uint16_t* src = P + size_t(in ? prow : 0) * ldp + pcol + ch * 8;
-          cp_async16(as + mn_offset(kk, ch), src, in ? 16u : 0u);
+          for (int i = 0; i < 8; ++i) {
+            const int c = tid + 128 * i;
+            const int kk = c >> 4, ch = c & 15;
+            const bool in = k0 + kk < w.rows;
+            int prow = w.base + k0 + kk;
+            if (w.kind == 3 && in && a.perm) prow = __ldg(a.perm + prow);
+            const uint16_t* src = P + size_t(in ? prow : 0) * ldp + pcol + ch * 8;
+            cp_async16(as + mn_offset(kk, ch), src, in ? 16u : 0u);
+          }
         }
         // Q: 64 rows x nchunk chunks
         for (int c = tid; c < kRowsPerStage * nchunk; c += 128) {
@@ -294,6 +322,8 @@ __global__ void __launch_bounds__(kThreads, 1) wgrad_kernel(const Args a) {
       if (!ok) break;
     }
     cp_async_wait_all();
+    // on an abort, wait (bounded) for every TMA fill issued by this thread
+    if (tid == 0 && aborted(abort_flag)) pend.drain(ctl->full);
   }
 
   tc_fence_before();
@@ -306,7 +336,7 @@ __global__ void __launch_bounds__(kThreads, 1) wgrad_kernel(const Args a) {
 
 }  // namespace wgrad
 
-int launch_wgrad(const tqp_moe_weights* w, const int32_t* offsets, const int32_t* perm, const uint16_t* dO,
+int launch_wgrad(const tqp_moe_weights* w, size_t A, const int32_t* offsets, const int32_t* perm, const uint16_t* dO,
                  const uint16_t* h, const uint16_t* dgu, const uint16_t* x16, const uint16_t* ha, const uint16_t* dha,
                  const uint16_t* xa, const uint16_t* dxa, const tqp_adapter_grads* g, const uint32_t* dmax,
                  int32_t* status, cudaStream_t s) {
@@ -343,9 +373,19 @@ int launch_wgrad(const tqp_moe_weights* w, const int32_t* offsets, const int32_t
   a.wait_ns = wait_limit_ns();
   static DeviceFlags attr_done;
   if (!attr_done.test_and_set_device(wgrad::wgrad_kernel, int(wgrad::kSmemBytes))) return TQP_ERR_CUDA;
+  CUtensorMap tp[4];
+  std::memset(tp, 0, sizeof(tp));
+  if (!perm) {
+    // the P matrices are expert-sorted rows [A][width]
+    const uint64_t rows = uint64_t(A);
+    if (!make_tile_map(&tp[0], dO, rows, uint64_t(w->d), 64) || !make_tile_map(&tp[1], h, rows, uint64_t(w->ffn), 64) ||
+        !make_tile_map(&tp[2], dgu, rows, uint64_t(2 * w->ffn), 64) ||
+        !make_tile_map(&tp[3], x16, rows, uint64_t(w->d), 64))
+      return TQP_ERR_CUDA;
+  }
   const int units = a.E * a.tile_prefix[4];
   const int grid = units < num_sms() ? units : num_sms();
-  wgrad::wgrad_kernel<<<grid, wgrad::kThreads, wgrad::kSmemBytes, s>>>(a);
+  wgrad::wgrad_kernel<<<grid, wgrad::kThreads, wgrad::kSmemBytes, s>>>(a, tp[0], tp[1], tp[2], tp[3]);
   return cudaGetLastError() == cudaSuccess ? TQP_OK : TQP_ERR_CUDA;
 }
 
