@@ -437,7 +437,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       const Unit un = us.take(u);
       const int feat = un.nt * 128 + lane_feature<BITS>(lrow);   // input feature m of this lane
       bool ok = true;
-      if (a.nkb_lora > 0 && grp == 0 && u + int(gridDim.x) < nunits) {
+      if (a.nkb_lora > 0 && !a.lt && grp == 0 && u + int(gridDim.x) < nunits) {
         // the next unit's rank-space columns into L2: for each j, this warp's 32
         // features are one 64-byte piece of row j of Ag^T / Au^T (Ad^T)
         const Unit nx = us.peek();
@@ -457,7 +457,21 @@ __global__ void __launch_bounds__(kThreads, 1)
         const uint32_t ph = uint32_t(n / kWStages) & 1u;
         if (!mbar_wait_warp(&ctl->w_empty[st], ph ^ 1u, abort_flag, a.status)) { ok = false; break; }
         tc_fence_after();
-        if (!main_stage) {
+        if (!main_stage && a.lt) {
+          // rank-space stage from the row copy: this feature's lt_w fp16 values are one
+          // contiguous row, loaded as up to eight 16-byte pieces at once; column c of
+          // the stage holds the pair j = 2c, 2c + 1 (zero past lora_k)
+          const uint4* rowp =
+              reinterpret_cast<const uint4*>(a.lt + (size_t(un.e) * a.in_dim + feat) * a.lt_w + kb * kK);
+          const int npc = (min(kK, a.lt_w - kb * kK)) >> 3;   // 16-byte pieces in this stage (lt_w % 8 == 0)
+          uint32_t v[32];
+#pragma unroll
+          for (int q = 0; q < 8; ++q) {
+            const uint4 p4 = q < npc ? __ldg(rowp + q) : make_uint4(0, 0, 0, 0);
+            v[4 * q] = p4.x; v[4 * q + 1] = p4.y; v[4 * q + 2] = p4.z; v[4 * q + 3] = p4.w;
+          }
+          tmem_st32(tw + uint32_t(st) * kWCols, v);
+        } else if (!main_stage) {
           // rank-space stage: A[m][j] = Ag^T[j][m] (j < r), Au^T[j - r][m] (r <= j < 2r), else 0,
           // written to TMEM in eight pieces of 4 columns (8 K values each)
           // dX: Ag^T then Au^T (lora_k = 2r); dH: Ad^T (lora_k = r)

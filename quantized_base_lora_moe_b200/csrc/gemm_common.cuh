@@ -47,6 +47,9 @@ struct GemmArgs {
   const uint16_t* lb0;     // DH / DX rank-space step: A^T sources read transposed (Ad^T | Ag^T)
   const uint16_t* lb1;     // DX: Au^T
   int lb_ld;
+  const uint16_t* lt;      // DH / DX rank-space step, if set: the same A values row by row in fp16,
+                           // [E][in][lt_w] (lt_w = lora_k), read as whole rows instead of lb0 / lb1
+  int lt_w;
   const int4* unit_tab;    // expert kernels: decoded units {e, n-tile, rows, base}, one per unit
   int bits;                // base-weight code width: 4 (packed int4) or 8 (int8)
   unsigned long long wait_ns;   // limit of one barrier wait (0: the default kWaitLimitNs)

@@ -1161,6 +1161,49 @@ __global__ void __launch_bounds__(256) rank_b_kernel(const uint16_t* __restrict_
   }
 }
 
+// Row copy of the adapter A factors for the rank-space stage of the dgrads, in fp16:
+//   which 0 (dH): out[e][n][j] = Ad^T[e][j][n]                                  [E][f][r]
+//   which 1 (dX): out[e][m][j] = Ag^T[e][j][m] (j < r), Au^T[e][j - r][m] (r <= j < 2r)   [E][d][2r]
+// so that a tensor-memory lane (one input feature) loads its values as one
+// contiguous row. One block per (64 input features, expert), transposed through
+// shared memory; a value beyond the fp16 range raises TQP_STATUS_NONFINITE.
+__global__ void __launch_bounds__(256) lora_a_rows_kernel(const uint16_t* __restrict__ a0,
+                                                          const uint16_t* __restrict__ a1, int which, int r, int in,
+                                                          uint16_t* __restrict__ out, int32_t* status) {
+  __shared__ __align__(16) uint16_t tile[64][136];   // [feature][j], fp16; j < 2r <= 128, row pitch 272 B
+  const int e = blockIdx.y, m0 = blockIdx.x * 64;
+  const int w = which == 0 ? r : 2 * r;
+  bool bad = false;
+  for (int i = threadIdx.x; i < w * 8; i += blockDim.x) {   // source rows j: 64 features = 8 pieces
+    const int j = i >> 3, c = i & 7;
+    const uint16_t* src = (j < r ? a0 + (size_t(e) * r + j) * in : a1 + (size_t(e) * r + (j - r)) * in) + m0 + c * 8;
+    const uint4 v = __ldg(reinterpret_cast<const uint4*>(src));
+    const uint32_t wv[4] = {v.x, v.y, v.z, v.w};
+#pragma unroll
+    for (int q = 0; q < 4; ++q) {
+      tile[c * 8 + 2 * q][j] = uint16_t(bf16_to_f16_bits_chk(uint16_t(wv[q] & 0xFFFFu), bad));
+      tile[c * 8 + 2 * q + 1][j] = uint16_t(bf16_to_f16_bits_chk(uint16_t(wv[q] >> 16), bad));
+    }
+  }
+  __syncthreads();
+  const int pcs = w >> 3;   // 16-byte pieces per output row (r % 8 == 0)
+  for (int i = threadIdx.x; i < 64 * pcs; i += blockDim.x) {
+    const int f = i / pcs, c = i - f * pcs;
+    *reinterpret_cast<uint4*>(out + (size_t(e) * in + m0 + f) * w + c * 8) =
+        *reinterpret_cast<const uint4*>(&tile[f][c * 8]);
+  }
+  if (__syncthreads_or(bad) && threadIdx.x == 0) raise_status(status, TQP_STATUS_NONFINITE);
+}
+
+int launch_lora_a_rows(int which, const tqp_moe_weights* w, uint16_t* out, int32_t* status, cudaStream_t s) {
+  const int r = w->rank;
+  if (r == 0) return TQP_OK;
+  const int in = which == 0 ? w->ffn : w->d;   // multiples of 64
+  lora_a_rows_kernel<<<dim3(unsigned(in / 64), unsigned(w->E)), 256, 0, s>>>(
+      which == 0 ? w->lora_a[2] : w->lora_a[0], which == 0 ? w->lora_a[2] : w->lora_a[1], which, r, in, out, status);
+  return cudaGetLastError() == cudaSuccess ? TQP_OK : TQP_ERR_CUDA;
+}
+
 int launch_rank_bwd(int which, const uint16_t* P, const int32_t* offsets, const int32_t* mb_prefix,
                     const tqp_moe_weights* w, int T, uint16_t* bk16, uint16_t* C, int32_t* status, cudaStream_t s) {
   const int r = w->rank, d = w->d, f = w->ffn;
@@ -1197,7 +1240,7 @@ int launch_rank_bwd(int which, const uint16_t* P, const int32_t* offsets, const 
 
 int launch_dgrad(int which, const uint16_t* a_src, const uint16_t* a_lora, const int32_t* offsets,
                  const int32_t* mb_prefix, const tqp_moe_weights* w, int T, const uint16_t* aux_gu, uint16_t* out,
-                 int32_t* status, cudaStream_t s, const int32_t* mb_prefix256, int4* unit_tab) {
+                 int32_t* status, cudaStream_t s, const int32_t* mb_prefix256, int4* unit_tab, const uint16_t* a_rows) {
   if (T == 0) return TQP_OK;
   const size_t A = size_t(T) * w->top_k;
   const int d = w->d, f = w->ffn, r = w->rank;
@@ -1231,6 +1274,8 @@ int launch_dgrad(int which, const uint16_t* a_src, const uint16_t* a_lora, const
     a.out_dim = d;
     a.lb0 = w->lora_a[2];
     a.lb_ld = f;
+    a.lt = r > 0 ? a_rows : nullptr;
+    a.lt_w = r;
     a.aux = const_cast<uint16_t*>(aux_gu);
     a.out_ld = 2 * f;
     a.n_valid = f;
@@ -1269,6 +1314,8 @@ int launch_dgrad(int which, const uint16_t* a_src, const uint16_t* a_lora, const
     a.lb0 = w->lora_a[0];
     a.lb1 = w->lora_a[1];
     a.lb_ld = d;
+    a.lt = r > 0 ? a_rows : nullptr;
+    a.lt_w = 2 * r;
     a.out_ld = d;
     a.n_valid = d;
     const uint32_t cbox = uint32_t(128 * bB / 8);   // one tile's 128 features of a code row

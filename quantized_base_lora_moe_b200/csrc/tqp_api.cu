@@ -120,6 +120,7 @@ struct BwdWs {
   uint16_t* dgu;    // dG | dU [A][2f] fp16
   uint16_t* dxa;    // s [dG|dU] [Bg|Bu]^T [A][2r] fp16
   uint16_t* bk16;   // K-major fp16 B operand of dha / dxa, E * max(r d, 4 r f) values
+  uint16_t* arow;   // row copy of Ad ([E][f][r]) or [Ag | Au] ([E][d][2r]) in fp16 for the dgrads
   uint32_t* dmax;   // max |dy| (sets the power-of-two scale of the fp16 intermediates)
 };
 
@@ -137,10 +138,16 @@ size_t rank_b_values(const tqp_moe_weights* w) {
   return size_t(w->E) * (rd > rf4 ? rd : rf4);
 }
 
+size_t arow_values(const tqp_moe_weights* w) {
+  const size_t fr = size_t(w->ffn) * w->rank, d2r = size_t(2) * w->d * w->rank;
+  return size_t(w->E) * (fr > d2r ? fr : d2r);
+}
+
 size_t bwd_extra_bytes(int T, const tqp_moe_weights* w) {
   const size_t A = size_t(T) * w->top_k;
   return align_up(A * 2 * w->ffn * 2, 256) * 2 + align_up(A * w->d * 2, 256) + align_up(A * w->rank * 2, 256) +
-         align_up(A * 2 * w->rank * 2, 256) + align_up(rank_b_values(w) * 2, 256) + 256 + 256;
+         align_up(A * 2 * w->rank * 2, 256) + align_up(rank_b_values(w) * 2, 256) + align_up(arow_values(w) * 2, 256) +
+         256 + 256;
 }
 
 BwdWs carve_bwd(void* p0, int T, const tqp_moe_weights* w) {
@@ -158,6 +165,7 @@ BwdWs carve_bwd(void* p0, int T, const tqp_moe_weights* w) {
   b.dgu = static_cast<uint16_t*>(take(A * 2 * w->ffn * 2));
   b.dxa = static_cast<uint16_t*>(take(A * 2 * w->rank * 2));
   b.bk16 = static_cast<uint16_t*>(take(rank_b_values(w) * 2));
+  b.arow = static_cast<uint16_t*>(take(arow_values(w) * 2));
   b.dmax = static_cast<uint32_t*>(take(sizeof(uint32_t)));
   return b;
 }
@@ -183,8 +191,9 @@ int layer_backward(const uint16_t* x, const float* dy, int T, const tqp_moe_weig
     return rc;
   if (r > 0 && (rc = launch_rank_bwd(0, B.dO, L.offsets, fb.mb_prefix, w, T, B.bk16, B.dha, status, s)) != TQP_OK)
     return rc;
+  if (r > 0 && (rc = launch_lora_a_rows(0, w, B.arow, status, s)) != TQP_OK) return rc;
   if ((rc = launch_dgrad(0, B.dO, B.dha, L.offsets, fb.mb_prefix, w, T, B.gu, B.dgu, status, s, fb.mb_prefix256,
-                         fb.unit_tab)) != TQP_OK)
+                         fb.unit_tab, B.arow)) != TQP_OK)
     return rc;
   if (r > 0) {
     if ((rc = launch_rank_bwd(1, B.dgu, L.offsets, fb.mb_prefix, w, T, B.bk16, B.dxa, status, s)) != TQP_OK)
@@ -207,8 +216,9 @@ int layer_backward(const uint16_t* x, const float* dy, int T, const tqp_moe_weig
       return rc;
   }
   uint16_t* dX = B.dO;  // dO is no longer needed
+  if (r > 0 && (rc = launch_lora_a_rows(1, w, B.arow, status, s)) != TQP_OK) return rc;
   if ((rc = launch_dgrad(1, B.dgu, B.dxa, L.offsets, fb.mb_prefix, w, T, nullptr, dX, status, s, fb.mb_prefix256,
-                         fb.unit_tab)) != TQP_OK)
+                         fb.unit_tab, B.arow)) != TQP_OK)
     return rc;
   return launch_gather_add(dX, L.inv, T, k, d, B.dmax, dx, s);
 }

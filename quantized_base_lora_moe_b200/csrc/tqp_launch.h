@@ -76,7 +76,11 @@ int launch_grouped_ffn_part(int part, const uint16_t* x, int T, const int32_t* o
 // tensor-memory dX kernel; null keeps the shared-memory engine.
 int launch_dgrad(int which, const uint16_t* a_src, const uint16_t* a_lora, const int32_t* offsets,
                  const int32_t* mb_prefix, const tqp_moe_weights* w, int T, const uint16_t* aux_gu, uint16_t* out,
-                 int32_t* status, cudaStream_t s, const int32_t* mb_prefix256 = nullptr, int4* unit_tab = nullptr);
+                 int32_t* status, cudaStream_t s, const int32_t* mb_prefix256 = nullptr, int4* unit_tab = nullptr,
+                 const uint16_t* a_rows = nullptr);
+// Row copy of the adapter A factors for the dgrads' rank-space stage (grouped_gemm.cu):
+// which 0: Ad as [E][f][r] (dH), which 1: [Ag | Au] as [E][d][2r] (dX), fp16.
+int launch_lora_a_rows(int which, const tqp_moe_weights* w, uint16_t* out, int32_t* status, cudaStream_t s);
 // rank-space products of the backward on the tensor cores (grouped_gemm.cu):
 //   which 0: dha = s dO Bd      (P = dO [A][d]      -> C [A][r])
 //   which 1: dxa = s [dG|dU] blockdiag(Bg, Bu)   (P = dgu [A][2f] -> C [A][2r])

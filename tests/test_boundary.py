@@ -101,14 +101,17 @@ def test_grouped_ffn_part_rejects_unknown_part():
 def test_backward_workspace_holds_its_scratch(cfg):
     # the backward adds, per routed row, G|U and dG|dU (2f each), dO (d), dha (r) and
     # dxa (2r) as fp16, plus the K-major fp16 B operand of the rank-space products:
-    # Bd as [E][r][d] or blockdiag(Bg, Bu) as [E][2r][2f], whichever is larger
+    # Bd as [E][r][d] or blockdiag(Bg, Bu) as [E][2r][2f], whichever is larger, and
+    # the row copy of the A factors for the dgrads: Ad as [E][f][r] or [Ag|Au] as
+    # [E][d][2r], whichever is larger
     L = Q.lib()
     w = _struct(cfg)
     A = cfg.T * cfg.k
     extra = (L.tqp_moe_layer_bwd_workspace_size(cfg.T, ctypes.byref(w))
              - L.tqp_moe_layer_workspace_size(cfg.T, ctypes.byref(w)))
-    need = A * (4 * cfg.f + cfg.d + 3 * cfg.r) * 2 + cfg.E * max(cfg.r * cfg.d, 4 * cfg.r * cfg.f) * 2
-    assert need <= extra <= need + 8 * 256 + 256
+    need = (A * (4 * cfg.f + cfg.d + 3 * cfg.r) * 2 + cfg.E * max(cfg.r * cfg.d, 4 * cfg.r * cfg.f) * 2
+            + cfg.E * max(cfg.f * cfg.r, 2 * cfg.d * cfg.r) * 2)
+    assert need <= extra <= need + 9 * 256 + 256
 
 
 def _grads(**bad):
