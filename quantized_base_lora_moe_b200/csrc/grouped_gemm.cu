@@ -1170,27 +1170,31 @@ __global__ void __launch_bounds__(256) rank_b_kernel(const uint16_t* __restrict_
 __global__ void __launch_bounds__(256) lora_a_rows_kernel(const uint16_t* __restrict__ a0,
                                                           const uint16_t* __restrict__ a1, int which, int r, int in,
                                                           uint16_t* __restrict__ out, int32_t* status) {
-  __shared__ __align__(16) uint16_t tile[64][136];   // [feature][j], fp16; j < 2r <= 128, row pitch 272 B
+  // [feature][j], fp16; j < 2r <= 128, row pitch 272 B. The 8-value pieces of row f
+  // are rotated by (f / 8) mod pieces, so that the eight threads that write one j
+  // of eight feature groups hit different banks.
+  __shared__ __align__(16) uint16_t tile[64][136];
   const int e = blockIdx.y, m0 = blockIdx.x * 64;
   const int w = which == 0 ? r : 2 * r;
+  const int pcs = w >> 3;   // 16-byte pieces per output row (r % 8 == 0)
   bool bad = false;
   for (int i = threadIdx.x; i < w * 8; i += blockDim.x) {   // source rows j: 64 features = 8 pieces
     const int j = i >> 3, c = i & 7;
     const uint16_t* src = (j < r ? a0 + (size_t(e) * r + j) * in : a1 + (size_t(e) * r + (j - r)) * in) + m0 + c * 8;
     const uint4 v = __ldg(reinterpret_cast<const uint4*>(src));
     const uint32_t wv[4] = {v.x, v.y, v.z, v.w};
+    const int jp = (((j >> 3) + c) % pcs) * 8 + (j & 7);   // rotation of row group c (rows 8c .. 8c + 7)
 #pragma unroll
     for (int q = 0; q < 4; ++q) {
-      tile[c * 8 + 2 * q][j] = uint16_t(bf16_to_f16_bits_chk(uint16_t(wv[q] & 0xFFFFu), bad));
-      tile[c * 8 + 2 * q + 1][j] = uint16_t(bf16_to_f16_bits_chk(uint16_t(wv[q] >> 16), bad));
+      tile[c * 8 + 2 * q][jp] = uint16_t(bf16_to_f16_bits_chk(uint16_t(wv[q] & 0xFFFFu), bad));
+      tile[c * 8 + 2 * q + 1][jp] = uint16_t(bf16_to_f16_bits_chk(uint16_t(wv[q] >> 16), bad));
     }
   }
   __syncthreads();
-  const int pcs = w >> 3;   // 16-byte pieces per output row (r % 8 == 0)
   for (int i = threadIdx.x; i < 64 * pcs; i += blockDim.x) {
     const int f = i / pcs, c = i - f * pcs;
     *reinterpret_cast<uint4*>(out + (size_t(e) * in + m0 + f) * w + c * 8) =
-        *reinterpret_cast<const uint4*>(&tile[f][c * 8]);
+        *reinterpret_cast<const uint4*>(&tile[f][((c + (f >> 3)) % pcs) * 8]);
   }
   if (__syncthreads_or(bad) && threadIdx.x == 0) raise_status(status, TQP_STATUS_NONFINITE);
 }
