@@ -127,15 +127,17 @@ __global__ void __launch_bounds__(256) bwd_combine_kernel(const uint16_t* __rest
   }
   if (__any_sync(0xFFFFFFFFu, bad != 0) && lane == 0) raise_status(status, TQP_STATUS_NONFINITE);
   __syncthreads();
-  if (threadIdx.x == 0) {
-    float sum = 0.0f;
-    for (int j = 0; j < k; ++j) {
-      float v = 0.0f;
-      for (int w = 0; w < nwarps; ++w) v += red[w][j];
-      dl_s[j] = v;
-      sum += g_s[j] * v;
-    }
-    for (int j = 0; j < k; ++j) dl_s[j] = g_s[j] * (dl_s[j] - sum);
+  if (wid == 0) {
+    // lane j < k: dgamma_j over the warps' partials, then the softmax backward over
+    // the chosen logits, dl_j = gamma_j (dgamma_j - sum_i gamma_i dgamma_i)
+    float v = 0.0f;
+    if (lane < k)
+      for (int w = 0; w < nwarps; ++w) v += red[w][lane];
+    const float gj = lane < k ? g_s[lane] : 0.0f;
+    float sum = gj * v;
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) sum += __shfl_xor_sync(0xFFFFFFFFu, sum, o);
+    if (lane < k) dl_s[lane] = gj * (v - sum);
   }
   __syncthreads();
   // dx[t] = addend[t] + sum_j dl_j W_r[id_j]  (through the frozen full-precision router)
