@@ -702,6 +702,21 @@ __global__ void unit_table_kernel(const int32_t* __restrict__ offsets, const int
   tab[u] = make_int4(lo, nt, min(block, cnt - mb * block), o0 + mb * block);
 }
 
+// 8 bf16 values -> 8 fp16 values, two per conversion instruction: a bf16 value is
+// the upper half of the fp32 with the same value, and the fp32 pair is rounded to
+// an fp16 pair (exact in fp16's normal range; round to nearest even below it,
+// inf past it, as the scalar conversion).
+__device__ __forceinline__ uint4 bf16x8_to_f16x8_pk(uint4 v) {
+  const uint32_t w[4] = {v.x, v.y, v.z, v.w};
+  uint32_t o[4];
+#pragma unroll
+  for (int i = 0; i < 4; ++i) {
+    const __half2 h = __floats2half2_rn(__uint_as_float(w[i] << 16), __uint_as_float(w[i] & 0xFFFF0000u));
+    o[i] = *reinterpret_cast<const uint32_t*>(&h);
+  }
+  return make_uint4(o[0], o[1], o[2], o[3]);
+}
+
 // bf16 -> fp16, 8 values per thread; values beyond the fp16 range (x, or a
 // LoRA factor) raise TQP_STATUS_NONFINITE (status may be null).
 __global__ void to_f16_kernel(const uint16_t* __restrict__ x, uint16_t* __restrict__ x16, size_t n8,
@@ -709,7 +724,7 @@ __global__ void to_f16_kernel(const uint16_t* __restrict__ x, uint16_t* __restri
   const size_t i = size_t(blockIdx.x) * blockDim.x + threadIdx.x;
   if (i >= n8) return;
   const uint4 v = __ldg(reinterpret_cast<const uint4*>(x) + i);
-  const uint4 o = bf16x8_to_f16x8(v);
+  const uint4 o = bf16x8_to_f16x8_pk(v);
   reinterpret_cast<uint4*>(x16)[i] = o;
   const uint32_t w[4] = {o.x, o.y, o.z, o.w};
   bool bad = false;
@@ -742,7 +757,7 @@ __global__ void __launch_bounds__(256) gather_rows_f16_kernel(const uint16_t* __
     for (int i = 0; i < 8; ++i) {
       const int c = c0 + 32 * i + lane;
       if (c < n16) {
-        const uint4 o = bf16x8_to_f16x8(v[i]);
+        const uint4 o = bf16x8_to_f16x8_pk(v[i]);
         dst[c] = o;
         bad |= f16x2_nonfinite(o.x) | f16x2_nonfinite(o.y) | f16x2_nonfinite(o.z) | f16x2_nonfinite(o.w);
       }
