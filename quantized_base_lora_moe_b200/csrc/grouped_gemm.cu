@@ -702,6 +702,12 @@ __global__ void unit_table_kernel(const int32_t* __restrict__ offsets, const int
   tab[u] = make_int4(lo, nt, min(block, cnt - mb * block), o0 + mb * block);
 }
 
+// 2 bf16 values (one 32-bit word) -> 2 fp16 values in one conversion instruction.
+__device__ __forceinline__ uint32_t bf16x2_to_f16x2_pk(uint32_t w) {
+  const __half2 h = __floats2half2_rn(__uint_as_float(w << 16), __uint_as_float(w & 0xFFFF0000u));
+  return *reinterpret_cast<const uint32_t*>(&h);
+}
+
 // 8 bf16 values -> 8 fp16 values, two per conversion instruction: a bf16 value is
 // the upper half of the fp32 with the same value, and the fp32 pair is rounded to
 // an fp16 pair (exact in fp16's normal range; round to nearest even below it,
@@ -1159,8 +1165,9 @@ __global__ void __launch_bounds__(256) rank_b_kernel(const uint16_t* __restrict_
     const uint32_t wv[4] = {v.x, v.y, v.z, v.w};
 #pragma unroll
     for (int q = 0; q < 4; ++q) {
-      tile[j8 * 8 + 2 * q][kk] = uint16_t(bf16_to_f16_bits(uint16_t(wv[q] & 0xFFFFu)));
-      tile[j8 * 8 + 2 * q + 1][kk] = uint16_t(bf16_to_f16_bits(uint16_t(wv[q] >> 16)));
+      const uint32_t h = bf16x2_to_f16x2_pk(wv[q]);
+      tile[j8 * 8 + 2 * q][kk] = uint16_t(h & 0xFFFFu);
+      tile[j8 * 8 + 2 * q + 1][kk] = uint16_t(h >> 16);
     }
   }
   __syncthreads();
@@ -1201,8 +1208,10 @@ __global__ void __launch_bounds__(256) lora_a_rows_kernel(const uint16_t* __rest
     const int jp = (((j >> 3) + c) % pcs) * 8 + (j & 7);   // rotation of row group c (rows 8c .. 8c + 7)
 #pragma unroll
     for (int q = 0; q < 4; ++q) {
-      tile[c * 8 + 2 * q][jp] = uint16_t(bf16_to_f16_bits_chk(uint16_t(wv[q] & 0xFFFFu), bad));
-      tile[c * 8 + 2 * q + 1][jp] = uint16_t(bf16_to_f16_bits_chk(uint16_t(wv[q] >> 16), bad));
+      const uint32_t h = bf16x2_to_f16x2_pk(wv[q]);
+      bad |= f16x2_nonfinite(h) != 0u;
+      tile[c * 8 + 2 * q][jp] = uint16_t(h & 0xFFFFu);
+      tile[c * 8 + 2 * q + 1][jp] = uint16_t(h >> 16);
     }
   }
   __syncthreads();

@@ -32,17 +32,10 @@ __device__ __forceinline__ uint32_t logit_key(float v) {
   return (b & 0x80000000u) ? (~b) : (b | 0x80000000u);
 }
 
-__device__ __forceinline__ uint32_t warp_max_u32(uint32_t v) {
-#pragma unroll
-  for (int o = 16; o > 0; o >>= 1) v = max(v, __shfl_xor_sync(0xFFFFFFFFu, v, o));
-  return v;
-}
+// (one warp-wide reduction instruction each)
+__device__ __forceinline__ uint32_t warp_max_u32(uint32_t v) { return __reduce_max_sync(0xFFFFFFFFu, v); }
 
-__device__ __forceinline__ uint32_t warp_min_u32(uint32_t v) {
-#pragma unroll
-  for (int o = 16; o > 0; o >>= 1) v = min(v, __shfl_xor_sync(0xFFFFFFFFu, v, o));
-  return v;
-}
+__device__ __forceinline__ uint32_t warp_min_u32(uint32_t v) { return __reduce_min_sync(0xFFFFFFFFu, v); }
 
 // One warp per token. Lane l holds the orderable keys of experts l, l+32, ...
 // Each of the k rounds takes every lane's best key not yet chosen (lowest
@@ -304,7 +297,8 @@ int launch_permute(const int32_t* ids, int T, int E, int k, int32_t* offsets, in
   if (smem1 > 48 * 1024 && !count_attr.test_and_set_device(permute_count_kernel, 64 * 1024)) return TQP_ERR_CUDA;
   permute_count_kernel<<<(W + wpb - 1) / wpb, wpb * 32, smem1, s>>>(ids, T, E, k, count, status);
   // pass 2
-  permute_colscan_kernel<<<(E + 31) / 32, W >= 1024 ? 1024 : ((W + 31) / 32) * 32, 0, s>>>(count, W, E, total);
+  // 32 warps per block whatever W: each warp's serial run over its chunks stays short
+  permute_colscan_kernel<<<(E + 31) / 32, 1024, 0, s>>>(count, W, E, total);
   // pass 3
   const size_t smem3 = size_t(E + 1 + 32) * 4 + size_t(wpb) * E * 4;
   if (smem3 > 48 * 1024 && !scatter_attr.test_and_set_device(permute_scatter_kernel, (4096 + 1 + 32) * 4 + 64 * 1024))
