@@ -297,7 +297,8 @@ int rev_couple_inv(const float* y1, const float* y2, int T, const tqp_moe_weight
  *   does not depend on the magnitude of dy (no fp16 underflow or overflow for
  *   small or large cotangents).
  *   ws: tqp_moe_layer_bwd_workspace_size (the layer's forward workspace plus
- *   G|U, dG|dU, dO, dha, dxa and the rank-space B operand in fp16).
+ *   G|U, dG|dU, dO, dha, dxa, the rank-space B operand and a row copy of the
+ *   adapter A factors in fp16).
  * ------------------------------------------------------------------------- */
 size_t tqp_moe_layer_bwd_workspace_size(int T, const tqp_moe_weights* w);
 int tqp_moe_layer_bwd(const uint16_t* x, const float* dy, int T, const tqp_moe_weights* w, float* dx,
