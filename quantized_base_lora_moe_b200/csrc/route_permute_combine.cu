@@ -43,8 +43,10 @@ __device__ __forceinline__ uint32_t warp_min_u32(uint32_t v) { return __reduce_m
 // id order), the warp maximum of those, and among the lanes that hold it the
 // lowest expert id (one ballot; a min-reduction only when several lanes tie).
 // The winner lane marks its element as chosen.
+// Up to 16 logits per lane (E <= 512) the kernel is held to 32 registers, so that
+// 8 blocks fit an SM and the 1024 blocks of an 8192-token batch run in one wave.
 template <int EPL>  // logits per lane kept in registers (E <= 32 * EPL)
-__global__ void __launch_bounds__(256) route_kernel(const float* __restrict__ logits, int T, int E, int k,
+__global__ void __launch_bounds__(256, EPL <= 16 ? 8 : 1) route_kernel(const float* __restrict__ logits, int T, int E, int k,
                                                     int32_t* __restrict__ ids, float* __restrict__ gates,
                                                     int32_t* status) {
   constexpr int NW = (EPL + 31) / 32;   // exclusion mask words
@@ -312,6 +314,8 @@ int launch_permute(const int32_t* ids, int T, int E, int k, int32_t* offsets, in
 // moe_combine
 // ----------------------------------------------------------------------------
 
+constexpr int kCombMaxK = 32;   // top-k limit of the C ABI
+
 // One block per token row; each thread owns 8 consecutive columns (16 B of bf16).
 __global__ void __launch_bounds__(256) combine_kernel(const uint16_t* __restrict__ out_perm,
                                                       const int32_t* __restrict__ inv,
@@ -319,21 +323,38 @@ __global__ void __launch_bounds__(256) combine_kernel(const uint16_t* __restrict
                                                       const void* __restrict__ residual, int residual_f32,
                                                       float sign, void* __restrict__ y, int y_f32,
                                                       uint16_t* __restrict__ y_bf16) {
+  // the token's slots (row, gate) in shared memory; the rows' pieces are then
+  // loaded four slots at a time so that their latencies overlap (the sum keeps
+  // the fixed j order)
+  __shared__ int32_t row_s[kCombMaxK];
+  __shared__ float g_s[kCombMaxK];
   const int t = blockIdx.x;
+  for (int i = threadIdx.x; i < k; i += blockDim.x) {
+    row_s[i] = __ldg(inv + size_t(t) * k + i);
+    g_s[i] = __ldg(gates + size_t(t) * k + i);
+  }
+  __syncthreads();
   const int c0 = threadIdx.x * 8;
   for (int c = c0; c < d; c += blockDim.x * 8) {
     float acc[8];
 #pragma unroll
     for (int i = 0; i < 8; ++i) acc[i] = 0.0f;
-    for (int j = 0; j < k; ++j) {
-      const int row = __ldg(inv + size_t(t) * k + j);
-      const float gmm = __ldg(gates + size_t(t) * k + j);
-      const uint4 v = __ldg(reinterpret_cast<const uint4*>(out_perm + size_t(row) * d + c));
-      const uint32_t w[4] = {v.x, v.y, v.z, v.w};
+    for (int j0 = 0; j0 < k; j0 += 4) {
+      uint4 ov[4];
 #pragma unroll
-      for (int i = 0; i < 4; ++i) {
-        acc[2 * i] = fmaf(gmm, f16_to_f32(uint16_t(w[i] & 0xFFFFu)), acc[2 * i]);
-        acc[2 * i + 1] = fmaf(gmm, f16_to_f32(uint16_t(w[i] >> 16)), acc[2 * i + 1]);
+      for (int b = 0; b < 4; ++b)
+        ov[b] = (j0 + b < k) ? __ldg(reinterpret_cast<const uint4*>(out_perm + size_t(row_s[j0 + b]) * d + c))
+                             : make_uint4(0, 0, 0, 0);
+#pragma unroll
+      for (int b = 0; b < 4; ++b) {
+        if (j0 + b >= k) break;
+        const float gmm = g_s[j0 + b];
+        const uint32_t w[4] = {ov[b].x, ov[b].y, ov[b].z, ov[b].w};
+#pragma unroll
+        for (int i = 0; i < 4; ++i) {
+          acc[2 * i] = fmaf(gmm, f16_to_f32(uint16_t(w[i] & 0xFFFFu)), acc[2 * i]);
+          acc[2 * i + 1] = fmaf(gmm, f16_to_f32(uint16_t(w[i] >> 16)), acc[2 * i + 1]);
+        }
       }
     }
     float out[8];
