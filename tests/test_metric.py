@@ -19,7 +19,7 @@ def test_excess_error_sees_real_errors():
     assert rel_err_bf16_out(O.round_bf16(bad), y) > 0.09
 
 
-def test_block_flop_counts_match_the_survey_estimates():
+def test_block_flop_counts_match_the_closed_forms():
     # one full-config layer: forward 996 GFLOP (router 15.4, experts 927.7, LoRA 53.2);
     # adapter-only backward: dgrad ~928 + adapter gradients ~106 GFLOP
     import bench
