@@ -129,10 +129,13 @@ __device__ __forceinline__ float inv_grad_scale(const uint32_t* dmax) {
   return ldexpf(1.0f, -max(-120, min(120, 8 - e)));
 }
 
-// tp[kind]: the P matrix of each kind as a box {64 m, 64 rows} map (unused when perm is set)
+// tp[kind]: the P matrix of each kind as a box {64 m, 64 rows} map, tq[kind] the Q
+// matrix as a box {64 columns, 64 rows} map (both unused when perm is set)
 __global__ void __launch_bounds__(kThreads, 1)
     wgrad_kernel(const Args a, const __grid_constant__ CUtensorMap tp0, const __grid_constant__ CUtensorMap tp1,
-                 const __grid_constant__ CUtensorMap tp2, const __grid_constant__ CUtensorMap tp3) {
+                 const __grid_constant__ CUtensorMap tp2, const __grid_constant__ CUtensorMap tp3,
+                 const __grid_constant__ CUtensorMap tq0, const __grid_constant__ CUtensorMap tq1,
+                 const __grid_constant__ CUtensorMap tq2, const __grid_constant__ CUtensorMap tq3) {
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   uint8_t* a_base = smem;
@@ -262,6 +265,10 @@ __global__ void __launch_bounds__(kThreads, 1)
       prefetch_tmap(&tp1);
       prefetch_tmap(&tp2);
       prefetch_tmap(&tp3);
+      prefetch_tmap(&tq0);
+      prefetch_tmap(&tq1);
+      prefetch_tmap(&tq2);
+      prefetch_tmap(&tq3);
     }
     for (int u = blockIdx.x; u < nunits; u += gridDim.x) {
       const WUnit w = decode(a, u);
@@ -286,14 +293,24 @@ __global__ void __launch_bounds__(kThreads, 1)
         const uint32_t as = smem_u32(a_base + size_t(rs.stage) * kABytes);
         const uint32_t bs = smem_u32(b_base + size_t(rs.stage) * kBBytes);
         const int k0 = s * kRowsPerStage;
+        // a stage whose 64 rows all belong to the expert takes Q by TMA as well;
+        // the expert's last, partial stage takes Q by cp.async, zero-filled past
+        // the expert's rows
+        const bool qtma = ptma && k0 + kRowsPerStage <= w.rows;
         if (ptma) {
           // P: two boxes of 64 m x 64 rows (rows past the expert are read, and
           // meet Q's zero rows; rows past the matrix are zero-filled)
           if (tid == 0) {
             const CUtensorMap* map = w.kind == 0 ? &tp0 : w.kind == 1 ? &tp1 : w.kind == 2 ? &tp2 : &tp3;
-            mbar_expect_tx(&ctl->full[rs.stage], uint32_t(2 * 64 * 128));
+            mbar_expect_tx(&ctl->full[rs.stage], uint32_t(2 * 64 * 128 + (qtma ? kBBytes : 0)));
             tma_load_2d(as, map, &ctl->full[rs.stage], pcol, w.base + k0);
             tma_load_2d(as + kAtomCol, map, &ctl->full[rs.stage], pcol + 64, w.base + k0);
+            if (qtma) {
+              // Q: one box of 64 columns x 64 rows (columns past the matrix zero-filled,
+              // columns past the kind's width never read by the MMA)
+              const CUtensorMap* qmap = w.kind == 0 ? &tq0 : w.kind == 1 ? &tq1 : w.kind == 2 ? &tq2 : &tq3;
+              tma_load_2d(bs, qmap, &ctl->full[rs.stage], qcol, w.base + k0);
+            }
             pend.issued(rs.stage, rs.phase);
           }
         } else {
@@ -310,7 +327,7 @@ __global__ void __launch_bounds__(kThreads, 1)
           }
         }
         // Q: 64 rows x nchunk chunks
-        for (int c = tid; c < kRowsPerStage * nchunk; c += 128) {
+        for (int c = tid; !qtma && c < kRowsPerStage * nchunk; c += 128) {
           const int kk = c / nchunk, ch = c - kk * nchunk;
           const bool in = k0 + kk < w.rows && ch < nreal;
           const uint16_t* src = Qs + size_t(in ? w.base + k0 + kk : 0) * ldq + qcol + (in ? ch * 8 : 0);
@@ -373,19 +390,23 @@ int launch_wgrad(const tqp_moe_weights* w, size_t A, const int32_t* offsets, con
   a.wait_ns = wait_limit_ns();
   static DeviceFlags attr_done;
   if (!attr_done.test_and_set_device(wgrad::wgrad_kernel, int(wgrad::kSmemBytes))) return TQP_ERR_CUDA;
-  CUtensorMap tp[4];
+  CUtensorMap tp[4], tq[4];
   std::memset(tp, 0, sizeof(tp));
+  std::memset(tq, 0, sizeof(tq));
   if (!perm) {
-    // the P matrices are expert-sorted rows [A][width]
+    // the P and Q matrices are expert-sorted rows [A][width]
     const uint64_t rows = uint64_t(A);
     if (!make_tile_map(&tp[0], dO, rows, uint64_t(w->d), 64) || !make_tile_map(&tp[1], h, rows, uint64_t(w->ffn), 64) ||
         !make_tile_map(&tp[2], dgu, rows, uint64_t(2 * w->ffn), 64) ||
-        !make_tile_map(&tp[3], x16, rows, uint64_t(w->d), 64))
+        !make_tile_map(&tp[3], x16, rows, uint64_t(w->d), 64) ||
+        !make_tile_map(&tq[0], ha, rows, uint64_t(r), 64) || !make_tile_map(&tq[1], dha, rows, uint64_t(r), 64) ||
+        !make_tile_map(&tq[2], xa, rows, uint64_t(2 * r), 64) || !make_tile_map(&tq[3], dxa, rows, uint64_t(2 * r), 64))
       return TQP_ERR_CUDA;
   }
   const int units = a.E * a.tile_prefix[4];
   const int grid = units < num_sms() ? units : num_sms();
-  wgrad::wgrad_kernel<<<grid, wgrad::kThreads, wgrad::kSmemBytes, s>>>(a, tp[0], tp[1], tp[2], tp[3]);
+  wgrad::wgrad_kernel<<<grid, wgrad::kThreads, wgrad::kSmemBytes, s>>>(a, tp[0], tp[1], tp[2], tp[3], tq[0], tq[1],
+                                                                        tq[2], tq[3]);
   return cudaGetLastError() == cudaSuccess ? TQP_OK : TQP_ERR_CUDA;
 }
 
