@@ -253,6 +253,7 @@ def time_rev_block(L_F, cfgF: synth.LayerConfig, dev, steps: int, warmup: int, f
     f = lambda t: t.view(torch.bfloat16).float()
     rms = torch.sqrt(torch.mean(torch.cat([f(x1), f(x2)]) ** 2))
     err = float(max((f(r1) - f(x1)).abs().max(), (f(r2) - f(x2)).abs().max()) / rms)
+    exact = exact_on_stream_grid(r1, x1) and exact_on_stream_grid(r2, x2)
     mean = {n: statistics.mean(v) for n, v in ms.items()}
     step_ms = mean["fwd"] + mean["adapter_bwd"]
     # forward: F and G; adapter backward: the inverse (F and G again) and both layers' backward
@@ -264,7 +265,16 @@ def time_rev_block(L_F, cfgF: synth.LayerConfig, dev, steps: int, warmup: int, f
             "ms_per_step": step_ms, "tokens_per_s": T / (step_ms * 1e-3), "ms": mean, "steps": steps,
             "flop_per_step": step_flop, "tflops": tflops,
             "roofline_frac_measured": tflops / pk["bf16_tflops"], "roofline_frac_nominal": tflops / 2250.0,
-            "reconstruction_max_err_rel_rms": err, "l2": "flushed before every call"}
+            "reconstruction_max_err_rel_rms": err, "reconstruction_exact_on_stream_grid": exact,
+            "l2": "flushed before every call"}
+
+
+def exact_on_stream_grid(r, x) -> bool:
+    """Whether the reconstructed bf16 r is x put on the coupling's stream grid
+    (multiples of 2^-16, half to even) bit for bit."""
+    import torch
+    f = lambda t: t.view(torch.bfloat16).double()
+    return bool(torch.equal(f(r), torch.round(f(x) * 65536.0) / 65536.0))
 
 
 def time_stack(dev, flush, depths=(1, 2, 4, 8)) -> dict:
@@ -302,7 +312,7 @@ def time_stack(dev, flush, depths=(1, 2, 4, 8)) -> dict:
     lib = Q.lib()
     per_layer_bwd_ws = max(lib.tqp_moe_layer_bwd_workspace_size(T, F.ref()), lib.tqp_moe_layer_bwd_workspace_size(T, G.ref()))
     out = {"workload": "L blocks of two full-size layers (460 experts, top-12, T=8192, d=2048; base weights and "
-                       "LoRA B x 1/2), fp32 streams between blocks", "depths": {}}
+                       "LoRA B x 1/2), fp32 streams on the 2^-16 grid between blocks", "depths": {}}
     bf = lambda t: t.view(torch.bfloat16).float()
     rms = float(torch.sqrt(torch.mean(torch.cat([bf(x1), bf(x2)]) ** 2)))
     for L in depths:
@@ -329,11 +339,13 @@ def time_stack(dev, flush, depths=(1, 2, 4, 8)) -> dict:
         if st.read() != 0:
             raise RuntimeError(f"device status {st.read()} in the reversible stack (L={L})")
         err = float(max((bf(r1) - bf(x1)).abs().max(), (bf(r2) - bf(x2)).abs().max())) / rms
+        exact = exact_on_stream_grid(r1, x1) and exact_on_stream_grid(r2, x2)
         store_all = L * (2 * T * d * 4 + 2 * per_layer_bwd_ws)
         out["depths"][str(L)] = {"fwd_ms": ms["fwd"][0], "bwd_ms": ms["bwd"][0],
                                  "workspace_bytes": ws.numel(), "peak_activation_bytes": peak,
                                  "store_all_estimate_bytes": store_all,
-                                 "reconstruction_max_err_rel_rms": err}
+                                 "reconstruction_max_err_rel_rms": err,
+                                 "reconstruction_exact_on_stream_grid": exact}
         del stack, gF, gG, arrays, ws
         torch.cuda.empty_cache()
     return out

@@ -41,7 +41,9 @@
  *       TQP_STATUS_RANGE      a nonzero group scale outside [2^-17, 8192): the
  *                             products q * scale are then not all exact in fp16
  *                             (the expert contractions run on exact fp16 weights
- *                             otherwise).
+ *                             otherwise); or, in the coupling and stack calls, a
+ *                             stream value of magnitude 256 or more (or not
+ *                             finite): the stream adds are then no longer exact.
  *     Nothing traps, prints or exits.
  *   - Every pointer argument is caller-owned DEVICE memory (unless stated),
  *     16-byte aligned, dense row-major. The library never allocates device
@@ -270,6 +272,13 @@ int tqp_moe_layer_fwd(const uint16_t* x, int T, const tqp_moe_weights* w, uint16
  *     x1, x2 [T][d] bf16 in; y1, y2 [T][d] fp32 out.
  *   rev_couple_inv: x2 = y2 - G(bf16(y1)); x1 = y1 - F(x2), rounded to bf16.
  *     y1, y2 fp32 in; x1, x2 bf16 out. Routing is recomputed (stateless).
+ *   Stream format: the streams are fp32 multiples of 2^-16 below 256 in
+ *   magnitude ("the grid"). x1, x2 and each layer's bf16 branch output are
+ *   rounded to the grid (half to even) before the add; F reads x2 on the
+ *   grid. On the grid every add and subtract is exact in fp32, and the layers
+ *   are deterministic, so rev_couple_inv returns x1, x2 on the grid bit for
+ *   bit: x itself wherever |x| >= 2^-9, else x moved by at most 2^-17. A
+ *   stream value leaving the range raises TQP_STATUS_RANGE.
  *   F and G must share d. ws: rev_couple_workspace_size (both calls).
  * ------------------------------------------------------------------------- */
 size_t rev_couple_workspace_size(int T, const tqp_moe_weights* F, const tqp_moe_weights* G);
@@ -332,8 +341,9 @@ int tqp_adapter_bwd(const float* y1, const float* y2, const float* dy1, const fl
  * Block l maps streams (a1, a2) to
  *   b1 = a1 + F_l(bf16(a2)),   b2 = a2 + G_l(bf16(b1)).
  * Block 0's inputs are x1, x2 (bf16); the streams between blocks are carried
- * in fp32 (each layer reads the bf16 rounding of its stream); the outputs of
- * block L-1 are y1, y2 (fp32). With L = 1 this is rev_couple_fwd exactly.
+ * in fp32 on the coupling's grid (each layer reads the bf16 rounding of its
+ * stream), so the inverse is exact at any depth; the outputs of block L-1 are
+ * y1, y2 (fp32). With L = 1 this is rev_couple_fwd exactly.
  *   F, G: arrays of L weight sets (all with the same d).
  *   rev_stack_fwd: x1, x2 [T][d] bf16 -> y1, y2 [T][d] fp32.
  *   rev_stack_inv: y1, y2 -> x1, x2 (bf16), walking the blocks from L-1 down

@@ -317,12 +317,17 @@ int launch_permute(const int32_t* ids, int T, int E, int k, int32_t* offsets, in
 constexpr int kCombMaxK = 32;   // top-k limit of the C ABI
 
 // One block per token row; each thread owns 8 consecutive columns (16 B of bf16).
+// grid (with a residual): the coupling's stream format. The residual and the
+// branch m are rounded to multiples of 2^-kStreamGridBits, so that
+// residual +- m is exact in fp32 while |y| < kStreamMax (24-bit significand);
+// a y outside that range raises TQP_STATUS_RANGE.
 __global__ void __launch_bounds__(256) combine_kernel(const uint16_t* __restrict__ out_perm,
                                                       const int32_t* __restrict__ inv,
                                                       const float* __restrict__ gates, int T, int k, int d,
                                                       const void* __restrict__ residual, int residual_f32,
                                                       float sign, void* __restrict__ y, int y_f32,
-                                                      uint16_t* __restrict__ y_bf16) {
+                                                      uint16_t* __restrict__ y_bf16, int grid,
+                                                      int32_t* __restrict__ status) {
   // the token's slots (row, gate) in shared memory; the rows' pieces are then
   // loaded four slots at a time so that their latencies overlap (the sum keeps
   // the fixed j order)
@@ -376,8 +381,18 @@ __global__ void __launch_bounds__(256) combine_kernel(const uint16_t* __restrict
           res[2 * i + 1] = __uint_as_float(w[i] & 0xFFFF0000u);
         }
       }
+      if (grid) {
+        bool in_range = true;
 #pragma unroll
-      for (int i = 0; i < 8; ++i) out[i] = res[i] + sign * out[i];
+        for (int i = 0; i < 8; ++i) {
+          out[i] = to_stream_grid(res[i]) + sign * to_stream_grid(out[i]);
+          in_range &= fabsf(out[i]) < kStreamMax;
+        }
+        if (!in_range && status) atomicOr(status, TQP_STATUS_RANGE);
+      } else {
+#pragma unroll
+        for (int i = 0; i < 8; ++i) out[i] = res[i] + sign * out[i];
+      }
     }
     uint4 ob;
     ob.x = pack_bf16x2(out[0], out[1]);
@@ -397,11 +412,11 @@ __global__ void __launch_bounds__(256) combine_kernel(const uint16_t* __restrict
 
 int launch_combine(const uint16_t* out_perm, const int32_t* inv, const float* gates, int T, int k, int d,
                    const void* residual, int residual_f32, float sign, void* y, int y_f32, uint16_t* y_bf16,
-                   cudaStream_t s) {
+                   cudaStream_t s, bool grid, int32_t* status) {
   if (T == 0) return TQP_OK;
   const int threads = d / 8 < 256 ? d / 8 : 256;
   combine_kernel<<<T, threads, 0, s>>>(out_perm, inv, gates, T, k, d, residual, residual_f32, sign, y, y_f32,
-                                       y_bf16);
+                                       y_bf16, grid ? 1 : 0, status);
   return cudaGetLastError() == cudaSuccess ? TQP_OK : TQP_ERR_CUDA;
 }
 

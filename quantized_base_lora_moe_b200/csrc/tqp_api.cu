@@ -223,13 +223,40 @@ int layer_backward(const uint16_t* x, const float* dy, int T, const tqp_moe_weig
   return launch_gather_add(dX, L.inv, T, k, d, B.dmax, dx, s);
 }
 
+// grid: the residual add is the coupling's, on the stream grid (exact adds)
 int layer_forward(const uint16_t* x, int T, const tqp_moe_weights* w, const void* residual, int res_f32,
                   float sign, void* y, int y_f32, uint16_t* y_bf16, void* ws, int32_t* status, cudaStream_t s,
-                  uint16_t* aux_gu = nullptr) {
+                  uint16_t* aux_gu = nullptr, bool grid = false) {
   const LayerWs L = carve_layer_ws(ws, T, w);
   int rc = layer_experts(x, T, w, L, status, s, aux_gu);
   if (rc != TQP_OK) return rc;
-  return launch_combine(L.out_perm, L.inv, L.gates, T, w->top_k, w->d, residual, res_f32, sign, y, y_f32, y_bf16, s);
+  return launch_combine(L.out_perm, L.inv, L.gates, T, w->top_k, w->d, residual, res_f32, sign, y, y_f32, y_bf16, s,
+                        grid, status);
+}
+
+// bf16(x) of a bf16 stream input put on the coupling's stream grid: the input
+// a coupling's first layer reads, so that its inverse, which can only return
+// the grid value, feeds that layer the same bits
+__global__ void stream_grid_bf16_kernel(const uint16_t* __restrict__ in, uint16_t* __restrict__ out, size_t n) {
+  const size_t i = (size_t(blockIdx.x) * blockDim.x + threadIdx.x) * 8;
+  if (i + 7 < n) {
+    const uint4 v = *reinterpret_cast<const uint4*>(in + i);
+    const uint32_t w[4] = {v.x, v.y, v.z, v.w};
+    uint32_t o[4];
+#pragma unroll
+    for (int q = 0; q < 4; ++q)
+      o[q] = pack_bf16x2(to_stream_grid(__uint_as_float(w[q] << 16)), to_stream_grid(__uint_as_float(w[q] & 0xFFFF0000u)));
+    *reinterpret_cast<uint4*>(out + i) = make_uint4(o[0], o[1], o[2], o[3]);
+  } else {
+    for (size_t j = i; j < n; ++j) out[j] = f32_to_bf16(to_stream_grid(bf16_to_f32(in[j])));
+  }
+}
+
+int to_stream_grid_bf16(const uint16_t* in, uint16_t* out, size_t n, cudaStream_t s) {
+  if (n == 0) return TQP_OK;
+  const size_t threads = (n + 7) / 8;
+  stream_grid_bf16_kernel<<<unsigned((threads + 255) / 256), 256, 0, s>>>(in, out, n);
+  return cudaGetLastError() == cudaSuccess ? TQP_OK : TQP_ERR_CUDA;
 }
 
 __global__ void f32_to_bf16_kernel(const float* __restrict__ in, uint16_t* __restrict__ out, size_t n) {
@@ -328,11 +355,11 @@ int block_backward_f32(const float* y1, const float* y2, const float* dy1, const
   int rc;
   if ((rc = to_bf16(y1, w.zb, Td, s)) != TQP_OK) return rc;
   uint16_t* gu = carve_bwd(static_cast<char*>(w.lws) + layer_ws_size(T, G), T, G).gu;
-  if ((rc = layer_forward(w.zb, T, G, y2, 1, -1.0f, a2, 1, w.ab, w.lws, status, s, gu)) != TQP_OK) return rc;
+  if ((rc = layer_forward(w.zb, T, G, y2, 1, -1.0f, a2, 1, w.ab, w.lws, status, s, gu, true)) != TQP_OK) return rc;
   // da1 = dy1 + J_G^T dy2, the sum taken inside G's backward
   if ((rc = layer_backward(w.zb, dy2, T, G, da1, gG, w.lws, status, s, false, dy1)) != TQP_OK) return rc;
   gu = carve_bwd(static_cast<char*>(w.lws) + layer_ws_size(T, F), T, F).gu;
-  if ((rc = layer_forward(w.ab, T, F, y1, 1, -1.0f, a1, 1, nullptr, w.lws, status, s, gu)) != TQP_OK) return rc;
+  if ((rc = layer_forward(w.ab, T, F, y1, 1, -1.0f, a1, 1, nullptr, w.lws, status, s, gu, true)) != TQP_OK) return rc;
   // da2 = dy2 + J_F^T da1
   return layer_backward(w.ab, da1, T, F, da2, gF, w.lws, status, s, false, dy2);
 }
@@ -456,7 +483,7 @@ int tqp_moe_layer_fwd(const uint16_t* x, int T, const tqp_moe_weights* w, uint16
 size_t rev_couple_workspace_size(int T, const tqp_moe_weights* F, const tqp_moe_weights* G) {
   if (check_weights(F) != TQP_OK || check_weights(G) != TQP_OK || T < 0 || F->d != G->d) return 0;
   const size_t a = layer_ws_size(T, F), b = layer_ws_size(T, G);
-  return (a > b ? a : b) + align_up(size_t(T) * F->d * 2, 256) + 256;
+  return (a > b ? a : b) + 2 * align_up(size_t(T) * F->d * 2, 256) + 256;
 }
 
 int rev_couple_fwd(const uint16_t* x1, const uint16_t* x2, int T, const tqp_moe_weights* F, const tqp_moe_weights* G,
@@ -471,12 +498,16 @@ int rev_couple_fwd(const uint16_t* x1, const uint16_t* x2, int T, const tqp_moe_
   if (ws_bytes < rev_couple_workspace_size(T, F, G)) return TQP_ERR_WORKSPACE;
   cudaStream_t s = static_cast<cudaStream_t>(stream);
   char* base = reinterpret_cast<char*>(align_up(reinterpret_cast<uintptr_t>(ws), 256));
+  const size_t Td = size_t(T) * F->d;
   uint16_t* y1b = reinterpret_cast<uint16_t*>(base);
-  void* lws = base + align_up(size_t(T) * F->d * 2, 256);
+  uint16_t* x2g = reinterpret_cast<uint16_t*>(base + align_up(Td * 2, 256));
+  void* lws = base + 2 * align_up(Td * 2, 256);
+  // the streams on the stream grid: F reads x2 on the grid, the value its inverse returns
+  if ((rc = to_stream_grid_bf16(x2, x2g, Td, s)) != TQP_OK) return rc;
   // y1 = x1 + F(x2) (fp32), plus its bf16 copy as G's input
-  if ((rc = layer_forward(x2, T, F, x1, 0, 1.0f, y1, 1, y1b, lws, dev_status, s)) != TQP_OK) return rc;
+  if ((rc = layer_forward(x2g, T, F, x1, 0, 1.0f, y1, 1, y1b, lws, dev_status, s, nullptr, true)) != TQP_OK) return rc;
   // y2 = x2 + G(bf16(y1))
-  return layer_forward(y1b, T, G, x2, 0, 1.0f, y2, 1, nullptr, lws, dev_status, s);
+  return layer_forward(y1b, T, G, x2, 0, 1.0f, y2, 1, nullptr, lws, dev_status, s, nullptr, true);
 }
 
 int rev_couple_inv(const float* y1, const float* y2, int T, const tqp_moe_weights* F, const tqp_moe_weights* G,
@@ -492,12 +523,13 @@ int rev_couple_inv(const float* y1, const float* y2, int T, const tqp_moe_weight
   cudaStream_t s = static_cast<cudaStream_t>(stream);
   char* base = reinterpret_cast<char*>(align_up(reinterpret_cast<uintptr_t>(ws), 256));
   uint16_t* y1b = reinterpret_cast<uint16_t*>(base);
-  void* lws = base + align_up(size_t(T) * F->d * 2, 256);
+  void* lws = base + 2 * align_up(size_t(T) * F->d * 2, 256);
   if ((rc = to_bf16(y1, y1b, size_t(T) * F->d, s)) != TQP_OK) return rc;
-  // x2 = y2 - G(bf16(y1)), rounded to bf16
-  if ((rc = layer_forward(y1b, T, G, y2, 1, -1.0f, x2, 0, nullptr, lws, dev_status, s)) != TQP_OK) return rc;
+  // x2 = y2 - G(bf16(y1)), exact on the stream grid, then rounded to bf16 (a no-op there)
+  if ((rc = layer_forward(y1b, T, G, y2, 1, -1.0f, x2, 0, nullptr, lws, dev_status, s, nullptr, true)) != TQP_OK)
+    return rc;
   // x1 = y1 - F(x2)
-  return layer_forward(x2, T, F, y1, 1, -1.0f, x1, 0, nullptr, lws, dev_status, s);
+  return layer_forward(x2, T, F, y1, 1, -1.0f, x1, 0, nullptr, lws, dev_status, s, nullptr, true);
 }
 
 size_t tqp_moe_layer_bwd_workspace_size(int T, const tqp_moe_weights* w) {
@@ -551,12 +583,12 @@ int tqp_adapter_bwd(const float* y1, const float* y2, const float* dy1, const fl
   // G-step: reconstruct x2 = y2 - G(bf16(y1)); G's grads for cotangent dy2
   if ((rc = to_bf16(y1, zb, Td, s)) != TQP_OK) return rc;
   uint16_t* gu = carve_bwd(static_cast<char*>(lws) + layer_ws_size(T, G), T, G).gu;
-  if ((rc = layer_forward(zb, T, G, y2, 1, -1.0f, x2, 0, nullptr, lws, dev_status, s, gu)) != TQP_OK) return rc;
+  if ((rc = layer_forward(zb, T, G, y2, 1, -1.0f, x2, 0, nullptr, lws, dev_status, s, gu, true)) != TQP_OK) return rc;
   // dz1 = dy1 + J_G^T dy2 -> dx1 (dx1 = dz1), the sum taken inside G's backward
   if ((rc = layer_backward(zb, dy2, T, G, dx1, gG, lws, dev_status, s, false, dy1)) != TQP_OK) return rc;
   // F-step: x1 = y1 - F(x2); F's grads for cotangent dz1; dx2 = dy2 + J_F^T dz1
   gu = carve_bwd(static_cast<char*>(lws) + layer_ws_size(T, F), T, F).gu;
-  if ((rc = layer_forward(x2, T, F, y1, 1, -1.0f, x1, 0, nullptr, lws, dev_status, s, gu)) != TQP_OK) return rc;
+  if ((rc = layer_forward(x2, T, F, y1, 1, -1.0f, x1, 0, nullptr, lws, dev_status, s, gu, true)) != TQP_OK) return rc;
   return layer_backward(x2, dx1, T, F, dx2, gF, lws, dev_status, s, false, dy2);
 }
 
@@ -582,16 +614,23 @@ int rev_stack_fwd(const uint16_t* x1, const uint16_t* x2, int T, int L, const tq
     float* b1 = (l == L - 1) ? y1 : w.s[l & 1][0];
     float* b2 = (l == L - 1) ? y2 : w.s[l & 1][1];
     if (l == 0) {
-      // b1 = x1 + F(x2), with bf16(b1) for G; b2 = x2 + G(bf16(b1))
-      if ((rc = layer_forward(x2, T, F[0], x1, 0, 1.0f, b1, 1, w.zb, w.lws, dev_status, s)) != TQP_OK) return rc;
-      if ((rc = layer_forward(w.zb, T, G[0], x2, 0, 1.0f, b2, 1, nullptr, w.lws, dev_status, s)) != TQP_OK)
+      // b1 = x1 + F(x2), with bf16(b1) for G; b2 = x2 + G(bf16(b1)) (x1, x2 and F's
+      // input put on the stream grid)
+      if ((rc = to_stream_grid_bf16(x2, w.ab, Td, s)) != TQP_OK) return rc;
+      if ((rc = layer_forward(w.ab, T, F[0], x1, 0, 1.0f, b1, 1, w.zb, w.lws, dev_status, s, nullptr, true)) != TQP_OK)
+        return rc;
+      if ((rc = layer_forward(w.zb, T, G[0], x2, 0, 1.0f, b2, 1, nullptr, w.lws, dev_status, s, nullptr, true)) !=
+          TQP_OK)
         return rc;
     } else {
       const float* a1 = w.s[(l - 1) & 1][0];
       const float* a2 = w.s[(l - 1) & 1][1];
       if ((rc = to_bf16(a2, w.ab, Td, s)) != TQP_OK) return rc;
-      if ((rc = layer_forward(w.ab, T, F[l], a1, 1, 1.0f, b1, 1, w.zb, w.lws, dev_status, s)) != TQP_OK) return rc;
-      if ((rc = layer_forward(w.zb, T, G[l], a2, 1, 1.0f, b2, 1, nullptr, w.lws, dev_status, s)) != TQP_OK)
+      if ((rc = layer_forward(w.ab, T, F[l], a1, 1, 1.0f, b1, 1, w.zb, w.lws, dev_status, s, nullptr, true)) !=
+          TQP_OK)
+        return rc;
+      if ((rc = layer_forward(w.zb, T, G[l], a2, 1, 1.0f, b2, 1, nullptr, w.lws, dev_status, s, nullptr, true)) !=
+          TQP_OK)
         return rc;
     }
   }
@@ -617,14 +656,18 @@ int rev_stack_inv(const float* y1, const float* y2, int T, int L, const tqp_moe_
     if ((rc = to_bf16(c1, w.zb, Td, s)) != TQP_OK) return rc;
     if (l == 0) {
       // the block inputs are bf16: x2 = y2 - G(bf16(y1)), x1 = y1 - F(x2)
-      if ((rc = layer_forward(w.zb, T, G[0], c2, 1, -1.0f, x2, 0, nullptr, w.lws, dev_status, s)) != TQP_OK)
+      if ((rc = layer_forward(w.zb, T, G[0], c2, 1, -1.0f, x2, 0, nullptr, w.lws, dev_status, s, nullptr, true)) !=
+          TQP_OK)
         return rc;
-      return layer_forward(x2, T, F[0], c1, 1, -1.0f, x1, 0, nullptr, w.lws, dev_status, s);
+      return layer_forward(x2, T, F[0], c1, 1, -1.0f, x1, 0, nullptr, w.lws, dev_status, s, nullptr, true);
     }
     float* a1 = w.s[l & 1][0];
     float* a2 = w.s[l & 1][1];
-    if ((rc = layer_forward(w.zb, T, G[l], c2, 1, -1.0f, a2, 1, w.ab, w.lws, dev_status, s)) != TQP_OK) return rc;
-    if ((rc = layer_forward(w.ab, T, F[l], c1, 1, -1.0f, a1, 1, nullptr, w.lws, dev_status, s)) != TQP_OK) return rc;
+    if ((rc = layer_forward(w.zb, T, G[l], c2, 1, -1.0f, a2, 1, w.ab, w.lws, dev_status, s, nullptr, true)) != TQP_OK)
+      return rc;
+    if ((rc = layer_forward(w.ab, T, F[l], c1, 1, -1.0f, a1, 1, nullptr, w.lws, dev_status, s, nullptr, true)) !=
+        TQP_OK)
+      return rc;
     c1 = a1;
     c2 = a2;
   }

@@ -512,6 +512,21 @@ __device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi) {
 }
 
 // ----------------------------------------------------------------------------
+// stream format of the additive coupling
+// ----------------------------------------------------------------------------
+// The coupling's streams are fp32 multiples of 2^-kStreamGridBits of magnitude
+// below kStreamMax. Such a value has at most 24 significant bits, so the sum or
+// difference of two of them is exact in fp32 while it stays below kStreamMax:
+// the inverse's subtraction then returns the forward's input bit for bit, at
+// any depth. Every bf16 value of magnitude 2^-9 or more lies on the grid; a
+// smaller one moves by at most 2^-17 and stays a bf16 value.
+constexpr int kStreamGridBits = 16;
+constexpr float kStreamScale = float(1 << kStreamGridBits);
+constexpr float kStreamMax = float(1 << (24 - kStreamGridBits));
+
+__device__ __forceinline__ float to_stream_grid(float v) { return rintf(v * kStreamScale) * (1.0f / kStreamScale); }
+
+// ----------------------------------------------------------------------------
 // fp16 (operand type of the expert contractions)
 // ----------------------------------------------------------------------------
 

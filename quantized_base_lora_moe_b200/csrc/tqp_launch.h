@@ -42,9 +42,11 @@ int launch_route(const float* logits, int T, int E, int k, int32_t* ids, float* 
 size_t permute_ws_bytes(int T, int E);
 int launch_permute(const int32_t* ids, int T, int E, int k, int32_t* offsets, int32_t* perm_token, int32_t* inv,
                    void* ws, int32_t* status, cudaStream_t s);
+// grid: round the residual and the branch to the coupling's stream grid (exact
+// adds; a result of magnitude >= 256 raises TQP_STATUS_RANGE into status)
 int launch_combine(const uint16_t* out_perm, const int32_t* inv, const float* gates, int T, int k, int d,
                    const void* residual, int residual_f32, float sign, void* y, int y_f32, uint16_t* y_bf16,
-                   cudaStream_t s);
+                   cudaStream_t s, bool grid = false, int32_t* status = nullptr);
 
 // grouped tensor-core GEMMs
 size_t router_ws_bytes(int T, const tqp_moe_weights* w);

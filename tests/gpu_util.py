@@ -28,6 +28,13 @@ def dev(a: np.ndarray, dtype=None) -> torch.Tensor:
     return (t.to(dtype) if dtype is not None else t).cuda()
 
 
+def stream_grid(x: np.ndarray) -> np.ndarray:
+    """x rounded to the coupling's stream grid, multiples of 2^-16 (half to
+    even): what the coupling's inverse returns for a bf16 input x. Every bf16
+    value of magnitude 2^-9 or more is unchanged."""
+    return np.rint(np.asarray(x, np.float64) * 65536.0) / 65536.0
+
+
 def rel_err(got, ref) -> float:
     got = np.asarray(got, np.float64)
     ref = np.asarray(ref, np.float64)

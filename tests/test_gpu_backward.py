@@ -20,7 +20,7 @@ import torch
 
 import synth
 from oracle import tqp_oracle as O
-from tests.gpu_util import dev, dev_bf16, host_bf16, near_tie_tokens, rel_err
+from tests.gpu_util import dev, dev_bf16, host_bf16, near_tie_tokens, rel_err, stream_grid
 
 pytestmark = pytest.mark.gpu
 
@@ -145,9 +145,11 @@ def test_adapter_bwd_block_matches_oracle(cfgs):
     dy1, dy2 = synth.make_grad(T, d, 4, "dy1"), synth.make_grad(T, d, 4, "dy2")
     got = gpu_block(cfgF, cfgG, rawF, rawG, x1b, x2b, dy1, dy2)
     x1, x2 = O.bf16_to_f64(x1b), O.bf16_to_f64(x2b)
-    # reconstruction is exact: the backward recomputes bit-identical F and G
+    # reconstruction is exact: the backward recomputes bit-identical F and G, and
+    # the stream adds are exact on the stream grid
     rms = np.sqrt(np.mean(np.concatenate([x1, x2]) ** 2))
     assert max(np.max(np.abs(got["x1"] - x1)), np.max(np.abs(got["x2"] - x2))) / rms <= 5e-3
+    assert np.array_equal(got["x1"], stream_grid(x1)) and np.array_equal(got["x2"], stream_grid(x2))
     LF, LG = O.Layer(rawF), O.Layer(rawG)
     z = g_input(got["y1"])
     dy1_, dy2_ = dy1.astype(np.float64), dy2.astype(np.float64)
@@ -209,6 +211,7 @@ def test_adapter_bwd_full_size_reconstruction_and_sampled_tokens():
     x1, x2 = O.bf16_to_f64(x1b), O.bf16_to_f64(x2b)
     rms = np.sqrt(np.mean(np.concatenate([x1, x2]) ** 2))
     assert max(np.max(np.abs(got["x1"] - x1)), np.max(np.abs(got["x2"] - x2))) / rms <= 5e-3
+    assert np.array_equal(got["x1"], stream_grid(x1)) and np.array_equal(got["x2"], stream_grid(x2))
     assert all(np.isfinite(got[k]).all() for k in ("dx1", "dx2"))
     LF, LG = O.Layer(rawF), O.Layer(rawG)
     toks = [0, T - 1, 1234, 4321, 777, 6000, 100, 8000]

@@ -18,7 +18,8 @@ import torch
 
 import synth
 from oracle import tqp_oracle as O
-from tests.gpu_util import dev, dev_bf16, dev_f16, host_bf16, host_f16, near_tie_tokens, rel_err, rel_err_bf16_out
+from tests.gpu_util import (dev, dev_bf16, dev_f16, host_bf16, host_f16, near_tie_tokens, rel_err, rel_err_bf16_out,
+                            stream_grid)
 
 pytestmark = pytest.mark.gpu
 
@@ -481,3 +482,27 @@ def test_rev_couple_full_size_reconstruction():
     rms = torch.sqrt(torch.mean(torch.cat([f(x1), f(x2)]) ** 2))
     err = max((f(r1) - f(x1)).abs().max(), (f(r2) - f(x2)).abs().max()) / rms
     assert float(err) <= 5e-3
+    # exact: the inverse returns the inputs on the stream grid bit for bit
+    for r, x in ((r1, x1), (r2, x2)):
+        assert np.array_equal(host_bf16(r), stream_grid(host_bf16(x)))
+
+
+def test_rev_couple_stream_out_of_range_raises_range_status():
+    """A stream value of magnitude 256 or more leaves the grid's exact range:
+    the coupling raises TQP_STATUS_RANGE (and nothing else)."""
+    cfgF, cfgG = REV_SMALL
+    F, G = device_layer(cfgF, cfgF.seed), device_layer(cfgG, cfgG.seed)
+    T, d = cfgF.T, cfgF.d
+    x1b = synth.make_tokens(T, d, 2).copy()
+    x1b[5, 7] = np.float32(300.0).view(np.uint32) >> 16        # bf16 300, exact
+    x2b = synth.make_tokens(T, d, 3)
+    y1 = torch.empty(T, d, dtype=torch.float32, device="cuda")
+    y2 = torch.empty_like(y1)
+    st = Q.Status()
+    Q.rev_couple_fwd(dev_bf16(x1b), dev_bf16(x2b), F, G, y1, y2, status=st)
+    torch.cuda.synchronize()
+    assert st.read() == Q.STATUS_RANGE
+    st = Q.Status()
+    Q.rev_couple_fwd(dev_bf16(synth.make_tokens(T, d, 2)), dev_bf16(x2b), F, G, y1, y2, status=st)
+    torch.cuda.synchronize()
+    assert st.read() == 0
