@@ -16,7 +16,7 @@ Scaling"):
   Abstract, "Single-node economics").
 * 460 routed experts with top-12 routing ("Architecture Details"; Abstract).
 * routing is stateless, so it is recomputed from the inputs during the inverse
-  ("Reversibility Implementation": "MoE routing: Stateless routing decisions").
+  (the routing item of "Reversibility Implementation").
 * reversible residual (RevNet-style) blocks whose inverse uses subtraction, and
   the backward pass reconstructs activations from the final state instead of
   storing them ("Principle 1: Reversible Recurrence Stack"; "Pattern 1";
@@ -151,8 +151,8 @@ class Layer:
 def router_logits(x, L: Layer) -> np.ndarray:
     """Full-precision router: l[t, e] = sum_i x[t, i] * W_r[e, i] (+ bias[e]).
 
-    "Router: Full precision (critical for routing quality)" (TQP Quantization
-    list). The additive bias is the skewed-load workload's per-expert
+    The pages keep the router at full precision because routing quality
+    depends on it (the router item of the TQP Quantization list). The additive bias is the skewed-load workload's per-expert
     popularity term, added before both top-k and the gates.
     """
     l = np.asarray(x, dtype=np.float64) @ L.router_w.T
@@ -345,8 +345,9 @@ def expert_backward(X, dO, P: dict, s: float, fwd: dict) -> dict:
     """Closed-form gradients of one expert for upstream dO (rows of X).
 
     Returns dX and the adapter gradients in storage layout: dA^T [r][in],
-    dB^T [out][r] for gate, up, down. Base weights get no gradient (frozen,
-    "Base expert weights: Quantized (fixed)").
+    dB^T [out][r] for gate, up, down. Base weights get no gradient: they stay
+    frozen in their quantised form (the base-weight item of the TQP
+    Quantization list).
     """
     h, gate, up = fwd["h"], fwd["gate"], fwd["up"]
     ha, xa_g, xa_u = fwd["ha"], fwd["xa_g"], fwd["xa_u"]
