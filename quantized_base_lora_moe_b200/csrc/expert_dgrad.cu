@@ -61,6 +61,7 @@ constexpr int kWWarp0 = 8;
 constexpr int kWWarps = 16;
 constexpr int kEpi1Warp0 = kWWarp0 + kWWarps;
 constexpr int kThreads = (kEpi1Warp0 + 4) * 32;
+constexpr int kDhBatch = 2;   // dH epilogue: 16-byte pieces whose G and U loads are in flight together
 constexpr int kRows = 256;
 constexpr int kK = 64;
 constexpr int kXStages = 3;
@@ -258,36 +259,56 @@ __global__ void __launch_bounds__(kThreads, 1)
         stage_tokens_pair<16, BITS == 4 ? 4 : 1>(ct, lane_feature<BITS>(row), w);
         if (!es.sync(abort_flag, a.status)) { stop = true; break; }   // the chunk tile is complete
         const int nt = min(32, un.rows - c);
-        for (int p = etid; p < nt * 16; p += 128) {
-          const int t = p >> 4, fg = p & 15;
-          const uint4 v = *reinterpret_cast<const uint4*>(ct + t * kTRow + fg * 16);
-          const size_t orow = size_t(un.base + c + t) * a.out_ld;
-          if (MODE == DX) {
+        if (MODE == DX) {
+          for (int p = etid; p < nt * 16; p += 128) {
+            const int t = p >> 4, fg = p & 15;
+            const uint4 v = *reinterpret_cast<const uint4*>(ct + t * kTRow + fg * 16);
+            const size_t orow = size_t(un.base + c + t) * a.out_ld;
             bad |= f16x2_nonfinite(v.x) | f16x2_nonfinite(v.y) | f16x2_nonfinite(v.z) | f16x2_nonfinite(v.w);
             *reinterpret_cast<uint4*>(out + orow + fg * 8) = v;
-          } else {
-            // SwiGLU backward of 8 features: dG = dH U s (1 + G (1 - s)), dU = dH G s, s = sigmoid(G)
-            const uint16_t* gu = a.aux + orow + un.nt * 128 + fg * 8;
-            const uint4 g4 = *reinterpret_cast<const uint4*>(gu);
-            const uint4 u4 = *reinterpret_cast<const uint4*>(gu + a.f_dim);
-            const uint32_t hw[4] = {v.x, v.y, v.z, v.w};
-            const uint32_t gw[4] = {g4.x, g4.y, g4.z, g4.w};
-            const uint32_t uw[4] = {u4.x, u4.y, u4.z, u4.w};
-            uint32_t dg[4], du[4];
+          }
+        } else {
+          // SwiGLU backward of 8 features: dG = dH U s (1 + G (1 - s)), dU = dH G s,
+          // s = sigmoid(G). The G and U pieces of kDhBatch pieces are loaded before
+          // any of them is used, so that their latencies overlap.
+          for (int p0 = etid; p0 < nt * 16; p0 += kDhBatch * 128) {
+            uint4 g4[kDhBatch], u4[kDhBatch];
 #pragma unroll
-            for (int q = 0; q < 4; ++q) {
-              const float2 dh = __half22float2(*reinterpret_cast<const __half2*>(&hw[q]));
-              const float2 g = __half22float2(*reinterpret_cast<const __half2*>(&gw[q]));
-              const float2 uu = __half22float2(*reinterpret_cast<const __half2*>(&uw[q]));
-              const float s0 = 1.0f / (1.0f + __expf(-g.x)), s1 = 1.0f / (1.0f + __expf(-g.y));
-              dg[q] = f32x2_to_f16x2(dh.x * uu.x * s0 * (1.0f + g.x * (1.0f - s0)),
-                                     dh.y * uu.y * s1 * (1.0f + g.y * (1.0f - s1)));
-              du[q] = f32x2_to_f16x2(dh.x * g.x * s0, dh.y * g.y * s1);
-              bad |= f16x2_nonfinite(dg[q]) | f16x2_nonfinite(du[q]);
+            for (int i = 0; i < kDhBatch; ++i) {
+              const int p = p0 + 128 * i;
+              g4[i] = u4[i] = make_uint4(0u, 0u, 0u, 0u);
+              if (p < nt * 16) {
+                const uint16_t* gu = a.aux + size_t(un.base + c + (p >> 4)) * a.out_ld + un.nt * 128 + (p & 15) * 8;
+                g4[i] = *reinterpret_cast<const uint4*>(gu);
+                u4[i] = *reinterpret_cast<const uint4*>(gu + a.f_dim);
+              }
             }
-            uint16_t* dgu = static_cast<uint16_t*>(a.out) + orow + un.nt * 128 + fg * 8;
-            *reinterpret_cast<uint4*>(dgu) = make_uint4(dg[0], dg[1], dg[2], dg[3]);
-            *reinterpret_cast<uint4*>(dgu + a.f_dim) = make_uint4(du[0], du[1], du[2], du[3]);
+#pragma unroll
+            for (int i = 0; i < kDhBatch; ++i) {
+              const int p = p0 + 128 * i;
+              if (p >= nt * 16) break;
+              const int t = p >> 4, fg = p & 15;
+              const uint4 v = *reinterpret_cast<const uint4*>(ct + t * kTRow + fg * 16);
+              const size_t orow = size_t(un.base + c + t) * a.out_ld;
+              const uint32_t hw[4] = {v.x, v.y, v.z, v.w};
+              const uint32_t gw[4] = {g4[i].x, g4[i].y, g4[i].z, g4[i].w};
+              const uint32_t uw[4] = {u4[i].x, u4[i].y, u4[i].z, u4[i].w};
+              uint32_t dg[4], du[4];
+#pragma unroll
+              for (int q = 0; q < 4; ++q) {
+                const float2 dh = __half22float2(*reinterpret_cast<const __half2*>(&hw[q]));
+                const float2 g = __half22float2(*reinterpret_cast<const __half2*>(&gw[q]));
+                const float2 uu = __half22float2(*reinterpret_cast<const __half2*>(&uw[q]));
+                const float s0 = 1.0f / (1.0f + __expf(-g.x)), s1 = 1.0f / (1.0f + __expf(-g.y));
+                dg[q] = f32x2_to_f16x2(dh.x * uu.x * s0 * (1.0f + g.x * (1.0f - s0)),
+                                       dh.y * uu.y * s1 * (1.0f + g.y * (1.0f - s1)));
+                du[q] = f32x2_to_f16x2(dh.x * g.x * s0, dh.y * g.y * s1);
+                bad |= f16x2_nonfinite(dg[q]) | f16x2_nonfinite(du[q]);
+              }
+              uint16_t* dgu = static_cast<uint16_t*>(a.out) + orow + un.nt * 128 + fg * 8;
+              *reinterpret_cast<uint4*>(dgu) = make_uint4(dg[0], dg[1], dg[2], dg[3]);
+              *reinterpret_cast<uint4*>(dgu + a.f_dim) = make_uint4(du[0], du[1], du[2], du[3]);
+            }
           }
         }
       }
