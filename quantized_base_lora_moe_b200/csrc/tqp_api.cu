@@ -283,9 +283,10 @@ int to_bf16(const float* in, uint16_t* out, size_t n, cudaStream_t s) {
 // reversible stack of L coupling blocks
 // ----------------------------------------------------------------------------
 // Block l maps fp32 streams (a1, a2) to (b1, b2):  b1 = a1 + F_l(bf16(a2)),
-// b2 = a2 + G_l(bf16(b1)). The streams stay fp32 between blocks; every layer
-// reads the bf16 rounding of its stream. For block 0 the inputs are the bf16
-// x1, x2 (exact in fp32), so one block is exactly rev_couple_fwd. The
+// b2 = a2 + G_l(bf16(b1)). The streams stay fp32 on the stream grid between
+// blocks, so every add and subtract is exact; every layer reads the bf16
+// rounding of its stream. Block 0 puts its bf16 inputs x1, x2 on the grid as
+// rev_couple_fwd does, so one block is exactly rev_couple_fwd. The
 // workspace holds two sets of stream buffers that the blocks alternate
 // between, two bf16 layer inputs, one fp32 input gradient and one layer's
 // workspace: activation memory does not grow with L.
