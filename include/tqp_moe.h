@@ -277,8 +277,10 @@ int tqp_moe_layer_fwd(const uint16_t* x, int T, const tqp_moe_weights* w, uint16
  *   rounded to the grid (half to even) before the add; F reads x2 on the
  *   grid. On the grid every add and subtract is exact in fp32, and the layers
  *   are deterministic, so rev_couple_inv returns x1, x2 on the grid bit for
- *   bit: x itself wherever |x| >= 2^-9, else x moved by at most 2^-17. A
- *   stream value leaving the range raises TQP_STATUS_RANGE.
+ *   bit: x itself wherever |x| >= 2^-9, else x moved by at most 2^-17. The
+ *   inverse rounds its inputs y1, y2 to the grid as well (a no-op on the
+ *   outputs of rev_couple_fwd). A stream value leaving the range raises
+ *   TQP_STATUS_RANGE.
  *   F and G must share d. ws: rev_couple_workspace_size (both calls).
  * ------------------------------------------------------------------------- */
 size_t rev_couple_workspace_size(int T, const tqp_moe_weights* F, const tqp_moe_weights* G);
